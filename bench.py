@@ -1,0 +1,384 @@
+"""Throughput of the Gated Delta Rule-2 operator on B200: one JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one chunkwise forward (gdn2_fwd) plus one gate-aware backward
+(gdn2_bwd, reusing the forward's workspace) over the training workload
+B=4, T=4096, H=16, d_k=d_v=128, chunk 64, bf16 q/k/v/o/dO and float32 gates
+and state, on seeded synthetic inputs already resident in HBM.  The metric is
+tokens/s (B*T per step).  With N > 1 (torchrun, one rank per GPU, NCCL) every
+rank runs its own batch of that shape (weak scaling: the (batch, head) units
+are independent, so no data-path collective exists); ranks only meet at
+barriers and at the max-over-ranks of the device time.
+
+--impl reference times the fp64 CPU oracle (the only other implementation of
+the operator: a token-by-token recurrence with reverse mode) on a bounded
+sample of the same workload, on this host's cores.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD_INDEX = 2
+METRIC = "GDR-2 fwd+bwd tokens/s (H16, dk=dv=128) and % of HBM/tensor roofline"
+NAMES = ("q", "k", "v", "g", "b", "w", "S0")
+# algorithmic bytes per token-head (bf16 q,k,v,o,dO,dq,dk,dv; f32 g,b,w,dg,db,dw)
+FWD_BYTES = 3 * 128 * 2 + 3 * 128 * 4 + 128 * 2           # 2560
+BWD_BYTES = 3 * 128 * 2 + 3 * 128 * 4 + 128 * 2 + 3 * 128 * 2 + 3 * 128 * 4   # 4864
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--e2e-steps", type=int, default=3)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def cores() -> int:
+    return max(1, len(os.sched_getaffinity(0)))
+
+
+# ------------------------------------------------------------ clock sampling
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 100 ms while active."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.gpu)], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for t, line in self.lines:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            rows.append((t, parts))
+        inside = [r for t, r in rows if self.t0 - 0.15 <= t <= self.t1 + 0.15] or [r for _, r in rows]
+        mhz = [float(r[1]) for r in inside if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in inside if r[2].replace(".", "").isdigit()]
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({names[i] for r in inside for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(mhz) if mhz else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(inside)}
+
+
+# ------------------------------------------------------------------ our arm
+
+def traffic_from_profiles(kernel_key: str, src_hash: str):
+    """DRAM bytes per launch recorded from an ncu capture (profiles/traffic.json),
+    only if the kernel's sources are unchanged since the capture."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        rec = json.load(open(path)).get(kernel_key)
+    except (OSError, ValueError):
+        return None
+    if not rec or rec.get("src_sha256") != src_hash:
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+def sources_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "gated_delta_rule_128_b200", "csrc")
+    for n in sorted(os.listdir(csrc)):
+        if n.endswith((".cu", ".cuh")):
+            h.update(open(os.path.join(csrc, n), "rb").read())
+    return h.hexdigest()
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import gated_delta_rule_128_b200 as gdn
+    from gated_delta_rule_128_b200 import workloads
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = workloads.WORKLOADS[WORKLOAD_INDEX]
+    B, T, H, dk, dv, C = wl.B, wl.T, wl.H, wl.dk, wl.dv, wl.chunk
+    x = workloads.draw(B, T, H, dk, dv, wl.seed + 7919 * rank, s0_std=wl.s0_std,
+                       erase_scale=wl.erase_scale)
+    io_names = ("q", "k", "v", "dO")
+    bf = torch.bfloat16
+    host = {n: (t.to(bf) if n in io_names else t).contiguous().pin_memory() for n, t in x.items()}
+    d = {n: t.to(dev) for n, t in host.items()}
+    ws = gdn.workspace(B, T, H, dk, dv, C, gdn.GDN2_IO_BF16, True, dev)
+    o = torch.empty(B, T, H, dv, dtype=bf, device=dev)
+    grads = dict(dq=torch.empty_like(d["q"]), dk=torch.empty_like(d["k"]),
+                 dv=torch.empty_like(d["v"]), dg=torch.empty_like(d["g"]),
+                 db=torch.empty_like(d["b"]), dw=torch.empty_like(d["w"]))
+    io = gdn.GDN2_IO_BF16
+    stream = torch.cuda.current_stream(dev)
+
+    def step(inp):
+        gdn.gdn2_fwd(*(inp[n] for n in NAMES), o, None, ws, ws.numel(), B, T, H, dk, dv, C, io,
+                     stream)
+        gdn.gdn2_bwd(*(inp[n] for n in NAMES), inp["dO"], None, grads["dq"], grads["dk"],
+                     grads["dv"], grads["dg"], grads["db"], grads["dw"], None, ws, ws.numel(), 1,
+                     B, T, H, dk, dv, C, io, stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    for _ in range(max(3, args.warmup)):
+        step(d)
+    torch.cuda.synchronize(dev)
+    if gdn.gdn2_get_device_status(stream) != 0:
+        raise RuntimeError("device status reports an error after warm-up")
+
+    # device-timed region: K steps, per-call events on the launching stream
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    launches0 = gdn.gdn2_kernel_launches()
+    sampler.mark_start()
+    start.record(stream)
+    for i in range(args.steps):
+        e0, e1, e2 = ev[i]
+        e0.record(stream)
+        gdn.gdn2_fwd(*(d[n] for n in NAMES), o, None, ws, ws.numel(), B, T, H, dk, dv, C, io,
+                     stream)
+        e1.record(stream)
+        gdn.gdn2_bwd(*(d[n] for n in NAMES), d["dO"], None, grads["dq"], grads["dk"],
+                     grads["dv"], grads["dg"], grads["db"], grads["dw"], None, ws, ws.numel(), 1,
+                     B, T, H, dk, dv, C, io, stream)
+        e2.record(stream)
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    sampler.mark_end()
+    barrier()
+    launches = gdn.gdn2_kernel_launches() - launches0
+    ms_total = start.elapsed_time(end)
+    fwd_ms = statistics.mean(a.elapsed_time(b) for a, b, _ in ev)
+    bwd_ms = statistics.mean(b.elapsed_time(c) for _, b, c in ev)
+    status = gdn.gdn2_get_device_status(stream)
+    if status != 0:
+        raise RuntimeError(f"device status {status} after the timed region")
+
+    # end-to-end through host buffers: H2D of the step's inputs, D2H of its outputs
+    host_out = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+                for n, t in [("o", o)] + list(grads.items())}
+    h2d = sum(t.numel() * t.element_size() for n, t in host.items() if n != "S0")
+    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+    stage = {n: torch.empty_like(t) for n, t in d.items()}
+    barrier()
+    torch.cuda.synchronize(dev)
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_start.record(stream)
+    for _ in range(args.e2e_steps):
+        for n, t in host.items():
+            if n != "S0":
+                stage[n].copy_(t, non_blocking=True)
+        stage["S0"] = d["S0"]
+        step(stage)
+        host_out["o"].copy_(o, non_blocking=True)
+        for n, t in grads.items():
+            host_out[n].copy_(t, non_blocking=True)
+    e_end.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e_start.elapsed_time(e_end) / args.e2e_steps
+    barrier()
+    clocks = sampler.stop()
+
+    ms_step = ms_total / args.steps
+    if world > 1:
+        t = torch.tensor([ms_step, e2e_ms, fwd_ms, bwd_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step, e2e_ms, fwd_ms, bwd_ms = (float(v) for v in t.tolist())
+    tokens = B * T * world
+    value = tokens / (ms_step * 1e-3)
+    token_heads = B * T * H
+    alg_bytes = token_heads * (FWD_BYTES + BWD_BYTES)
+    achieved = alg_bytes / (ms_step * 1e-3) / 1e9
+    peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) \
+        if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")) else {}
+    peak = peaks.get("hbm_gbs", 6650.0)
+    peak_src = "measured" if "hbm_gbs" in peaks else "fallback"
+    traffic = traffic_from_profiles("fwd+bwd step, workload 2", sources_hash())
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic (seeded; BASELINE workload generators)",
+        "config": {"workload": wl.name, "B": B, "T": T, "H": H, "d_k": dk, "d_v": dv,
+                   "chunk": C, "io": "bf16 q/k/v/o/dO/dq/dk/dv, f32 g/b/w/state",
+                   "global_batch": B * world, "seq_len": T, "parallelism": f"dp{world}",
+                   "l2": "inputs 0.67 GB per step (> 126 MB L2), no flush"},
+        "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
+        "roofline": {"bound": "hbm", "kernel": "whole fwd+bwd step (all launches)",
+                     "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_source": peak_src,
+                     "algorithmic_bytes_per_step": alg_bytes, "traffic": traffic},
+        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches,
+        "clocks": clocks,
+    }
+    return line
+
+
+# -------------------------------------------------------------- oracle arm
+
+def oracle_sample(seconds_budget: float, nthreads: int):
+    """Time the fp64 oracle (forward + reverse mode) on whole-sequence (b, h)
+    pairs of the workload: about `seconds_budget` of CPU work on `nthreads`
+    threads.  Returns (tokens/s scaled to the workload's H heads, sample text)."""
+    import numpy as np
+
+    import oracle
+    from gated_delta_rule_128_b200 import workloads
+
+    wl = workloads.WORKLOADS[WORKLOAD_INDEX]
+    B, T, H, dk, dv = wl.B, wl.T, wl.H, wl.dk, wl.dv
+    # one batch row's inputs (all heads), bf16-rounded like the GPU's
+    x = workloads.draw(1, T, H, dk, dv, wl.seed, s0_std=wl.s0_std, erase_scale=wl.erase_scale)
+    for n in ("q", "k", "v", "dO"):
+        x[n] = workloads.round_bf16(x[n])
+
+    def run(npairs, tlen):
+        sl = {n: np.ascontiguousarray(t[:, :tlen, :npairs].double().numpy())
+              for n, t in x.items() if n not in ("S0",)}
+        S0 = np.zeros((1, npairs, dk, dv))
+        t0 = time.perf_counter()
+        oracle.forward(sl["q"], sl["k"], sl["v"], sl["g"], sl["b"], sl["w"], S0, nthreads=nthreads)
+        oracle.backward(sl["q"], sl["k"], sl["v"], sl["g"], sl["b"], sl["w"], S0, sl["dO"], None,
+                        nthreads=nthreads)
+        return time.perf_counter() - t0
+
+    probe_t = 256
+    dt = run(1, probe_t)                       # one pair, short: cost per token-head
+    per_th = dt / probe_t
+    pairs = min(H, max(1, nthreads))
+    tlen = int(min(T, max(64, seconds_budget / (per_th * pairs / min(pairs, nthreads)))))
+    elapsed = run(pairs, tlen)
+    token_heads = pairs * tlen
+    tokens_per_s = token_heads / elapsed / H
+    sample = (f"{pairs} (batch 0, head) pairs x {tlen} tokens of {wl.name}, fp64 forward + "
+              f"reverse mode, {nthreads} threads, {elapsed:.1f} s")
+    return tokens_per_s, sample, elapsed
+
+
+def run_reference(args, rank, world):
+    """The oracle arm: rank 0 only."""
+    if rank != 0:
+        return None
+    n = cores()
+    total = max(1, args.steps + max(3, args.warmup))
+    per_step = max(0.5, min(20.0, 150.0 / total))
+    vals = []
+    sample = ""
+    for i in range(total):
+        v, sample, _ = oracle_sample(per_step, n)
+        if i >= max(3, args.warmup):
+            vals.append(v)
+    value = statistics.mean(vals)
+    from gated_delta_rule_128_b200 import workloads
+    wl = workloads.WORKLOADS[WORKLOAD_INDEX]
+    return {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": None,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded; BASELINE workload generators)",
+        "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "H": wl.H, "d_k": wl.dk,
+                   "d_v": wl.dv, "chunk": wl.chunk, "global_batch": wl.B * world,
+                   "seq_len": wl.T, "parallelism": f"dp{world}"},
+        "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": n, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(args, rank, world, local_rank)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            v, sample, _ = oracle_sample(15.0, cores())
+            line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores(),
+                                    "kind": "oracle", "sample": sample}
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

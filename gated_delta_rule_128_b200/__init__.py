@@ -1,0 +1,187 @@
+"""Python binding of libgdn2.so, the B200 (sm_100a) Gated Delta Rule-2 operator.
+
+Argument marshalling only: every step of the operator runs in the CUDA
+library.  There is no CPU path; importing works anywhere, but the first call
+raises if ``libgdn2.so`` has not been built (``python -m
+gated_delta_rule_128_b200.build``).
+
+Two layers:
+
+* ``gdn2_fwd``, ``gdn2_bwd``, ``gdn2_decode_step``, ``gdn2_workspace_bytes``,
+  ``gdn2_get_device_status``: the C entry points of ``include/gdn2.h`` under
+  the same names, taking torch tensors (or None) where the C call takes
+  pointers, and raising ``Gdn2Error`` on a non-zero status.
+* ``forward``, ``backward``, ``decode_step``: allocate outputs and workspace
+  with torch (device memory is PyTorch's job here) and call the above on the
+  current CUDA stream.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, Optional
+
+import torch
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libgdn2.so")
+
+GDN2_IO_F32 = 0
+GDN2_IO_BF16 = 1
+STATUS = {0: "GDN2_OK", 1: "GDN2_ERR_INVALID_ARG", 2: "GDN2_ERR_UNSUPPORTED",
+          3: "GDN2_ERR_WORKSPACE", 4: "GDN2_ERR_CUDA", 5: "GDN2_ERR_TIMEOUT"}
+
+
+class Gdn2Error(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        msg = lib().gdn2_status_string(status).decode()
+        super().__init__(f"{fn} returned {STATUS.get(status, status)}: {msg}")
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libgdn2.so (raises if it is missing: there is no fallback)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is not built; run "
+                               "`python -m gated_delta_rule_128_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        L.gdn2_workspace_bytes.argtypes = [i] * 8
+        L.gdn2_workspace_bytes.restype = sz
+        L.gdn2_fwd.argtypes = [vp] * 10 + [sz] + [i] * 7 + [vp]
+        L.gdn2_fwd.restype = i
+        L.gdn2_bwd.argtypes = [vp] * 17 + [sz, i] + [i] * 7 + [vp]
+        L.gdn2_bwd.restype = i
+        L.gdn2_decode_step.argtypes = [vp] * 8 + [i] * 5 + [vp]
+        L.gdn2_decode_step.restype = i
+        L.gdn2_get_device_status.argtypes = [vp]
+        L.gdn2_get_device_status.restype = i
+        L.gdn2_status_string.argtypes = [i]
+        L.gdn2_status_string.restype = ctypes.c_char_p
+        L.gdn2_version.argtypes = []
+        L.gdn2_version.restype = i
+        L.gdn2_kernel_launches.argtypes = []
+        L.gdn2_kernel_launches.restype = ctypes.c_ulonglong
+        _lib = L
+    return _lib
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libgdn2 must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _io_of(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return GDN2_IO_BF16
+    if t.dtype == torch.float32:
+        return GDN2_IO_F32
+    raise TypeError(f"q/k/v must be float32 or bfloat16, got {t.dtype}")
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(fn: str, rc: int):
+    if rc != 0:
+        raise Gdn2Error(fn, rc)
+
+
+# ------------------------------------------------------------- C entry points
+
+def gdn2_workspace_bytes(B, T, H, d_k, d_v, chunk, io, for_bwd) -> int:
+    return int(lib().gdn2_workspace_bytes(B, T, H, d_k, d_v, chunk, io, int(for_bwd)))
+
+
+def gdn2_fwd(q, k, v, g, b, w, S0, o, ST, ws, ws_bytes, B, T, H, d_k, d_v, chunk, io,
+             stream=None):
+    rc = lib().gdn2_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b), _ptr(w), _ptr(S0), _ptr(o),
+                        _ptr(ST), _ptr(ws), ws_bytes, B, T, H, d_k, d_v, chunk, io,
+                        _stream(stream))
+    _check("gdn2_fwd", rc)
+
+
+def gdn2_bwd(q, k, v, g, b, w, S0, dO, dST, dq, dk, dv, dg, db, dw, dS0, ws, ws_bytes,
+             ws_has_fwd, B, T, H, d_k, d_v, chunk, io, stream=None):
+    rc = lib().gdn2_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b), _ptr(w), _ptr(S0), _ptr(dO),
+                        _ptr(dST), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg), _ptr(db), _ptr(dw),
+                        _ptr(dS0), _ptr(ws), ws_bytes, int(ws_has_fwd), B, T, H, d_k, d_v, chunk,
+                        io, _stream(stream))
+    _check("gdn2_bwd", rc)
+
+
+def gdn2_decode_step(q, k, v, g, b, w, S, o, N, H, d_k, d_v, io, stream=None):
+    rc = lib().gdn2_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b), _ptr(w), _ptr(S),
+                                _ptr(o), N, H, d_k, d_v, io, _stream(stream))
+    _check("gdn2_decode_step", rc)
+
+
+def gdn2_get_device_status(stream=None) -> int:
+    return int(lib().gdn2_get_device_status(_stream(stream)))
+
+
+def gdn2_kernel_launches() -> int:
+    return int(lib().gdn2_kernel_launches())
+
+
+# ------------------------------------------------------- tensor conveniences
+
+def workspace(B, T, H, d_k, d_v, chunk, io, for_bwd, device="cuda") -> torch.Tensor:
+    n = gdn2_workspace_bytes(B, T, H, d_k, d_v, chunk, io, for_bwd)
+    if n == 0:
+        raise Gdn2Error("gdn2_workspace_bytes", 2)
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def forward(q, k, v, g, b, w, S0=None, *, chunk: int = 64, want_state: bool = True,
+            ws: Optional[torch.Tensor] = None, for_bwd: bool = False, stream=None):
+    """Returns (o, S_T or None, ws).  Shapes: q, k, g, b [B,T,H,dk]; v, w [B,T,H,dv]."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    io = _io_of(q)
+    if ws is None:
+        ws = workspace(B, T, H, dk, dv, chunk, io, for_bwd, q.device)
+    o = torch.empty(B, T, H, dv, dtype=q.dtype, device=q.device)
+    ST = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device) if want_state else None
+    gdn2_fwd(q, k, v, g, b, w, S0, o, ST, ws, ws.numel(), B, T, H, dk, dv, chunk, io, stream)
+    return o, ST, ws
+
+
+def backward(q, k, v, g, b, w, S0, dO, dST=None, *, chunk: int = 64,
+             ws: Optional[torch.Tensor] = None, ws_has_fwd: bool = False,
+             want_dS0: bool = True, stream=None) -> Dict[str, torch.Tensor]:
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    io = _io_of(q)
+    if ws is None:
+        ws = workspace(B, T, H, dk, dv, chunk, io, True, q.device)
+        ws_has_fwd = False
+    out = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
+               dg=torch.empty_like(g), db=torch.empty_like(b), dw=torch.empty_like(w))
+    out["dS0"] = (torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device)
+                  if want_dS0 else None)
+    gdn2_bwd(q, k, v, g, b, w, S0, dO, dST, out["dq"], out["dk"], out["dv"], out["dg"], out["db"],
+             out["dw"], out["dS0"], ws, ws.numel(), ws_has_fwd, B, T, H, dk, dv, chunk, io, stream)
+    return out
+
+
+def decode_step(q, k, v, g, b, w, S, o=None, stream=None):
+    """One token for N sequences: q, k, g, b [N,H,dk]; v, w [N,H,dv]; S [N,H,dk,dv]
+    float32, updated in place.  Returns o [N,H,dv]."""
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    if o is None:
+        o = torch.empty(N, H, dv, dtype=q.dtype, device=q.device)
+    gdn2_decode_step(q, k, v, g, b, w, S, o, N, H, dk, dv, _io_of(q), stream)
+    return o

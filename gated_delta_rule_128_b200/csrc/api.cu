@@ -1,0 +1,169 @@
+// Host side of the C ABI in include/gdn2.h: argument checks, workspace sizing
+// and kernel dispatch.  No allocation, no synchronisation (except
+// gdn2_get_device_status), no CPU fallback.
+
+#include <stdint.h>
+
+#include <atomic>
+
+#include "common.cuh"
+
+namespace gdn2 {
+
+// kernels and launchers of the other translation units
+template <typename E>
+cudaError_t simt_prep_launch(const void *, const void *, const void *, const float *, const float *,
+                             const float *, void *, const Dims &, cudaStream_t);
+cudaError_t simt_state_fwd_launch(const float *, float *, const void *, int, void *, const Dims &,
+                                  cudaStream_t);
+template <typename E>
+cudaError_t simt_out_launch(const void *, void *, void *, const Dims &, cudaStream_t);
+template <typename E>
+cudaError_t simt_bwd_launch(const void *, const void *, const void *, const float *, const float *,
+                            const void *, const float *, void *, void *, void *, float *, float *,
+                            float *, float *, void *, const Dims &, cudaStream_t);
+cudaError_t decode_launch(const void *, const void *, const void *, const float *, const float *,
+                          const float *, float *, void *, int, int, int, int, gdn2_io,
+                          cudaStream_t);
+
+__device__ unsigned int g_status_word;
+
+static std::atomic<unsigned long long> g_launches{0};
+void count_launches(unsigned long long n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+static bool supported_d(int x) { return x == 32 || x == 64 || x == 128; }
+static bool supported_chunk(int c) { return c == 16 || c == 32 || c == 64; }
+static bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+static gdn2_status check_dims(int B, int T, int H, int dk, int dv, int chunk, gdn2_io io) {
+    if (B < 1 || T < 1 || H < 1) return GDN2_ERR_INVALID_ARG;
+    if (io != GDN2_IO_F32 && io != GDN2_IO_BF16) return GDN2_ERR_INVALID_ARG;
+    if (!supported_d(dk) || !supported_d(dv) || !supported_chunk(chunk)) return GDN2_ERR_UNSUPPORTED;
+    // grid limits: chunks per sequence in grid.x, H in grid.y, B in grid.z
+    if (H > 65535 || B > 65535) return GDN2_ERR_UNSUPPORTED;
+    if ((long long)B * T * H * (dk > dv ? dk : dv) > (1LL << 40)) return GDN2_ERR_UNSUPPORTED;
+    return GDN2_OK;
+}
+
+static Dims make_dims(int B, int T, int H, int dk, int dv, int chunk) {
+    return Dims{B, T, H, dk, dv, chunk, (T + chunk - 1) / chunk};
+}
+
+// every required pointer non-null and 16-byte aligned; optional ones aligned
+static gdn2_status check_ptrs(std::initializer_list<const void *> required,
+                              std::initializer_list<const void *> optional) {
+    for (const void *p : required)
+        if (!p || !aligned16(p)) return GDN2_ERR_INVALID_ARG;
+    for (const void *p : optional)
+        if (p && !aligned16(p)) return GDN2_ERR_INVALID_ARG;
+    return GDN2_OK;
+}
+
+static gdn2_status cuda_status(cudaError_t e) { return e == cudaSuccess ? GDN2_OK : GDN2_ERR_CUDA; }
+
+static cudaError_t run_forward(const void *q, const void *k, const void *v, const float *g,
+                               const float *b, const float *w, const float *S0, void *o, float *ST,
+                               void *ws, const Dims &d, gdn2_io io, cudaStream_t s) {
+    cudaError_t e;
+    if (io == GDN2_IO_BF16) {
+        if ((e = simt_prep_launch<__nv_bfloat16>(q, k, v, g, b, w, ws, d, s)) != cudaSuccess) return e;
+    } else {
+        if ((e = simt_prep_launch<float>(q, k, v, g, b, w, ws, d, s)) != cudaSuccess) return e;
+    }
+    if ((e = simt_state_fwd_launch(S0, ST, k, io == GDN2_IO_BF16, ws, d, s)) != cudaSuccess) return e;
+    if (o) {
+        if (io == GDN2_IO_BF16) return simt_out_launch<__nv_bfloat16>(q, o, ws, d, s);
+        return simt_out_launch<float>(q, o, ws, d, s);
+    }
+    return cudaSuccess;
+}
+
+}  // namespace gdn2
+
+using namespace gdn2;
+
+extern "C" {
+
+size_t gdn2_workspace_bytes(int B, int T, int H, int d_k, int d_v, int chunk, gdn2_io io,
+                            int for_bwd) {
+    if (check_dims(B, T, H, d_k, d_v, chunk, io) != GDN2_OK) return 0;
+    SimtWs lay = simt_ws_layout(make_dims(B, T, H, d_k, d_v, chunk));
+    return for_bwd ? lay.bwd_end : lay.fwd_end;
+}
+
+gdn2_status gdn2_fwd(const void *q, const void *k, const void *v, const float *g, const float *b,
+                     const float *w, const float *S0, void *o, float *ST, void *ws,
+                     size_t ws_bytes, int B, int T, int H, int d_k, int d_v, int chunk,
+                     gdn2_io io, gdn2_stream_t stream) {
+    gdn2_status st = check_dims(B, T, H, d_k, d_v, chunk, io);
+    if (st != GDN2_OK) return st;
+    st = check_ptrs({q, k, v, g, b, w, o}, {S0, ST});
+    if (st != GDN2_OK) return st;
+    Dims d = make_dims(B, T, H, d_k, d_v, chunk);
+    if (!ws || !aligned16(ws) || ws_bytes < simt_ws_layout(d).fwd_end) return GDN2_ERR_WORKSPACE;
+    return cuda_status(run_forward(q, k, v, g, b, w, S0, o, ST, ws, d, io, (cudaStream_t)stream));
+}
+
+gdn2_status gdn2_bwd(const void *q, const void *k, const void *v, const float *g, const float *b,
+                     const float *w, const float *S0, const void *dO, const float *dST, void *dq,
+                     void *dk, void *dv, float *dg, float *db, float *dw, float *dS0, void *ws,
+                     size_t ws_bytes, int ws_has_fwd, int B, int T, int H, int d_k, int d_v,
+                     int chunk, gdn2_io io, gdn2_stream_t stream) {
+    gdn2_status st = check_dims(B, T, H, d_k, d_v, chunk, io);
+    if (st != GDN2_OK) return st;
+    st = check_ptrs({q, k, v, g, b, w, dO, dq, dk, dv, dg, db, dw}, {S0, dST, dS0});
+    if (st != GDN2_OK) return st;
+    Dims d = make_dims(B, T, H, d_k, d_v, chunk);
+    if (!ws || !aligned16(ws) || ws_bytes < simt_ws_layout(d).bwd_end) return GDN2_ERR_WORKSPACE;
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e;
+    if (!ws_has_fwd) {
+        e = run_forward(q, k, v, g, b, w, S0, nullptr, nullptr, ws, d, io, s);
+        if (e != cudaSuccess) return GDN2_ERR_CUDA;
+    }
+    if (io == GDN2_IO_BF16)
+        e = simt_bwd_launch<__nv_bfloat16>(q, k, v, b, w, dO, dST, dq, dk, dv, dg, db, dw, dS0, ws,
+                                           d, s);
+    else
+        e = simt_bwd_launch<float>(q, k, v, b, w, dO, dST, dq, dk, dv, dg, db, dw, dS0, ws, d, s);
+    return cuda_status(e);
+}
+
+gdn2_status gdn2_decode_step(const void *q, const void *k, const void *v, const float *g,
+                             const float *b, const float *w, float *S, void *o, int N, int H,
+                             int d_k, int d_v, gdn2_io io, gdn2_stream_t stream) {
+    if (N < 1 || H < 1 || (io != GDN2_IO_F32 && io != GDN2_IO_BF16)) return GDN2_ERR_INVALID_ARG;
+    if (!supported_d(d_k) || !supported_d(d_v)) return GDN2_ERR_UNSUPPORTED;
+    if ((long long)N * H > 0x7fffffffLL) return GDN2_ERR_UNSUPPORTED;
+    gdn2_status st = check_ptrs({q, k, v, g, b, w, S, o}, {});
+    if (st != GDN2_OK) return st;
+    return cuda_status(decode_launch(q, k, v, g, b, w, S, o, N, H, d_k, d_v, io,
+                                     (cudaStream_t)stream));
+}
+
+gdn2_status gdn2_get_device_status(gdn2_stream_t stream) {
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return GDN2_ERR_CUDA;
+    unsigned int word = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&word, g_status_word, sizeof(word)) != cudaSuccess) return GDN2_ERR_CUDA;
+    if (word != 0 && cudaMemcpyToSymbol(g_status_word, &zero, sizeof(zero)) != cudaSuccess)
+        return GDN2_ERR_CUDA;
+    return (gdn2_status)word;
+}
+
+const char *gdn2_status_string(gdn2_status status) {
+    switch (status) {
+        case GDN2_OK: return "ok";
+        case GDN2_ERR_INVALID_ARG: return "invalid argument (null or misaligned pointer, bad size)";
+        case GDN2_ERR_UNSUPPORTED: return "unsupported size (d_k, d_v in {32,64,128}; chunk in {16,32,64})";
+        case GDN2_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+        case GDN2_ERR_CUDA: return "CUDA error";
+        case GDN2_ERR_TIMEOUT: return "a kernel gave up on a bounded wait";
+    }
+    return "unknown status";
+}
+
+int gdn2_version(void) { return 100; }
+
+unsigned long long gdn2_kernel_launches(void) { return g_launches.load(); }
+
+}  // extern "C"

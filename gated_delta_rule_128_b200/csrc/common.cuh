@@ -1,0 +1,106 @@
+// Shared device helpers, sizes and the workspace layout of libgdn2.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "gdn2.h"
+
+namespace gdn2 {
+
+constexpr int kMaxD = 128;     // largest d_k / d_v
+constexpr int kMaxChunk = 64;  // largest chunk
+
+struct Dims {
+    int B, T, H, dk, dv, C, NC;
+};
+
+// ---- element access in the io type (float or bf16), computing in float
+template <typename E> __device__ __forceinline__ float ldx(const E *p, size_t i);
+template <> __device__ __forceinline__ float ldx<float>(const float *p, size_t i) { return p[i]; }
+template <> __device__ __forceinline__ float ldx<__nv_bfloat16>(const __nv_bfloat16 *p, size_t i) {
+    return __bfloat162float(p[i]);
+}
+template <typename E> __device__ __forceinline__ void stx(E *p, size_t i, float x);
+template <> __device__ __forceinline__ void stx<float>(float *p, size_t i, float x) { p[i] = x; }
+template <> __device__ __forceinline__ void stx<__nv_bfloat16>(__nv_bfloat16 *p, size_t i, float x) {
+    p[i] = __float2bfloat16_rn(x);
+}
+
+// offset of element (bb, t, h, 0) in a [B, T, H, width] tensor
+__device__ __forceinline__ size_t tok(const Dims &d, int bb, int t, int h, int width) {
+    return (((size_t)bb * d.T + t) * d.H + h) * (size_t)width;
+}
+// offset of the (bb, h) state in a [B, H, dk, dv] tensor
+__device__ __forceinline__ size_t st_off(const Dims &d, int bb, int h) {
+    return ((size_t)bb * d.H + h) * (size_t)d.dk * d.dv;
+}
+// index of chunk tile (bb, h, c)
+__device__ __forceinline__ size_t tile(const Dims &d, int bb, int h, int c) {
+    return ((size_t)bb * d.H + h) * d.NC + c;
+}
+
+// ---- the device status word (GDN2_OK or the first error recorded); kernels
+// that can give up on a bounded wait receive its device address.
+__device__ __forceinline__ void record_status(unsigned int *status, unsigned int s) {
+    atomicCAS(status, 0u, s);
+}
+
+// ---- workspace of the CUDA-core (fp32) path: per-chunk float32 tiles
+struct SimtWs {
+    size_t gam;     // [B,H,NC,C,dk]  in-chunk cumulative log-decay
+    size_t Tinv;    // [B,H,NC,C,C]   (I + A)^-1
+    size_t P;       // [B,H,NC,C,C]   lower-incl(Qb Kh^T)
+    size_t W;       // [B,H,NC,C,dk]  T Kc
+    size_t Up;      // [B,H,NC,C,dv]  T U
+    size_t Delta;   // [B,H,NC,C,dv]  U' - W S_c
+    size_t Sc;      // [B,H,NC,dk,dv] chunk-entry states
+    size_t fwd_end;
+    size_t dSn;     // [B,H,NC,dk,dv] dL/dS at the chunk's exit
+    size_t dDelta;  // [B,H,NC,C,dv]
+    size_t dP;      // [B,H,NC,C,C]   lower-incl(dO Delta^T)
+    size_t dA;      // [B,H,NC,C,C]   -strictly-lower(dU Delta^T)
+    size_t X1;      // [B,H,NC,C,dk]  dO S_c^T
+    size_t X2;      // [B,H,NC,C,dk]  dU S_c^T
+    size_t X3;      // [B,H,NC,C,dk]  Delta dSn^T
+    size_t X4;      // [B,H,NC,dk]    rowsum(dSn . S_c)
+    size_t bwd_end;
+};
+
+// ---- host-side launch counter (gdn2_kernel_launches)
+void count_launches(unsigned long long n);
+
+inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+inline SimtWs simt_ws_layout(const Dims &d) {
+    SimtWs w;
+    size_t tiles = (size_t)d.B * d.H * d.NC;
+    size_t o = 0;
+    auto take = [&](size_t floats) { size_t at = o; o = align256(o + floats * sizeof(float)); return at; };
+    w.gam = take(tiles * d.C * d.dk);
+    w.Tinv = take(tiles * d.C * d.C);
+    w.P = take(tiles * d.C * d.C);
+    w.W = take(tiles * d.C * d.dk);
+    w.Up = take(tiles * d.C * d.dv);
+    w.Delta = take(tiles * d.C * d.dv);
+    w.Sc = take(tiles * (size_t)d.dk * d.dv);
+    w.fwd_end = o;
+    w.dSn = take(tiles * (size_t)d.dk * d.dv);
+    w.dDelta = take(tiles * d.C * d.dv);
+    w.dP = take(tiles * d.C * d.C);
+    w.dA = take(tiles * d.C * d.C);
+    w.X1 = take(tiles * d.C * d.dk);
+    w.X2 = take(tiles * d.C * d.dk);
+    w.X3 = take(tiles * d.C * d.dk);
+    w.X4 = take(tiles * d.dk);
+    w.bwd_end = o;
+    return w;
+}
+
+template <typename T> __host__ __device__ __forceinline__ T *at(void *base, size_t off) {
+    return reinterpret_cast<T *>(static_cast<char *>(base) + off);
+}
+
+}  // namespace gdn2

@@ -1,0 +1,147 @@
+/*
+ * gdn2.h - C ABI of the B200 (sm_100a) Gated Delta Rule-2 operator library
+ * (libgdn2.so).
+ *
+ * The operator ("Gated DeltaNet-2: Decoupling Erase and Write in Linear
+ * Attention"; anthology-of-the-sota LIT-802 review, "Key takeaways" 1, paper
+ * Sec. 3.1 Eqs. 8-10) is, for every batch row b and head h independently,
+ *
+ *     S_t = (I - k_t (b_t . k_t)^T) D_t S_{t-1} + k_t (w_t . v_t)^T,
+ *     D_t = diag(exp g_t),          o_t = S_t^T q_t,
+ *
+ * with a channel-wise log-decay g_t (key axis), erase gate b_t (key axis) and
+ * write gate w_t (value axis).  The read o_t = S_t^T q_t (after the update, no
+ * scale) is the reading taken for this library; the pages never print it.
+ * Gate activations (sigmoid, logsigmoid) and any q/k normalisation or 1/sqrt(d)
+ * scale belong to the caller: the library takes the activated values.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Layouts (all contiguous, innermost dimension fastest):
+ *   q, k, g, b, dq, dk, dg, db : [B, T, H, d_k]
+ *   v, w, o, dO, dv, dw        : [B, T, H, d_v]
+ *   S0, ST, dST, dS0           : [B, H, d_k, d_v]   (row = key channel)
+ * Decode uses the same layouts with T = 1 removed: [N, H, d] and
+ * [N, H, d_k, d_v].
+ * Element types: q, k, v, o, dO, dq, dk, dv are float32 (GDN2_IO_F32) or
+ *   bfloat16 (GDN2_IO_BF16); g, b, w, dg, db, dw and every state are float32.
+ * Supported sizes: B, T, H, N >= 1; d_k, d_v in {32, 64, 128}; chunk in
+ *   {16, 32, 64}.  T need not be a multiple of chunk (the last chunk is short).
+ *   The chunk size changes only the order of rounding, never the result.
+ * Pointers: device memory owned by the caller; the library allocates nothing
+ *   and keeps no pointer after a call returns.  Every pointer must be 16-byte
+ *   aligned.  Input and output buffers must not overlap (except S in
+ *   gdn2_decode_step, which is updated in place).
+ * Streams: every call only enqueues work on `stream` (NULL = the legacy
+ *   default stream) and returns without synchronising, except
+ *   gdn2_get_device_status.
+ * Errors: arguments are checked on the host before anything is launched; a
+ *   failed check returns a status and enqueues nothing.  A failed launch
+ *   returns GDN2_ERR_CUDA.  Kernels never trap: a kernel that gives up on a
+ *   bounded wait records GDN2_ERR_TIMEOUT in a device status word that
+ *   gdn2_get_device_status reports.
+ */
+#ifndef GDN2_H
+#define GDN2_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Identical to cudaStream_t / CUstream. */
+struct CUstream_st;
+typedef struct CUstream_st *gdn2_stream_t;
+
+typedef enum {
+    GDN2_OK = 0,
+    GDN2_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misaligned pointer   */
+    GDN2_ERR_UNSUPPORTED = 2,  /* d_k, d_v or chunk outside the supported set  */
+    GDN2_ERR_WORKSPACE = 3,    /* workspace missing or smaller than required   */
+    GDN2_ERR_CUDA = 4,         /* a CUDA launch or runtime call failed          */
+    GDN2_ERR_TIMEOUT = 5       /* a kernel gave up on a bounded wait            */
+} gdn2_status;
+
+typedef enum {
+    GDN2_IO_F32 = 0,
+    GDN2_IO_BF16 = 1
+} gdn2_io;
+
+/* Bytes of caller-provided device workspace that gdn2_fwd (for_bwd = 0) or
+ * gdn2_fwd followed by gdn2_bwd (for_bwd = 1) needs for these sizes.  Returns
+ * 0 when the sizes are unsupported.  A workspace sized with for_bwd = 1 also
+ * serves gdn2_fwd, and then keeps what gdn2_bwd can reuse (see ws_has_fwd). */
+size_t gdn2_workspace_bytes(int B, int T, int H, int d_k, int d_v, int chunk, gdn2_io io,
+                            int for_bwd);
+
+/* Chunkwise forward ("Gated DeltaNet-2" LIT-802 review, "Key takeaways" 2;
+ * paper Secs. 3.3-3.4 and Apps. A-B: the state is normalised by the
+ * cumulative decay so that D_t folds into the two factors of each rank-one
+ * erase, and one WY inverse serves the erase and the write side; only the
+ * state crosses chunk borders).
+ *   q, k, v, g, b, w : inputs (layouts above).
+ *   S0  : initial state, or NULL for zero.
+ *   o   : output [B, T, H, d_v] in the io type.
+ *   ST  : final state, or NULL if not wanted.
+ *   ws  : workspace of ws_bytes >= gdn2_workspace_bytes(..., for_bwd = 0).
+ *         If ws_bytes >= gdn2_workspace_bytes(..., for_bwd = 1), the call also
+ *         leaves in ws what gdn2_bwd reuses with ws_has_fwd = 1. */
+gdn2_status gdn2_fwd(const void *q, const void *k, const void *v, const float *g,
+                     const float *b, const float *w, const float *S0, void *o, float *ST,
+                     void *ws, size_t ws_bytes, int B, int T, int H, int d_k, int d_v,
+                     int chunk, gdn2_io io, gdn2_stream_t stream);
+
+/* Gate-aware backward of L = <o, dO> + <S_T, dST> ("Gated DeltaNet-2"
+ * LIT-802 review, "Key takeaways" 2: the per-channel gates stay inside the
+ * dot products that accumulate dA instead of being pulled outside as a scalar
+ * beta would be; digg thread 11/).
+ *   q ... S0   : the forward's inputs (S0 may be NULL for zero).
+ *   dO  : upstream gradient of o, io type.   dST : of S_T, or NULL for zero.
+ *   dq, dk, dv (io type), dg, db, dw (float32) : gradients, same layouts as
+ *         the inputs.  dS0 : gradient of S0 (float32), or NULL if not wanted.
+ *   ws, ws_bytes >= gdn2_workspace_bytes(..., for_bwd = 1).
+ *   ws_has_fwd : 1 if ws holds what gdn2_fwd left there for these same inputs
+ *         and sizes (the training pattern: fwd then bwd with one workspace);
+ *         0 makes the call recompute it first.  Passing 1 for a workspace that
+ *         does not hold the matching forward gives wrong gradients. */
+gdn2_status gdn2_bwd(const void *q, const void *k, const void *v, const float *g,
+                     const float *b, const float *w, const float *S0, const void *dO,
+                     const float *dST, void *dq, void *dk, void *dv, float *dg, float *db,
+                     float *dw, float *dS0, void *ws, size_t ws_bytes, int ws_has_fwd,
+                     int B, int T, int H, int d_k, int d_v, int chunk, gdn2_io io,
+                     gdn2_stream_t stream);
+
+/* One token of the recurrence for N independent sequences ("Gated DeltaNet-2"
+ * abstract: linear-time mixing with constant-memory decoding; the update of
+ * LIT-802 "Key takeaways" 1):
+ *   S <- D S;  delta = w.v - S^T (b.k);  S <- S + k delta^T;  o = S^T q.
+ *   q, k, v : [N, H, d] in the io type;  g, b : [N, H, d_k];  w : [N, H, d_v].
+ *   S : [N, H, d_k, d_v] float32, read and overwritten in place.
+ *   o : [N, H, d_v] in the io type.
+ * Needs no workspace. */
+gdn2_status gdn2_decode_step(const void *q, const void *k, const void *v, const float *g,
+                             const float *b, const float *w, float *S, void *o, int N, int H,
+                             int d_k, int d_v, gdn2_io io, gdn2_stream_t stream);
+
+/* Waits for `stream`, then returns and clears the device status word: GDN2_OK,
+ * or the first error a kernel recorded since the last call (GDN2_ERR_TIMEOUT).
+ * Returns GDN2_ERR_CUDA if the stream reports a CUDA error. */
+gdn2_status gdn2_get_device_status(gdn2_stream_t stream);
+
+/* Static, never NULL. */
+const char *gdn2_status_string(gdn2_status status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int gdn2_version(void);
+
+/* Number of kernels this library has enqueued in the calling process since it
+ * was loaded (all threads, all devices).  A diagnostic for counting launches
+ * around a region of work; not tied to any entry in the pages. */
+unsigned long long gdn2_kernel_launches(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN2_H */

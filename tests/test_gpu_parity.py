@@ -1,0 +1,255 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle on the
+same seeded inputs.
+
+Tolerances (max|gpu - ref| / max|ref| per output tensor): float32 path 1e-4;
+bf16-I/O path 5e-3 on o and S_T, 1e-2 on gradients.  bf16 inputs are rounded
+once on the host and the oracle consumes exactly the rounded values.
+
+Small cases span several chunks and a ragged tail; the five workloads run at
+full size on the GPU and are compared on sampled (batch, head) pairs that the
+oracle computes one by one.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import gated_delta_rule_128_b200 as gdn
+from gated_delta_rule_128_b200 import workloads
+from _util import TOL_BF16_GRAD, TOL_BF16_OUT, TOL_F32, io_round, rel, to_device, to_np64
+
+pytestmark = pytest.mark.gpu
+
+NAMES = ("q", "k", "v", "g", "b", "w", "S0")
+GRADS = ("dq", "dk", "dv", "dg", "db", "dw", "dS0")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    gdn.lib()
+
+
+def tols(io):
+    return (TOL_F32, TOL_F32) if io == "f32" else (TOL_BF16_OUT, TOL_BF16_GRAD)
+
+
+def gpu_fwd_bwd(x, io, chunk, backward=True, use_dST=True):
+    d = to_device(x, io)
+    o, ST, ws = gdn.forward(*(d[n] for n in NAMES), chunk=chunk, for_bwd=backward)
+    out = {"o": o, "ST": ST}
+    if backward:
+        gr = gdn.backward(*(d[n] for n in NAMES), d["dO"], d.get("dST") if use_dST else None,
+                          chunk=chunk, ws=ws, ws_has_fwd=True)
+        out.update(gr)
+    torch.cuda.synchronize()
+    assert gdn.gdn2_get_device_status() == 0
+    return {n: t.float().cpu().numpy() for n, t in out.items() if t is not None}
+
+
+def oracle_fwd_bwd(x, io, backward=True, use_dST=True, pairs=None):
+    """Oracle on all (b, h) pairs, or on the listed ones (results stacked in
+    the order given, as batch 1 with len(pairs) heads)."""
+    if pairs is not None:
+        x = {n: (torch.stack([t[bb, h] for bb, h in pairs])[None] if n in ("S0", "dST")
+                 else torch.stack([t[bb, :, h] for bb, h in pairs], dim=1)[None]).contiguous()
+             for n, t in x.items() if t.dim() == 4}
+    r = to_np64(io_round(x, io))
+    o, ST = oracle.forward(*(r[n] for n in NAMES))
+    out = {"o": o, "ST": ST}
+    if backward:
+        out.update(oracle.backward(*(r[n] for n in NAMES), r["dO"],
+                                   r.get("dST") if use_dST else None, ckpt=64))
+    return out
+
+
+def compare(gpu, ref, io, names, pairs=None):
+    tol_out, tol_grad = tols(io)
+    errs = {}
+    for n in names:
+        a = gpu[n]
+        if pairs is not None:
+            if n in ("ST", "dS0"):
+                a = np.stack([a[bb, h] for bb, h in pairs])[None]
+            else:
+                a = np.stack([a[bb, :, h] for bb, h in pairs], axis=1)[None]
+        assert np.isfinite(a).all(), n
+        errs[n] = rel(a, ref[n])
+    bad = {n: e for n, e in errs.items()
+           if e > (tol_out if n in ("o", "ST") else tol_grad)}
+    assert not bad, f"parity failures {bad} (all: {errs})"
+    return errs
+
+
+# ------------------------------------------------------------- workload 0
+
+def test_workload0_fp32_forward_backward():
+    x = workloads.draw_workload(0)
+    gpu = gpu_fwd_bwd(x, "f32", 64, use_dST=False)
+    ref = oracle_fwd_bwd(x, "f32", use_dST=False)
+    compare(gpu, ref, "f32", ("o", "ST") + GRADS)
+
+
+@pytest.mark.parametrize("tie", ["kda", "gdn"])
+def test_workload0_fp32_tied_gates(tie):
+    """b = w = beta 1 gives KDA; a scalar decay as well gives Gated DeltaNet."""
+    x = workloads.draw_workload(0, tie=tie)
+    gpu = gpu_fwd_bwd({n: t for n, t in x.items() if n not in ("beta", "alpha_log")}, "f32", 64,
+                      use_dST=False)
+    r = to_np64(x)
+    if tie == "kda":
+        o, ST = oracle.kda_forward(r["q"], r["k"], r["v"], r["g"], r["beta"], r["S0"])
+    else:
+        o, ST = oracle.gdn_forward(r["q"], r["k"], r["v"], r["alpha_log"], r["beta"], r["S0"])
+    assert rel(gpu["o"], o) < TOL_F32 and rel(gpu["ST"], ST) < TOL_F32
+    ref = oracle.backward(*(r[n] for n in NAMES), r["dO"], None)
+    compare(gpu, ref, "f32", GRADS)
+    # the tied scalar's gradient: dbeta = sum_c db + sum_c dw
+    dbeta = gpu["db"].sum(-1) + gpu["dw"].sum(-1)
+    assert rel(dbeta, ref["db"].sum(-1) + ref["dw"].sum(-1)) < TOL_F32
+
+
+# ------------------------------------------------------ small grids, ragged
+
+CASES = [
+    # B, T, H, dk, dv, chunk
+    (2, 200, 2, 128, 128, 64),
+    (1, 77, 3, 64, 128, 32),
+    (2, 33, 2, 32, 64, 16),
+    (1, 64, 2, 128, 32, 64),
+    (1, 65, 1, 64, 64, 64),
+    (3, 1, 2, 128, 128, 64),
+    (1, 130, 2, 32, 32, 16),
+]
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "B{}T{}H{}k{}v{}C{}".format(*c))
+def test_small_grids(case, io):
+    B, T, H, dk, dv, chunk = case
+    x = workloads.draw(B, T, H, dk, dv, 500 + T + dk, s0_std=0.3, with_dST=True)
+    gpu = gpu_fwd_bwd(x, io, chunk)
+    ref = oracle_fwd_bwd(x, io)
+    compare(gpu, ref, io, ("o", "ST") + GRADS)
+
+
+def test_negative_eigenvalue_erase_range():
+    x = workloads.draw(1, 150, 2, 64, 64, 77, erase_scale=2.0, s0_std=0.1, with_dST=True)
+    for io in ("f32", "bf16"):
+        compare(gpu_fwd_bwd(x, io, 64), oracle_fwd_bwd(x, io), io, ("o", "ST") + GRADS)
+
+
+def test_backward_recompute_equals_reuse_and_is_deterministic():
+    x = workloads.draw(2, 150, 2, 128, 128, 91, s0_std=0.1, with_dST=True)
+    d = to_device(x, "bf16")
+    o, ST, ws = gdn.forward(*(d[n] for n in NAMES), chunk=64, for_bwd=True)
+    a = gdn.backward(*(d[n] for n in NAMES), d["dO"], d["dST"], chunk=64, ws=ws, ws_has_fwd=True)
+    b = gdn.backward(*(d[n] for n in NAMES), d["dO"], d["dST"], chunk=64)  # fresh ws, recompute
+    o2, ST2, _ = gdn.forward(*(d[n] for n in NAMES), chunk=64)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o2) and torch.equal(ST, ST2)
+    for n in GRADS:
+        assert torch.equal(a[n], b[n]), n
+
+
+def test_every_output_written_and_no_nan_read():
+    """Outputs and workspace pre-filled with NaN: every output element must be
+    written, and nothing uninitialised may reach an output."""
+    x = workloads.draw(1, 100, 2, 64, 64, 92, s0_std=0.1, with_dST=True)
+    d = to_device(x, "bf16")
+    B, T, H, dk, dv = 1, 100, 2, 64, 64
+    ws = gdn.workspace(B, T, H, dk, dv, 32, 1, True)
+    ws.view(torch.uint8).fill_(0xFF)   # NaN pattern in every float32 slot
+    o = torch.full((B, T, H, dv), float("nan"), dtype=torch.bfloat16, device="cuda")
+    ST = torch.full((B, H, dk, dv), float("nan"), device="cuda")
+    gdn.gdn2_fwd(*(d[n] for n in NAMES), o, ST, ws, ws.numel(), B, T, H, dk, dv, 32, 1)
+    outs = {n: torch.full_like(d[m], float("nan")) for n, m in
+            (("dq", "q"), ("dk", "k"), ("dv", "v"), ("dg", "g"), ("db", "b"), ("dw", "w"))}
+    outs["dS0"] = torch.full_like(ST, float("nan"))
+    gdn.gdn2_bwd(*(d[n] for n in NAMES), d["dO"], d["dST"], outs["dq"], outs["dk"], outs["dv"],
+                 outs["dg"], outs["db"], outs["dw"], outs["dS0"], ws, ws.numel(), 1,
+                 B, T, H, dk, dv, 32, 1)
+    torch.cuda.synchronize()
+    for n, t in list(outs.items()) + [("o", o), ("ST", ST)]:
+        assert torch.isfinite(t.float()).all(), n
+
+
+# --------------------------------------------- full-size workloads, sampled
+
+SAMPLE = {1: [(0, 0), (7, 15), (3, 9)], 2: [(0, 0), (3, 15), (1, 7)], 3: [(0, 0), (0, 15), (0, 6)]}
+
+
+@pytest.mark.parametrize("index", [1, 2, 3])
+def test_full_workload_sampled_heads(index):
+    wl = workloads.WORKLOADS[index]
+    x = workloads.draw_workload(index)
+    if wl.backward:
+        x["dST"] = torch.zeros(wl.B, wl.H, wl.dk, wl.dv)   # training: no gradient on S_T
+    gpu = gpu_fwd_bwd(x, wl.io, wl.chunk, backward=wl.backward)
+    ref = oracle_fwd_bwd(x, wl.io, backward=wl.backward, pairs=SAMPLE[index])
+    names = ("o", "ST") + (GRADS if wl.backward else ())
+    compare(gpu, ref, wl.io, names, pairs=SAMPLE[index])
+
+
+# ------------------------------------------------------------------ decode
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 32), (32, 128)])
+def test_decode_small_step_by_step(io, dk, dv):
+    N, H, steps = 3, 2, 12
+    S_gpu = (workloads.decode_state(N, H, dk, dv, 7, 0.3)).cuda()
+    S_ref = S_gpu.double().cpu().numpy()
+    dt = torch.bfloat16 if io == "bf16" else torch.float32
+    tol = TOL_F32 if io == "f32" else TOL_BF16_OUT
+    for s in range(steps):
+        x = workloads.decode_step_inputs(N, H, dk, dv, 7, s, erase_scale=2.0 if s % 2 else 1.0)
+        xr = io_round(x, io)
+        d = {n: (t.to(dt) if n in ("q", "k", "v") else t).cuda() for n, t in x.items()}
+        o = gdn.decode_step(d["q"], d["k"], d["v"], d["g"], d["b"], d["w"], S_gpu)
+        r = {n: t.double().numpy()[:, None] for n, t in xr.items()}
+        o_ref, S_ref = oracle.forward(r["q"], r["k"], r["v"], r["g"], r["b"], r["w"], S_ref)
+        assert rel(o.float().cpu().numpy(), o_ref[:, 0]) < tol, s
+        assert rel(S_gpu.cpu().numpy(), S_ref) < tol, s
+
+
+def test_decode_equals_chunked_forward():
+    """T decode steps reproduce the chunked forward's outputs and final state."""
+    B, T, H, dk, dv = 2, 40, 2, 128, 128
+    x = workloads.draw(B, T, H, dk, dv, 93, s0_std=0.1, with_dO=False)
+    d = to_device(x, "f32")
+    o, ST, _ = gdn.forward(*(d[n] for n in NAMES), chunk=16)
+    S = d["S0"].clone()
+    outs = []
+    for t in range(T):
+        outs.append(gdn.decode_step(*(d[n][:, t].contiguous() for n in NAMES[:-1]), S))
+    torch.cuda.synchronize()
+    assert rel(torch.stack(outs, 1).cpu().numpy(), o.cpu().numpy()) < TOL_F32
+    assert rel(S.cpu().numpy(), ST.cpu().numpy()) < TOL_F32
+
+
+def test_workload4_decode_sampled_every_step():
+    """256 sequences x 16 heads, 1024 consecutive steps, bf16 q/k/v, float32
+    state carried in HBM; sampled (sequence, head) pairs checked after every
+    step against the oracle stepped from the same state, never re-synchronised."""
+    wl = workloads.WORKLOADS[4]
+    N, H, dk, dv = wl.B, wl.H, wl.dk, wl.dv
+    pairs = [(0, 0), (255, 15), (100, 7), (17, 3)]
+    S = workloads.decode_state(N, H, dk, dv, wl.seed, wl.s0_std).cuda()
+    S_ref = np.stack([S[n, h].double().cpu().numpy() for n, h in pairs])[None]
+    worst_o = worst_S = 0.0
+    for s in range(wl.decode_steps):
+        x = workloads.decode_step_inputs(N, H, dk, dv, wl.seed, s)
+        d = {n: (t.to(torch.bfloat16) if n in ("q", "k", "v") else t).cuda() for n, t in x.items()}
+        o = gdn.decode_step(d["q"], d["k"], d["v"], d["g"], d["b"], d["w"], S)
+        xr = io_round(x, "bf16")
+        r = {n: np.stack([t[nn, hh].double().numpy() for nn, hh in pairs])[None, None]
+             for n, t in xr.items()}
+        o_ref, S_ref = oracle.forward(r["q"], r["k"], r["v"], r["g"], r["b"], r["w"], S_ref)
+        o_s = np.stack([o[nn, hh].float().cpu().numpy() for nn, hh in pairs])
+        worst_o = max(worst_o, rel(o_s, o_ref[0, 0]))
+        if s % 64 == 63 or s == wl.decode_steps - 1:
+            S_s = np.stack([S[nn, hh].cpu().numpy() for nn, hh in pairs])
+            worst_S = max(worst_S, rel(S_s, S_ref[0]))
+    assert worst_o < TOL_BF16_OUT and worst_S < TOL_BF16_OUT, (worst_o, worst_S)
