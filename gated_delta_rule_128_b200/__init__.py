@@ -66,6 +66,8 @@ def lib() -> ctypes.CDLL:
         L.gdn2_status_string.restype = ctypes.c_char_p
         L.gdn2_version.argtypes = []
         L.gdn2_version.restype = i
+        L.gdn2_fwd_noalloc.argtypes = [vp] * 9 + [i] * 7 + [vp]
+        L.gdn2_fwd_noalloc.restype = i
         L.gdn2_kernel_launches.argtypes = []
         L.gdn2_kernel_launches.restype = ctypes.c_ulonglong
         _lib = L
@@ -110,6 +112,12 @@ def gdn2_fwd(q, k, v, g, b, w, S0, o, ST, ws, ws_bytes, B, T, H, d_k, d_v, chunk
                         _ptr(ST), _ptr(ws), ws_bytes, B, T, H, d_k, d_v, chunk, io,
                         _stream(stream))
     _check("gdn2_fwd", rc)
+
+
+def gdn2_fwd_noalloc(q, k, v, g, b, w, S0, o, ST, B, T, H, d_k, d_v, chunk, io, stream=None):
+    rc = lib().gdn2_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b), _ptr(w), _ptr(S0),
+                                _ptr(o), _ptr(ST), B, T, H, d_k, d_v, chunk, io, _stream(stream))
+    _check("gdn2_fwd_noalloc", rc)
 
 
 def gdn2_bwd(q, k, v, g, b, w, S0, dO, dST, dq, dk, dv, dg, db, dw, dS0, ws, ws_bytes,

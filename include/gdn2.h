@@ -124,6 +124,34 @@ gdn2_status gdn2_decode_step(const void *q, const void *k, const void *v, const 
                              const float *b, const float *w, float *S, void *o, int N, int H,
                              int d_k, int d_v, gdn2_io io, gdn2_stream_t stream);
 
+/* Bytes of the scratch array behind gdn2_fwd_noalloc (64 MiB). */
+#define GDN2_NOALLOC_SCRATCH_BYTES (64u << 20)
+
+/* gdn2_fwd without a workspace argument, for callers that cannot allocate
+ * device memory.  The pages have no counterpart; it is a deployment aid.
+ * Examples: a plugin handed only input and output pointers by a host framework
+ * whose allocator owns all device memory, or a latency-critical path where the
+ * implicit device synchronisation of cudaMalloc/cudaFree is unacceptable.
+ * It computes the same forward as gdn2_fwd on the float32 CUDA-core path, and
+ * takes the same arguments minus ws and ws_bytes.
+ * Scratch: a file-scope device array of GDN2_NOALLOC_SCRATCH_BYTES, held by
+ *   every GPU that loads this library until the process exits.  The call
+ *   never calls cudaMalloc, cudaFree or any allocating routine.
+ * Limit: problems with gdn2_workspace_bytes(B, T, H, d_k, d_v, chunk, io, 0)
+ *   above GDN2_NOALLOC_SCRATCH_BYTES are rejected with GDN2_ERR_WORKSPACE
+ *   before anything is enqueued (e.g. d_k = d_v = 128, chunk 64: B*H*chunks
+ *   up to 292).
+ * Set-up: the first call on a device looks up the array's device address
+ *   (the current device must be the stream's device); make that first call
+ *   before any stream capture.
+ * Sharing: all calls use the same array, and it keeps the last call's
+ *   contents.  Calls whose work overlaps on the GPU (other streams, other
+ *   threads) race on it; serialise them. */
+gdn2_status gdn2_fwd_noalloc(const void *q, const void *k, const void *v, const float *g,
+                             const float *b, const float *w, const float *S0, void *o, float *ST,
+                             int B, int T, int H, int d_k, int d_v, int chunk, gdn2_io io,
+                             gdn2_stream_t stream);
+
 /* Waits for `stream`, then returns and clears the device status word: GDN2_OK,
  * or the first error a kernel recorded since the last call (GDN2_ERR_TIMEOUT).
  * Returns GDN2_ERR_CUDA if the stream reports a CUDA error. */
