@@ -30,7 +30,8 @@ LIB_PATH = os.path.join(PKG, "libgdn2.so")
 GDN2_IO_F32 = 0
 GDN2_IO_BF16 = 1
 STATUS = {0: "GDN2_OK", 1: "GDN2_ERR_INVALID_ARG", 2: "GDN2_ERR_UNSUPPORTED",
-          3: "GDN2_ERR_WORKSPACE", 4: "GDN2_ERR_CUDA", 5: "GDN2_ERR_TIMEOUT"}
+          3: "GDN2_ERR_WORKSPACE", 4: "GDN2_ERR_CUDA", 5: "GDN2_ERR_TIMEOUT",
+          6: "GDN2_ERR_RANGE"}
 
 
 class Gdn2Error(RuntimeError):

@@ -5,6 +5,7 @@
 #include <stdint.h>
 
 #include <atomic>
+#include <mutex>
 
 #include "common.cuh"
 
@@ -25,8 +26,32 @@ cudaError_t simt_bwd_launch(const void *, const void *, const void *, const floa
 cudaError_t decode_launch(const void *, const void *, const void *, const float *, const float *,
                           const float *, float *, void *, int, int, int, int, gdn2_io,
                           cudaStream_t);
+size_t tc_fwd_ckpt_bytes(const Dims &d);
+cudaError_t tc_fwd_launch(const void *, const void *, const void *, const float *, const float *,
+                          const float *, const float *, void *, float *, void *, unsigned int *,
+                          const Dims &, cudaStream_t);
 
 __device__ unsigned int g_status_word;
+
+// device address of g_status_word on the current device (looked up once per device)
+static unsigned int *status_word() {
+    static unsigned int *addr[64];
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+        addr[dev] = static_cast<unsigned int *>(p);
+    }
+    return addr[dev];
+}
+
+// the tensor-core path: bf16 I/O, d_k = d_v = 128, chunk 64
+static bool use_tc(const Dims &d, gdn2_io io) {
+    return io == GDN2_IO_BF16 && d.dk == 128 && d.dv == 128 && d.C == 64;
+}
 
 static std::atomic<unsigned long long> g_launches{0};
 void count_launches(unsigned long long n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
@@ -84,11 +109,20 @@ using namespace gdn2;
 
 extern "C" {
 
+static size_t ws_bytes_for(const Dims &d, gdn2_io io, int for_bwd) {
+    SimtWs lay = simt_ws_layout(d);
+    if (use_tc(d, io)) {
+        if (!for_bwd) return 256;  // the tensor-core forward keeps nothing between phases
+        size_t a = tc_fwd_ckpt_bytes(d), b = lay.bwd_end;
+        return a > b ? a : b;
+    }
+    return for_bwd ? lay.bwd_end : lay.fwd_end;
+}
+
 size_t gdn2_workspace_bytes(int B, int T, int H, int d_k, int d_v, int chunk, gdn2_io io,
                             int for_bwd) {
     if (check_dims(B, T, H, d_k, d_v, chunk, io) != GDN2_OK) return 0;
-    SimtWs lay = simt_ws_layout(make_dims(B, T, H, d_k, d_v, chunk));
-    return for_bwd ? lay.bwd_end : lay.fwd_end;
+    return ws_bytes_for(make_dims(B, T, H, d_k, d_v, chunk), io, for_bwd);
 }
 
 gdn2_status gdn2_fwd(const void *q, const void *k, const void *v, const float *g, const float *b,
@@ -100,7 +134,14 @@ gdn2_status gdn2_fwd(const void *q, const void *k, const void *v, const float *g
     st = check_ptrs({q, k, v, g, b, w, o}, {S0, ST});
     if (st != GDN2_OK) return st;
     Dims d = make_dims(B, T, H, d_k, d_v, chunk);
-    if (!ws || !aligned16(ws) || ws_bytes < simt_ws_layout(d).fwd_end) return GDN2_ERR_WORKSPACE;
+    if (!ws || !aligned16(ws) || ws_bytes < ws_bytes_for(d, io, 0)) return GDN2_ERR_WORKSPACE;
+    if (use_tc(d, io)) {
+        unsigned int *status = status_word();
+        if (!status) return GDN2_ERR_CUDA;
+        void *ckpt = (ws && ws_bytes >= ws_bytes_for(d, io, 1)) ? ws : nullptr;
+        return cuda_status(tc_fwd_launch(q, k, v, g, b, w, S0, o, ST, ckpt, status, d,
+                                         (cudaStream_t)stream));
+    }
     return cuda_status(run_forward(q, k, v, g, b, w, S0, o, ST, ws, d, io, (cudaStream_t)stream));
 }
 
@@ -114,9 +155,11 @@ gdn2_status gdn2_bwd(const void *q, const void *k, const void *v, const float *g
     st = check_ptrs({q, k, v, g, b, w, dO, dq, dk, dv, dg, db, dw}, {S0, dST, dS0});
     if (st != GDN2_OK) return st;
     Dims d = make_dims(B, T, H, d_k, d_v, chunk);
-    if (!ws || !aligned16(ws) || ws_bytes < simt_ws_layout(d).bwd_end) return GDN2_ERR_WORKSPACE;
+    if (!ws || !aligned16(ws) || ws_bytes < ws_bytes_for(d, io, 1)) return GDN2_ERR_WORKSPACE;
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e;
+    // the float32 backward below needs the float32 forward's tiles
+    if (use_tc(d, io)) ws_has_fwd = 0;
     if (!ws_has_fwd) {
         e = run_forward(q, k, v, g, b, w, S0, nullptr, nullptr, ws, d, io, s);
         if (e != cudaSuccess) return GDN2_ERR_CUDA;
@@ -158,6 +201,7 @@ const char *gdn2_status_string(gdn2_status status) {
         case GDN2_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
         case GDN2_ERR_CUDA: return "CUDA error";
         case GDN2_ERR_TIMEOUT: return "a kernel gave up on a bounded wait";
+        case GDN2_ERR_RANGE: return "input outside the tensor-core path's range (see gdn2.h)";
     }
     return "unknown status";
 }

@@ -1,0 +1,547 @@
+// Fused chunkwise forward of Gated Delta Rule-2 on the sm_100a tensor cores,
+// for bf16 q/k/v/o, float32 gates and state, d_k = d_v = 128, chunk 64.
+//
+// "Gated DeltaNet-2" (LIT-802 review, Key takeaways 2; paper Secs. 3.3-3.4,
+// Apps. A-B): the state is normalised by the in-chunk cumulative decay, so the
+// channel-wise decay folds into the two factors of every rank-one erase, one
+// WY/UT inverse serves the erase and the write side, and only the state
+// crosses chunk borders.  Per chunk of 64 tokens entering with state S:
+//   G = cumsum(g);  Qb = q.e^G,  Kc = b.k.e^G,  Kh = k.e^-G,  U = w.v
+//   A = strictly-lower(Kc Kh^T),  P = lower-incl(Qb Kh^T),  T = (I + A)^-1
+//   W = T Kc,  U' = T U,  Delta = U' - W S
+//   O = Qb S + P Delta,   S_next = diag(e^G_L) (S + Kh^T Delta)
+//
+// One CTA owns one (b, h) and one 64-column half of d_v, and walks the
+// sequence's chunks in order with its fp32 state slice resident in tensor
+// memory.  Per chunk: TMA brings the raw q, k, v, w, g, b tiles into shared
+// memory (the next chunk's tiles are requested as soon as this chunk's are
+// consumed); the CUDA cores form the decay-scaled fp16 operands; seven
+// tcgen05.mma groups (kind::f16 with fp16 operands, f32 accumulators in TMEM)
+// form A, P, QbS, W|U', WS, P Delta and Kh^T Delta; the unit-lower-triangular
+// T is inverted in float32 on the CUDA cores by blocked forward substitution
+// (16x16 diagonal blocks, then three block levels).  The fp16 copy of each
+// chunk-entry state is written to the workspace for the backward pass.
+//
+// Precision and range: fp16 operands carry 11 significant bits (bf16 carries
+// 8, which left the output error at the 5e-3 tolerance).  To keep them in
+// fp16 range the decay factors are taken relative to the chunk's middle row
+// m = 31: Qb = q.e^(G-G_m), Kc = b.k.e^(G-G_m), Kh = k.e^(G_m-G); the state
+// products then use S_m = diag(e^G_m) S, and the update becomes
+// S_next = diag(e^(G_L-G_m)) (S_m + Kh^T Delta).  Any operand beyond 6e4 in
+// magnitude is reported as GDN2_ERR_RANGE.
+
+#include "common.cuh"
+#include "tc.cuh"
+#include "tmap.cuh"
+
+namespace gdn2 {
+using namespace tc;
+
+namespace tfwd {
+constexpr int kThreads = 256;
+// shared memory map (bytes from a 1024-aligned base)
+constexpr uint32_t RAW_Q = 0, RAW_K = 16384, RAW_V = 32768, RAW_W = 40960, RAW_G = 57344,
+                   RAW_B = 90112;
+constexpr uint32_t OP_KC = 122880;  // Kc, later W        [64 pos][128 key]  K-major
+constexpr uint32_t OP_QB = 139264;  // Qb                 [64 pos][128 key]
+constexpr uint32_t OP_KH = 155648;  // Kh                 [64 pos][128 key]
+constexpr uint32_t OP_S = 172032;   // S (fp16)           [128 key][64 v]    MN-major B
+constexpr uint32_t OP_U = 188416;   // U, later Delta     [64 pos][64 v]     MN-major B
+constexpr uint32_t OP_T = 196608;   // T                  [64 r][64 j]       K-major
+constexpr uint32_t OP_P = 204800;   // P                  [64 r][64 j]       K-major
+constexpr uint32_t MISC = 212992;   // e^(G_L-G_m), e^G_m [128] f32 each, mbarriers, TMEM slot
+constexpr uint32_t SMEM_BYTES = MISC + 1024 + 128 + 1024;
+// float32 scratch while inverting T (inside the raw g/b tiles, reloaded after)
+constexpr uint32_t SCR_A = RAW_G, SCR_T = RAW_G + 64 * 65 * 4, SCR_M = SCR_T + 64 * 65 * 4;
+constexpr uint32_t SCR_SCAN = OP_T;  // per-warp cumsum totals [8][128] f32 during phase 1
+// tensor memory columns (512 allocated)
+constexpr uint32_t TM_S = 0, TM_A = 64, TM_P = 128, TM_WU = 192, TM_WS = 384, TM_O = 448;
+constexpr uint32_t ID_KK64 = idesc_f16(64, 64, false, false);
+constexpr uint32_t ID_KM64 = idesc_f16(64, 64, false, true);
+constexpr uint32_t ID_KM128 = idesc_f16(64, 128, false, true);
+constexpr uint32_t ID_MM128x64 = idesc_f16(128, 64, true, true);
+constexpr long long kWait = 2000000000LL;  // ~1 s of SM clocks per wait
+constexpr float kRange = 6.0e4f;           // largest operand magnitude kept in fp16
+}  // namespace tfwd
+
+__device__ __forceinline__ void st_h4(unsigned char *p, float a, float b, float c, float d) {
+    uint2 v = make_uint2(pack_f16(a, b), pack_f16(c, d));
+    *reinterpret_cast<uint2 *>(p) = v;
+}
+__device__ __forceinline__ void st_h8(unsigned char *p, const float *x) {
+    uint4 v = make_uint4(pack_f16(x[0], x[1]), pack_f16(x[2], x[3]), pack_f16(x[4], x[5]),
+                         pack_f16(x[6], x[7]));
+    *reinterpret_cast<uint4 *>(p) = v;
+}
+__device__ __forceinline__ float absmax8(const float *x, float m) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(x[i]));
+    return m;
+}
+__device__ __forceinline__ void st_bf16x8(unsigned char *p, const float *x) {
+    uint4 v = make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]),
+                         pack_bf16(x[6], x[7]));
+    *reinterpret_cast<uint4 *>(p) = v;
+}
+
+__global__ void __launch_bounds__(tfwd::kThreads, 1)
+tc_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
+              const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mg,
+              const __grid_constant__ CUtensorMap mb, const __grid_constant__ CUtensorMap mw,
+              const float *__restrict__ S0, __nv_bfloat16 *__restrict__ o, float *__restrict__ ST,
+              __nv_bfloat16 *__restrict__ ckpt, unsigned int *status, Dims d) {
+    using namespace tfwd;
+    extern __shared__ unsigned char smraw[];
+    unsigned char *sm = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smraw) + 1023) & ~static_cast<uintptr_t>(1023));
+    float *sGam = reinterpret_cast<float *>(sm + MISC);        // e^(G_L - G_m)
+    float *sRef = reinterpret_cast<float *>(sm + MISC + 512);  // e^G_m
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + MISC + 1024);  // 0 qkvw, 1 gb, 2..5 mma
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + MISC + 1024 + 64);
+    float big = 0.f;  // largest operand magnitude seen (range check)
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int vh = blockIdx.x, h = blockIdx.y, bb = blockIdx.z, v0 = vh * 64;
+    const int NC = d.NC, T = d.T, H = d.H;
+    const int quarter = warp & 3, half = warp >> 2;
+
+    if (warp == 0) {
+        tmem_alloc(tslot, 512);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        for (int i = 0; i < 6; ++i) mbar_init(&bars[i], 1);
+        mbar_fence_init();
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tm = *tslot;
+
+    int issued_qkvw = 0, issued_gb = 0;  // loads requested so far (thread 0)
+    auto load_qkvw = [&](int cc) {
+        mbar_expect_tx(&bars[0], 16384 * 2 + 8192 + 16384);
+        tma_load_4d(sm + RAW_Q, &mq, 0, h, cc * 64, bb, &bars[0]);
+        tma_load_4d(sm + RAW_K, &mk, 0, h, cc * 64, bb, &bars[0]);
+        tma_load_4d(sm + RAW_V, &mv, v0, h, cc * 64, bb, &bars[0]);
+        tma_load_4d(sm + RAW_W, &mw, v0, h, cc * 64, bb, &bars[0]);
+        ++issued_qkvw;
+    };
+    auto load_gb = [&](int cc) {
+        mbar_expect_tx(&bars[1], 32768 * 2);
+        tma_load_4d(sm + RAW_G, &mg, 0, h, cc * 64, bb, &bars[1]);
+        tma_load_4d(sm + RAW_B, &mb, 0, h, cc * 64, bb, &bars[1]);
+        ++issued_gb;
+    };
+    if (tid == 0) {
+        load_qkvw(0);
+        load_gb(0);
+    }
+
+    const size_t so = st_off(d, bb, h);
+    // initial state slice: fp32 into TMEM, fp16 into OP_S
+    {
+        const int key = quarter * 32 + lane, c0 = half * 32;
+        float x[32];
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) {
+            float4 t = S0 ? *reinterpret_cast<const float4 *>(S0 + so + (size_t)key * 128 + v0 + c0 + j)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+            x[j] = t.x; x[j + 1] = t.y; x[j + 2] = t.z; x[j + 3] = t.w;
+        }
+        tmem_st16(taddr(tm + TM_S, quarter * 32, c0), x);
+        tmem_st16(taddr(tm + TM_S, quarter * 32, c0 + 16), x + 16);
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+            st_h8(sm + OP_S + sw128_chunk(key, half * 4 + jj, 128), x + 8 * jj);
+            big = absmax8(x + 8 * jj, big);
+        }
+        tmem_wait_st();
+    }
+    fence_proxy_async();
+    fence_before_sync();
+    __syncthreads();
+    const size_t ck_head = ((size_t)bb * H + h) * NC;
+    if (tid == 0 && ckpt) {
+        bulk_store(ckpt + ((ck_head + 0) * 2 + vh) * 8192, sm + OP_S, 16384);
+        bulk_commit();
+    }
+
+    bool abort = false;
+    int c = 0;
+    for (; c < NC; ++c) {
+        const uint32_t par = c & 1;
+        const int c0 = c * 64;
+        // ---------------- phase 1: cumulative decay and operands
+        bool ok = mbar_wait(&bars[0], par, kWait);
+        ok = ok && mbar_wait(&bars[1], par, kWait);
+        float G[8][4];
+        {
+            const float *rg = reinterpret_cast<const float *>(sm + RAW_G);
+            float run[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+                float4 t = *reinterpret_cast<const float4 *>(rg + (8 * warp + m) * 128 + 4 * lane);
+                run[0] += t.x; run[1] += t.y; run[2] += t.z; run[3] += t.w;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) G[m][i] = run[i];
+            }
+            float *scan = reinterpret_cast<float *>(sm + SCR_SCAN);
+            *reinterpret_cast<float4 *>(scan + warp * 128 + 4 * lane) =
+                make_float4(run[0], run[1], run[2], run[3]);
+        }
+        if (__syncthreads_or(!ok)) { abort = true; break; }
+        {
+            const float *scan = reinterpret_cast<const float *>(sm + SCR_SCAN);
+            float pre[4] = {0.f, 0.f, 0.f, 0.f}, tot[4] = {0.f, 0.f, 0.f, 0.f};
+            float ref[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int w2 = 0; w2 < 8; ++w2) {
+                float4 t = *reinterpret_cast<const float4 *>(scan + w2 * 128 + 4 * lane);
+                float tv[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    if (w2 < warp) pre[i] += tv[i];
+                    if (w2 < 4) ref[i] += tv[i];   // G at row 31
+                    tot[i] += tv[i];
+                }
+            }
+            // G relative to the reference row
+#pragma unroll
+            for (int m = 0; m < 8; ++m)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) G[m][i] += pre[i] - ref[i];
+            if (warp == 0)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    sGam[4 * lane + i] = __expf(tot[i] - ref[i]);
+                    sRef[4 * lane + i] = __expf(ref[i]);
+                }
+        }
+        {
+            const unsigned char *rq = sm + RAW_Q, *rk = sm + RAW_K;
+            const float *rb = reinterpret_cast<const float *>(sm + RAW_B);
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+                const int r = 8 * warp + m;
+                uint2 qr = *reinterpret_cast<const uint2 *>(rq + r * 256 + lane * 8);
+                uint2 kr = *reinterpret_cast<const uint2 *>(rk + r * 256 + lane * 8);
+                float4 bv = *reinterpret_cast<const float4 *>(rb + r * 128 + 4 * lane);
+                const __nv_bfloat162 *q2 = reinterpret_cast<const __nv_bfloat162 *>(&qr);
+                const __nv_bfloat162 *k2 = reinterpret_cast<const __nv_bfloat162 *>(&kr);
+                float qf[4] = {__low2float(q2[0]), __high2float(q2[0]), __low2float(q2[1]), __high2float(q2[1])};
+                float kf[4] = {__low2float(k2[0]), __high2float(k2[0]), __low2float(k2[1]), __high2float(k2[1])};
+                float bf[4] = {bv.x, bv.y, bv.z, bv.w};
+                float qb[4], kc[4], kh[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float ep = __expf(G[m][i]), em = __expf(-G[m][i]);
+                    qb[i] = qf[i] * ep;
+                    kc[i] = bf[i] * kf[i] * ep;
+                    kh[i] = kf[i] * em;
+                }
+                const uint32_t off = sw128_off(r, 4 * lane, 64);
+                st_h4(sm + OP_QB + off, qb[0], qb[1], qb[2], qb[3]);
+                st_h4(sm + OP_KC + off, kc[0], kc[1], kc[2], kc[3]);
+                st_h4(sm + OP_KH + off, kh[0], kh[1], kh[2], kh[3]);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    big = fmaxf(big, fmaxf(fabsf(qb[i]), fmaxf(fabsf(kc[i]), fabsf(kh[i]))));
+                if (lane < 16) {
+                    uint2 vr = *reinterpret_cast<const uint2 *>(sm + RAW_V + r * 128 + lane * 8);
+                    float4 wv = *reinterpret_cast<const float4 *>(sm + RAW_W + r * 256 + lane * 16);
+                    const __nv_bfloat162 *v2 = reinterpret_cast<const __nv_bfloat162 *>(&vr);
+                    float u[4] = {wv.x * __low2float(v2[0]), wv.y * __high2float(v2[0]),
+                                  wv.z * __low2float(v2[1]), wv.w * __high2float(v2[1])};
+                    st_h4(sm + OP_U + sw128_off(r, 4 * lane, 64), u[0], u[1], u[2], u[3]);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) big = fmaxf(big, fabsf(u[i]));
+                }
+            }
+        }
+        if (tid == 0 && ckpt) bulk_wait_read();  // OP_S is rewritten just below
+        __syncthreads();
+        // state in the chunk's reference frame: S_m = diag(e^G_m) S (TMEM and fp16 copy)
+        {
+            const int key = quarter * 32 + lane;
+            float sv[32];
+            tmem_ld16(taddr(tm + TM_S, quarter * 32, 32 * half), sv);
+            tmem_ld16(taddr(tm + TM_S, quarter * 32, 32 * half + 16), sv + 16);
+            tmem_wait_ld();
+            const float e = sRef[key];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) sv[j] *= e;
+            tmem_st16(taddr(tm + TM_S, quarter * 32, 32 * half), sv);
+            tmem_st16(taddr(tm + TM_S, quarter * 32, 32 * half + 16), sv + 16);
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                st_h8(sm + OP_S + sw128_chunk(key, 4 * half + jj, 128), sv + 8 * jj);
+                big = absmax8(sv + 8 * jj, big);
+            }
+            tmem_wait_st();
+        }
+        fence_proxy_async();
+        fence_before_sync();
+        __syncthreads();
+        if (tid == 0) {
+            fence_after_sync();
+            if (c + 1 < NC) load_qkvw(c + 1);
+            const uint32_t kc = smem_addr(sm + OP_KC), qb = smem_addr(sm + OP_QB),
+                           kh = smem_addr(sm + OP_KH), s = smem_addr(sm + OP_S);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                mma_bf16(tm + TM_A, desc_kmajor(kc, 64, ks), desc_kmajor(kh, 64, ks), ID_KK64, ks > 0);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                mma_bf16(tm + TM_P, desc_kmajor(qb, 64, ks), desc_kmajor(kh, 64, ks), ID_KK64, ks > 0);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                mma_bf16(tm + TM_O, desc_kmajor(qb, 64, ks), desc_mnmajor(s, 128, ks), ID_KM64, ks > 0);
+            mma_commit(&bars[2]);
+        }
+        // ---------------- phase 3: T = (I + A)^-1 and the masked P
+        ok = mbar_wait(&bars[2], par, kWait);
+        fence_after_sync();
+        float *sA = reinterpret_cast<float *>(sm + SCR_A);
+        float *sT = reinterpret_cast<float *>(sm + SCR_T);
+        {
+            float row[64];
+            const uint32_t base = warp < 4 ? tm + TM_A : tm + TM_P;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) tmem_ld16(taddr(base, quarter * 32, 16 * j), row + 16 * j);
+            tmem_wait_ld();
+            if (lane < 16) {
+                const int r = quarter * 16 + lane;
+                if (warp < 4) {
+#pragma unroll
+                    for (int j = 0; j < 64; ++j) sA[r * 65 + j] = j < r ? row[j] : 0.f;
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 64; ++j) row[j] = j <= r ? row[j] : 0.f;
+#pragma unroll
+                    for (int jj = 0; jj < 8; ++jj) {
+                        st_h8(sm + OP_P + sw128_chunk(r, jj, 64), row + 8 * jj);
+                        big = absmax8(row + 8 * jj, big);
+                    }
+                }
+            }
+        }
+        if (__syncthreads_or(!ok)) { abort = true; break; }
+        // diagonal 16x16 blocks, one column per thread; zero the upper blocks
+        if (tid < 64) {
+            const int o16 = (tid >> 4) * 16, cl = tid & 15;
+            float x[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                float acc = r == cl ? 1.f : 0.f;
+#pragma unroll
+                for (int j = 0; j < r; ++j) acc -= sA[(o16 + r) * 65 + o16 + j] * x[j];
+                x[r] = acc;
+            }
+#pragma unroll
+            for (int r = 0; r < 16; ++r) sT[(o16 + r) * 65 + o16 + cl] = x[r];
+        }
+        for (int e = tid; e < 64 * 64; e += kThreads) {
+            const int r = e >> 6, j = e & 63;
+            if ((j >> 4) > (r >> 4)) sT[r * 65 + j] = 0.f;
+        }
+        __syncthreads();
+        // block levels: T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ, I - J = lvl
+        float *sM = reinterpret_cast<float *>(sm + SCR_M);
+        for (int lvl = 1; lvl < 4; ++lvl) {
+            const int nb = 4 - lvl;
+            for (int e = tid; e < nb * 256; e += kThreads) {
+                const int bi = e >> 8, r = (e >> 4) & 15, cl = e & 15;
+                const int I = bi + lvl, J = bi;
+                float acc = 0.f;
+                for (int K = J; K < I; ++K)
+#pragma unroll
+                    for (int kk = 0; kk < 16; ++kk)
+                        acc += sA[(16 * I + r) * 65 + 16 * K + kk] * sT[(16 * K + kk) * 65 + 16 * J + cl];
+                sM[bi * 272 + r * 17 + cl] = acc;
+            }
+            __syncthreads();
+            for (int e = tid; e < nb * 256; e += kThreads) {
+                const int bi = e >> 8, r = (e >> 4) & 15, cl = e & 15;
+                const int I = bi + lvl, J = bi;
+                float acc = 0.f;
+#pragma unroll
+                for (int kk = 0; kk < 16; ++kk)
+                    acc += sT[(16 * I + r) * 65 + 16 * I + kk] * sM[bi * 272 + kk * 17 + cl];
+                sT[(16 * I + r) * 65 + 16 * J + cl] = -acc;
+            }
+            __syncthreads();
+        }
+        for (int e = tid; e < 64 * 8; e += kThreads) {
+            const int r = e >> 3, jj = e & 7;
+            st_h8(sm + OP_T + sw128_chunk(r, jj, 64), sT + r * 65 + 8 * jj);
+            big = absmax8(sT + r * 65 + 8 * jj, big);
+        }
+        fence_proxy_async();
+        fence_before_sync();
+        __syncthreads();
+        if (tid == 0) {
+            fence_after_sync();
+            if (c + 1 < NC) load_gb(c + 1);
+            const uint32_t t = smem_addr(sm + OP_T), kc = smem_addr(sm + OP_KC),
+                           u = smem_addr(sm + OP_U);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(tm + TM_WU, desc_kmajor(t, 64, ks), desc_mnmajor(kc, 64, ks), ID_KM128, ks > 0);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(tm + TM_WU + 128, desc_kmajor(t, 64, ks), desc_mnmajor(u, 64, ks), ID_KM64, ks > 0);
+            mma_commit(&bars[3]);
+        }
+        // ---------------- phase 5: W to shared memory (keep U' in registers)
+        ok = mbar_wait(&bars[3], par, kWait);
+        fence_after_sync();
+        float up[32];
+        {
+            float wv[64];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) tmem_ld16(taddr(tm + TM_WU, quarter * 32, 64 * half + 16 * j), wv + 16 * j);
+            tmem_ld16(taddr(tm + TM_WU, quarter * 32, 128 + 32 * half), up);
+            tmem_ld16(taddr(tm + TM_WU, quarter * 32, 128 + 32 * half + 16), up + 16);
+            tmem_wait_ld();
+            if (lane < 16) {
+                const int r = quarter * 16 + lane;
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj) {
+                    st_h8(sm + OP_KC + sw128_chunk(r, 8 * half + jj, 64), wv + 8 * jj);
+                    big = absmax8(wv + 8 * jj, big);
+                }
+            }
+        }
+        fence_proxy_async();
+        fence_before_sync();
+        if (__syncthreads_or(!ok)) { abort = true; break; }
+        if (tid == 0) {
+            fence_after_sync();
+            const uint32_t w = smem_addr(sm + OP_KC), s = smem_addr(sm + OP_S);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                mma_bf16(tm + TM_WS, desc_kmajor(w, 64, ks), desc_mnmajor(s, 128, ks), ID_KM64, ks > 0);
+            mma_commit(&bars[4]);
+        }
+        // ---------------- phase 7: Delta = U' - W S
+        ok = mbar_wait(&bars[4], par, kWait);
+        fence_after_sync();
+        {
+            float ws[32];
+            tmem_ld16(taddr(tm + TM_WS, quarter * 32, 32 * half), ws);
+            tmem_ld16(taddr(tm + TM_WS, quarter * 32, 32 * half + 16), ws + 16);
+            tmem_wait_ld();
+            if (lane < 16) {
+                const int r = quarter * 16 + lane;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) ws[j] = up[j] - ws[j];
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    st_h8(sm + OP_U + sw128_chunk(r, 4 * half + jj, 64), ws + 8 * jj);
+                    big = absmax8(ws + 8 * jj, big);
+                }
+            }
+        }
+        fence_proxy_async();
+        fence_before_sync();
+        if (__syncthreads_or(!ok)) { abort = true; break; }
+        if (tid == 0) {
+            fence_after_sync();
+            const uint32_t p = smem_addr(sm + OP_P), dl = smem_addr(sm + OP_U),
+                           kh = smem_addr(sm + OP_KH);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(tm + TM_O, desc_kmajor(p, 64, ks), desc_mnmajor(dl, 64, ks), ID_KM64, 1);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(tm + TM_S, desc_mnmajor(kh, 64, ks), desc_mnmajor(dl, 64, ks), ID_MM128x64, 1);
+            mma_commit(&bars[5]);
+        }
+        // ---------------- phase 9: output rows, state update and checkpoint
+        ok = mbar_wait(&bars[5], par, kWait);
+        fence_after_sync();
+        {
+            float ov[32];
+            tmem_ld16(taddr(tm + TM_O, quarter * 32, 32 * half), ov);
+            tmem_ld16(taddr(tm + TM_O, quarter * 32, 32 * half + 16), ov + 16);
+            tmem_wait_ld();
+            if (lane < 16) {
+                const int r = quarter * 16 + lane;
+                if (c0 + r < T) {
+                    unsigned char *dst = reinterpret_cast<unsigned char *>(
+                        o + tok(d, bb, c0 + r, h, 128) + v0 + 32 * half);
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) st_bf16x8(dst + 16 * jj, ov + 8 * jj);
+                }
+            }
+            const int key = quarter * 32 + lane;
+            float sv[32];
+            tmem_ld16(taddr(tm + TM_S, quarter * 32, 32 * half), sv);
+            tmem_ld16(taddr(tm + TM_S, quarter * 32, 32 * half + 16), sv + 16);
+            tmem_wait_ld();
+            const float gk = sGam[key];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) sv[j] *= gk;
+            tmem_st16(taddr(tm + TM_S, quarter * 32, 32 * half), sv);
+            tmem_st16(taddr(tm + TM_S, quarter * 32, 32 * half + 16), sv + 16);
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                st_h8(sm + OP_S + sw128_chunk(key, 4 * half + jj, 128), sv + 8 * jj);
+                big = absmax8(sv + 8 * jj, big);
+            }
+            if (c == NC - 1 && ST) {
+                float *dst = ST + so + (size_t)key * 128 + v0 + 32 * half;
+#pragma unroll
+                for (int j = 0; j < 32; j += 4)
+                    *reinterpret_cast<float4 *>(dst + j) = make_float4(sv[j], sv[j + 1], sv[j + 2], sv[j + 3]);
+            }
+            tmem_wait_st();
+        }
+        fence_proxy_async();
+        fence_before_sync();
+        if (__syncthreads_or(!ok)) { abort = true; break; }
+        if (tid == 0 && ckpt && c + 1 < NC) {
+            bulk_store(ckpt + ((ck_head + c + 1) * 2 + vh) * 8192, sm + OP_S, 16384);
+            bulk_commit();
+        }
+    }
+    if (!(big <= kRange)) record_status(status, GDN2_ERR_RANGE);
+    if (tid == 0) {
+        if (ckpt) bulk_wait_all();
+        if (abort) {
+            record_status(status, GDN2_ERR_TIMEOUT);
+            // let every requested tile land before the CTA's shared memory goes away
+            if (issued_qkvw > 0) mbar_wait(&bars[0], (issued_qkvw - 1) & 1, kWait);
+            if (issued_gb > 0) mbar_wait(&bars[1], (issued_gb - 1) & 1, kWait);
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tm, 512);
+}
+
+// ---------------------------------------------------------------- launcher
+size_t tc_fwd_ckpt_bytes(const Dims &d) { return (size_t)d.B * d.H * d.NC * 2 * 16384; }
+
+cudaError_t tc_fwd_launch(const void *q, const void *k, const void *v, const float *g,
+                          const float *b, const float *w, const float *S0, void *o, float *ST,
+                          void *ckpt, unsigned int *status, const Dims &d, cudaStream_t s) {
+    CUtensorMap mq, mk, mv, mg, mb, mw;
+    if (!make_btHd_map(&mq, q, true, d.B, d.T, d.H, 128, 64, 128) ||
+        !make_btHd_map(&mk, k, true, d.B, d.T, d.H, 128, 64, 128) ||
+        !make_btHd_map(&mv, v, true, d.B, d.T, d.H, 128, 64, 64) ||
+        !make_btHd_map(&mg, g, false, d.B, d.T, d.H, 128, 64, 128) ||
+        !make_btHd_map(&mb, b, false, d.B, d.T, d.H, 128, 64, 128) ||
+        !make_btHd_map(&mw, w, false, d.B, d.T, d.H, 128, 64, 64))
+        return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(tc_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)tfwd::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    count_launches(1);
+    tc_fwd_kernel<<<dim3(2, d.H, d.B), tfwd::kThreads, tfwd::SMEM_BYTES, s>>>(
+        mq, mk, mv, mg, mb, mw, S0, (__nv_bfloat16 *)o, ST, (__nv_bfloat16 *)ckpt, status, d);
+    return cudaGetLastError();
+}
+
+}  // namespace gdn2

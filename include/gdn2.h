@@ -40,6 +40,15 @@
  *   returns GDN2_ERR_CUDA.  Kernels never trap: a kernel that gives up on a
  *   bounded wait records GDN2_ERR_TIMEOUT in a device status word that
  *   gdn2_get_device_status reports.
+ * Paths: bf16 I/O with d_k = d_v = 128 and chunk 64 runs on the tensor cores
+ *   (fp16 operands, fp32 accumulation and state); every other combination
+ *   runs on the float32 CUDA-core path.  The tensor-core path forms the decay
+ *   factors relative to the middle of each chunk, so it needs every key
+ *   channel's cumulative log-decay to move by at most 9 within any 32-token
+ *   half-chunk (and |q|, |k| <= 8 per element, |w v| and the state below
+ *   6e4); a kernel that meets an input outside that range records
+ *   GDN2_ERR_RANGE (the results of that call are then not valid).  The
+ *   float32 path has no such limit.
  */
 #ifndef GDN2_H
 #define GDN2_H
@@ -60,7 +69,8 @@ typedef enum {
     GDN2_ERR_UNSUPPORTED = 2,  /* d_k, d_v or chunk outside the supported set  */
     GDN2_ERR_WORKSPACE = 3,    /* workspace missing or smaller than required   */
     GDN2_ERR_CUDA = 4,         /* a CUDA launch or runtime call failed          */
-    GDN2_ERR_TIMEOUT = 5       /* a kernel gave up on a bounded wait            */
+    GDN2_ERR_TIMEOUT = 5,      /* a kernel gave up on a bounded wait            */
+    GDN2_ERR_RANGE = 6         /* inputs outside the tensor-core path's range   */
 } gdn2_status;
 
 typedef enum {
@@ -69,8 +79,8 @@ typedef enum {
 } gdn2_io;
 
 /* Bytes of caller-provided device workspace that gdn2_fwd (for_bwd = 0) or
- * gdn2_fwd followed by gdn2_bwd (for_bwd = 1) needs for these sizes.  Returns
- * 0 when the sizes are unsupported.  A workspace sized with for_bwd = 1 also
+ * gdn2_fwd followed by gdn2_bwd (for_bwd = 1) needs for these sizes (at
+ * least 256).  Returns 0 when the sizes are unsupported.  A workspace sized with for_bwd = 1 also
  * serves gdn2_fwd, and then keeps what gdn2_bwd can reuse (see ws_has_fwd). */
 size_t gdn2_workspace_bytes(int B, int T, int H, int d_k, int d_v, int chunk, gdn2_io io,
                             int for_bwd);
@@ -137,10 +147,11 @@ gdn2_status gdn2_decode_step(const void *q, const void *k, const void *v, const 
  * Scratch: a file-scope device array of GDN2_NOALLOC_SCRATCH_BYTES, held by
  *   every GPU that loads this library until the process exits.  The call
  *   never calls cudaMalloc, cudaFree or any allocating routine.
- * Limit: problems with gdn2_workspace_bytes(B, T, H, d_k, d_v, chunk, io, 0)
- *   above GDN2_NOALLOC_SCRATCH_BYTES are rejected with GDN2_ERR_WORKSPACE
- *   before anything is enqueued (e.g. d_k = d_v = 128, chunk 64: B*H*chunks
- *   up to 292).
+ * Limit: problems whose float32-path workspace,
+ *   gdn2_workspace_bytes(B, T, H, d_k, d_v, chunk, GDN2_IO_F32, 0), exceeds
+ *   GDN2_NOALLOC_SCRATCH_BYTES are rejected with GDN2_ERR_WORKSPACE before
+ *   anything is enqueued (e.g. d_k = d_v = 128, chunk 64: B*H*chunks up to
+ *   292), whatever the io type.
  * Set-up: the first call on a device looks up the array's device address
  *   (the current device must be the stream's device); make that first call
  *   before any stream capture.

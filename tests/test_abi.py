@@ -50,7 +50,7 @@ def test_library_links_no_torch(L):
 
 
 def test_status_strings_and_version(L):
-    for s in range(6):
+    for s in range(7):
         assert len(L.gdn2_status_string(s)) > 0
     assert L.gdn2_status_string(99) == b"unknown status"
     assert L.gdn2_version() >= 100

@@ -24,8 +24,9 @@ def test_noalloc_rejects_problems_beyond_its_scratch():
     L = gdn.lib()
     limit = 64 << 20
     # d = 128, chunk 64: 292 chunk tiles fit, 293 do not
-    assert gdn.gdn2_workspace_bytes(1, 292 * 64, 1, 128, 128, 64, 1, 0) <= limit
-    assert gdn.gdn2_workspace_bytes(1, 293 * 64, 1, 128, 128, 64, 1, 0) > limit
+    f32 = gdn.GDN2_IO_F32   # the limit is the float32 path's workspace, whatever the io type
+    assert gdn.gdn2_workspace_bytes(1, 292 * 64, 1, 128, 128, 64, f32, 0) <= limit
+    assert gdn.gdn2_workspace_bytes(1, 293 * 64, 1, 128, 128, 64, f32, 0) > limit
     call = lambda T: L.gdn2_fwd_noalloc(*([FAKE] * 6), None, FAKE, None,  # noqa: E731
                                         1, T, 1, 128, 128, 64, 1, None)
     assert call(293 * 64) == 3            # GDN2_ERR_WORKSPACE, nothing enqueued
