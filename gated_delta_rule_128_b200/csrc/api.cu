@@ -26,10 +26,13 @@ cudaError_t simt_bwd_launch(const void *, const void *, const void *, const floa
 cudaError_t decode_launch(const void *, const void *, const void *, const float *, const float *,
                           const float *, float *, void *, int, int, int, int, gdn2_io,
                           cudaStream_t);
-size_t tc_fwd_ckpt_bytes(const Dims &d);
 cudaError_t tc_fwd_launch(const void *, const void *, const void *, const float *, const float *,
                           const float *, const float *, void *, float *, void *, unsigned int *,
                           const Dims &, cudaStream_t);
+cudaError_t tc_bwd_launch(const void *, const void *, const void *, const float *, const float *,
+                          const float *, const void *, const float *, void *, void *, void *,
+                          float *, float *, float *, float *, void *, unsigned int *, const Dims &,
+                          cudaStream_t);
 
 __device__ unsigned int g_status_word;
 
@@ -113,8 +116,7 @@ static size_t ws_bytes_for(const Dims &d, gdn2_io io, int for_bwd) {
     SimtWs lay = simt_ws_layout(d);
     if (use_tc(d, io)) {
         if (!for_bwd) return 256;  // the tensor-core forward keeps nothing between phases
-        size_t a = tc_fwd_ckpt_bytes(d), b = lay.bwd_end;
-        return a > b ? a : b;
+        return tc_ws_layout(d).bwd_end;
     }
     return for_bwd ? lay.bwd_end : lay.fwd_end;
 }
@@ -138,8 +140,8 @@ gdn2_status gdn2_fwd(const void *q, const void *k, const void *v, const float *g
     if (use_tc(d, io)) {
         unsigned int *status = status_word();
         if (!status) return GDN2_ERR_CUDA;
-        void *ckpt = (ws && ws_bytes >= ws_bytes_for(d, io, 1)) ? ws : nullptr;
-        return cuda_status(tc_fwd_launch(q, k, v, g, b, w, S0, o, ST, ckpt, status, d,
+        void *keep = ws_bytes >= ws_bytes_for(d, io, 1) ? ws : nullptr;
+        return cuda_status(tc_fwd_launch(q, k, v, g, b, w, S0, o, ST, keep, status, d,
                                          (cudaStream_t)stream));
     }
     return cuda_status(run_forward(q, k, v, g, b, w, S0, o, ST, ws, d, io, (cudaStream_t)stream));
@@ -158,8 +160,16 @@ gdn2_status gdn2_bwd(const void *q, const void *k, const void *v, const float *g
     if (!ws || !aligned16(ws) || ws_bytes < ws_bytes_for(d, io, 1)) return GDN2_ERR_WORKSPACE;
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e;
-    // the float32 backward below needs the float32 forward's tiles
-    if (use_tc(d, io)) ws_has_fwd = 0;
+    if (use_tc(d, io)) {
+        unsigned int *status = status_word();
+        if (!status) return GDN2_ERR_CUDA;
+        if (!ws_has_fwd) {
+            e = tc_fwd_launch(q, k, v, g, b, w, S0, nullptr, nullptr, ws, status, d, s);
+            if (e != cudaSuccess) return GDN2_ERR_CUDA;
+        }
+        return cuda_status(tc_bwd_launch(q, k, v, g, b, w, dO, dST, dq, dk, dv, dg, db, dw, dS0, ws,
+                                         status, d, s));
+    }
     if (!ws_has_fwd) {
         e = run_forward(q, k, v, g, b, w, S0, nullptr, nullptr, ws, d, io, s);
         if (e != cudaSuccess) return GDN2_ERR_CUDA;

@@ -99,6 +99,34 @@ inline SimtWs simt_ws_layout(const Dims &d) {
     return w;
 }
 
+// ---- workspace of the tensor-core path (d_k = d_v = 128, chunk 64): fp16
+// tiles in their 128-byte swizzled shared-memory layout, so that they move
+// with plain bulk copies.  Offsets in bytes; bh = b * H + h.
+//   ckS   [bh][NC + 1][2 halves] 16 KB  chunk-entry states S_c (and S_T), true scale
+//   ckTP  [bh][NC]               16 KB  T (8 KB) then P (8 KB)
+//   ckD   [bh][NC][2]             8 KB  Delta (columns of one d_v half)
+//   ckdS  [bh][NC][2]            16 KB  e^(G_L - G_m) dS_next
+//   ckndU [bh][NC][2]             8 KB  -dU
+//   ckEnd [bh][NC][2]           512 B  half-sums of rowsum(dS_next . S_next)
+struct TcWs {
+    size_t ckS, ckTP, ckD, ckdS, ckndU, ckEnd, fwd_end, bwd_end;
+};
+inline TcWs tc_ws_layout(const Dims &d) {
+    const size_t bh = (size_t)d.B * d.H, nc = (size_t)d.NC;
+    TcWs w;
+    size_t o = 0;
+    auto take = [&](size_t bytes) { size_t at = o; o = align256(o + bytes); return at; };
+    w.ckS = take(bh * (nc + 1) * 2 * 16384);
+    w.ckTP = take(bh * nc * 16384);
+    w.ckD = take(bh * nc * 2 * 8192);
+    w.fwd_end = o;
+    w.ckdS = take(bh * nc * 2 * 16384);
+    w.ckndU = take(bh * nc * 2 * 8192);
+    w.ckEnd = take(bh * nc * 2 * 512);
+    w.bwd_end = o;
+    return w;
+}
+
 template <typename T> __host__ __device__ __forceinline__ T *at(void *base, size_t off) {
     return reinterpret_cast<T *>(static_cast<char *>(base) + off);
 }

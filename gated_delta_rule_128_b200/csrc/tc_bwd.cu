@@ -1,0 +1,651 @@
+// Gate-aware chunkwise backward of Gated Delta Rule-2 on the sm_100a tensor
+// cores (bf16 I/O, d_k = d_v = 128, chunk 64), after tc_fwd_kernel has left
+// its chunk states, T, P and Delta in the workspace.
+//
+// "Gated DeltaNet-2" (LIT-802 review, Key takeaways 2; paper Secs. 3.3-3.4,
+// Apps. A-B, D.6; digg thread 11/): the per-channel gates cannot be pulled
+// out of the products that accumulate the gradient of the strictly-lower A,
+// so they stay inside them: b enters dA and dKc through Kc in every channel
+// sum below.
+//
+// Chunk equations (decay factors relative to the chunk's middle row m, see
+// tc_common.cuh; dS = dL/dS_next entering the chunk from the right):
+//   dS_m  = diag(e^(G_L-G_m)) dS
+//   dDelta = P^T dO + Kh dS_m,         dU = T^T dDelta,   dw = dU.v, dv = dU.w
+//   dS_c  = diag(e^G_m) (dS_m + Qb^T dO - Kc^T dU)                (carried left)
+//   S_m   = diag(e^G_m) S_c
+//   dP = lower-incl(dO Delta^T),       dA = -strictly-lower(dU Delta^T)
+//   Y1 = dO S_m^T + dP Kh              dq  = Y1.E
+//   Y2 = -dU S_m^T + dA Kh             dKc.e^G = Y2.E,  db = Y2.E.k
+//   Y3 = Delta dS_m^T + dP^T Qb + dA^T Kc            dk = Y2.E.b + Y3/E
+//   dG = dq.q + Y2.E.b.k - (Y3/E).k, plus rowsum(dS . S_next) on the last row
+//   dg = reverse in-chunk cumsum of dG
+// (E = e^(G - G_m); the chunk-end term rowsum(dS_next . S_next) is the
+// derivative through the chunk's total decay, since S_next = e^G_L (...).)
+//
+// Two kernels:
+//  * tc_bwd_state_kernel: one CTA per (b, h, half of d_v), walking the chunks
+//    in reverse with dS in tensor memory; three tcgen05.mma round trips per
+//    chunk (dDelta, dU, dS).  Writes dw, dv, dS0, and per chunk dS_m, -dU and
+//    the half-sums of the chunk-end term to the workspace.
+//  * tc_bwd_grad_kernel: one CTA per (b, h, chunk), all chunks in parallel,
+//    full d_v; five products, then three accumulations, then dq, dk, db, dg.
+
+#include "common.cuh"
+#include "tc.cuh"
+#include "tc_common.cuh"
+#include "tmap.cuh"
+
+namespace gdn2 {
+using namespace tc;
+using namespace tcc;
+
+// ============================================================ state kernel
+namespace tbs {
+constexpr int kThreads = 256;
+constexpr uint32_t RAW_Q = 0, RAW_K = 16384, RAW_DO = 32768, RAW_G = 40960, RAW_B = 73728;
+constexpr uint32_t OP_QB = 106496, OP_KC = 122880, OP_KH = 139264;  // [64 pos][128 key]
+constexpr uint32_t OP_T = 155648, OP_P = 163840;                      // [64][64], adjacent
+constexpr uint32_t OP_DS = 172032;   // dS_m fp16 [128 key][64 v]  MN-major B
+constexpr uint32_t OP_DO = 188416;   // dO fp16   [64 pos][64 v]   MN-major B
+constexpr uint32_t OP_DD = 196608;   // dDelta, later -dU [64 pos][64 v]
+constexpr uint32_t STG_S = 204800;   // S_c (true scale) fp16 [128 key][64 v]
+constexpr uint32_t MISC = 221184;    // sGam, sRef [128] f32; sEnd [2][128] f32; mbarriers; slot
+constexpr uint32_t SMEM_BYTES = MISC + 2176 + 1024;
+constexpr uint32_t SCR_SCAN = OP_DD;  // cumsum totals during phase 1
+constexpr uint32_t TM_DS = 0, TM_DD = 64, TM_DU = 128;  // 256 columns allocated
+constexpr uint32_t ID_MM64 = idesc_f16(64, 64, true, true);
+constexpr uint32_t ID_KM64 = idesc_f16(64, 64, false, true);
+constexpr uint32_t ID_MM128x64 = idesc_f16(128, 64, true, true);
+constexpr long long kWait = 2000000000LL;
+constexpr float kRange = 6.0e4f;
+}  // namespace tbs
+
+__global__ void __launch_bounds__(tbs::kThreads, 1)
+tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
+                    const __grid_constant__ CUtensorMap mdo, const __grid_constant__ CUtensorMap mg,
+                    const __grid_constant__ CUtensorMap mb, const __nv_bfloat16 *__restrict__ v,
+                    const float *__restrict__ w, const float *__restrict__ dST,
+                    __nv_bfloat16 *__restrict__ dvout, float *__restrict__ dwout,
+                    float *__restrict__ dS0, unsigned char *__restrict__ ws, TcWs lay,
+                    unsigned int *status, Dims d) {
+    using namespace tbs;
+    extern __shared__ unsigned char smraw[];
+    unsigned char *sm = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smraw) + 1023) & ~static_cast<uintptr_t>(1023));
+    float *sGam = reinterpret_cast<float *>(sm + MISC);
+    float *sRef = reinterpret_cast<float *>(sm + MISC + 512);
+    float *sEnd = reinterpret_cast<float *>(sm + MISC + 1024);  // [2][128]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + MISC + 2048);  // 0..7
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + MISC + 2048 + 64);
+    float big = 0.f;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int vh = blockIdx.x, h = blockIdx.y, bb = blockIdx.z, v0 = vh * 64;
+    const int NC = d.NC, T = d.T, H = d.H;
+    const int quarter = warp & 3, half = warp >> 2;
+    const int key = quarter * 32 + lane;
+    const size_t bh = (size_t)bb * H + h;
+
+    if (warp == 0) {
+        tmem_alloc(tslot, 256);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        for (int i = 0; i < 8; ++i) mbar_init(&bars[i], 1);
+        mbar_fence_init();
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tm = *tslot;
+
+    int issued[4] = {0, 0, 0, 0};
+    auto load_inputs = [&](int cc) {  // bar0: q, k, dO half; bar1: g, b
+        mbar_expect_tx(&bars[0], 16384 * 2 + 8192);
+        tma_load_4d(sm + RAW_Q, &mq, 0, h, cc * 64, bb, &bars[0]);
+        tma_load_4d(sm + RAW_K, &mk, 0, h, cc * 64, bb, &bars[0]);
+        tma_load_4d(sm + RAW_DO, &mdo, v0, h, cc * 64, bb, &bars[0]);
+        mbar_expect_tx(&bars[1], 32768 * 2);
+        tma_load_4d(sm + RAW_G, &mg, 0, h, cc * 64, bb, &bars[1]);
+        tma_load_4d(sm + RAW_B, &mb, 0, h, cc * 64, bb, &bars[1]);
+        ++issued[0];
+        ++issued[1];
+    };
+    auto load_tp = [&](int cc) {  // bar2: T and P of chunk cc
+        mbar_expect_tx(&bars[2], 16384);
+        bulk_load(sm + OP_T, ws + lay.ckTP + (bh * NC + cc) * 16384, 16384, &bars[2]);
+        ++issued[2];
+    };
+    auto load_s = [&](int slot, uint64_t *bar) {  // state checkpoint `slot` of this half
+        mbar_expect_tx(bar, 16384);
+        bulk_load(sm + STG_S, ws + lay.ckS + ((bh * (NC + 1) + slot) * 2 + vh) * 16384, 16384, bar);
+    };
+
+    // dS entering the last chunk: dS_T (or zero)
+    float x[32];
+    {
+        const size_t so = st_off(d, bb, h);
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) {
+            float4 t = dST ? *reinterpret_cast<const float4 *>(dST + so + (size_t)key * 128 + v0 + 32 * half + j)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+            x[j] = t.x; x[j + 1] = t.y; x[j + 2] = t.z; x[j + 3] = t.w;
+        }
+        tmem_st16(taddr(tm + TM_DS, quarter * 32, 32 * half), x);
+        tmem_st16(taddr(tm + TM_DS, quarter * 32, 32 * half + 16), x + 16);
+        tmem_wait_st();
+    }
+    // chunk-end term of the last chunk: rowsum(dS_T . S_T), this half's columns
+    bool ok = true;
+    if (tid == 0) load_s(NC, &bars[7]);
+    ok = mbar_wait(&bars[7], 0, kWait);
+    {
+        float acc = 0.f;
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+            float s8[8];
+            ld_h8(sm + STG_S + sw128_chunk(key, 4 * half + jj, 128), s8);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc += x[8 * jj + i] * s8[i];
+        }
+        sEnd[half * 128 + key] = acc;
+    }
+    fence_before_sync();
+    bool abort = __syncthreads_or(!ok);
+    if (!abort) {
+        if (half == 0)
+            reinterpret_cast<float *>(ws + lay.ckEnd + ((bh * NC + NC - 1) * 2 + vh) * 512)[key] =
+                sEnd[key] + sEnd[128 + key];
+        if (tid == 0) {
+            load_inputs(NC - 1);
+            load_tp(NC - 1);
+            load_s(NC - 1, &bars[3]);
+            ++issued[3];
+        }
+    }
+
+    for (int i = 0; i < NC && !abort; ++i) {
+        const int c = NC - 1 - i, c0 = c * 64;
+        const uint32_t par = i & 1;
+        // ---------------- phase 1: decay, operands, dS_m
+        ok = mbar_wait(&bars[0], par, kWait);
+        ok = ok && mbar_wait(&bars[1], par, kWait);
+        ok = ok && mbar_wait(&bars[2], par, kWait);
+        float G[8][4];
+        cumsum_local(reinterpret_cast<const float *>(sm + RAW_G), reinterpret_cast<float *>(sm + SCR_SCAN),
+                     warp, lane, G);
+        if (__syncthreads_or(!ok)) { abort = true; break; }
+        cumsum_finish(reinterpret_cast<const float *>(sm + SCR_SCAN), warp, lane, G, sGam, sRef);
+        big = fmaxf(big, write_factors(sm + RAW_Q, sm + RAW_K, reinterpret_cast<const float *>(sm + RAW_B),
+                                       G, sm + OP_QB, sm + OP_KC, sm + OP_KH, warp, lane));
+        if (lane < 16) {  // dO half -> fp16 operand [pos][v]
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+                const int r = 8 * warp + m;
+                uint2 dr = *reinterpret_cast<const uint2 *>(sm + RAW_DO + r * 128 + lane * 8);
+                const __nv_bfloat162 *d2 = reinterpret_cast<const __nv_bfloat162 *>(&dr);
+                st_h4(sm + OP_DO + sw128_off(r, 4 * lane, 64), __low2float(d2[0]), __high2float(d2[0]),
+                      __low2float(d2[1]), __high2float(d2[1]));
+            }
+        }
+        __syncthreads();
+        if (tid == 0 && c > 0) load_inputs(c - 1);  // raw tiles consumed
+        {
+            float sv[32];
+            tmem_ld16(taddr(tm + TM_DS, quarter * 32, 32 * half), sv);
+            tmem_ld16(taddr(tm + TM_DS, quarter * 32, 32 * half + 16), sv + 16);
+            tmem_wait_ld();
+            const float gm = sGam[key];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) sv[j] *= gm;
+            tmem_st16(taddr(tm + TM_DS, quarter * 32, 32 * half), sv);
+            tmem_st16(taddr(tm + TM_DS, quarter * 32, 32 * half + 16), sv + 16);
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                st_h8(sm + OP_DS + sw128_chunk(key, 4 * half + jj, 128), sv + 8 * jj);
+                big = absmax8(sv + 8 * jj, big);
+            }
+            tmem_wait_st();
+        }
+        fence_proxy_async();
+        fence_before_sync();
+        __syncthreads();
+        if (tid == 0) {
+            fence_after_sync();
+            bulk_store(ws + lay.ckdS + ((bh * NC + c) * 2 + vh) * 16384, sm + OP_DS, 16384);
+            bulk_commit();
+            const uint32_t p = smem_addr(sm + OP_P), dO = smem_addr(sm + OP_DO),
+                           kh = smem_addr(sm + OP_KH), ds = smem_addr(sm + OP_DS);
+            // dDelta = P^T dO + Kh dS_m
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(tm + TM_DD, desc_mnmajor(p, 64, ks), desc_mnmajor(dO, 64, ks), ID_MM64, ks > 0);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                mma_bf16(tm + TM_DD, desc_kmajor(kh, 64, ks), desc_mnmajor(ds, 128, ks), ID_KM64, 1);
+            mma_commit(&bars[4]);
+        }
+        // ---------------- phase 2: dDelta to shared memory, dU = T^T dDelta
+        ok = mbar_wait(&bars[4], par, kWait);
+        fence_after_sync();
+        {
+            float dd[32];
+            tmem_ld16(taddr(tm + TM_DD, quarter * 32, 32 * half), dd);
+            tmem_ld16(taddr(tm + TM_DD, quarter * 32, 32 * half + 16), dd + 16);
+            tmem_wait_ld();
+            if (lane < 16) {
+                const int r = quarter * 16 + lane;
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    st_h8(sm + OP_DD + sw128_chunk(r, 4 * half + jj, 64), dd + 8 * jj);
+                    big = absmax8(dd + 8 * jj, big);
+                }
+            }
+        }
+        fence_proxy_async();
+        fence_before_sync();
+        if (__syncthreads_or(!ok)) { abort = true; break; }
+        if (tid == 0) {
+            fence_after_sync();
+            const uint32_t t = smem_addr(sm + OP_T), dd = smem_addr(sm + OP_DD);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(tm + TM_DU, desc_mnmajor(t, 64, ks), desc_mnmajor(dd, 64, ks), ID_MM64, ks > 0);
+            mma_commit(&bars[5]);
+        }
+        // ---------------- phase 3: dw, dv; -dU to shared memory; dS update
+        ok = mbar_wait(&bars[5], par, kWait);
+        fence_after_sync();
+        {
+            float du[32];
+            tmem_ld16(taddr(tm + TM_DU, quarter * 32, 32 * half), du);
+            tmem_ld16(taddr(tm + TM_DU, quarter * 32, 32 * half + 16), du + 16);
+            tmem_wait_ld();
+            if (lane < 16) {
+                const int r = quarter * 16 + lane;
+                if (c0 + r < T) {
+                    const size_t ov = tok(d, bb, c0 + r, h, 128) + v0 + 32 * half;
+                    float dwv[32], dvv[32];
+#pragma unroll
+                    for (int j = 0; j < 32; j += 8) {
+                        uint4 vr = *reinterpret_cast<const uint4 *>(v + ov + j);
+                        const __nv_bfloat162 *v2 = reinterpret_cast<const __nv_bfloat162 *>(&vr);
+                        float4 w0 = *reinterpret_cast<const float4 *>(w + ov + j);
+                        float4 w1 = *reinterpret_cast<const float4 *>(w + ov + j + 4);
+                        float wf[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            dwv[j + 2 * e] = du[j + 2 * e] * __low2float(v2[e]);
+                            dwv[j + 2 * e + 1] = du[j + 2 * e + 1] * __high2float(v2[e]);
+                        }
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) dvv[j + e] = du[j + e] * wf[e];
+                    }
+#pragma unroll
+                    for (int j = 0; j < 32; j += 4)
+                        *reinterpret_cast<float4 *>(dwout + ov + j) =
+                            make_float4(dwv[j], dwv[j + 1], dwv[j + 2], dwv[j + 3]);
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj)
+                        st_bf16x8(reinterpret_cast<unsigned char *>(dvout + ov) + 16 * jj, dvv + 8 * jj);
+                }
+#pragma unroll
+                for (int j = 0; j < 32; ++j) du[j] = -du[j];
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    st_h8(sm + OP_DD + sw128_chunk(r, 4 * half + jj, 64), du + 8 * jj);
+                    big = absmax8(du + 8 * jj, big);
+                }
+            }
+        }
+        fence_proxy_async();
+        fence_before_sync();
+        if (__syncthreads_or(!ok)) { abort = true; break; }
+        if (tid == 0) {
+            fence_after_sync();
+            bulk_store(ws + lay.ckndU + ((bh * NC + c) * 2 + vh) * 8192, sm + OP_DD, 8192);
+            bulk_commit();
+            if (c > 0) load_tp(c - 1);  // T and P consumed
+            const uint32_t qb = smem_addr(sm + OP_QB), kc = smem_addr(sm + OP_KC),
+                           dO = smem_addr(sm + OP_DO), ndu = smem_addr(sm + OP_DD);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(tm + TM_DS, desc_mnmajor(qb, 64, ks), desc_mnmajor(dO, 64, ks), ID_MM128x64, 1);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(tm + TM_DS, desc_mnmajor(kc, 64, ks), desc_mnmajor(ndu, 64, ks), ID_MM128x64, 1);
+            mma_commit(&bars[6]);
+        }
+        // ---------------- phase 4: dS_c = e^G_m (...), chunk-end term of chunk c-1
+        ok = mbar_wait(&bars[6], par, kWait);
+        ok = ok && mbar_wait(&bars[3], par, kWait);
+        fence_after_sync();
+        {
+            float sv[32];
+            tmem_ld16(taddr(tm + TM_DS, quarter * 32, 32 * half), sv);
+            tmem_ld16(taddr(tm + TM_DS, quarter * 32, 32 * half + 16), sv + 16);
+            tmem_wait_ld();
+            const float e = sRef[key];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) sv[j] *= e;
+            tmem_st16(taddr(tm + TM_DS, quarter * 32, 32 * half), sv);
+            tmem_st16(taddr(tm + TM_DS, quarter * 32, 32 * half + 16), sv + 16);
+            float acc = 0.f;
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                float s8[8];
+                ld_h8(sm + STG_S + sw128_chunk(key, 4 * half + jj, 128), s8);
+#pragma unroll
+                for (int e2 = 0; e2 < 8; ++e2) acc += sv[8 * jj + e2] * s8[e2];
+            }
+            sEnd[half * 128 + key] = acc;
+            if (c == 0 && dS0) {
+                float *dst = dS0 + st_off(d, bb, h) + (size_t)key * 128 + v0 + 32 * half;
+#pragma unroll
+                for (int j = 0; j < 32; j += 4)
+                    *reinterpret_cast<float4 *>(dst + j) = make_float4(sv[j], sv[j + 1], sv[j + 2], sv[j + 3]);
+            }
+            tmem_wait_st();
+        }
+        if (tid == 0) bulk_wait_read();  // OP_DS, OP_DD copies done before they are rewritten
+        fence_proxy_async();
+        fence_before_sync();
+        if (__syncthreads_or(!ok)) { abort = true; break; }
+        if (c > 0 && half == 0)
+            reinterpret_cast<float *>(ws + lay.ckEnd + ((bh * NC + c - 1) * 2 + vh) * 512)[key] =
+                sEnd[key] + sEnd[128 + key];
+        if (tid == 0 && c > 0) {
+            load_s(c - 1, &bars[3]);
+            ++issued[3];
+        }
+    }
+    if (!(big <= kRange)) record_status(status, GDN2_ERR_RANGE);
+    if (tid == 0) {
+        bulk_wait_all();
+        if (abort) {
+            record_status(status, GDN2_ERR_TIMEOUT);
+            for (int k2 = 0; k2 < 4; ++k2)
+                if (issued[k2] > 0) mbar_wait(&bars[k2], (issued[k2] - 1) & 1, kWait);
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tm, 256);
+}
+
+// ============================================================ chunk kernel
+namespace tbg {
+constexpr int kThreads = 256;
+constexpr uint32_t RAW_Q = 0, RAW_K = 16384, RAW_B = 32768, RAW_G = 65536;  // g, later G - G_m
+constexpr uint32_t OP_DO = 98304;     // dO fp16 [64 pos][128 v] K-major (in place of raw dO)
+constexpr uint32_t BL_S = 114688;     // S_m [128 key][128 v] K-major B   (later Qb, Kc, Kh; then dG)
+constexpr uint32_t BL_DS = 147456;    // dS_m [128 key][128 v]
+constexpr uint32_t BL_D = 180224;     // Delta [64 pos][128 v]              (later dP, dA)
+constexpr uint32_t BL_NDU = 196608;   // -dU [64 pos][128 v]
+constexpr uint32_t OP_QB = BL_S, OP_KC = BL_S + 16384, OP_KH = BL_S + 32768;
+constexpr uint32_t OP_DP = BL_D, OP_DA = BL_D + 8192;
+constexpr uint32_t SCR_DG = BL_S;     // dG [64][128] f32, after the last products
+constexpr uint32_t MISC = 212992;     // sGam, sRef [128]; sEnd [128]; scan [8][128]; mbarriers; slot
+constexpr uint32_t SMEM_BYTES = MISC + 1536 + 4096 + 128 + 1024;
+constexpr uint32_t TM_DP = 0, TM_DA = 64, TM_Y1 = 128, TM_Y2 = 256, TM_Y3 = 384;
+constexpr uint32_t ID_KK64 = idesc_f16(64, 64, false, false);
+constexpr uint32_t ID_KK128 = idesc_f16(64, 128, false, false);
+constexpr uint32_t ID_KM128 = idesc_f16(64, 128, false, true);
+constexpr uint32_t ID_MM128 = idesc_f16(64, 128, true, true);
+constexpr long long kWait = 2000000000LL;
+constexpr float kRange = 6.0e4f;
+}  // namespace tbg
+
+__global__ void __launch_bounds__(tbg::kThreads, 1)
+tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
+                   const __grid_constant__ CUtensorMap mdo, const __grid_constant__ CUtensorMap mg,
+                   const __grid_constant__ CUtensorMap mb, __nv_bfloat16 *__restrict__ dqout,
+                   __nv_bfloat16 *__restrict__ dkout, float *__restrict__ dbout,
+                   float *__restrict__ dgout, unsigned char *__restrict__ ws, TcWs lay,
+                   unsigned int *status, Dims d) {
+    using namespace tbg;
+    extern __shared__ unsigned char smraw[];
+    unsigned char *sm = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smraw) + 1023) & ~static_cast<uintptr_t>(1023));
+    float *sGam = reinterpret_cast<float *>(sm + MISC);
+    float *sRef = reinterpret_cast<float *>(sm + MISC + 512);
+    float *sEnd = reinterpret_cast<float *>(sm + MISC + 1024);
+    float *scan = reinterpret_cast<float *>(sm + MISC + 1536);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + MISC + 1536 + 4096);
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + MISC + 1536 + 4096 + 64);
+    float big = 0.f;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int c = blockIdx.x, h = blockIdx.y, bb = blockIdx.z, c0 = c * 64;
+    const int NC = d.NC, T = d.T, H = d.H, L = min(64, T - c0);
+    const int quarter = warp & 3, half = warp >> 2;
+    const size_t bh = (size_t)bb * H + h;
+
+    if (warp == 0) {
+        tmem_alloc(tslot, 512);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        for (int i = 0; i < 3; ++i) mbar_init(&bars[i], 1);
+        mbar_fence_init();
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tm = *tslot;
+
+    if (tid == 0) {
+        mbar_expect_tx(&bars[0], 16384 * 2 + 32768 * 2 + 16384 + 32768 * 2 + 16384 * 2);
+        tma_load_4d(sm + RAW_Q, &mq, 0, h, c0, bb, &bars[0]);
+        tma_load_4d(sm + RAW_K, &mk, 0, h, c0, bb, &bars[0]);
+        tma_load_4d(sm + RAW_B, &mb, 0, h, c0, bb, &bars[0]);
+        tma_load_4d(sm + RAW_G, &mg, 0, h, c0, bb, &bars[0]);
+        tma_load_4d(sm + OP_DO, &mdo, 0, h, c0, bb, &bars[0]);
+        bulk_load(sm + BL_S, ws + lay.ckS + ((bh * (NC + 1) + c) * 2) * 16384, 32768, &bars[0]);
+        bulk_load(sm + BL_DS, ws + lay.ckdS + ((bh * NC + c) * 2) * 16384, 32768, &bars[0]);
+        bulk_load(sm + BL_D, ws + lay.ckD + ((bh * NC + c) * 2) * 8192, 16384, &bars[0]);
+        bulk_load(sm + BL_NDU, ws + lay.ckndU + ((bh * NC + c) * 2) * 8192, 16384, &bars[0]);
+    }
+    if (tid < 128) {
+        const float *e0 = reinterpret_cast<const float *>(ws + lay.ckEnd + ((bh * NC + c) * 2) * 512);
+        sEnd[tid] = e0[tid] + e0[128 + tid];
+    }
+    bool ok = mbar_wait(&bars[0], 0, kWait);
+    // ---------------- G1: decay, S_m, dO operand; five products
+    float G[8][4];
+    cumsum_local(reinterpret_cast<const float *>(sm + RAW_G), scan, warp, lane, G);
+    // dO: raw bf16 rows [64][128] -> fp16 K-major tile in place (values held in registers)
+    uint2 dor[8];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) dor[m] = *reinterpret_cast<const uint2 *>(sm + OP_DO + (8 * warp + m) * 256 + lane * 8);
+    bool abort = __syncthreads_or(!ok);
+    if (!abort) {
+        cumsum_finish(scan, warp, lane, G, sGam, sRef);
+        float *sG = reinterpret_cast<float *>(sm + RAW_G);
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+            const int r = 8 * warp + m;
+            *reinterpret_cast<float4 *>(sG + r * 128 + 4 * lane) = make_float4(G[m][0], G[m][1], G[m][2], G[m][3]);
+            const __nv_bfloat162 *d2 = reinterpret_cast<const __nv_bfloat162 *>(&dor[m]);
+            st_h4(sm + OP_DO + sw128_off(r, 4 * lane, 64), __low2float(d2[0]), __high2float(d2[0]),
+                  __low2float(d2[1]), __high2float(d2[1]));
+        }
+        __syncthreads();
+        // S_m = diag(e^G_m) S_c, in place: thread -> (key, 64 value columns)
+        {
+            const int kr = tid >> 1, hb = tid & 1;
+            const float e = sRef[kr];
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) {
+                unsigned char *p = sm + BL_S + sw128_chunk(kr, hb * 8 + jj, 128);
+                float s8[8];
+                ld_h8(p, s8);
+#pragma unroll
+                for (int e2 = 0; e2 < 8; ++e2) s8[e2] *= e;
+                st_h8(p, s8);
+                big = absmax8(s8, big);
+            }
+        }
+        fence_proxy_async();
+        fence_before_sync();
+        __syncthreads();
+        if (tid == 0) {
+            fence_after_sync();
+            const uint32_t dO = smem_addr(sm + OP_DO), S = smem_addr(sm + BL_S),
+                           DS = smem_addr(sm + BL_DS), D = smem_addr(sm + BL_D),
+                           NDU = smem_addr(sm + BL_NDU);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                mma_bf16(tm + TM_DP, desc_kmajor(dO, 64, ks), desc_kmajor(D, 64, ks), ID_KK64, ks > 0);
+                mma_bf16(tm + TM_DA, desc_kmajor(NDU, 64, ks), desc_kmajor(D, 64, ks), ID_KK64, ks > 0);
+                mma_bf16(tm + TM_Y1, desc_kmajor(dO, 64, ks), desc_kmajor(S, 128, ks), ID_KK128, ks > 0);
+                mma_bf16(tm + TM_Y2, desc_kmajor(NDU, 64, ks), desc_kmajor(S, 128, ks), ID_KK128, ks > 0);
+                mma_bf16(tm + TM_Y3, desc_kmajor(D, 64, ks), desc_kmajor(DS, 128, ks), ID_KK128, ks > 0);
+            }
+            mma_commit(&bars[1]);
+        }
+        // ---------------- G2: masked dP, dA; Qb, Kc, Kh; three accumulations
+        ok = mbar_wait(&bars[1], 0, kWait);
+        fence_after_sync();
+        {
+            float row[64];
+            const uint32_t base = warp < 4 ? tm + TM_DP : tm + TM_DA;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) tmem_ld16(taddr(base, quarter * 32, 16 * j), row + 16 * j);
+            tmem_wait_ld();
+            if (lane < 16) {
+                const int r = quarter * 16 + lane;
+                // dP keeps j <= r; dA = -strictly-lower(dU Delta^T) = strictly-lower of (-dU) Delta^T
+#pragma unroll
+                for (int j = 0; j < 64; ++j) row[j] = (warp < 4 ? j <= r : j < r) ? row[j] : 0.f;
+                unsigned char *dst = sm + (warp < 4 ? OP_DP : OP_DA);
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj) {
+                    st_h8(dst + sw128_chunk(r, jj, 64), row + 8 * jj);
+                    big = absmax8(row + 8 * jj, big);
+                }
+            }
+        }
+        big = fmaxf(big, write_factors(sm + RAW_Q, sm + RAW_K, reinterpret_cast<const float *>(sm + RAW_B),
+                                       G, sm + OP_QB, sm + OP_KC, sm + OP_KH, warp, lane));
+        fence_proxy_async();
+        fence_before_sync();
+        abort = __syncthreads_or(!ok);
+    }
+    if (!abort) {
+        if (tid == 0) {
+            fence_after_sync();
+            const uint32_t dP = smem_addr(sm + OP_DP), dA = smem_addr(sm + OP_DA),
+                           qb = smem_addr(sm + OP_QB), kc = smem_addr(sm + OP_KC),
+                           kh = smem_addr(sm + OP_KH);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                mma_bf16(tm + TM_Y1, desc_kmajor(dP, 64, ks), desc_mnmajor(kh, 64, ks), ID_KM128, 1);
+                mma_bf16(tm + TM_Y2, desc_kmajor(dA, 64, ks), desc_mnmajor(kh, 64, ks), ID_KM128, 1);
+                mma_bf16(tm + TM_Y3, desc_mnmajor(dP, 64, ks), desc_mnmajor(qb, 64, ks), ID_MM128, 1);
+                mma_bf16(tm + TM_Y3, desc_mnmajor(dA, 64, ks), desc_mnmajor(kc, 64, ks), ID_MM128, 1);
+            }
+            mma_commit(&bars[2]);
+        }
+        // ---------------- G3: dq, dk, db and dG per (row, channel)
+        ok = mbar_wait(&bars[2], 0, kWait);
+        fence_after_sync();
+        float *sG = reinterpret_cast<float *>(sm + RAW_G);
+        float *sdG = reinterpret_cast<float *>(sm + SCR_DG);  // Qb/Kc/Kh are consumed
+        const float *rb = reinterpret_cast<const float *>(sm + RAW_B);
+        __syncthreads();  // every thread is past the products before dG overwrites their operands
+        const int r = quarter * 16 + lane;
+#pragma unroll 1
+        for (int cb = 0; cb < 4; ++cb) {
+            const int i0 = 64 * half + 16 * cb;
+            float y1[16], y2[16], y3[16];
+            tmem_ld16(taddr(tm + TM_Y1, quarter * 32, i0), y1);
+            tmem_ld16(taddr(tm + TM_Y2, quarter * 32, i0), y2);
+            tmem_ld16(taddr(tm + TM_Y3, quarter * 32, i0), y3);
+            tmem_wait_ld();
+            if (lane < 16) {
+                float dq[16], dk[16], db[16];
+                const uint4 *q8 = reinterpret_cast<const uint4 *>(sm + RAW_Q + r * 256 + i0 * 2);
+                const uint4 *k8 = reinterpret_cast<const uint4 *>(sm + RAW_K + r * 256 + i0 * 2);
+                uint4 qv[2] = {q8[0], q8[1]}, kv[2] = {k8[0], k8[1]};
+                const __nv_bfloat16 *qh = reinterpret_cast<const __nv_bfloat16 *>(qv);
+                const __nv_bfloat16 *kh = reinterpret_cast<const __nv_bfloat16 *>(kv);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const int i = i0 + e;
+                    const float E = __expf(sG[r * 128 + i]);
+                    const float qf = __bfloat162float(qh[e]), kf = __bfloat162float(kh[e]);
+                    const float bf = rb[r * 128 + i];
+                    const float dqv = y1[e] * E, dkc = y2[e] * E, dkh = y3[e] * __frcp_rn(E);
+                    dq[e] = dqv;
+                    db[e] = dkc * kf;
+                    dk[e] = dkc * bf + dkh;
+                    sdG[r * 128 + i] = dqv * qf + dkc * bf * kf - dkh * kf;
+                }
+                if (r < L) {
+                    const size_t ok_ = tok(d, bb, c0 + r, h, 128) + i0;
+                    st_bf16x8(reinterpret_cast<unsigned char *>(dqout + ok_), dq);
+                    st_bf16x8(reinterpret_cast<unsigned char *>(dqout + ok_) + 16, dq + 8);
+                    st_bf16x8(reinterpret_cast<unsigned char *>(dkout + ok_), dk);
+                    st_bf16x8(reinterpret_cast<unsigned char *>(dkout + ok_) + 16, dk + 8);
+#pragma unroll
+                    for (int e = 0; e < 16; e += 4)
+                        *reinterpret_cast<float4 *>(dbout + ok_ + e) = make_float4(db[e], db[e + 1], db[e + 2], db[e + 3]);
+                }
+            }
+        }
+        abort = __syncthreads_or(!ok);
+        if (!abort && tid < 128) {
+            // dg = reverse in-chunk cumsum of dG, chunk-end term on the last row
+            float acc = sEnd[tid];
+            for (int rr = L - 1; rr >= 0; --rr) {
+                acc += sdG[rr * 128 + tid];
+                dgout[tok(d, bb, c0 + rr, h, 128) + tid] = acc;
+            }
+        }
+    }
+    if (!(big <= kRange)) record_status(status, GDN2_ERR_RANGE);
+    if (abort && tid == 0) {
+        record_status(status, GDN2_ERR_TIMEOUT);
+        mbar_wait(&bars[0], 0, kWait);
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tm, 512);
+}
+
+// ---------------------------------------------------------------- launchers
+cudaError_t tc_bwd_launch(const void *q, const void *k, const void *v, const float *g,
+                          const float *b, const float *w, const void *dO, const float *dST,
+                          void *dq, void *dk, void *dv, float *dg, float *db, float *dw,
+                          float *dS0, void *ws, unsigned int *status, const Dims &d,
+                          cudaStream_t s) {
+    CUtensorMap mq, mk, mdo_half, mdo, mg, mb;
+    if (!make_btHd_map(&mq, q, true, d.B, d.T, d.H, 128, 64, 128) ||
+        !make_btHd_map(&mk, k, true, d.B, d.T, d.H, 128, 64, 128) ||
+        !make_btHd_map(&mdo_half, dO, true, d.B, d.T, d.H, 128, 64, 64) ||
+        !make_btHd_map(&mdo, dO, true, d.B, d.T, d.H, 128, 64, 128) ||
+        !make_btHd_map(&mg, g, false, d.B, d.T, d.H, 128, 64, 128) ||
+        !make_btHd_map(&mb, b, false, d.B, d.T, d.H, 128, 64, 128))
+        return cudaErrorInvalidValue;
+    const TcWs lay = tc_ws_layout(d);
+    cudaError_t e = cudaFuncSetAttribute(tc_bwd_state_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tbs::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(tc_bwd_grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)tbg::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    count_launches(1);
+    tc_bwd_state_kernel<<<dim3(2, d.H, d.B), tbs::kThreads, tbs::SMEM_BYTES, s>>>(
+        mq, mk, mdo_half, mg, mb, (const __nv_bfloat16 *)v, w, dST, (__nv_bfloat16 *)dv, dw, dS0,
+        (unsigned char *)ws, lay, status, d);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    count_launches(1);
+    tc_bwd_grad_kernel<<<dim3(d.NC, d.H, d.B), tbg::kThreads, tbg::SMEM_BYTES, s>>>(
+        mq, mk, mdo, mg, mb, (__nv_bfloat16 *)dq, (__nv_bfloat16 *)dk, db, dg, (unsigned char *)ws,
+        lay, status, d);
+    return cudaGetLastError();
+}
+
+}  // namespace gdn2

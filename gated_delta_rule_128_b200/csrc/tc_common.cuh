@@ -1,0 +1,134 @@
+// Pieces shared by the tensor-core forward and backward kernels: the in-chunk
+// cumulative log-decay, the decay-scaled fp16 operand tiles, and small store
+// helpers.  Thread layout of these helpers (256 threads, 64-row chunk, 128 key
+// channels): warp w owns rows 8w..8w+7, lane l owns channels 4l..4l+3.
+//
+// Decay factors are taken relative to the chunk's middle row m = 31
+// ("Gated DeltaNet-2", LIT-802 review, Key takeaways 2: the state is
+// normalised by the cumulative decay; here the normalisation point is moved
+// to the chunk's middle to keep every factor within fp16 range):
+//   E = e^(G - G_m),  Qb = q.E,  Kc = b.k.E,  Kh = k / E,
+//   gamma_m = e^(G_L - G_m) (sGam),  e^(G_m) (sRef).
+#pragma once
+
+#include "common.cuh"
+#include "tc.cuh"
+
+namespace gdn2 {
+namespace tcc {
+using namespace tc;
+
+__device__ __forceinline__ void st_h4(unsigned char *p, float a, float b, float c, float d) {
+    uint2 v = make_uint2(pack_f16(a, b), pack_f16(c, d));
+    *reinterpret_cast<uint2 *>(p) = v;
+}
+__device__ __forceinline__ void st_h8(unsigned char *p, const float *x) {
+    uint4 v = make_uint4(pack_f16(x[0], x[1]), pack_f16(x[2], x[3]), pack_f16(x[4], x[5]),
+                         pack_f16(x[6], x[7]));
+    *reinterpret_cast<uint4 *>(p) = v;
+}
+__device__ __forceinline__ void st_bf16x8(unsigned char *p, const float *x) {
+    uint4 v = make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]),
+                         pack_bf16(x[6], x[7]));
+    *reinterpret_cast<uint4 *>(p) = v;
+}
+__device__ __forceinline__ float absmax8(const float *x, float m) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(x[i]));
+    return m;
+}
+// 8 fp16 values of a 16-B chunk, widened
+__device__ __forceinline__ void ld_h8(const unsigned char *p, float *x) {
+    uint4 v = *reinterpret_cast<const uint4 *>(p);
+    const __half2 *h = reinterpret_cast<const __half2 *>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float2 f = __half22float2(h[i]);
+        x[2 * i] = f.x;
+        x[2 * i + 1] = f.y;
+    }
+}
+
+// Step 1 of the cumsum: local inclusive prefix over the warp's 8 rows (raw g
+// tile row-major [64][128] f32); the warp's totals go to scan[warp][128].
+__device__ __forceinline__ void cumsum_local(const float *rg, float *scan, int warp, int lane,
+                                             float G[8][4]) {
+    float run[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+        float4 t = *reinterpret_cast<const float4 *>(rg + (8 * warp + m) * 128 + 4 * lane);
+        run[0] += t.x; run[1] += t.y; run[2] += t.z; run[3] += t.w;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) G[m][i] = run[i];
+    }
+    *reinterpret_cast<float4 *>(scan + warp * 128 + 4 * lane) = make_float4(run[0], run[1], run[2], run[3]);
+}
+
+// Step 2 (after a block barrier): add the earlier warps' totals and express G
+// relative to row 31; warp 0 writes e^(G_L - G_m) and e^(G_m) per channel.
+// Rows past the chunk's end hold g = 0 (zero-filled tiles), so row 63
+// carries G_L of a short last chunk.
+__device__ __forceinline__ void cumsum_finish(const float *scan, int warp, int lane, float G[8][4],
+                                              float *sGam, float *sRef) {
+    float pre[4] = {0.f, 0.f, 0.f, 0.f}, tot[4] = {0.f, 0.f, 0.f, 0.f}, ref[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int w2 = 0; w2 < 8; ++w2) {
+        float4 t = *reinterpret_cast<const float4 *>(scan + w2 * 128 + 4 * lane);
+        float tv[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            if (w2 < warp) pre[i] += tv[i];
+            if (w2 < 4) ref[i] += tv[i];
+            tot[i] += tv[i];
+        }
+    }
+#pragma unroll
+    for (int m = 0; m < 8; ++m)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) G[m][i] += pre[i] - ref[i];
+    if (warp == 0)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            sGam[4 * lane + i] = __expf(tot[i] - ref[i]);
+            sRef[4 * lane + i] = __expf(ref[i]);
+        }
+}
+
+// Operand tiles Qb, Kc, Kh ([64 pos][128 key] fp16, 128-B swizzled, R = 64)
+// from the raw q, k (bf16 [64][128]) and b (f32 [64][128]) tiles.  Any null
+// destination is skipped.  Returns the largest magnitude written.
+__device__ __forceinline__ float write_factors(const unsigned char *rq, const unsigned char *rk,
+                                               const float *rb, const float G[8][4],
+                                               unsigned char *oQb, unsigned char *oKc,
+                                               unsigned char *oKh, int warp, int lane) {
+    float big = 0.f;
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+        const int r = 8 * warp + m;
+        uint2 qr = *reinterpret_cast<const uint2 *>(rq + r * 256 + lane * 8);
+        uint2 kr = *reinterpret_cast<const uint2 *>(rk + r * 256 + lane * 8);
+        float4 bv = *reinterpret_cast<const float4 *>(rb + r * 128 + 4 * lane);
+        const __nv_bfloat162 *q2 = reinterpret_cast<const __nv_bfloat162 *>(&qr);
+        const __nv_bfloat162 *k2 = reinterpret_cast<const __nv_bfloat162 *>(&kr);
+        float qf[4] = {__low2float(q2[0]), __high2float(q2[0]), __low2float(q2[1]), __high2float(q2[1])};
+        float kf[4] = {__low2float(k2[0]), __high2float(k2[0]), __low2float(k2[1]), __high2float(k2[1])};
+        float bf[4] = {bv.x, bv.y, bv.z, bv.w};
+        float qb[4], kc[4], kh[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float e = __expf(G[m][i]);
+            qb[i] = qf[i] * e;
+            kc[i] = bf[i] * kf[i] * e;
+            kh[i] = kf[i] * __frcp_rn(e);
+            big = fmaxf(big, fmaxf(fabsf(qb[i]), fmaxf(fabsf(kc[i]), fabsf(kh[i]))));
+        }
+        const uint32_t off = sw128_off(r, 4 * lane, 64);
+        if (oQb) st_h4(oQb + off, qb[0], qb[1], qb[2], qb[3]);
+        if (oKc) st_h4(oKc + off, kc[0], kc[1], kc[2], kc[3]);
+        if (oKh) st_h4(oKh + off, kh[0], kh[1], kh[2], kh[3]);
+    }
+    return big;
+}
+
+}  // namespace tcc
+}  // namespace gdn2

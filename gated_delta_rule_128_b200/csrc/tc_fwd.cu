@@ -19,23 +19,26 @@
 // tcgen05.mma groups (kind::f16 with fp16 operands, f32 accumulators in TMEM)
 // form A, P, QbS, W|U', WS, P Delta and Kh^T Delta; the unit-lower-triangular
 // T is inverted in float32 on the CUDA cores by blocked forward substitution
-// (16x16 diagonal blocks, then three block levels).  The fp16 copy of each
-// chunk-entry state is written to the workspace for the backward pass.
+// (16x16 diagonal blocks, then three block levels).
 //
 // Precision and range: fp16 operands carry 11 significant bits (bf16 carries
 // 8, which left the output error at the 5e-3 tolerance).  To keep them in
 // fp16 range the decay factors are taken relative to the chunk's middle row
-// m = 31: Qb = q.e^(G-G_m), Kc = b.k.e^(G-G_m), Kh = k.e^(G_m-G); the state
-// products then use S_m = diag(e^G_m) S, and the update becomes
-// S_next = diag(e^(G_L-G_m)) (S_m + Kh^T Delta).  Any operand beyond 6e4 in
-// magnitude is reported as GDN2_ERR_RANGE.
+// m = 31 (see tc_common.cuh); the state products then use S_m = diag(e^G_m) S
+// and the update becomes S_next = diag(e^(G_L-G_m)) (S_m + Kh^T Delta).  Any
+// operand beyond 6e4 in magnitude is reported as GDN2_ERR_RANGE.
+//
+// For the backward the call can also leave in the workspace (TcWs): every
+// chunk-entry state and S_T (fp16), T and P per chunk, and Delta per chunk.
 
 #include "common.cuh"
 #include "tc.cuh"
+#include "tc_common.cuh"
 #include "tmap.cuh"
 
 namespace gdn2 {
 using namespace tc;
+using namespace tcc;
 
 namespace tfwd {
 constexpr int kThreads = 256;
@@ -45,7 +48,7 @@ constexpr uint32_t RAW_Q = 0, RAW_K = 16384, RAW_V = 32768, RAW_W = 40960, RAW_G
 constexpr uint32_t OP_KC = 122880;  // Kc, later W        [64 pos][128 key]  K-major
 constexpr uint32_t OP_QB = 139264;  // Qb                 [64 pos][128 key]
 constexpr uint32_t OP_KH = 155648;  // Kh                 [64 pos][128 key]
-constexpr uint32_t OP_S = 172032;   // S (fp16)           [128 key][64 v]    MN-major B
+constexpr uint32_t OP_S = 172032;   // S_m (fp16)         [128 key][64 v]    MN-major B
 constexpr uint32_t OP_U = 188416;   // U, later Delta     [64 pos][64 v]     MN-major B
 constexpr uint32_t OP_T = 196608;   // T                  [64 r][64 j]       K-major
 constexpr uint32_t OP_P = 204800;   // P                  [64 r][64 j]       K-major
@@ -64,24 +67,53 @@ constexpr long long kWait = 2000000000LL;  // ~1 s of SM clocks per wait
 constexpr float kRange = 6.0e4f;           // largest operand magnitude kept in fp16
 }  // namespace tfwd
 
-__device__ __forceinline__ void st_h4(unsigned char *p, float a, float b, float c, float d) {
-    uint2 v = make_uint2(pack_f16(a, b), pack_f16(c, d));
-    *reinterpret_cast<uint2 *>(p) = v;
-}
-__device__ __forceinline__ void st_h8(unsigned char *p, const float *x) {
-    uint4 v = make_uint4(pack_f16(x[0], x[1]), pack_f16(x[2], x[3]), pack_f16(x[4], x[5]),
-                         pack_f16(x[6], x[7]));
-    *reinterpret_cast<uint4 *>(p) = v;
-}
-__device__ __forceinline__ float absmax8(const float *x, float m) {
+// T = (I + A)^-1 for the strictly-lower 64x64 A in sA ([64][65] f32), into
+// sT ([64][65] f32): 16x16 diagonal blocks by forward substitution (one
+// column per thread), then T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ level by
+// level.  All 256 threads; ends with a barrier.
+__device__ __forceinline__ void invert_unit_lower(const float *sA, float *sT, float *sM, int tid) {
+    if (tid < 64) {
+        const int o16 = (tid >> 4) * 16, cl = tid & 15;
+        float x[16];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(x[i]));
-    return m;
-}
-__device__ __forceinline__ void st_bf16x8(unsigned char *p, const float *x) {
-    uint4 v = make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]),
-                         pack_bf16(x[6], x[7]));
-    *reinterpret_cast<uint4 *>(p) = v;
+        for (int r = 0; r < 16; ++r) {
+            float acc = r == cl ? 1.f : 0.f;
+#pragma unroll
+            for (int j = 0; j < r; ++j) acc -= sA[(o16 + r) * 65 + o16 + j] * x[j];
+            x[r] = acc;
+        }
+#pragma unroll
+        for (int r = 0; r < 16; ++r) sT[(o16 + r) * 65 + o16 + cl] = x[r];
+    }
+    for (int e = tid; e < 64 * 64; e += 256) {
+        const int r = e >> 6, j = e & 63;
+        if ((j >> 4) > (r >> 4)) sT[r * 65 + j] = 0.f;
+    }
+    __syncthreads();
+    for (int lvl = 1; lvl < 4; ++lvl) {
+        const int nb = 4 - lvl;
+        for (int e = tid; e < nb * 256; e += 256) {
+            const int bi = e >> 8, r = (e >> 4) & 15, cl = e & 15;
+            const int I = bi + lvl, J = bi;
+            float acc = 0.f;
+            for (int K = J; K < I; ++K)
+#pragma unroll
+                for (int kk = 0; kk < 16; ++kk)
+                    acc += sA[(16 * I + r) * 65 + 16 * K + kk] * sT[(16 * K + kk) * 65 + 16 * J + cl];
+            sM[bi * 272 + r * 17 + cl] = acc;
+        }
+        __syncthreads();
+        for (int e = tid; e < nb * 256; e += 256) {
+            const int bi = e >> 8, r = (e >> 4) & 15, cl = e & 15;
+            const int I = bi + lvl, J = bi;
+            float acc = 0.f;
+#pragma unroll
+            for (int kk = 0; kk < 16; ++kk)
+                acc += sT[(16 * I + r) * 65 + 16 * I + kk] * sM[bi * 272 + kk * 17 + cl];
+            sT[(16 * I + r) * 65 + 16 * J + cl] = -acc;
+        }
+        __syncthreads();
+    }
 }
 
 __global__ void __launch_bounds__(tfwd::kThreads, 1)
@@ -89,7 +121,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CU
               const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mg,
               const __grid_constant__ CUtensorMap mb, const __grid_constant__ CUtensorMap mw,
               const float *__restrict__ S0, __nv_bfloat16 *__restrict__ o, float *__restrict__ ST,
-              __nv_bfloat16 *__restrict__ ckpt, unsigned int *status, Dims d) {
+              unsigned char *__restrict__ ws, TcWs lay, unsigned int *status, Dims d) {
     using namespace tfwd;
     extern __shared__ unsigned char smraw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(
@@ -104,6 +136,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CU
     const int vh = blockIdx.x, h = blockIdx.y, bb = blockIdx.z, v0 = vh * 64;
     const int NC = d.NC, T = d.T, H = d.H;
     const int quarter = warp & 3, half = warp >> 2;
+    const size_t bh = (size_t)bb * H + h;
 
     if (warp == 0) {
         tmem_alloc(tslot, 512);
@@ -139,7 +172,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CU
     }
 
     const size_t so = st_off(d, bb, h);
-    // initial state slice: fp32 into TMEM, fp16 into OP_S
+    // initial state slice: fp32 into TMEM, fp16 (true scale) into OP_S for the checkpoint
     {
         const int key = quarter * 32 + lane, c0 = half * 32;
         float x[32];
@@ -161,105 +194,40 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CU
     fence_proxy_async();
     fence_before_sync();
     __syncthreads();
-    const size_t ck_head = ((size_t)bb * H + h) * NC;
-    if (tid == 0 && ckpt) {
-        bulk_store(ckpt + ((ck_head + 0) * 2 + vh) * 8192, sm + OP_S, 16384);
+    if (tid == 0 && ws) {
+        bulk_store(ws + lay.ckS + ((bh * (NC + 1) + 0) * 2 + vh) * 16384, sm + OP_S, 16384);
         bulk_commit();
     }
 
     bool abort = false;
-    int c = 0;
-    for (; c < NC; ++c) {
+    for (int c = 0; c < NC; ++c) {
         const uint32_t par = c & 1;
         const int c0 = c * 64;
         // ---------------- phase 1: cumulative decay and operands
         bool ok = mbar_wait(&bars[0], par, kWait);
         ok = ok && mbar_wait(&bars[1], par, kWait);
         float G[8][4];
-        {
-            const float *rg = reinterpret_cast<const float *>(sm + RAW_G);
-            float run[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int m = 0; m < 8; ++m) {
-                float4 t = *reinterpret_cast<const float4 *>(rg + (8 * warp + m) * 128 + 4 * lane);
-                run[0] += t.x; run[1] += t.y; run[2] += t.z; run[3] += t.w;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) G[m][i] = run[i];
-            }
-            float *scan = reinterpret_cast<float *>(sm + SCR_SCAN);
-            *reinterpret_cast<float4 *>(scan + warp * 128 + 4 * lane) =
-                make_float4(run[0], run[1], run[2], run[3]);
-        }
+        cumsum_local(reinterpret_cast<const float *>(sm + RAW_G), reinterpret_cast<float *>(sm + SCR_SCAN),
+                     warp, lane, G);
         if (__syncthreads_or(!ok)) { abort = true; break; }
-        {
-            const float *scan = reinterpret_cast<const float *>(sm + SCR_SCAN);
-            float pre[4] = {0.f, 0.f, 0.f, 0.f}, tot[4] = {0.f, 0.f, 0.f, 0.f};
-            float ref[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int w2 = 0; w2 < 8; ++w2) {
-                float4 t = *reinterpret_cast<const float4 *>(scan + w2 * 128 + 4 * lane);
-                float tv[4] = {t.x, t.y, t.z, t.w};
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    if (w2 < warp) pre[i] += tv[i];
-                    if (w2 < 4) ref[i] += tv[i];   // G at row 31
-                    tot[i] += tv[i];
-                }
-            }
-            // G relative to the reference row
-#pragma unroll
-            for (int m = 0; m < 8; ++m)
-#pragma unroll
-                for (int i = 0; i < 4; ++i) G[m][i] += pre[i] - ref[i];
-            if (warp == 0)
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    sGam[4 * lane + i] = __expf(tot[i] - ref[i]);
-                    sRef[4 * lane + i] = __expf(ref[i]);
-                }
-        }
-        {
-            const unsigned char *rq = sm + RAW_Q, *rk = sm + RAW_K;
-            const float *rb = reinterpret_cast<const float *>(sm + RAW_B);
+        cumsum_finish(reinterpret_cast<const float *>(sm + SCR_SCAN), warp, lane, G, sGam, sRef);
+        big = fmaxf(big, write_factors(sm + RAW_Q, sm + RAW_K, reinterpret_cast<const float *>(sm + RAW_B),
+                                       G, sm + OP_QB, sm + OP_KC, sm + OP_KH, warp, lane));
+        if (lane < 16) {
 #pragma unroll
             for (int m = 0; m < 8; ++m) {
                 const int r = 8 * warp + m;
-                uint2 qr = *reinterpret_cast<const uint2 *>(rq + r * 256 + lane * 8);
-                uint2 kr = *reinterpret_cast<const uint2 *>(rk + r * 256 + lane * 8);
-                float4 bv = *reinterpret_cast<const float4 *>(rb + r * 128 + 4 * lane);
-                const __nv_bfloat162 *q2 = reinterpret_cast<const __nv_bfloat162 *>(&qr);
-                const __nv_bfloat162 *k2 = reinterpret_cast<const __nv_bfloat162 *>(&kr);
-                float qf[4] = {__low2float(q2[0]), __high2float(q2[0]), __low2float(q2[1]), __high2float(q2[1])};
-                float kf[4] = {__low2float(k2[0]), __high2float(k2[0]), __low2float(k2[1]), __high2float(k2[1])};
-                float bf[4] = {bv.x, bv.y, bv.z, bv.w};
-                float qb[4], kc[4], kh[4];
+                uint2 vr = *reinterpret_cast<const uint2 *>(sm + RAW_V + r * 128 + lane * 8);
+                float4 wv = *reinterpret_cast<const float4 *>(sm + RAW_W + r * 256 + lane * 16);
+                const __nv_bfloat162 *v2 = reinterpret_cast<const __nv_bfloat162 *>(&vr);
+                float u[4] = {wv.x * __low2float(v2[0]), wv.y * __high2float(v2[0]),
+                              wv.z * __low2float(v2[1]), wv.w * __high2float(v2[1])};
+                st_h4(sm + OP_U + sw128_off(r, 4 * lane, 64), u[0], u[1], u[2], u[3]);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float ep = __expf(G[m][i]), em = __expf(-G[m][i]);
-                    qb[i] = qf[i] * ep;
-                    kc[i] = bf[i] * kf[i] * ep;
-                    kh[i] = kf[i] * em;
-                }
-                const uint32_t off = sw128_off(r, 4 * lane, 64);
-                st_h4(sm + OP_QB + off, qb[0], qb[1], qb[2], qb[3]);
-                st_h4(sm + OP_KC + off, kc[0], kc[1], kc[2], kc[3]);
-                st_h4(sm + OP_KH + off, kh[0], kh[1], kh[2], kh[3]);
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    big = fmaxf(big, fmaxf(fabsf(qb[i]), fmaxf(fabsf(kc[i]), fabsf(kh[i]))));
-                if (lane < 16) {
-                    uint2 vr = *reinterpret_cast<const uint2 *>(sm + RAW_V + r * 128 + lane * 8);
-                    float4 wv = *reinterpret_cast<const float4 *>(sm + RAW_W + r * 256 + lane * 16);
-                    const __nv_bfloat162 *v2 = reinterpret_cast<const __nv_bfloat162 *>(&vr);
-                    float u[4] = {wv.x * __low2float(v2[0]), wv.y * __high2float(v2[0]),
-                                  wv.z * __low2float(v2[1]), wv.w * __high2float(v2[1])};
-                    st_h4(sm + OP_U + sw128_off(r, 4 * lane, 64), u[0], u[1], u[2], u[3]);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) big = fmaxf(big, fabsf(u[i]));
-                }
+                for (int i = 0; i < 4; ++i) big = fmaxf(big, fabsf(u[i]));
             }
         }
-        if (tid == 0 && ckpt) bulk_wait_read();  // OP_S is rewritten just below
+        if (tid == 0 && ws) bulk_wait_read();  // OP_S is rewritten just below
         __syncthreads();
         // state in the chunk's reference frame: S_m = diag(e^G_m) S (TMEM and fp16 copy)
         {
@@ -327,51 +295,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CU
             }
         }
         if (__syncthreads_or(!ok)) { abort = true; break; }
-        // diagonal 16x16 blocks, one column per thread; zero the upper blocks
-        if (tid < 64) {
-            const int o16 = (tid >> 4) * 16, cl = tid & 15;
-            float x[16];
-#pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                float acc = r == cl ? 1.f : 0.f;
-#pragma unroll
-                for (int j = 0; j < r; ++j) acc -= sA[(o16 + r) * 65 + o16 + j] * x[j];
-                x[r] = acc;
-            }
-#pragma unroll
-            for (int r = 0; r < 16; ++r) sT[(o16 + r) * 65 + o16 + cl] = x[r];
-        }
-        for (int e = tid; e < 64 * 64; e += kThreads) {
-            const int r = e >> 6, j = e & 63;
-            if ((j >> 4) > (r >> 4)) sT[r * 65 + j] = 0.f;
-        }
-        __syncthreads();
-        // block levels: T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ, I - J = lvl
-        float *sM = reinterpret_cast<float *>(sm + SCR_M);
-        for (int lvl = 1; lvl < 4; ++lvl) {
-            const int nb = 4 - lvl;
-            for (int e = tid; e < nb * 256; e += kThreads) {
-                const int bi = e >> 8, r = (e >> 4) & 15, cl = e & 15;
-                const int I = bi + lvl, J = bi;
-                float acc = 0.f;
-                for (int K = J; K < I; ++K)
-#pragma unroll
-                    for (int kk = 0; kk < 16; ++kk)
-                        acc += sA[(16 * I + r) * 65 + 16 * K + kk] * sT[(16 * K + kk) * 65 + 16 * J + cl];
-                sM[bi * 272 + r * 17 + cl] = acc;
-            }
-            __syncthreads();
-            for (int e = tid; e < nb * 256; e += kThreads) {
-                const int bi = e >> 8, r = (e >> 4) & 15, cl = e & 15;
-                const int I = bi + lvl, J = bi;
-                float acc = 0.f;
-#pragma unroll
-                for (int kk = 0; kk < 16; ++kk)
-                    acc += sT[(16 * I + r) * 65 + 16 * I + kk] * sM[bi * 272 + kk * 17 + cl];
-                sT[(16 * I + r) * 65 + 16 * J + cl] = -acc;
-            }
-            __syncthreads();
-        }
+        invert_unit_lower(sA, sT, reinterpret_cast<float *>(sm + SCR_M), tid);
         for (int e = tid; e < 64 * 8; e += kThreads) {
             const int r = e >> 3, jj = e & 7;
             st_h8(sm + OP_T + sw128_chunk(r, jj, 64), sT + r * 65 + 8 * jj);
@@ -383,6 +307,12 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CU
         if (tid == 0) {
             fence_after_sync();
             if (c + 1 < NC) load_gb(c + 1);
+            if (ws && vh == 0) {  // T and P of this chunk, for the backward
+                unsigned char *dst = ws + lay.ckTP + (bh * NC + c) * 16384;
+                bulk_store(dst, sm + OP_T, 8192);
+                bulk_store(dst + 8192, sm + OP_P, 8192);
+                bulk_commit();
+            }
             const uint32_t t = smem_addr(sm + OP_T), kc = smem_addr(sm + OP_KC),
                            u = smem_addr(sm + OP_U);
 #pragma unroll
@@ -428,18 +358,18 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CU
         ok = mbar_wait(&bars[4], par, kWait);
         fence_after_sync();
         {
-            float ws[32];
-            tmem_ld16(taddr(tm + TM_WS, quarter * 32, 32 * half), ws);
-            tmem_ld16(taddr(tm + TM_WS, quarter * 32, 32 * half + 16), ws + 16);
+            float ws_[32];
+            tmem_ld16(taddr(tm + TM_WS, quarter * 32, 32 * half), ws_);
+            tmem_ld16(taddr(tm + TM_WS, quarter * 32, 32 * half + 16), ws_ + 16);
             tmem_wait_ld();
             if (lane < 16) {
                 const int r = quarter * 16 + lane;
 #pragma unroll
-                for (int j = 0; j < 32; ++j) ws[j] = up[j] - ws[j];
+                for (int j = 0; j < 32; ++j) ws_[j] = up[j] - ws_[j];
 #pragma unroll
                 for (int jj = 0; jj < 4; ++jj) {
-                    st_h8(sm + OP_U + sw128_chunk(r, 4 * half + jj, 64), ws + 8 * jj);
-                    big = absmax8(ws + 8 * jj, big);
+                    st_h8(sm + OP_U + sw128_chunk(r, 4 * half + jj, 64), ws_ + 8 * jj);
+                    big = absmax8(ws_ + 8 * jj, big);
                 }
             }
         }
@@ -448,6 +378,10 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CU
         if (__syncthreads_or(!ok)) { abort = true; break; }
         if (tid == 0) {
             fence_after_sync();
+            if (ws) {  // Delta of this chunk and half, for the backward
+                bulk_store(ws + lay.ckD + ((bh * NC + c) * 2 + vh) * 8192, sm + OP_U, 8192);
+                bulk_commit();
+            }
             const uint32_t p = smem_addr(sm + OP_P), dl = smem_addr(sm + OP_U),
                            kh = smem_addr(sm + OP_KH);
 #pragma unroll
@@ -468,7 +402,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CU
             tmem_wait_ld();
             if (lane < 16) {
                 const int r = quarter * 16 + lane;
-                if (c0 + r < T) {
+                if (o && c0 + r < T) {
                     unsigned char *dst = reinterpret_cast<unsigned char *>(
                         o + tok(d, bb, c0 + r, h, 128) + v0 + 32 * half);
 #pragma unroll
@@ -498,17 +432,19 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CU
             }
             tmem_wait_st();
         }
+        // the T/P and Delta copies read OP_T, OP_P and OP_U, all rewritten next chunk
+        if (tid == 0 && ws) bulk_wait_read();
         fence_proxy_async();
         fence_before_sync();
         if (__syncthreads_or(!ok)) { abort = true; break; }
-        if (tid == 0 && ckpt && c + 1 < NC) {
-            bulk_store(ckpt + ((ck_head + c + 1) * 2 + vh) * 8192, sm + OP_S, 16384);
+        if (tid == 0 && ws) {  // S_{c+1} (S_T after the last chunk), true scale
+            bulk_store(ws + lay.ckS + ((bh * (NC + 1) + c + 1) * 2 + vh) * 16384, sm + OP_S, 16384);
             bulk_commit();
         }
     }
     if (!(big <= kRange)) record_status(status, GDN2_ERR_RANGE);
     if (tid == 0) {
-        if (ckpt) bulk_wait_all();
+        if (ws) bulk_wait_all();
         if (abort) {
             record_status(status, GDN2_ERR_TIMEOUT);
             // let every requested tile land before the CTA's shared memory goes away
@@ -522,11 +458,9 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CU
 }
 
 // ---------------------------------------------------------------- launcher
-size_t tc_fwd_ckpt_bytes(const Dims &d) { return (size_t)d.B * d.H * d.NC * 2 * 16384; }
-
 cudaError_t tc_fwd_launch(const void *q, const void *k, const void *v, const float *g,
                           const float *b, const float *w, const float *S0, void *o, float *ST,
-                          void *ckpt, unsigned int *status, const Dims &d, cudaStream_t s) {
+                          void *ws, unsigned int *status, const Dims &d, cudaStream_t s) {
     CUtensorMap mq, mk, mv, mg, mb, mw;
     if (!make_btHd_map(&mq, q, true, d.B, d.T, d.H, 128, 64, 128) ||
         !make_btHd_map(&mk, k, true, d.B, d.T, d.H, 128, 64, 128) ||
@@ -540,7 +474,8 @@ cudaError_t tc_fwd_launch(const void *q, const void *k, const void *v, const flo
     if (e != cudaSuccess) return e;
     count_launches(1);
     tc_fwd_kernel<<<dim3(2, d.H, d.B), tfwd::kThreads, tfwd::SMEM_BYTES, s>>>(
-        mq, mk, mv, mg, mb, mw, S0, (__nv_bfloat16 *)o, ST, (__nv_bfloat16 *)ckpt, status, d);
+        mq, mk, mv, mg, mb, mw, S0, (__nv_bfloat16 *)o, ST, (unsigned char *)ws, tc_ws_layout(d),
+        status, d);
     return cudaGetLastError();
 }
 

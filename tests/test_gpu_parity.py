@@ -154,23 +154,24 @@ def test_backward_recompute_equals_reuse_and_is_deterministic():
         assert torch.equal(a[n], b[n]), n
 
 
-def test_every_output_written_and_no_nan_read():
+@pytest.mark.parametrize("dk,chunk", [(64, 32), (128, 64)])
+def test_every_output_written_and_no_nan_read(dk, chunk):
     """Outputs and workspace pre-filled with NaN: every output element must be
     written, and nothing uninitialised may reach an output."""
-    x = workloads.draw(1, 100, 2, 64, 64, 92, s0_std=0.1, with_dST=True)
+    B, T, H, dv = 1, 100, 2, dk
+    x = workloads.draw(B, T, H, dk, dv, 92, s0_std=0.1, with_dST=True)
     d = to_device(x, "bf16")
-    B, T, H, dk, dv = 1, 100, 2, 64, 64
-    ws = gdn.workspace(B, T, H, dk, dv, 32, 1, True)
+    ws = gdn.workspace(B, T, H, dk, dv, chunk, 1, True)
     ws.view(torch.uint8).fill_(0xFF)   # NaN pattern in every float32 slot
     o = torch.full((B, T, H, dv), float("nan"), dtype=torch.bfloat16, device="cuda")
     ST = torch.full((B, H, dk, dv), float("nan"), device="cuda")
-    gdn.gdn2_fwd(*(d[n] for n in NAMES), o, ST, ws, ws.numel(), B, T, H, dk, dv, 32, 1)
+    gdn.gdn2_fwd(*(d[n] for n in NAMES), o, ST, ws, ws.numel(), B, T, H, dk, dv, chunk, 1)
     outs = {n: torch.full_like(d[m], float("nan")) for n, m in
             (("dq", "q"), ("dk", "k"), ("dv", "v"), ("dg", "g"), ("db", "b"), ("dw", "w"))}
     outs["dS0"] = torch.full_like(ST, float("nan"))
     gdn.gdn2_bwd(*(d[n] for n in NAMES), d["dO"], d["dST"], outs["dq"], outs["dk"], outs["dv"],
                  outs["dg"], outs["db"], outs["dw"], outs["dS0"], ws, ws.numel(), 1,
-                 B, T, H, dk, dv, 32, 1)
+                 B, T, H, dk, dv, chunk, 1)
     torch.cuda.synchronize()
     for n, t in list(outs.items()) + [("o", o), ("ST", ST)]:
         assert torch.isfinite(t.float()).all(), n
