@@ -37,6 +37,15 @@ NAMES = ("q", "k", "v", "g", "b", "w", "S0")
 # algorithmic bytes per token-head (bf16 q,k,v,o,dO,dq,dk,dv; f32 g,b,w,dg,db,dw)
 FWD_BYTES = 3 * 128 * 2 + 3 * 128 * 4 + 128 * 2           # 2560
 BWD_BYTES = 3 * 128 * 2 + 3 * 128 * 4 + 128 * 2 + 3 * 128 * 2 + 3 * 128 * 4   # 4864
+# ... attributed to the kernel that first reads (or writes) each tensor
+KERNEL_BYTES = {
+    "tc_fwd": FWD_BYTES,
+    # q, k, g, b, dO, v, w read; dv, dw written
+    "tc_bwd_state": 2 * 128 * 2 + 2 * 128 * 4 + 128 * 2 + 128 * 2 + 128 * 4 + 128 * 2 + 128 * 4,
+    # dq, dk, db, dg written
+    "tc_bwd_grad": 2 * 128 * 2 + 2 * 128 * 4,
+}
+assert KERNEL_BYTES["tc_bwd_state"] + KERNEL_BYTES["tc_bwd_grad"] == BWD_BYTES
 
 
 def parse():
@@ -47,6 +56,8 @@ def parse():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--batch", type=int, default=None,
+                   help="override B (smaller cases for profiling captures only)")
     return p.parse_args()
 
 
@@ -150,7 +161,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     wl = workloads.WORKLOADS[WORKLOAD_INDEX]
-    B, T, H, dk, dv, C = wl.B, wl.T, wl.H, wl.dk, wl.dv, wl.chunk
+    B, T, H, dk, dv, C = args.batch or wl.B, wl.T, wl.H, wl.dk, wl.dv, wl.chunk
     x = workloads.draw(B, T, H, dk, dv, wl.seed + 7919 * rank, s0_std=wl.s0_std,
                        erase_scale=wl.erase_scale)
     io_names = ("q", "k", "v", "dO")
@@ -191,6 +202,7 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     torch.cuda.synchronize(dev)
     launches0 = gdn.gdn2_kernel_launches()
+    gdn.gdn2_set_kernel_timer(True)
     sampler.mark_start()
     start.record(stream)
     for i in range(args.steps):
@@ -208,6 +220,8 @@ def run_ours(args, rank, world, local_rank):
     sampler.mark_end()
     barrier()
     launches = gdn.gdn2_kernel_launches() - launches0
+    ktimes = gdn.gdn2_kernel_times()
+    gdn.gdn2_set_kernel_timer(False)
     ms_total = start.elapsed_time(end)
     fwd_ms = statistics.mean(a.elapsed_time(b) for a, b, _ in ev)
     bwd_ms = statistics.mean(b.elapsed_time(c) for _, b, c in ev)
@@ -249,26 +263,44 @@ def run_ours(args, rank, world, local_rank):
     value = tokens / (ms_step * 1e-3)
     token_heads = B * T * H
     alg_bytes = token_heads * (FWD_BYTES + BWD_BYTES)
-    achieved = alg_bytes / (ms_step * 1e-3) / 1e9
     peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) \
         if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")) else {}
     peak = peaks.get("hbm_gbs", 6650.0)
-    peak_src = "measured" if "hbm_gbs" in peaks else "fallback"
-    traffic = traffic_from_profiles("fwd+bwd step, workload 2", sources_hash())
+    peak_src = "of measured" if "hbm_gbs" in peaks else "of fallback"
+    src = sources_hash()
+    kernels = {}
+    for name, (cnt, tot) in ktimes.items():
+        avg = tot / cnt
+        per = KERNEL_BYTES.get(name)
+        ent = {"launches": cnt, "avg_ms": avg}
+        if per is not None:
+            gbs = per * token_heads / (avg * 1e-3) / 1e9
+            ent.update(alg_bytes_per_launch=per * token_heads, achieved_gbs=gbs, frac=gbs / peak)
+        kernels[name] = ent
+    dom = max(kernels, key=lambda n: kernels[n]["launches"] * kernels[n]["avg_ms"])
+    dk_ = kernels[dom]
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": dk_.get("achieved_gbs"), "peak": peak,
+                "unit": "GB/s", "frac": dk_.get("frac"), "peak_source": peak_src,
+                "alg_bytes_per_launch": dk_.get("alg_bytes_per_launch"),
+                "avg_launch_ms": dk_["avg_ms"],
+                "traffic": traffic_from_profiles(dom, src)}
+    step_achieved = alg_bytes / (ms_step * 1e-3) / 1e9
+    roofline_step = {"bound": "hbm", "achieved": step_achieved, "peak": peak, "unit": "GB/s",
+                     "frac": step_achieved / peak, "alg_bytes_per_step": alg_bytes}
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f32", "data": "synthetic (seeded; BASELINE workload generators)",
+        "dtype": "f16", "data": "synthetic (seeded; BASELINE workload generators)",
         "config": {"workload": wl.name, "B": B, "T": T, "H": H, "d_k": dk, "d_v": dv,
                    "chunk": C, "io": "bf16 q/k/v/o/dO/dq/dk/dv, f32 g/b/w/state",
                    "global_batch": B * world, "seq_len": T, "parallelism": f"dp{world}",
-                   "l2": "inputs 0.67 GB per step (> 126 MB L2), no flush"},
+                   "l2": "inputs 0.67 GB per step (> 126 MB L2), no flush",
+                   "arithmetic": "fp16 tensor-core operands, fp32 accumulation and state"},
         "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
-        "roofline": {"bound": "hbm", "kernel": "whole fwd+bwd step (all launches)",
-                     "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "peak_source": peak_src,
-                     "algorithmic_bytes_per_step": alg_bytes, "traffic": traffic},
+        "roofline": roofline,
+        "roofline_step": roofline_step,
+        "kernels": kernels,
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches,

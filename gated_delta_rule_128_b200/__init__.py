@@ -71,6 +71,14 @@ def lib() -> ctypes.CDLL:
         L.gdn2_fwd_noalloc.restype = i
         L.gdn2_kernel_launches.argtypes = []
         L.gdn2_kernel_launches.restype = ctypes.c_ulonglong
+        L.gdn2_set_kernel_timer.argtypes = [i]
+        L.gdn2_set_kernel_timer.restype = None
+        L.gdn2_kernel_kinds.argtypes = []
+        L.gdn2_kernel_kinds.restype = i
+        L.gdn2_kernel_name.argtypes = [i]
+        L.gdn2_kernel_name.restype = ctypes.c_char_p
+        L.gdn2_kernel_times.argtypes = [vp, vp, i]
+        L.gdn2_kernel_times.restype = i
         _lib = L
     return _lib
 
@@ -142,6 +150,21 @@ def gdn2_get_device_status(stream=None) -> int:
 
 def gdn2_kernel_launches() -> int:
     return int(lib().gdn2_kernel_launches())
+
+
+def gdn2_set_kernel_timer(enable: bool) -> None:
+    lib().gdn2_set_kernel_timer(int(enable))
+
+
+def gdn2_kernel_times() -> Dict[str, tuple]:
+    """{kernel name: (launches, total ms)} for the kernels timed since the
+    timer was enabled (only kinds that launched)."""
+    n = lib().gdn2_kernel_kinds()
+    counts = (ctypes.c_ulonglong * n)()
+    ms = (ctypes.c_double * n)()
+    _check("gdn2_kernel_times", lib().gdn2_kernel_times(ctypes.cast(counts, ctypes.c_void_p),
+                                                         ctypes.cast(ms, ctypes.c_void_p), n))
+    return {lib().gdn2_kernel_name(i).decode(): (counts[i], ms[i]) for i in range(n) if counts[i]}
 
 
 # ------------------------------------------------------- tensor conveniences

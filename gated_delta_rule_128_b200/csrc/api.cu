@@ -6,6 +6,7 @@
 
 #include <atomic>
 #include <mutex>
+#include <vector>
 
 #include "common.cuh"
 
@@ -57,7 +58,44 @@ static bool use_tc(const Dims &d, gdn2_io io) {
 }
 
 static std::atomic<unsigned long long> g_launches{0};
-void count_launches(unsigned long long n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+// ---- optional per-kernel event timing (gdn2_set_kernel_timer)
+struct PendingTiming {
+    int kind;
+    cudaEvent_t start, end;
+};
+static std::mutex g_timer_mu;
+static std::atomic<bool> g_timer_on{false};
+static std::vector<PendingTiming> g_pending;
+static cudaEvent_t g_open_start[K_KINDS];
+static unsigned long long g_kind_count[K_KINDS];
+static double g_kind_ms[K_KINDS];
+static const char *const g_kind_names[K_KINDS] = {
+    "simt_chunk_prep", "simt_state_fwd", "simt_out_fwd", "simt_state_bwd", "simt_chunk_bwd_a",
+    "simt_chunk_bwd_b", "decode_step", "tc_fwd", "tc_bwd_state", "tc_bwd_grad"};
+
+void launch_begin(int kind, cudaStream_t s) {
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    if (!g_timer_on.load(std::memory_order_relaxed)) return;
+    std::lock_guard<std::mutex> lock(g_timer_mu);
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) == cudaSuccess) cudaEventRecord(e, s);
+    g_open_start[kind] = e;
+}
+
+void launch_end(int kind, cudaStream_t s) {
+    if (!g_timer_on.load(std::memory_order_relaxed)) return;
+    std::lock_guard<std::mutex> lock(g_timer_mu);
+    cudaEvent_t st = g_open_start[kind], e = nullptr;
+    g_open_start[kind] = nullptr;
+    if (!st) return;
+    if (cudaEventCreate(&e) != cudaSuccess) {
+        cudaEventDestroy(st);
+        return;
+    }
+    cudaEventRecord(e, s);
+    g_pending.push_back({kind, st, e});
+}
 
 static bool supported_d(int x) { return x == 32 || x == 64 || x == 128; }
 static bool supported_chunk(int c) { return c == 16 || c == 32 || c == 64; }
@@ -219,5 +257,46 @@ const char *gdn2_status_string(gdn2_status status) {
 int gdn2_version(void) { return 100; }
 
 unsigned long long gdn2_kernel_launches(void) { return g_launches.load(); }
+
+void gdn2_set_kernel_timer(int enable) {
+    std::lock_guard<std::mutex> lock(g_timer_mu);
+    for (auto &p : g_pending) {
+        cudaEventDestroy(p.start);
+        cudaEventDestroy(p.end);
+    }
+    g_pending.clear();
+    for (int i = 0; i < K_KINDS; ++i) {
+        g_kind_count[i] = 0;
+        g_kind_ms[i] = 0.0;
+    }
+    g_timer_on.store(enable != 0);
+}
+
+int gdn2_kernel_kinds(void) { return K_KINDS; }
+
+const char *gdn2_kernel_name(int id) { return id >= 0 && id < K_KINDS ? g_kind_names[id] : nullptr; }
+
+gdn2_status gdn2_kernel_times(unsigned long long *count, double *ms, int n) {
+    std::lock_guard<std::mutex> lock(g_timer_mu);
+    gdn2_status st = GDN2_OK;
+    for (auto &p : g_pending) {
+        float t = 0.f;
+        if (cudaEventSynchronize(p.end) != cudaSuccess ||
+            cudaEventElapsedTime(&t, p.start, p.end) != cudaSuccess)
+            st = GDN2_ERR_CUDA;
+        else {
+            g_kind_count[p.kind] += 1;
+            g_kind_ms[p.kind] += t;
+        }
+        cudaEventDestroy(p.start);
+        cudaEventDestroy(p.end);
+    }
+    g_pending.clear();
+    for (int i = 0; i < n && i < K_KINDS; ++i) {
+        if (count) count[i] = g_kind_count[i];
+        if (ms) ms[i] = g_kind_ms[i];
+    }
+    return st;
+}
 
 }  // extern "C"

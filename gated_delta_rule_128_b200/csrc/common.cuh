@@ -69,8 +69,14 @@ struct SimtWs {
     size_t bwd_end;
 };
 
-// ---- host-side launch counter (gdn2_kernel_launches)
-void count_launches(unsigned long long n);
+// ---- host-side launch accounting: every launch site brackets its launch
+// with launch_begin / launch_end (kernel kind ids below)
+enum KernelKind {
+    K_SIMT_PREP = 0, K_SIMT_STATE_FWD, K_SIMT_OUT, K_SIMT_STATE_BWD, K_SIMT_BWD_A, K_SIMT_BWD_B,
+    K_DECODE, K_TC_FWD, K_TC_BWD_STATE, K_TC_BWD_GRAD, K_KINDS
+};
+void launch_begin(int kind, cudaStream_t s);
+void launch_end(int kind, cudaStream_t s);
 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 

@@ -105,9 +105,10 @@ template <typename E, int DK, int DV>
 static cudaError_t launch_dec(const void *q, const void *k, const void *v, const float *g,
                               const float *b, const float *w, float *S, void *o, int N, int H,
                               cudaStream_t s) {
-    count_launches(1);
+    launch_begin(K_DECODE, s);
     decode_step_kernel<E, DK, DV><<<(unsigned)N * (unsigned)H, kDecThreads, 0, s>>>(
         (const E *)q, (const E *)k, (const E *)v, g, b, w, S, (E *)o, H);
+    launch_end(K_DECODE, s);
     return cudaGetLastError();
 }
 

@@ -275,22 +275,25 @@ cudaError_t simt_bwd_launch(const void *q, const void *k, const void *v, const f
     size_t sm1 = sizeof(float) * ((size_t)d.dk * kSliceB + 3 * (size_t)d.C * d.dk + d.C * d.C +
                                   2 * d.C * kSliceB + d.dk);
     if ((e = allow_smem_b(simt_state_bwd<E>, sm1)) != cudaSuccess) return e;
-    count_launches(1);
+    launch_begin(K_SIMT_STATE_BWD, s);
     simt_state_bwd<E><<<dim3(d.dv / kSliceB, d.H, d.B), kThreadsB, sm1, s>>>(
         (const E *)q, (const E *)k, (const E *)dO, dST, dS0, ws, lay, d);
+    launch_end(K_SIMT_STATE_BWD, s);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     size_t sm2 = sizeof(float) * ((size_t)d.C * d.C + 4 * (size_t)d.C * (d.dv + 1) +
                                   (size_t)d.dk * (d.dv + 1));
     if ((e = allow_smem_b(simt_chunk_bwd_a<E>, sm2)) != cudaSuccess) return e;
-    count_launches(1);
+    launch_begin(K_SIMT_BWD_A, s);
     simt_chunk_bwd_a<E><<<dim3(d.NC, d.H, d.B), kThreadsB, sm2, s>>>(
         (const E *)v, w, (const E *)dO, (E *)dv, dw, ws, lay, d);
+    launch_end(K_SIMT_BWD_A, s);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     size_t sm3 = sizeof(float) * (5 * (size_t)d.dk * (d.C + 1) + 2 * (size_t)d.C * d.C);
     if ((e = allow_smem_b(simt_chunk_bwd_b<E>, sm3)) != cudaSuccess) return e;
-    count_launches(1);
+    launch_begin(K_SIMT_BWD_B, s);
     simt_chunk_bwd_b<E><<<dim3(d.NC, d.H, d.B), kThreadsB, sm3, s>>>(
         (const E *)q, (const E *)k, b, (E *)dq, (E *)dk, db, dg, ws, lay, d);
+    launch_end(K_SIMT_BWD_B, s);
     return cudaGetLastError();
 }
 

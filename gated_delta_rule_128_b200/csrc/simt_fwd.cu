@@ -257,9 +257,10 @@ cudaError_t simt_prep_launch(const void *q, const void *k, const void *v, const 
     size_t sm = prep_smem(d);
     cudaError_t e = allow_smem(simt_chunk_prep<E>, sm);
     if (e != cudaSuccess) return e;
-    count_launches(1);
+    launch_begin(K_SIMT_PREP, s);
     simt_chunk_prep<E><<<dim3(d.NC, d.H, d.B), kThreads, sm, s>>>(
         (const E *)q, (const E *)k, (const E *)v, g, b, w, ws, lay, d);
+    launch_end(K_SIMT_PREP, s);
     return cudaGetLastError();
 }
 
@@ -269,9 +270,10 @@ cudaError_t simt_state_fwd_launch(const float *S0, float *ST, const void *k, int
     size_t sm = state_smem(d);
     cudaError_t e = allow_smem(simt_state_fwd_kernel, sm);
     if (e != cudaSuccess) return e;
-    count_launches(1);
+    launch_begin(K_SIMT_STATE_FWD, s);
     simt_state_fwd_kernel<<<dim3(d.dv / kSlice, d.H, d.B), kThreads, sm, s>>>(S0, ST, k, k_is_bf16,
                                                                               ws, lay, d);
+    launch_end(K_SIMT_STATE_FWD, s);
     return cudaGetLastError();
 }
 
@@ -281,8 +283,9 @@ cudaError_t simt_out_launch(const void *q, void *o, void *ws, const Dims &d, cud
     size_t sm = out_smem(d);
     cudaError_t e = allow_smem(simt_out_fwd<E>, sm);
     if (e != cudaSuccess) return e;
-    count_launches(1);
+    launch_begin(K_SIMT_OUT, s);
     simt_out_fwd<E><<<dim3(d.NC, d.H, d.B), kThreads, sm, s>>>((const E *)q, (E *)o, ws, lay, d);
+    launch_end(K_SIMT_OUT, s);
     return cudaGetLastError();
 }
 

@@ -78,7 +78,7 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
     float *sEnd = reinterpret_cast<float *>(sm + MISC + 1024);  // [2][128]
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + MISC + 2048);  // 0..7
     uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + MISC + 2048 + 64);
-    float big = 0.f;
+    float big = 0.f, gbig = 0.f;  // range checks: operand magnitude, |G - G_m|
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int vh = blockIdx.x, h = blockIdx.y, bb = blockIdx.z, v0 = vh * 64;
@@ -177,7 +177,7 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
                      warp, lane, G);
         if (__syncthreads_or(!ok)) { abort = true; break; }
         cumsum_finish(reinterpret_cast<const float *>(sm + SCR_SCAN), warp, lane, G, sGam, sRef);
-        big = fmaxf(big, write_factors(sm + RAW_Q, sm + RAW_K, reinterpret_cast<const float *>(sm + RAW_B),
+        gbig = fmaxf(gbig, write_factors(sm + RAW_Q, sm + RAW_K, reinterpret_cast<const float *>(sm + RAW_B),
                                        G, sm + OP_QB, sm + OP_KC, sm + OP_KH, warp, lane));
         if (lane < 16) {  // dO half -> fp16 operand [pos][v]
 #pragma unroll
@@ -360,7 +360,7 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
             ++issued[3];
         }
     }
-    if (!(big <= kRange)) record_status(status, GDN2_ERR_RANGE);
+    if (!(big <= kRange) || !(gbig <= 9.f)) record_status(status, GDN2_ERR_RANGE);
     if (tid == 0) {
         bulk_wait_all();
         if (abort) {
@@ -414,7 +414,7 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
     float *scan = reinterpret_cast<float *>(sm + MISC + 1536);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + MISC + 1536 + 4096);
     uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + MISC + 1536 + 4096 + 64);
-    float big = 0.f;
+    float big = 0.f, gbig = 0.f;  // range checks: operand magnitude, |G - G_m|
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int c = blockIdx.x, h = blockIdx.y, bb = blockIdx.z, c0 = c * 64;
@@ -527,7 +527,7 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
                 }
             }
         }
-        big = fmaxf(big, write_factors(sm + RAW_Q, sm + RAW_K, reinterpret_cast<const float *>(sm + RAW_B),
+        gbig = fmaxf(gbig, write_factors(sm + RAW_Q, sm + RAW_K, reinterpret_cast<const float *>(sm + RAW_B),
                                        G, sm + OP_QB, sm + OP_KC, sm + OP_KH, warp, lane));
         fence_proxy_async();
         fence_before_sync();
@@ -605,7 +605,7 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
             }
         }
     }
-    if (!(big <= kRange)) record_status(status, GDN2_ERR_RANGE);
+    if (!(big <= kRange) || !(gbig <= 9.f)) record_status(status, GDN2_ERR_RANGE);
     if (abort && tid == 0) {
         record_status(status, GDN2_ERR_TIMEOUT);
         mbar_wait(&bars[0], 0, kWait);
@@ -636,15 +636,17 @@ cudaError_t tc_bwd_launch(const void *q, const void *k, const void *v, const flo
     e = cudaFuncSetAttribute(tc_bwd_grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)tbg::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    count_launches(1);
+    launch_begin(K_TC_BWD_STATE, s);
     tc_bwd_state_kernel<<<dim3(2, d.H, d.B), tbs::kThreads, tbs::SMEM_BYTES, s>>>(
         mq, mk, mdo_half, mg, mb, (const __nv_bfloat16 *)v, w, dST, (__nv_bfloat16 *)dv, dw, dS0,
         (unsigned char *)ws, lay, status, d);
+    launch_end(K_TC_BWD_STATE, s);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    count_launches(1);
+    launch_begin(K_TC_BWD_GRAD, s);
     tc_bwd_grad_kernel<<<dim3(d.NC, d.H, d.B), tbg::kThreads, tbg::SMEM_BYTES, s>>>(
         mq, mk, mdo, mg, mb, (__nv_bfloat16 *)dq, (__nv_bfloat16 *)dk, db, dg, (unsigned char *)ws,
         lay, status, d);
+    launch_end(K_TC_BWD_GRAD, s);
     return cudaGetLastError();
 }
 

@@ -67,10 +67,40 @@ constexpr long long kWait = 2000000000LL;  // ~1 s of SM clocks per wait
 constexpr float kRange = 6.0e4f;           // largest operand magnitude kept in fp16
 }  // namespace tfwd
 
+// Warp-level tensor-core tile product D = A B + C (m16n8k8, tf32 operands,
+// f32 accumulate) for the small 16x16 block products of the T inversion.
+// Fragment layout (g = lane / 4, t = lane % 4): a0 (g, t), a1 (g + 8, t),
+// a2 (g, t + 4), a3 (g + 8, t + 4); b0 (t, g), b1 (t + 4, g);
+// c0 (g, 2t), c1 (g, 2t + 1), c2 (g + 8, 2t), c3 (g + 8, 2t + 1).
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ void mma_tf32_16x8x8(float *c, const uint32_t *a, const uint32_t *b) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+// c += X[r0.., k0..k0+8) * Y[k0..k0+8, n0..n0+8) for row-major [.][65] f32 tiles
+__device__ __forceinline__ void tile_mma(float *c, const float *X, int r0, int k0, const float *Y,
+                                         int n0, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    uint32_t a[4] = {to_tf32(X[(r0 + g) * 65 + k0 + t]), to_tf32(X[(r0 + g + 8) * 65 + k0 + t]),
+                     to_tf32(X[(r0 + g) * 65 + k0 + t + 4]), to_tf32(X[(r0 + g + 8) * 65 + k0 + t + 4])};
+    uint32_t b[2] = {to_tf32(Y[(k0 + t) * 65 + n0 + g]), to_tf32(Y[(k0 + t + 4) * 65 + n0 + g])};
+    mma_tf32_16x8x8(c, a, b);
+}
+
 // T = (I + A)^-1 for the strictly-lower 64x64 A in sA ([64][65] f32), into
-// sT ([64][65] f32): 16x16 diagonal blocks by forward substitution (one
-// column per thread), then T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ level by
-// level.  All 256 threads; ends with a barrier.
+// sT ([64][65] f32), by blocks of 16: the diagonal blocks by forward
+// substitution (one column per thread), then level by level
+// T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ (I - J = 1, 2, 3) as warp-level
+// tf32 tile products, each warp owning 8 columns of one block.  sM holds one
+// 16x8 intermediate per warp ([8][16][9] f32).  All 256 threads; ends with a
+// barrier.
 __device__ __forceinline__ void invert_unit_lower(const float *sA, float *sT, float *sM, int tid) {
     if (tid < 64) {
         const int o16 = (tid >> 4) * 16, cl = tid & 15;
@@ -90,27 +120,36 @@ __device__ __forceinline__ void invert_unit_lower(const float *sA, float *sT, fl
         if ((j >> 4) > (r >> 4)) sT[r * 65 + j] = 0.f;
     }
     __syncthreads();
+    const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+    float *mw = sM + warp * 16 * 9;
     for (int lvl = 1; lvl < 4; ++lvl) {
-        const int nb = 4 - lvl;
-        for (int e = tid; e < nb * 256; e += 256) {
-            const int bi = e >> 8, r = (e >> 4) & 15, cl = e & 15;
-            const int I = bi + lvl, J = bi;
-            float acc = 0.f;
-            for (int K = J; K < I; ++K)
+        const int nb = 4 - lvl;  // blocks on this level, two warps each
+        if (warp < 2 * nb) {
+            const int J = warp >> 1, I = J + lvl, n0 = 16 * J + 8 * (warp & 1);
+            float c[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int K = J; K < I; ++K) {
+                tile_mma(c, sA, 16 * I, 16 * K, sT, n0, lane);
+                tile_mma(c, sA, 16 * I, 16 * K + 8, sT, n0, lane);
+            }
+            mw[g * 9 + 2 * t] = c[0];
+            mw[g * 9 + 2 * t + 1] = c[1];
+            mw[(g + 8) * 9 + 2 * t] = c[2];
+            mw[(g + 8) * 9 + 2 * t + 1] = c[3];
+            __syncwarp();
+            float e[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int kk = 0; kk < 16; ++kk)
-                    acc += sA[(16 * I + r) * 65 + 16 * K + kk] * sT[(16 * K + kk) * 65 + 16 * J + cl];
-            sM[bi * 272 + r * 17 + cl] = acc;
-        }
-        __syncthreads();
-        for (int e = tid; e < nb * 256; e += 256) {
-            const int bi = e >> 8, r = (e >> 4) & 15, cl = e & 15;
-            const int I = bi + lvl, J = bi;
-            float acc = 0.f;
-#pragma unroll
-            for (int kk = 0; kk < 16; ++kk)
-                acc += sT[(16 * I + r) * 65 + 16 * I + kk] * sM[bi * 272 + kk * 17 + cl];
-            sT[(16 * I + r) * 65 + 16 * J + cl] = -acc;
+            for (int k0 = 0; k0 < 16; k0 += 8) {
+                uint32_t a[4] = {to_tf32(sT[(16 * I + g) * 65 + 16 * I + k0 + t]),
+                                 to_tf32(sT[(16 * I + g + 8) * 65 + 16 * I + k0 + t]),
+                                 to_tf32(sT[(16 * I + g) * 65 + 16 * I + k0 + t + 4]),
+                                 to_tf32(sT[(16 * I + g + 8) * 65 + 16 * I + k0 + t + 4])};
+                uint32_t b[2] = {to_tf32(mw[(k0 + t) * 9 + g]), to_tf32(mw[(k0 + t + 4) * 9 + g])};
+                mma_tf32_16x8x8(e, a, b);
+            }
+            sT[(16 * I + g) * 65 + n0 + 2 * t] = -e[0];
+            sT[(16 * I + g) * 65 + n0 + 2 * t + 1] = -e[1];
+            sT[(16 * I + g + 8) * 65 + n0 + 2 * t] = -e[2];
+            sT[(16 * I + g + 8) * 65 + n0 + 2 * t + 1] = -e[3];
         }
         __syncthreads();
     }
@@ -130,7 +169,8 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CU
     float *sRef = reinterpret_cast<float *>(sm + MISC + 512);  // e^G_m
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + MISC + 1024);  // 0 qkvw, 1 gb, 2..5 mma
     uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + MISC + 1024 + 64);
-    float big = 0.f;  // largest operand magnitude seen (range check)
+    float big = 0.f;   // largest operand magnitude seen (range check)
+    float gbig = 0.f;  // largest |G - G_m| seen (range check of the decay factors)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int vh = blockIdx.x, h = blockIdx.y, bb = blockIdx.z, v0 = vh * 64;
@@ -211,7 +251,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CU
                      warp, lane, G);
         if (__syncthreads_or(!ok)) { abort = true; break; }
         cumsum_finish(reinterpret_cast<const float *>(sm + SCR_SCAN), warp, lane, G, sGam, sRef);
-        big = fmaxf(big, write_factors(sm + RAW_Q, sm + RAW_K, reinterpret_cast<const float *>(sm + RAW_B),
+        gbig = fmaxf(gbig, write_factors(sm + RAW_Q, sm + RAW_K, reinterpret_cast<const float *>(sm + RAW_B),
                                        G, sm + OP_QB, sm + OP_KC, sm + OP_KH, warp, lane));
         if (lane < 16) {
 #pragma unroll
@@ -442,7 +482,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CU
             bulk_commit();
         }
     }
-    if (!(big <= kRange)) record_status(status, GDN2_ERR_RANGE);
+    if (!(big <= kRange) || !(gbig <= 9.f)) record_status(status, GDN2_ERR_RANGE);
     if (tid == 0) {
         if (ws) bulk_wait_all();
         if (abort) {
@@ -472,10 +512,11 @@ cudaError_t tc_fwd_launch(const void *q, const void *k, const void *v, const flo
     cudaError_t e = cudaFuncSetAttribute(tc_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)tfwd::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    count_launches(1);
+    launch_begin(K_TC_FWD, s);
     tc_fwd_kernel<<<dim3(2, d.H, d.B), tfwd::kThreads, tfwd::SMEM_BYTES, s>>>(
         mq, mk, mv, mg, mb, mw, S0, (__nv_bfloat16 *)o, ST, (unsigned char *)ws, tc_ws_layout(d),
         status, d);
+    launch_end(K_TC_FWD, s);
     return cudaGetLastError();
 }
 

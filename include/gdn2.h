@@ -45,7 +45,7 @@
  *   runs on the float32 CUDA-core path.  The tensor-core path forms the decay
  *   factors relative to the middle of each chunk, so it needs every key
  *   channel's cumulative log-decay to move by at most 9 within any 32-token
- *   half-chunk (and |q|, |k| <= 8 per element, |w v| and the state below
+ *   half-chunk (and |q|, |k|, |b| <= 8 per element, |w v| and the state below
  *   6e4); a kernel that meets an input outside that range records
  *   GDN2_ERR_RANGE (the results of that call are then not valid).  The
  *   float32 path has no such limit.
@@ -178,6 +178,21 @@ int gdn2_version(void);
  * was loaded (all threads, all devices).  A diagnostic for counting launches
  * around a region of work; not tied to any entry in the pages. */
 unsigned long long gdn2_kernel_launches(void);
+
+/* Per-kernel device timing, for benchmarks.  While enabled, every kernel the
+ * library launches is bracketed by two CUDA events recorded on its launch
+ * stream; gdn2_kernel_times waits for them and adds each kernel's elapsed
+ * time to a per-kernel total.  Enabling resets the totals.  Not tied to any
+ * entry in the pages. */
+void gdn2_set_kernel_timer(int enable);
+/* Number of kernel kinds the library can launch. */
+int gdn2_kernel_kinds(void);
+/* Static name of kernel kind `id`, or NULL. */
+const char *gdn2_kernel_name(int id);
+/* Waits for the recorded events, then writes for kind i < n the launches
+ * counted (count[i]) and their summed device time in milliseconds (ms[i]).
+ * Returns GDN2_ERR_CUDA if an event query fails. */
+gdn2_status gdn2_kernel_times(unsigned long long *count, double *ms, int n);
 
 #ifdef __cplusplus
 }
