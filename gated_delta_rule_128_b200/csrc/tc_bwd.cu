@@ -226,6 +226,19 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
                 mma_bf16(tm + TM_DD, desc_kmajor(kh, 64, ks), desc_mnmajor(ds, 128, ks), ID_KM64, 1);
             mma_commit(&bars[4]);
         }
+        // v and w of this thread's row and columns, for dw and dv in phase 3:
+        // requested now so that the loads overlap phase 2
+        uint4 vreg[4];
+        float4 wreg[8];
+        const int r_own = quarter * 16 + lane;
+        const bool row_ok = lane < 16 && c0 + r_own < T;
+        {
+            const size_t ov = tok(d, bb, row_ok ? c0 + r_own : 0, h, 128) + v0 + 32 * half;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) vreg[j] = row_ok ? *reinterpret_cast<const uint4 *>(v + ov + 8 * j) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) wreg[j] = row_ok ? *reinterpret_cast<const float4 *>(w + ov + 4 * j) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
         // ---------------- phase 2: dDelta to shared memory, dU = T^T dDelta
         ok = mbar_wait(&bars[4], par, kWait);
         fence_after_sync();
@@ -264,15 +277,13 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
             tmem_wait_ld();
             if (lane < 16) {
                 const int r = quarter * 16 + lane;
-                if (c0 + r < T) {
+                if (row_ok) {
                     const size_t ov = tok(d, bb, c0 + r, h, 128) + v0 + 32 * half;
                     float dwv[32], dvv[32];
 #pragma unroll
                     for (int j = 0; j < 32; j += 8) {
-                        uint4 vr = *reinterpret_cast<const uint4 *>(v + ov + j);
-                        const __nv_bfloat162 *v2 = reinterpret_cast<const __nv_bfloat162 *>(&vr);
-                        float4 w0 = *reinterpret_cast<const float4 *>(w + ov + j);
-                        float4 w1 = *reinterpret_cast<const float4 *>(w + ov + j + 4);
+                        const __nv_bfloat162 *v2 = reinterpret_cast<const __nv_bfloat162 *>(&vreg[j / 8]);
+                        const float4 w0 = wreg[j / 4], w1 = wreg[j / 4 + 1];
                         float wf[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
@@ -549,59 +560,88 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
             mma_commit(&bars[2]);
         }
         // ---------------- G3: dq, dk, db and dG per (row, channel)
+        // The three accumulators go through shared memory (YS, [3][64][128]
+        // f32 with 16-byte chunks XOR-swizzled by row) so that every warp then
+        // walks whole rows with lanes across channels: conflict-free reads and
+        // coalesced output rows.
         ok = mbar_wait(&bars[2], 0, kWait);
         fence_after_sync();
-        float *sG = reinterpret_cast<float *>(sm + RAW_G);
-        float *sdG = reinterpret_cast<float *>(sm + SCR_DG);  // Qb/Kc/Kh are consumed
-        const float *rb = reinterpret_cast<const float *>(sm + RAW_B);
-        __syncthreads();  // every thread is past the products before dG overwrites their operands
-        const int r = quarter * 16 + lane;
+        float *YS = reinterpret_cast<float *>(sm + BL_S);  // operands of G2 are consumed
+        {
+            const int r = quarter * 16 + lane;
 #pragma unroll 1
-        for (int cb = 0; cb < 4; ++cb) {
-            const int i0 = 64 * half + 16 * cb;
-            float y1[16], y2[16], y3[16];
-            tmem_ld16(taddr(tm + TM_Y1, quarter * 32, i0), y1);
-            tmem_ld16(taddr(tm + TM_Y2, quarter * 32, i0), y2);
-            tmem_ld16(taddr(tm + TM_Y3, quarter * 32, i0), y3);
-            tmem_wait_ld();
-            if (lane < 16) {
-                float dq[16], dk[16], db[16];
-                const uint4 *q8 = reinterpret_cast<const uint4 *>(sm + RAW_Q + r * 256 + i0 * 2);
-                const uint4 *k8 = reinterpret_cast<const uint4 *>(sm + RAW_K + r * 256 + i0 * 2);
-                uint4 qv[2] = {q8[0], q8[1]}, kv[2] = {k8[0], k8[1]};
-                const __nv_bfloat16 *qh = reinterpret_cast<const __nv_bfloat16 *>(qv);
-                const __nv_bfloat16 *kh = reinterpret_cast<const __nv_bfloat16 *>(kv);
+            for (int a = 0; a < 3; ++a) {
+                const uint32_t col0 = (a == 0 ? TM_Y1 : a == 1 ? TM_Y2 : TM_Y3) + 64 * half;
+                float y[64];
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int i = i0 + e;
-                    const float E = __expf(sG[r * 128 + i]);
-                    const float qf = __bfloat162float(qh[e]), kf = __bfloat162float(kh[e]);
-                    const float bf = rb[r * 128 + i];
-                    const float dqv = y1[e] * E, dkc = y2[e] * E, dkh = y3[e] * __frcp_rn(E);
-                    dq[e] = dqv;
-                    db[e] = dkc * kf;
-                    dk[e] = dkc * bf + dkh;
-                    sdG[r * 128 + i] = dqv * qf + dkc * bf * kf - dkh * kf;
+                for (int j = 0; j < 4; ++j) tmem_ld16(taddr(tm + col0, quarter * 32, 16 * j), y + 16 * j);
+                tmem_wait_ld();
+                if (lane < 16) {
+                    float *row = YS + (a * 64 + r) * 128;
+#pragma unroll
+                    for (int ch = 0; ch < 16; ++ch) {  // logical 16-B chunk 16 * half + ch
+                        const int lc = 16 * half + ch, pc = lc ^ (r & 31);
+                        *reinterpret_cast<float4 *>(row + 4 * pc) =
+                            make_float4(y[4 * ch], y[4 * ch + 1], y[4 * ch + 2], y[4 * ch + 3]);
+                    }
                 }
-                if (r < L) {
-                    const size_t ok_ = tok(d, bb, c0 + r, h, 128) + i0;
-                    st_bf16x8(reinterpret_cast<unsigned char *>(dqout + ok_), dq);
-                    st_bf16x8(reinterpret_cast<unsigned char *>(dqout + ok_) + 16, dq + 8);
-                    st_bf16x8(reinterpret_cast<unsigned char *>(dkout + ok_), dk);
-                    st_bf16x8(reinterpret_cast<unsigned char *>(dkout + ok_) + 16, dk + 8);
+            }
+        }
+        __syncthreads();
+        {
+            const float *sG = reinterpret_cast<const float *>(sm + RAW_G);
+            const float *rb = reinterpret_cast<const float *>(sm + RAW_B);
+            float *sdG = YS;  // row r of dG overwrites row r of Y1 (read first, same warp)
+#pragma unroll 1
+            for (int i8 = 0; i8 < 8; ++i8) {
+                const int r = warp + 8 * i8, pc = lane ^ (r & 31);
+                const float4 y1 = *reinterpret_cast<const float4 *>(YS + (0 * 64 + r) * 128 + 4 * pc);
+                const float4 y2 = *reinterpret_cast<const float4 *>(YS + (1 * 64 + r) * 128 + 4 * pc);
+                const float4 y3 = *reinterpret_cast<const float4 *>(YS + (2 * 64 + r) * 128 + 4 * pc);
+                const float4 G4 = *reinterpret_cast<const float4 *>(sG + r * 128 + 4 * lane);
+                const float4 b4 = *reinterpret_cast<const float4 *>(rb + r * 128 + 4 * lane);
+                const uint2 qr = *reinterpret_cast<const uint2 *>(sm + RAW_Q + r * 256 + 8 * lane);
+                const uint2 kr = *reinterpret_cast<const uint2 *>(sm + RAW_K + r * 256 + 8 * lane);
+                const __nv_bfloat162 *q2 = reinterpret_cast<const __nv_bfloat162 *>(&qr);
+                const __nv_bfloat162 *k2 = reinterpret_cast<const __nv_bfloat162 *>(&kr);
+                const float Y1[4] = {y1.x, y1.y, y1.z, y1.w}, Y2[4] = {y2.x, y2.y, y2.z, y2.w},
+                            Y3[4] = {y3.x, y3.y, y3.z, y3.w}, Gv[4] = {G4.x, G4.y, G4.z, G4.w},
+                            bf[4] = {b4.x, b4.y, b4.z, b4.w};
+                const float qf[4] = {__low2float(q2[0]), __high2float(q2[0]), __low2float(q2[1]), __high2float(q2[1])};
+                const float kf[4] = {__low2float(k2[0]), __high2float(k2[0]), __low2float(k2[1]), __high2float(k2[1])};
+                float dq[4], dk[4], db[4], dG[4];
 #pragma unroll
-                    for (int e = 0; e < 16; e += 4)
-                        *reinterpret_cast<float4 *>(dbout + ok_ + e) = make_float4(db[e], db[e + 1], db[e + 2], db[e + 3]);
+                for (int e = 0; e < 4; ++e) {
+                    const float E = __expf(Gv[e]), Ei = __expf(-Gv[e]);
+                    const float dkc = Y2[e] * E, dkh = Y3[e] * Ei;
+                    dq[e] = Y1[e] * E;
+                    db[e] = dkc * kf[e];
+                    dk[e] = dkc * bf[e] + dkh;
+                    dG[e] = dq[e] * qf[e] + dkc * bf[e] * kf[e] - dkh * kf[e];
+                }
+                *reinterpret_cast<float4 *>(sdG + r * 128 + 4 * lane) = make_float4(dG[0], dG[1], dG[2], dG[3]);
+                if (r < L) {
+                    const size_t o4 = tok(d, bb, c0 + r, h, 128) + 4 * lane;
+                    *reinterpret_cast<uint2 *>(dqout + o4) = make_uint2(pack_bf16(dq[0], dq[1]), pack_bf16(dq[2], dq[3]));
+                    *reinterpret_cast<uint2 *>(dkout + o4) = make_uint2(pack_bf16(dk[0], dk[1]), pack_bf16(dk[2], dk[3]));
+                    *reinterpret_cast<float4 *>(dbout + o4) = make_float4(db[0], db[1], db[2], db[3]);
                 }
             }
         }
         abort = __syncthreads_or(!ok);
-        if (!abort && tid < 128) {
-            // dg = reverse in-chunk cumsum of dG, chunk-end term on the last row
-            float acc = sEnd[tid];
-            for (int rr = L - 1; rr >= 0; --rr) {
-                acc += sdG[rr * 128 + tid];
-                dgout[tok(d, bb, c0 + rr, h, 128) + tid] = acc;
+        if (!abort) {
+            // dg = reverse in-chunk cumsum of dG with the chunk-end term on the last row;
+            // thread (channel, part): part 1 scans rows 32..63, part 0 rows 0..31 after
+            // adding the sum of rows 32..63 itself
+            const float *sdG = YS;
+            const int ch = tid & 127, part = tid >> 7;
+            float acc = sEnd[ch];
+            if (part == 0)
+                for (int rr = 32; rr < 64; ++rr) acc += sdG[rr * 128 + ch];
+            const int hi = part ? 63 : 31, lo = part ? 32 : 0;
+            for (int rr = hi; rr >= lo; --rr) {
+                acc += sdG[rr * 128 + ch];
+                if (rr < L) dgout[tok(d, bb, c0 + rr, h, 128) + ch] = acc;
             }
         }
     }
