@@ -56,6 +56,7 @@ def parse():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-decode", action="store_true")
     p.add_argument("--batch", type=int, default=None,
                    help="override B (smaller cases for profiling captures only)")
     return p.parse_args()
@@ -153,16 +154,17 @@ def sources_hash() -> str:
 
 def run_ours(args, rank, world, local_rank):
     import torch
-    import torch.distributed as dist
 
     import gated_delta_rule_128_b200 as gdn
     from gated_delta_rule_128_b200 import workloads
+
+    from gated_delta_rule_128_b200 import dist as gd
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     wl = workloads.WORKLOADS[WORKLOAD_INDEX]
     B, T, H, dk, dv, C = args.batch or wl.B, wl.T, wl.H, wl.dk, wl.dv, wl.chunk
-    x = workloads.draw(B, T, H, dk, dv, wl.seed + 7919 * rank, s0_std=wl.s0_std,
+    x = workloads.draw(B, T, H, dk, dv, gd.rank_seed(wl.seed, rank), s0_std=wl.s0_std,
                        erase_scale=wl.erase_scale)
     io_names = ("q", "k", "v", "dO")
     bf = torch.bfloat16
@@ -183,9 +185,7 @@ def run_ours(args, rank, world, local_rank):
                      grads["dv"], grads["dg"], grads["db"], grads["dw"], None, ws, ws.numel(), 1,
                      B, T, H, dk, dv, C, io, stream)
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
+    barrier = gd.barrier
 
     sampler = ClockSampler(local_rank)
     sampler.start()
@@ -255,10 +255,10 @@ def run_ours(args, rank, world, local_rank):
     clocks = sampler.stop()
 
     ms_step = ms_total / args.steps
-    if world > 1:
-        t = torch.tensor([ms_step, e2e_ms, fwd_ms, bwd_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step, e2e_ms, fwd_ms, bwd_ms = (float(v) for v in t.tolist())
+    decode = run_decode(args, rank, dev) if not args.no_decode else None
+    ms_step, e2e_ms, fwd_ms, bwd_ms = gd.max_over_ranks([ms_step, e2e_ms, fwd_ms, bwd_ms], dev)
+    if decode is not None:
+        decode["us_per_step"] = gd.max_over_ranks([decode["us_per_step"]], dev)[0]
     tokens = B * T * world
     value = tokens / (ms_step * 1e-3)
     token_heads = B * T * H
@@ -306,7 +306,63 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": launches,
         "clocks": clocks,
     }
+    if decode is not None:
+        us = decode["us_per_step"]
+        dec_bytes = decode["bytes_per_step"]
+        gbs = dec_bytes / (us * 1e-6) / 1e9
+        decode.update(tokens_per_s=decode["N"] * world / (us * 1e-6),
+                      roofline={"bound": "hbm", "kernel": "decode_step", "achieved": gbs,
+                                "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                                "alg_bytes_per_launch": dec_bytes, "peak_source": peak_src})
+        line["decode"] = decode
     return line
+
+
+def run_decode(args, rank, dev):
+    """Recurrent decode, workload 4 (256 sequences x 16 heads, d = 128, bf16
+    q/k/v/o, f32 gates and state): 1024 consecutive steps timed with CUDA
+    events on the launch stream, inputs of 8 seeded steps cycled, state
+    resident in HBM."""
+    import torch
+
+    import gated_delta_rule_128_b200 as gdn
+    from gated_delta_rule_128_b200 import dist as gd
+    from gated_delta_rule_128_b200 import workloads
+
+    wl = workloads.WORKLOADS[4]
+    N, H, dk, dv = wl.B, wl.H, wl.dk, wl.dv
+    seed = gd.rank_seed(wl.seed, rank)
+    S = workloads.decode_state(N, H, dk, dv, seed, wl.s0_std).to(dev)
+    steps = []
+    for st in range(8):
+        x = workloads.decode_step_inputs(N, H, dk, dv, seed, st)
+        steps.append({n: (t.to(torch.bfloat16) if n in ("q", "k", "v") else t).to(dev)
+                      for n, t in x.items()})
+    o = torch.empty(N, H, dv, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.Stream(dev)
+    io = gdn.GDN2_IO_BF16
+
+    def run(n):
+        for i in range(n):
+            d = steps[i % 8]
+            gdn.gdn2_decode_step(d["q"], d["k"], d["v"], d["g"], d["b"], d["w"], S, o, N, H, dk,
+                                 dv, io, stream)
+
+    nsteps = wl.decode_steps
+    run(16)  # warm-up
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    run(nsteps)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    us = e0.elapsed_time(e1) * 1e3 / nsteps
+    if gdn.gdn2_get_device_status() != 0:
+        raise RuntimeError("device status reports an error after decode")
+    per_head = 2 * dk * dv * 4 + (2 * dk + dv) * 2 + (2 * dk + dv) * 4 + dv * 2
+    return {"workload": wl.name, "N": N, "H": H, "steps": nsteps,
+            "us_per_step": us, "bytes_per_step": per_head * N * H,
+            "inputs": "8 seeded steps cycled; 1024 consecutive launches on one stream"}
 
 
 # -------------------------------------------------------------- oracle arm
@@ -397,13 +453,8 @@ def main():
         if line is not None:
             print(json.dumps(line), flush=True)
         return
-    import torch
-    import torch.distributed as dist
-    if world > 1:
-        import datetime
-        torch.cuda.set_device(local_rank)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local_rank))
+    from gated_delta_rule_128_b200 import dist as gd
+    gd.init("nccl", gd.rank_info(), timeout_s=120)
     try:
         line = run_ours(args, rank, world, local_rank)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -413,8 +464,7 @@ def main():
         if rank == 0:
             print(json.dumps(line), flush=True)
     finally:
-        if world > 1:
-            dist.destroy_process_group()
+        gd.shutdown()
 
 
 if __name__ == "__main__":

@@ -396,7 +396,6 @@ constexpr uint32_t BL_D = 180224;     // Delta [64 pos][128 v]              (lat
 constexpr uint32_t BL_NDU = 196608;   // -dU [64 pos][128 v]
 constexpr uint32_t OP_QB = BL_S, OP_KC = BL_S + 16384, OP_KH = BL_S + 32768;
 constexpr uint32_t OP_DP = BL_D, OP_DA = BL_D + 8192;
-constexpr uint32_t SCR_DG = BL_S;     // dG [64][128] f32, after the last products
 constexpr uint32_t MISC = 212992;     // sGam, sRef [128]; sEnd [128]; scan [8][128]; mbarriers; slot
 constexpr uint32_t SMEM_BYTES = MISC + 1536 + 4096 + 128 + 1024;
 constexpr uint32_t TM_DP = 0, TM_DA = 64, TM_Y1 = 128, TM_Y2 = 256, TM_Y3 = 384;
