@@ -39,12 +39,16 @@ FWD_BYTES = 3 * 128 * 2 + 3 * 128 * 4 + 128 * 2           # 2560
 BWD_BYTES = 3 * 128 * 2 + 3 * 128 * 4 + 128 * 2 + 3 * 128 * 2 + 3 * 128 * 4   # 4864
 # ... attributed to the kernel that first reads (or writes) each tensor
 KERNEL_BYTES = {
-    "tc_fwd": FWD_BYTES,
+    # q, k, g, b read
+    "tc_prep": 2 * 128 * 2 + 2 * 128 * 4,
+    # v, w read; o written
+    "tc_fwd": 128 * 2 + 128 * 4 + 128 * 2,
     # q, k, g, b, dO, v, w read; dv, dw written
     "tc_bwd_state": 2 * 128 * 2 + 2 * 128 * 4 + 128 * 2 + 128 * 2 + 128 * 4 + 128 * 2 + 128 * 4,
     # dq, dk, db, dg written
     "tc_bwd_grad": 2 * 128 * 2 + 2 * 128 * 4,
 }
+assert KERNEL_BYTES["tc_prep"] + KERNEL_BYTES["tc_fwd"] == FWD_BYTES
 assert KERNEL_BYTES["tc_bwd_state"] + KERNEL_BYTES["tc_bwd_grad"] == BWD_BYTES
 
 
@@ -291,7 +295,7 @@ def run_ours(args, rank, world, local_rank):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f16", "data": "synthetic (seeded; BASELINE workload generators)",
+        "dtype": "f16", "data": "synthetic (seeded workload generators)",
         "config": {"workload": wl.name, "B": B, "T": T, "H": H, "d_k": dk, "d_v": dv,
                    "chunk": C, "io": "bf16 q/k/v/o/dO/dq/dk/dv, f32 g/b/w/state",
                    "global_batch": B * world, "seq_len": T, "parallelism": f"dp{world}",
@@ -431,7 +435,7 @@ def run_reference(args, rank, world):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": None,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic (seeded; BASELINE workload generators)",
+        "data": "synthetic (seeded workload generators)",
         "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "H": wl.H, "d_k": wl.dk,
                    "d_v": wl.dv, "chunk": wl.chunk, "global_batch": wl.B * world,
                    "seq_len": wl.T, "parallelism": f"dp{world}"},

@@ -28,8 +28,8 @@ cudaError_t decode_launch(const void *, const void *, const void *, const float 
                           const float *, float *, void *, int, int, int, int, gdn2_io,
                           cudaStream_t);
 cudaError_t tc_fwd_launch(const void *, const void *, const void *, const float *, const float *,
-                          const float *, const float *, void *, float *, void *, unsigned int *,
-                          const Dims &, cudaStream_t);
+                          const float *, const float *, void *, float *, void *, int,
+                          unsigned int *, const Dims &, cudaStream_t);
 cudaError_t tc_bwd_launch(const void *, const void *, const void *, const float *, const float *,
                           const float *, const void *, const float *, void *, void *, void *,
                           float *, float *, float *, float *, void *, unsigned int *, const Dims &,
@@ -72,7 +72,7 @@ static unsigned long long g_kind_count[K_KINDS];
 static double g_kind_ms[K_KINDS];
 static const char *const g_kind_names[K_KINDS] = {
     "simt_chunk_prep", "simt_state_fwd", "simt_out_fwd", "simt_state_bwd", "simt_chunk_bwd_a",
-    "simt_chunk_bwd_b", "decode_step", "tc_fwd", "tc_bwd_state", "tc_bwd_grad"};
+    "simt_chunk_bwd_b", "decode_step", "tc_prep", "tc_fwd", "tc_bwd_state", "tc_bwd_grad"};
 
 void launch_begin(int kind, cudaStream_t s) {
     g_launches.fetch_add(1, std::memory_order_relaxed);
@@ -153,8 +153,8 @@ extern "C" {
 static size_t ws_bytes_for(const Dims &d, gdn2_io io, int for_bwd) {
     SimtWs lay = simt_ws_layout(d);
     if (use_tc(d, io)) {
-        if (!for_bwd) return 256;  // the tensor-core forward keeps nothing between phases
-        return tc_ws_layout(d).bwd_end;
+        const TcWs t = tc_ws_layout(d);
+        return for_bwd ? t.bwd_end : t.rec_end;
     }
     return for_bwd ? lay.bwd_end : lay.fwd_end;
 }
@@ -178,8 +178,8 @@ gdn2_status gdn2_fwd(const void *q, const void *k, const void *v, const float *g
     if (use_tc(d, io)) {
         unsigned int *status = status_word();
         if (!status) return GDN2_ERR_CUDA;
-        void *keep = ws_bytes >= ws_bytes_for(d, io, 1) ? ws : nullptr;
-        return cuda_status(tc_fwd_launch(q, k, v, g, b, w, S0, o, ST, keep, status, d,
+        const int keep = ws_bytes >= ws_bytes_for(d, io, 1);
+        return cuda_status(tc_fwd_launch(q, k, v, g, b, w, S0, o, ST, ws, keep, status, d,
                                          (cudaStream_t)stream));
     }
     return cuda_status(run_forward(q, k, v, g, b, w, S0, o, ST, ws, d, io, (cudaStream_t)stream));
@@ -202,7 +202,7 @@ gdn2_status gdn2_bwd(const void *q, const void *k, const void *v, const float *g
         unsigned int *status = status_word();
         if (!status) return GDN2_ERR_CUDA;
         if (!ws_has_fwd) {
-            e = tc_fwd_launch(q, k, v, g, b, w, S0, nullptr, nullptr, ws, status, d, s);
+            e = tc_fwd_launch(q, k, v, g, b, w, S0, nullptr, nullptr, ws, 1, status, d, s);
             if (e != cudaSuccess) return GDN2_ERR_CUDA;
         }
         return cuda_status(tc_bwd_launch(q, k, v, g, b, w, dO, dST, dq, dk, dv, dg, db, dw, dS0, ws,

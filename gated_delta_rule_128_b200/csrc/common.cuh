@@ -73,7 +73,7 @@ struct SimtWs {
 // with launch_begin / launch_end (kernel kind ids below)
 enum KernelKind {
     K_SIMT_PREP = 0, K_SIMT_STATE_FWD, K_SIMT_OUT, K_SIMT_STATE_BWD, K_SIMT_BWD_A, K_SIMT_BWD_B,
-    K_DECODE, K_TC_FWD, K_TC_BWD_STATE, K_TC_BWD_GRAD, K_KINDS
+    K_DECODE, K_TC_PREP, K_TC_FWD, K_TC_BWD_STATE, K_TC_BWD_GRAD, K_KINDS
 };
 void launch_begin(int kind, cudaStream_t s);
 void launch_end(int kind, cudaStream_t s);
@@ -108,22 +108,36 @@ inline SimtWs simt_ws_layout(const Dims &d) {
 // ---- workspace of the tensor-core path (d_k = d_v = 128, chunk 64): fp16
 // tiles in their 128-byte swizzled shared-memory layout, so that they move
 // with plain bulk copies.  Offsets in bytes; bh = b * H + h.
+//   rec   [bh][NC]        66560 B  the chunk's record, written by the chunk-
+//                                  parallel prep kernel (layout REC_* below)
 //   ckS   [bh][NC + 1][2 halves] 16 KB  chunk-entry states S_c (and S_T), true scale
-//   ckTP  [bh][NC]               16 KB  T (8 KB) then P (8 KB)
 //   ckD   [bh][NC][2]             8 KB  Delta (columns of one d_v half)
 //   ckdS  [bh][NC][2]            16 KB  e^(G_L - G_m) dS_next
 //   ckndU [bh][NC][2]             8 KB  -dU
 //   ckEnd [bh][NC][2]           512 B  half-sums of rowsum(dS_next . S_next)
+// A forward that is not followed by a backward needs `rec` only.
+//
+// Chunk record: decay-scaled operands relative to the chunk's middle row
+// (fp16, 128-byte swizzled, [64 pos][128 key] K-major unless noted)
+//   REC_QB   Qb = q.e^(G-G_m)
+//   REC_KH   Kh = k.e^-(G-G_m)
+//   REC_WN   -W = -T Kc
+//   REC_T    T = (I + A)^-1            [64][64]
+//   REC_P    P = lower-incl(Qb Kh^T)   [64][64]
+//   REC_FAC  e^(G_L - G_m) [128] f32, then e^G_m [128] f32
+constexpr uint32_t REC_QB = 0, REC_KH = 16384, REC_WN = 32768, REC_T = 49152, REC_P = 57344,
+                   REC_FAC = 65536, REC_BYTES = 66560;
 struct TcWs {
-    size_t ckS, ckTP, ckD, ckdS, ckndU, ckEnd, fwd_end, bwd_end;
+    size_t rec, rec_end, ckS, ckD, fwd_end, ckdS, ckndU, ckEnd, bwd_end;
 };
 inline TcWs tc_ws_layout(const Dims &d) {
     const size_t bh = (size_t)d.B * d.H, nc = (size_t)d.NC;
     TcWs w;
     size_t o = 0;
     auto take = [&](size_t bytes) { size_t at = o; o = align256(o + bytes); return at; };
+    w.rec = take(bh * nc * REC_BYTES);
+    w.rec_end = o;
     w.ckS = take(bh * (nc + 1) * 2 * 16384);
-    w.ckTP = take(bh * nc * 16384);
     w.ckD = take(bh * nc * 2 * 8192);
     w.fwd_end = o;
     w.ckdS = take(bh * nc * 2 * 16384);

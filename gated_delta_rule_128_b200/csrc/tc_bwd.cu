@@ -1,6 +1,6 @@
 // Gate-aware chunkwise backward of Gated Delta Rule-2 on the sm_100a tensor
-// cores (bf16 I/O, d_k = d_v = 128, chunk 64), after tc_fwd_kernel has left
-// its chunk states, T, P and Delta in the workspace.
+// cores (bf16 I/O, d_k = d_v = 128, chunk 64), after the forward has left
+// its chunk records (T, P among them), chunk states and Delta in the workspace.
 //
 // "Gated DeltaNet-2" (LIT-802 review, Key takeaways 2; paper Secs. 3.3-3.4,
 // Apps. A-B, D.6; digg thread 11/): the per-channel gates cannot be pulled
@@ -12,7 +12,8 @@
 // tc_common.cuh; dS = dL/dS_next entering the chunk from the right):
 //   dS_m  = diag(e^(G_L-G_m)) dS
 //   dDelta = P^T dO + Kh dS_m,         dU = T^T dDelta,   dw = dU.v, dv = dU.w
-//   dS_c  = diag(e^G_m) (dS_m + Qb^T dO - Kc^T dU)                (carried left)
+//   dS_c  = diag(e^G_m) (dS_m + Qb^T dO - W^T dDelta)             (carried left)
+//   (W^T dDelta = Kc^T dU, since W = T Kc)
 //   S_m   = diag(e^G_m) S_c
 //   dP = lower-incl(dO Delta^T),       dA = -strictly-lower(dU Delta^T)
 //   Y1 = dO S_m^T + dP Kh              dq  = Y1.E
@@ -25,9 +26,10 @@
 //
 // Two kernels:
 //  * tc_bwd_state_kernel: one CTA per (b, h, half of d_v), walking the chunks
-//    in reverse with dS in tensor memory; three tcgen05.mma round trips per
-//    chunk (dDelta, dU, dS).  Writes dw, dv, dS0, and per chunk dS_m, -dU and
-//    the half-sums of the chunk-end term to the workspace.
+//    in reverse with dS in tensor memory and the chunk records double-
+//    buffered; two tcgen05.mma round trips per chunk (dDelta; then dS and
+//    dU together).  Writes dw, dv, dS0, and per chunk dS_m, -dU and the
+//    half-sums of the chunk-end term to the workspace.
 //  * tc_bwd_grad_kernel: one CTA per (b, h, chunk), all chunks in parallel,
 //    full d_v; five products, then three accumulations, then dq, dk, db, dg.
 
@@ -43,16 +45,14 @@ using namespace tcc;
 // ============================================================ state kernel
 namespace tbs {
 constexpr int kThreads = 256;
-constexpr uint32_t RAW_Q = 0, RAW_K = 16384, RAW_DO = 32768, RAW_G = 40960, RAW_B = 73728;
-constexpr uint32_t OP_QB = 106496, OP_KC = 122880, OP_KH = 139264;  // [64 pos][128 key]
-constexpr uint32_t OP_T = 155648, OP_P = 163840;                      // [64][64], adjacent
-constexpr uint32_t OP_DS = 172032;   // dS_m fp16 [128 key][64 v]  MN-major B
-constexpr uint32_t OP_DO = 188416;   // dO fp16   [64 pos][64 v]   MN-major B
-constexpr uint32_t OP_DD = 196608;   // dDelta, later -dU [64 pos][64 v]
-constexpr uint32_t STG_S = 204800;   // S_c (true scale) fp16 [128 key][64 v]
-constexpr uint32_t MISC = 221184;    // sGam, sRef [128] f32; sEnd [2][128] f32; mbarriers; slot
-constexpr uint32_t SMEM_BYTES = MISC + 2176 + 1024;
-constexpr uint32_t SCR_SCAN = OP_DD;  // cumsum totals during phase 1
+constexpr uint32_t STG = 0;                   // two chunk records, REC_BYTES each
+constexpr uint32_t RAW_DO = 2 * REC_BYTES;    // dO half, bf16 [64 pos][64]
+constexpr uint32_t OP_DO = RAW_DO + 8192;     // dO fp16      [64 pos][64 v]  MN-major B
+constexpr uint32_t OP_DS = OP_DO + 8192;      // dX fp16      [128 key][64 v] MN-major B
+constexpr uint32_t OP_DD = OP_DS + 16384;     // dDelta fp16  [64 pos][64 v]  MN-major B
+constexpr uint32_t STG_S = OP_DD + 8192;      // S_c (true scale) fp16 [128 key][64 v]
+constexpr uint32_t MISC = STG_S + 16384;      // sEnd [2][128] f32; mbarriers; TMEM slot
+constexpr uint32_t SMEM_BYTES = MISC + 1024 + 128 + 1024;
 constexpr uint32_t TM_DS = 0, TM_DD = 64, TM_DU = 128;  // 256 columns allocated
 constexpr uint32_t ID_MM64 = idesc_f16(64, 64, true, true);
 constexpr uint32_t ID_KM64 = idesc_f16(64, 64, false, true);
@@ -61,10 +61,16 @@ constexpr long long kWait = 2000000000LL;
 constexpr float kRange = 6.0e4f;
 }  // namespace tbs
 
+// One CTA per (b, h, half of d_v), walking the chunks in reverse with
+// dX = diag(e^(G_L - G_m)) dS_next in tensor memory.  Per chunk, from the
+// chunk's record (Qb, Kh, -W, T, P, factors):
+//   (1) dDelta = P^T dO + Kh dX,        dS_m = dX + Qb^T dO
+//   (2) dS_m += (-W)^T dDelta,          dU = T^T dDelta
+// then dS_c = diag(e^G_m) dS_m, the previous chunk's dX = diag(e^(G_L - G_m))
+// dS_c, dv = dU.w, dw = dU.v, and the workspace copies of dX, -dU and the
+// chunk-end half-sums for the gradient kernel.
 __global__ void __launch_bounds__(tbs::kThreads, 1)
-tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
-                    const __grid_constant__ CUtensorMap mdo, const __grid_constant__ CUtensorMap mg,
-                    const __grid_constant__ CUtensorMap mb, const __nv_bfloat16 *__restrict__ v,
+tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __nv_bfloat16 *__restrict__ v,
                     const float *__restrict__ w, const float *__restrict__ dST,
                     __nv_bfloat16 *__restrict__ dvout, float *__restrict__ dwout,
                     float *__restrict__ dS0, unsigned char *__restrict__ ws, TcWs lay,
@@ -73,12 +79,11 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
     extern __shared__ unsigned char smraw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smraw) + 1023) & ~static_cast<uintptr_t>(1023));
-    float *sGam = reinterpret_cast<float *>(sm + MISC);
-    float *sRef = reinterpret_cast<float *>(sm + MISC + 512);
-    float *sEnd = reinterpret_cast<float *>(sm + MISC + 1024);  // [2][128]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + MISC + 2048);  // 0..7
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + MISC + 2048 + 64);
-    float big = 0.f, gbig = 0.f;  // range checks: operand magnitude, |G - G_m|
+    float *sEnd = reinterpret_cast<float *>(sm + MISC);  // [2][128]
+    // 0, 1 records of stages 0, 1; 2 dO; 3 state checkpoint; 4, 5 product groups
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + MISC + 1024);
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + MISC + 1024 + 64);
+    float big = 0.f;  // range check: operand magnitude
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int vh = blockIdx.x, h = blockIdx.y, bb = blockIdx.z, v0 = vh * 64;
@@ -86,13 +91,14 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
     const int quarter = warp & 3, half = warp >> 2;
     const int key = quarter * 32 + lane;
     const size_t bh = (size_t)bb * H + h;
+    const unsigned char *recs = ws + lay.rec + bh * NC * (size_t)REC_BYTES;
 
     if (warp == 0) {
         tmem_alloc(tslot, 256);
         tmem_relinquish();
     }
     if (tid == 0) {
-        for (int i = 0; i < 8; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < 6; ++i) mbar_init(&bars[i], 1);
         mbar_fence_init();
     }
     fence_before_sync();
@@ -101,30 +107,61 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
     const uint32_t tm = *tslot;
 
     int issued[4] = {0, 0, 0, 0};
-    auto load_inputs = [&](int cc) {  // bar0: q, k, dO half; bar1: g, b
-        mbar_expect_tx(&bars[0], 16384 * 2 + 8192);
-        tma_load_4d(sm + RAW_Q, &mq, 0, h, cc * 64, bb, &bars[0]);
-        tma_load_4d(sm + RAW_K, &mk, 0, h, cc * 64, bb, &bars[0]);
-        tma_load_4d(sm + RAW_DO, &mdo, v0, h, cc * 64, bb, &bars[0]);
-        mbar_expect_tx(&bars[1], 32768 * 2);
-        tma_load_4d(sm + RAW_G, &mg, 0, h, cc * 64, bb, &bars[1]);
-        tma_load_4d(sm + RAW_B, &mb, 0, h, cc * 64, bb, &bars[1]);
-        ++issued[0];
-        ++issued[1];
+    auto load_rec = [&](int cc) {
+        const int s = cc & 1;
+        mbar_expect_tx(&bars[s], REC_BYTES);
+        bulk_load(sm + STG + s * REC_BYTES, recs + (size_t)cc * REC_BYTES, REC_BYTES, &bars[s]);
+        ++issued[s];
     };
-    auto load_tp = [&](int cc) {  // bar2: T and P of chunk cc
-        mbar_expect_tx(&bars[2], 16384);
-        bulk_load(sm + OP_T, ws + lay.ckTP + (bh * NC + cc) * 16384, 16384, &bars[2]);
+    auto load_do = [&](int cc) {
+        mbar_expect_tx(&bars[2], 8192);
+        tma_load_4d(sm + RAW_DO, &mdo, v0, h, cc * 64, bb, &bars[2]);
         ++issued[2];
     };
-    auto load_s = [&](int slot, uint64_t *bar) {  // state checkpoint `slot` of this half
-        mbar_expect_tx(bar, 16384);
-        bulk_load(sm + STG_S, ws + lay.ckS + ((bh * (NC + 1) + slot) * 2 + vh) * 16384, 16384, bar);
+    auto load_s = [&](int slot) {  // state checkpoint `slot` of this half
+        mbar_expect_tx(&bars[3], 16384);
+        bulk_load(sm + STG_S, ws + lay.ckS + ((bh * (NC + 1) + slot) * 2 + vh) * 16384, 16384, &bars[3]);
+        ++issued[3];
+    };
+    auto rec_fac = [&](int cc) {  // e^(G_L - G_m) of chunk cc (then e^G_m at +128)
+        return reinterpret_cast<const float *>(sm + STG + (cc & 1) * REC_BYTES + REC_FAC);
+    };
+    // dX of chunk c, this thread's row and 32 columns: TMEM, fp16 operand, workspace copy
+    auto put_dx = [&](int c, float *x) {
+        tmem_st16(taddr(tm + TM_DS, quarter * 32, 32 * half), x);
+        tmem_st16(taddr(tm + TM_DS, quarter * 32, 32 * half + 16), x + 16);
+        unsigned char *dst = ws + lay.ckdS + ((bh * NC + c) * 2 + vh) * 16384;
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+            const uint32_t off = sw128_chunk(key, 4 * half + jj, 128);
+            st_h8(sm + OP_DS + off, x + 8 * jj);
+            st_h8(dst + off, x + 8 * jj);
+            big = absmax8(x + 8 * jj, big);
+        }
+    };
+    // rowsum over this thread's 32 columns of x . S (S from STG_S)
+    auto end_term = [&](const float *x) {
+        float acc = 0.f;
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+            float s8[8];
+            ld_h8(sm + STG_S + sw128_chunk(key, 4 * half + jj, 128), s8);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc += x[8 * jj + e] * s8[e];
+        }
+        return acc;
     };
 
-    // dS entering the last chunk: dS_T (or zero)
-    float x[32];
+    if (tid == 0) {
+        load_rec(NC - 1);
+        if (NC > 1) load_rec(NC - 2);
+        load_do(NC - 1);
+        load_s(NC);
+    }
+    // dS_T (or zero); the last chunk's end term rowsum(dS_T . S_T); its dX
+    bool ok;
     {
+        float x[32];
         const size_t so = st_off(d, bb, h);
 #pragma unroll
         for (int j = 0; j < 32; j += 4) {
@@ -132,102 +169,69 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
                            : make_float4(0.f, 0.f, 0.f, 0.f);
             x[j] = t.x; x[j + 1] = t.y; x[j + 2] = t.z; x[j + 3] = t.w;
         }
-        tmem_st16(taddr(tm + TM_DS, quarter * 32, 32 * half), x);
-        tmem_st16(taddr(tm + TM_DS, quarter * 32, 32 * half + 16), x + 16);
+        ok = mbar_wait(&bars[3], 0, kWait);
+        ok = ok && mbar_wait(&bars[(NC - 1) & 1], 0, kWait);
+        sEnd[half * 128 + key] = end_term(x);
+        const float gam = rec_fac(NC - 1)[key];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) x[j] *= gam;
+        put_dx(NC - 1, x);
         tmem_wait_st();
     }
-    // chunk-end term of the last chunk: rowsum(dS_T . S_T), this half's columns
-    bool ok = true;
-    if (tid == 0) load_s(NC, &bars[7]);
-    ok = mbar_wait(&bars[7], 0, kWait);
-    {
-        float acc = 0.f;
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-            float s8[8];
-            ld_h8(sm + STG_S + sw128_chunk(key, 4 * half + jj, 128), s8);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) acc += x[8 * jj + i] * s8[i];
-        }
-        sEnd[half * 128 + key] = acc;
-    }
+    fence_proxy_async();
     fence_before_sync();
     bool abort = __syncthreads_or(!ok);
     if (!abort) {
         if (half == 0)
             reinterpret_cast<float *>(ws + lay.ckEnd + ((bh * NC + NC - 1) * 2 + vh) * 512)[key] =
                 sEnd[key] + sEnd[128 + key];
-        if (tid == 0) {
-            load_inputs(NC - 1);
-            load_tp(NC - 1);
-            load_s(NC - 1, &bars[3]);
-            ++issued[3];
-        }
+        if (tid == 0 && NC > 1) load_s(NC - 1);
     }
 
     for (int i = 0; i < NC && !abort; ++i) {
         const int c = NC - 1 - i, c0 = c * 64;
         const uint32_t par = i & 1;
-        // ---------------- phase 1: decay, operands, dS_m
-        ok = mbar_wait(&bars[0], par, kWait);
-        ok = ok && mbar_wait(&bars[1], par, kWait);
+        unsigned char *stg = sm + STG + (c & 1) * REC_BYTES;
+        // ---------------- dO to fp16, product group 1
+        ok = mbar_wait(&bars[c & 1], (i >> 1) & 1, kWait);
         ok = ok && mbar_wait(&bars[2], par, kWait);
-        float G[8][4];
-        cumsum_local(reinterpret_cast<const float *>(sm + RAW_G), reinterpret_cast<float *>(sm + SCR_SCAN),
-                     warp, lane, G);
-        if (__syncthreads_or(!ok)) { abort = true; break; }
-        cumsum_finish(reinterpret_cast<const float *>(sm + SCR_SCAN), warp, lane, G, sGam, sRef);
-        gbig = fmaxf(gbig, write_factors(sm + RAW_Q, sm + RAW_K, reinterpret_cast<const float *>(sm + RAW_B),
-                                       G, sm + OP_QB, sm + OP_KC, sm + OP_KH, warp, lane));
-        if (lane < 16) {  // dO half -> fp16 operand [pos][v]
-#pragma unroll
-            for (int m = 0; m < 8; ++m) {
-                const int r = 8 * warp + m;
-                uint2 dr = *reinterpret_cast<const uint2 *>(sm + RAW_DO + r * 128 + lane * 8);
-                const __nv_bfloat162 *d2 = reinterpret_cast<const __nv_bfloat162 *>(&dr);
-                st_h4(sm + OP_DO + sw128_off(r, 4 * lane, 64), __low2float(d2[0]), __high2float(d2[0]),
-                      __low2float(d2[1]), __high2float(d2[1]));
-            }
-        }
-        __syncthreads();
-        if (tid == 0 && c > 0) load_inputs(c - 1);  // raw tiles consumed
         {
-            float sv[32];
-            tmem_ld16(taddr(tm + TM_DS, quarter * 32, 32 * half), sv);
-            tmem_ld16(taddr(tm + TM_DS, quarter * 32, 32 * half + 16), sv + 16);
-            tmem_wait_ld();
-            const float gm = sGam[key];
+            const int r = tid >> 2, cg = tid & 3;  // row, 16-column group
+            const uint4 d0 = *reinterpret_cast<const uint4 *>(sm + RAW_DO + r * 128 + cg * 32);
+            const uint4 d1 = *reinterpret_cast<const uint4 *>(sm + RAW_DO + r * 128 + cg * 32 + 16);
+            const __nv_bfloat162 *a = reinterpret_cast<const __nv_bfloat162 *>(&d0);
+            const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&d1);
+            float x[16];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) sv[j] *= gm;
-            tmem_st16(taddr(tm + TM_DS, quarter * 32, 32 * half), sv);
-            tmem_st16(taddr(tm + TM_DS, quarter * 32, 32 * half + 16), sv + 16);
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                st_h8(sm + OP_DS + sw128_chunk(key, 4 * half + jj, 128), sv + 8 * jj);
-                big = absmax8(sv + 8 * jj, big);
+            for (int e = 0; e < 4; ++e) {
+                x[2 * e] = __low2float(a[e]);
+                x[2 * e + 1] = __high2float(a[e]);
+                x[8 + 2 * e] = __low2float(b2[e]);
+                x[8 + 2 * e + 1] = __high2float(b2[e]);
             }
-            tmem_wait_st();
+            st_h8(sm + OP_DO + sw128_chunk(r, 2 * cg, 64), x);
+            st_h8(sm + OP_DO + sw128_chunk(r, 2 * cg + 1, 64), x + 8);
         }
         fence_proxy_async();
         fence_before_sync();
-        __syncthreads();
+        if (__syncthreads_or(!ok)) { abort = true; break; }
         if (tid == 0) {
             fence_after_sync();
-            bulk_store(ws + lay.ckdS + ((bh * NC + c) * 2 + vh) * 16384, sm + OP_DS, 16384);
-            bulk_commit();
-            const uint32_t p = smem_addr(sm + OP_P), dO = smem_addr(sm + OP_DO),
-                           kh = smem_addr(sm + OP_KH), ds = smem_addr(sm + OP_DS);
-            // dDelta = P^T dO + Kh dS_m
+            if (c > 0) load_do(c - 1);  // raw dO consumed
+            const uint32_t st = smem_addr(stg), dO = smem_addr(sm + OP_DO), dx = smem_addr(sm + OP_DS);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tm + TM_DD, desc_mnmajor(p, 64, ks), desc_mnmajor(dO, 64, ks), ID_MM64, ks > 0);
+                mma_bf16(tm + TM_DD, desc_mnmajor(st + REC_P, 64, ks), desc_mnmajor(dO, 64, ks), ID_MM64, ks > 0);
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks)
-                mma_bf16(tm + TM_DD, desc_kmajor(kh, 64, ks), desc_mnmajor(ds, 128, ks), ID_KM64, 1);
+                mma_bf16(tm + TM_DD, desc_kmajor(st + REC_KH, 64, ks), desc_mnmajor(dx, 128, ks), ID_KM64, 1);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(tm + TM_DS, desc_mnmajor(st + REC_QB, 64, ks), desc_mnmajor(dO, 64, ks), ID_MM128x64, 1);
             mma_commit(&bars[4]);
         }
-        // v and w of this thread's row and columns, for dw and dv in phase 3:
-        // requested now so that the loads overlap phase 2
+        // v and w of this thread's row and columns, for dw and dv below:
+        // requested now so that the loads overlap the products
         uint4 vreg[4];
         float4 wreg[8];
         const int r_own = quarter * 16 + lane;
@@ -239,7 +243,7 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
 #pragma unroll
             for (int j = 0; j < 8; ++j) wreg[j] = row_ok ? *reinterpret_cast<const float4 *>(w + ov + 4 * j) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        // ---------------- phase 2: dDelta to shared memory, dU = T^T dDelta
+        // ---------------- dDelta to fp16, product group 2
         ok = mbar_wait(&bars[4], par, kWait);
         fence_after_sync();
         {
@@ -261,20 +265,46 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
         if (__syncthreads_or(!ok)) { abort = true; break; }
         if (tid == 0) {
             fence_after_sync();
-            const uint32_t t = smem_addr(sm + OP_T), dd = smem_addr(sm + OP_DD);
+            const uint32_t st = smem_addr(stg), dd = smem_addr(sm + OP_DD);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tm + TM_DU, desc_mnmajor(t, 64, ks), desc_mnmajor(dd, 64, ks), ID_MM64, ks > 0);
+                mma_bf16(tm + TM_DS, desc_mnmajor(st + REC_WN, 64, ks), desc_mnmajor(dd, 64, ks), ID_MM128x64, 1);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(tm + TM_DU, desc_mnmajor(st + REC_T, 64, ks), desc_mnmajor(dd, 64, ks), ID_MM64, ks > 0);
             mma_commit(&bars[5]);
         }
-        // ---------------- phase 3: dw, dv; -dU to shared memory; dS update
+        // ---------------- dS_c, the previous chunk's dX and end term; dv, dw, -dU
         ok = mbar_wait(&bars[5], par, kWait);
+        if (c > 0) {
+            ok = ok && mbar_wait(&bars[3], (i + 1) & 1, kWait);                 // S_c
+            ok = ok && mbar_wait(&bars[(c - 1) & 1], ((i + 1) >> 1) & 1, kWait);  // record c-1
+        }
         fence_after_sync();
         {
-            float du[32];
+            float sv[32], du[32];
+            tmem_ld16(taddr(tm + TM_DS, quarter * 32, 32 * half), sv);
+            tmem_ld16(taddr(tm + TM_DS, quarter * 32, 32 * half + 16), sv + 16);
             tmem_ld16(taddr(tm + TM_DU, quarter * 32, 32 * half), du);
             tmem_ld16(taddr(tm + TM_DU, quarter * 32, 32 * half + 16), du + 16);
             tmem_wait_ld();
+            const float e = reinterpret_cast<const float *>(stg + REC_FAC)[128 + key];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) sv[j] *= e;  // dS_c
+            if (c == 0) {
+                if (dS0) {
+                    float *dst = dS0 + st_off(d, bb, h) + (size_t)key * 128 + v0 + 32 * half;
+#pragma unroll
+                    for (int j = 0; j < 32; j += 4)
+                        *reinterpret_cast<float4 *>(dst + j) = make_float4(sv[j], sv[j + 1], sv[j + 2], sv[j + 3]);
+                }
+            } else {
+                sEnd[half * 128 + key] = end_term(sv);
+                const float gam = rec_fac(c - 1)[key];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) sv[j] *= gam;
+                put_dx(c - 1, sv);
+            }
             if (lane < 16) {
                 const int r = quarter * 16 + lane;
                 if (row_ok) {
@@ -286,12 +316,12 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
                         const float4 w0 = wreg[j / 4], w1 = wreg[j / 4 + 1];
                         float wf[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            dwv[j + 2 * e] = du[j + 2 * e] * __low2float(v2[e]);
-                            dwv[j + 2 * e + 1] = du[j + 2 * e + 1] * __high2float(v2[e]);
+                        for (int e2 = 0; e2 < 4; ++e2) {
+                            dwv[j + 2 * e2] = du[j + 2 * e2] * __low2float(v2[e2]);
+                            dwv[j + 2 * e2 + 1] = du[j + 2 * e2 + 1] * __high2float(v2[e2]);
                         }
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) dvv[j + e] = du[j + e] * wf[e];
+                        for (int e2 = 0; e2 < 8; ++e2) dvv[j + e2] = du[j + e2] * wf[e2];
                     }
 #pragma unroll
                     for (int j = 0; j < 32; j += 4)
@@ -303,82 +333,31 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
                 }
 #pragma unroll
                 for (int j = 0; j < 32; ++j) du[j] = -du[j];
+                unsigned char *dst = ws + lay.ckndU + ((bh * NC + c) * 2 + vh) * 8192;
 #pragma unroll
                 for (int jj = 0; jj < 4; ++jj) {
-                    st_h8(sm + OP_DD + sw128_chunk(r, 4 * half + jj, 64), du + 8 * jj);
+                    st_h8(dst + sw128_chunk(r, 4 * half + jj, 64), du + 8 * jj);
                     big = absmax8(du + 8 * jj, big);
                 }
             }
-        }
-        fence_proxy_async();
-        fence_before_sync();
-        if (__syncthreads_or(!ok)) { abort = true; break; }
-        if (tid == 0) {
-            fence_after_sync();
-            bulk_store(ws + lay.ckndU + ((bh * NC + c) * 2 + vh) * 8192, sm + OP_DD, 8192);
-            bulk_commit();
-            if (c > 0) load_tp(c - 1);  // T and P consumed
-            const uint32_t qb = smem_addr(sm + OP_QB), kc = smem_addr(sm + OP_KC),
-                           dO = smem_addr(sm + OP_DO), ndu = smem_addr(sm + OP_DD);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tm + TM_DS, desc_mnmajor(qb, 64, ks), desc_mnmajor(dO, 64, ks), ID_MM128x64, 1);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tm + TM_DS, desc_mnmajor(kc, 64, ks), desc_mnmajor(ndu, 64, ks), ID_MM128x64, 1);
-            mma_commit(&bars[6]);
-        }
-        // ---------------- phase 4: dS_c = e^G_m (...), chunk-end term of chunk c-1
-        ok = mbar_wait(&bars[6], par, kWait);
-        ok = ok && mbar_wait(&bars[3], par, kWait);
-        fence_after_sync();
-        {
-            float sv[32];
-            tmem_ld16(taddr(tm + TM_DS, quarter * 32, 32 * half), sv);
-            tmem_ld16(taddr(tm + TM_DS, quarter * 32, 32 * half + 16), sv + 16);
-            tmem_wait_ld();
-            const float e = sRef[key];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) sv[j] *= e;
-            tmem_st16(taddr(tm + TM_DS, quarter * 32, 32 * half), sv);
-            tmem_st16(taddr(tm + TM_DS, quarter * 32, 32 * half + 16), sv + 16);
-            float acc = 0.f;
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                float s8[8];
-                ld_h8(sm + STG_S + sw128_chunk(key, 4 * half + jj, 128), s8);
-#pragma unroll
-                for (int e2 = 0; e2 < 8; ++e2) acc += sv[8 * jj + e2] * s8[e2];
-            }
-            sEnd[half * 128 + key] = acc;
-            if (c == 0 && dS0) {
-                float *dst = dS0 + st_off(d, bb, h) + (size_t)key * 128 + v0 + 32 * half;
-#pragma unroll
-                for (int j = 0; j < 32; j += 4)
-                    *reinterpret_cast<float4 *>(dst + j) = make_float4(sv[j], sv[j + 1], sv[j + 2], sv[j + 3]);
-            }
             tmem_wait_st();
         }
-        if (tid == 0) bulk_wait_read();  // OP_DS, OP_DD copies done before they are rewritten
         fence_proxy_async();
         fence_before_sync();
         if (__syncthreads_or(!ok)) { abort = true; break; }
         if (c > 0 && half == 0)
             reinterpret_cast<float *>(ws + lay.ckEnd + ((bh * NC + c - 1) * 2 + vh) * 512)[key] =
                 sEnd[key] + sEnd[128 + key];
-        if (tid == 0 && c > 0) {
-            load_s(c - 1, &bars[3]);
-            ++issued[3];
+        if (tid == 0) {
+            if (c > 0) load_s(c - 1);     // S_c consumed
+            if (c >= 2) load_rec(c - 2);  // this chunk's record consumed
         }
     }
-    if (!(big <= kRange) || !(gbig <= 9.f)) record_status(status, GDN2_ERR_RANGE);
-    if (tid == 0) {
-        bulk_wait_all();
-        if (abort) {
-            record_status(status, GDN2_ERR_TIMEOUT);
-            for (int k2 = 0; k2 < 4; ++k2)
-                if (issued[k2] > 0) mbar_wait(&bars[k2], (issued[k2] - 1) & 1, kWait);
-        }
+    if (!(big <= kRange)) record_status(status, GDN2_ERR_RANGE);
+    if (tid == 0 && abort) {
+        record_status(status, GDN2_ERR_TIMEOUT);
+        for (int k2 = 0; k2 < 4; ++k2)
+            if (issued[k2] > 0) mbar_wait(&bars[k2], (issued[k2] - 1) & 1, kWait);
     }
     fence_before_sync();
     __syncthreads();
@@ -677,7 +656,7 @@ cudaError_t tc_bwd_launch(const void *q, const void *k, const void *v, const flo
     if (e != cudaSuccess) return e;
     launch_begin(K_TC_BWD_STATE, s);
     tc_bwd_state_kernel<<<dim3(2, d.H, d.B), tbs::kThreads, tbs::SMEM_BYTES, s>>>(
-        mq, mk, mdo_half, mg, mb, (const __nv_bfloat16 *)v, w, dST, (__nv_bfloat16 *)dv, dw, dS0,
+        mdo_half, (const __nv_bfloat16 *)v, w, dST, (__nv_bfloat16 *)dv, dw, dS0,
         (unsigned char *)ws, lay, status, d);
     launch_end(K_TC_BWD_STATE, s);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
