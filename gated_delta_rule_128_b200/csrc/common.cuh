@@ -118,15 +118,15 @@ inline SimtWs simt_ws_layout(const Dims &d) {
 // A forward that is not followed by a backward needs `rec` only.
 //
 // Chunk record: decay-scaled operands relative to the chunk's middle row
-// (fp16, 128-byte swizzled, [64 pos][128 key] K-major unless noted)
-//   REC_QB   Qb = q.e^(G-G_m)
-//   REC_KH   Kh = k.e^-(G-G_m)
-//   REC_WN   -W = -T Kc
-//   REC_T    T = (I + A)^-1            [64][64]
-//   REC_P    P = lower-incl(Qb Kh^T)   [64][64]
+// (fp16, 128-byte swizzled; see tc.cuh for the layouts)
+//   REC_WQ   [-W; Qb] as one [128 rows][128 key] K-major tile: rows 0..63
+//            -W = -T Kc, rows 64..127 Qb = q.e^(G-G_m) (32 KB)
+//   REC_KH   Kh = k.e^-(G-G_m)          [64 pos][128 key] K-major (16 KB)
+//   REC_T    T = (I + A)^-1             [64][64] K-major (8 KB)
+//   REC_P    P = lower-incl(Qb Kh^T)    [64][64] K-major (8 KB)
 //   REC_FAC  e^(G_L - G_m) [128] f32, then e^G_m [128] f32
-constexpr uint32_t REC_QB = 0, REC_KH = 16384, REC_WN = 32768, REC_T = 49152, REC_P = 57344,
-                   REC_FAC = 65536, REC_BYTES = 66560;
+constexpr uint32_t REC_WQ = 0, REC_KH = 32768, REC_T = 49152, REC_P = 57344, REC_FAC = 65536,
+                   REC_BYTES = 66560;
 struct TcWs {
     size_t rec, rec_end, ckS, ckD, fwd_end, ckdS, ckndU, ckEnd, bwd_end;
 };

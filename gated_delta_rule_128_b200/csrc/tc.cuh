@@ -74,6 +74,22 @@ __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool a_mn, bool b
     return idesc_f16kind(M, N, a_mn, b_mn, 0u);
 }
 
+// MN-major operand whose 64-wide MN blocks lie `lbo` bytes apart (for tiles
+// interleaved with another tile of the same shape), K step kstep
+__device__ __forceinline__ uint64_t desc_mnmajor_lbo(uint32_t base, uint32_t lbo, int kstep) {
+    return sdesc(base + (uint32_t)(kstep * 2048), lbo, 1024);
+}
+
+// The same descriptors from the descriptor of K step 0 (d0 = desc_kmajor(base,
+// R, 0) or desc_mnmajor(base, Krows, 0)): only the start-address field moves,
+// and for shared addresses below 256 KB it cannot carry out of its 14 bits.
+__device__ __forceinline__ uint64_t kstep_kmajor(uint64_t d0, int R, int kstep) {
+    return d0 + (uint64_t)((((kstep >> 2) * (R * 128)) + (kstep & 3) * 32) >> 4);
+}
+__device__ __forceinline__ uint64_t kstep_mnmajor(uint64_t d0, int kstep) {
+    return d0 + (uint64_t)(kstep * (2048 >> 4));
+}
+
 // D[tmem] (+)= A * B, issued by one thread
 __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
                                          uint32_t accumulate) {
@@ -199,6 +215,30 @@ __device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, i
         "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3),
         "r"(smem_addr(bar))
         : "memory");
+}
+
+// ---- TMA: 4-D tiled store shared -> global, tracked by the issuing
+// thread's bulk group (coordinates must not be negative)
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap *map, const void *src, int c0, int c1,
+                                             int c2, int c3) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(smem_addr(src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+        : "memory");
+}
+
+// ---- per-thread asynchronous copies (16 B, global -> shared), tracked per
+// thread: the issuing thread waits for its own copies before reading them
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
 // ---- bulk (non-tensor) copies

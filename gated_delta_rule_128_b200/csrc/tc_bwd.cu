@@ -27,9 +27,10 @@
 // Two kernels:
 //  * tc_bwd_state_kernel: one CTA per (b, h, half of d_v), walking the chunks
 //    in reverse with dS in tensor memory and the chunk records double-
-//    buffered; two tcgen05.mma round trips per chunk (dDelta; then dS and
-//    dU together).  Writes dw, dv, dS0, and per chunk dS_m, -dU and the
-//    half-sums of the chunk-end term to the workspace.
+//    buffered; two tcgen05.mma round trips per chunk on the state's path
+//    (dDelta; then dS), with dU and its outputs off that path.  Writes dw,
+//    dv, dS0, and per chunk dS_m, -dU and the half-sums of the chunk-end
+//    term to the workspace.
 //  * tc_bwd_grad_kernel: one CTA per (b, h, chunk), all chunks in parallel,
 //    full d_v; five products, then three accumulations, then dq, dk, db, dg.
 
@@ -50,8 +51,11 @@ constexpr uint32_t RAW_DO = 2 * REC_BYTES;    // dO half, bf16 [64 pos][64]
 constexpr uint32_t OP_DO = RAW_DO + 8192;     // dO fp16      [64 pos][64 v]  MN-major B
 constexpr uint32_t OP_DS = OP_DO + 8192;      // dX fp16      [128 key][64 v] MN-major B
 constexpr uint32_t OP_DD = OP_DS + 16384;     // dDelta fp16  [64 pos][64 v]  MN-major B
-constexpr uint32_t STG_S = OP_DD + 8192;      // S_c (true scale) fp16 [128 key][64 v]
-constexpr uint32_t MISC = STG_S + 16384;      // sEnd [2][128] f32; mbarriers; TMEM slot
+constexpr uint32_t STG_S = OP_DD + 8192;      // checkpoint S_m fp16 [128 key][64 v]
+constexpr uint32_t VV = STG_S + 16384;        // v half bf16 [64][64], 128-B swizzled; dv in place
+constexpr uint32_t VW = VV + 8192;            // w half f32, two [64][32] 128-B swizzled boxes; dw in place
+constexpr uint32_t NDU = VW + 16384;          // -dU fp16 [64 pos][64 v] (the workspace layout)
+constexpr uint32_t MISC = NDU + 8192;         // sEnd [2][128] f32; mbarriers; TMEM slot
 constexpr uint32_t SMEM_BYTES = MISC + 1024 + 128 + 1024;
 constexpr uint32_t TM_DS = 0, TM_DD = 64, TM_DU = 128;  // 256 columns allocated
 constexpr uint32_t ID_MM64 = idesc_f16(64, 64, true, true);
@@ -59,20 +63,23 @@ constexpr uint32_t ID_KM64 = idesc_f16(64, 64, false, true);
 constexpr uint32_t ID_MM128x64 = idesc_f16(128, 64, true, true);
 constexpr long long kWait = 2000000000LL;
 constexpr float kRange = 6.0e4f;
+static_assert(MISC % 1024 == 0, "alignment");
 }  // namespace tbs
 
 // One CTA per (b, h, half of d_v), walking the chunks in reverse with
 // dX = diag(e^(G_L - G_m)) dS_next in tensor memory.  Per chunk, from the
 // chunk's record (Qb, Kh, -W, T, P, factors):
-//   (1) dDelta = P^T dO + Kh dX,        dS_m = dX + Qb^T dO
-//   (2) dS_m += (-W)^T dDelta,          dU = T^T dDelta
-// then dS_c = diag(e^G_m) dS_m, the previous chunk's dX = diag(e^(G_L - G_m))
-// dS_c, dv = dU.w, dw = dU.v, and the workspace copies of dX, -dU and the
-// chunk-end half-sums for the gradient kernel.
+//   (1) dDelta = P^T dO + Kh dX  (committed alone),  then dS_m = dX + Qb^T dO
+//   (2) dS_m += (-W)^T dDelta  (committed alone),     then dU = T^T dDelta
+// then dS_c = diag(e^G_m) dS_m and the previous chunk's dX = diag(e^(G_L -
+// G_m)) dS_c.  dU is read while the next chunk's first products run: dv =
+// dU.w and dw = dU.v are formed in place of the v and w tiles (128-B
+// swizzled TMA tiles) and leave by TMA stores; -dU, dX and the chunk-end
+// half-sums go to the workspace for the gradient kernel.
 __global__ void __launch_bounds__(tbs::kThreads, 1)
-tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __nv_bfloat16 *__restrict__ v,
-                    const float *__restrict__ w, const float *__restrict__ dST,
-                    __nv_bfloat16 *__restrict__ dvout, float *__restrict__ dwout,
+tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_constant__ CUtensorMap mv,
+                    const __grid_constant__ CUtensorMap mw, const __grid_constant__ CUtensorMap mdv,
+                    const __grid_constant__ CUtensorMap mdw, const float *__restrict__ dST,
                     float *__restrict__ dS0, unsigned char *__restrict__ ws, TcWs lay,
                     unsigned int *status, Dims d) {
     using namespace tbs;
@@ -80,16 +87,18 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __nv_bfloat16
     unsigned char *sm = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smraw) + 1023) & ~static_cast<uintptr_t>(1023));
     float *sEnd = reinterpret_cast<float *>(sm + MISC);  // [2][128]
-    // 0, 1 records of stages 0, 1; 2 dO; 3 state checkpoint; 4, 5 product groups
+    // 0, 1 records of stages 0, 1; 2 dO; 3 state checkpoint; 4 v and w;
+    // 5 dDelta ready; 6 dS ready; 7 dU ready
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + MISC + 1024);
     uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + MISC + 1024 + 64);
     float big = 0.f;  // range check: operand magnitude
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int vh = blockIdx.x, h = blockIdx.y, bb = blockIdx.z, v0 = vh * 64;
-    const int NC = d.NC, T = d.T, H = d.H;
+    const int NC = d.NC, H = d.H;
     const int quarter = warp & 3, half = warp >> 2;
     const int key = quarter * 32 + lane;
+    const int r16 = quarter * 16 + lane;  // row of an M = 64 accumulator (lanes 0..15)
     const size_t bh = (size_t)bb * H + h;
     const unsigned char *recs = ws + lay.rec + bh * NC * (size_t)REC_BYTES;
 
@@ -98,7 +107,7 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __nv_bfloat16
         tmem_relinquish();
     }
     if (tid == 0) {
-        for (int i = 0; i < 6; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < 8; ++i) mbar_init(&bars[i], 1);
         mbar_fence_init();
     }
     fence_before_sync();
@@ -106,7 +115,8 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __nv_bfloat16
     fence_after_sync();
     const uint32_t tm = *tslot;
 
-    int issued[4] = {0, 0, 0, 0};
+    int issued[5] = {0, 0, 0, 0, 0};  // loads requested per barrier (thread 0)
+    int groups[3] = {0, 0, 0};        // commits to barriers 5, 6, 7 (thread 0)
     auto load_rec = [&](int cc) {
         const int s = cc & 1;
         mbar_expect_tx(&bars[s], REC_BYTES);
@@ -123,19 +133,43 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __nv_bfloat16
         bulk_load(sm + STG_S, ws + lay.ckS + ((bh * (NC + 1) + slot) * 2 + vh) * 16384, 16384, &bars[3]);
         ++issued[3];
     };
+    auto load_vw = [&](int cc) {
+        mbar_expect_tx(&bars[4], 8192 + 16384);
+        tma_load_4d(sm + VV, &mv, v0, h, cc * 64, bb, &bars[4]);
+        tma_load_4d(sm + VW, &mw, v0, h, cc * 64, bb, &bars[4]);
+        tma_load_4d(sm + VW + 8192, &mw, v0 + 32, h, cc * 64, bb, &bars[4]);
+        ++issued[4];
+    };
     auto rec_fac = [&](int cc) {  // e^(G_L - G_m) of chunk cc (then e^G_m at +128)
         return reinterpret_cast<const float *>(sm + STG + (cc & 1) * REC_BYTES + REC_FAC);
     };
-    // dX of chunk c, this thread's row and 32 columns: TMEM, fp16 operand, workspace copy
-    auto put_dx = [&](int c, float *x) {
+    // dO of the chunk in RAW_DO -> fp16 operand (each thread 16 values)
+    auto convert_do = [&]() {
+        const int r = tid >> 2, cg = tid & 3;
+        const uint4 d0 = *reinterpret_cast<const uint4 *>(sm + RAW_DO + r * 128 + cg * 32);
+        const uint4 d1 = *reinterpret_cast<const uint4 *>(sm + RAW_DO + r * 128 + cg * 32 + 16);
+        const __nv_bfloat162 *a = reinterpret_cast<const __nv_bfloat162 *>(&d0);
+        const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&d1);
+        float x[16];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            x[2 * e] = __low2float(a[e]);
+            x[2 * e + 1] = __high2float(a[e]);
+            x[8 + 2 * e] = __low2float(b2[e]);
+            x[8 + 2 * e + 1] = __high2float(b2[e]);
+        }
+        st_h8(sm + OP_DO + sw128_chunk(r, 2 * cg, 64), x);
+        st_h8(sm + OP_DO + sw128_chunk(r, 2 * cg + 1, 64), x + 8);
+        big = absmax8(x, big);
+        big = absmax8(x + 8, big);
+    };
+    // dX of chunk c into TMEM and the fp16 operand (this thread's row, 32 columns)
+    auto put_dx = [&](float *x) {
         tmem_st16(taddr(tm + TM_DS, quarter * 32, 32 * half), x);
         tmem_st16(taddr(tm + TM_DS, quarter * 32, 32 * half + 16), x + 16);
-        unsigned char *dst = ws + lay.ckdS + ((bh * NC + c) * 2 + vh) * 16384;
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
-            const uint32_t off = sw128_chunk(key, 4 * half + jj, 128);
-            st_h8(sm + OP_DS + off, x + 8 * jj);
-            st_h8(dst + off, x + 8 * jj);
+            st_h8(sm + OP_DS + sw128_chunk(key, 4 * half + jj, 128), x + 8 * jj);
             big = absmax8(x + 8 * jj, big);
         }
     };
@@ -151,14 +185,68 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __nv_bfloat16
         }
         return acc;
     };
+    // dU of chunk cc (TMEM) -> dv, dw in place of v, w; -dU staged; then the
+    // stores, and the next v, w tiles (chunk cc - 1).  All threads.
+    auto flush_du = [&](int cc, uint32_t vw_par, uint32_t du_par) {
+        bool fine = mbar_wait(&bars[7], du_par, kWait);
+        fine = mbar_wait(&bars[4], vw_par, kWait) && fine;
+        fence_after_sync();
+        float du[32];
+        tmem_ld16(taddr(tm + TM_DU, quarter * 32, 32 * half), du);
+        tmem_ld16(taddr(tm + TM_DU, quarter * 32, 32 * half + 16), du + 16);
+        tmem_wait_ld();
+        if (lane < 16) {
+            const int r = r16;
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {  // v chunk 4 * half + jj: 8 columns
+                unsigned char *pv = sm + VV + sw128_chunk(r, 4 * half + jj, 64);
+                const uint4 vq = *reinterpret_cast<const uint4 *>(pv);
+                const __nv_bfloat162 *v2 = reinterpret_cast<const __nv_bfloat162 *>(&vq);
+                unsigned char *pw0 = sm + VW + half * 8192 + sw128_chunk(r, 2 * jj, 64);
+                unsigned char *pw1 = sm + VW + half * 8192 + sw128_chunk(r, 2 * jj + 1, 64);
+                const float4 w0 = *reinterpret_cast<const float4 *>(pw0);
+                const float4 w1 = *reinterpret_cast<const float4 *>(pw1);
+                const float *u = du + 8 * jj;
+                float dv8[8] = {u[0] * w0.x, u[1] * w0.y, u[2] * w0.z, u[3] * w0.w,
+                                u[4] * w1.x, u[5] * w1.y, u[6] * w1.z, u[7] * w1.w};
+                *reinterpret_cast<float4 *>(pw0) = make_float4(
+                    u[0] * __low2float(v2[0]), u[1] * __high2float(v2[0]), u[2] * __low2float(v2[1]),
+                    u[3] * __high2float(v2[1]));
+                *reinterpret_cast<float4 *>(pw1) = make_float4(
+                    u[4] * __low2float(v2[2]), u[5] * __high2float(v2[2]), u[6] * __low2float(v2[3]),
+                    u[7] * __high2float(v2[3]));
+                st_bf16x8(pv, dv8);
+            }
+#pragma unroll
+            for (int j = 0; j < 32; ++j) du[j] = -du[j];
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                st_h8(sm + NDU + sw128_chunk(r, 4 * half + jj, 64), du + 8 * jj);
+                big = absmax8(du + 8 * jj, big);
+            }
+        }
+        fence_proxy_async();
+        __syncthreads();
+        if (tid == 0) {
+            tma_store_4d(&mdv, sm + VV, v0, h, cc * 64, bb);
+            tma_store_4d(&mdw, sm + VW, v0, h, cc * 64, bb);
+            tma_store_4d(&mdw, sm + VW + 8192, v0 + 32, h, cc * 64, bb);
+            bulk_store(ws + lay.ckndU + ((bh * NC + cc) * 2 + vh) * 8192, sm + NDU, 8192);
+            bulk_commit();
+            bulk_wait_read();  // VV, VW and NDU may be rewritten
+            if (cc > 0) load_vw(cc - 1);
+        }
+        return fine;
+    };
 
     if (tid == 0) {
         load_rec(NC - 1);
         if (NC > 1) load_rec(NC - 2);
         load_do(NC - 1);
         load_s(NC);
+        load_vw(NC - 1);
     }
-    // dS_T (or zero); the last chunk's end term rowsum(dS_T . S_T); its dX
+    // ---------------- prologue: dS_T (or zero), the last chunk's end term and dX; dO
     bool ok;
     {
         float x[32];
@@ -170,12 +258,14 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __nv_bfloat16
             x[j] = t.x; x[j + 1] = t.y; x[j + 2] = t.z; x[j + 3] = t.w;
         }
         ok = mbar_wait(&bars[3], 0, kWait);
-        ok = ok && mbar_wait(&bars[(NC - 1) & 1], 0, kWait);
-        sEnd[half * 128 + key] = end_term(x);
+        ok = mbar_wait(&bars[(NC - 1) & 1], 0, kWait) && ok;
+        ok = mbar_wait(&bars[2], 0, kWait) && ok;
+        sEnd[half * 128 + key] = end_term(x);  // the last checkpoint is S_T itself
         const float gam = rec_fac(NC - 1)[key];
 #pragma unroll
         for (int j = 0; j < 32; ++j) x[j] *= gam;
-        put_dx(NC - 1, x);
+        put_dx(x);
+        convert_do();
         tmem_wait_st();
     }
     fence_proxy_async();
@@ -185,66 +275,45 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __nv_bfloat16
         if (half == 0)
             reinterpret_cast<float *>(ws + lay.ckEnd + ((bh * NC + NC - 1) * 2 + vh) * 512)[key] =
                 sEnd[key] + sEnd[128 + key];
-        if (tid == 0 && NC > 1) load_s(NC - 1);
+        if (tid == 0) {
+            fence_after_sync();
+            bulk_store(ws + lay.ckdS + ((bh * NC + NC - 1) * 2 + vh) * 16384, sm + OP_DS, 16384);
+            bulk_commit();
+            if (NC > 1) {
+                load_s(NC - 1);
+                load_do(NC - 2);
+            }
+        }
     }
 
     for (int i = 0; i < NC && !abort; ++i) {
-        const int c = NC - 1 - i, c0 = c * 64;
+        const int c = NC - 1 - i;
         const uint32_t par = i & 1;
         unsigned char *stg = sm + STG + (c & 1) * REC_BYTES;
-        // ---------------- dO to fp16, product group 1
-        ok = mbar_wait(&bars[c & 1], (i >> 1) & 1, kWait);
-        ok = ok && mbar_wait(&bars[2], par, kWait);
-        {
-            const int r = tid >> 2, cg = tid & 3;  // row, 16-column group
-            const uint4 d0 = *reinterpret_cast<const uint4 *>(sm + RAW_DO + r * 128 + cg * 32);
-            const uint4 d1 = *reinterpret_cast<const uint4 *>(sm + RAW_DO + r * 128 + cg * 32 + 16);
-            const __nv_bfloat162 *a = reinterpret_cast<const __nv_bfloat162 *>(&d0);
-            const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&d1);
-            float x[16];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                x[2 * e] = __low2float(a[e]);
-                x[2 * e + 1] = __high2float(a[e]);
-                x[8 + 2 * e] = __low2float(b2[e]);
-                x[8 + 2 * e + 1] = __high2float(b2[e]);
-            }
-            st_h8(sm + OP_DO + sw128_chunk(r, 2 * cg, 64), x);
-            st_h8(sm + OP_DO + sw128_chunk(r, 2 * cg + 1, 64), x + 8);
-        }
-        fence_proxy_async();
-        fence_before_sync();
-        if (__syncthreads_or(!ok)) { abort = true; break; }
+        // ---------------- (1) dDelta products, then Qb^T dO
+        ok = mbar_wait(&bars[c & 1], (i >> 1) & 1, kWait) && ok;  // record c
         if (tid == 0) {
-            fence_after_sync();
-            if (c > 0) load_do(c - 1);  // raw dO consumed
-            const uint32_t st = smem_addr(stg), dO = smem_addr(sm + OP_DO), dx = smem_addr(sm + OP_DS);
+            const uint32_t st = smem_addr(stg);
+            // Qb is rows 64..127 of the [-W; Qb] tile: 64-key blocks 16 KB apart
+            const uint64_t dP = desc_mnmajor(st + REC_P, 64, 0), dO = desc_mnmajor(smem_addr(sm + OP_DO), 64, 0),
+                           dK = desc_kmajor(st + REC_KH, 64, 0), dX = desc_mnmajor(smem_addr(sm + OP_DS), 128, 0),
+                           dQ = desc_mnmajor_lbo(st + REC_WQ + 8192, 16384, 0);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tm + TM_DD, desc_mnmajor(st + REC_P, 64, ks), desc_mnmajor(dO, 64, ks), ID_MM64, ks > 0);
+                mma_bf16(tm + TM_DD, kstep_mnmajor(dP, ks), kstep_mnmajor(dO, ks), ID_MM64, ks > 0);
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks)
-                mma_bf16(tm + TM_DD, desc_kmajor(st + REC_KH, 64, ks), desc_mnmajor(dx, 128, ks), ID_KM64, 1);
+                mma_bf16(tm + TM_DD, kstep_kmajor(dK, 64, ks), kstep_mnmajor(dX, ks), ID_KM64, 1);
+            mma_commit(&bars[5]);
+            ++groups[0];
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tm + TM_DS, desc_mnmajor(st + REC_QB, 64, ks), desc_mnmajor(dO, 64, ks), ID_MM128x64, 1);
-            mma_commit(&bars[4]);
+                mma_bf16(tm + TM_DS, kstep_mnmajor(dQ, ks), kstep_mnmajor(dO, ks), ID_MM128x64, 1);
         }
-        // v and w of this thread's row and columns, for dw and dv below:
-        // requested now so that the loads overlap the products
-        uint4 vreg[4];
-        float4 wreg[8];
-        const int r_own = quarter * 16 + lane;
-        const bool row_ok = lane < 16 && c0 + r_own < T;
-        {
-            const size_t ov = tok(d, bb, row_ok ? c0 + r_own : 0, h, 128) + v0 + 32 * half;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) vreg[j] = row_ok ? *reinterpret_cast<const uint4 *>(v + ov + 8 * j) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) wreg[j] = row_ok ? *reinterpret_cast<const float4 *>(w + ov + 4 * j) : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-        // ---------------- dDelta to fp16, product group 2
-        ok = mbar_wait(&bars[4], par, kWait);
+        // the next chunk's dU, while these products run
+        if (c + 1 < NC) ok = flush_du(c + 1, (i - 1) & 1, (i - 1) & 1) && ok;
+        // ---------------- dDelta to fp16, (2) products
+        ok = mbar_wait(&bars[5], par, kWait) && ok;
         fence_after_sync();
         {
             float dd[32];
@@ -252,41 +321,45 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __nv_bfloat16
             tmem_ld16(taddr(tm + TM_DD, quarter * 32, 32 * half + 16), dd + 16);
             tmem_wait_ld();
             if (lane < 16) {
-                const int r = quarter * 16 + lane;
 #pragma unroll
                 for (int jj = 0; jj < 4; ++jj) {
-                    st_h8(sm + OP_DD + sw128_chunk(r, 4 * half + jj, 64), dd + 8 * jj);
+                    st_h8(sm + OP_DD + sw128_chunk(r16, 4 * half + jj, 64), dd + 8 * jj);
                     big = absmax8(dd + 8 * jj, big);
                 }
             }
         }
         fence_proxy_async();
         fence_before_sync();
-        if (__syncthreads_or(!ok)) { abort = true; break; }
+        __syncthreads();
         if (tid == 0) {
             fence_after_sync();
-            const uint32_t st = smem_addr(stg), dd = smem_addr(sm + OP_DD);
+            const uint32_t st = smem_addr(stg);
+            const uint64_t dW = desc_mnmajor_lbo(st + REC_WQ, 16384, 0), dT = desc_mnmajor(st + REC_T, 64, 0),
+                           dD = desc_mnmajor(smem_addr(sm + OP_DD), 64, 0);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tm + TM_DS, desc_mnmajor(st + REC_WN, 64, ks), desc_mnmajor(dd, 64, ks), ID_MM128x64, 1);
+                mma_bf16(tm + TM_DS, kstep_mnmajor(dW, ks), kstep_mnmajor(dD, ks), ID_MM128x64, 1);
+            mma_commit(&bars[6]);
+            ++groups[1];
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tm + TM_DU, desc_mnmajor(st + REC_T, 64, ks), desc_mnmajor(dd, 64, ks), ID_MM64, ks > 0);
-            mma_commit(&bars[5]);
+                mma_bf16(tm + TM_DU, kstep_mnmajor(dT, ks), kstep_mnmajor(dD, ks), ID_MM64, ks > 0);
+            mma_commit(&bars[7]);
+            ++groups[2];
+            bulk_wait_read();  // the dX copy has left OP_DS
         }
-        // ---------------- dS_c, the previous chunk's dX and end term; dv, dw, -dU
-        ok = mbar_wait(&bars[5], par, kWait);
+        // ---------------- dS_c; the previous chunk's end term, dX and dO
+        ok = mbar_wait(&bars[6], par, kWait) && ok;
         if (c > 0) {
-            ok = ok && mbar_wait(&bars[3], (i + 1) & 1, kWait);                 // S_c
-            ok = ok && mbar_wait(&bars[(c - 1) & 1], ((i + 1) >> 1) & 1, kWait);  // record c-1
+            ok = mbar_wait(&bars[3], (i + 1) & 1, kWait) && ok;                 // S_m of chunk c
+            ok = mbar_wait(&bars[(c - 1) & 1], ((i + 1) >> 1) & 1, kWait) && ok;  // record c-1
+            ok = mbar_wait(&bars[2], (i + 1) & 1, kWait) && ok;                 // dO of chunk c-1
         }
         fence_after_sync();
         {
-            float sv[32], du[32];
+            float sv[32];
             tmem_ld16(taddr(tm + TM_DS, quarter * 32, 32 * half), sv);
             tmem_ld16(taddr(tm + TM_DS, quarter * 32, 32 * half + 16), sv + 16);
-            tmem_ld16(taddr(tm + TM_DU, quarter * 32, 32 * half), du);
-            tmem_ld16(taddr(tm + TM_DU, quarter * 32, 32 * half + 16), du + 16);
             tmem_wait_ld();
             const float e = reinterpret_cast<const float *>(stg + REC_FAC)[128 + key];
 #pragma unroll
@@ -299,65 +372,46 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __nv_bfloat16
                         *reinterpret_cast<float4 *>(dst + j) = make_float4(sv[j], sv[j + 1], sv[j + 2], sv[j + 3]);
                 }
             } else {
-                sEnd[half * 128 + key] = end_term(sv);
+                // the checkpoint holds S_m = diag(e^G_m) S_c
+                sEnd[half * 128 + key] = end_term(sv) / e;
                 const float gam = rec_fac(c - 1)[key];
 #pragma unroll
                 for (int j = 0; j < 32; ++j) sv[j] *= gam;
-                put_dx(c - 1, sv);
+                put_dx(sv);
+                convert_do();
+                tmem_wait_st();
             }
-            if (lane < 16) {
-                const int r = quarter * 16 + lane;
-                if (row_ok) {
-                    const size_t ov = tok(d, bb, c0 + r, h, 128) + v0 + 32 * half;
-                    float dwv[32], dvv[32];
-#pragma unroll
-                    for (int j = 0; j < 32; j += 8) {
-                        const __nv_bfloat162 *v2 = reinterpret_cast<const __nv_bfloat162 *>(&vreg[j / 8]);
-                        const float4 w0 = wreg[j / 4], w1 = wreg[j / 4 + 1];
-                        float wf[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-#pragma unroll
-                        for (int e2 = 0; e2 < 4; ++e2) {
-                            dwv[j + 2 * e2] = du[j + 2 * e2] * __low2float(v2[e2]);
-                            dwv[j + 2 * e2 + 1] = du[j + 2 * e2 + 1] * __high2float(v2[e2]);
-                        }
-#pragma unroll
-                        for (int e2 = 0; e2 < 8; ++e2) dvv[j + e2] = du[j + e2] * wf[e2];
-                    }
-#pragma unroll
-                    for (int j = 0; j < 32; j += 4)
-                        *reinterpret_cast<float4 *>(dwout + ov + j) =
-                            make_float4(dwv[j], dwv[j + 1], dwv[j + 2], dwv[j + 3]);
-#pragma unroll
-                    for (int jj = 0; jj < 4; ++jj)
-                        st_bf16x8(reinterpret_cast<unsigned char *>(dvout + ov) + 16 * jj, dvv + 8 * jj);
-                }
-#pragma unroll
-                for (int j = 0; j < 32; ++j) du[j] = -du[j];
-                unsigned char *dst = ws + lay.ckndU + ((bh * NC + c) * 2 + vh) * 8192;
-#pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                    st_h8(dst + sw128_chunk(r, 4 * half + jj, 64), du + 8 * jj);
-                    big = absmax8(du + 8 * jj, big);
-                }
-            }
-            tmem_wait_st();
         }
         fence_proxy_async();
         fence_before_sync();
         if (__syncthreads_or(!ok)) { abort = true; break; }
-        if (c > 0 && half == 0)
-            reinterpret_cast<float *>(ws + lay.ckEnd + ((bh * NC + c - 1) * 2 + vh) * 512)[key] =
-                sEnd[key] + sEnd[128 + key];
-        if (tid == 0) {
-            if (c > 0) load_s(c - 1);     // S_c consumed
-            if (c >= 2) load_rec(c - 2);  // this chunk's record consumed
+        if (c > 0) {
+            if (half == 0)
+                reinterpret_cast<float *>(ws + lay.ckEnd + ((bh * NC + c - 1) * 2 + vh) * 512)[key] =
+                    sEnd[key] + sEnd[128 + key];
+            if (tid == 0) {
+                fence_after_sync();
+                bulk_store(ws + lay.ckdS + ((bh * NC + c - 1) * 2 + vh) * 16384, sm + OP_DS, 16384);
+                bulk_commit();
+                load_s(c - 1);                // S_m of chunk c consumed
+                if (c >= 2) {
+                    load_do(c - 2);           // raw dO consumed
+                    // this chunk's record is consumed once T^T dDelta has read T
+                    if (!mbar_wait(&bars[7], par, kWait)) record_status(status, GDN2_ERR_TIMEOUT);
+                    load_rec(c - 2);
+                }
+            }
         }
     }
+    if (!abort) ok = flush_du(0, (NC - 1) & 1, (NC - 1) & 1);
     if (!(big <= kRange)) record_status(status, GDN2_ERR_RANGE);
-    if (tid == 0 && abort) {
+    if (tid == 0) bulk_wait_all();
+    if (tid == 0 && (abort || !ok)) {
         record_status(status, GDN2_ERR_TIMEOUT);
-        for (int k2 = 0; k2 < 4; ++k2)
+        for (int k2 = 0; k2 < 5; ++k2)
             if (issued[k2] > 0) mbar_wait(&bars[k2], (issued[k2] - 1) & 1, kWait);
+        for (int k2 = 0; k2 < 3; ++k2)
+            if (groups[k2] > 0) mbar_wait(&bars[5 + k2], (groups[k2] - 1) & 1, kWait);
     }
     fence_before_sync();
     __syncthreads();
@@ -369,7 +423,7 @@ namespace tbg {
 constexpr int kThreads = 256;
 constexpr uint32_t RAW_Q = 0, RAW_K = 16384, RAW_B = 32768, RAW_G = 65536;  // g, later G - G_m
 constexpr uint32_t OP_DO = 98304;     // dO fp16 [64 pos][128 v] K-major (in place of raw dO)
-constexpr uint32_t BL_S = 114688;     // S_m [128 key][128 v] K-major B   (later Qb, Kc, Kh; then dG)
+constexpr uint32_t BL_S = 114688;     // S_m [128 key][128 v] K-major B (the checkpoint; later Qb, Kc, Kh; then dG)
 constexpr uint32_t BL_DS = 147456;    // dS_m [128 key][128 v]
 constexpr uint32_t BL_D = 180224;     // Delta [64 pos][128 v]              (later dP, dA)
 constexpr uint32_t BL_NDU = 196608;   // -dU [64 pos][128 v]
@@ -441,7 +495,7 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
         sEnd[tid] = e0[tid] + e0[128 + tid];
     }
     bool ok = mbar_wait(&bars[0], 0, kWait);
-    // ---------------- G1: decay, S_m, dO operand; five products
+    // ---------------- G1: decay, dO operand; five products (the checkpoint holds S_m)
     float G[8][4];
     cumsum_local(reinterpret_cast<const float *>(sm + RAW_G), scan, warp, lane, G);
     // dO: raw bf16 rows [64][128] -> fp16 K-major tile in place (values held in registers)
@@ -460,37 +514,25 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
             st_h4(sm + OP_DO + sw128_off(r, 4 * lane, 64), __low2float(d2[0]), __high2float(d2[0]),
                   __low2float(d2[1]), __high2float(d2[1]));
         }
-        __syncthreads();
-        // S_m = diag(e^G_m) S_c, in place: thread -> (key, 64 value columns)
-        {
-            const int kr = tid >> 1, hb = tid & 1;
-            const float e = sRef[kr];
-#pragma unroll
-            for (int jj = 0; jj < 8; ++jj) {
-                unsigned char *p = sm + BL_S + sw128_chunk(kr, hb * 8 + jj, 128);
-                float s8[8];
-                ld_h8(p, s8);
-#pragma unroll
-                for (int e2 = 0; e2 < 8; ++e2) s8[e2] *= e;
-                st_h8(p, s8);
-                big = absmax8(s8, big);
-            }
-        }
         fence_proxy_async();
         fence_before_sync();
         __syncthreads();
         if (tid == 0) {
             fence_after_sync();
-            const uint32_t dO = smem_addr(sm + OP_DO), S = smem_addr(sm + BL_S),
-                           DS = smem_addr(sm + BL_DS), D = smem_addr(sm + BL_D),
-                           NDU = smem_addr(sm + BL_NDU);
+            const uint64_t dO = desc_kmajor(smem_addr(sm + OP_DO), 64, 0),
+                           S = desc_kmajor(smem_addr(sm + BL_S), 128, 0),
+                           DS = desc_kmajor(smem_addr(sm + BL_DS), 128, 0),
+                           D = desc_kmajor(smem_addr(sm + BL_D), 64, 0),
+                           NDU = desc_kmajor(smem_addr(sm + BL_NDU), 64, 0);
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
-                mma_bf16(tm + TM_DP, desc_kmajor(dO, 64, ks), desc_kmajor(D, 64, ks), ID_KK64, ks > 0);
-                mma_bf16(tm + TM_DA, desc_kmajor(NDU, 64, ks), desc_kmajor(D, 64, ks), ID_KK64, ks > 0);
-                mma_bf16(tm + TM_Y1, desc_kmajor(dO, 64, ks), desc_kmajor(S, 128, ks), ID_KK128, ks > 0);
-                mma_bf16(tm + TM_Y2, desc_kmajor(NDU, 64, ks), desc_kmajor(S, 128, ks), ID_KK128, ks > 0);
-                mma_bf16(tm + TM_Y3, desc_kmajor(D, 64, ks), desc_kmajor(DS, 128, ks), ID_KK128, ks > 0);
+                const uint64_t a_do = kstep_kmajor(dO, 64, ks), a_ndu = kstep_kmajor(NDU, 64, ks),
+                               a_d = kstep_kmajor(D, 64, ks), b_s = kstep_kmajor(S, 128, ks);
+                mma_bf16(tm + TM_DP, a_do, a_d, ID_KK64, ks > 0);
+                mma_bf16(tm + TM_DA, a_ndu, a_d, ID_KK64, ks > 0);
+                mma_bf16(tm + TM_Y1, a_do, b_s, ID_KK128, ks > 0);
+                mma_bf16(tm + TM_Y2, a_ndu, b_s, ID_KK128, ks > 0);
+                mma_bf16(tm + TM_Y3, a_d, kstep_kmajor(DS, 128, ks), ID_KK128, ks > 0);
             }
             mma_commit(&bars[1]);
         }
@@ -525,15 +567,19 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
     if (!abort) {
         if (tid == 0) {
             fence_after_sync();
-            const uint32_t dP = smem_addr(sm + OP_DP), dA = smem_addr(sm + OP_DA),
-                           qb = smem_addr(sm + OP_QB), kc = smem_addr(sm + OP_KC),
-                           kh = smem_addr(sm + OP_KH);
+            const uint32_t dP = smem_addr(sm + OP_DP), dA = smem_addr(sm + OP_DA);
+            const uint64_t kP = desc_kmajor(dP, 64, 0), kA = desc_kmajor(dA, 64, 0),
+                           mP = desc_mnmajor(dP, 64, 0), mA = desc_mnmajor(dA, 64, 0),
+                           qb = desc_mnmajor(smem_addr(sm + OP_QB), 64, 0),
+                           kc = desc_mnmajor(smem_addr(sm + OP_KC), 64, 0),
+                           kh = desc_mnmajor(smem_addr(sm + OP_KH), 64, 0);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
-                mma_bf16(tm + TM_Y1, desc_kmajor(dP, 64, ks), desc_mnmajor(kh, 64, ks), ID_KM128, 1);
-                mma_bf16(tm + TM_Y2, desc_kmajor(dA, 64, ks), desc_mnmajor(kh, 64, ks), ID_KM128, 1);
-                mma_bf16(tm + TM_Y3, desc_mnmajor(dP, 64, ks), desc_mnmajor(qb, 64, ks), ID_MM128, 1);
-                mma_bf16(tm + TM_Y3, desc_mnmajor(dA, 64, ks), desc_mnmajor(kc, 64, ks), ID_MM128, 1);
+                const uint64_t b_kh = kstep_mnmajor(kh, ks);
+                mma_bf16(tm + TM_Y1, kstep_kmajor(kP, 64, ks), b_kh, ID_KM128, 1);
+                mma_bf16(tm + TM_Y2, kstep_kmajor(kA, 64, ks), b_kh, ID_KM128, 1);
+                mma_bf16(tm + TM_Y3, kstep_mnmajor(mP, ks), kstep_mnmajor(qb, ks), ID_MM128, 1);
+                mma_bf16(tm + TM_Y3, kstep_mnmajor(mA, ks), kstep_mnmajor(kc, ks), ID_MM128, 1);
             }
             mma_commit(&bars[2]);
         }
@@ -639,10 +685,14 @@ cudaError_t tc_bwd_launch(const void *q, const void *k, const void *v, const flo
                           void *dq, void *dk, void *dv, float *dg, float *db, float *dw,
                           float *dS0, void *ws, unsigned int *status, const Dims &d,
                           cudaStream_t s) {
-    CUtensorMap mq, mk, mdo_half, mdo, mg, mb;
+    CUtensorMap mq, mk, mdo_half, mdo, mg, mb, mv, mw, mdv, mdw;
     if (!make_btHd_map(&mq, q, true, d.B, d.T, d.H, 128, 64, 128) ||
         !make_btHd_map(&mk, k, true, d.B, d.T, d.H, 128, 64, 128) ||
         !make_btHd_map(&mdo_half, dO, true, d.B, d.T, d.H, 128, 64, 64) ||
+        !make_btHd_map(&mv, v, true, d.B, d.T, d.H, 128, 64, 64, true) ||
+        !make_btHd_map(&mw, w, false, d.B, d.T, d.H, 128, 64, 32, true) ||
+        !make_btHd_map(&mdv, dv, true, d.B, d.T, d.H, 128, 64, 64, true) ||
+        !make_btHd_map(&mdw, dw, false, d.B, d.T, d.H, 128, 64, 32, true) ||
         !make_btHd_map(&mdo, dO, true, d.B, d.T, d.H, 128, 64, 128) ||
         !make_btHd_map(&mg, g, false, d.B, d.T, d.H, 128, 64, 128) ||
         !make_btHd_map(&mb, b, false, d.B, d.T, d.H, 128, 64, 128))
@@ -656,8 +706,7 @@ cudaError_t tc_bwd_launch(const void *q, const void *k, const void *v, const flo
     if (e != cudaSuccess) return e;
     launch_begin(K_TC_BWD_STATE, s);
     tc_bwd_state_kernel<<<dim3(2, d.H, d.B), tbs::kThreads, tbs::SMEM_BYTES, s>>>(
-        mdo_half, (const __nv_bfloat16 *)v, w, dST, (__nv_bfloat16 *)dv, dw, dS0,
-        (unsigned char *)ws, lay, status, d);
+        mdo_half, mv, mw, mdv, mdw, dST, dS0, (unsigned char *)ws, lay, status, d);
     launch_end(K_TC_BWD_STATE, s);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     launch_begin(K_TC_BWD_GRAD, s);

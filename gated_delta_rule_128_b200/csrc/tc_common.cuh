@@ -132,5 +132,40 @@ __device__ __forceinline__ float write_factors(const unsigned char *rq, const un
     return gmax;
 }
 
+// The same operands for the chunk record's layout: Kc into rows 0..63 and Qb
+// into rows 64..127 of the [128][128] K-major tile at oWQ, Kh into the
+// [64][128] K-major tile at oKh.  Returns the largest |G - G_m| seen.
+__device__ __forceinline__ float write_factors_rec(const unsigned char *rq, const unsigned char *rk,
+                                                   const float *rb, const float G[8][4],
+                                                   unsigned char *oWQ, unsigned char *oKh,
+                                                   int warp, int lane) {
+    float gmax = 0.f;
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+        const int r = 8 * warp + m;
+        uint2 qr = *reinterpret_cast<const uint2 *>(rq + r * 256 + lane * 8);
+        uint2 kr = *reinterpret_cast<const uint2 *>(rk + r * 256 + lane * 8);
+        float4 bv = *reinterpret_cast<const float4 *>(rb + r * 128 + 4 * lane);
+        const __nv_bfloat162 *q2 = reinterpret_cast<const __nv_bfloat162 *>(&qr);
+        const __nv_bfloat162 *k2 = reinterpret_cast<const __nv_bfloat162 *>(&kr);
+        float qf[4] = {__low2float(q2[0]), __high2float(q2[0]), __low2float(q2[1]), __high2float(q2[1])};
+        float kf[4] = {__low2float(k2[0]), __high2float(k2[0]), __low2float(k2[1]), __high2float(k2[1])};
+        float bf[4] = {bv.x, bv.y, bv.z, bv.w};
+        float qb[4], kc[4], kh[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float e = __expf(G[m][i]), ei = __expf(-G[m][i]);
+            qb[i] = qf[i] * e;
+            kc[i] = bf[i] * kf[i] * e;
+            kh[i] = kf[i] * ei;
+            gmax = fmaxf(gmax, fabsf(G[m][i]));
+        }
+        st_h4(oWQ + sw128_off(r, 4 * lane, 128), kc[0], kc[1], kc[2], kc[3]);
+        st_h4(oWQ + sw128_off(r + 64, 4 * lane, 128), qb[0], qb[1], qb[2], qb[3]);
+        st_h4(oKh + sw128_off(r, 4 * lane, 64), kh[0], kh[1], kh[2], kh[3]);
+    }
+    return gmax;
+}
+
 }  // namespace tcc
 }  // namespace gdn2

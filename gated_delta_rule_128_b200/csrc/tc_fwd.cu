@@ -11,14 +11,18 @@
 //
 // One CTA owns one (b, h) and one 64-column half of d_v and walks the
 // sequence's chunks in order with its fp32 state slice resident in tensor
-// memory.  The chunk records (Qb, Kh, -W, T, P, decay factors; 65 KB) are
-// double-buffered in shared memory and requested two chunks ahead, since
-// they do not depend on the state; v and w arrive by TMA one chunk ahead.
-// Per chunk two tcgen05.mma round trips sit on the state's path:
-//   (1) D = T U + (-W) S_m,  O = Qb S_m          (D in TMEM is Delta)
-//   (2) O += P Delta,        S += Kh^T Delta
-// then the state is rescaled into the next chunk's frame in TMEM and copied
-// to fp16 for the next chunk's products.
+// memory.  The chunk records are double-buffered in shared memory and
+// requested two chunks ahead, since they do not depend on the state.
+//
+// Both state-side products are M = 128 tcgen05.mma groups into one
+// [Delta; O] accumulator (rows 0..63 Delta, 64..127 O; two such accumulators
+// alternate between chunks):
+//   (1) [T; 0] U + [-W; Qb] S_m            -> Delta and Qb S_m
+//   (2) [0; P] Delta,  and  S += Kh^T Delta
+// Warp roles: warps 0, 1, 4, 5 (TMEM lanes 0..63) read Delta; warps 2, 3,
+// 6, 7 (lanes 64..127) read the previous chunk's O and form the next chunk's
+// U = w.v off the state's path; all warps rescale the state into the next
+// chunk's frame.
 //
 // Precision and range: fp16 operands carry 11 significant bits (bf16 carries
 // 8, which left the output error at the 5e-3 tolerance); Delta is formed in
@@ -26,7 +30,8 @@
 // GDN2_ERR_RANGE.
 //
 // For the backward the call can also leave in the workspace (TcWs): every
-// chunk-entry state and S_T (fp16, true scale) and Delta per chunk.
+// chunk's entry state in its own frame, S_m (fp16, a copy of the operand),
+// S_T (fp16, true scale) and Delta per chunk.
 
 #include "common.cuh"
 #include "tc.cuh"
@@ -39,22 +44,31 @@ using namespace tcc;
 
 namespace tfwd {
 constexpr int kThreads = 256;
+// one record stage: the record with an 8 KB zero tile between T and P, so
+// that [T; 0] and [0; P] are M = 128 operands
+constexpr uint32_t S_WQ = 0, S_KH = 32768, S_T = 49152, S_Z = 57344, S_P = 65536, S_FAC = 73728;
+constexpr uint32_t STAGE = 74752;
 // shared memory map (bytes from a 1024-aligned base)
-constexpr uint32_t STG = 0;                  // two chunk records, REC_BYTES each
-constexpr uint32_t RAW_V = 2 * REC_BYTES;    // v half, bf16 [64 pos][64]
+constexpr uint32_t STG = 0;                  // two record stages
+constexpr uint32_t RAW_V = 2 * STAGE;        // v half, bf16 [64 pos][64]
 constexpr uint32_t RAW_W = RAW_V + 8192;     // w half, f32  [64 pos][64]
-constexpr uint32_t OP_U = RAW_W + 16384;     // U = w.v      [64 pos][64 v]  MN-major B
-constexpr uint32_t OP_S = OP_U + 8192;       // S_m (fp16)   [128 key][64 v] MN-major B
-constexpr uint32_t OP_D = OP_S + 16384;      // Delta        [64 pos][64 v]  MN-major B
+constexpr uint32_t OP_U = RAW_W + 16384;     // two U = w.v tiles [64 pos][64 v] MN-major, 8 KB each
+constexpr uint32_t OP_S = OP_U + 16384;      // S_m (fp16)   [128 key][64 v] MN-major
+constexpr uint32_t OP_D = OP_S + 16384;      // Delta        [64 pos][64 v]  MN-major
 constexpr uint32_t MISC = OP_D + 8192;       // mbarriers, TMEM slot
 constexpr uint32_t SMEM_BYTES = MISC + 128 + 1024;
-// tensor memory columns (256 allocated)
-constexpr uint32_t TM_S = 0, TM_D = 64, TM_O = 128;
-constexpr uint32_t ID_KM64 = idesc_f16(64, 64, false, true);
+// tensor memory columns (256 allocated): state, then two [Delta; O] accumulators
+constexpr uint32_t TM_S = 0, TM_X = 64;
+constexpr uint32_t ID_KM128x64 = idesc_f16(128, 64, false, true);
 constexpr uint32_t ID_MM128x64 = idesc_f16(128, 64, true, true);
 constexpr long long kWait = 2000000000LL;  // ~1 s of SM clocks per wait
 constexpr float kRange = 6.0e4f;           // largest operand magnitude kept in fp16
+static_assert(STAGE % 1024 == 0 && MISC % 1024 == 0, "alignment");
 }  // namespace tfwd
+
+__device__ __forceinline__ void named_sync(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
 
 __global__ void __launch_bounds__(tfwd::kThreads, 1)
 tc_fwd_kernel(const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mw,
@@ -73,7 +87,9 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mv, const __grid_constant__ CU
     const int vh = blockIdx.x, h = blockIdx.y, bb = blockIdx.z, v0 = vh * 64;
     const int NC = d.NC, T = d.T, H = d.H;
     const int quarter = warp & 3, half = warp >> 2;
-    const int key = quarter * 32 + lane;  // state row of this thread
+    const int key = quarter * 32 + lane;          // state row (TMEM lane) of this thread
+    const bool dwarp = quarter < 2;               // reads Delta (lanes 0..63), else O (64..127)
+    const int ot = (half * 2 + (quarter - 2)) * 32 + lane;  // 0..127 among the O warps
     const size_t bh = (size_t)bb * H + h;
     const unsigned char *recs = ws + lay.rec + bh * NC * (size_t)REC_BYTES;
 
@@ -85,33 +101,92 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mv, const __grid_constant__ CU
         for (int i = 0; i < 5; ++i) mbar_init(&bars[i], 1);
         mbar_fence_init();
     }
+    // zero tiles of both stages
+    for (int i = tid; i < 2 * 8192 / 16; i += kThreads)
+        *reinterpret_cast<uint4 *>(sm + STG + (i >> 9) * STAGE + S_Z + (i & 511) * 16) = make_uint4(0, 0, 0, 0);
+    fence_proxy_async();
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
     const uint32_t tm = *tslot;
 
-    int issued[3] = {0, 0, 0};  // loads requested per barrier (thread 0)
-    auto load_rec = [&](int cc) {
+    int issued[3] = {0, 0, 0};  // loads requested per barrier
+    int groups[2] = {0, 0};     // product groups 1 and 2 issued (thread 0)
+    auto load_rec = [&](int cc) {  // thread 0
         const int s = cc & 1;
+        unsigned char *dst = sm + STG + s * STAGE;
+        const unsigned char *src = recs + (size_t)cc * REC_BYTES;
         mbar_expect_tx(&bars[s], REC_BYTES);
-        bulk_load(sm + STG + s * REC_BYTES, recs + (size_t)cc * REC_BYTES, REC_BYTES, &bars[s]);
+        bulk_load(dst, src, REC_P, &bars[s]);                        // [-W; Qb], Kh, T
+        bulk_load(dst + S_P, src + REC_P, 8192, &bars[s]);           // P
+        bulk_load(dst + S_FAC, src + REC_FAC, REC_BYTES - REC_FAC, &bars[s]);
         ++issued[s];
     };
-    auto load_vw = [&](int cc) {
+    auto load_vw = [&](int cc) {  // thread 64
         mbar_expect_tx(&bars[2], 8192 + 16384);
         tma_load_4d(sm + RAW_V, &mv, v0, h, cc * 64, bb, &bars[2]);
         tma_load_4d(sm + RAW_W, &mw, v0, h, cc * 64, bb, &bars[2]);
         ++issued[2];
     };
+    // U = w.v of chunk cc into OP_U[cc & 1] (O warps: 4 rows x 8 columns each)
+    auto make_u = [&](int cc) {
+        const int jv = ot & 7;
+        unsigned char *dst = sm + OP_U + (cc & 1) * 8192;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int r = (ot >> 3) + 16 * i;
+            const uint4 vr = *reinterpret_cast<const uint4 *>(sm + RAW_V + r * 128 + jv * 16);
+            const float4 w0 = *reinterpret_cast<const float4 *>(sm + RAW_W + r * 256 + jv * 32);
+            const float4 w1 = *reinterpret_cast<const float4 *>(sm + RAW_W + r * 256 + jv * 32 + 16);
+            const __nv_bfloat162 *v2 = reinterpret_cast<const __nv_bfloat162 *>(&vr);
+            float u[8] = {w0.x * __low2float(v2[0]), w0.y * __high2float(v2[0]),
+                          w0.z * __low2float(v2[1]), w0.w * __high2float(v2[1]),
+                          w1.x * __low2float(v2[2]), w1.y * __high2float(v2[2]),
+                          w1.z * __low2float(v2[3]), w1.w * __high2float(v2[3])};
+            st_h8(dst + sw128_chunk(r, jv, 64), u);
+            big = absmax8(u, big);
+        }
+    };
+    // product group 1 of chunk cc (thread 0)
+    auto group1 = [&](int cc) {
+        const uint32_t st = smem_addr(sm + STG + (cc & 1) * STAGE);
+        const uint32_t x = tm + TM_X + 64 * (cc & 1);
+        const uint64_t dT = desc_kmajor(st + S_T, 128, 0),
+                       dU = desc_mnmajor(smem_addr(sm + OP_U + (cc & 1) * 8192), 64, 0),
+                       dW = desc_kmajor(st + S_WQ, 128, 0),
+                       dS = desc_mnmajor(smem_addr(sm + OP_S), 128, 0);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+            mma_bf16(x, kstep_kmajor(dT, 128, ks), kstep_mnmajor(dU, ks), ID_KM128x64, ks > 0);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+            mma_bf16(x, kstep_kmajor(dW, 128, ks), kstep_mnmajor(dS, ks), ID_KM128x64, 1);
+        mma_commit(&bars[3]);
+        ++groups[0];
+    };
+    auto ckpt = [&](int c) { return ws + lay.ckS + ((bh * (NC + 1) + c) * 2 + vh) * 16384; };
+    // O rows of chunk cc (O warps): accumulator rows 64..127, this warp's 32 columns
+    auto store_o = [&](int cc) {
+        float ov[32];
+        const uint32_t x = tm + TM_X + 64 * (cc & 1);
+        tmem_ld16(taddr(x, quarter * 32, 32 * half), ov);
+        tmem_ld16(taddr(x, quarter * 32, 32 * half + 16), ov + 16);
+        tmem_wait_ld();
+        const int t = cc * 64 + key - 64;
+        if (o && t < T) {
+            unsigned char *dst = reinterpret_cast<unsigned char *>(o + tok(d, bb, t, h, 128) + v0 + 32 * half);
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) st_bf16x8(dst + 16 * jj, ov + 8 * jj);
+        }
+    };
+
     if (tid == 0) {
         load_rec(0);
         if (NC > 1) load_rec(1);
-        load_vw(0);
     }
-    // state checkpoint c of this half: [128 key][64 v] fp16, true scale
-    auto ckpt = [&](int c) { return ws + lay.ckS + ((bh * (NC + 1) + c) * 2 + vh) * 16384; };
+    if (tid == 64) load_vw(0);
 
-    // initial state slice: S_m of chunk 0 into TMEM and OP_S; S0 itself to checkpoint 0
+    // ---------------- prologue: S_m of chunk 0 (TMEM, OP_S); U of chunk 0
     bool ok = mbar_wait(&bars[0], 0, kWait);
     {
         const size_t so = st_off(d, bb, h);
@@ -122,10 +197,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mv, const __grid_constant__ CU
                           : make_float4(0.f, 0.f, 0.f, 0.f);
             x[j] = t.x; x[j + 1] = t.y; x[j + 2] = t.z; x[j + 3] = t.w;
         }
-        if (keep)
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) st_h8(ckpt(0) + sw128_chunk(key, 4 * half + jj, 128), x + 8 * jj);
-        const float e = ok ? reinterpret_cast<const float *>(sm + STG + REC_FAC)[128 + key] : 0.f;
+        const float e = reinterpret_cast<const float *>(sm + STG + S_FAC)[128 + key];
 #pragma unroll
         for (int j = 0; j < 32; ++j) x[j] *= e;
         tmem_st16(taddr(tm + TM_S, quarter * 32, 32 * half), x);
@@ -137,129 +209,91 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mv, const __grid_constant__ CU
         }
         tmem_wait_st();
     }
+    if (!dwarp) {
+        ok = mbar_wait(&bars[2], 0, kWait) && ok;
+        make_u(0);
+        named_sync(2, 128);  // raw v, w consumed
+        if (tid == 64 && NC > 1) load_vw(1);
+    }
     fence_proxy_async();
     fence_before_sync();
     bool abort = __syncthreads_or(!ok);
+    if (tid == 0 && !abort) {
+        fence_after_sync();
+        if (keep) {
+            bulk_store(ckpt(0), sm + OP_S, 16384);
+            bulk_commit();
+        }
+        group1(0);
+    }
 
     for (int c = 0; c < NC && !abort; ++c) {
-        const int s = c & 1, c0 = c * 64;
+        const int s = c & 1;
         const uint32_t par = c & 1;
-        unsigned char *stg = sm + STG + s * REC_BYTES;
-        // ---------------- U = w.v for this half, then product group 1
-        ok = mbar_wait(&bars[s], (c >> 1) & 1, kWait);
-        ok = ok && mbar_wait(&bars[2], par, kWait);
-        const float gam = reinterpret_cast<const float *>(stg + REC_FAC)[key];  // e^(G_L - G_m)
-        {
-            const int r = tid >> 2, cg = tid & 3;  // row, 16-column group
-            const uint4 vr0 = *reinterpret_cast<const uint4 *>(sm + RAW_V + r * 128 + cg * 32);
-            const uint4 vr1 = *reinterpret_cast<const uint4 *>(sm + RAW_V + r * 128 + cg * 32 + 16);
-            const float4 *wr = reinterpret_cast<const float4 *>(sm + RAW_W + r * 256 + cg * 64);
-            const __nv_bfloat162 *va = reinterpret_cast<const __nv_bfloat162 *>(&vr0);
-            const __nv_bfloat162 *vb = reinterpret_cast<const __nv_bfloat162 *>(&vr1);
-            float u[16];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float4 w4 = wr[i];
-                const __nv_bfloat162 p0 = i < 2 ? va[2 * i] : vb[2 * i - 4];
-                const __nv_bfloat162 p1 = i < 2 ? va[2 * i + 1] : vb[2 * i - 3];
-                u[4 * i] = w4.x * __low2float(p0);
-                u[4 * i + 1] = w4.y * __high2float(p0);
-                u[4 * i + 2] = w4.z * __low2float(p1);
-                u[4 * i + 3] = w4.w * __high2float(p1);
-            }
-            st_h8(sm + OP_U + sw128_chunk(r, 2 * cg, 64), u);
-            st_h8(sm + OP_U + sw128_chunk(r, 2 * cg + 1, 64), u + 8);
-            big = absmax8(u, big);
-            big = absmax8(u + 8, big);
-        }
-        fence_proxy_async();
-        fence_before_sync();
-        if (__syncthreads_or(!ok)) { abort = true; break; }
-        if (tid == 0) {
+        unsigned char *stg = sm + STG + s * STAGE;
+        const uint32_t x = tm + TM_X + 64 * s;
+        if (dwarp) {
+            // ---------------- Delta rows to fp16
+            ok = mbar_wait(&bars[3], par, kWait);
             fence_after_sync();
-            if (c + 1 < NC) load_vw(c + 1);  // raw v and w consumed
-            const uint32_t st = smem_addr(stg), u = smem_addr(sm + OP_U), sS = smem_addr(sm + OP_S);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tm + TM_D, desc_kmajor(st + REC_T, 64, ks), desc_mnmajor(u, 64, ks), ID_KM64, ks > 0);
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-                mma_bf16(tm + TM_D, desc_kmajor(st + REC_WN, 64, ks), desc_mnmajor(sS, 128, ks), ID_KM64, 1);
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-                mma_bf16(tm + TM_O, desc_kmajor(st + REC_QB, 64, ks), desc_mnmajor(sS, 128, ks), ID_KM64, ks > 0);
-            mma_commit(&bars[3]);
-        }
-        // ---------------- Delta to fp16, product group 2
-        ok = mbar_wait(&bars[3], par, kWait);
-        fence_after_sync();
-        {
             float dl[32];
-            tmem_ld16(taddr(tm + TM_D, quarter * 32, 32 * half), dl);
-            tmem_ld16(taddr(tm + TM_D, quarter * 32, 32 * half + 16), dl + 16);
+            tmem_ld16(taddr(x, quarter * 32, 32 * half), dl);
+            tmem_ld16(taddr(x, quarter * 32, 32 * half + 16), dl + 16);
             tmem_wait_ld();
-            if (lane < 16) {
-                const int r = quarter * 16 + lane;
 #pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                    st_h8(sm + OP_D + sw128_chunk(r, 4 * half + jj, 64), dl + 8 * jj);
-                    big = absmax8(dl + 8 * jj, big);
+            for (int jj = 0; jj < 4; ++jj) {
+                st_h8(sm + OP_D + sw128_chunk(key, 4 * half + jj, 64), dl + 8 * jj);
+                big = absmax8(dl + 8 * jj, big);
+            }
+            fence_proxy_async();
+            fence_before_sync();
+            named_sync(1, 128);
+            if (tid == 0) {
+                fence_after_sync();
+                bulk_wait_read();  // the checkpoint copy has left OP_S
+                const uint32_t st = smem_addr(stg);
+                const uint64_t dZP = desc_kmajor(st + S_Z, 128, 0), dK = desc_mnmajor(st + S_KH, 64, 0),
+                               dD = desc_mnmajor(smem_addr(sm + OP_D), 64, 0);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16(x, kstep_kmajor(dZP, 128, ks), kstep_mnmajor(dD, ks), ID_KM128x64, 1);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16(tm + TM_S, kstep_mnmajor(dK, ks), kstep_mnmajor(dD, ks), ID_MM128x64, 1);
+                mma_commit(&bars[4]);
+                ++groups[1];
+                if (keep) {  // Delta of this chunk and half, for the backward
+                    bulk_store(ws + lay.ckD + ((bh * NC + c) * 2 + vh) * 8192, sm + OP_D, 8192);
+                    bulk_commit();
                 }
             }
-        }
-        fence_proxy_async();
-        fence_before_sync();
-        if (__syncthreads_or(!ok)) { abort = true; break; }
-        if (tid == 0) {
-            fence_after_sync();
-            if (keep) {  // Delta of this chunk and half, for the backward
-                bulk_store(ws + lay.ckD + ((bh * NC + c) * 2 + vh) * 8192, sm + OP_D, 8192);
-                bulk_commit();
+        } else {
+            // ---------------- previous chunk's O; next chunk's U
+            if (c > 0) store_o(c - 1);
+            if (c + 1 < NC) {
+                ok = mbar_wait(&bars[2], (c + 1) & 1, kWait) && ok;
+                make_u(c + 1);
+                fence_proxy_async();
+                named_sync(2, 128);  // raw v, w consumed
+                if (tid == 64 && c + 2 < NC) load_vw(c + 2);
             }
-            const uint32_t st = smem_addr(stg), dl = smem_addr(sm + OP_D);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tm + TM_O, desc_kmajor(st + REC_P, 64, ks), desc_mnmajor(dl, 64, ks), ID_KM64, 1);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tm + TM_S, desc_mnmajor(st + REC_KH, 64, ks), desc_mnmajor(dl, 64, ks), ID_MM128x64, 1);
-            mma_commit(&bars[4]);
         }
-        // ---------------- output rows; state into the next chunk's frame
-        ok = mbar_wait(&bars[4], par, kWait);
-        float ref = 1.f;  // e^G_m of the next chunk
+        // ---------------- state into the next chunk's frame
+        ok = mbar_wait(&bars[4], par, kWait) && ok;
+        const float gam = reinterpret_cast<const float *>(stg + S_FAC)[key];  // e^(G_L - G_m)
+        float ref = 1.f;                                                      // next e^G_m
         if (c + 1 < NC) {
-            ok = ok && mbar_wait(&bars[s ^ 1], ((c + 1) >> 1) & 1, kWait);
-            ref = reinterpret_cast<const float *>(sm + STG + (s ^ 1) * REC_BYTES + REC_FAC)[128 + key];
+            ok = mbar_wait(&bars[s ^ 1], ((c + 1) >> 1) & 1, kWait) && ok;
+            ref = reinterpret_cast<const float *>(sm + STG + (s ^ 1) * STAGE + S_FAC)[128 + key];
         }
         fence_after_sync();
         {
-            float ov[32], sv[32];
-            tmem_ld16(taddr(tm + TM_O, quarter * 32, 32 * half), ov);
-            tmem_ld16(taddr(tm + TM_O, quarter * 32, 32 * half + 16), ov + 16);
+            float sv[32];
             tmem_ld16(taddr(tm + TM_S, quarter * 32, 32 * half), sv);
             tmem_ld16(taddr(tm + TM_S, quarter * 32, 32 * half + 16), sv + 16);
             tmem_wait_ld();
-            if (lane < 16) {
-                const int r = quarter * 16 + lane;
-                if (o && c0 + r < T) {
-                    unsigned char *dst = reinterpret_cast<unsigned char *>(
-                        o + tok(d, bb, c0 + r, h, 128) + v0 + 32 * half);
-#pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) st_bf16x8(dst + 16 * jj, ov + 8 * jj);
-                }
-            }
 #pragma unroll
             for (int j = 0; j < 32; ++j) sv[j] *= gam;  // S_{c+1}, true scale
-            if (keep)
-#pragma unroll
-                for (int jj = 0; jj < 4; ++jj) st_h8(ckpt(c + 1) + sw128_chunk(key, 4 * half + jj, 128), sv + 8 * jj);
-            if (c == NC - 1 && ST) {
-                float *dst = ST + st_off(d, bb, h) + (size_t)key * 128 + v0 + 32 * half;
-#pragma unroll
-                for (int j = 0; j < 32; j += 4)
-                    *reinterpret_cast<float4 *>(dst + j) = make_float4(sv[j], sv[j + 1], sv[j + 2], sv[j + 3]);
-            }
             if (c + 1 < NC) {
 #pragma unroll
                 for (int j = 0; j < 32; ++j) sv[j] *= ref;  // S_m of the next chunk
@@ -271,23 +305,45 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mv, const __grid_constant__ CU
                     big = absmax8(sv + 8 * jj, big);
                 }
                 tmem_wait_st();
+            } else {
+                if (ST) {
+                    float *dst = ST + st_off(d, bb, h) + (size_t)key * 128 + v0 + 32 * half;
+#pragma unroll
+                    for (int j = 0; j < 32; j += 4)
+                        *reinterpret_cast<float4 *>(dst + j) = make_float4(sv[j], sv[j + 1], sv[j + 2], sv[j + 3]);
+                }
+                if (keep)
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) st_h8(ckpt(NC) + sw128_chunk(key, 4 * half + jj, 128), sv + 8 * jj);
             }
         }
-        if (tid == 0 && keep) bulk_wait_read();  // the Delta copy reads OP_D, rewritten next chunk
+        if (tid == 0) bulk_wait_read();  // the Delta copy has left OP_D
         fence_proxy_async();
         fence_before_sync();
         if (__syncthreads_or(!ok)) { abort = true; break; }
-        if (tid == 0 && c + 2 < NC) load_rec(c + 2);  // this stage's record is consumed
-    }
-    if (!(big <= kRange)) record_status(status, GDN2_ERR_RANGE);
-    if (tid == 0) {
-        bulk_wait_all();
-        if (abort) {
-            record_status(status, GDN2_ERR_TIMEOUT);
-            // let every requested copy land before the CTA's shared memory goes away
-            for (int i = 0; i < 3; ++i)
-                if (issued[i] > 0) mbar_wait(&bars[i], (issued[i] - 1) & 1, kWait);
+        if (tid == 0) {
+            fence_after_sync();
+            if (c + 2 < NC) load_rec(c + 2);  // this stage's record is consumed
+            if (c + 1 < NC) {
+                if (keep) {
+                    bulk_store(ckpt(c + 1), sm + OP_S, 16384);
+                    bulk_commit();
+                }
+                group1(c + 1);
+            }
         }
+    }
+    if (!abort && !dwarp) store_o(NC - 1);
+    if (!(big <= kRange)) record_status(status, GDN2_ERR_RANGE);
+    if (tid == 0) bulk_wait_all();
+    if (abort && (tid == 0 || tid == 64)) {
+        if (tid == 0) record_status(status, GDN2_ERR_TIMEOUT);
+        // let every requested copy land before the CTA's shared memory goes away
+        for (int i = 0; i < 3; ++i)
+            if (issued[i] > 0) mbar_wait(&bars[i], (issued[i] - 1) & 1, kWait);
+        // and every issued product finish before the tensor memory is freed
+        for (int i = 0; i < 2; ++i)
+            if (groups[i] > 0) mbar_wait(&bars[3 + i], (groups[i] - 1) & 1, kWait);
     }
     fence_before_sync();
     __syncthreads();

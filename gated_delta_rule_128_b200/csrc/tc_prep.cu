@@ -13,7 +13,8 @@
 // The kernel writes Qb, Kh, -W, T, P and the per-channel factors
 // e^(G_L - G_m), e^G_m to the chunk's record in the workspace (layout REC_*
 // in common.cuh); the sequential state kernel (tc_fwd.cu) and the backward
-// read them from there.
+// read them from there.  Kc and Qb share one [128][128] tile (Kc on top), so
+// that A and P come out of one M = 128 product: [Kc; Qb] Kh^T.
 //
 // Persistent: one CTA per SM walks the (b, h, chunk) tiles with a stride of
 // the grid size.  TMA brings the raw q, k, g, b tiles; as soon as the
@@ -35,16 +36,16 @@ namespace tprep {
 constexpr int kThreads = 256;
 constexpr uint32_t RAW_Q = 0, RAW_K = 16384, RAW_G = 32768, RAW_B = 65536;
 constexpr uint32_t REC = 98304;  // the tile's record, laid out as in the workspace
-constexpr uint32_t OP_QB = REC + REC_QB, OP_KH = REC + REC_KH;
-constexpr uint32_t OP_KC = REC + REC_WN;  // Kc, later -W
+constexpr uint32_t OP_WQ = REC + REC_WQ;  // [Kc; Qb], later [-W; Qb]
+constexpr uint32_t OP_KH = REC + REC_KH;
 constexpr uint32_t OP_T = REC + REC_T, OP_P = REC + REC_P, FAC = REC + REC_FAC;
 constexpr uint32_t SCR = REC + REC_BYTES;  // float32 scratch of the inversion
 constexpr uint32_t SCR_A = SCR, SCR_T = SCR + 64 * 65 * 4, SCR_M = SCR_T + 64 * 65 * 4;
 constexpr uint32_t SCR_SCAN = SCR;  // per-warp cumsum totals [8][128] f32, before the inversion
 constexpr uint32_t MISC = SCR_M + 8 * 16 * 9 * 4;  // mbarriers, TMEM slot
 constexpr uint32_t SMEM_BYTES = MISC + 128 + 1024;
-constexpr uint32_t TM_A = 0, TM_P = 64, TM_W = 128;  // 256 columns
-constexpr uint32_t ID_KK64 = idesc_f16(64, 64, false, false);
+constexpr uint32_t TM_AP = 0, TM_W = 128;  // [A; P] (M = 128), W; 256 columns
+constexpr uint32_t ID_KK128x64 = idesc_f16(128, 64, false, false);
 constexpr uint32_t ID_KM128 = idesc_f16(64, 128, false, true);
 constexpr long long kWait = 2000000000LL;  // ~1 s of SM clocks per wait
 constexpr float kRange = 6.0e4f;
@@ -196,24 +197,19 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
         if (tid == 0) bulk_wait_read();  // the previous tile's record has left shared memory
         if (__syncthreads_or(!ok)) { abort = true; break; }
         cumsum_finish(reinterpret_cast<const float *>(sm + SCR_SCAN), warp, lane, G, sGam, sRef);
-        gbig = fmaxf(gbig, write_factors(sm + RAW_Q, sm + RAW_K, reinterpret_cast<const float *>(sm + RAW_B),
-                                       G, sm + OP_QB, sm + OP_KC, sm + OP_KH, warp, lane));
+        gbig = fmaxf(gbig, write_factors_rec(sm + RAW_Q, sm + RAW_K, reinterpret_cast<const float *>(sm + RAW_B),
+                                           G, sm + OP_WQ, sm + OP_KH, warp, lane));
         fence_proxy_async();
         fence_before_sync();
         __syncthreads();
         if (tid == 0) {
             fence_after_sync();
             if (it + (int)gridDim.x < ntiles) load_raw(it + gridDim.x);  // raw tiles consumed
-            bulk_store(rec + REC_QB, sm + OP_QB, 32768);                  // Qb, Kh
-            bulk_commit();
-            const uint32_t kc = smem_addr(sm + OP_KC), qb = smem_addr(sm + OP_QB),
-                           kh = smem_addr(sm + OP_KH);
+            const uint64_t kq = desc_kmajor(smem_addr(sm + OP_WQ), 128, 0),
+                           kh = desc_kmajor(smem_addr(sm + OP_KH), 64, 0);
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks)
-                mma_bf16(tm + TM_A, desc_kmajor(kc, 64, ks), desc_kmajor(kh, 64, ks), ID_KK64, ks > 0);
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-                mma_bf16(tm + TM_P, desc_kmajor(qb, 64, ks), desc_kmajor(kh, 64, ks), ID_KK64, ks > 0);
+                mma_bf16(tm + TM_AP, kstep_kmajor(kq, 128, ks), kstep_kmajor(kh, 64, ks), ID_KK128x64, ks > 0);
             mma_commit(&bars[1]);
         }
         // ---------------- strictly-lower A to float32, masked P to fp16; T = (I + A)^-1
@@ -222,24 +218,24 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
         float *sA = reinterpret_cast<float *>(sm + SCR_A);
         float *sT = reinterpret_cast<float *>(sm + SCR_T);
         {
-            float row[64];
-            const uint32_t base = warp < 4 ? tm + TM_A : tm + TM_P;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) tmem_ld16(taddr(base, quarter * 32, 16 * j), row + 16 * j);
+            // accumulator row quarter * 32 + lane: rows 0..63 are A, 64..127 are P;
+            // this warp's 32 columns start at 32 * half
+            float row[32];
+            tmem_ld16(taddr(tm + TM_AP, quarter * 32, 32 * half), row);
+            tmem_ld16(taddr(tm + TM_AP, quarter * 32, 32 * half + 16), row + 16);
             tmem_wait_ld();
-            if (lane < 16) {
-                const int r = quarter * 16 + lane;
-                if (warp < 4) {
+            if (quarter < 2) {
+                const int r = quarter * 32 + lane;
 #pragma unroll
-                    for (int j = 0; j < 64; ++j) sA[r * 65 + j] = j < r ? row[j] : 0.f;
-                } else {
+                for (int j = 0; j < 32; ++j) sA[r * 65 + 32 * half + j] = 32 * half + j < r ? row[j] : 0.f;
+            } else {
+                const int r = quarter * 32 + lane - 64;
 #pragma unroll
-                    for (int j = 0; j < 64; ++j) row[j] = j <= r ? row[j] : 0.f;
+                for (int j = 0; j < 32; ++j) row[j] = 32 * half + j <= r ? row[j] : 0.f;
 #pragma unroll
-                    for (int jj = 0; jj < 8; ++jj) {
-                        st_h8(sm + OP_P + sw128_chunk(r, jj, 64), row + 8 * jj);
-                        big = absmax8(row + 8 * jj, big);
-                    }
+                for (int jj = 0; jj < 4; ++jj) {
+                    st_h8(sm + OP_P + sw128_chunk(r, 4 * half + jj, 64), row + 8 * jj);
+                    big = absmax8(row + 8 * jj, big);
                 }
             }
         }
@@ -255,13 +251,16 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
         __syncthreads();
         if (tid == 0) {
             fence_after_sync();
-            const uint32_t t = smem_addr(sm + OP_T), kc = smem_addr(sm + OP_KC);
+            // Kc (rows 0..63 of the [Kc; Qb] tile) as the MN-major B: its two
+            // 64-key blocks lie 16 KB apart
+            const uint64_t t = desc_kmajor(smem_addr(sm + OP_T), 64, 0),
+                           kc = desc_mnmajor_lbo(smem_addr(sm + OP_WQ), 16384, 0);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tm + TM_W, desc_kmajor(t, 64, ks), desc_mnmajor(kc, 64, ks), ID_KM128, ks > 0);
+                mma_bf16(tm + TM_W, kstep_kmajor(t, 64, ks), kstep_mnmajor(kc, ks), ID_KM128, ks > 0);
             mma_commit(&bars[1]);
         }
-        // ---------------- -W to fp16 (over Kc, consumed by the product)
+        // ---------------- -W to fp16 (over Kc, consumed by the product); the record
         ok = mbar_wait(&bars[1], 1, kWait);
         fence_after_sync();
         {
@@ -275,7 +274,7 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
                 for (int j = 0; j < 64; ++j) wv[j] = -wv[j];
 #pragma unroll
                 for (int jj = 0; jj < 8; ++jj) {
-                    st_h8(sm + OP_KC + sw128_chunk(r, 8 * half + jj, 64), wv + 8 * jj);
+                    st_h8(sm + OP_WQ + sw128_chunk(r, 8 * half + jj, 128), wv + 8 * jj);
                     big = absmax8(wv + 8 * jj, big);
                 }
             }
@@ -285,7 +284,7 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
         if (__syncthreads_or(!ok)) { abort = true; break; }
         if (tid == 0) {
             fence_after_sync();
-            bulk_store(rec + REC_WN, sm + OP_KC, REC_BYTES - REC_WN);  // -W, T, P, factors
+            bulk_store(rec, sm + REC, REC_BYTES);
             bulk_commit();
         }
     }

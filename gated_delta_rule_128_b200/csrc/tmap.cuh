@@ -31,9 +31,12 @@ inline EncodeTiledFn encode_fn() {
 // Map of a contiguous [B, T, H, D] tensor whose box is `rows` consecutive
 // tokens x `cols` channels (starting at a channel multiple of cols) of one
 // (b, h).  Coordinates (innermost first): {channel, h, t, b}.  Rows past T
-// read as zero.  Returns false if the driver refuses the map.
+// read as zero and are not written by stores.  With swizzle128 the box's
+// rows (cols x element size = 128 bytes) land in shared memory with their
+// 16-byte chunks XOR-ed by (row % 8), the layout of tc.cuh's sw128 tiles.
+// Returns false if the driver refuses the map.
 inline bool make_btHd_map(CUtensorMap *map, const void *base, bool bf16, int B, int T, int H,
-                          int D, int rows, int cols) {
+                          int D, int rows, int cols, bool swizzle128 = false) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t es = bf16 ? 2 : 4;
@@ -43,7 +46,8 @@ inline bool make_btHd_map(CUtensorMap *map, const void *base, bool bf16, int B, 
     cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
                     4, const_cast<void *>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
