@@ -170,6 +170,11 @@ __device__ __forceinline__ uint32_t taddr(uint32_t base, int lane, int col) {
     return base + ((uint32_t)lane << 16) + (uint32_t)col;
 }
 
+// barrier `id` (1..15) among `nthreads` threads (whole warps) of the CTA
+__device__ __forceinline__ void named_sync(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 // ---- mbarriers
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)

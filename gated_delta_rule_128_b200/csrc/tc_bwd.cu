@@ -420,19 +420,24 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
 
 // ============================================================ chunk kernel
 namespace tbg {
-constexpr int kThreads = 256;
-constexpr uint32_t RAW_Q = 0, RAW_K = 16384, RAW_B = 32768, RAW_G = 65536;  // g, later G - G_m
-constexpr uint32_t OP_DO = 98304;     // dO fp16 [64 pos][128 v] K-major (in place of raw dO)
-constexpr uint32_t BL_S = 114688;     // S_m [128 key][128 v] K-major B (the checkpoint; later Qb, Kc, Kh; then dG)
-constexpr uint32_t BL_DS = 147456;    // dS_m [128 key][128 v]
-constexpr uint32_t BL_D = 180224;     // Delta [64 pos][128 v]              (later dP, dA)
-constexpr uint32_t BL_NDU = 196608;   // -dU [64 pos][128 v]
-constexpr uint32_t OP_QB = BL_S, OP_KC = BL_S + 16384, OP_KH = BL_S + 32768;
-constexpr uint32_t OP_DP = BL_D, OP_DA = BL_D + 8192;
-constexpr uint32_t MISC = 212992;     // sGam, sRef [128]; sEnd [128]; scan [8][128]; mbarriers; slot
-constexpr uint32_t SMEM_BYTES = MISC + 1536 + 4096 + 128 + 1024;
-constexpr uint32_t TM_DP = 0, TM_DA = 64, TM_Y1 = 128, TM_Y2 = 256, TM_Y3 = 384;
-constexpr uint32_t ID_KK64 = idesc_f16(64, 64, false, false);
+constexpr int kCompute = 512;             // warps 0..15 form operands and outputs
+constexpr int kThreads = kCompute + 32;   // warp 16 issues the copies and products
+constexpr int kWarps = kCompute / 32;
+constexpr uint32_t RQ = 0;        // q: two 128-B swizzled [64][64] bf16 boxes; Qb, then dq, in place
+constexpr uint32_t RK = 16384;    // k (bf16); dk in place
+constexpr uint32_t RB = 32768;    // b: four [64][32] f32 boxes; db in place
+constexpr uint32_t RG = 65536;    // g (f32); G - G_m, then dG, then dg in place
+constexpr uint32_t DN = 98304;    // [dO; -dU] [128][128] K-major (K-blocks of 16 KB)
+constexpr uint32_t DL = 131072;   // Delta [64 pos][128 v] K-major
+constexpr uint32_t SMT = 147456;  // S_m [128 key][128 v] K-major (then Kh, Kc)
+constexpr uint32_t DXT = 180224;  // dX  [128 key][128 v] K-major (then [dP; dA])
+constexpr uint32_t KH = SMT, KC = SMT + 16384, PA = DXT;  // after the first products
+constexpr uint32_t TE = DXT + 16384, TEI = DL;              // E = e^(G - G_m), 1/E (fp16 [64][128])
+constexpr uint32_t MISC = 212992; // sEnd [128]; sRef [128]; scan [16][128]; mbarriers; slot
+constexpr uint32_t SMEM_BYTES = MISC + 1024 + 8192 + 128 + 1024;
+constexpr uint32_t LOAD_BYTES = 212992;
+constexpr uint32_t TM_Y1 = 0, TM_Y2 = 128, TM_Y3 = 256, TM_PA = 384;  // 512 columns
+constexpr uint32_t ID_PA = idesc_f16(128, 64, false, false);
 constexpr uint32_t ID_KK128 = idesc_f16(64, 128, false, false);
 constexpr uint32_t ID_KM128 = idesc_f16(64, 128, false, true);
 constexpr uint32_t ID_MM128 = idesc_f16(64, 128, true, true);
@@ -440,36 +445,57 @@ constexpr long long kWait = 2000000000LL;
 constexpr float kRange = 6.0e4f;
 }  // namespace tbg
 
+// descriptor of K step kstep of a K-major operand whose 64-wide K-blocks lie
+// blk bytes apart (d0 = its K step 0)
+__device__ __forceinline__ uint64_t kstep_kmajor_blk(uint64_t d0, uint32_t blk, int kstep) {
+    return d0 + (uint64_t)((((uint32_t)(kstep >> 2) * blk) + (kstep & 3) * 32) >> 4);
+}
+
+// One CTA per (b, h, chunk), all chunks in parallel, full d_v.  Warp 16
+// loads the tile (raw q, k, b, g, dO as 128-B swizzled TMA boxes; S_m, dX,
+// Delta, -dU from the workspace) and issues the products; warps 0..15 form
+// the operands and the outputs:
+//   (1) [dP; dA] = [dO; -dU] Delta^T (M = 128), Y1 = dO S_m^T, Y2 = -dU S_m^T,
+//       Y3 = Delta dX^T, while the decay factors Qb (in place of q), Kc, Kh
+//       are formed
+//   (2) Y1 += dP Kh, Y2 += dA Kh, Y3 += dP^T Qb + dA^T Kc (masked dP, dA)
+// then, per (row, channel) straight from tensor memory: dq = Y1.E,
+// db = Y2.E.k, dk = Y2.E.b + Y3/E, dG = Y1.Qb + Y2.Kc - Y3.Kh, written in
+// place of q, k, b, g; dg is the reverse in-chunk cumsum of dG plus the
+// chunk-end term, and the four tiles leave by TMA stores.  Sixteen compute
+// warps (four rows each in the row-wise phases) hide the latency of the
+// per-element work; E and 1/E are kept as fp16 tiles between the factor
+// phase and the outputs.
 __global__ void __launch_bounds__(tbg::kThreads, 1)
 tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
-                   const __grid_constant__ CUtensorMap mdo, const __grid_constant__ CUtensorMap mg,
-                   const __grid_constant__ CUtensorMap mb, __nv_bfloat16 *__restrict__ dqout,
-                   __nv_bfloat16 *__restrict__ dkout, float *__restrict__ dbout,
-                   float *__restrict__ dgout, unsigned char *__restrict__ ws, TcWs lay,
+                   const __grid_constant__ CUtensorMap mb, const __grid_constant__ CUtensorMap mg,
+                   const __grid_constant__ CUtensorMap mdo, const __grid_constant__ CUtensorMap mdq,
+                   const __grid_constant__ CUtensorMap mdk, const __grid_constant__ CUtensorMap mdb,
+                   const __grid_constant__ CUtensorMap mdg, unsigned char *__restrict__ ws, TcWs lay,
                    unsigned int *status, Dims d) {
     using namespace tbg;
     extern __shared__ unsigned char smraw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smraw) + 1023) & ~static_cast<uintptr_t>(1023));
-    float *sGam = reinterpret_cast<float *>(sm + MISC);
-    float *sRef = reinterpret_cast<float *>(sm + MISC + 512);
-    float *sEnd = reinterpret_cast<float *>(sm + MISC + 1024);
-    float *scan = reinterpret_cast<float *>(sm + MISC + 1536);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + MISC + 1536 + 4096);
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + MISC + 1536 + 4096 + 64);
+    float *sEnd = reinterpret_cast<float *>(sm + MISC);        // chunk-end term per channel
+    float *sRef = reinterpret_cast<float *>(sm + MISC + 512);  // G of the middle row per channel
+    float *scan = reinterpret_cast<float *>(sm + MISC + 1024);  // per-warp totals [16][128]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + MISC + 1024 + 8192);  // 0 loads, 1, 2 products
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + MISC + 1024 + 8192 + 64);
     float big = 0.f, gbig = 0.f;  // range checks: operand magnitude, |G - G_m|
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int c = blockIdx.x, h = blockIdx.y, bb = blockIdx.z, c0 = c * 64;
-    const int NC = d.NC, T = d.T, H = d.H, L = min(64, T - c0);
-    const int quarter = warp & 3, half = warp >> 2;
+    const int NC = d.NC, H = d.H;
+    const int quarter = warp & 3, cgrp = (warp >> 2) & 3;  // TMEM lane quarter; column group
     const size_t bh = (size_t)bb * H + h;
+    const bool compute = warp < kWarps, issuer = tid == kCompute;
 
     if (warp == 0) {
         tmem_alloc(tslot, 512);
         tmem_relinquish();
     }
-    if (tid == 0) {
+    if (issuer) {
         for (int i = 0; i < 3; ++i) mbar_init(&bars[i], 1);
         mbar_fence_init();
     }
@@ -478,201 +504,302 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
     fence_after_sync();
     const uint32_t tm = *tslot;
 
-    if (tid == 0) {
-        mbar_expect_tx(&bars[0], 16384 * 2 + 32768 * 2 + 16384 + 32768 * 2 + 16384 * 2);
-        tma_load_4d(sm + RAW_Q, &mq, 0, h, c0, bb, &bars[0]);
-        tma_load_4d(sm + RAW_K, &mk, 0, h, c0, bb, &bars[0]);
-        tma_load_4d(sm + RAW_B, &mb, 0, h, c0, bb, &bars[0]);
-        tma_load_4d(sm + RAW_G, &mg, 0, h, c0, bb, &bars[0]);
-        tma_load_4d(sm + OP_DO, &mdo, 0, h, c0, bb, &bars[0]);
-        bulk_load(sm + BL_S, ws + lay.ckS + ((bh * (NC + 1) + c) * 2) * 16384, 32768, &bars[0]);
-        bulk_load(sm + BL_DS, ws + lay.ckdS + ((bh * NC + c) * 2) * 16384, 32768, &bars[0]);
-        bulk_load(sm + BL_D, ws + lay.ckD + ((bh * NC + c) * 2) * 8192, 16384, &bars[0]);
-        bulk_load(sm + BL_NDU, ws + lay.ckndU + ((bh * NC + c) * 2) * 8192, 16384, &bars[0]);
+    if (issuer) {
+        mbar_expect_tx(&bars[0], LOAD_BYTES);
+        for (int x = 0; x < 2; ++x) {
+            tma_load_4d(sm + RQ + x * 8192, &mq, 64 * x, h, c0, bb, &bars[0]);
+            tma_load_4d(sm + RK + x * 8192, &mk, 64 * x, h, c0, bb, &bars[0]);
+            tma_load_4d(sm + DN + x * 16384, &mdo, 64 * x, h, c0, bb, &bars[0]);
+            bulk_load(sm + DN + x * 16384 + 8192, ws + lay.ckndU + ((bh * NC + c) * 2 + x) * 8192, 8192,
+                      &bars[0]);
+        }
+        for (int x = 0; x < 4; ++x) {
+            tma_load_4d(sm + RB + x * 8192, &mb, 32 * x, h, c0, bb, &bars[0]);
+            tma_load_4d(sm + RG + x * 8192, &mg, 32 * x, h, c0, bb, &bars[0]);
+        }
+        bulk_load(sm + DL, ws + lay.ckD + ((bh * NC + c) * 2) * 8192, 16384, &bars[0]);
+        bulk_load(sm + SMT, ws + lay.ckS + ((bh * (NC + 1) + c) * 2) * 16384, 32768, &bars[0]);
+        bulk_load(sm + DXT, ws + lay.ckdS + ((bh * NC + c) * 2) * 16384, 32768, &bars[0]);
     }
     if (tid < 128) {
         const float *e0 = reinterpret_cast<const float *>(ws + lay.ckEnd + ((bh * NC + c) * 2) * 512);
         sEnd[tid] = e0[tid] + e0[128 + tid];
     }
     bool ok = mbar_wait(&bars[0], 0, kWait);
-    // ---------------- G1: decay, dO operand; five products (the checkpoint holds S_m)
-    float G[8][4];
-    cumsum_local(reinterpret_cast<const float *>(sm + RAW_G), scan, warp, lane, G);
-    // dO: raw bf16 rows [64][128] -> fp16 K-major tile in place (values held in registers)
-    uint2 dor[8];
+
+    // ---------------- cumulative decay (rows 4w..4w+3, channels 4l..4l+3); dO to fp16
+    float G[4][4];
+    if (compute) {
+        float run[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int m = 0; m < 8; ++m) dor[m] = *reinterpret_cast<const uint2 *>(sm + OP_DO + (8 * warp + m) * 256 + lane * 8);
-    bool abort = __syncthreads_or(!ok);
-    if (!abort) {
-        cumsum_finish(scan, warp, lane, G, sGam, sRef);
-        float *sG = reinterpret_cast<float *>(sm + RAW_G);
+        for (int m = 0; m < 4; ++m) {
+            const float4 t = *reinterpret_cast<const float4 *>(sm + RG + sw128_chunk(4 * warp + m, lane, 64));
+            run[0] += t.x; run[1] += t.y; run[2] += t.z; run[3] += t.w;
 #pragma unroll
-        for (int m = 0; m < 8; ++m) {
-            const int r = 8 * warp + m;
-            *reinterpret_cast<float4 *>(sG + r * 128 + 4 * lane) = make_float4(G[m][0], G[m][1], G[m][2], G[m][3]);
-            const __nv_bfloat162 *d2 = reinterpret_cast<const __nv_bfloat162 *>(&dor[m]);
-            st_h4(sm + OP_DO + sw128_off(r, 4 * lane, 64), __low2float(d2[0]), __high2float(d2[0]),
-                  __low2float(d2[1]), __high2float(d2[1]));
+            for (int i = 0; i < 4; ++i) G[m][i] = run[i];
         }
-        fence_proxy_async();
-        fence_before_sync();
-        __syncthreads();
-        if (tid == 0) {
-            fence_after_sync();
-            const uint64_t dO = desc_kmajor(smem_addr(sm + OP_DO), 64, 0),
-                           S = desc_kmajor(smem_addr(sm + BL_S), 128, 0),
-                           DS = desc_kmajor(smem_addr(sm + BL_DS), 128, 0),
-                           D = desc_kmajor(smem_addr(sm + BL_D), 64, 0),
-                           NDU = desc_kmajor(smem_addr(sm + BL_NDU), 64, 0);
+        *reinterpret_cast<float4 *>(scan + warp * 128 + 4 * lane) = make_float4(run[0], run[1], run[2], run[3]);
+        named_sync(1, kCompute);
+        if (tid < 128) {  // per channel: exclusive prefix over the warps' totals, in place
+            float acc = 0.f;
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint64_t a_do = kstep_kmajor(dO, 64, ks), a_ndu = kstep_kmajor(NDU, 64, ks),
-                               a_d = kstep_kmajor(D, 64, ks), b_s = kstep_kmajor(S, 128, ks);
-                mma_bf16(tm + TM_DP, a_do, a_d, ID_KK64, ks > 0);
-                mma_bf16(tm + TM_DA, a_ndu, a_d, ID_KK64, ks > 0);
-                mma_bf16(tm + TM_Y1, a_do, b_s, ID_KK128, ks > 0);
-                mma_bf16(tm + TM_Y2, a_ndu, b_s, ID_KK128, ks > 0);
-                mma_bf16(tm + TM_Y3, a_d, kstep_kmajor(DS, 128, ks), ID_KK128, ks > 0);
-            }
-            mma_commit(&bars[1]);
-        }
-        // ---------------- G2: masked dP, dA; Qb, Kc, Kh; three accumulations
-        ok = mbar_wait(&bars[1], 0, kWait);
-        fence_after_sync();
-        {
-            float row[64];
-            const uint32_t base = warp < 4 ? tm + TM_DP : tm + TM_DA;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) tmem_ld16(taddr(base, quarter * 32, 16 * j), row + 16 * j);
-            tmem_wait_ld();
-            if (lane < 16) {
-                const int r = quarter * 16 + lane;
-                // dP keeps j <= r; dA = -strictly-lower(dU Delta^T) = strictly-lower of (-dU) Delta^T
-#pragma unroll
-                for (int j = 0; j < 64; ++j) row[j] = (warp < 4 ? j <= r : j < r) ? row[j] : 0.f;
-                unsigned char *dst = sm + (warp < 4 ? OP_DP : OP_DA);
-#pragma unroll
-                for (int jj = 0; jj < 8; ++jj) {
-                    st_h8(dst + sw128_chunk(r, jj, 64), row + 8 * jj);
-                    big = absmax8(row + 8 * jj, big);
-                }
+            for (int w2 = 0; w2 < kWarps; ++w2) {
+                const float t = scan[w2 * 128 + tid];
+                scan[w2 * 128 + tid] = acc;
+                acc += t;
+                if (w2 == kWarps / 2 - 1) sRef[tid] = acc;  // rows 0..31: G of the middle row
             }
         }
-        gbig = fmaxf(gbig, write_factors(sm + RAW_Q, sm + RAW_K, reinterpret_cast<const float *>(sm + RAW_B),
-                                       G, sm + OP_QB, sm + OP_KC, sm + OP_KH, warp, lane));
-        fence_proxy_async();
-        fence_before_sync();
-        abort = __syncthreads_or(!ok);
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {  // the dO rows of [dO; -dU], in place
+            const int i = tid + kCompute * m;
+            unsigned char *p = sm + DN + (i >> 9) * 16384 + (i & 511) * 16;
+            uint4 raw = *reinterpret_cast<const uint4 *>(p);
+            const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+            float x[8];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                x[2 * e] = __low2float(b2[e]);
+                x[2 * e + 1] = __high2float(b2[e]);
+            }
+            st_h8(p, x);
+        }
     }
-    if (!abort) {
-        if (tid == 0) {
-            fence_after_sync();
-            const uint32_t dP = smem_addr(sm + OP_DP), dA = smem_addr(sm + OP_DA);
-            const uint64_t kP = desc_kmajor(dP, 64, 0), kA = desc_kmajor(dA, 64, 0),
-                           mP = desc_mnmajor(dP, 64, 0), mA = desc_mnmajor(dA, 64, 0),
-                           qb = desc_mnmajor(smem_addr(sm + OP_QB), 64, 0),
-                           kc = desc_mnmajor(smem_addr(sm + OP_KC), 64, 0),
-                           kh = desc_mnmajor(smem_addr(sm + OP_KH), 64, 0);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-                const uint64_t b_kh = kstep_mnmajor(kh, ks);
-                mma_bf16(tm + TM_Y1, kstep_kmajor(kP, 64, ks), b_kh, ID_KM128, 1);
-                mma_bf16(tm + TM_Y2, kstep_kmajor(kA, 64, ks), b_kh, ID_KM128, 1);
-                mma_bf16(tm + TM_Y3, kstep_mnmajor(mP, ks), kstep_mnmajor(qb, ks), ID_MM128, 1);
-                mma_bf16(tm + TM_Y3, kstep_mnmajor(mA, ks), kstep_mnmajor(kc, ks), ID_MM128, 1);
-            }
-            mma_commit(&bars[2]);
-        }
-        // ---------------- G3: dq, dk, db and dG per (row, channel)
-        // The three accumulators go through shared memory (YS, [3][64][128]
-        // f32 with 16-byte chunks XOR-swizzled by row) so that every warp then
-        // walks whole rows with lanes across channels: conflict-free reads and
-        // coalesced output rows.
-        ok = mbar_wait(&bars[2], 0, kWait);
+    fence_proxy_async();
+    fence_before_sync();
+    ok = !__syncthreads_or(!ok);
+    if (issuer) {
         fence_after_sync();
-        float *YS = reinterpret_cast<float *>(sm + BL_S);  // operands of G2 are consumed
+        const uint64_t dn = desc_kmajor(smem_addr(sm + DN), 128, 0), dl = desc_kmajor(smem_addr(sm + DL), 64, 0),
+                       s = desc_kmajor(smem_addr(sm + SMT), 128, 0), dx = desc_kmajor(smem_addr(sm + DXT), 128, 0),
+                       ado = desc_kmajor(smem_addr(sm + DN), 64, 0), andu = desc_kmajor(smem_addr(sm + DN + 8192), 64, 0);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            const uint64_t b_s = kstep_kmajor(s, 128, ks), a_dl = kstep_kmajor(dl, 64, ks);
+            mma_bf16(tm + TM_PA, kstep_kmajor(dn, 128, ks), a_dl, ID_PA, ks > 0);
+            mma_bf16(tm + TM_Y1, kstep_kmajor_blk(ado, 16384, ks), b_s, ID_KK128, ks > 0);
+            mma_bf16(tm + TM_Y2, kstep_kmajor_blk(andu, 16384, ks), b_s, ID_KK128, ks > 0);
+            mma_bf16(tm + TM_Y3, a_dl, kstep_kmajor(dx, 128, ks), ID_KK128, ks > 0);
+        }
+        mma_commit(&bars[1]);
+    }
+    // ---------------- decay factors while the products run: Qb in place of q;
+    // Kh, Kc kept in registers until S_m is consumed
+    uint2 khr[4], kcr[4], er[4], eir[4];
+    if (compute) {
+        const float4 pre4 = *reinterpret_cast<const float4 *>(scan + warp * 128 + 4 * lane);
+        const float4 ref4 = *reinterpret_cast<const float4 *>(sRef + 4 * lane);
+        const float pre[4] = {pre4.x, pre4.y, pre4.z, pre4.w}, ref[4] = {ref4.x, ref4.y, ref4.z, ref4.w};
+        uint2 qr[4], kr[4];
+        float4 bv[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {  // every input row before the first store
+            const int r = 4 * warp + m;
+            qr[m] = *reinterpret_cast<const uint2 *>(sm + RQ + sw128_chunk(r, lane >> 1, 64) + (lane & 1) * 8);
+            kr[m] = *reinterpret_cast<const uint2 *>(sm + RK + sw128_chunk(r, lane >> 1, 64) + (lane & 1) * 8);
+            bv[m] = *reinterpret_cast<const float4 *>(sm + RB + sw128_chunk(r, lane, 64));
+        }
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const int r = 4 * warp + m;
+            float Gv[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                Gv[i] = G[m][i] + pre[i] - ref[i];
+                gbig = fmaxf(gbig, fabsf(Gv[i]));
+            }
+            const __nv_bfloat162 *q2 = reinterpret_cast<const __nv_bfloat162 *>(&qr[m]);
+            const __nv_bfloat162 *k2 = reinterpret_cast<const __nv_bfloat162 *>(&kr[m]);
+            const float qf[4] = {__low2float(q2[0]), __high2float(q2[0]), __low2float(q2[1]), __high2float(q2[1])};
+            const float kf[4] = {__low2float(k2[0]), __high2float(k2[0]), __low2float(k2[1]), __high2float(k2[1])};
+            const float bf[4] = {bv[m].x, bv[m].y, bv[m].z, bv[m].w};
+            float qb[4], kc[4], kh[4], e[4], ei[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                e[i] = __expf(Gv[i]);
+                ei[i] = __expf(-Gv[i]);
+                qb[i] = qf[i] * e[i];
+                kc[i] = bf[i] * kf[i] * e[i];
+                kh[i] = kf[i] * ei[i];
+            }
+            st_h4(sm + RQ + sw128_chunk(r, lane >> 1, 64) + (lane & 1) * 8, qb[0], qb[1], qb[2], qb[3]);
+            khr[m] = make_uint2(pack_f16(kh[0], kh[1]), pack_f16(kh[2], kh[3]));
+            kcr[m] = make_uint2(pack_f16(kc[0], kc[1]), pack_f16(kc[2], kc[3]));
+            er[m] = make_uint2(pack_f16(e[0], e[1]), pack_f16(e[2], e[3]));
+            eir[m] = make_uint2(pack_f16(ei[0], ei[1]), pack_f16(ei[2], ei[3]));
+#pragma unroll
+            for (int i = 0; i < 4; ++i) big = fmaxf(big, fmaxf(fabsf(qb[i]), fmaxf(fabsf(kc[i]), fabsf(kh[i]))));
+        }
+        // ---------------- masked dP, dA; Kh, Kc into the space of S_m
+        ok = mbar_wait(&bars[1], 0, kWait) && ok;
+        fence_after_sync();
         {
-            const int r = quarter * 16 + lane;
-#pragma unroll 1
-            for (int a = 0; a < 3; ++a) {
-                const uint32_t col0 = (a == 0 ? TM_Y1 : a == 1 ? TM_Y2 : TM_Y3) + 64 * half;
-                float y[64];
+            // accumulator row quarter * 32 + lane: 0..63 dP, 64..127 dA; 16 columns from 16 * cgrp
+            float row[16];
+            tmem_ld16(taddr(tm + TM_PA, quarter * 32, 16 * cgrp), row);
+            tmem_wait_ld();
+            const int pr = quarter * 32 + lane, r = pr & 63;
+            // dP keeps j <= r; dA = strictly-lower of (-dU) Delta^T
 #pragma unroll
-                for (int j = 0; j < 4; ++j) tmem_ld16(taddr(tm + col0, quarter * 32, 16 * j), y + 16 * j);
-                tmem_wait_ld();
-                if (lane < 16) {
-                    float *row = YS + (a * 64 + r) * 128;
+            for (int j = 0; j < 16; ++j) row[j] = (pr < 64 ? 16 * cgrp + j <= r : 16 * cgrp + j < r) ? row[j] : 0.f;
 #pragma unroll
-                    for (int ch = 0; ch < 16; ++ch) {  // logical 16-B chunk 16 * half + ch
-                        const int lc = 16 * half + ch, pc = lc ^ (r & 31);
-                        *reinterpret_cast<float4 *>(row + 4 * pc) =
-                            make_float4(y[4 * ch], y[4 * ch + 1], y[4 * ch + 2], y[4 * ch + 3]);
-                    }
-                }
+            for (int jj = 0; jj < 2; ++jj) {
+                st_h8(sm + PA + sw128_chunk(pr, 2 * cgrp + jj, 128), row + 8 * jj);
+                big = absmax8(row + 8 * jj, big);
             }
         }
-        __syncthreads();
-        {
-            const float *sG = reinterpret_cast<const float *>(sm + RAW_G);
-            const float *rb = reinterpret_cast<const float *>(sm + RAW_B);
-            float *sdG = YS;  // row r of dG overwrites row r of Y1 (read first, same warp)
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const uint32_t off = sw128_off(4 * warp + m, 4 * lane, 64);
+            *reinterpret_cast<uint2 *>(sm + KH + off) = khr[m];
+            *reinterpret_cast<uint2 *>(sm + KC + off) = kcr[m];
+            *reinterpret_cast<uint2 *>(sm + TE + off) = er[m];
+            *reinterpret_cast<uint2 *>(sm + TEI + off) = eir[m];
+        }
+    }
+    fence_proxy_async();
+    fence_before_sync();
+    __syncthreads();
+    if (issuer) {
+        fence_after_sync();
+        const uint64_t kP = desc_kmajor(smem_addr(sm + PA), 128, 0), kA = desc_kmajor(smem_addr(sm + PA + 8192), 128, 0),
+                       mP = desc_mnmajor(smem_addr(sm + PA), 64, 0), mA = desc_mnmajor(smem_addr(sm + PA + 8192), 64, 0),
+                       qb = desc_mnmajor(smem_addr(sm + RQ), 64, 0), kc = desc_mnmajor(smem_addr(sm + KC), 64, 0),
+                       kh = desc_mnmajor(smem_addr(sm + KH), 64, 0);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+            const uint64_t b_kh = kstep_mnmajor(kh, ks);
+            mma_bf16(tm + TM_Y1, kstep_kmajor(kP, 128, ks), b_kh, ID_KM128, 1);
+            mma_bf16(tm + TM_Y2, kstep_kmajor(kA, 128, ks), b_kh, ID_KM128, 1);
+            mma_bf16(tm + TM_Y3, kstep_mnmajor(mP, ks), kstep_mnmajor(qb, ks), ID_MM128, 1);
+            mma_bf16(tm + TM_Y3, kstep_mnmajor(mA, ks), kstep_mnmajor(kc, ks), ID_MM128, 1);
+        }
+        mma_commit(&bars[2]);
+    }
+    // ---------------- dq, dk, db, dG per (row, channel), from tensor memory.
+    // The M = 64 accumulators hold row quarter * 16 + l in lane l < 16; each
+    // 16-channel group is split by shuffles: lane l keeps channels 0..7 of
+    // row l, lane l + 16 takes channels 8..15 of the same row.
+    if (compute) {
+        ok = mbar_wait(&bars[2], 0, kWait) && ok;
+        fence_after_sync();
+        const int r = quarter * 16 + (lane & 15), hi = lane >> 4;
 #pragma unroll 1
-            for (int i8 = 0; i8 < 8; ++i8) {
-                const int r = warp + 8 * i8, pc = lane ^ (r & 31);
-                const float4 y1 = *reinterpret_cast<const float4 *>(YS + (0 * 64 + r) * 128 + 4 * pc);
-                const float4 y2 = *reinterpret_cast<const float4 *>(YS + (1 * 64 + r) * 128 + 4 * pc);
-                const float4 y3 = *reinterpret_cast<const float4 *>(YS + (2 * 64 + r) * 128 + 4 * pc);
-                const float4 G4 = *reinterpret_cast<const float4 *>(sG + r * 128 + 4 * lane);
-                const float4 b4 = *reinterpret_cast<const float4 *>(rb + r * 128 + 4 * lane);
-                const uint2 qr = *reinterpret_cast<const uint2 *>(sm + RAW_Q + r * 256 + 8 * lane);
-                const uint2 kr = *reinterpret_cast<const uint2 *>(sm + RAW_K + r * 256 + 8 * lane);
-                const __nv_bfloat162 *q2 = reinterpret_cast<const __nv_bfloat162 *>(&qr);
-                const __nv_bfloat162 *k2 = reinterpret_cast<const __nv_bfloat162 *>(&kr);
-                const float Y1[4] = {y1.x, y1.y, y1.z, y1.w}, Y2[4] = {y2.x, y2.y, y2.z, y2.w},
-                            Y3[4] = {y3.x, y3.y, y3.z, y3.w}, Gv[4] = {G4.x, G4.y, G4.z, G4.w},
-                            bf[4] = {b4.x, b4.y, b4.z, b4.w};
-                const float qf[4] = {__low2float(q2[0]), __high2float(q2[0]), __low2float(q2[1]), __high2float(q2[1])};
-                const float kf[4] = {__low2float(k2[0]), __high2float(k2[0]), __low2float(k2[1]), __high2float(k2[1])};
-                float dq[4], dk[4], db[4], dG[4];
+        for (int g2 = 0; g2 < 2; ++g2) {
+            const int ch0 = 32 * cgrp + 16 * g2, ch = ch0 + 8 * hi;
+            float y1[16], y2[16], y3[16];
+            tmem_ld16(taddr(tm + TM_Y1 + ch0, quarter * 32, 0), y1);
+            tmem_ld16(taddr(tm + TM_Y2 + ch0, quarter * 32, 0), y2);
+            tmem_ld16(taddr(tm + TM_Y3 + ch0, quarter * 32, 0), y3);
+            tmem_wait_ld();
+            float a1[8], a2[8], a3[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float s1 = __shfl_sync(0xffffffffu, y1[8 + i], lane & 15);
+                const float s2 = __shfl_sync(0xffffffffu, y2[8 + i], lane & 15);
+                const float s3 = __shfl_sync(0xffffffffu, y3[8 + i], lane & 15);
+                a1[i] = hi ? s1 : y1[i];
+                a2[i] = hi ? s2 : y2[i];
+                a3[i] = hi ? s3 : y3[i];
+            }
+            const uint32_t o16 = sw128_chunk(r, ch >> 3, 64);
+            const uint32_t o32a = sw128_chunk(r, ch >> 2, 64), o32b = sw128_chunk(r, (ch >> 2) + 1, 64);
+            const uint4 qbr = *reinterpret_cast<const uint4 *>(sm + RQ + o16);
+            const uint4 kcr2 = *reinterpret_cast<const uint4 *>(sm + KC + o16);
+            const uint4 khr2 = *reinterpret_cast<const uint4 *>(sm + KH + o16);
+            const uint4 kr2 = *reinterpret_cast<const uint4 *>(sm + RK + o16);
+            const uint4 e2 = *reinterpret_cast<const uint4 *>(sm + TE + o16);
+            const uint4 ei2 = *reinterpret_cast<const uint4 *>(sm + TEI + o16);
+            const float4 b0 = *reinterpret_cast<const float4 *>(sm + RB + o32a);
+            const float4 b1 = *reinterpret_cast<const float4 *>(sm + RB + o32b);
+            float qb[8], kc[8], kh[8], kf[8], E[8], Ei[8];
+            {
+                const __half2 *x1 = reinterpret_cast<const __half2 *>(&qbr);
+                const __half2 *x2 = reinterpret_cast<const __half2 *>(&kcr2);
+                const __half2 *x3 = reinterpret_cast<const __half2 *>(&khr2);
+                const __half2 *x4 = reinterpret_cast<const __half2 *>(&e2);
+                const __half2 *x5 = reinterpret_cast<const __half2 *>(&ei2);
+                const __nv_bfloat162 *x6 = reinterpret_cast<const __nv_bfloat162 *>(&kr2);
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const float E = __expf(Gv[e]), Ei = __expf(-Gv[e]);
-                    const float dkc = Y2[e] * E, dkh = Y3[e] * Ei;
-                    dq[e] = Y1[e] * E;
-                    db[e] = dkc * kf[e];
-                    dk[e] = dkc * bf[e] + dkh;
-                    dG[e] = dq[e] * qf[e] + dkc * bf[e] * kf[e] - dkh * kf[e];
-                }
-                *reinterpret_cast<float4 *>(sdG + r * 128 + 4 * lane) = make_float4(dG[0], dG[1], dG[2], dG[3]);
-                if (r < L) {
-                    const size_t o4 = tok(d, bb, c0 + r, h, 128) + 4 * lane;
-                    *reinterpret_cast<uint2 *>(dqout + o4) = make_uint2(pack_bf16(dq[0], dq[1]), pack_bf16(dq[2], dq[3]));
-                    *reinterpret_cast<uint2 *>(dkout + o4) = make_uint2(pack_bf16(dk[0], dk[1]), pack_bf16(dk[2], dk[3]));
-                    *reinterpret_cast<float4 *>(dbout + o4) = make_float4(db[0], db[1], db[2], db[3]);
+                    qb[2 * e] = __low2float(x1[e]); qb[2 * e + 1] = __high2float(x1[e]);
+                    kc[2 * e] = __low2float(x2[e]); kc[2 * e + 1] = __high2float(x2[e]);
+                    kh[2 * e] = __low2float(x3[e]); kh[2 * e + 1] = __high2float(x3[e]);
+                    E[2 * e] = __low2float(x4[e]); E[2 * e + 1] = __high2float(x4[e]);
+                    Ei[2 * e] = __low2float(x5[e]); Ei[2 * e + 1] = __high2float(x5[e]);
+                    kf[2 * e] = __low2float(x6[e]); kf[2 * e + 1] = __high2float(x6[e]);
                 }
             }
-        }
-        abort = __syncthreads_or(!ok);
-        if (!abort) {
-            // dg = reverse in-chunk cumsum of dG with the chunk-end term on the last row;
-            // thread (channel, part): part 1 scans rows 32..63, part 0 rows 0..31 after
-            // adding the sum of rows 32..63 itself
-            const float *sdG = YS;
-            const int ch = tid & 127, part = tid >> 7;
-            float acc = sEnd[ch];
-            if (part == 0)
-                for (int rr = 32; rr < 64; ++rr) acc += sdG[rr * 128 + ch];
-            const int hi = part ? 63 : 31, lo = part ? 32 : 0;
-            for (int rr = hi; rr >= lo; --rr) {
-                acc += sdG[rr * 128 + ch];
-                if (rr < L) dgout[tok(d, bb, c0 + rr, h, 128) + ch] = acc;
+            const float bf[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+            float dq[8], dk[8], db[8], dG[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float dkc = a2[i] * E[i], dkh = a3[i] * Ei[i];
+                dq[i] = a1[i] * E[i];
+                db[i] = dkc * kf[i];
+                dk[i] = dkc * bf[i] + dkh;
+                dG[i] = a1[i] * qb[i] + a2[i] * kc[i] - a3[i] * kh[i];
             }
+            st_bf16x8(sm + RQ + o16, dq);
+            st_bf16x8(sm + RK + o16, dk);
+            *reinterpret_cast<float4 *>(sm + RB + o32a) = make_float4(db[0], db[1], db[2], db[3]);
+            *reinterpret_cast<float4 *>(sm + RB + o32b) = make_float4(db[4], db[5], db[6], db[7]);
+            *reinterpret_cast<float4 *>(sm + RG + o32a) = make_float4(dG[0], dG[1], dG[2], dG[3]);
+            *reinterpret_cast<float4 *>(sm + RG + o32b) = make_float4(dG[4], dG[5], dG[6], dG[7]);
         }
     }
+    fence_before_sync();
+    __syncthreads();
+    // ---------------- dg: reverse in-chunk cumsum of dG with the chunk-end term
+    if (compute) {
+        float run[4] = {0.f, 0.f, 0.f, 0.f}, x[4][4];
+#pragma unroll
+        for (int m = 3; m >= 0; --m) {
+            const float4 t = *reinterpret_cast<const float4 *>(sm + RG + sw128_chunk(4 * warp + m, lane, 64));
+            run[0] += t.x; run[1] += t.y; run[2] += t.z; run[3] += t.w;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) x[m][i] = run[i];
+        }
+        *reinterpret_cast<float4 *>(scan + warp * 128 + 4 * lane) = make_float4(run[0], run[1], run[2], run[3]);
+        named_sync(1, kCompute);
+        if (tid < 128) {  // per channel: the end term plus the later warps' totals, in place
+            float acc = sEnd[tid];
+#pragma unroll
+            for (int w2 = kWarps - 1; w2 >= 0; --w2) {
+                const float t = scan[w2 * 128 + tid];
+                scan[w2 * 128 + tid] = acc;
+                acc += t;
+            }
+        }
+        named_sync(1, kCompute);
+        const float4 a4 = *reinterpret_cast<const float4 *>(scan + warp * 128 + 4 * lane);
+        const float after[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+            *reinterpret_cast<float4 *>(sm + RG + sw128_chunk(4 * warp + m, lane, 64)) =
+                make_float4(x[m][0] + after[0], x[m][1] + after[1], x[m][2] + after[2], x[m][3] + after[3]);
+    }
+    fence_proxy_async();
+    fence_before_sync();
+    __syncthreads();
+    if (issuer) {
+        for (int x = 0; x < 2; ++x) {
+            tma_store_4d(&mdq, sm + RQ + x * 8192, 64 * x, h, c0, bb);
+            tma_store_4d(&mdk, sm + RK + x * 8192, 64 * x, h, c0, bb);
+        }
+        for (int x = 0; x < 4; ++x) {
+            tma_store_4d(&mdb, sm + RB + x * 8192, 32 * x, h, c0, bb);
+            tma_store_4d(&mdg, sm + RG + x * 8192, 32 * x, h, c0, bb);
+        }
+        bulk_commit();
+        bulk_wait_all();
+    }
     if (!(big <= kRange) || !(gbig <= 9.f)) record_status(status, GDN2_ERR_RANGE);
-    if (abort && tid == 0) {
+    if (!ok && tid == 0) {
         record_status(status, GDN2_ERR_TIMEOUT);
-        mbar_wait(&bars[0], 0, kWait);
+        // every issued product done before the tensor memory is freed
+        mbar_wait(&bars[1], 0, kWait);
+        mbar_wait(&bars[2], 0, kWait);
     }
     fence_before_sync();
     __syncthreads();
@@ -685,17 +812,21 @@ cudaError_t tc_bwd_launch(const void *q, const void *k, const void *v, const flo
                           void *dq, void *dk, void *dv, float *dg, float *db, float *dw,
                           float *dS0, void *ws, unsigned int *status, const Dims &d,
                           cudaStream_t s) {
-    CUtensorMap mq, mk, mdo_half, mdo, mg, mb, mv, mw, mdv, mdw;
-    if (!make_btHd_map(&mq, q, true, d.B, d.T, d.H, 128, 64, 128) ||
-        !make_btHd_map(&mk, k, true, d.B, d.T, d.H, 128, 64, 128) ||
-        !make_btHd_map(&mdo_half, dO, true, d.B, d.T, d.H, 128, 64, 64) ||
+    CUtensorMap mdo_half, mv, mw, mdv, mdw, mq, mk, mb, mg, mdo, mdq, mdk, mdb, mdg;
+    if (!make_btHd_map(&mdo_half, dO, true, d.B, d.T, d.H, 128, 64, 64) ||
         !make_btHd_map(&mv, v, true, d.B, d.T, d.H, 128, 64, 64, true) ||
         !make_btHd_map(&mw, w, false, d.B, d.T, d.H, 128, 64, 32, true) ||
         !make_btHd_map(&mdv, dv, true, d.B, d.T, d.H, 128, 64, 64, true) ||
         !make_btHd_map(&mdw, dw, false, d.B, d.T, d.H, 128, 64, 32, true) ||
-        !make_btHd_map(&mdo, dO, true, d.B, d.T, d.H, 128, 64, 128) ||
-        !make_btHd_map(&mg, g, false, d.B, d.T, d.H, 128, 64, 128) ||
-        !make_btHd_map(&mb, b, false, d.B, d.T, d.H, 128, 64, 128))
+        !make_btHd_map(&mq, q, true, d.B, d.T, d.H, 128, 64, 64, true) ||
+        !make_btHd_map(&mk, k, true, d.B, d.T, d.H, 128, 64, 64, true) ||
+        !make_btHd_map(&mb, b, false, d.B, d.T, d.H, 128, 64, 32, true) ||
+        !make_btHd_map(&mg, g, false, d.B, d.T, d.H, 128, 64, 32, true) ||
+        !make_btHd_map(&mdo, dO, true, d.B, d.T, d.H, 128, 64, 64, true) ||
+        !make_btHd_map(&mdq, dq, true, d.B, d.T, d.H, 128, 64, 64, true) ||
+        !make_btHd_map(&mdk, dk, true, d.B, d.T, d.H, 128, 64, 64, true) ||
+        !make_btHd_map(&mdb, db, false, d.B, d.T, d.H, 128, 64, 32, true) ||
+        !make_btHd_map(&mdg, dg, false, d.B, d.T, d.H, 128, 64, 32, true))
         return cudaErrorInvalidValue;
     const TcWs lay = tc_ws_layout(d);
     cudaError_t e = cudaFuncSetAttribute(tc_bwd_state_kernel,
@@ -711,8 +842,7 @@ cudaError_t tc_bwd_launch(const void *q, const void *k, const void *v, const flo
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     launch_begin(K_TC_BWD_GRAD, s);
     tc_bwd_grad_kernel<<<dim3(d.NC, d.H, d.B), tbg::kThreads, tbg::SMEM_BYTES, s>>>(
-        mq, mk, mdo, mg, mb, (__nv_bfloat16 *)dq, (__nv_bfloat16 *)dk, db, dg, (unsigned char *)ws,
-        lay, status, d);
+        mq, mk, mb, mg, mdo, mdq, mdk, mdb, mdg, (unsigned char *)ws, lay, status, d);
     launch_end(K_TC_BWD_GRAD, s);
     return cudaGetLastError();
 }

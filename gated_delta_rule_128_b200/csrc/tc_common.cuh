@@ -94,63 +94,35 @@ __device__ __forceinline__ void cumsum_finish(const float *scan, int warp, int l
         }
 }
 
-// Operand tiles Qb, Kc, Kh ([64 pos][128 key] fp16, 128-B swizzled, R = 64)
-// from the raw q, k (bf16 [64][128]) and b (f32 [64][128]) tiles.  Any null
-// destination is skipped.  Returns the largest |G - G_m| seen: with |q|, |k|,
-// |b| <= 8 every factor stays below 8 e^|G|, so the fp16 range holds while
-// that value stays below 9.
-__device__ __forceinline__ float write_factors(const unsigned char *rq, const unsigned char *rk,
-                                               const float *rb, const float G[8][4],
-                                               unsigned char *oQb, unsigned char *oKc,
-                                               unsigned char *oKh, int warp, int lane) {
-    float gmax = 0.f;
-#pragma unroll
-    for (int m = 0; m < 8; ++m) {
-        const int r = 8 * warp + m;
-        uint2 qr = *reinterpret_cast<const uint2 *>(rq + r * 256 + lane * 8);
-        uint2 kr = *reinterpret_cast<const uint2 *>(rk + r * 256 + lane * 8);
-        float4 bv = *reinterpret_cast<const float4 *>(rb + r * 128 + 4 * lane);
-        const __nv_bfloat162 *q2 = reinterpret_cast<const __nv_bfloat162 *>(&qr);
-        const __nv_bfloat162 *k2 = reinterpret_cast<const __nv_bfloat162 *>(&kr);
-        float qf[4] = {__low2float(q2[0]), __high2float(q2[0]), __low2float(q2[1]), __high2float(q2[1])};
-        float kf[4] = {__low2float(k2[0]), __high2float(k2[0]), __low2float(k2[1]), __high2float(k2[1])};
-        float bf[4] = {bv.x, bv.y, bv.z, bv.w};
-        float qb[4], kc[4], kh[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float e = __expf(G[m][i]), ei = __expf(-G[m][i]);
-            qb[i] = qf[i] * e;
-            kc[i] = bf[i] * kf[i] * e;
-            kh[i] = kf[i] * ei;
-            gmax = fmaxf(gmax, fabsf(G[m][i]));
-        }
-        const uint32_t off = sw128_off(r, 4 * lane, 64);
-        if (oQb) st_h4(oQb + off, qb[0], qb[1], qb[2], qb[3]);
-        if (oKc) st_h4(oKc + off, kc[0], kc[1], kc[2], kc[3]);
-        if (oKh) st_h4(oKh + off, kh[0], kh[1], kh[2], kh[3]);
-    }
-    return gmax;
-}
-
-// The same operands for the chunk record's layout: Kc into rows 0..63 and Qb
-// into rows 64..127 of the [128][128] K-major tile at oWQ, Kh into the
-// [64][128] K-major tile at oKh.  Returns the largest |G - G_m| seen.
+// Operands of the chunk record from the raw q, k (bf16 [64][128]) and b (f32
+// [64][128]) tiles: Kc = b.k.E into rows 0..63 and Qb = q.E into rows
+// 64..127 of the [128][128] K-major tile at oWQ, Kh = k / E into the
+// [64][128] K-major tile at oKh (E = e^(G - G_m)).  Every input row is loaded
+// before the first store, so that the loads overlap.  Returns the largest
+// |G - G_m| seen: with |q|, |k|, |b| <= 8 every factor stays below 8 e^|G|,
+// so the fp16 range holds while that value stays below 9.
 __device__ __forceinline__ float write_factors_rec(const unsigned char *rq, const unsigned char *rk,
                                                    const float *rb, const float G[8][4],
                                                    unsigned char *oWQ, unsigned char *oKh,
                                                    int warp, int lane) {
+    uint2 qr[8], kr[8];
+    float4 bv[8];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+        const int r = 8 * warp + m;
+        qr[m] = *reinterpret_cast<const uint2 *>(rq + r * 256 + lane * 8);
+        kr[m] = *reinterpret_cast<const uint2 *>(rk + r * 256 + lane * 8);
+        bv[m] = *reinterpret_cast<const float4 *>(rb + r * 128 + 4 * lane);
+    }
     float gmax = 0.f;
 #pragma unroll
     for (int m = 0; m < 8; ++m) {
         const int r = 8 * warp + m;
-        uint2 qr = *reinterpret_cast<const uint2 *>(rq + r * 256 + lane * 8);
-        uint2 kr = *reinterpret_cast<const uint2 *>(rk + r * 256 + lane * 8);
-        float4 bv = *reinterpret_cast<const float4 *>(rb + r * 128 + 4 * lane);
-        const __nv_bfloat162 *q2 = reinterpret_cast<const __nv_bfloat162 *>(&qr);
-        const __nv_bfloat162 *k2 = reinterpret_cast<const __nv_bfloat162 *>(&kr);
-        float qf[4] = {__low2float(q2[0]), __high2float(q2[0]), __low2float(q2[1]), __high2float(q2[1])};
-        float kf[4] = {__low2float(k2[0]), __high2float(k2[0]), __low2float(k2[1]), __high2float(k2[1])};
-        float bf[4] = {bv.x, bv.y, bv.z, bv.w};
+        const __nv_bfloat162 *q2 = reinterpret_cast<const __nv_bfloat162 *>(&qr[m]);
+        const __nv_bfloat162 *k2 = reinterpret_cast<const __nv_bfloat162 *>(&kr[m]);
+        const float qf[4] = {__low2float(q2[0]), __high2float(q2[0]), __low2float(q2[1]), __high2float(q2[1])};
+        const float kf[4] = {__low2float(k2[0]), __high2float(k2[0]), __low2float(k2[1]), __high2float(k2[1])};
+        const float bf[4] = {bv[m].x, bv[m].y, bv[m].z, bv[m].w};
         float qb[4], kc[4], kh[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {

@@ -66,10 +66,6 @@ constexpr float kRange = 6.0e4f;           // largest operand magnitude kept in 
 static_assert(STAGE % 1024 == 0 && MISC % 1024 == 0, "alignment");
 }  // namespace tfwd
 
-__device__ __forceinline__ void named_sync(int id, int nthreads) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
 __global__ void __launch_bounds__(tfwd::kThreads, 1)
 tc_fwd_kernel(const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mw,
               const float *__restrict__ S0, __nv_bfloat16 *__restrict__ o, float *__restrict__ ST,
