@@ -80,6 +80,19 @@ void launch_end(int kind, cudaStream_t s);
 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
+// number of SMs of the current device (grid size of the persistent kernels)
+inline int sm_count() {
+    static int cached[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 1;
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) n = 1;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
 inline SimtWs simt_ws_layout(const Dims &d) {
     SimtWs w;
     size_t tiles = (size_t)d.B * d.H * d.NC;

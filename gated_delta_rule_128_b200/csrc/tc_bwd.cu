@@ -435,7 +435,8 @@ constexpr uint32_t KH = SMT, KC = SMT + 16384, PA = DXT;  // after the first pro
 constexpr uint32_t TE = DXT + 16384, TEI = DL;              // E = e^(G - G_m), 1/E (fp16 [64][128])
 constexpr uint32_t MISC = 212992; // sEnd [128]; sRef [128]; scan [16][128]; mbarriers; slot
 constexpr uint32_t SMEM_BYTES = MISC + 1024 + 8192 + 128 + 1024;
-constexpr uint32_t LOAD_BYTES = 212992;
+constexpr uint32_t LOAD_A = 114688;  // dO, -dU, Delta, S_m, dX (the first products' operands)
+constexpr uint32_t LOAD_B = 98304;   // raw q, k, b, g
 constexpr uint32_t TM_Y1 = 0, TM_Y2 = 128, TM_Y3 = 256, TM_PA = 384;  // 512 columns
 constexpr uint32_t ID_PA = idesc_f16(128, 64, false, false);
 constexpr uint32_t ID_KK128 = idesc_f16(64, 128, false, false);
@@ -451,7 +452,7 @@ __device__ __forceinline__ uint64_t kstep_kmajor_blk(uint64_t d0, uint32_t blk, 
     return d0 + (uint64_t)((((uint32_t)(kstep >> 2) * blk) + (kstep & 3) * 32) >> 4);
 }
 
-// One CTA per (b, h, chunk), all chunks in parallel, full d_v.  Warp 16
+// Persistent: one CTA per SM walks the (b, h, chunk) tiles, full d_v.  Warp 16
 // loads the tile (raw q, k, b, g, dO as 128-B swizzled TMA boxes; S_m, dX,
 // Delta, -dU from the workspace) and issues the products; warps 0..15 form
 // the operands and the outputs:
@@ -465,7 +466,10 @@ __device__ __forceinline__ uint64_t kstep_kmajor_blk(uint64_t d0, uint32_t blk, 
 // chunk-end term, and the four tiles leave by TMA stores.  Sixteen compute
 // warps (four rows each in the row-wise phases) hide the latency of the
 // per-element work; E and 1/E are kept as fp16 tiles between the factor
-// phase and the outputs.
+// phase and the outputs.  The next tile's copies are requested as soon as
+// their buffers are free: dO and -dU after the first products, Delta, S_m
+// and dX after the outputs are formed, the raw tiles once the TMA stores have
+// read them.
 __global__ void __launch_bounds__(tbg::kThreads, 1)
 tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                    const __grid_constant__ CUtensorMap mb, const __grid_constant__ CUtensorMap mg,
@@ -480,15 +484,15 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
     float *sEnd = reinterpret_cast<float *>(sm + MISC);        // chunk-end term per channel
     float *sRef = reinterpret_cast<float *>(sm + MISC + 512);  // G of the middle row per channel
     float *scan = reinterpret_cast<float *>(sm + MISC + 1024);  // per-warp totals [16][128]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + MISC + 1024 + 8192);  // 0 loads, 1, 2 products
+    // 0 first-product operands (two parts), 1, 2 products, 3 raw tiles
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + MISC + 1024 + 8192);
     uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + MISC + 1024 + 8192 + 64);
     float big = 0.f, gbig = 0.f;  // range checks: operand magnitude, |G - G_m|
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int c = blockIdx.x, h = blockIdx.y, bb = blockIdx.z, c0 = c * 64;
     const int NC = d.NC, H = d.H;
+    const int ntiles = d.B * H * NC;
     const int quarter = warp & 3, cgrp = (warp >> 2) & 3;  // TMEM lane quarter; column group
-    const size_t bh = (size_t)bb * H + h;
     const bool compute = warp < kWarps, issuer = tid == kCompute;
 
     if (warp == 0) {
@@ -496,7 +500,8 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
         tmem_relinquish();
     }
     if (issuer) {
-        for (int i = 0; i < 3; ++i) mbar_init(&bars[i], 1);
+        mbar_init(&bars[0], 2);
+        for (int i = 1; i < 4; ++i) mbar_init(&bars[i], 1);
         mbar_fence_init();
     }
     fence_before_sync();
@@ -504,302 +509,348 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
     fence_after_sync();
     const uint32_t tm = *tslot;
 
-    if (issuer) {
-        mbar_expect_tx(&bars[0], LOAD_BYTES);
+    // tile `it` = (b * H + h) * NC + c; copies requested by the issuer
+    int issued[3] = {0, 0, 0};  // operand parts 1, 2 and raw tiles
+    auto load_a1 = [&](int it) {  // dO (TMA) and -dU: [dO; -dU]
+        const int c = it % NC, bhi = it / NC, h = bhi % H, bb = bhi / H;
+        mbar_expect_tx(&bars[0], 32768);
         for (int x = 0; x < 2; ++x) {
-            tma_load_4d(sm + RQ + x * 8192, &mq, 64 * x, h, c0, bb, &bars[0]);
-            tma_load_4d(sm + RK + x * 8192, &mk, 64 * x, h, c0, bb, &bars[0]);
-            tma_load_4d(sm + DN + x * 16384, &mdo, 64 * x, h, c0, bb, &bars[0]);
-            bulk_load(sm + DN + x * 16384 + 8192, ws + lay.ckndU + ((bh * NC + c) * 2 + x) * 8192, 8192,
-                      &bars[0]);
+            tma_load_4d(sm + DN + x * 16384, &mdo, 64 * x, h, c * 64, bb, &bars[0]);
+            bulk_load(sm + DN + x * 16384 + 8192, ws + lay.ckndU + ((size_t)it * 2 + x) * 8192, 8192, &bars[0]);
+        }
+        ++issued[0];
+    };
+    auto load_a2 = [&](int it) {  // Delta, S_m, dX
+        mbar_expect_tx(&bars[0], LOAD_A - 32768);
+        bulk_load(sm + DL, ws + lay.ckD + ((size_t)it * 2) * 8192, 16384, &bars[0]);
+        bulk_load(sm + SMT, ws + lay.ckS + ((size_t)(it + it / NC) * 2) * 16384, 32768, &bars[0]);
+        bulk_load(sm + DXT, ws + lay.ckdS + ((size_t)it * 2) * 16384, 32768, &bars[0]);
+        ++issued[1];
+    };
+    auto load_b = [&](int it) {  // raw q, k, b, g
+        const int c = it % NC, bhi = it / NC, h = bhi % H, bb = bhi / H;
+        mbar_expect_tx(&bars[3], LOAD_B);
+        for (int x = 0; x < 2; ++x) {
+            tma_load_4d(sm + RQ + x * 8192, &mq, 64 * x, h, c * 64, bb, &bars[3]);
+            tma_load_4d(sm + RK + x * 8192, &mk, 64 * x, h, c * 64, bb, &bars[3]);
         }
         for (int x = 0; x < 4; ++x) {
-            tma_load_4d(sm + RB + x * 8192, &mb, 32 * x, h, c0, bb, &bars[0]);
-            tma_load_4d(sm + RG + x * 8192, &mg, 32 * x, h, c0, bb, &bars[0]);
+            tma_load_4d(sm + RB + x * 8192, &mb, 32 * x, h, c * 64, bb, &bars[3]);
+            tma_load_4d(sm + RG + x * 8192, &mg, 32 * x, h, c * 64, bb, &bars[3]);
         }
-        bulk_load(sm + DL, ws + lay.ckD + ((bh * NC + c) * 2) * 8192, 16384, &bars[0]);
-        bulk_load(sm + SMT, ws + lay.ckS + ((bh * (NC + 1) + c) * 2) * 16384, 32768, &bars[0]);
-        bulk_load(sm + DXT, ws + lay.ckdS + ((bh * NC + c) * 2) * 16384, 32768, &bars[0]);
+        ++issued[2];
+    };
+    if (issuer && (int)blockIdx.x < ntiles) {
+        load_a1(blockIdx.x);
+        load_a2(blockIdx.x);
+        load_b(blockIdx.x);
     }
-    if (tid < 128) {
-        const float *e0 = reinterpret_cast<const float *>(ws + lay.ckEnd + ((bh * NC + c) * 2) * 512);
-        sEnd[tid] = e0[tid] + e0[128 + tid];
-    }
-    bool ok = mbar_wait(&bars[0], 0, kWait);
 
-    // ---------------- cumulative decay (rows 4w..4w+3, channels 4l..4l+3); dO to fp16
-    float G[4][4];
-    if (compute) {
-        float run[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            const float4 t = *reinterpret_cast<const float4 *>(sm + RG + sw128_chunk(4 * warp + m, lane, 64));
-            run[0] += t.x; run[1] += t.y; run[2] += t.z; run[3] += t.w;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) G[m][i] = run[i];
+    bool ok = true;
+    for (int it = blockIdx.x, n = 0; it < ntiles; it += gridDim.x, ++n) {
+        const int c = it % NC, bhi = it / NC, h = bhi % H, bb = bhi / H, c0 = c * 64;
+        const uint32_t par = n & 1;
+        const int nxt = it + (int)gridDim.x;
+        const bool more = nxt < ntiles;
+        if (tid < 128) {
+            const float *e0 = reinterpret_cast<const float *>(ws + lay.ckEnd + ((size_t)it * 2) * 512);
+            sEnd[tid] = e0[tid] + e0[128 + tid];
         }
-        *reinterpret_cast<float4 *>(scan + warp * 128 + 4 * lane) = make_float4(run[0], run[1], run[2], run[3]);
-        named_sync(1, kCompute);
-        if (tid < 128) {  // per channel: exclusive prefix over the warps' totals, in place
-            float acc = 0.f;
+        ok = mbar_wait(&bars[0], par, kWait) && ok;
+
+        // ---------------- dO to fp16; then, while the first products run, the
+        // cumulative decay (rows 4w..4w+3, channels 4l..4l+3)
+        if (compute) {
 #pragma unroll
-            for (int w2 = 0; w2 < kWarps; ++w2) {
-                const float t = scan[w2 * 128 + tid];
-                scan[w2 * 128 + tid] = acc;
-                acc += t;
-                if (w2 == kWarps / 2 - 1) sRef[tid] = acc;  // rows 0..31: G of the middle row
-            }
-        }
-#pragma unroll
-        for (int m = 0; m < 2; ++m) {  // the dO rows of [dO; -dU], in place
-            const int i = tid + kCompute * m;
-            unsigned char *p = sm + DN + (i >> 9) * 16384 + (i & 511) * 16;
-            uint4 raw = *reinterpret_cast<const uint4 *>(p);
-            const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-            float x[8];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                x[2 * e] = __low2float(b2[e]);
-                x[2 * e + 1] = __high2float(b2[e]);
-            }
-            st_h8(p, x);
-        }
-    }
-    fence_proxy_async();
-    fence_before_sync();
-    ok = !__syncthreads_or(!ok);
-    if (issuer) {
-        fence_after_sync();
-        const uint64_t dn = desc_kmajor(smem_addr(sm + DN), 128, 0), dl = desc_kmajor(smem_addr(sm + DL), 64, 0),
-                       s = desc_kmajor(smem_addr(sm + SMT), 128, 0), dx = desc_kmajor(smem_addr(sm + DXT), 128, 0),
-                       ado = desc_kmajor(smem_addr(sm + DN), 64, 0), andu = desc_kmajor(smem_addr(sm + DN + 8192), 64, 0);
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-            const uint64_t b_s = kstep_kmajor(s, 128, ks), a_dl = kstep_kmajor(dl, 64, ks);
-            mma_bf16(tm + TM_PA, kstep_kmajor(dn, 128, ks), a_dl, ID_PA, ks > 0);
-            mma_bf16(tm + TM_Y1, kstep_kmajor_blk(ado, 16384, ks), b_s, ID_KK128, ks > 0);
-            mma_bf16(tm + TM_Y2, kstep_kmajor_blk(andu, 16384, ks), b_s, ID_KK128, ks > 0);
-            mma_bf16(tm + TM_Y3, a_dl, kstep_kmajor(dx, 128, ks), ID_KK128, ks > 0);
-        }
-        mma_commit(&bars[1]);
-    }
-    // ---------------- decay factors while the products run: Qb in place of q;
-    // Kh, Kc kept in registers until S_m is consumed
-    uint2 khr[4], kcr[4], er[4], eir[4];
-    if (compute) {
-        const float4 pre4 = *reinterpret_cast<const float4 *>(scan + warp * 128 + 4 * lane);
-        const float4 ref4 = *reinterpret_cast<const float4 *>(sRef + 4 * lane);
-        const float pre[4] = {pre4.x, pre4.y, pre4.z, pre4.w}, ref[4] = {ref4.x, ref4.y, ref4.z, ref4.w};
-        uint2 qr[4], kr[4];
-        float4 bv[4];
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {  // every input row before the first store
-            const int r = 4 * warp + m;
-            qr[m] = *reinterpret_cast<const uint2 *>(sm + RQ + sw128_chunk(r, lane >> 1, 64) + (lane & 1) * 8);
-            kr[m] = *reinterpret_cast<const uint2 *>(sm + RK + sw128_chunk(r, lane >> 1, 64) + (lane & 1) * 8);
-            bv[m] = *reinterpret_cast<const float4 *>(sm + RB + sw128_chunk(r, lane, 64));
-        }
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            const int r = 4 * warp + m;
-            float Gv[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                Gv[i] = G[m][i] + pre[i] - ref[i];
-                gbig = fmaxf(gbig, fabsf(Gv[i]));
-            }
-            const __nv_bfloat162 *q2 = reinterpret_cast<const __nv_bfloat162 *>(&qr[m]);
-            const __nv_bfloat162 *k2 = reinterpret_cast<const __nv_bfloat162 *>(&kr[m]);
-            const float qf[4] = {__low2float(q2[0]), __high2float(q2[0]), __low2float(q2[1]), __high2float(q2[1])};
-            const float kf[4] = {__low2float(k2[0]), __high2float(k2[0]), __low2float(k2[1]), __high2float(k2[1])};
-            const float bf[4] = {bv[m].x, bv[m].y, bv[m].z, bv[m].w};
-            float qb[4], kc[4], kh[4], e[4], ei[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                e[i] = __expf(Gv[i]);
-                ei[i] = __expf(-Gv[i]);
-                qb[i] = qf[i] * e[i];
-                kc[i] = bf[i] * kf[i] * e[i];
-                kh[i] = kf[i] * ei[i];
-            }
-            st_h4(sm + RQ + sw128_chunk(r, lane >> 1, 64) + (lane & 1) * 8, qb[0], qb[1], qb[2], qb[3]);
-            khr[m] = make_uint2(pack_f16(kh[0], kh[1]), pack_f16(kh[2], kh[3]));
-            kcr[m] = make_uint2(pack_f16(kc[0], kc[1]), pack_f16(kc[2], kc[3]));
-            er[m] = make_uint2(pack_f16(e[0], e[1]), pack_f16(e[2], e[3]));
-            eir[m] = make_uint2(pack_f16(ei[0], ei[1]), pack_f16(ei[2], ei[3]));
-#pragma unroll
-            for (int i = 0; i < 4; ++i) big = fmaxf(big, fmaxf(fabsf(qb[i]), fmaxf(fabsf(kc[i]), fabsf(kh[i]))));
-        }
-        // ---------------- masked dP, dA; Kh, Kc into the space of S_m
-        ok = mbar_wait(&bars[1], 0, kWait) && ok;
-        fence_after_sync();
-        {
-            // accumulator row quarter * 32 + lane: 0..63 dP, 64..127 dA; 16 columns from 16 * cgrp
-            float row[16];
-            tmem_ld16(taddr(tm + TM_PA, quarter * 32, 16 * cgrp), row);
-            tmem_wait_ld();
-            const int pr = quarter * 32 + lane, r = pr & 63;
-            // dP keeps j <= r; dA = strictly-lower of (-dU) Delta^T
-#pragma unroll
-            for (int j = 0; j < 16; ++j) row[j] = (pr < 64 ? 16 * cgrp + j <= r : 16 * cgrp + j < r) ? row[j] : 0.f;
-#pragma unroll
-            for (int jj = 0; jj < 2; ++jj) {
-                st_h8(sm + PA + sw128_chunk(pr, 2 * cgrp + jj, 128), row + 8 * jj);
-                big = absmax8(row + 8 * jj, big);
-            }
-        }
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            const uint32_t off = sw128_off(4 * warp + m, 4 * lane, 64);
-            *reinterpret_cast<uint2 *>(sm + KH + off) = khr[m];
-            *reinterpret_cast<uint2 *>(sm + KC + off) = kcr[m];
-            *reinterpret_cast<uint2 *>(sm + TE + off) = er[m];
-            *reinterpret_cast<uint2 *>(sm + TEI + off) = eir[m];
-        }
-    }
-    fence_proxy_async();
-    fence_before_sync();
-    __syncthreads();
-    if (issuer) {
-        fence_after_sync();
-        const uint64_t kP = desc_kmajor(smem_addr(sm + PA), 128, 0), kA = desc_kmajor(smem_addr(sm + PA + 8192), 128, 0),
-                       mP = desc_mnmajor(smem_addr(sm + PA), 64, 0), mA = desc_mnmajor(smem_addr(sm + PA + 8192), 64, 0),
-                       qb = desc_mnmajor(smem_addr(sm + RQ), 64, 0), kc = desc_mnmajor(smem_addr(sm + KC), 64, 0),
-                       kh = desc_mnmajor(smem_addr(sm + KH), 64, 0);
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t b_kh = kstep_mnmajor(kh, ks);
-            mma_bf16(tm + TM_Y1, kstep_kmajor(kP, 128, ks), b_kh, ID_KM128, 1);
-            mma_bf16(tm + TM_Y2, kstep_kmajor(kA, 128, ks), b_kh, ID_KM128, 1);
-            mma_bf16(tm + TM_Y3, kstep_mnmajor(mP, ks), kstep_mnmajor(qb, ks), ID_MM128, 1);
-            mma_bf16(tm + TM_Y3, kstep_mnmajor(mA, ks), kstep_mnmajor(kc, ks), ID_MM128, 1);
-        }
-        mma_commit(&bars[2]);
-    }
-    // ---------------- dq, dk, db, dG per (row, channel), from tensor memory.
-    // The M = 64 accumulators hold row quarter * 16 + l in lane l < 16; each
-    // 16-channel group is split by shuffles: lane l keeps channels 0..7 of
-    // row l, lane l + 16 takes channels 8..15 of the same row.
-    if (compute) {
-        ok = mbar_wait(&bars[2], 0, kWait) && ok;
-        fence_after_sync();
-        const int r = quarter * 16 + (lane & 15), hi = lane >> 4;
-#pragma unroll 1
-        for (int g2 = 0; g2 < 2; ++g2) {
-            const int ch0 = 32 * cgrp + 16 * g2, ch = ch0 + 8 * hi;
-            float y1[16], y2[16], y3[16];
-            tmem_ld16(taddr(tm + TM_Y1 + ch0, quarter * 32, 0), y1);
-            tmem_ld16(taddr(tm + TM_Y2 + ch0, quarter * 32, 0), y2);
-            tmem_ld16(taddr(tm + TM_Y3 + ch0, quarter * 32, 0), y3);
-            tmem_wait_ld();
-            float a1[8], a2[8], a3[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float s1 = __shfl_sync(0xffffffffu, y1[8 + i], lane & 15);
-                const float s2 = __shfl_sync(0xffffffffu, y2[8 + i], lane & 15);
-                const float s3 = __shfl_sync(0xffffffffu, y3[8 + i], lane & 15);
-                a1[i] = hi ? s1 : y1[i];
-                a2[i] = hi ? s2 : y2[i];
-                a3[i] = hi ? s3 : y3[i];
-            }
-            const uint32_t o16 = sw128_chunk(r, ch >> 3, 64);
-            const uint32_t o32a = sw128_chunk(r, ch >> 2, 64), o32b = sw128_chunk(r, (ch >> 2) + 1, 64);
-            const uint4 qbr = *reinterpret_cast<const uint4 *>(sm + RQ + o16);
-            const uint4 kcr2 = *reinterpret_cast<const uint4 *>(sm + KC + o16);
-            const uint4 khr2 = *reinterpret_cast<const uint4 *>(sm + KH + o16);
-            const uint4 kr2 = *reinterpret_cast<const uint4 *>(sm + RK + o16);
-            const uint4 e2 = *reinterpret_cast<const uint4 *>(sm + TE + o16);
-            const uint4 ei2 = *reinterpret_cast<const uint4 *>(sm + TEI + o16);
-            const float4 b0 = *reinterpret_cast<const float4 *>(sm + RB + o32a);
-            const float4 b1 = *reinterpret_cast<const float4 *>(sm + RB + o32b);
-            float qb[8], kc[8], kh[8], kf[8], E[8], Ei[8];
-            {
-                const __half2 *x1 = reinterpret_cast<const __half2 *>(&qbr);
-                const __half2 *x2 = reinterpret_cast<const __half2 *>(&kcr2);
-                const __half2 *x3 = reinterpret_cast<const __half2 *>(&khr2);
-                const __half2 *x4 = reinterpret_cast<const __half2 *>(&e2);
-                const __half2 *x5 = reinterpret_cast<const __half2 *>(&ei2);
-                const __nv_bfloat162 *x6 = reinterpret_cast<const __nv_bfloat162 *>(&kr2);
+            for (int m = 0; m < 2; ++m) {  // the dO rows of [dO; -dU], in place
+                const int i = tid + kCompute * m;
+                unsigned char *p = sm + DN + (i >> 9) * 16384 + (i & 511) * 16;
+                uint4 raw = *reinterpret_cast<const uint4 *>(p);
+                const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+                float x[8];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    qb[2 * e] = __low2float(x1[e]); qb[2 * e + 1] = __high2float(x1[e]);
-                    kc[2 * e] = __low2float(x2[e]); kc[2 * e + 1] = __high2float(x2[e]);
-                    kh[2 * e] = __low2float(x3[e]); kh[2 * e + 1] = __high2float(x3[e]);
-                    E[2 * e] = __low2float(x4[e]); E[2 * e + 1] = __high2float(x4[e]);
-                    Ei[2 * e] = __low2float(x5[e]); Ei[2 * e + 1] = __high2float(x5[e]);
-                    kf[2 * e] = __low2float(x6[e]); kf[2 * e + 1] = __high2float(x6[e]);
+                    x[2 * e] = __low2float(b2[e]);
+                    x[2 * e + 1] = __high2float(b2[e]);
+                }
+                st_h8(p, x);
+            }
+        }
+        fence_proxy_async();
+        fence_before_sync();
+        __syncthreads();
+        if (issuer) {
+            fence_after_sync();
+            const uint64_t dn = desc_kmajor(smem_addr(sm + DN), 128, 0), dl = desc_kmajor(smem_addr(sm + DL), 64, 0),
+                           s = desc_kmajor(smem_addr(sm + SMT), 128, 0), dx = desc_kmajor(smem_addr(sm + DXT), 128, 0),
+                           ado = desc_kmajor(smem_addr(sm + DN), 64, 0), andu = desc_kmajor(smem_addr(sm + DN + 8192), 64, 0);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint64_t b_s = kstep_kmajor(s, 128, ks), a_dl = kstep_kmajor(dl, 64, ks);
+                mma_bf16(tm + TM_PA, kstep_kmajor(dn, 128, ks), a_dl, ID_PA, ks > 0);
+                mma_bf16(tm + TM_Y1, kstep_kmajor_blk(ado, 16384, ks), b_s, ID_KK128, ks > 0);
+                mma_bf16(tm + TM_Y2, kstep_kmajor_blk(andu, 16384, ks), b_s, ID_KK128, ks > 0);
+                mma_bf16(tm + TM_Y3, a_dl, kstep_kmajor(dx, 128, ks), ID_KK128, ks > 0);
+            }
+            mma_commit(&bars[1]);
+        }
+        float G[4][4];
+        if (compute) {
+            ok = mbar_wait(&bars[3], par, kWait) && ok;
+            float run[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const float4 t = *reinterpret_cast<const float4 *>(sm + RG + sw128_chunk(4 * warp + m, lane, 64));
+                run[0] += t.x; run[1] += t.y; run[2] += t.z; run[3] += t.w;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) G[m][i] = run[i];
+            }
+            *reinterpret_cast<float4 *>(scan + warp * 128 + 4 * lane) = make_float4(run[0], run[1], run[2], run[3]);
+            named_sync(1, kCompute);
+            if (tid < 128) {  // per channel: exclusive prefix over the warps' totals, in place
+                float acc = 0.f;
+#pragma unroll
+                for (int w2 = 0; w2 < kWarps; ++w2) {
+                    const float t = scan[w2 * 128 + tid];
+                    scan[w2 * 128 + tid] = acc;
+                    acc += t;
+                    if (w2 == kWarps / 2 - 1) sRef[tid] = acc;  // rows 0..31: G of the middle row
                 }
             }
-            const float bf[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-            float dq[8], dk[8], db[8], dG[8];
+            named_sync(1, kCompute);
+        }
+        // ---------------- decay factors while the products run: Qb in place of q;
+        // Kh, Kc kept in registers until S_m is consumed
+        uint2 khr[4], kcr[4], er[4], eir[4];
+        if (compute) {
+            const float4 pre4 = *reinterpret_cast<const float4 *>(scan + warp * 128 + 4 * lane);
+            const float4 ref4 = *reinterpret_cast<const float4 *>(sRef + 4 * lane);
+            const float pre[4] = {pre4.x, pre4.y, pre4.z, pre4.w}, ref[4] = {ref4.x, ref4.y, ref4.z, ref4.w};
+            uint2 qr[4], kr[4];
+            float4 bv[4];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float dkc = a2[i] * E[i], dkh = a3[i] * Ei[i];
-                dq[i] = a1[i] * E[i];
-                db[i] = dkc * kf[i];
-                dk[i] = dkc * bf[i] + dkh;
-                dG[i] = a1[i] * qb[i] + a2[i] * kc[i] - a3[i] * kh[i];
+            for (int m = 0; m < 4; ++m) {  // every input row before the first store
+                const int r = 4 * warp + m;
+                qr[m] = *reinterpret_cast<const uint2 *>(sm + RQ + sw128_chunk(r, lane >> 1, 64) + (lane & 1) * 8);
+                kr[m] = *reinterpret_cast<const uint2 *>(sm + RK + sw128_chunk(r, lane >> 1, 64) + (lane & 1) * 8);
+                bv[m] = *reinterpret_cast<const float4 *>(sm + RB + sw128_chunk(r, lane, 64));
             }
-            st_bf16x8(sm + RQ + o16, dq);
-            st_bf16x8(sm + RK + o16, dk);
-            *reinterpret_cast<float4 *>(sm + RB + o32a) = make_float4(db[0], db[1], db[2], db[3]);
-            *reinterpret_cast<float4 *>(sm + RB + o32b) = make_float4(db[4], db[5], db[6], db[7]);
-            *reinterpret_cast<float4 *>(sm + RG + o32a) = make_float4(dG[0], dG[1], dG[2], dG[3]);
-            *reinterpret_cast<float4 *>(sm + RG + o32b) = make_float4(dG[4], dG[5], dG[6], dG[7]);
-        }
-    }
-    fence_before_sync();
-    __syncthreads();
-    // ---------------- dg: reverse in-chunk cumsum of dG with the chunk-end term
-    if (compute) {
-        float run[4] = {0.f, 0.f, 0.f, 0.f}, x[4][4];
 #pragma unroll
-        for (int m = 3; m >= 0; --m) {
-            const float4 t = *reinterpret_cast<const float4 *>(sm + RG + sw128_chunk(4 * warp + m, lane, 64));
-            run[0] += t.x; run[1] += t.y; run[2] += t.z; run[3] += t.w;
+            for (int m = 0; m < 4; ++m) {
+                const int r = 4 * warp + m;
+                float Gv[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) x[m][i] = run[i];
-        }
-        *reinterpret_cast<float4 *>(scan + warp * 128 + 4 * lane) = make_float4(run[0], run[1], run[2], run[3]);
-        named_sync(1, kCompute);
-        if (tid < 128) {  // per channel: the end term plus the later warps' totals, in place
-            float acc = sEnd[tid];
+                for (int i = 0; i < 4; ++i) {
+                    Gv[i] = G[m][i] + pre[i] - ref[i];
+                    gbig = fmaxf(gbig, fabsf(Gv[i]));
+                }
+                const __nv_bfloat162 *q2 = reinterpret_cast<const __nv_bfloat162 *>(&qr[m]);
+                const __nv_bfloat162 *k2 = reinterpret_cast<const __nv_bfloat162 *>(&kr[m]);
+                const float qf[4] = {__low2float(q2[0]), __high2float(q2[0]), __low2float(q2[1]), __high2float(q2[1])};
+                const float kf[4] = {__low2float(k2[0]), __high2float(k2[0]), __low2float(k2[1]), __high2float(k2[1])};
+                const float bf[4] = {bv[m].x, bv[m].y, bv[m].z, bv[m].w};
+                float qb[4], kc[4], kh[4], e[4], ei[4];
 #pragma unroll
-            for (int w2 = kWarps - 1; w2 >= 0; --w2) {
-                const float t = scan[w2 * 128 + tid];
-                scan[w2 * 128 + tid] = acc;
-                acc += t;
+                for (int i = 0; i < 4; ++i) {
+                    e[i] = __expf(Gv[i]);
+                    ei[i] = __expf(-Gv[i]);
+                    qb[i] = qf[i] * e[i];
+                    kc[i] = bf[i] * kf[i] * e[i];
+                    kh[i] = kf[i] * ei[i];
+                }
+                st_h4(sm + RQ + sw128_chunk(r, lane >> 1, 64) + (lane & 1) * 8, qb[0], qb[1], qb[2], qb[3]);
+                khr[m] = make_uint2(pack_f16(kh[0], kh[1]), pack_f16(kh[2], kh[3]));
+                kcr[m] = make_uint2(pack_f16(kc[0], kc[1]), pack_f16(kc[2], kc[3]));
+                er[m] = make_uint2(pack_f16(e[0], e[1]), pack_f16(e[2], e[3]));
+                eir[m] = make_uint2(pack_f16(ei[0], ei[1]), pack_f16(ei[2], ei[3]));
+#pragma unroll
+                for (int i = 0; i < 4; ++i) big = fmaxf(big, fmaxf(fabsf(qb[i]), fmaxf(fabsf(kc[i]), fabsf(kh[i]))));
+            }
+            // ---------------- masked dP, dA; Kh, Kc into the space of S_m
+            ok = mbar_wait(&bars[1], par, kWait) && ok;
+            fence_after_sync();
+            {
+                // accumulator row quarter * 32 + lane: 0..63 dP, 64..127 dA; 16 columns from 16 * cgrp
+                float row[16];
+                tmem_ld16(taddr(tm + TM_PA, quarter * 32, 16 * cgrp), row);
+                tmem_wait_ld();
+                const int pr = quarter * 32 + lane, r = pr & 63;
+                // dP keeps j <= r; dA = strictly-lower of (-dU) Delta^T
+#pragma unroll
+                for (int j = 0; j < 16; ++j) row[j] = (pr < 64 ? 16 * cgrp + j <= r : 16 * cgrp + j < r) ? row[j] : 0.f;
+#pragma unroll
+                for (int jj = 0; jj < 2; ++jj) {
+                    st_h8(sm + PA + sw128_chunk(pr, 2 * cgrp + jj, 128), row + 8 * jj);
+                    big = absmax8(row + 8 * jj, big);
+                }
+            }
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const uint32_t off = sw128_off(4 * warp + m, 4 * lane, 64);
+                *reinterpret_cast<uint2 *>(sm + KH + off) = khr[m];
+                *reinterpret_cast<uint2 *>(sm + KC + off) = kcr[m];
+                *reinterpret_cast<uint2 *>(sm + TE + off) = er[m];
+                *reinterpret_cast<uint2 *>(sm + TEI + off) = eir[m];
             }
         }
-        named_sync(1, kCompute);
-        const float4 a4 = *reinterpret_cast<const float4 *>(scan + warp * 128 + 4 * lane);
-        const float after[4] = {a4.x, a4.y, a4.z, a4.w};
+        if (issuer) {  // dO and -dU of the next tile, once the first products have read them
+            ok = mbar_wait(&bars[1], par, kWait) && ok;
+            if (more) load_a1(nxt);
+        }
+        fence_proxy_async();
+        fence_before_sync();
+        __syncthreads();
+        if (issuer) {
+            fence_after_sync();
+            const uint64_t kP = desc_kmajor(smem_addr(sm + PA), 128, 0), kA = desc_kmajor(smem_addr(sm + PA + 8192), 128, 0),
+                           mP = desc_mnmajor(smem_addr(sm + PA), 64, 0), mA = desc_mnmajor(smem_addr(sm + PA + 8192), 64, 0),
+                           qb = desc_mnmajor(smem_addr(sm + RQ), 64, 0), kc = desc_mnmajor(smem_addr(sm + KC), 64, 0),
+                           kh = desc_mnmajor(smem_addr(sm + KH), 64, 0);
 #pragma unroll
-        for (int m = 0; m < 4; ++m)
-            *reinterpret_cast<float4 *>(sm + RG + sw128_chunk(4 * warp + m, lane, 64)) =
-                make_float4(x[m][0] + after[0], x[m][1] + after[1], x[m][2] + after[2], x[m][3] + after[3]);
-    }
-    fence_proxy_async();
-    fence_before_sync();
-    __syncthreads();
-    if (issuer) {
-        for (int x = 0; x < 2; ++x) {
-            tma_store_4d(&mdq, sm + RQ + x * 8192, 64 * x, h, c0, bb);
-            tma_store_4d(&mdk, sm + RK + x * 8192, 64 * x, h, c0, bb);
+            for (int ks = 0; ks < 4; ++ks) {
+                const uint64_t b_kh = kstep_mnmajor(kh, ks);
+                mma_bf16(tm + TM_Y1, kstep_kmajor(kP, 128, ks), b_kh, ID_KM128, 1);
+                mma_bf16(tm + TM_Y2, kstep_kmajor(kA, 128, ks), b_kh, ID_KM128, 1);
+                mma_bf16(tm + TM_Y3, kstep_mnmajor(mP, ks), kstep_mnmajor(qb, ks), ID_MM128, 1);
+                mma_bf16(tm + TM_Y3, kstep_mnmajor(mA, ks), kstep_mnmajor(kc, ks), ID_MM128, 1);
+            }
+            mma_commit(&bars[2]);
         }
-        for (int x = 0; x < 4; ++x) {
-            tma_store_4d(&mdb, sm + RB + x * 8192, 32 * x, h, c0, bb);
-            tma_store_4d(&mdg, sm + RG + x * 8192, 32 * x, h, c0, bb);
+        // ---------------- dq, dk, db, dG per (row, channel), from tensor memory.
+        // The M = 64 accumulators hold row quarter * 16 + l in lane l < 16; each
+        // 16-channel group is split by shuffles: lane l keeps channels 0..7 of
+        // row l, lane l + 16 takes channels 8..15 of the same row.
+        if (compute) {
+            ok = mbar_wait(&bars[2], par, kWait) && ok;
+            fence_after_sync();
+            const int r = quarter * 16 + (lane & 15), hi = lane >> 4;
+#pragma unroll 1
+            for (int g2 = 0; g2 < 2; ++g2) {
+                const int ch0 = 32 * cgrp + 16 * g2, ch = ch0 + 8 * hi;
+                float y1[16], y2[16], y3[16];
+                tmem_ld16(taddr(tm + TM_Y1 + ch0, quarter * 32, 0), y1);
+                tmem_ld16(taddr(tm + TM_Y2 + ch0, quarter * 32, 0), y2);
+                tmem_ld16(taddr(tm + TM_Y3 + ch0, quarter * 32, 0), y3);
+                tmem_wait_ld();
+                float a1[8], a2[8], a3[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float s1 = __shfl_sync(0xffffffffu, y1[8 + i], lane & 15);
+                    const float s2 = __shfl_sync(0xffffffffu, y2[8 + i], lane & 15);
+                    const float s3 = __shfl_sync(0xffffffffu, y3[8 + i], lane & 15);
+                    a1[i] = hi ? s1 : y1[i];
+                    a2[i] = hi ? s2 : y2[i];
+                    a3[i] = hi ? s3 : y3[i];
+                }
+                const uint32_t o16 = sw128_chunk(r, ch >> 3, 64);
+                const uint32_t o32a = sw128_chunk(r, ch >> 2, 64), o32b = sw128_chunk(r, (ch >> 2) + 1, 64);
+                const uint4 qbr = *reinterpret_cast<const uint4 *>(sm + RQ + o16);
+                const uint4 kcr2 = *reinterpret_cast<const uint4 *>(sm + KC + o16);
+                const uint4 khr2 = *reinterpret_cast<const uint4 *>(sm + KH + o16);
+                const uint4 kr2 = *reinterpret_cast<const uint4 *>(sm + RK + o16);
+                const uint4 e2 = *reinterpret_cast<const uint4 *>(sm + TE + o16);
+                const uint4 ei2 = *reinterpret_cast<const uint4 *>(sm + TEI + o16);
+                const float4 b0 = *reinterpret_cast<const float4 *>(sm + RB + o32a);
+                const float4 b1 = *reinterpret_cast<const float4 *>(sm + RB + o32b);
+                float qb[8], kc[8], kh[8], kf[8], E[8], Ei[8];
+                {
+                    const __half2 *x1 = reinterpret_cast<const __half2 *>(&qbr);
+                    const __half2 *x2 = reinterpret_cast<const __half2 *>(&kcr2);
+                    const __half2 *x3 = reinterpret_cast<const __half2 *>(&khr2);
+                    const __half2 *x4 = reinterpret_cast<const __half2 *>(&e2);
+                    const __half2 *x5 = reinterpret_cast<const __half2 *>(&ei2);
+                    const __nv_bfloat162 *x6 = reinterpret_cast<const __nv_bfloat162 *>(&kr2);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        qb[2 * e] = __low2float(x1[e]); qb[2 * e + 1] = __high2float(x1[e]);
+                        kc[2 * e] = __low2float(x2[e]); kc[2 * e + 1] = __high2float(x2[e]);
+                        kh[2 * e] = __low2float(x3[e]); kh[2 * e + 1] = __high2float(x3[e]);
+                        E[2 * e] = __low2float(x4[e]); E[2 * e + 1] = __high2float(x4[e]);
+                        Ei[2 * e] = __low2float(x5[e]); Ei[2 * e + 1] = __high2float(x5[e]);
+                        kf[2 * e] = __low2float(x6[e]); kf[2 * e + 1] = __high2float(x6[e]);
+                    }
+                }
+                const float bf[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+                float dq[8], dk[8], db[8], dG[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float dkc = a2[i] * E[i], dkh = a3[i] * Ei[i];
+                    dq[i] = a1[i] * E[i];
+                    db[i] = dkc * kf[i];
+                    dk[i] = dkc * bf[i] + dkh;
+                    dG[i] = a1[i] * qb[i] + a2[i] * kc[i] - a3[i] * kh[i];
+                }
+                st_bf16x8(sm + RQ + o16, dq);
+                st_bf16x8(sm + RK + o16, dk);
+                *reinterpret_cast<float4 *>(sm + RB + o32a) = make_float4(db[0], db[1], db[2], db[3]);
+                *reinterpret_cast<float4 *>(sm + RB + o32b) = make_float4(db[4], db[5], db[6], db[7]);
+                *reinterpret_cast<float4 *>(sm + RG + o32a) = make_float4(dG[0], dG[1], dG[2], dG[3]);
+                *reinterpret_cast<float4 *>(sm + RG + o32b) = make_float4(dG[4], dG[5], dG[6], dG[7]);
+            }
         }
-        bulk_commit();
-        bulk_wait_all();
+        fence_proxy_async();
+        fence_before_sync();
+        __syncthreads();
+        if (issuer) {
+            if (more) load_a2(nxt);  // Kh, Kc, E, 1/E, dP, dA are consumed
+            for (int x = 0; x < 2; ++x) {
+                tma_store_4d(&mdq, sm + RQ + x * 8192, 64 * x, h, c0, bb);
+                tma_store_4d(&mdk, sm + RK + x * 8192, 64 * x, h, c0, bb);
+            }
+            for (int x = 0; x < 4; ++x) tma_store_4d(&mdb, sm + RB + x * 8192, 32 * x, h, c0, bb);
+            bulk_commit();
+        }
+        // ---------------- dg: reverse in-chunk cumsum of dG with the chunk-end term
+        if (compute) {
+            float run[4] = {0.f, 0.f, 0.f, 0.f}, x[4][4];
+#pragma unroll
+            for (int m = 3; m >= 0; --m) {
+                const float4 t = *reinterpret_cast<const float4 *>(sm + RG + sw128_chunk(4 * warp + m, lane, 64));
+                run[0] += t.x; run[1] += t.y; run[2] += t.z; run[3] += t.w;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) x[m][i] = run[i];
+            }
+            *reinterpret_cast<float4 *>(scan + warp * 128 + 4 * lane) = make_float4(run[0], run[1], run[2], run[3]);
+            named_sync(1, kCompute);
+            if (tid < 128) {  // per channel: the end term plus the later warps' totals, in place
+                float acc = sEnd[tid];
+#pragma unroll
+                for (int w2 = kWarps - 1; w2 >= 0; --w2) {
+                    const float t = scan[w2 * 128 + tid];
+                    scan[w2 * 128 + tid] = acc;
+                    acc += t;
+                }
+            }
+            named_sync(1, kCompute);
+            const float4 a4 = *reinterpret_cast<const float4 *>(scan + warp * 128 + 4 * lane);
+            const float after[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+            for (int m = 0; m < 4; ++m)
+                *reinterpret_cast<float4 *>(sm + RG + sw128_chunk(4 * warp + m, lane, 64)) =
+                    make_float4(x[m][0] + after[0], x[m][1] + after[1], x[m][2] + after[2], x[m][3] + after[3]);
+        }
+        fence_proxy_async();
+        fence_before_sync();
+        if (__syncthreads_or(!ok)) break;
+        if (issuer) {
+            for (int x = 0; x < 4; ++x) tma_store_4d(&mdg, sm + RG + x * 8192, 32 * x, h, c0, bb);
+            bulk_commit();
+            bulk_wait_read();  // the tiles may be refilled
+            if (more) load_b(nxt);
+        }
     }
+    if (issuer) bulk_wait_all();
     if (!(big <= kRange) || !(gbig <= 9.f)) record_status(status, GDN2_ERR_RANGE);
-    if (!ok && tid == 0) {
+    if (!ok && issuer) {
         record_status(status, GDN2_ERR_TIMEOUT);
-        // every issued product done before the tensor memory is freed
+        // every copy landed and every issued product done before the shared
+        // and tensor memory go away
+        if (issued[0] > 0) mbar_wait(&bars[0], (issued[0] - 1) & 1, kWait);
+        if (issued[2] > 0) mbar_wait(&bars[3], (issued[2] - 1) & 1, kWait);
         mbar_wait(&bars[1], 0, kWait);
+        mbar_wait(&bars[1], 1, kWait);
         mbar_wait(&bars[2], 0, kWait);
+        mbar_wait(&bars[2], 1, kWait);
     }
     fence_before_sync();
     __syncthreads();
@@ -841,7 +892,9 @@ cudaError_t tc_bwd_launch(const void *q, const void *k, const void *v, const flo
     launch_end(K_TC_BWD_STATE, s);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     launch_begin(K_TC_BWD_GRAD, s);
-    tc_bwd_grad_kernel<<<dim3(d.NC, d.H, d.B), tbg::kThreads, tbg::SMEM_BYTES, s>>>(
+    const long long ntiles = (long long)d.B * d.H * d.NC;
+    const int grid = (int)(ntiles < sm_count() ? ntiles : sm_count());
+    tc_bwd_grad_kernel<<<grid, tbg::kThreads, tbg::SMEM_BYTES, s>>>(
         mq, mk, mb, mg, mdo, mdq, mdk, mdb, mdg, (unsigned char *)ws, lay, status, d);
     launch_end(K_TC_BWD_GRAD, s);
     return cudaGetLastError();

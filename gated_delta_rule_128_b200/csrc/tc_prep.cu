@@ -302,17 +302,6 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
     if (warp == 0) tmem_dealloc(tm, 256);
 }
 
-static int sm_count() {
-    static int n = 0;
-    if (n == 0) {
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
-            n = 1;
-    }
-    return n;
-}
-
 cudaError_t tc_prep_launch(const void *q, const void *k, const float *g, const float *b, void *ws,
                            unsigned int *status, const Dims &d, cudaStream_t s) {
     CUtensorMap mq, mk, mg, mb;
