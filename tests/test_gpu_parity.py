@@ -135,6 +135,41 @@ def test_small_grids(case, io):
     compare(gpu, ref, io, ("o", "ST") + GRADS)
 
 
+# The tensor-core path (bf16, d = 128, chunk 64): one and two chunks, a ragged
+# tail, more tiles than SMs with one chunk each, and several tiles per
+# persistent CTA; non-zero S0 and dS_T throughout.
+TC_CASES = [
+    # B, T, H
+    (1, 64, 1),
+    (1, 128, 1),
+    (1, 127, 3),
+    (2, 64, 80),
+    (3, 700, 11),
+]
+
+
+@pytest.mark.parametrize("case", TC_CASES, ids=lambda c: "B{}T{}H{}".format(*c))
+def test_tensor_core_path_tiles(case):
+    B, T, H = case
+    x = workloads.draw(B, T, H, 128, 128, 700 + T + H, s0_std=0.3, with_dST=True)
+    gpu = gpu_fwd_bwd(x, "bf16", 64)
+    ref = oracle_fwd_bwd(x, "bf16")
+    compare(gpu, ref, "bf16", ("o", "ST") + GRADS)
+
+
+def test_forward_only_workspace_gives_the_same_outputs():
+    """A workspace sized for the forward alone (chunk records only) and one
+    sized for the backward run the same products: o and S_T agree bit for bit."""
+    x = workloads.draw(2, 300, 3, 128, 128, 94, s0_std=0.2, with_dO=False)
+    d = to_device(x, "bf16")
+    o1, ST1, ws1 = gdn.forward(*(d[n] for n in NAMES), chunk=64, for_bwd=False)
+    o2, ST2, ws2 = gdn.forward(*(d[n] for n in NAMES), chunk=64, for_bwd=True)
+    torch.cuda.synchronize()
+    assert ws1.numel() < ws2.numel()
+    assert gdn.gdn2_get_device_status() == 0
+    assert torch.equal(o1, o2) and torch.equal(ST1, ST2)
+
+
 def test_negative_eigenvalue_erase_range():
     x = workloads.draw(1, 150, 2, 64, 64, 77, erase_scale=2.0, s0_std=0.1, with_dST=True)
     for io in ("f32", "bf16"):
