@@ -98,7 +98,6 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
     const int NC = d.NC, H = d.H;
     const int quarter = warp & 3, half = warp >> 2;
     const int key = quarter * 32 + lane;
-    const int r16 = quarter * 16 + lane;  // row of an M = 64 accumulator (lanes 0..15)
     const size_t bh = (size_t)bb * H + h;
     const unsigned char *recs = ws + lay.rec + bh * NC * (size_t)REC_BYTES;
 
@@ -195,10 +194,17 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
         tmem_ld16(taddr(tm + TM_DU, quarter * 32, 32 * half), du);
         tmem_ld16(taddr(tm + TM_DU, quarter * 32, 32 * half + 16), du + 16);
         tmem_wait_ld();
-        if (lane < 16) {
-            const int r = r16;
+        {
+            // lanes 0..15 hold the rows; lane l + 16 takes columns 16..31 of row l
+            const int r = quarter * 16 + (lane & 15), hi = lane >> 4;
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {  // v chunk 4 * half + jj: 8 columns
+            for (int j = 0; j < 16; ++j) {
+                const float t = __shfl_sync(0xffffffffu, du[16 + j], lane & 15);
+                if (hi) du[j] = t;
+            }
+#pragma unroll
+            for (int j2 = 0; j2 < 2; ++j2) {  // v chunk 4 * half + jj: 8 columns
+                const int jj = 2 * hi + j2;
                 unsigned char *pv = sm + VV + sw128_chunk(r, 4 * half + jj, 64);
                 const uint4 vq = *reinterpret_cast<const uint4 *>(pv);
                 const __nv_bfloat162 *v2 = reinterpret_cast<const __nv_bfloat162 *>(&vq);
@@ -206,7 +212,7 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
                 unsigned char *pw1 = sm + VW + half * 8192 + sw128_chunk(r, 2 * jj + 1, 64);
                 const float4 w0 = *reinterpret_cast<const float4 *>(pw0);
                 const float4 w1 = *reinterpret_cast<const float4 *>(pw1);
-                const float *u = du + 8 * jj;
+                const float *u = du + 8 * j2;
                 float dv8[8] = {u[0] * w0.x, u[1] * w0.y, u[2] * w0.z, u[3] * w0.w,
                                 u[4] * w1.x, u[5] * w1.y, u[6] * w1.z, u[7] * w1.w};
                 *reinterpret_cast<float4 *>(pw0) = make_float4(
@@ -218,11 +224,11 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
                 st_bf16x8(pv, dv8);
             }
 #pragma unroll
-            for (int j = 0; j < 32; ++j) du[j] = -du[j];
+            for (int j = 0; j < 16; ++j) du[j] = -du[j];
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                st_h8(sm + NDU + sw128_chunk(r, 4 * half + jj, 64), du + 8 * jj);
-                big = absmax8(du + 8 * jj, big);
+            for (int j2 = 0; j2 < 2; ++j2) {
+                st_h8(sm + NDU + sw128_chunk(r, 4 * half + 2 * hi + j2, 64), du + 8 * j2);
+                big = absmax8(du + 8 * j2, big);
             }
         }
         fence_proxy_async();
@@ -320,12 +326,16 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
             tmem_ld16(taddr(tm + TM_DD, quarter * 32, 32 * half), dd);
             tmem_ld16(taddr(tm + TM_DD, quarter * 32, 32 * half + 16), dd + 16);
             tmem_wait_ld();
-            if (lane < 16) {
+            const int hi = lane >> 4;  // lane l + 16 stores columns 16..31 of row l
 #pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                    st_h8(sm + OP_DD + sw128_chunk(r16, 4 * half + jj, 64), dd + 8 * jj);
-                    big = absmax8(dd + 8 * jj, big);
-                }
+            for (int j = 0; j < 16; ++j) {
+                const float t = __shfl_sync(0xffffffffu, dd[16 + j], lane & 15);
+                if (hi) dd[j] = t;
+            }
+#pragma unroll
+            for (int j2 = 0; j2 < 2; ++j2) {
+                st_h8(sm + OP_DD + sw128_chunk(quarter * 16 + (lane & 15), 4 * half + 2 * hi + j2, 64), dd + 8 * j2);
+                big = absmax8(dd + 8 * j2, big);
             }
         }
         fence_proxy_async();

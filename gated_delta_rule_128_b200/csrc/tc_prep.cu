@@ -268,15 +268,17 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
 #pragma unroll
             for (int j = 0; j < 4; ++j) tmem_ld16(taddr(tm + TM_W, quarter * 32, 64 * half + 16 * j), wv + 16 * j);
             tmem_wait_ld();
-            if (lane < 16) {
-                const int r = quarter * 16 + lane;
+            // lanes 0..15 hold the rows; lane l + 16 takes columns 32..63 of row l
+            const int r = quarter * 16 + (lane & 15), hi = lane >> 4;
 #pragma unroll
-                for (int j = 0; j < 64; ++j) wv[j] = -wv[j];
+            for (int j = 0; j < 32; ++j) {
+                const float t = __shfl_sync(0xffffffffu, wv[32 + j], lane & 15);
+                wv[j] = -(hi ? t : wv[j]);
+            }
 #pragma unroll
-                for (int jj = 0; jj < 8; ++jj) {
-                    st_h8(sm + OP_WQ + sw128_chunk(r, 8 * half + jj, 128), wv + 8 * jj);
-                    big = absmax8(wv + 8 * jj, big);
-                }
+            for (int j2 = 0; j2 < 4; ++j2) {
+                st_h8(sm + OP_WQ + sw128_chunk(r, 8 * half + 4 * hi + j2, 128), wv + 8 * j2);
+                big = absmax8(wv + 8 * j2, big);
             }
         }
         fence_proxy_async();
