@@ -45,7 +45,8 @@ using namespace tcc;
 
 // ============================================================ state kernel
 namespace tbs {
-constexpr int kThreads = 256;
+constexpr int kCompute = 256;            // warps 0..7: readouts, dU outputs, the next dX
+constexpr int kThreads = kCompute + 64;  // warp 8 issues the products; warp 9 the copies
 constexpr uint32_t STG = 0;                   // two chunk records, REC_BYTES each
 constexpr uint32_t RAW_DO = 2 * REC_BYTES;    // dO half, bf16 [64 pos][64]
 constexpr uint32_t OP_DO = RAW_DO + 8192;     // dO fp16      [64 pos][64 v]  MN-major B
@@ -75,7 +76,10 @@ static_assert(MISC % 1024 == 0, "alignment");
 // G_m)) dS_c.  dU is read while the next chunk's first products run: dv =
 // dU.w and dw = dU.v are formed in place of the v and w tiles (128-B
 // swizzled TMA tiles) and leave by TMA stores; -dU, dX and the chunk-end
-// half-sums go to the workspace for the gradient kernel.
+// half-sums go to the workspace for the gradient kernel.  Warps 0..7 read
+// the accumulators and form the operands and outputs; warp 8 issues the
+// products (an issuing thread is held for about as long as the products
+// run); warp 9 requests every copy, so that neither delays the readouts.
 __global__ void __launch_bounds__(tbs::kThreads, 1)
 tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_constant__ CUtensorMap mv,
                     const __grid_constant__ CUtensorMap mw, const __grid_constant__ CUtensorMap mdv,
@@ -96,7 +100,8 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int vh = blockIdx.x, h = blockIdx.y, bb = blockIdx.z, v0 = vh * 64;
     const int NC = d.NC, H = d.H;
-    const int quarter = warp & 3, half = warp >> 2;
+    const bool compute = tid < kCompute, issuer = tid == kCompute, copier = tid == kCompute + 32;
+    const int quarter = warp & 3, half = (warp >> 2) & 1;
     const int key = quarter * 32 + lane;
     const size_t bh = (size_t)bb * H + h;
     const unsigned char *recs = ws + lay.rec + bh * NC * (size_t)REC_BYTES;
@@ -114,8 +119,8 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
     fence_after_sync();
     const uint32_t tm = *tslot;
 
-    int issued[5] = {0, 0, 0, 0, 0};  // loads requested per barrier (thread 0)
-    int groups[3] = {0, 0, 0};        // commits to barriers 5, 6, 7 (thread 0)
+    int issued[5] = {0, 0, 0, 0, 0};  // loads requested per barrier (the copier)
+    int groups[3] = {0, 0, 0};        // commits to barriers 5, 6, 7 (the issuer)
     auto load_rec = [&](int cc) {
         const int s = cc & 1;
         mbar_expect_tx(&bars[s], REC_BYTES);
@@ -184,8 +189,8 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
         }
         return acc;
     };
-    // dU of chunk cc (TMEM) -> dv, dw in place of v, w; -dU staged; then the
-    // stores, and the next v, w tiles (chunk cc - 1).  All threads.
+    // dU of chunk cc (TMEM) -> dv, dw in place of v, w; -dU staged (compute
+    // threads; the copier stores them after the next barrier: store_du)
     auto flush_du = [&](int cc, uint32_t vw_par, uint32_t du_par) {
         bool fine = mbar_wait(&bars[7], du_par, kWait);
         fine = mbar_wait(&bars[4], vw_par, kWait) && fine;
@@ -232,20 +237,20 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
             }
         }
         fence_proxy_async();
-        __syncthreads();
-        if (tid == 0) {
-            tma_store_4d(&mdv, sm + VV, v0, h, cc * 64, bb);
-            tma_store_4d(&mdw, sm + VW, v0, h, cc * 64, bb);
-            tma_store_4d(&mdw, sm + VW + 8192, v0 + 32, h, cc * 64, bb);
-            bulk_store(ws + lay.ckndU + ((bh * NC + cc) * 2 + vh) * 8192, sm + NDU, 8192);
-            bulk_commit();
-            bulk_wait_read();  // VV, VW and NDU may be rewritten
-            if (cc > 0) load_vw(cc - 1);
-        }
         return fine;
     };
+    // the copier: dv, dw and -dU of chunk cc out, then the v, w tiles of chunk cc - 1
+    auto store_du = [&](int cc) {
+        tma_store_4d(&mdv, sm + VV, v0, h, cc * 64, bb);
+        tma_store_4d(&mdw, sm + VW, v0, h, cc * 64, bb);
+        tma_store_4d(&mdw, sm + VW + 8192, v0 + 32, h, cc * 64, bb);
+        bulk_store(ws + lay.ckndU + ((bh * NC + cc) * 2 + vh) * 8192, sm + NDU, 8192);
+        bulk_commit();
+        bulk_wait_read();  // VV, VW and NDU may be rewritten
+        if (cc > 0) load_vw(cc - 1);
+    };
 
-    if (tid == 0) {
+    if (copier) {
         load_rec(NC - 1);
         if (NC > 1) load_rec(NC - 2);
         load_do(NC - 1);
@@ -253,8 +258,8 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
         load_vw(NC - 1);
     }
     // ---------------- prologue: dS_T (or zero), the last chunk's end term and dX; dO
-    bool ok;
-    {
+    bool ok = true;
+    if (compute) {
         float x[32];
         const size_t so = st_off(d, bb, h);
 #pragma unroll
@@ -278,10 +283,10 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
     fence_before_sync();
     bool abort = __syncthreads_or(!ok);
     if (!abort) {
-        if (half == 0)
+        if (compute && half == 0)
             reinterpret_cast<float *>(ws + lay.ckEnd + ((bh * NC + NC - 1) * 2 + vh) * 512)[key] =
                 sEnd[key] + sEnd[128 + key];
-        if (tid == 0) {
+        if (copier) {
             fence_after_sync();
             bulk_store(ws + lay.ckdS + ((bh * NC + NC - 1) * 2 + vh) * 16384, sm + OP_DS, 16384);
             bulk_commit();
@@ -289,6 +294,7 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
                 load_s(NC - 1);
                 load_do(NC - 2);
             }
+            bulk_wait_read();  // the dX copy has left OP_DS
         }
     }
 
@@ -297,8 +303,8 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
         const uint32_t par = i & 1;
         unsigned char *stg = sm + STG + (c & 1) * REC_BYTES;
         // ---------------- (1) dDelta products, then Qb^T dO
-        ok = mbar_wait(&bars[c & 1], (i >> 1) & 1, kWait) && ok;  // record c
-        if (tid == 0) {
+        if (!copier) ok = mbar_wait(&bars[c & 1], (i >> 1) & 1, kWait) && ok;  // record c
+        if (issuer) {
             const uint32_t st = smem_addr(stg);
             // Qb is rows 64..127 of the [-W; Qb] tile: 64-key blocks 16 KB apart
             const uint64_t dP = desc_mnmajor(st + REC_P, 64, 0), dO = desc_mnmajor(smem_addr(sm + OP_DO), 64, 0),
@@ -317,11 +323,11 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
                 mma_bf16(tm + TM_DS, kstep_mnmajor(dQ, ks), kstep_mnmajor(dO, ks), ID_MM128x64, 1);
         }
         // the next chunk's dU, while these products run
-        if (c + 1 < NC) ok = flush_du(c + 1, (i - 1) & 1, (i - 1) & 1) && ok;
+        if (compute && c + 1 < NC) ok = flush_du(c + 1, (i - 1) & 1, (i - 1) & 1) && ok;
         // ---------------- dDelta to fp16, (2) products
-        ok = mbar_wait(&bars[5], par, kWait) && ok;
-        fence_after_sync();
-        {
+        if (compute) {
+            ok = mbar_wait(&bars[5], par, kWait) && ok;
+            fence_after_sync();
             float dd[32];
             tmem_ld16(taddr(tm + TM_DD, quarter * 32, 32 * half), dd);
             tmem_ld16(taddr(tm + TM_DD, quarter * 32, 32 * half + 16), dd + 16);
@@ -341,7 +347,8 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
         fence_proxy_async();
         fence_before_sync();
         __syncthreads();
-        if (tid == 0) {
+        if (copier && c + 1 < NC) store_du(c + 1);
+        if (issuer) {
             fence_after_sync();
             const uint32_t st = smem_addr(stg);
             const uint64_t dW = desc_mnmajor_lbo(st + REC_WQ, 16384, 0), dT = desc_mnmajor(st + REC_T, 64, 0),
@@ -356,9 +363,9 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
                 mma_bf16(tm + TM_DU, kstep_mnmajor(dT, ks), kstep_mnmajor(dD, ks), ID_MM64, ks > 0);
             mma_commit(&bars[7]);
             ++groups[2];
-            bulk_wait_read();  // the dX copy has left OP_DS
         }
         // ---------------- dS_c; the previous chunk's end term, dX and dO
+        if (compute) {
         ok = mbar_wait(&bars[6], par, kWait) && ok;
         if (c > 0) {
             ok = mbar_wait(&bars[3], (i + 1) & 1, kWait) && ok;                 // S_m of chunk c
@@ -392,14 +399,15 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
                 tmem_wait_st();
             }
         }
+        }
         fence_proxy_async();
         fence_before_sync();
         if (__syncthreads_or(!ok)) { abort = true; break; }
         if (c > 0) {
-            if (half == 0)
+            if (compute && half == 0)
                 reinterpret_cast<float *>(ws + lay.ckEnd + ((bh * NC + c - 1) * 2 + vh) * 512)[key] =
                     sEnd[key] + sEnd[128 + key];
-            if (tid == 0) {
+            if (copier) {
                 fence_after_sync();
                 bulk_store(ws + lay.ckdS + ((bh * NC + c - 1) * 2 + vh) * 16384, sm + OP_DS, 16384);
                 bulk_commit();
@@ -410,16 +418,22 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
                     if (!mbar_wait(&bars[7], par, kWait)) record_status(status, GDN2_ERR_TIMEOUT);
                     load_rec(c - 2);
                 }
+                bulk_wait_read();  // the dX copy has left OP_DS before it is rewritten
             }
         }
     }
-    if (!abort) ok = flush_du(0, (NC - 1) & 1, (NC - 1) & 1);
+    if (!abort && compute) ok = flush_du(0, (NC - 1) & 1, (NC - 1) & 1);
+    fence_before_sync();
+    const bool bad = __syncthreads_or(abort || !ok);
+    if (!bad && copier) store_du(0);
     if (!(big <= kRange)) record_status(status, GDN2_ERR_RANGE);
-    if (tid == 0) bulk_wait_all();
-    if (tid == 0 && (abort || !ok)) {
+    if (copier) bulk_wait_all();
+    if (bad && copier) {
         record_status(status, GDN2_ERR_TIMEOUT);
         for (int k2 = 0; k2 < 5; ++k2)
             if (issued[k2] > 0) mbar_wait(&bars[k2], (issued[k2] - 1) & 1, kWait);
+    }
+    if (bad && issuer) {
         for (int k2 = 0; k2 < 3; ++k2)
             if (groups[k2] > 0) mbar_wait(&bars[5 + k2], (groups[k2] - 1) & 1, kWait);
     }
