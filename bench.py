@@ -58,7 +58,7 @@ def parse():
     p.add_argument("--steps", type=int, default=50)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--e2e-steps", type=int, default=3)
+    p.add_argument("--e2e-steps", type=int, default=8)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-decode", action="store_true")
     p.add_argument("--batch", type=int, default=None,
@@ -182,11 +182,12 @@ def run_ours(args, rank, world, local_rank):
     io = gdn.GDN2_IO_BF16
     stream = torch.cuda.current_stream(dev)
 
-    def step(inp):
-        gdn.gdn2_fwd(*(inp[n] for n in NAMES), o, None, ws, ws.numel(), B, T, H, dk, dv, C, io,
-                     stream)
-        gdn.gdn2_bwd(*(inp[n] for n in NAMES), inp["dO"], None, grads["dq"], grads["dk"],
-                     grads["dv"], grads["dg"], grads["db"], grads["dw"], None, ws, ws.numel(), 1,
+    def step(inp, out=None):
+        out = out or dict(o=o, **grads)
+        gdn.gdn2_fwd(*(inp[n] for n in NAMES), out["o"], None, ws, ws.numel(), B, T, H, dk, dv, C,
+                     io, stream)
+        gdn.gdn2_bwd(*(inp[n] for n in NAMES), inp["dO"], None, out["dq"], out["dk"],
+                     out["dv"], out["dg"], out["db"], out["dw"], None, ws, ws.numel(), 1,
                      B, T, H, dk, dv, C, io, stream)
 
     barrier = gd.barrier
@@ -233,25 +234,48 @@ def run_ours(args, rank, world, local_rank):
     if status != 0:
         raise RuntimeError(f"device status {status} after the timed region")
 
-    # end-to-end through host buffers: H2D of the step's inputs, D2H of its outputs
-    host_out = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
-                for n, t in [("o", o)] + list(grads.items())}
+    # end-to-end through host buffers: every step copies its inputs H2D from
+    # pinned memory and its outputs D2H.  The input copies run on one stream,
+    # the step on the launch stream and the output copies on a third, with two
+    # sets of device buffers, so that step i's D2H overlaps step i+1's H2D
+    # (PCIe moves both directions at once).  The timed region spans the first
+    # H2D to the last D2H.
+    outs = [dict(o=torch.empty_like(o), **{n: torch.empty_like(t) for n, t in grads.items()})
+            for _ in range(2)]
+    host_out = [{n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for n, t in ob.items()}
+                for ob in outs]
     h2d = sum(t.numel() * t.element_size() for n, t in host.items() if n != "S0")
-    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
-    stage = {n: torch.empty_like(t) for n, t in d.items()}
+    d2h = sum(t.numel() * t.element_size() for t in host_out[0].values())
+    stage = [{n: (d[n] if n == "S0" else torch.empty_like(t)) for n, t in d.items()} for _ in range(2)]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()
+    ev_in, ev_done, ev_out = [ev(), ev()], [ev(), ev()], [ev(), ev()]
     barrier()
     torch.cuda.synchronize(dev)
     e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e_start.record(stream)
-    for _ in range(args.e2e_steps):
-        for n, t in host.items():
-            if n != "S0":
-                stage[n].copy_(t, non_blocking=True)
-        stage["S0"] = d["S0"]
-        step(stage)
-        host_out["o"].copy_(o, non_blocking=True)
-        for n, t in grads.items():
-            host_out[n].copy_(t, non_blocking=True)
+    s_in.wait_stream(stream)
+    s_out.wait_stream(stream)
+    for i in range(args.e2e_steps):
+        k = i % 2
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(ev_done[k])  # step i - 2 has read this stage
+            for n, t in host.items():
+                if n != "S0":
+                    stage[k][n].copy_(t, non_blocking=True)
+            ev_in[k].record(s_in)
+        stream.wait_event(ev_in[k])
+        if i >= 2:
+            stream.wait_event(ev_out[k])  # step i - 2's outputs have left these buffers
+        step(stage[k], outs[k])
+        ev_done[k].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_done[k])
+            for n, t in outs[k].items():
+                host_out[k][n].copy_(t, non_blocking=True)
+            ev_out[k].record(s_out)
+    stream.wait_stream(s_out)
     e_end.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = e_start.elapsed_time(e_end) / args.e2e_steps
@@ -306,7 +330,9 @@ def run_ours(args, rank, world, local_rank):
         "roofline_step": roofline_step,
         "kernels": kernels,
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
+                "copies": "pinned host buffers; H2D, step and D2H on three streams with two "
+                          "device buffer sets, step i's D2H overlapping step i+1's H2D"},
         "gpu_launches": launches,
         "clocks": clocks,
     }
