@@ -63,6 +63,8 @@ def parse():
     p.add_argument("--no-decode", action="store_true")
     p.add_argument("--batch", type=int, default=None,
                    help="override B (smaller cases for profiling captures only)")
+    p.add_argument("--workload", type=int, choices=[2, 3], default=2,
+                   help="fwd+bwd workload: 2 = B4 T4096 (the default line), 3 = B1 T16384")
     return p.parse_args()
 
 
@@ -320,10 +322,11 @@ def run_ours(args, rank, world, local_rank):
         "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f16", "data": "synthetic (seeded workload generators)",
-        "config": {"workload": wl.name, "B": B, "T": T, "H": H, "d_k": dk, "d_v": dv,
+        "config": {"workload": wl.name if B == wl.B else f"{wl.name}, B overridden to {B}",
+                   "B": B, "T": T, "H": H, "d_k": dk, "d_v": dv,
                    "chunk": C, "io": "bf16 q/k/v/o/dO/dq/dk/dv, f32 g/b/w/state",
                    "global_batch": B * world, "seq_len": T, "parallelism": f"dp{world}",
-                   "l2": "inputs 0.67 GB per step (> 126 MB L2), no flush",
+                   "l2": f"inputs {h2d / 1e9:.2f} GB per step (> 126 MB L2), no flush",
                    "arithmetic": "fp16 tensor-core operands, fp32 accumulation and state"},
         "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
         "roofline": roofline,
@@ -474,7 +477,9 @@ def run_reference(args, rank, world):
 
 
 def main():
+    global WORKLOAD_INDEX
     args = parse()
+    WORKLOAD_INDEX = args.workload
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
