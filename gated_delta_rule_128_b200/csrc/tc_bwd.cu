@@ -457,8 +457,8 @@ constexpr uint32_t SMT = 147456;  // S_m [128 key][128 v] K-major (then Kh, Kc)
 constexpr uint32_t DXT = 180224;  // dX  [128 key][128 v] K-major (then [dP; dA])
 constexpr uint32_t KH = SMT, KC = SMT + 16384, PA = DXT;  // after the first products
 constexpr uint32_t TE = DXT + 16384, TEI = DL;              // E = e^(G - G_m), 1/E (fp16 [64][128])
-constexpr uint32_t MISC = 212992; // sEnd [128]; sRef [128]; scan [16][128]; mbarriers; slot
-constexpr uint32_t SMEM_BYTES = MISC + 1024 + 8192 + 128 + 1024;
+constexpr uint32_t MISC = 212992; // sEnd [2][256]; sRef [128]; scan [16][128]; mbarriers; slot
+constexpr uint32_t SMEM_BYTES = MISC + 2560 + 8192 + 128 + 1024;
 constexpr uint32_t LOAD_A = 114688;  // dO, -dU, Delta, S_m, dX (the first products' operands)
 constexpr uint32_t LOAD_B = 98304;   // raw q, k, b, g
 constexpr uint32_t TM_Y1 = 0, TM_Y2 = 128, TM_Y3 = 256, TM_PA = 384;  // 512 columns
@@ -505,12 +505,15 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
     extern __shared__ unsigned char smraw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smraw) + 1023) & ~static_cast<uintptr_t>(1023));
-    float *sEnd = reinterpret_cast<float *>(sm + MISC);        // chunk-end term per channel
-    float *sRef = reinterpret_cast<float *>(sm + MISC + 512);  // G of the middle row per channel
-    float *scan = reinterpret_cast<float *>(sm + MISC + 1024);  // per-warp totals [16][128]
-    // 0 first-product operands (two parts), 1, 2 products, 3 raw tiles
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + MISC + 1024 + 8192);
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + MISC + 1024 + 8192 + 64);
+    // chunk-end term per channel as the two d_v halves' partials [2][128],
+    // double-buffered by tile parity (copied in with Delta, S_m, dX)
+    float *sEnd2 = reinterpret_cast<float *>(sm + MISC);
+    float *sRef = reinterpret_cast<float *>(sm + MISC + 2048);  // G of the middle row per channel
+    float *scan = reinterpret_cast<float *>(sm + MISC + 2560);  // per-warp totals [16][128]
+    // 0 first-product operands (two parts), 1, 2 products, 3 raw tiles, 4 dO
+    // converted (one arrival per compute warp)
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + MISC + 2560 + 8192);
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + MISC + 2560 + 8192 + 64);
     float big = 0.f, gbig = 0.f;  // range checks: operand magnitude, |G - G_m|
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -526,6 +529,7 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
     if (issuer) {
         mbar_init(&bars[0], 2);
         for (int i = 1; i < 4; ++i) mbar_init(&bars[i], 1);
+        mbar_init(&bars[4], kWarps);
         mbar_fence_init();
     }
     fence_before_sync();
@@ -544,8 +548,9 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
         }
         ++issued[0];
     };
-    auto load_a2 = [&](int it) {  // Delta, S_m, dX
-        mbar_expect_tx(&bars[0], LOAD_A - 32768);
+    auto load_a2 = [&](int it, int pb) {  // Delta, S_m, dX and the chunk-end partials
+        mbar_expect_tx(&bars[0], LOAD_A - 32768 + 1024);
+        bulk_load(sEnd2 + 256 * pb, ws + lay.ckEnd + (size_t)it * 1024, 1024, &bars[0]);
         bulk_load(sm + DL, ws + lay.ckD + ((size_t)it * 2) * 8192, 16384, &bars[0]);
         bulk_load(sm + SMT, ws + lay.ckS + ((size_t)(it + it / NC) * 2) * 16384, 32768, &bars[0]);
         bulk_load(sm + DXT, ws + lay.ckdS + ((size_t)it * 2) * 16384, 32768, &bars[0]);
@@ -566,7 +571,7 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
     };
     if (issuer && (int)blockIdx.x < ntiles) {
         load_a1(blockIdx.x);
-        load_a2(blockIdx.x);
+        load_a2(blockIdx.x, 0);
         load_b(blockIdx.x);
     }
 
@@ -576,10 +581,6 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
         const uint32_t par = n & 1;
         const int nxt = it + (int)gridDim.x;
         const bool more = nxt < ntiles;
-        if (tid < 128) {
-            const float *e0 = reinterpret_cast<const float *>(ws + lay.ckEnd + ((size_t)it * 2) * 512);
-            sEnd[tid] = e0[tid] + e0[128 + tid];
-        }
         ok = mbar_wait(&bars[0], par, kWait) && ok;
 
         // ---------------- dO to fp16; then, while the first products run, the
@@ -599,11 +600,13 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
                 }
                 st_h8(p, x);
             }
+            // the issuer waits for this, the compute warps go on to the decay
+            fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[4]);
         }
-        fence_proxy_async();
-        fence_before_sync();
-        __syncthreads();
         if (issuer) {
+            ok = mbar_wait(&bars[4], par, kWait) && ok;
             fence_after_sync();
             const uint64_t dn = desc_kmajor(smem_addr(sm + DN), 128, 0), dl = desc_kmajor(smem_addr(sm + DL), 64, 0),
                            s = desc_kmajor(smem_addr(sm + SMT), 128, 0), dx = desc_kmajor(smem_addr(sm + DXT), 128, 0),
@@ -816,7 +819,7 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
         fence_before_sync();
         __syncthreads();
         if (issuer) {
-            if (more) load_a2(nxt);  // Kh, Kc, E, 1/E, dP, dA are consumed
+            if (more) load_a2(nxt, (n + 1) & 1);  // Kh, Kc, E, 1/E, dP, dA are consumed
             for (int x = 0; x < 2; ++x) {
                 tma_store_4d(&mdq, sm + RQ + x * 8192, 64 * x, h, c0, bb);
                 tma_store_4d(&mdk, sm + RK + x * 8192, 64 * x, h, c0, bb);
@@ -837,7 +840,7 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
             *reinterpret_cast<float4 *>(scan + warp * 128 + 4 * lane) = make_float4(run[0], run[1], run[2], run[3]);
             named_sync(1, kCompute);
             if (tid < 128) {  // per channel: the end term plus the later warps' totals, in place
-                float acc = sEnd[tid];
+                float acc = sEnd2[256 * par + tid] + sEnd2[256 * par + 128 + tid];
 #pragma unroll
                 for (int w2 = kWarps - 1; w2 >= 0; --w2) {
                     const float t = scan[w2 * 128 + tid];
