@@ -31,8 +31,9 @@
 //    (dDelta; then dS), with dU and its outputs off that path.  Writes dw,
 //    dv, dS0, and per chunk dS_m, -dU and the half-sums of the chunk-end
 //    term to the workspace.
-//  * tc_bwd_grad_kernel: one CTA per (b, h, chunk), all chunks in parallel,
-//    full d_v; five products, then three accumulations, then dq, dk, db, dg.
+//  * tc_bwd_grad_kernel: persistent, one CTA per SM walking the (b, h, chunk)
+//    tiles, all chunks in parallel, full d_v; five products, then three
+//    accumulations, then dq, dk, db, dg.
 
 #include "common.cuh"
 #include "tc.cuh"
