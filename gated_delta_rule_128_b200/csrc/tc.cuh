@@ -146,6 +146,34 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float *v) {
 #pragma unroll
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
+// 16 TMEM lanes x 16 columns (two 256-bit blocks), spread over the warp
+// without waste: thread t gets lane base + t/4 in v[0..1] and base + t/4 + 8
+// in v[2..3] (columns c + 2 (t % 4) and c + 2 (t % 4) + 1), then the same for
+// columns c + 8 + 2 (t % 4), + 1 in v[4..7] (checked on the device against
+// values stored with the 32x32b shape).  Reads an M = 64 accumulator, whose
+// rows occupy lanes 0..15 of each warp's quarter, with every thread busy.
+__device__ __forceinline__ void tmem_ld16x256x2(uint32_t taddr, float *v) {
+    uint32_t r[8];
+    asm volatile("tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                   "=r"(r[7])
+                 : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+// As tmem_ld16x256x2 for 32 columns: v[4j .. 4j+3] cover columns c + 8j +
+// 2 (t % 4), + 1 of the two lanes, j = 0..3.
+__device__ __forceinline__ void tmem_ld16x256x4(uint32_t taddr, float *v) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+          "=r"(r[15])
+        : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
 // store 16 consecutive 32-bit columns of this thread's TMEM lane
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float *v) {
     asm volatile(

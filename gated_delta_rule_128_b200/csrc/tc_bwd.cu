@@ -196,45 +196,25 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
         bool fine = mbar_wait(&bars[7], du_par, kWait);
         fine = mbar_wait(&bars[4], vw_par, kWait) && fine;
         fence_after_sync();
-        float du[32];
-        tmem_ld16(taddr(tm + TM_DU, quarter * 32, 32 * half), du);
-        tmem_ld16(taddr(tm + TM_DU, quarter * 32, 32 * half + 16), du + 16);
+        float du[16];
+        tmem_ld16x256x4(taddr(tm + TM_DU, quarter * 32, 32 * half), du);
         tmem_wait_ld();
         {
-            // lanes 0..15 hold the rows; lane l + 16 takes columns 16..31 of row l
-            const int r = quarter * 16 + (lane & 15), hi = lane >> 4;
+            // 16x256b: rows quarter * 16 + t/4 and + 8, column pairs 32 * half +
+            // 8 jb + 2 (t % 4); dv, dw in place of v, w and -dU, pair by pair
+            const int rA = quarter * 16 + (lane >> 2), cp0 = 32 * half + 2 * (lane & 3);
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const float t = __shfl_sync(0xffffffffu, du[16 + j], lane & 15);
-                if (hi) du[j] = t;
-            }
-#pragma unroll
-            for (int j2 = 0; j2 < 2; ++j2) {  // v chunk 4 * half + jj: 8 columns
-                const int jj = 2 * hi + j2;
-                unsigned char *pv = sm + VV + sw128_chunk(r, 4 * half + jj, 64);
-                const uint4 vq = *reinterpret_cast<const uint4 *>(pv);
-                const __nv_bfloat162 *v2 = reinterpret_cast<const __nv_bfloat162 *>(&vq);
-                unsigned char *pw0 = sm + VW + half * 8192 + sw128_chunk(r, 2 * jj, 64);
-                unsigned char *pw1 = sm + VW + half * 8192 + sw128_chunk(r, 2 * jj + 1, 64);
-                const float4 w0 = *reinterpret_cast<const float4 *>(pw0);
-                const float4 w1 = *reinterpret_cast<const float4 *>(pw1);
-                const float *u = du + 8 * j2;
-                float dv8[8] = {u[0] * w0.x, u[1] * w0.y, u[2] * w0.z, u[3] * w0.w,
-                                u[4] * w1.x, u[5] * w1.y, u[6] * w1.z, u[7] * w1.w};
-                *reinterpret_cast<float4 *>(pw0) = make_float4(
-                    u[0] * __low2float(v2[0]), u[1] * __high2float(v2[0]), u[2] * __low2float(v2[1]),
-                    u[3] * __high2float(v2[1]));
-                *reinterpret_cast<float4 *>(pw1) = make_float4(
-                    u[4] * __low2float(v2[2]), u[5] * __high2float(v2[2]), u[6] * __low2float(v2[3]),
-                    u[7] * __high2float(v2[3]));
-                st_bf16x8(pv, dv8);
-            }
-#pragma unroll
-            for (int j = 0; j < 16; ++j) du[j] = -du[j];
-#pragma unroll
-            for (int j2 = 0; j2 < 2; ++j2) {
-                st_h8(sm + NDU + sw128_chunk(r, 4 * half + 2 * hi + j2, 64), du + 8 * j2);
-                big = absmax8(du + 8 * j2, big);
+            for (int p = 0; p < 8; ++p) {
+                const int rr = rA + 8 * (p & 1), jb = p >> 1, c = cp0 + 8 * jb;
+                const float u0 = du[4 * jb + 2 * (p & 1)], u1 = du[4 * jb + 2 * (p & 1) + 1];
+                unsigned char *pv = sm + VV + sw128_off(rr, c, 64);
+                unsigned char *pw = sm + VW + (c >> 5) * 8192 + sw128_chunk(rr, (c & 31) >> 2, 64) + (c & 3) * 4;
+                const float2 vf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(pv));
+                const float2 wf = *reinterpret_cast<const float2 *>(pw);
+                *reinterpret_cast<uint32_t *>(pv) = pack_bf16(u0 * wf.x, u1 * wf.y);
+                *reinterpret_cast<float2 *>(pw) = make_float2(u0 * vf.x, u1 * vf.y);
+                *reinterpret_cast<uint32_t *>(sm + NDU + sw128_off(rr, c, 64)) = pack_f16(-u0, -u1);
+                big = fmaxf(big, fmaxf(fabsf(u0), fabsf(u1)));
             }
         }
         fence_proxy_async();
@@ -329,20 +309,16 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
         if (compute) {
             ok = mbar_wait(&bars[5], par, kWait) && ok;
             fence_after_sync();
-            float dd[32];
-            tmem_ld16(taddr(tm + TM_DD, quarter * 32, 32 * half), dd);
-            tmem_ld16(taddr(tm + TM_DD, quarter * 32, 32 * half + 16), dd + 16);
+            float dd[16];
+            tmem_ld16x256x4(taddr(tm + TM_DD, quarter * 32, 32 * half), dd);
             tmem_wait_ld();
-            const int hi = lane >> 4;  // lane l + 16 stores columns 16..31 of row l
+            const int rA = quarter * 16 + (lane >> 2), cp0 = 32 * half + 2 * (lane & 3);
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const float t = __shfl_sync(0xffffffffu, dd[16 + j], lane & 15);
-                if (hi) dd[j] = t;
-            }
-#pragma unroll
-            for (int j2 = 0; j2 < 2; ++j2) {
-                st_h8(sm + OP_DD + sw128_chunk(quarter * 16 + (lane & 15), 4 * half + 2 * hi + j2, 64), dd + 8 * j2);
-                big = absmax8(dd + 8 * j2, big);
+            for (int p = 0; p < 8; ++p) {  // 16x256b pairs, as in the dU flush
+                const int rr = rA + 8 * (p & 1), jb = p >> 1, c = cp0 + 8 * jb;
+                const float x0 = dd[4 * jb + 2 * (p & 1)], x1 = dd[4 * jb + 2 * (p & 1) + 1];
+                *reinterpret_cast<uint32_t *>(sm + OP_DD + sw128_off(rr, c, 64)) = pack_f16(x0, x1);
+                big = fmaxf(big, fmaxf(fabsf(x0), fabsf(x1)));
             }
         }
         fence_proxy_async();
@@ -745,75 +721,53 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
             mma_commit(&bars[2]);
         }
         // ---------------- dq, dk, db, dG per (row, channel), from tensor memory.
-        // The M = 64 accumulators hold row quarter * 16 + l in lane l < 16; each
-        // 16-channel group is split by shuffles: lane l keeps channels 0..7 of
-        // row l, lane l + 16 takes channels 8..15 of the same row.
+        // The M = 64 accumulators hold row quarter * 16 + l in lane l < 16; the
+        // 16x256b loads give each thread two rows x two column pairs of every
+        // 16-channel group.
         if (compute) {
             ok = mbar_wait(&bars[2], par, kWait) && ok;
             fence_after_sync();
-            const int r = quarter * 16 + (lane & 15), hi = lane >> 4;
+            // 16x256b loads: thread t holds rows q16 + t/4 and q16 + t/4 + 8, column
+            // pairs 2 (t % 4) and 8 + 2 (t % 4) of each 16-column group
+            const int rA = quarter * 16 + (lane >> 2), cp0 = 2 * (lane & 3);
 #pragma unroll 1
             for (int g2 = 0; g2 < 2; ++g2) {
-                const int ch0 = 32 * cgrp + 16 * g2, ch = ch0 + 8 * hi;
-                float y1[16], y2[16], y3[16];
-                tmem_ld16(taddr(tm + TM_Y1 + ch0, quarter * 32, 0), y1);
-                tmem_ld16(taddr(tm + TM_Y2 + ch0, quarter * 32, 0), y2);
-                tmem_ld16(taddr(tm + TM_Y3 + ch0, quarter * 32, 0), y3);
+                const int ch0 = 32 * cgrp + 16 * g2;
+                float y1[8], y2[8], y3[8];
+                tmem_ld16x256x2(taddr(tm + TM_Y1 + ch0, quarter * 32, 0), y1);
+                tmem_ld16x256x2(taddr(tm + TM_Y2 + ch0, quarter * 32, 0), y2);
+                tmem_ld16x256x2(taddr(tm + TM_Y3 + ch0, quarter * 32, 0), y3);
                 tmem_wait_ld();
-                float a1[8], a2[8], a3[8];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float s1 = __shfl_sync(0xffffffffu, y1[8 + i], lane & 15);
-                    const float s2 = __shfl_sync(0xffffffffu, y2[8 + i], lane & 15);
-                    const float s3 = __shfl_sync(0xffffffffu, y3[8 + i], lane & 15);
-                    a1[i] = hi ? s1 : y1[i];
-                    a2[i] = hi ? s2 : y2[i];
-                    a3[i] = hi ? s3 : y3[i];
-                }
-                const uint32_t o16 = sw128_chunk(r, ch >> 3, 64);
-                const uint32_t o32a = sw128_chunk(r, ch >> 2, 64), o32b = sw128_chunk(r, (ch >> 2) + 1, 64);
-                const uint4 qbr = *reinterpret_cast<const uint4 *>(sm + RQ + o16);
-                const uint4 kcr2 = *reinterpret_cast<const uint4 *>(sm + KC + o16);
-                const uint4 khr2 = *reinterpret_cast<const uint4 *>(sm + KH + o16);
-                const uint4 kr2 = *reinterpret_cast<const uint4 *>(sm + RK + o16);
-                const uint4 e2 = *reinterpret_cast<const uint4 *>(sm + TE + o16);
-                const uint4 ei2 = *reinterpret_cast<const uint4 *>(sm + TEI + o16);
-                const float4 b0 = *reinterpret_cast<const float4 *>(sm + RB + o32a);
-                const float4 b1 = *reinterpret_cast<const float4 *>(sm + RB + o32b);
-                float qb[8], kc[8], kh[8], kf[8], E[8], Ei[8];
-                {
-                    const __half2 *x1 = reinterpret_cast<const __half2 *>(&qbr);
-                    const __half2 *x2 = reinterpret_cast<const __half2 *>(&kcr2);
-                    const __half2 *x3 = reinterpret_cast<const __half2 *>(&khr2);
-                    const __half2 *x4 = reinterpret_cast<const __half2 *>(&e2);
-                    const __half2 *x5 = reinterpret_cast<const __half2 *>(&ei2);
-                    const __nv_bfloat162 *x6 = reinterpret_cast<const __nv_bfloat162 *>(&kr2);
+                for (int p = 0; p < 4; ++p) {  // (row, column pair): p & 1 picks the row, p >> 1 the pair
+                    const int rr = rA + 8 * (p & 1), c = ch0 + cp0 + 8 * (p >> 1);
+                    const int ri = 2 * (p & 1) + 4 * (p >> 1);  // register index of the pair
+                    const uint32_t o16 = sw128_off(rr, c, 64);
+                    const uint32_t o32 = sw128_chunk(rr, c >> 2, 64) + (c & 3) * 4;
+                    const float2 qb = __half22float2(*reinterpret_cast<const __half2 *>(sm + RQ + o16));
+                    const float2 kc = __half22float2(*reinterpret_cast<const __half2 *>(sm + KC + o16));
+                    const float2 kh = __half22float2(*reinterpret_cast<const __half2 *>(sm + KH + o16));
+                    const float2 E = __half22float2(*reinterpret_cast<const __half2 *>(sm + TE + o16));
+                    const float2 Ei = __half22float2(*reinterpret_cast<const __half2 *>(sm + TEI + o16));
+                    const float2 kf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(sm + RK + o16));
+                    const float2 bf = *reinterpret_cast<const float2 *>(sm + RB + o32);
+                    const float a1[2] = {y1[ri], y1[ri + 1]}, a2[2] = {y2[ri], y2[ri + 1]}, a3[2] = {y3[ri], y3[ri + 1]};
+                    const float qv[2] = {qb.x, qb.y}, kcv[2] = {kc.x, kc.y}, khv[2] = {kh.x, kh.y};
+                    const float Ev[2] = {E.x, E.y}, Eiv[2] = {Ei.x, Ei.y}, kv[2] = {kf.x, kf.y}, bv[2] = {bf.x, bf.y};
+                    float dq[2], dk[2], db[2], dG[2];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        qb[2 * e] = __low2float(x1[e]); qb[2 * e + 1] = __high2float(x1[e]);
-                        kc[2 * e] = __low2float(x2[e]); kc[2 * e + 1] = __high2float(x2[e]);
-                        kh[2 * e] = __low2float(x3[e]); kh[2 * e + 1] = __high2float(x3[e]);
-                        E[2 * e] = __low2float(x4[e]); E[2 * e + 1] = __high2float(x4[e]);
-                        Ei[2 * e] = __low2float(x5[e]); Ei[2 * e + 1] = __high2float(x5[e]);
-                        kf[2 * e] = __low2float(x6[e]); kf[2 * e + 1] = __high2float(x6[e]);
+                    for (int i = 0; i < 2; ++i) {
+                        const float dkc = a2[i] * Ev[i], dkh = a3[i] * Eiv[i];
+                        dq[i] = a1[i] * Ev[i];
+                        db[i] = dkc * kv[i];
+                        dk[i] = dkc * bv[i] + dkh;
+                        dG[i] = a1[i] * qv[i] + a2[i] * kcv[i] - a3[i] * khv[i];
                     }
+                    *reinterpret_cast<uint32_t *>(sm + RQ + o16) = pack_bf16(dq[0], dq[1]);
+                    *reinterpret_cast<uint32_t *>(sm + RK + o16) = pack_bf16(dk[0], dk[1]);
+                    *reinterpret_cast<float2 *>(sm + RB + o32) = make_float2(db[0], db[1]);
+                    *reinterpret_cast<float2 *>(sm + RG + o32) = make_float2(dG[0], dG[1]);
                 }
-                const float bf[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-                float dq[8], dk[8], db[8], dG[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float dkc = a2[i] * E[i], dkh = a3[i] * Ei[i];
-                    dq[i] = a1[i] * E[i];
-                    db[i] = dkc * kf[i];
-                    dk[i] = dkc * bf[i] + dkh;
-                    dG[i] = a1[i] * qb[i] + a2[i] * kc[i] - a3[i] * kh[i];
-                }
-                st_bf16x8(sm + RQ + o16, dq);
-                st_bf16x8(sm + RK + o16, dk);
-                *reinterpret_cast<float4 *>(sm + RB + o32a) = make_float4(db[0], db[1], db[2], db[3]);
-                *reinterpret_cast<float4 *>(sm + RB + o32b) = make_float4(db[4], db[5], db[6], db[7]);
-                *reinterpret_cast<float4 *>(sm + RG + o32a) = make_float4(dG[0], dG[1], dG[2], dG[3]);
-                *reinterpret_cast<float4 *>(sm + RG + o32b) = make_float4(dG[4], dG[5], dG[6], dG[7]);
             }
         }
         fence_proxy_async();
