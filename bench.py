@@ -149,12 +149,17 @@ def traffic_from_profiles(kernel_key: str, src_hash: str):
     return rec.get("dram_bytes_per_launch")
 
 
+# the files that make up the tensor-core kernels whose DRAM traffic
+# profiles/traffic.json records; the captured figures apply while these match
+TC_KERNEL_SOURCES = ("tc_prep.cu", "tc_fwd.cu", "tc_bwd.cu", "common.cuh", "tc.cuh", "tc_common.cuh",
+                     "tmap.cuh")
+
+
 def sources_hash() -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gated_delta_rule_128_b200", "csrc")
-    for n in sorted(os.listdir(csrc)):
-        if n.endswith((".cu", ".cuh")):
-            h.update(open(os.path.join(csrc, n), "rb").read())
+    for n in TC_KERNEL_SOURCES:
+        h.update(open(os.path.join(csrc, n), "rb").read())
     return h.hexdigest()
 
 

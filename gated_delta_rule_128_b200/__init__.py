@@ -63,6 +63,8 @@ def lib() -> ctypes.CDLL:
         L.gdn2_decode_step.restype = i
         L.gdn2_get_device_status.argtypes = [vp]
         L.gdn2_get_device_status.restype = i
+        L.gdn2_selftest_timeout.argtypes = [ctypes.c_longlong, vp]
+        L.gdn2_selftest_timeout.restype = i
         L.gdn2_status_string.argtypes = [i]
         L.gdn2_status_string.restype = ctypes.c_char_p
         L.gdn2_version.argtypes = []
@@ -146,6 +148,10 @@ def gdn2_decode_step(q, k, v, g, b, w, S, o, N, H, d_k, d_v, io, stream=None):
 
 def gdn2_get_device_status(stream=None) -> int:
     return int(lib().gdn2_get_device_status(_stream(stream)))
+
+
+def gdn2_selftest_timeout(limit_cycles: int = 2_000_000, stream=None) -> None:
+    _check("gdn2_selftest_timeout", lib().gdn2_selftest_timeout(int(limit_cycles), _stream(stream)))
 
 
 def gdn2_kernel_launches() -> int:

@@ -9,6 +9,7 @@
 #include <vector>
 
 #include "common.cuh"
+#include "tc.cuh"
 
 namespace gdn2 {
 
@@ -230,6 +231,26 @@ gdn2_status gdn2_decode_step(const void *q, const void *k, const void *v, const 
     if (st != GDN2_OK) return st;
     return cuda_status(decode_launch(q, k, v, g, b, w, S, o, N, H, d_k, d_v, io,
                                      (cudaStream_t)stream));
+}
+
+// One block, one waiting thread: an mbarrier that no copy or product will
+// complete, waited on with the same bounded wait the kernels use.
+static __global__ void selftest_timeout_kernel(unsigned int *status, long long limit) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        tc::mbar_init(&bar, 1);
+        tc::mbar_fence_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && !tc::mbar_wait(&bar, 0, limit)) record_status(status, GDN2_ERR_TIMEOUT);
+}
+
+gdn2_status gdn2_selftest_timeout(long long limit_cycles, gdn2_stream_t stream) {
+    unsigned int *st = status_word();
+    if (!st) return GDN2_ERR_CUDA;
+    const long long lim = limit_cycles < 1000 ? 1000 : (limit_cycles > 4000000000LL ? 4000000000LL : limit_cycles);
+    selftest_timeout_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(st, lim);
+    return cuda_status(cudaGetLastError());
 }
 
 gdn2_status gdn2_get_device_status(gdn2_stream_t stream) {

@@ -168,6 +168,16 @@ gdn2_status gdn2_fwd_noalloc(const void *q, const void *k, const void *v, const 
  * Returns GDN2_ERR_CUDA if the stream reports a CUDA error. */
 gdn2_status gdn2_get_device_status(gdn2_stream_t stream);
 
+/* Self-test of the bounded-wait path every kernel uses.  Enqueues one block
+ * on `stream` that waits on an mbarrier nothing will complete, gives up after
+ * about `limit_cycles` SM clocks (clamped to [1e3, 4e9]) and records
+ * GDN2_ERR_TIMEOUT in the device status word, as a kernel whose copy or
+ * product never arrives does.  No copy or product is in flight when it
+ * returns, and the context stays usable; the next gdn2_get_device_status
+ * reports the timeout and clears it.  Returns GDN2_ERR_CUDA if the launch
+ * fails.  Not tied to any entry in the pages. */
+gdn2_status gdn2_selftest_timeout(long long limit_cycles, gdn2_stream_t stream);
+
 /* Static, never NULL. */
 const char *gdn2_status_string(gdn2_status status);
 

@@ -289,3 +289,22 @@ def test_workload4_decode_sampled_every_step():
             S_s = np.stack([S[nn, hh].cpu().numpy() for nn, hh in pairs])
             worst_S = max(worst_S, rel(S_s, S_ref[0]))
     assert worst_o < TOL_BF16_OUT and worst_S < TOL_BF16_OUT, (worst_o, worst_S)
+
+
+# ------------------------------------------------------ bounded waits
+def test_bounded_wait_reports_timeout_and_context_stays_usable():
+    """A wait that nothing completes gives up, records GDN2_ERR_TIMEOUT in the
+    status word (read once, then cleared), and later calls still run and
+    still agree with the oracle."""
+    assert gdn.gdn2_get_device_status() == 0
+    gdn.gdn2_selftest_timeout(2_000_000)
+    assert gdn.gdn2_get_device_status() == 5          # GDN2_ERR_TIMEOUT
+    assert gdn.gdn2_get_device_status() == 0          # cleared by the read
+    x = workloads.draw(1, 70, 2, 64, 64, 31, s0_std=0.1, with_dO=False)
+    d = to_device(x, "f32")
+    o, ST, _ = gdn.forward(*(d[n] for n in ("q", "k", "v", "g", "b", "w", "S0")), chunk=64)
+    torch.cuda.synchronize()
+    assert gdn.gdn2_get_device_status() == 0
+    r = to_np64(x)
+    o_ref, S_ref = oracle.forward(r["q"], r["k"], r["v"], r["g"], r["b"], r["w"], r["S0"])
+    assert rel(o.cpu().numpy(), o_ref) < TOL_F32 and rel(ST.cpu().numpy(), S_ref) < TOL_F32
