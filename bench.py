@@ -358,9 +358,9 @@ def run_ours(args, rank, world, local_rank):
 
 def run_decode(args, rank, dev):
     """Recurrent decode, workload 4 (256 sequences x 16 heads, d = 128, bf16
-    q/k/v/o, f32 gates and state): 1024 consecutive steps timed with CUDA
-    events on the launch stream, inputs of 8 seeded steps cycled, state
-    resident in HBM."""
+    q/k/v/o, f32 gates and state): 1024 consecutive steps captured in one CUDA
+    graph and replayed on the stream the events are recorded on, inputs of 8
+    seeded steps cycled, state resident in HBM."""
     import torch
 
     import gated_delta_rule_128_b200 as gdn
@@ -387,20 +387,27 @@ def run_decode(args, rank, dev):
                                  dv, io, stream)
 
     nsteps = wl.decode_steps
-    run(16)  # warm-up
+    with torch.cuda.stream(stream):
+        run(16)  # warm-up, eager
     torch.cuda.synchronize(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    run(nsteps)
-    e1.record(stream)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        run(nsteps)
+    with torch.cuda.stream(stream):
+        graph.replay()  # warm-up replay
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        graph.replay()
+        e1.record(stream)
     torch.cuda.synchronize(dev)
     us = e0.elapsed_time(e1) * 1e3 / nsteps
+    del graph
     if gdn.gdn2_get_device_status() != 0:
         raise RuntimeError("device status reports an error after decode")
     per_head = 2 * dk * dv * 4 + (2 * dk + dv) * 2 + (2 * dk + dv) * 4 + dv * 2
     return {"workload": wl.name, "N": N, "H": H, "steps": nsteps,
             "us_per_step": us, "bytes_per_step": per_head * N * H,
-            "inputs": "8 seeded steps cycled; 1024 consecutive launches on one stream"}
+            "inputs": "8 seeded steps cycled; 1024 consecutive steps in one CUDA graph"}
 
 
 # -------------------------------------------------------------- oracle arm

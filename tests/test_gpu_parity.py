@@ -308,3 +308,40 @@ def test_bounded_wait_reports_timeout_and_context_stays_usable():
     r = to_np64(x)
     o_ref, S_ref = oracle.forward(r["q"], r["k"], r["v"], r["g"], r["b"], r["w"], r["S0"])
     assert rel(o.cpu().numpy(), o_ref) < TOL_F32 and rel(ST.cpu().numpy(), S_ref) < TOL_F32
+
+
+# ------------------------------------------------------ CUDA graph capture
+def test_decode_steps_capture_in_a_cuda_graph():
+    """Launches through the C ABI on a capturing stream are captured, not run:
+    the state is untouched after capture, and one replay of 16 captured decode
+    steps leaves it bit for bit where 16 eager steps do."""
+    N, H, dk, dv = 32, 4, 128, 128
+    S0 = workloads.decode_state(N, H, dk, dv, 11, 0.3).cuda()
+    x = workloads.decode_step_inputs(N, H, dk, dv, 11, 0)
+    d = {n: (t.to(torch.bfloat16) if n in ("q", "k", "v") else t).cuda() for n, t in x.items()}
+    o = torch.empty(N, H, dv, dtype=torch.bfloat16, device="cuda")
+    s = torch.cuda.Stream()
+
+    def run(S, n):
+        for _ in range(n):
+            gdn.gdn2_decode_step(d["q"], d["k"], d["v"], d["g"], d["b"], d["w"], S, o, N, H, dk, dv,
+                                 gdn.GDN2_IO_BF16, s)
+
+    Sw = S0.clone()
+    with torch.cuda.stream(s):
+        run(Sw, 1)
+    torch.cuda.synchronize()
+    Sg = S0.clone()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        run(Sg, 16)
+    torch.cuda.synchronize()
+    assert torch.equal(Sg, S0)
+    with torch.cuda.stream(s):
+        g.replay()
+    Se = S0.clone()
+    with torch.cuda.stream(s):
+        run(Se, 16)
+    torch.cuda.synchronize()
+    assert torch.equal(Sg, Se) and not torch.equal(Se, S0)
+    assert gdn.gdn2_get_device_status() == 0
