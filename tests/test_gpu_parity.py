@@ -345,3 +345,24 @@ def test_decode_steps_capture_in_a_cuda_graph():
     torch.cuda.synchronize()
     assert torch.equal(Sg, Se) and not torch.equal(Se, S0)
     assert gdn.gdn2_get_device_status() == 0
+
+
+# ------------------------------------------------------ tensor-core range check
+def test_tensor_core_path_reports_decay_out_of_range():
+    """A log-decay steep enough that e^(G - G_m) leaves fp16's range within a
+    chunk (here -0.5 per token and channel: |G - G_m| reaches 16 > 9) makes
+    the tensor-core kernels record GDN2_ERR_RANGE instead of silently
+    returning overflowed results; the word clears once read, and an in-range
+    call afterwards reports nothing."""
+    x = workloads.draw(1, 128, 2, 128, 128, 41, with_dO=False)
+    x["g"] = torch.full_like(x["g"], -0.5)
+    d = to_device(x, "bf16")
+    gdn.forward(*(d[n] for n in NAMES), chunk=64)
+    torch.cuda.synchronize()
+    assert gdn.gdn2_get_device_status() == 6          # GDN2_ERR_RANGE
+    assert gdn.gdn2_get_device_status() == 0
+    x2 = workloads.draw(1, 128, 2, 128, 128, 42, with_dO=False)
+    d2 = to_device(x2, "bf16")
+    gdn.forward(*(d2[n] for n in NAMES), chunk=64)
+    torch.cuda.synchronize()
+    assert gdn.gdn2_get_device_status() == 0
