@@ -390,24 +390,35 @@ def run_decode(args, rank, dev):
     with torch.cuda.stream(stream):
         run(16)  # warm-up, eager
     torch.cuda.synchronize(dev)
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=stream):
-        run(nsteps)
-    with torch.cuda.stream(stream):
-        graph.replay()  # warm-up replay
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # thread-local capture: other threads' CUDA calls (a process group's
+    # watchdog under torchrun) cannot invalidate it
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    how = "1024 consecutive steps in one CUDA graph"
+    try:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream, capture_error_mode="thread_local"):
+            run(nsteps)
+        with torch.cuda.stream(stream):
+            graph.replay()  # warm-up replay
+            e0.record(stream)
+            graph.replay()
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        del graph
+    except RuntimeError as err:
+        torch.cuda.synchronize(dev)
+        how = f"1024 consecutive launches on one stream (graph capture failed: {str(err)[:80]})"
         e0.record(stream)
-        graph.replay()
+        run(nsteps)
         e1.record(stream)
-    torch.cuda.synchronize(dev)
+        torch.cuda.synchronize(dev)
     us = e0.elapsed_time(e1) * 1e3 / nsteps
-    del graph
     if gdn.gdn2_get_device_status() != 0:
         raise RuntimeError("device status reports an error after decode")
     per_head = 2 * dk * dv * 4 + (2 * dk + dv) * 2 + (2 * dk + dv) * 4 + dv * 2
     return {"workload": wl.name, "N": N, "H": H, "steps": nsteps,
             "us_per_step": us, "bytes_per_step": per_head * N * H,
-            "inputs": "8 seeded steps cycled; 1024 consecutive steps in one CUDA graph"}
+            "inputs": "8 seeded steps cycled; " + how}
 
 
 # -------------------------------------------------------------- oracle arm
