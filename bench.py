@@ -63,8 +63,9 @@ def parse():
     p.add_argument("--no-decode", action="store_true")
     p.add_argument("--batch", type=int, default=None,
                    help="override B (smaller cases for profiling captures only)")
-    p.add_argument("--workload", type=int, choices=[2, 3], default=2,
-                   help="fwd+bwd workload: 2 = B4 T4096 (the default line), 3 = B1 T16384")
+    p.add_argument("--workload", type=int, choices=[1, 2, 3], default=2,
+                   help="2 = fwd+bwd B4 T4096 (the default line), 3 = fwd+bwd B1 T16384, "
+                        "1 = forward only B8 T2048 (a line of its own metric)")
     return p.parse_args()
 
 
@@ -421,6 +422,66 @@ def run_decode(args, rank, dev):
             "inputs": "8 seeded steps cycled; " + how}
 
 
+def run_forward_only(args, rank, world, local_rank):
+    """Workload 1: the forward alone (bf16 q/k/v/o, f32 gates and state, S0 ~
+    N(0, 0.02), B8 T2048 H16 d128 C64), device-timed per call; algorithmic
+    bytes are the forward's per token-head plus S0 read and S_T written."""
+    import torch
+
+    import gated_delta_rule_128_b200 as gdn
+    from gated_delta_rule_128_b200 import dist as gd
+    from gated_delta_rule_128_b200 import workloads
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = workloads.WORKLOADS[1]
+    B, T, H, dk, dv, C = args.batch or wl.B, wl.T, wl.H, wl.dk, wl.dv, wl.chunk
+    x = workloads.draw(B, T, H, dk, dv, gd.rank_seed(wl.seed, rank), s0_std=wl.s0_std,
+                       erase_scale=wl.erase_scale, with_dO=False)
+    d = {n: (t.to(torch.bfloat16) if n in ("q", "k", "v") else t).contiguous().to(dev)
+         for n, t in x.items()}
+    io = gdn.GDN2_IO_BF16
+    ws = gdn.workspace(B, T, H, dk, dv, C, io, False, dev)
+    o = torch.empty(B, T, H, dv, dtype=torch.bfloat16, device=dev)
+    ST = torch.empty(B, H, dk, dv, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        gdn.gdn2_fwd(*(d[n] for n in NAMES), o, ST, ws, ws.numel(), B, T, H, dk, dv, C, io, stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    gd.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    gdn.gdn2_set_kernel_timer(True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ktimes = gdn.gdn2_kernel_times()
+    gdn.gdn2_set_kernel_timer(False)
+    if gdn.gdn2_get_device_status(stream) != 0:
+        raise RuntimeError("device status reports an error after the timed region")
+    ms = gd.max_over_ranks([e0.elapsed_time(e1) / args.steps], dev)[0]
+    peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) \
+        if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")) else {}
+    peak = peaks.get("hbm_gbs", 6650.0)
+    alg = B * T * H * FWD_BYTES + 2 * B * H * dk * dv * 4
+    gbs = alg / (ms * 1e-3) / 1e9
+    return {
+        "metric": "GDR-2 fwd tokens/s (H16, dk=dv=128) and % of HBM roofline", "value": B * T * world / (ms * 1e-3),
+        "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup),
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f16", "data": "synthetic (seeded workload generators)",
+        "config": {"workload": wl.name, "B": B, "T": T, "H": H, "d_k": dk, "d_v": dv, "chunk": C},
+        "roofline_step": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                          "alg_bytes_per_step": alg},
+        "kernels": {k: {"launches": c, "avg_ms": t / c} for k, (c, t) in ktimes.items()},
+    }
+
+
 # -------------------------------------------------------------- oracle arm
 
 def oracle_sample(seconds_budget: float, nthreads: int):
@@ -513,6 +574,14 @@ def main():
         return
     from gated_delta_rule_128_b200 import dist as gd
     gd.init("nccl", gd.rank_info(), timeout_s=120)
+    if args.workload == 1:
+        try:
+            line = run_forward_only(args, rank, world, local_rank)
+            if rank == 0:
+                print(json.dumps(line), flush=True)
+        finally:
+            gd.shutdown()
+        return
     try:
         line = run_ours(args, rank, world, local_rank)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
