@@ -61,6 +61,8 @@ def parse():
     p.add_argument("--e2e-steps", type=int, default=8)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-decode", action="store_true")
+    p.add_argument("--no-sub", action="store_true",
+                   help="skip the workload 1 and 3 sub-objects of the default line")
     p.add_argument("--batch", type=int, default=None,
                    help="override B (smaller cases for profiling captures only)")
     p.add_argument("--workload", type=int, choices=[1, 2, 3], default=2,
@@ -164,83 +166,182 @@ def sources_hash() -> str:
     return h.hexdigest()
 
 
+def _peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    peaks = json.load(open(path)) if os.path.exists(path) else {}
+    return peaks.get("hbm_gbs", 6650.0), ("of measured" if "hbm_gbs" in peaks else "of fallback")
+
+
+def kernel_split(gdn, run_steps, steps, token_heads, peak, stream):
+    """Per-kernel device time from the library's event timer, taken in a pass
+    of its own (the timer records two events around every launch, so it is
+    never on while a headline number is timed)."""
+    import torch
+
+    torch.cuda.synchronize()
+    gdn.gdn2_set_kernel_timer(True)
+    run_steps(steps)
+    torch.cuda.synchronize()
+    ktimes = gdn.gdn2_kernel_times()
+    gdn.gdn2_set_kernel_timer(False)
+    kernels = {}
+    for name, (cnt, tot) in ktimes.items():
+        avg = tot / cnt
+        ent = {"launches": cnt, "avg_ms": avg}
+        per = KERNEL_BYTES.get(name)
+        if per is not None:
+            gbs = per * token_heads / (avg * 1e-3) / 1e9
+            ent.update(alg_bytes_per_launch=per * token_heads, achieved_gbs=gbs, frac=gbs / peak)
+        kernels[name] = ent
+    return kernels
+
+
+class FwdBwdCase:
+    """Device buffers and the fwd+bwd step of one workload shape (bf16 I/O,
+    float32 gates and state), inputs resident in HBM."""
+
+    def __init__(self, wl, B, seed, dev, with_bwd=True):
+        import torch
+
+        import gated_delta_rule_128_b200 as gdn
+        from gated_delta_rule_128_b200 import workloads
+
+        self.gdn, self.wl, self.dev = gdn, wl, dev
+        self.B, self.T, self.H, self.dk, self.dv, self.C = B, wl.T, wl.H, wl.dk, wl.dv, wl.chunk
+        self.with_bwd = with_bwd
+        x = workloads.draw(B, wl.T, wl.H, wl.dk, wl.dv, seed, s0_std=wl.s0_std,
+                           erase_scale=wl.erase_scale, with_dO=with_bwd)
+        bf = torch.bfloat16
+        io_names = ("q", "k", "v", "dO")
+        self.host = {n: (t.to(bf) if n in io_names else t).contiguous() for n, t in x.items()}
+        self.d = {n: t.to(dev) for n, t in self.host.items()}
+        self.io = gdn.GDN2_IO_BF16
+        self.ws = gdn.workspace(B, wl.T, wl.H, wl.dk, wl.dv, wl.chunk, self.io, with_bwd, dev)
+        self.o = torch.empty(B, wl.T, wl.H, wl.dv, dtype=bf, device=dev)
+        self.ST = None if with_bwd else torch.empty(B, wl.H, wl.dk, wl.dv, device=dev)
+        d = self.d
+        self.grads = dict(dq=torch.empty_like(d["q"]), dk=torch.empty_like(d["k"]),
+                          dv=torch.empty_like(d["v"]), dg=torch.empty_like(d["g"]),
+                          db=torch.empty_like(d["b"]), dw=torch.empty_like(d["w"])) if with_bwd else {}
+        self.stream = torch.cuda.current_stream(dev)
+
+    @property
+    def token_heads(self):
+        return self.B * self.T * self.H
+
+    def fwd(self, inp=None, out=None):
+        inp, out = inp or self.d, out or dict(o=self.o, **self.grads)
+        g = self.gdn
+        g.gdn2_fwd(*(inp[n] for n in NAMES), out["o"], self.ST, self.ws, self.ws.numel(), self.B,
+                   self.T, self.H, self.dk, self.dv, self.C, self.io, self.stream)
+
+    def bwd(self, inp=None, out=None):
+        inp, out = inp or self.d, out or dict(o=self.o, **self.grads)
+        self.gdn.gdn2_bwd(*(inp[n] for n in NAMES), inp["dO"], None, out["dq"], out["dk"],
+                          out["dv"], out["dg"], out["db"], out["dw"], None, self.ws,
+                          self.ws.numel(), 1, self.B, self.T, self.H, self.dk, self.dv, self.C,
+                          self.io, self.stream)
+
+    def step(self, inp=None, out=None):
+        self.fwd(inp, out)
+        if self.with_bwd:
+            self.bwd(inp, out)
+
+    def run(self, n):
+        for _ in range(n):
+            self.step()
+
+    def timed(self, steps, warmup, barrier=lambda: None):
+        """(ms per step, fwd ms, bwd ms, launches) over `steps` device-timed
+        steps after `warmup` untimed ones; the kernel timer is off."""
+        import torch
+
+        for _ in range(max(3, warmup)):
+            self.step()
+        torch.cuda.synchronize(self.dev)
+        if self.gdn.gdn2_get_device_status(self.stream) != 0:
+            raise RuntimeError("device status reports an error after warm-up")
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+               torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize(self.dev)
+        launches0 = self.gdn.gdn2_kernel_launches()
+        start.record(self.stream)
+        for i in range(steps):
+            e0, e1, e2 = ev[i]
+            e0.record(self.stream)
+            self.fwd()
+            e1.record(self.stream)
+            if self.with_bwd:
+                self.bwd()
+            e2.record(self.stream)
+        end.record(self.stream)
+        torch.cuda.synchronize(self.dev)
+        launches = self.gdn.gdn2_kernel_launches() - launches0
+        barrier()
+        if self.gdn.gdn2_get_device_status(self.stream) != 0:
+            raise RuntimeError("device status reports an error after the timed region")
+        fwd_ms = statistics.mean(a.elapsed_time(b) for a, b, _ in ev)
+        bwd_ms = statistics.mean(b.elapsed_time(c) for _, b, c in ev)
+        return start.elapsed_time(end) / steps, fwd_ms, bwd_ms, launches
+
+
+def sub_workload(index, args, rank, dev, peak, peak_src):
+    """A secondary workload of the default line (1: forward only B8 T2048;
+    3: fwd+bwd B1 T16384 with b in [0, 2]), device-timed like the headline."""
+    import torch
+
+    from gated_delta_rule_128_b200 import dist as gd
+    from gated_delta_rule_128_b200 import workloads
+
+    wl = workloads.WORKLOADS[index]
+    case = FwdBwdCase(wl, wl.B, gd.rank_seed(wl.seed, rank), dev, with_bwd=wl.backward)
+    steps = max(5, args.steps // 2)
+    ms, fwd_ms, bwd_ms, _ = case.timed(steps, args.warmup, gd.barrier)
+    kernels = kernel_split(case.gdn, case.run, steps, case.token_heads, peak, case.stream)
+    ms = gd.max_over_ranks([ms], dev)[0]
+    if wl.backward:
+        alg = case.token_heads * (FWD_BYTES + BWD_BYTES)
+    else:  # the forward's bytes per token-head plus S0 read and S_T written
+        alg = case.token_heads * FWD_BYTES + 2 * wl.B * wl.H * wl.dk * wl.dv * 4
+    gbs = alg / (ms * 1e-3) / 1e9
+    out = {"workload": wl.name, "ms_per_step": ms, "steps": steps,
+           "tokens_per_s": wl.B * wl.T / (ms * 1e-3),
+           "roofline_step": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
+                             "frac": gbs / peak, "alg_bytes_per_step": alg,
+                             "peak_source": peak_src},
+           "kernels": kernels}
+    if wl.backward:
+        out.update(fwd_ms=fwd_ms, bwd_ms=bwd_ms)
+    del case
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
 
     import gated_delta_rule_128_b200 as gdn
-    from gated_delta_rule_128_b200 import workloads
-
     from gated_delta_rule_128_b200 import dist as gd
+    from gated_delta_rule_128_b200 import workloads
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     wl = workloads.WORKLOADS[WORKLOAD_INDEX]
-    B, T, H, dk, dv, C = args.batch or wl.B, wl.T, wl.H, wl.dk, wl.dv, wl.chunk
-    x = workloads.draw(B, T, H, dk, dv, gd.rank_seed(wl.seed, rank), s0_std=wl.s0_std,
-                       erase_scale=wl.erase_scale)
-    io_names = ("q", "k", "v", "dO")
-    bf = torch.bfloat16
-    host = {n: (t.to(bf) if n in io_names else t).contiguous().pin_memory() for n, t in x.items()}
-    d = {n: t.to(dev) for n, t in host.items()}
-    ws = gdn.workspace(B, T, H, dk, dv, C, gdn.GDN2_IO_BF16, True, dev)
-    o = torch.empty(B, T, H, dv, dtype=bf, device=dev)
-    grads = dict(dq=torch.empty_like(d["q"]), dk=torch.empty_like(d["k"]),
-                 dv=torch.empty_like(d["v"]), dg=torch.empty_like(d["g"]),
-                 db=torch.empty_like(d["b"]), dw=torch.empty_like(d["w"]))
-    io = gdn.GDN2_IO_BF16
-    stream = torch.cuda.current_stream(dev)
-
-    def step(inp, out=None):
-        out = out or dict(o=o, **grads)
-        gdn.gdn2_fwd(*(inp[n] for n in NAMES), out["o"], None, ws, ws.numel(), B, T, H, dk, dv, C,
-                     io, stream)
-        gdn.gdn2_bwd(*(inp[n] for n in NAMES), inp["dO"], None, out["dq"], out["dk"],
-                     out["dv"], out["dg"], out["db"], out["dw"], None, ws, ws.numel(), 1,
-                     B, T, H, dk, dv, C, io, stream)
-
-    barrier = gd.barrier
+    B = args.batch or wl.B
+    case = FwdBwdCase(wl, B, gd.rank_seed(wl.seed, rank), dev)
+    T, H, dk, dv = wl.T, wl.H, wl.dk, wl.dv
+    peak, peak_src = _peak()
+    host = {n: t.pin_memory() for n, t in case.host.items()}
 
     sampler = ClockSampler(local_rank)
     sampler.start()
-    for _ in range(max(3, args.warmup)):
-        step(d)
-    torch.cuda.synchronize(dev)
-    if gdn.gdn2_get_device_status(stream) != 0:
-        raise RuntimeError("device status reports an error after warm-up")
-
-    # device-timed region: K steps, per-call events on the launching stream
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
-    torch.cuda.synchronize(dev)
-    launches0 = gdn.gdn2_kernel_launches()
-    gdn.gdn2_set_kernel_timer(True)
     sampler.mark_start()
-    start.record(stream)
-    for i in range(args.steps):
-        e0, e1, e2 = ev[i]
-        e0.record(stream)
-        gdn.gdn2_fwd(*(d[n] for n in NAMES), o, None, ws, ws.numel(), B, T, H, dk, dv, C, io,
-                     stream)
-        e1.record(stream)
-        gdn.gdn2_bwd(*(d[n] for n in NAMES), d["dO"], None, grads["dq"], grads["dk"],
-                     grads["dv"], grads["dg"], grads["db"], grads["dw"], None, ws, ws.numel(), 1,
-                     B, T, H, dk, dv, C, io, stream)
-        e2.record(stream)
-    end.record(stream)
-    torch.cuda.synchronize(dev)
+    ms_step, fwd_ms, bwd_ms, launches = case.timed(args.steps, args.warmup, gd.barrier)
     sampler.mark_end()
-    barrier()
-    launches = gdn.gdn2_kernel_launches() - launches0
-    ktimes = gdn.gdn2_kernel_times()
-    gdn.gdn2_set_kernel_timer(False)
-    ms_total = start.elapsed_time(end)
-    fwd_ms = statistics.mean(a.elapsed_time(b) for a, b, _ in ev)
-    bwd_ms = statistics.mean(b.elapsed_time(c) for _, b, c in ev)
-    status = gdn.gdn2_get_device_status(stream)
-    if status != 0:
-        raise RuntimeError(f"device status {status} after the timed region")
+    # the per-kernel split, in a pass of its own
+    kernels = kernel_split(gdn, case.run, args.steps, case.token_heads, peak, case.stream)
 
     # end-to-end through host buffers: every step copies its inputs H2D from
     # pinned memory and its outputs D2H.  The input copies run on one stream,
@@ -248,7 +349,8 @@ def run_ours(args, rank, world, local_rank):
     # sets of device buffers, so that step i's D2H overlaps step i+1's H2D
     # (PCIe moves both directions at once).  The timed region spans the first
     # H2D to the last D2H.
-    outs = [dict(o=torch.empty_like(o), **{n: torch.empty_like(t) for n, t in grads.items()})
+    d, stream = case.d, case.stream
+    outs = [dict(o=torch.empty_like(case.o), **{n: torch.empty_like(t) for n, t in case.grads.items()})
             for _ in range(2)]
     host_out = [{n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for n, t in ob.items()}
                 for ob in outs]
@@ -256,9 +358,9 @@ def run_ours(args, rank, world, local_rank):
     d2h = sum(t.numel() * t.element_size() for t in host_out[0].values())
     stage = [{n: (d[n] if n == "S0" else torch.empty_like(t)) for n, t in d.items()} for _ in range(2)]
     s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    ev = lambda: torch.cuda.Event()
+    ev = lambda: torch.cuda.Event()  # noqa: E731
     ev_in, ev_done, ev_out = [ev(), ev()], [ev(), ev()], [ev(), ev()]
-    barrier()
+    gd.barrier()
     torch.cuda.synchronize(dev)
     e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e_start.record(stream)
@@ -276,7 +378,7 @@ def run_ours(args, rank, world, local_rank):
         stream.wait_event(ev_in[k])
         if i >= 2:
             stream.wait_event(ev_out[k])  # step i - 2's outputs have left these buffers
-        step(stage[k], outs[k])
+        case.step(stage[k], outs[k])
         ev_done[k].record(stream)
         with torch.cuda.stream(s_out):
             s_out.wait_event(ev_done[k])
@@ -287,32 +389,25 @@ def run_ours(args, rank, world, local_rank):
     e_end.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = e_start.elapsed_time(e_end) / args.e2e_steps
-    barrier()
+    gd.barrier()
     clocks = sampler.stop()
+    if gdn.gdn2_get_device_status(stream) != 0:
+        raise RuntimeError("device status reports an error after the end-to-end steps")
+    del outs, host_out, stage
+    token_heads = case.token_heads
+    del case
+    torch.cuda.empty_cache()
 
-    ms_step = ms_total / args.steps
     decode = run_decode(args, rank, dev) if not args.no_decode else None
+    subs = {} if (args.no_sub or WORKLOAD_INDEX != 2) else {
+        f"workload{i}": sub_workload(i, args, rank, dev, peak, peak_src) for i in (1, 3)}
     ms_step, e2e_ms, fwd_ms, bwd_ms = gd.max_over_ranks([ms_step, e2e_ms, fwd_ms, bwd_ms], dev)
     if decode is not None:
         decode["us_per_step"] = gd.max_over_ranks([decode["us_per_step"]], dev)[0]
     tokens = B * T * world
     value = tokens / (ms_step * 1e-3)
-    token_heads = B * T * H
     alg_bytes = token_heads * (FWD_BYTES + BWD_BYTES)
-    peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) \
-        if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")) else {}
-    peak = peaks.get("hbm_gbs", 6650.0)
-    peak_src = "of measured" if "hbm_gbs" in peaks else "of fallback"
     src = sources_hash()
-    kernels = {}
-    for name, (cnt, tot) in ktimes.items():
-        avg = tot / cnt
-        per = KERNEL_BYTES.get(name)
-        ent = {"launches": cnt, "avg_ms": avg}
-        if per is not None:
-            gbs = per * token_heads / (avg * 1e-3) / 1e9
-            ent.update(alg_bytes_per_launch=per * token_heads, achieved_gbs=gbs, frac=gbs / peak)
-        kernels[name] = ent
     dom = max(kernels, key=lambda n: kernels[n]["launches"] * kernels[n]["avg_ms"])
     dk_ = kernels[dom]
     roofline = {"bound": "hbm", "kernel": dom, "achieved": dk_.get("achieved_gbs"), "peak": peak,
@@ -322,7 +417,8 @@ def run_ours(args, rank, world, local_rank):
                 "traffic": traffic_from_profiles(dom, src)}
     step_achieved = alg_bytes / (ms_step * 1e-3) / 1e9
     roofline_step = {"bound": "hbm", "achieved": step_achieved, "peak": peak, "unit": "GB/s",
-                     "frac": step_achieved / peak, "alg_bytes_per_step": alg_bytes}
+                     "frac": step_achieved / peak, "alg_bytes_per_step": alg_bytes,
+                     "peak_source": peak_src}
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_step,
@@ -330,14 +426,16 @@ def run_ours(args, rank, world, local_rank):
         "dtype": "f16", "data": "synthetic (seeded workload generators)",
         "config": {"workload": wl.name if B == wl.B else f"{wl.name}, B overridden to {B}",
                    "B": B, "T": T, "H": H, "d_k": dk, "d_v": dv,
-                   "chunk": C, "io": "bf16 q/k/v/o/dO/dq/dk/dv, f32 g/b/w/state",
+                   "chunk": wl.chunk, "io": "bf16 q/k/v/o/dO/dq/dk/dv, f32 g/b/w/state",
                    "global_batch": B * world, "seq_len": T, "parallelism": f"dp{world}",
                    "l2": f"inputs {h2d / 1e9:.2f} GB per step (> 126 MB L2), no flush",
-                   "arithmetic": "fp16 tensor-core operands, fp32 accumulation and state"},
+                   "arithmetic": "fp16 and tf32 tensor-core operands, fp32 accumulation and state"},
         "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
         "roofline": roofline,
         "roofline_step": roofline_step,
         "kernels": kernels,
+        "kernel_timing": "per-kernel split from a separate pass of the same steps with the "
+                         "library's event timer on; the headline region runs with it off",
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
                 "copies": "pinned host buffers; H2D, step and D2H on three streams with two "
@@ -354,6 +452,7 @@ def run_ours(args, rank, world, local_rank):
                                 "peak": peak, "unit": "GB/s", "frac": gbs / peak,
                                 "alg_bytes_per_launch": dec_bytes, "peak_source": peak_src})
         line["decode"] = decode
+    line.update(subs)
     return line
 
 
@@ -423,62 +522,36 @@ def run_decode(args, rank, dev):
 
 
 def run_forward_only(args, rank, world, local_rank):
-    """Workload 1: the forward alone (bf16 q/k/v/o, f32 gates and state, S0 ~
-    N(0, 0.02), B8 T2048 H16 d128 C64), device-timed per call; algorithmic
-    bytes are the forward's per token-head plus S0 read and S_T written."""
+    """Workload 1 as a line of its own: the forward alone (bf16 q/k/v/o, f32
+    gates and state, S0 ~ N(0, 0.02), B8 T2048 H16 d128 C64), device-timed per
+    call; algorithmic bytes are the forward's per token-head plus S0 read and
+    S_T written."""
     import torch
 
-    import gated_delta_rule_128_b200 as gdn
     from gated_delta_rule_128_b200 import dist as gd
     from gated_delta_rule_128_b200 import workloads
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     wl = workloads.WORKLOADS[1]
-    B, T, H, dk, dv, C = args.batch or wl.B, wl.T, wl.H, wl.dk, wl.dv, wl.chunk
-    x = workloads.draw(B, T, H, dk, dv, gd.rank_seed(wl.seed, rank), s0_std=wl.s0_std,
-                       erase_scale=wl.erase_scale, with_dO=False)
-    d = {n: (t.to(torch.bfloat16) if n in ("q", "k", "v") else t).contiguous().to(dev)
-         for n, t in x.items()}
-    io = gdn.GDN2_IO_BF16
-    ws = gdn.workspace(B, T, H, dk, dv, C, io, False, dev)
-    o = torch.empty(B, T, H, dv, dtype=torch.bfloat16, device=dev)
-    ST = torch.empty(B, H, dk, dv, dtype=torch.float32, device=dev)
-    stream = torch.cuda.current_stream(dev)
-
-    def step():
-        gdn.gdn2_fwd(*(d[n] for n in NAMES), o, ST, ws, ws.numel(), B, T, H, dk, dv, C, io, stream)
-
-    for _ in range(max(3, args.warmup)):
-        step()
-    torch.cuda.synchronize(dev)
-    gd.barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    gdn.gdn2_set_kernel_timer(True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    ktimes = gdn.gdn2_kernel_times()
-    gdn.gdn2_set_kernel_timer(False)
-    if gdn.gdn2_get_device_status(stream) != 0:
-        raise RuntimeError("device status reports an error after the timed region")
-    ms = gd.max_over_ranks([e0.elapsed_time(e1) / args.steps], dev)[0]
-    peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) \
-        if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")) else {}
-    peak = peaks.get("hbm_gbs", 6650.0)
-    alg = B * T * H * FWD_BYTES + 2 * B * H * dk * dv * 4
+    B = args.batch or wl.B
+    case = FwdBwdCase(wl, B, gd.rank_seed(wl.seed, rank), dev, with_bwd=False)
+    peak, _ = _peak()
+    ms, _, _, launches = case.timed(args.steps, args.warmup, gd.barrier)
+    kernels = kernel_split(case.gdn, case.run, args.steps, case.token_heads, peak, case.stream)
+    ms = gd.max_over_ranks([ms], dev)[0]
+    alg = case.token_heads * FWD_BYTES + 2 * B * wl.H * wl.dk * wl.dv * 4
     gbs = alg / (ms * 1e-3) / 1e9
     return {
-        "metric": "GDR-2 fwd tokens/s (H16, dk=dv=128) and % of HBM roofline", "value": B * T * world / (ms * 1e-3),
+        "metric": "GDR-2 fwd tokens/s (H16, dk=dv=128) and % of HBM roofline", "value": B * wl.T * world / (ms * 1e-3),
         "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup),
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f16", "data": "synthetic (seeded workload generators)",
-        "config": {"workload": wl.name, "B": B, "T": T, "H": H, "d_k": dk, "d_v": dv, "chunk": C},
+        "config": {"workload": wl.name, "B": B, "T": wl.T, "H": wl.H, "d_k": wl.dk, "d_v": wl.dv,
+                   "chunk": wl.chunk},
         "roofline_step": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
                           "alg_bytes_per_step": alg},
-        "kernels": {k: {"launches": c, "avg_ms": t / c} for k, (c, t) in ktimes.items()},
+        "kernels": kernels, "gpu_launches": launches,
     }
 
 

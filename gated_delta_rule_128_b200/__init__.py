@@ -13,7 +13,8 @@ Two layers:
   pointers, and raising ``Gdn2Error`` on a non-zero status.
 * ``forward``, ``backward``, ``decode_step``: allocate outputs and workspace
   with torch (device memory is PyTorch's job here) and call the above on the
-  current CUDA stream.
+  current CUDA stream; ``forward`` and ``backward`` then read the device
+  status word and raise on a recorded error unless called with check=False.
 """
 
 from __future__ import annotations
@@ -182,9 +183,23 @@ def workspace(B, T, H, d_k, d_v, chunk, io, for_bwd, device="cuda") -> torch.Ten
     return torch.empty(n, dtype=torch.uint8, device=device)
 
 
+def check_device_status(stream=None) -> None:
+    """Raise Gdn2Error if a kernel recorded an error (a bounded wait that gave
+    up, or an operand outside the tensor-core path's fp16 range) since the
+    status word was last read.  Waits for `stream`."""
+    st = gdn2_get_device_status(stream)
+    if st != 0:
+        raise Gdn2Error("device status", st)
+
+
 def forward(q, k, v, g, b, w, S0=None, *, chunk: int = 64, want_state: bool = True,
-            ws: Optional[torch.Tensor] = None, for_bwd: bool = False, stream=None):
-    """Returns (o, S_T or None, ws).  Shapes: q, k, g, b [B,T,H,dk]; v, w [B,T,H,dv]."""
+            ws: Optional[torch.Tensor] = None, for_bwd: bool = False, stream=None,
+            check: bool = True):
+    """Returns (o, S_T or None, ws).  Shapes: q, k, g, b [B,T,H,dk]; v, w [B,T,H,dv].
+
+    check=True (the default) waits for the stream and raises Gdn2Error if a
+    kernel recorded an error during the call; check=False leaves the call
+    asynchronous (read the status later with check_device_status)."""
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     io = _io_of(q)
@@ -193,12 +208,16 @@ def forward(q, k, v, g, b, w, S0=None, *, chunk: int = 64, want_state: bool = Tr
     o = torch.empty(B, T, H, dv, dtype=q.dtype, device=q.device)
     ST = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device) if want_state else None
     gdn2_fwd(q, k, v, g, b, w, S0, o, ST, ws, ws.numel(), B, T, H, dk, dv, chunk, io, stream)
+    if check:
+        check_device_status(stream)
     return o, ST, ws
 
 
 def backward(q, k, v, g, b, w, S0, dO, dST=None, *, chunk: int = 64,
              ws: Optional[torch.Tensor] = None, ws_has_fwd: bool = False,
-             want_dS0: bool = True, stream=None) -> Dict[str, torch.Tensor]:
+             want_dS0: bool = True, stream=None, check: bool = True) -> Dict[str, torch.Tensor]:
+    """Gradients dq, dk, dv, dg, db, dw, dS0 (None unless want_dS0).  check as
+    in forward()."""
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     io = _io_of(q)
@@ -211,6 +230,8 @@ def backward(q, k, v, g, b, w, S0, dO, dST=None, *, chunk: int = 64,
                   if want_dS0 else None)
     gdn2_bwd(q, k, v, g, b, w, S0, dO, dST, out["dq"], out["dk"], out["dv"], out["dg"], out["db"],
              out["dw"], out["dS0"], ws, ws.numel(), ws_has_fwd, B, T, H, dk, dv, chunk, io, stream)
+    if check:
+        check_device_status(stream)
     return out
 
 

@@ -36,22 +36,24 @@ cudaError_t tc_bwd_launch(const void *, const void *, const void *, const float 
                           float *, float *, float *, float *, void *, unsigned int *, const Dims &,
                           cudaStream_t);
 
+// The device status word (GDN2_OK or the first error a kernel recorded), and
+// the slot that gdn2_get_device_status moves it into.  One pair per device,
+// shared by every stream.
 __device__ unsigned int g_status_word;
+__device__ unsigned int g_status_taken;
 
-// device address of g_status_word on the current device (looked up once per device)
+// device address of g_status_word in the current device's context, looked up
+// on every call (cheap, allocates nothing, and never stale after a reset)
 static unsigned int *status_word() {
-    static unsigned int *addr[64];
-    static std::mutex mu;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    std::lock_guard<std::mutex> lock(mu);
-    if (!addr[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
-        addr[dev] = static_cast<unsigned int *>(p);
-    }
-    return addr[dev];
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+    return static_cast<unsigned int *>(p);
 }
+
+// reads and clears the status word in one atomic step, after the work
+// enqueued on the stream before it
+static __global__ void status_take_kernel() { g_status_taken = atomicExch(&g_status_word, 0u); }
+static std::mutex g_status_mu;
 
 // the tensor-core path: bf16 I/O, d_k = d_v = 128, chunk 64
 static bool use_tc(const Dims &d, gdn2_io io) {
@@ -254,10 +256,16 @@ gdn2_status gdn2_selftest_timeout(long long limit_cycles, gdn2_stream_t stream) 
 }
 
 gdn2_status gdn2_get_device_status(gdn2_stream_t stream) {
-    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return GDN2_ERR_CUDA;
-    unsigned int word = 0, zero = 0;
-    if (cudaMemcpyFromSymbol(&word, g_status_word, sizeof(word)) != cudaSuccess) return GDN2_ERR_CUDA;
-    if (word != 0 && cudaMemcpyToSymbol(g_status_word, &zero, sizeof(zero)) != cudaSuccess)
+    // one reader at a time: the taken value goes through one device slot
+    std::lock_guard<std::mutex> lock(g_status_mu);
+    cudaStream_t s = (cudaStream_t)stream;
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    status_take_kernel<<<1, 1, 0, s>>>();
+    unsigned int word = 0;
+    if (cudaGetLastError() != cudaSuccess ||
+        cudaMemcpyFromSymbolAsync(&word, g_status_taken, sizeof(word), 0, cudaMemcpyDeviceToHost, s) !=
+            cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
         return GDN2_ERR_CUDA;
     return (gdn2_status)word;
 }

@@ -3,8 +3,6 @@
 // array of GDN2_NOALLOC_SCRATCH_BYTES that every GPU which loads this library
 // holds until the process exits.  All calls share it.
 
-#include <mutex>
-
 #include "common.cuh"
 
 namespace gdn2 {
@@ -22,26 +20,18 @@ cudaError_t simt_out_launch(const void *, void *, void *, const Dims &, cudaStre
 // returns for the current device.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[GDN2_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-static void *g_scratch_addr[kMaxDevices];
-static std::mutex g_scratch_mu;
-
-// Device address of the scratch on the current device, looked up once per
-// device (the first call on a device does this set-up).
+// Device address of the scratch in the current device's context.  It is
+// looked up on every call (cudaGetSymbolAddress allocates nothing), so a call
+// made after cudaDeviceReset, or in a new primary context, never receives an
+// address from a context that no longer exists.  The first lookup in a
+// context also loads the library's device code there, which is why the first
+// call on a device should come before any stream capture.
 static cudaError_t scratch_address(void **out) {
-    int dev = -1;
-    cudaError_t e = cudaGetDevice(&dev);
+    void *p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (!g_scratch_addr[dev]) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess) return e;
-        if (!p) return cudaErrorInvalidSymbol;
-        g_scratch_addr[dev] = p;
-    }
-    *out = g_scratch_addr[dev];
+    if (!p) return cudaErrorInvalidSymbol;
+    *out = p;
     return cudaSuccess;
 }
 

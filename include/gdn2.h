@@ -152,9 +152,12 @@ gdn2_status gdn2_decode_step(const void *q, const void *k, const void *v, const 
  *   GDN2_NOALLOC_SCRATCH_BYTES are rejected with GDN2_ERR_WORKSPACE before
  *   anything is enqueued (e.g. d_k = d_v = 128, chunk 64: B*H*chunks up to
  *   292), whatever the io type.
- * Set-up: the first call on a device looks up the array's device address
- *   (the current device must be the stream's device); make that first call
- *   before any stream capture.
+ * Set-up: every call looks up the array's device address in the calling
+ *   thread's current context (the current device must be the stream's
+ *   device); the lookup allocates nothing, and no address is kept between
+ *   calls, so a call after cudaDeviceReset never uses a stale address.  The
+ *   first call in a context also loads the library's device code there: make
+ *   that first call before any stream capture.
  * Sharing: all calls use the same array, and it keeps the last call's
  *   contents.  Calls whose work overlaps on the GPU (other streams, other
  *   threads) race on it; serialise them. */
@@ -163,8 +166,17 @@ gdn2_status gdn2_fwd_noalloc(const void *q, const void *k, const void *v, const 
                              int B, int T, int H, int d_k, int d_v, int chunk, gdn2_io io,
                              gdn2_stream_t stream);
 
-/* Waits for `stream`, then returns and clears the device status word: GDN2_OK,
- * or the first error a kernel recorded since the last call (GDN2_ERR_TIMEOUT).
+/* Returns and clears the device status word once the work enqueued on
+ * `stream` before this call has run: GDN2_OK, or the first error a kernel
+ * recorded since the word was last read (GDN2_ERR_TIMEOUT, GDN2_ERR_RANGE).
+ * The word is read and cleared in one atomic step by a one-thread kernel on
+ * `stream`, and the call then waits for `stream`.
+ * There is ONE status word per device, shared by every stream and thread of
+ * the process: an error recorded by a call on one stream is reported to
+ * whichever caller reads the word next, and work still running on other
+ * streams may record an error after this call returns.  Callers that need
+ * per-call attribution serialise their calls, or read the status after
+ * synchronising the device.
  * Returns GDN2_ERR_CUDA if the stream reports a CUDA error. */
 gdn2_status gdn2_get_device_status(gdn2_stream_t stream);
 

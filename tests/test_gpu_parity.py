@@ -111,6 +111,28 @@ def test_workload0_fp32_tied_gates(tie):
     assert rel(dbeta, ref["db"].sum(-1) + ref["dw"].sum(-1)) < TOL_F32
 
 
+@pytest.mark.parametrize("tie", ["kda", "gdn"])
+def test_tensor_core_path_tied_gates(tie):
+    """The ties on the tensor-core path (bf16, d = 128, chunk 64): b = w = beta 1
+    reproduces KDA, and a scalar decay as well reproduces Gated DeltaNet, at the
+    bf16 tolerances; the tied scalar's gradient is sum_c db + sum_c dw."""
+    x = workloads.draw(1, 256, 2, 128, 128, 810 + len(tie), tie=tie, s0_std=0.1)
+    xr = io_round({n: t for n, t in x.items() if n not in ("beta", "alpha_log")}, "bf16")
+    gpu = gpu_fwd_bwd({n: t for n, t in x.items() if n not in ("beta", "alpha_log")}, "bf16", 64,
+                      use_dST=False)
+    r = to_np64(xr)
+    beta, alpha = x["beta"].double().numpy(), x.get("alpha_log")
+    if tie == "kda":
+        o, ST = oracle.kda_forward(r["q"], r["k"], r["v"], r["g"], beta, r["S0"])
+    else:
+        o, ST = oracle.gdn_forward(r["q"], r["k"], r["v"], alpha.double().numpy(), beta, r["S0"])
+    assert rel(gpu["o"], o) < TOL_BF16_OUT and rel(gpu["ST"], ST) < TOL_BF16_OUT
+    ref = oracle.backward(*(r[n] for n in NAMES), r["dO"], None)
+    compare(gpu, ref, "bf16", GRADS)
+    dbeta = gpu["db"].sum(-1) + gpu["dw"].sum(-1)
+    assert rel(dbeta, ref["db"].sum(-1) + ref["dw"].sum(-1)) < TOL_BF16_GRAD
+
+
 # ------------------------------------------------------ small grids, ragged
 
 CASES = [
@@ -214,7 +236,10 @@ def test_every_output_written_and_no_nan_read(dk, chunk):
 
 # --------------------------------------------- full-size workloads, sampled
 
-SAMPLE = {1: [(0, 0), (7, 15), (3, 9)], 2: [(0, 0), (3, 15), (1, 7)], 3: [(0, 0), (0, 15), (0, 6)]}
+# eight (batch, head) pairs per workload, the first and the last pair included
+SAMPLE = {1: [(0, 0), (7, 15), (3, 9), (1, 4), (5, 12), (6, 1), (2, 14), (4, 7)],
+          2: [(0, 0), (3, 15), (1, 7), (2, 3), (0, 12), (3, 0), (1, 14), (2, 9)],
+          3: [(0, 0), (0, 15), (0, 6), (0, 3), (0, 9), (0, 12), (0, 1), (0, 13)]}
 
 
 @pytest.mark.parametrize("index", [1, 2, 3])
@@ -357,7 +382,7 @@ def test_tensor_core_path_reports_decay_out_of_range():
     x = workloads.draw(1, 128, 2, 128, 128, 41, with_dO=False)
     x["g"] = torch.full_like(x["g"], -0.5)
     d = to_device(x, "bf16")
-    gdn.forward(*(d[n] for n in NAMES), chunk=64)
+    gdn.forward(*(d[n] for n in NAMES), chunk=64, check=False)
     torch.cuda.synchronize()
     assert gdn.gdn2_get_device_status() == 6          # GDN2_ERR_RANGE
     assert gdn.gdn2_get_device_status() == 0
