@@ -123,25 +123,24 @@ inline SimtWs simt_ws_layout(const Dims &d) {
 // with plain bulk copies.  Offsets in bytes; bh = b * H + h.
 //   rec   [bh][NC]        66560 B  the chunk's record, written by the chunk-
 //                                  parallel prep kernel (layout REC_* below)
-//   ckS   [bh][NC + 1][2 halves] 16 KB  chunk-entry states S_c (and S_T), true scale
-//   ckD   [bh][NC][2]             8 KB  Delta (columns of one d_v half)
-//   ckdS  [bh][NC][2]            16 KB  e^(G_L - G_m) dS_next
-//   ckndU [bh][NC][2]             8 KB  -dU
-//   ckEnd [bh][NC][2]           512 B  half-sums of rowsum(dS_next . S_next)
+//   ckS   [bh][NC][2 halves]  16 KB  chunk-entry states S_c (true scale)
+//   ckD   [bh][NC][2]          8 KB  Delta (columns of one d_v half)
+//   ckdS  [bh][NC][2]         16 KB  dL/dS_{c+1}, the state gradient leaving chunk c
+//   ckndU [bh][NC][2]          8 KB  -dU
 // A forward that is not followed by a backward needs `rec` only.
 //
-// Chunk record: decay-scaled operands relative to the chunk's middle row
-// (fp16, 128-byte swizzled; see tc.cuh for the layouts)
+// Chunk record: chunk-start-frame operands (fp16, 128-byte swizzled; see
+// tc.cuh for the layouts and tc_common.cuh for the frames)
 //   REC_WQ   [-W; Qb] as one [128 rows][128 key] K-major tile: rows 0..63
-//            -W = -T Kc, rows 64..127 Qb = q.e^(G-G_m) (32 KB)
-//   REC_KH   Kh = k.e^-(G-G_m)          [64 pos][128 key] K-major (16 KB)
+//            -W = -T Kc (Kc = b.k.e^G), rows 64..127 Qb = q.e^G (32 KB)
+//   REC_KH   Kb = k.e^(G_63 - G)        [64 pos][128 key] K-major (16 KB)
 //   REC_T    T = (I + A)^-1             [64][64] K-major (8 KB)
-//   REC_P    P = lower-incl(Qb Kh^T)    [64][64] K-major (8 KB)
-//   REC_FAC  e^(G_L - G_m) [128] f32, then e^G_m [128] f32
+//   REC_P    P                          [64][64] K-major (8 KB)
+//   REC_FAC  gamma = e^G_63 [128] f32, then 128 unused floats
 constexpr uint32_t REC_WQ = 0, REC_KH = 32768, REC_T = 49152, REC_P = 57344, REC_FAC = 65536,
                    REC_BYTES = 66560;
 struct TcWs {
-    size_t rec, rec_end, ckS, ckD, fwd_end, ckdS, ckndU, ckEnd, bwd_end;
+    size_t rec, rec_end, ckS, ckD, fwd_end, ckdS, ckndU, bwd_end;
 };
 inline TcWs tc_ws_layout(const Dims &d) {
     const size_t bh = (size_t)d.B * d.H, nc = (size_t)d.NC;
@@ -150,12 +149,11 @@ inline TcWs tc_ws_layout(const Dims &d) {
     auto take = [&](size_t bytes) { size_t at = o; o = align256(o + bytes); return at; };
     w.rec = take(bh * nc * REC_BYTES);
     w.rec_end = o;
-    w.ckS = take(bh * (nc + 1) * 2 * 16384);
+    w.ckS = take(bh * nc * 2 * 16384);
     w.ckD = take(bh * nc * 2 * 8192);
     w.fwd_end = o;
     w.ckdS = take(bh * nc * 2 * 16384);
     w.ckndU = take(bh * nc * 2 * 8192);
-    w.ckEnd = take(bh * nc * 2 * 512);
     w.bwd_end = o;
     return w;
 }

@@ -8,32 +8,31 @@
 // so they stay inside them: b enters dA and dKc through Kc in every channel
 // sum below.
 //
-// Chunk equations (decay factors relative to the chunk's middle row m, see
-// tc_common.cuh; dS = dL/dS_next entering the chunk from the right):
-//   dS_m  = diag(e^(G_L-G_m)) dS
-//   dDelta = P^T dO + Kh dS_m,         dU = T^T dDelta,   dw = dU.v, dv = dU.w
-//   dS_c  = diag(e^G_m) (dS_m + Qb^T dO - W^T dDelta)             (carried left)
-//   (W^T dDelta = Kc^T dU, since W = T Kc)
-//   S_m   = diag(e^G_m) S_c
-//   dP = lower-incl(dO Delta^T),       dA = -strictly-lower(dU Delta^T)
-//   Y1 = dO S_m^T + dP Kh              dq  = Y1.E
-//   Y2 = -dU S_m^T + dA Kh             dKc.e^G = Y2.E,  db = Y2.E.k
-//   Y3 = Delta dS_m^T + dP^T Qb + dA^T Kc            dk = Y2.E.b + Y3/E
-//   dG = dq.q + Y2.E.b.k - (Y3/E).k, plus rowsum(dS . S_next) on the last row
+// Chunk equations (chunk-start frame, tc_common.cuh; dS' = dL/dS_{c+1}
+// entering the chunk from the right; E = e^G, F = e^(G_63 - G)):
+//   dDelta = P^T dO + Kb dS',           dU = T^T dDelta,   dw = dU.v, dv = dU.w
+//   dS_c  = diag(gamma) dS' + Qb^T dO - W^T dDelta                 (carried left)
+//   dP = lower-incl(dO Delta^T),        dA = -strictly-lower(dU Delta^T)
+//   Y1 = dO S_c^T,  Y2 = -dU S_c^T,  Y3 = Delta dS'^T        (state parts)
+//   Z1_r = sum_j dP_rj k_j e^(G_r - G_j),   Z2_r = sum_j dA_rj k_j e^(G_r - G_j)
+//   Z3_j = sum_r (dP_rj q_r + dA_rj b_r k_r) e^(G_r - G_j)   (pair parts)
+//   dq = Y1 E + Z1,   dKc = Y2 E + Z2,   dk = Y3 F + Z3 + dKc b,   db = dKc k
+//   dG = q dq + 2 b k dKc - k dk, plus on the last row the chunk-end term
+//        rowsum(dS' . S_{c+1}) = gamma rowsum(dS' . S_c) + sum_t Kb_t Y3_t
 //   dg = reverse in-chunk cumsum of dG
-// (E = e^(G - G_m); the chunk-end term rowsum(dS_next . S_next) is the
-// derivative through the chunk's total decay, since S_next = e^G_L (...).)
+// (the chunk-end term is the derivative through the chunk's total decay,
+// since S_{c+1} = diag(e^G_63) S_c + Kb^T Delta).
 //
 // Two kernels:
 //  * tc_bwd_state_kernel: one CTA per (b, h, half of d_v), walking the chunks
 //    in reverse with dS in tensor memory and the chunk records double-
 //    buffered; two tcgen05.mma round trips per chunk on the state's path
 //    (dDelta; then dS), with dU and its outputs off that path.  Writes dw,
-//    dv, dS0, and per chunk dS_m, -dU and the half-sums of the chunk-end
-//    term to the workspace.
+//    dv, dS0, and per chunk dS' and -dU to the workspace.
 //  * tc_bwd_grad_kernel: persistent, one CTA per SM walking the (b, h, chunk)
-//    tiles, all chunks in parallel, full d_v; five products, then three
-//    accumulations, then dq, dk, db, dg.
+//    tiles, all chunks in parallel, full d_v: the state parts and dP, dA on
+//    the tensor cores, the pair parts as warp-level products in the block
+//    frames of tc_common.cuh, then dq, dk, db, dg.
 
 #include "common.cuh"
 #include "tc.cuh"
@@ -53,12 +52,11 @@ constexpr uint32_t RAW_DO = 2 * REC_BYTES;    // dO half, bf16 [64 pos][64]
 constexpr uint32_t OP_DO = RAW_DO + 8192;     // dO fp16      [64 pos][64 v]  MN-major B
 constexpr uint32_t OP_DS = OP_DO + 8192;      // dX fp16      [128 key][64 v] MN-major B
 constexpr uint32_t OP_DD = OP_DS + 16384;     // dDelta fp16  [64 pos][64 v]  MN-major B
-constexpr uint32_t STG_S = OP_DD + 8192;      // checkpoint S_m fp16 [128 key][64 v]
-constexpr uint32_t VV = STG_S + 16384;        // v half bf16 [64][64], 128-B swizzled; dv in place
+constexpr uint32_t VV = OP_DD + 8192;         // v half bf16 [64][64], 128-B swizzled; dv in place
 constexpr uint32_t VW = VV + 8192;            // w half f32, two [64][32] 128-B swizzled boxes; dw in place
 constexpr uint32_t NDU = VW + 16384;          // -dU fp16 [64 pos][64 v] (the workspace layout)
-constexpr uint32_t MISC = NDU + 8192;         // sEnd [2][128] f32; mbarriers; TMEM slot
-constexpr uint32_t SMEM_BYTES = MISC + 1024 + 128 + 1024;
+constexpr uint32_t MISC = NDU + 8192;         // mbarriers; TMEM slot
+constexpr uint32_t SMEM_BYTES = MISC + 128 + 1024;
 constexpr uint32_t TM_DS = 0, TM_DD = 64, TM_DU = 128;  // 256 columns allocated
 constexpr uint32_t ID_MM64 = idesc_f16(64, 64, true, true);
 constexpr uint32_t ID_KM64 = idesc_f16(64, 64, false, true);
@@ -68,16 +66,16 @@ constexpr float kRange = 6.0e4f;
 static_assert(MISC % 1024 == 0, "alignment");
 }  // namespace tbs
 
-// One CTA per (b, h, half of d_v), walking the chunks in reverse with
-// dX = diag(e^(G_L - G_m)) dS_next in tensor memory.  Per chunk, from the
-// chunk's record (Qb, Kh, -W, T, P, factors):
-//   (1) dDelta = P^T dO + Kh dX  (committed alone),  then dS_m = dX + Qb^T dO
-//   (2) dS_m += (-W)^T dDelta  (committed alone),     then dU = T^T dDelta
-// then dS_c = diag(e^G_m) dS_m and the previous chunk's dX = diag(e^(G_L -
-// G_m)) dS_c.  dU is read while the next chunk's first products run: dv =
-// dU.w and dw = dU.v are formed in place of the v and w tiles (128-B
-// swizzled TMA tiles) and leave by TMA stores; -dU, dX and the chunk-end
-// half-sums go to the workspace for the gradient kernel.  Warps 0..7 read
+// One CTA per (b, h, half of d_v), walking the chunks in reverse.  Entering
+// chunk c, the compute warps put diag(gamma) dS' in tensor memory and dS' as
+// an fp16 operand.  Per chunk, from the chunk's record (Qb, Kb, -W, T, P,
+// gamma):
+//   (1) dDelta = P^T dO + Kb dS'  (committed alone),  then dS += Qb^T dO
+//   (2) dS += (-W)^T dDelta  (committed alone),       then dU = T^T dDelta
+// after which tensor memory holds dS_c, the dS' of chunk c - 1.  dU is read
+// while the next chunk's first products run: dv = dU.w and dw = dU.v are
+// formed in place of the v and w tiles (128-B swizzled TMA tiles) and leave
+// by TMA stores; -dU and dS' go to the workspace for the gradient kernel.  Warps 0..7 read
 // the accumulators and form the operands and outputs; warp 8 issues the
 // products (an issuing thread is held for about as long as the products
 // run); warp 9 requests every copy, so that neither delays the readouts.
@@ -91,11 +89,10 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
     extern __shared__ unsigned char smraw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smraw) + 1023) & ~static_cast<uintptr_t>(1023));
-    float *sEnd = reinterpret_cast<float *>(sm + MISC);  // [2][128]
-    // 0, 1 records of stages 0, 1; 2 dO; 3 state checkpoint; 4 v and w;
+    // 0, 1 records of stages 0, 1; 2 dO; 3 (unused); 4 v and w;
     // 5 dDelta ready; 6 dS ready; 7 dU ready
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + MISC + 1024);
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + MISC + 1024 + 64);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + MISC);
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + MISC + 64);
     float big = 0.f;  // range check: operand magnitude
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -133,11 +130,6 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
         tma_load_4d(sm + RAW_DO, &mdo, v0, h, cc * 64, bb, &bars[2]);
         ++issued[2];
     };
-    auto load_s = [&](int slot) {  // state checkpoint `slot` of this half
-        mbar_expect_tx(&bars[3], 16384);
-        bulk_load(sm + STG_S, ws + lay.ckS + ((bh * (NC + 1) + slot) * 2 + vh) * 16384, 16384, &bars[3]);
-        ++issued[3];
-    };
     auto load_vw = [&](int cc) {
         mbar_expect_tx(&bars[4], 8192 + 16384);
         tma_load_4d(sm + VV, &mv, v0, h, cc * 64, bb, &bars[4]);
@@ -145,8 +137,8 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
         tma_load_4d(sm + VW + 8192, &mw, v0 + 32, h, cc * 64, bb, &bars[4]);
         ++issued[4];
     };
-    auto rec_fac = [&](int cc) {  // e^(G_L - G_m) of chunk cc (then e^G_m at +128)
-        return reinterpret_cast<const float *>(sm + STG + (cc & 1) * REC_BYTES + REC_FAC);
+    auto rec_gamma = [&](int cc) {  // gamma = e^G_63 of chunk cc
+        return reinterpret_cast<const float *>(sm + STG + (cc & 1) * REC_BYTES + REC_FAC)[key];
     };
     // dO of the chunk in RAW_DO -> fp16 operand (each thread 16 values)
     auto convert_do = [&]() {
@@ -168,27 +160,20 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
         big = absmax8(x, big);
         big = absmax8(x + 8, big);
     };
-    // dX of chunk c into TMEM and the fp16 operand (this thread's row, 32 columns)
-    auto put_dx = [&](float *x) {
-        tmem_st16(taddr(tm + TM_DS, quarter * 32, 32 * half), x);
-        tmem_st16(taddr(tm + TM_DS, quarter * 32, 32 * half + 16), x + 16);
+    // dS' of the next chunk to process: diag(gamma) dS' into TMEM (the
+    // products add the rest of dS_c to it), dS' as the fp16 operand (this
+    // thread's row, 32 columns)
+    auto put_ds = [&](const float *x, float gam) {
+        float y[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) y[j] = gam * x[j];
+        tmem_st16(taddr(tm + TM_DS, quarter * 32, 32 * half), y);
+        tmem_st16(taddr(tm + TM_DS, quarter * 32, 32 * half + 16), y + 16);
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
             st_h8(sm + OP_DS + sw128_chunk(key, 4 * half + jj, 128), x + 8 * jj);
             big = absmax8(x + 8 * jj, big);
         }
-    };
-    // rowsum over this thread's 32 columns of x . S (S from STG_S)
-    auto end_term = [&](const float *x) {
-        float acc = 0.f;
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-            float s8[8];
-            ld_h8(sm + STG_S + sw128_chunk(key, 4 * half + jj, 128), s8);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) acc += x[8 * jj + e] * s8[e];
-        }
-        return acc;
     };
     // dU of chunk cc (TMEM) -> dv, dw in place of v, w; -dU staged (compute
     // threads; the copier stores them after the next barrier: store_du)
@@ -235,10 +220,9 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
         load_rec(NC - 1);
         if (NC > 1) load_rec(NC - 2);
         load_do(NC - 1);
-        load_s(NC);
         load_vw(NC - 1);
     }
-    // ---------------- prologue: dS_T (or zero), the last chunk's end term and dX; dO
+    // ---------------- prologue: dS' = dS_T (or zero) for the last chunk; dO
     bool ok = true;
     if (compute) {
         float x[32];
@@ -249,34 +233,21 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
                            : make_float4(0.f, 0.f, 0.f, 0.f);
             x[j] = t.x; x[j + 1] = t.y; x[j + 2] = t.z; x[j + 3] = t.w;
         }
-        ok = mbar_wait(&bars[3], 0, kWait);
-        ok = mbar_wait(&bars[(NC - 1) & 1], 0, kWait) && ok;
+        ok = mbar_wait(&bars[(NC - 1) & 1], 0, kWait);
         ok = mbar_wait(&bars[2], 0, kWait) && ok;
-        sEnd[half * 128 + key] = end_term(x);  // the last checkpoint is S_T itself
-        const float gam = rec_fac(NC - 1)[key];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) x[j] *= gam;
-        put_dx(x);
+        put_ds(x, rec_gamma(NC - 1));
         convert_do();
         tmem_wait_st();
     }
     fence_proxy_async();
     fence_before_sync();
     bool abort = __syncthreads_or(!ok);
-    if (!abort) {
-        if (compute && half == 0)
-            reinterpret_cast<float *>(ws + lay.ckEnd + ((bh * NC + NC - 1) * 2 + vh) * 512)[key] =
-                sEnd[key] + sEnd[128 + key];
-        if (copier) {
-            fence_after_sync();
-            bulk_store(ws + lay.ckdS + ((bh * NC + NC - 1) * 2 + vh) * 16384, sm + OP_DS, 16384);
-            bulk_commit();
-            if (NC > 1) {
-                load_s(NC - 1);
-                load_do(NC - 2);
-            }
-            bulk_wait_read();  // the dX copy has left OP_DS
-        }
+    if (!abort && copier) {
+        fence_after_sync();
+        bulk_store(ws + lay.ckdS + ((bh * NC + NC - 1) * 2 + vh) * 16384, sm + OP_DS, 16384);
+        bulk_commit();
+        if (NC > 1) load_do(NC - 2);
+        bulk_wait_read();  // the dS' copy has left OP_DS
     }
 
     for (int i = 0; i < NC && !abort; ++i) {
@@ -341,23 +312,18 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
             mma_commit(&bars[7]);
             ++groups[2];
         }
-        // ---------------- dS_c; the previous chunk's end term, dX and dO
+        // ---------------- dS_c: dS' of chunk c - 1; its dO
         if (compute) {
-        ok = mbar_wait(&bars[6], par, kWait) && ok;
-        if (c > 0) {
-            ok = mbar_wait(&bars[3], (i + 1) & 1, kWait) && ok;                 // S_m of chunk c
-            ok = mbar_wait(&bars[(c - 1) & 1], ((i + 1) >> 1) & 1, kWait) && ok;  // record c-1
-            ok = mbar_wait(&bars[2], (i + 1) & 1, kWait) && ok;                 // dO of chunk c-1
-        }
-        fence_after_sync();
-        {
+            ok = mbar_wait(&bars[6], par, kWait) && ok;
+            if (c > 0) {
+                ok = mbar_wait(&bars[(c - 1) & 1], ((i + 1) >> 1) & 1, kWait) && ok;  // record c-1
+                ok = mbar_wait(&bars[2], (i + 1) & 1, kWait) && ok;                 // dO of chunk c-1
+            }
+            fence_after_sync();
             float sv[32];
             tmem_ld16(taddr(tm + TM_DS, quarter * 32, 32 * half), sv);
             tmem_ld16(taddr(tm + TM_DS, quarter * 32, 32 * half + 16), sv + 16);
             tmem_wait_ld();
-            const float e = reinterpret_cast<const float *>(stg + REC_FAC)[128 + key];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) sv[j] *= e;  // dS_c
             if (c == 0) {
                 if (dS0) {
                     float *dst = dS0 + st_off(d, bb, h) + (size_t)key * 128 + v0 + 32 * half;
@@ -366,36 +332,26 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
                         *reinterpret_cast<float4 *>(dst + j) = make_float4(sv[j], sv[j + 1], sv[j + 2], sv[j + 3]);
                 }
             } else {
-                // the checkpoint holds S_m = diag(e^G_m) S_c
-                sEnd[half * 128 + key] = end_term(sv) / e;
-                const float gam = rec_fac(c - 1)[key];
-#pragma unroll
-                for (int j = 0; j < 32; ++j) sv[j] *= gam;
-                put_dx(sv);
+                put_ds(sv, rec_gamma(c - 1));
                 convert_do();
                 tmem_wait_st();
             }
-        }
         }
         fence_proxy_async();
         fence_before_sync();
         if (__syncthreads_or(!ok)) { abort = true; break; }
         if (c > 0) {
-            if (compute && half == 0)
-                reinterpret_cast<float *>(ws + lay.ckEnd + ((bh * NC + c - 1) * 2 + vh) * 512)[key] =
-                    sEnd[key] + sEnd[128 + key];
             if (copier) {
                 fence_after_sync();
                 bulk_store(ws + lay.ckdS + ((bh * NC + c - 1) * 2 + vh) * 16384, sm + OP_DS, 16384);
                 bulk_commit();
-                load_s(c - 1);                // S_m of chunk c consumed
                 if (c >= 2) {
                     load_do(c - 2);           // raw dO consumed
                     // this chunk's record is consumed once T^T dDelta has read T
                     if (!mbar_wait(&bars[7], par, kWait)) record_status(status, GDN2_ERR_TIMEOUT);
                     load_rec(c - 2);
                 }
-                bulk_wait_read();  // the dX copy has left OP_DS before it is rewritten
+                bulk_wait_read();  // the dS' copy has left OP_DS before it is rewritten
             }
         }
     }
@@ -424,27 +380,40 @@ namespace tbg {
 constexpr int kCompute = 512;             // warps 0..15 form operands and outputs
 constexpr int kThreads = kCompute + 32;   // warp 16 issues the copies and products
 constexpr int kWarps = kCompute / 32;
-constexpr uint32_t RQ = 0;        // q: two 128-B swizzled [64][64] bf16 boxes; Qb, then dq, in place
-constexpr uint32_t RK = 16384;    // k (bf16); dk in place
-constexpr uint32_t RB = 32768;    // b: four [64][32] f32 boxes; db in place
-constexpr uint32_t RG = 65536;    // g (f32); G - G_m, then dG, then dg in place
+// raw tiles (128-B swizzled TMA boxes, tc_common.cuh raw16 / raw32); the
+// outputs are formed in place
+constexpr uint32_t RQ = 0;        // q (bf16), then dq
+constexpr uint32_t RK = 16384;    // k (bf16), then dk
+constexpr uint32_t RB = 32768;    // b (f32), then db
+constexpr uint32_t RG = 65536;    // g (f32), then d = G' - G'_m, then dG, then dg
+// operands of the tensor-core products
 constexpr uint32_t DN = 98304;    // [dO; -dU] [128][128] K-major (K-blocks of 16 KB)
 constexpr uint32_t DL = 131072;   // Delta [64 pos][128 v] K-major
-constexpr uint32_t SMT = 147456;  // S_m [128 key][128 v] K-major (then Kh, Kc)
-constexpr uint32_t DXT = 180224;  // dX  [128 key][128 v] K-major (then [dP; dA])
-constexpr uint32_t KH = SMT, KC = SMT + 16384, PA = DXT;  // after the first products
-constexpr uint32_t TE = DXT + 16384, TEI = DL;              // E = e^(G - G_m), 1/E (fp16 [64][128])
-constexpr uint32_t MISC = 212992; // sEnd [2][256]; sRef [128]; scan [16][128]; mbarriers; slot
-constexpr uint32_t SMEM_BYTES = MISC + 2560 + 8192 + 128 + 1024;
-constexpr uint32_t LOAD_A = 114688;  // dO, -dU, Delta, S_m, dX (the first products' operands)
-constexpr uint32_t LOAD_B = 98304;   // raw q, k, b, g
+constexpr uint32_t SMT = 147456;  // S_c [128 key][128 v] K-major
+constexpr uint32_t DXT = 180224;  // dS' [128 key][128 v] K-major
+// once the products have read them, the same 112 KB hold the pair-term data
+// ([64 rows][128 channels] fp16 tiles, swizzled as raw16)
+constexpr uint32_t KA = 98304;    // k e^(e_I - G)
+constexpr uint32_t QA = 114688;   // q e^(G - s_I)
+constexpr uint32_t BA = 131072;   // b k e^(G - s_I)
+constexpr uint32_t AL = 147456;   // e^(G - s_I)
+constexpr uint32_t AB = 163840;   // e^(e_I - G)
+constexpr uint32_t PD = 180224;   // masked dP [64][64] fp16 (sw128, R = 64)
+constexpr uint32_t AD = 188416;   // masked dA
+constexpr uint32_t DG32 = 196608; // diagonal blocks of dP, dA in f32 [2][4][16][17]
+constexpr uint32_t MISC = 212992; // per-channel values (below), mbarriers, TMEM slot
+constexpr uint32_t M_TOT = 0, M_ES = 2048, M_EF = 4096, M_CHI = 6144, M_END1 = 9216, M_ENDK = 11264,
+                   M_GAM = 13312, M_BAR = 13824;
+constexpr uint32_t SMEM_BYTES = MISC + M_BAR + 128 + 1024;
+constexpr uint32_t LOAD_A = 32768 + 81920;  // dO, -dU; Delta, S_c, dS'
+constexpr uint32_t LOAD_B = 98304;          // raw q, k, b, g
 constexpr uint32_t TM_Y1 = 0, TM_Y2 = 128, TM_Y3 = 256, TM_PA = 384;  // 512 columns
 constexpr uint32_t ID_PA = idesc_f16(128, 64, false, false);
 constexpr uint32_t ID_KK128 = idesc_f16(64, 128, false, false);
-constexpr uint32_t ID_KM128 = idesc_f16(64, 128, false, true);
-constexpr uint32_t ID_MM128 = idesc_f16(64, 128, true, true);
 constexpr long long kWait = 2000000000LL;
 constexpr float kRange = 6.0e4f;
+static_assert(DG32 + 2 * 4 * 16 * 17 * 4 <= MISC, "pair-term data fits over the operands");
+static_assert(SMEM_BYTES <= 232448, "shared memory");
 }  // namespace tbg
 
 // descriptor of K step kstep of a K-major operand whose 64-wide K-blocks lie
@@ -453,24 +422,36 @@ __device__ __forceinline__ uint64_t kstep_kmajor_blk(uint64_t d0, uint32_t blk, 
     return d0 + (uint64_t)((((uint32_t)(kstep >> 2) * blk) + (kstep & 3) * 32) >> 4);
 }
 
+// 16 TMEM lanes x 8 columns in the m16n8 accumulator-fragment layout: rows
+// base + t/4 (v0, v1) and base + t/4 + 8 (v2, v3), columns c + 2 (t % 4), + 1
+__device__ __forceinline__ void tmem_ld16x256x1(uint32_t taddr, float *v) {
+    uint32_t r[4];
+    asm volatile("tcgen05.ld.sync.aligned.16x256b.x1.b32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// index of the block pair (I, J), I > J, among the six
+__host__ __device__ constexpr int pair_ix(int I, int J) { return I * (I - 1) / 2 + J; }
+
 // Persistent: one CTA per SM walks the (b, h, chunk) tiles, full d_v.  Warp 16
-// loads the tile (raw q, k, b, g, dO as 128-B swizzled TMA boxes; S_m, dX,
-// Delta, -dU from the workspace) and issues the products; warps 0..15 form
-// the operands and the outputs:
-//   (1) [dP; dA] = [dO; -dU] Delta^T (M = 128), Y1 = dO S_m^T, Y2 = -dU S_m^T,
-//       Y3 = Delta dX^T, while the decay factors Qb (in place of q), Kc, Kh
-//       are formed
-//   (2) Y1 += dP Kh, Y2 += dA Kh, Y3 += dP^T Qb + dA^T Kc (masked dP, dA)
-// then, per (row, channel) straight from tensor memory: dq = Y1.E,
-// db = Y2.E.k, dk = Y2.E.b + Y3/E, dG = Y1.Qb + Y2.Kc - Y3.Kh, written in
-// place of q, k, b, g; dg is the reverse in-chunk cumsum of dG plus the
-// chunk-end term, and the four tiles leave by TMA stores.  Sixteen compute
-// warps (four rows each in the row-wise phases) hide the latency of the
-// per-element work; E and 1/E are kept as fp16 tiles between the factor
-// phase and the outputs.  The next tile's copies are requested as soon as
-// their buffers are free: dO and -dU after the first products, Delta, S_m
-// and dX after the outputs are formed, the raw tiles once the TMA stores have
-// read them.
+// loads the tile (raw q, k, b, g, dO as 128-B swizzled TMA boxes; S_c, dS',
+// Delta, -dU from the workspace) and issues the tensor-core products; compute
+// warp w owns row block I = w % 4 (16 rows, TMEM lane quarter I) and channel
+// quarter Q = w / 4 (32 channels):
+//   (1) [dP; dA] = [dO; -dU] Delta^T (M = 128), Y1 = dO S_c^T, Y2 = -dU S_c^T,
+//       Y3 = Delta dS'^T on the tensor cores, while the warps form the
+//       cumulative decay and the block factors;
+//   (2) the chunk-end sum rowsum(dS' . S_c) and the masked dP, dA;
+//   (3) the pair terms Z1, Z2, Z3 as warp-level products: blocks below the
+//       diagonal in fp16 (m16n8k16) with the block-boundary frames, the
+//       diagonal blocks in tf32 (m16n8k8) with the clamped mid-block frame;
+//   (4) dq, dk, db, dG per (row, channel) in the accumulator-fragment layout,
+//       which the 16x256b tensor-memory loads share, written in place of q,
+//       k, b, g; then dg, the reverse in-chunk cumsum of dG plus the chunk-end
+//       term, and TMA stores.
 __global__ void __launch_bounds__(tbg::kThreads, 1)
 tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                    const __grid_constant__ CUtensorMap mb, const __grid_constant__ CUtensorMap mg,
@@ -482,21 +463,24 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
     extern __shared__ unsigned char smraw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smraw) + 1023) & ~static_cast<uintptr_t>(1023));
-    // chunk-end term per channel as the two d_v halves' partials [2][128],
-    // double-buffered by tile parity (copied in with Delta, S_m, dX)
-    float *sEnd2 = reinterpret_cast<float *>(sm + MISC);
-    float *sRef = reinterpret_cast<float *>(sm + MISC + 2048);  // G of the middle row per channel
-    float *scan = reinterpret_cast<float *>(sm + MISC + 2560);  // per-warp totals [16][128]
-    // 0 first-product operands (two parts), 1, 2 products, 3 raw tiles, 4 dO
+    float *mtot = reinterpret_cast<float *>(sm + MISC + M_TOT);    // [4][128] block totals
+    float *mes = reinterpret_cast<float *>(sm + MISC + M_ES);      // [4][128] e^s_I
+    float *mef = reinterpret_cast<float *>(sm + MISC + M_EF);      // [4][128] e^(G_63 - e_I)
+    float *mchi = reinterpret_cast<float *>(sm + MISC + M_CHI);    // [6][128] chi_IJ
+    float *mend1 = reinterpret_cast<float *>(sm + MISC + M_END1);  // [4][128] rowsum(dS' . S_c) parts
+    float *mendk = reinterpret_cast<float *>(sm + MISC + M_ENDK);  // [4][128] sum_t Kb Y3 parts
+    float *mgam = reinterpret_cast<float *>(sm + MISC + M_GAM);    // [128] gamma
+    // 0 first-product operands (two parts), 1 products, 3 raw tiles, 4 dO
     // converted (one arrival per compute warp)
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + MISC + 2560 + 8192);
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + MISC + 2560 + 8192 + 64);
-    float big = 0.f, gbig = 0.f;  // range checks: operand magnitude, |G - G_m|
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + MISC + M_BAR);
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + MISC + M_BAR + 64);
+    float big = 0.f;  // range check: largest fp16 operand magnitude
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int NC = d.NC, H = d.H;
     const int ntiles = d.B * H * NC;
-    const int quarter = warp & 3, cgrp = (warp >> 2) & 3;  // TMEM lane quarter; column group
+    const int I = warp & 3, Q = (warp >> 2) & 3;  // row block (TMEM lane quarter); channel quarter
+    const int gq = lane >> 2, tq = lane & 3;
     const bool compute = warp < kWarps, issuer = tid == kCompute;
 
     if (warp == 0) {
@@ -525,11 +509,10 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
         }
         ++issued[0];
     };
-    auto load_a2 = [&](int it, int pb) {  // Delta, S_m, dX and the chunk-end partials
-        mbar_expect_tx(&bars[0], LOAD_A - 32768 + 1024);
-        bulk_load(sEnd2 + 256 * pb, ws + lay.ckEnd + (size_t)it * 1024, 1024, &bars[0]);
+    auto load_a2 = [&](int it) {  // Delta, S_c, dS'
+        mbar_expect_tx(&bars[0], LOAD_A - 32768);
         bulk_load(sm + DL, ws + lay.ckD + ((size_t)it * 2) * 8192, 16384, &bars[0]);
-        bulk_load(sm + SMT, ws + lay.ckS + ((size_t)(it + it / NC) * 2) * 16384, 32768, &bars[0]);
+        bulk_load(sm + SMT, ws + lay.ckS + ((size_t)it * 2) * 16384, 32768, &bars[0]);
         bulk_load(sm + DXT, ws + lay.ckdS + ((size_t)it * 2) * 16384, 32768, &bars[0]);
         ++issued[1];
     };
@@ -548,7 +531,7 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
     };
     if (issuer && (int)blockIdx.x < ntiles) {
         load_a1(blockIdx.x);
-        load_a2(blockIdx.x, 0);
+        load_a2(blockIdx.x);
         load_b(blockIdx.x);
     }
 
@@ -560,8 +543,8 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
         const bool more = nxt < ntiles;
         ok = mbar_wait(&bars[0], par, kWait) && ok;
 
-        // ---------------- dO to fp16; then, while the first products run, the
-        // cumulative decay (rows 4w..4w+3, channels 4l..4l+3)
+        // ---------------- dO to fp16; the issuer waits for this, then the
+        // first products run while the warps form the block factors
         if (compute) {
 #pragma unroll
             for (int m = 0; m < 2; ++m) {  // the dO rows of [dO; -dU], in place
@@ -577,7 +560,6 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
                 }
                 st_h8(p, x);
             }
-            // the issuer waits for this, the compute warps go on to the decay
             fence_proxy_async();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[4]);
@@ -598,183 +580,356 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
             }
             mma_commit(&bars[1]);
         }
-        float G[4][4];
+        // factor ownership: channel fc = 32 Q + lane, the 16 rows of block I
+        const int fc = 32 * Q + lane;
+        uint32_t pk[8][5];  // rows (2 i, 2 i + 1) as f16 pairs: k a_bar, q a, b k a, a, a_bar
         if (compute) {
             ok = mbar_wait(&bars[3], par, kWait) && ok;
-            float run[4] = {0.f, 0.f, 0.f, 0.f};
+            float gl[16], gc[16];
+            {
+                float run = 0.f, runc = 0.f;
 #pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const float4 t = *reinterpret_cast<const float4 *>(sm + RG + sw128_chunk(4 * warp + m, lane, 64));
-                run[0] += t.x; run[1] += t.y; run[2] += t.z; run[3] += t.w;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) G[m][i] = run[i];
-            }
-            *reinterpret_cast<float4 *>(scan + warp * 128 + 4 * lane) = make_float4(run[0], run[1], run[2], run[3]);
-            named_sync(1, kCompute);
-            if (tid < 128) {  // per channel: exclusive prefix over the warps' totals, in place
-                float acc = 0.f;
-#pragma unroll
-                for (int w2 = 0; w2 < kWarps; ++w2) {
-                    const float t = scan[w2 * 128 + tid];
-                    scan[w2 * 128 + tid] = acc;
-                    acc += t;
-                    if (w2 == kWarps / 2 - 1) sRef[tid] = acc;  // rows 0..31: G of the middle row
+                for (int r = 0; r < 16; ++r) {
+                    const float gv = *reinterpret_cast<const float *>(sm + RG + raw32(16 * I + r, fc));
+                    run += gv;
+                    runc += fmaxf(gv, -kClampG);
+                    gl[r] = run;
+                    gc[r] = runc;
                 }
+                mtot[I * 128 + fc] = run;
             }
             named_sync(1, kCompute);
-        }
-        // ---------------- decay factors while the products run: Qb in place of q;
-        // Kh, Kc kept in registers until S_m is consumed
-        uint2 khr[4], kcr[4], er[4], eir[4];
-        if (compute) {
-            const float4 pre4 = *reinterpret_cast<const float4 *>(scan + warp * 128 + 4 * lane);
-            const float4 ref4 = *reinterpret_cast<const float4 *>(sRef + 4 * lane);
-            const float pre[4] = {pre4.x, pre4.y, pre4.z, pre4.w}, ref[4] = {ref4.x, ref4.y, ref4.z, ref4.w};
-            uint2 qr[4], kr[4];
-            float4 bv[4];
+            float T4[4];
 #pragma unroll
-            for (int m = 0; m < 4; ++m) {  // every input row before the first store
-                const int r = 4 * warp + m;
-                qr[m] = *reinterpret_cast<const uint2 *>(sm + RQ + sw128_chunk(r, lane >> 1, 64) + (lane & 1) * 8);
-                kr[m] = *reinterpret_cast<const uint2 *>(sm + RK + sw128_chunk(r, lane >> 1, 64) + (lane & 1) * 8);
-                bv[m] = *reinterpret_cast<const float4 *>(sm + RB + sw128_chunk(r, lane, 64));
+            for (int J = 0; J < 4; ++J) T4[J] = mtot[J * 128 + fc];
+            {
+                float s = 0.f, all = 0.f;
+#pragma unroll
+                for (int J = 0; J < 4; ++J) {
+                    if (J < I) s += T4[J];
+                    all += T4[J];
+                }
+                mes[I * 128 + fc] = __expf(s);
+                mef[I * 128 + fc] = __expf(all - s - T4[I]);
+                if (I == 0) mgam[fc] = __expf(all);
+                float between = 0.f;
+#pragma unroll
+                for (int I2 = 1; I2 < 4; ++I2)
+                    if (I2 > I) {
+                        mchi[pair_ix(I2, I) * 128 + fc] = I2 == I + 1 ? 1.f : __expf(between);
+                        between += T4[I2];
+                    }
             }
 #pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const int r = 4 * warp + m;
-                float Gv[4];
+            for (int r2 = 0; r2 < 8; ++r2) {
+                float v[2][5];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    Gv[i] = G[m][i] + pre[i] - ref[i];
-                    gbig = fmaxf(gbig, fabsf(Gv[i]));
+                for (int e = 0; e < 2; ++e) {
+                    const int r = 2 * r2 + e, t = 16 * I + r;
+                    const float qv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + RQ + raw16(t, fc)));
+                    const float kv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + RK + raw16(t, fc)));
+                    const float bv = *reinterpret_cast<const float *>(sm + RB + raw32(t, fc));
+                    const float a = __expf(gl[r]), ab = __expf(T4[I] - gl[r]);
+                    v[e][0] = kv * ab;
+                    v[e][1] = qv * a;
+                    v[e][2] = bv * kv * a;
+                    v[e][3] = a;
+                    v[e][4] = ab;
+                    big = fmaxf(big, fmaxf(fabsf(v[e][0]), fmaxf(fabsf(v[e][1]), fabsf(v[e][2]))));
+                    *reinterpret_cast<float *>(sm + RG + raw32(t, fc)) = gc[r] - gc[7];
                 }
-                const __nv_bfloat162 *q2 = reinterpret_cast<const __nv_bfloat162 *>(&qr[m]);
-                const __nv_bfloat162 *k2 = reinterpret_cast<const __nv_bfloat162 *>(&kr[m]);
-                const float qf[4] = {__low2float(q2[0]), __high2float(q2[0]), __low2float(q2[1]), __high2float(q2[1])};
-                const float kf[4] = {__low2float(k2[0]), __high2float(k2[0]), __low2float(k2[1]), __high2float(k2[1])};
-                const float bf[4] = {bv[m].x, bv[m].y, bv[m].z, bv[m].w};
-                float qb[4], kc[4], kh[4], e[4], ei[4];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    e[i] = __expf(Gv[i]);
-                    ei[i] = __expf(-Gv[i]);
-                    qb[i] = qf[i] * e[i];
-                    kc[i] = bf[i] * kf[i] * e[i];
-                    kh[i] = kf[i] * ei[i];
-                }
-                st_h4(sm + RQ + sw128_chunk(r, lane >> 1, 64) + (lane & 1) * 8, qb[0], qb[1], qb[2], qb[3]);
-                khr[m] = make_uint2(pack_f16(kh[0], kh[1]), pack_f16(kh[2], kh[3]));
-                kcr[m] = make_uint2(pack_f16(kc[0], kc[1]), pack_f16(kc[2], kc[3]));
-                er[m] = make_uint2(pack_f16(e[0], e[1]), pack_f16(e[2], e[3]));
-                eir[m] = make_uint2(pack_f16(ei[0], ei[1]), pack_f16(ei[2], ei[3]));
-#pragma unroll
-                for (int i = 0; i < 4; ++i) big = fmaxf(big, fmaxf(fabsf(qb[i]), fmaxf(fabsf(kc[i]), fabsf(kh[i]))));
+                for (int x = 0; x < 5; ++x) pk[r2][x] = pack_f16(v[0][x], v[1][x]);
             }
-            // ---------------- masked dP, dA; Kh, Kc into the space of S_m
+            // ---------------- chunk-end sum, once the products have read S_c and dS'
             ok = mbar_wait(&bars[1], par, kWait) && ok;
             fence_after_sync();
             {
-                // accumulator row quarter * 32 + lane: 0..63 dP, 64..127 dA; 16 columns from 16 * cgrp
-                float row[16];
-                tmem_ld16(taddr(tm + TM_PA, quarter * 32, 16 * cgrp), row);
-                tmem_wait_ld();
-                const int pr = quarter * 32 + lane, r = pr & 63;
-                // dP keeps j <= r; dA = strictly-lower of (-dU) Delta^T
+                // channel fc, d_v quarter I: 32 values of S_c and dS'
+                float acc = 0.f;
 #pragma unroll
-                for (int j = 0; j < 16; ++j) row[j] = (pr < 64 ? 16 * cgrp + j <= r : 16 * cgrp + j < r) ? row[j] : 0.f;
+                for (int jj = 0; jj < 4; ++jj) {
+                    const uint32_t off = (uint32_t)((I >> 1) * 16384) + sw128_chunk(fc, 4 * (I & 1) + jj, 128);
+                    float s8[8], d8[8];
+                    ld_h8(sm + SMT + off, s8);
+                    ld_h8(sm + DXT + off, d8);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) acc = fmaf(s8[e], d8[e], acc);
+                }
+                mend1[I * 128 + fc] = acc;
+            }
+            named_sync(1, kCompute);  // S_c, dS', Delta, [dO; -dU] are consumed
+            // ---------------- masked dP, dA (TMEM lanes 0..63 dP, 64..127 dA)
+            {
+                float row[16];
+                tmem_ld16(taddr(tm + TM_PA, I * 32, 16 * Q), row);
+                tmem_wait_ld();
+                const int pr = I * 32 + lane, r = pr & 63;
+                const bool isA = pr >= 64;
+#pragma unroll
+                for (int j = 0; j < 16; ++j) row[j] = (isA ? 16 * Q + j < r : 16 * Q + j <= r) ? row[j] : 0.f;
+                unsigned char *dst = sm + (isA ? AD : PD);
 #pragma unroll
                 for (int jj = 0; jj < 2; ++jj) {
-                    st_h8(sm + PA + sw128_chunk(pr, 2 * cgrp + jj, 128), row + 8 * jj);
+                    st_h8(dst + sw128_chunk(r, 2 * Q + jj, 64), row + 8 * jj);
                     big = absmax8(row + 8 * jj, big);
                 }
+                if ((r >> 4) == Q) {
+                    float *dg32 = reinterpret_cast<float *>(sm + DG32) + ((isA ? 4 : 0) + Q) * 16 * 17 + (r & 15) * 17;
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) dg32[j] = row[j];
+                }
             }
+            // ---------------- the block factors as fp16 tiles
 #pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const uint32_t off = sw128_off(4 * warp + m, 4 * lane, 64);
-                *reinterpret_cast<uint2 *>(sm + KH + off) = khr[m];
-                *reinterpret_cast<uint2 *>(sm + KC + off) = kcr[m];
-                *reinterpret_cast<uint2 *>(sm + TE + off) = er[m];
-                *reinterpret_cast<uint2 *>(sm + TEI + off) = eir[m];
-            }
-        }
-        if (issuer) {  // dO and -dU of the next tile, once the first products have read them
-            ok = mbar_wait(&bars[1], par, kWait) && ok;
-            if (more) load_a1(nxt);
-        }
-        fence_proxy_async();
-        fence_before_sync();
-        __syncthreads();
-        if (issuer) {
-            fence_after_sync();
-            const uint64_t kP = desc_kmajor(smem_addr(sm + PA), 128, 0), kA = desc_kmajor(smem_addr(sm + PA + 8192), 128, 0),
-                           mP = desc_mnmajor(smem_addr(sm + PA), 64, 0), mA = desc_mnmajor(smem_addr(sm + PA + 8192), 64, 0),
-                           qb = desc_mnmajor(smem_addr(sm + RQ), 64, 0), kc = desc_mnmajor(smem_addr(sm + KC), 64, 0),
-                           kh = desc_mnmajor(smem_addr(sm + KH), 64, 0);
+            for (int r2 = 0; r2 < 8; ++r2) {
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-                const uint64_t b_kh = kstep_mnmajor(kh, ks);
-                mma_bf16(tm + TM_Y1, kstep_kmajor(kP, 128, ks), b_kh, ID_KM128, 1);
-                mma_bf16(tm + TM_Y2, kstep_kmajor(kA, 128, ks), b_kh, ID_KM128, 1);
-                mma_bf16(tm + TM_Y3, kstep_mnmajor(mP, ks), kstep_mnmajor(qb, ks), ID_MM128, 1);
-                mma_bf16(tm + TM_Y3, kstep_mnmajor(mA, ks), kstep_mnmajor(kc, ks), ID_MM128, 1);
-            }
-            mma_commit(&bars[2]);
-        }
-        // ---------------- dq, dk, db, dG per (row, channel), from tensor memory.
-        // The M = 64 accumulators hold row quarter * 16 + l in lane l < 16; the
-        // 16x256b loads give each thread two rows x two column pairs of every
-        // 16-channel group.
-        if (compute) {
-            ok = mbar_wait(&bars[2], par, kWait) && ok;
-            fence_after_sync();
-            // 16x256b loads: thread t holds rows q16 + t/4 and q16 + t/4 + 8, column
-            // pairs 2 (t % 4) and 8 + 2 (t % 4) of each 16-column group
-            const int rA = quarter * 16 + (lane >> 2), cp0 = 2 * (lane & 3);
-#pragma unroll 1
-            for (int g2 = 0; g2 < 2; ++g2) {
-                const int ch0 = 32 * cgrp + 16 * g2;
-                float y1[8], y2[8], y3[8];
-                tmem_ld16x256x2(taddr(tm + TM_Y1 + ch0, quarter * 32, 0), y1);
-                tmem_ld16x256x2(taddr(tm + TM_Y2 + ch0, quarter * 32, 0), y2);
-                tmem_ld16x256x2(taddr(tm + TM_Y3 + ch0, quarter * 32, 0), y3);
-                tmem_wait_ld();
+                for (int e = 0; e < 2; ++e) {
+                    const uint32_t off = raw16(16 * I + 2 * r2 + e, fc);
 #pragma unroll
-                for (int p = 0; p < 4; ++p) {  // (row, column pair): p & 1 picks the row, p >> 1 the pair
-                    const int rr = rA + 8 * (p & 1), c = ch0 + cp0 + 8 * (p >> 1);
-                    const int ri = 2 * (p & 1) + 4 * (p >> 1);  // register index of the pair
-                    const uint32_t o16 = sw128_off(rr, c, 64);
-                    const uint32_t o32 = sw128_chunk(rr, c >> 2, 64) + (c & 3) * 4;
-                    const float2 qb = __half22float2(*reinterpret_cast<const __half2 *>(sm + RQ + o16));
-                    const float2 kc = __half22float2(*reinterpret_cast<const __half2 *>(sm + KC + o16));
-                    const float2 kh = __half22float2(*reinterpret_cast<const __half2 *>(sm + KH + o16));
-                    const float2 E = __half22float2(*reinterpret_cast<const __half2 *>(sm + TE + o16));
-                    const float2 Ei = __half22float2(*reinterpret_cast<const __half2 *>(sm + TEI + o16));
-                    const float2 kf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(sm + RK + o16));
-                    const float2 bf = *reinterpret_cast<const float2 *>(sm + RB + o32);
-                    const float a1[2] = {y1[ri], y1[ri + 1]}, a2[2] = {y2[ri], y2[ri + 1]}, a3[2] = {y3[ri], y3[ri + 1]};
-                    const float qv[2] = {qb.x, qb.y}, kcv[2] = {kc.x, kc.y}, khv[2] = {kh.x, kh.y};
-                    const float Ev[2] = {E.x, E.y}, Eiv[2] = {Ei.x, Ei.y}, kv[2] = {kf.x, kf.y}, bv[2] = {bf.x, bf.y};
-                    float dq[2], dk[2], db[2], dG[2];
-#pragma unroll
-                    for (int i = 0; i < 2; ++i) {
-                        const float dkc = a2[i] * Ev[i], dkh = a3[i] * Eiv[i];
-                        dq[i] = a1[i] * Ev[i];
-                        db[i] = dkc * kv[i];
-                        dk[i] = dkc * bv[i] + dkh;
-                        dG[i] = a1[i] * qv[i] + a2[i] * kcv[i] - a3[i] * khv[i];
+                    for (int x = 0; x < 5; ++x) {
+                        const uint32_t hv = e ? (pk[r2][x] >> 16) : (pk[r2][x] & 0xffffu);
+                        *reinterpret_cast<uint16_t *>(sm + KA + x * 16384 + off) = (uint16_t)hv;
                     }
-                    *reinterpret_cast<uint32_t *>(sm + RQ + o16) = pack_bf16(dq[0], dq[1]);
-                    *reinterpret_cast<uint32_t *>(sm + RK + o16) = pack_bf16(dk[0], dk[1]);
-                    *reinterpret_cast<float2 *>(sm + RB + o32) = make_float2(db[0], db[1]);
-                    *reinterpret_cast<float2 *>(sm + RG + o32) = make_float2(dG[0], dG[1]);
                 }
             }
         }
+        __syncthreads();  // dP, dA and the factor tiles are in place
+        if (compute) {
+            const uint32_t spd = smem_addr(sm + PD), sad = smem_addr(sm + AD);
+            const float *dgP = reinterpret_cast<const float *>(sm + DG32) + I * 16 * 17;
+            const float *dgA = dgP + 4 * 16 * 17;
+            const int r0 = 16 * I + gq;  // this thread's fragment rows r0, r0 + 8
+            // ---------------- Z1, Z2: rows of block I, channels of quarter Q
+            float z1[4][4], z2[4][4];
+            {
+                float c1[4][4] = {}, c2[4][4] = {};
+                for (int J = 0; J < I; ++J) {
+                    uint32_t aP[4], aA[4], bk[8];
+                    // A: rows 16 I + (l & 7) + 8 ((l >> 3) & 1), columns 16 J + 8 (l >> 4)
+                    const int ar = 16 * I + (lane & 7) + 8 * ((lane >> 3) & 1), ac = 16 * J + 8 * (lane >> 4);
+                    ldsm_x4(aP, spd + sw128_off(ar, ac, 64));
+                    ldsm_x4(aA, sad + sw128_off(ar, ac, 64));
+                    // B: rows 16 J + (l & 7) + 8 ((l >> 3) & 1), channels 32 Q + 16 p + 8 (l >> 4)
+                    const int br = 16 * J + (lane & 7) + 8 * ((lane >> 3) & 1);
+                    ldsm_x4_t(bk, smem_addr(sm + KA + raw16(br, 32 * Q + 8 * (lane >> 4))));
+                    ldsm_x4_t(bk + 4, smem_addr(sm + KA + raw16(br, 32 * Q + 16 + 8 * (lane >> 4))));
+                    if (J + 1 < I) {
+#pragma unroll
+                        for (int nt = 0; nt < 4; ++nt) {
+                            const float chi = mchi[pair_ix(I, J) * 128 + 32 * Q + 8 * nt + gq];
+                            bk[2 * nt] = h2scale(bk[2 * nt], chi);
+                            bk[2 * nt + 1] = h2scale(bk[2 * nt + 1], chi);
+                        }
+                    }
+#pragma unroll
+                    for (int nt = 0; nt < 4; ++nt) {
+                        mma_f16_16x8x16(c1[nt], aP, bk + 2 * nt);
+                        mma_f16_16x8x16(c2[nt], aA, bk + 2 * nt);
+                    }
+                }
+                // scale by a = e^(G_r - s_I)
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt) {
+                    const int cc = 32 * Q + 8 * nt + 2 * tq;
+#pragma unroll
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(sm + AL + raw16(r0 + 8 * h2, cc)));
+                        z1[nt][2 * h2] = a.x * c1[nt][2 * h2];
+                        z1[nt][2 * h2 + 1] = a.y * c1[nt][2 * h2 + 1];
+                        z2[nt][2 * h2] = a.x * c2[nt][2 * h2];
+                        z2[nt][2 * h2 + 1] = a.y * c2[nt][2 * h2 + 1];
+                    }
+                }
+            }
+            {
+                // diagonal block: rows and columns of block I, tf32
+                float c1[4][4] = {}, c2[4][4] = {};
+#pragma unroll
+                for (int k0 = 0; k0 < 16; k0 += 8) {
+                    const uint32_t aP[4] = {to_tf32(dgP[gq * 17 + k0 + tq]), to_tf32(dgP[(gq + 8) * 17 + k0 + tq]),
+                                            to_tf32(dgP[gq * 17 + k0 + tq + 4]), to_tf32(dgP[(gq + 8) * 17 + k0 + tq + 4])};
+                    const uint32_t aA[4] = {to_tf32(dgA[gq * 17 + k0 + tq]), to_tf32(dgA[(gq + 8) * 17 + k0 + tq]),
+                                            to_tf32(dgA[gq * 17 + k0 + tq + 4]), to_tf32(dgA[(gq + 8) * 17 + k0 + tq + 4])};
+#pragma unroll
+                    for (int nt = 0; nt < 4; ++nt) {
+                        const int cc = 32 * Q + 8 * nt + gq;
+                        uint32_t bkd[2];
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int j = 16 * I + k0 + tq + 4 * e;
+                            const float kv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + RK + raw16(j, cc)));
+                            const float dv = *reinterpret_cast<const float *>(sm + RG + raw32(j, cc));
+                            bkd[e] = to_tf32(kv * __expf(-dv));
+                        }
+                        mma_tf32_16x8x8(c1[nt], aP, bkd);
+                        mma_tf32_16x8x8(c2[nt], aA, bkd);
+                    }
+                }
+                // scale by l = e^(G'_r - G'_m) and add
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt) {
+                    const int cc = 32 * Q + 8 * nt + 2 * tq;
+#pragma unroll
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        const float2 dv = *reinterpret_cast<const float2 *>(sm + RG + raw32(r0 + 8 * h2, cc));
+                        const float l0 = __expf(dv.x), l1 = __expf(dv.y);
+                        z1[nt][2 * h2] += l0 * c1[nt][2 * h2];
+                        z1[nt][2 * h2 + 1] += l1 * c1[nt][2 * h2 + 1];
+                        z2[nt][2 * h2] += l0 * c2[nt][2 * h2];
+                        z2[nt][2 * h2 + 1] += l1 * c2[nt][2 * h2 + 1];
+                    }
+                }
+            }
+            // ---------------- Z3: rows j of block I (as a column block), channels of quarter Q
+            float z3[4][4];
+            {
+                float c3[4][4] = {};
+                for (int I2 = I + 1; I2 < 4; ++I2) {
+                    uint32_t aP[4], aA[4], bq[8], bb2[8];
+                    // A = dP[r in I2][j in I]^T: stored rows 16 I2 + (l & 7) + 8 (l >> 4),
+                    // columns 16 I + 8 ((l >> 3) & 1)
+                    const int sr = 16 * I2 + (lane & 7) + 8 * (lane >> 4), sc = 16 * I + 8 * ((lane >> 3) & 1);
+                    ldsm_x4_t(aP, spd + sw128_off(sr, sc, 64));
+                    ldsm_x4_t(aA, sad + sw128_off(sr, sc, 64));
+                    const int br = 16 * I2 + (lane & 7) + 8 * ((lane >> 3) & 1);
+                    ldsm_x4_t(bq, smem_addr(sm + QA + raw16(br, 32 * Q + 8 * (lane >> 4))));
+                    ldsm_x4_t(bq + 4, smem_addr(sm + QA + raw16(br, 32 * Q + 16 + 8 * (lane >> 4))));
+                    ldsm_x4_t(bb2, smem_addr(sm + BA + raw16(br, 32 * Q + 8 * (lane >> 4))));
+                    ldsm_x4_t(bb2 + 4, smem_addr(sm + BA + raw16(br, 32 * Q + 16 + 8 * (lane >> 4))));
+                    if (I2 > I + 1) {
+#pragma unroll
+                        for (int nt = 0; nt < 4; ++nt) {
+                            const float chi = mchi[pair_ix(I2, I) * 128 + 32 * Q + 8 * nt + gq];
+#pragma unroll
+                            for (int e = 0; e < 2; ++e) {
+                                bq[2 * nt + e] = h2scale(bq[2 * nt + e], chi);
+                                bb2[2 * nt + e] = h2scale(bb2[2 * nt + e], chi);
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int nt = 0; nt < 4; ++nt) {
+                        mma_f16_16x8x16(c3[nt], aP, bq + 2 * nt);
+                        mma_f16_16x8x16(c3[nt], aA, bb2 + 2 * nt);
+                    }
+                }
+                // scale by a_bar = e^(e_I - G_j)
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt) {
+                    const int cc = 32 * Q + 8 * nt + 2 * tq;
+#pragma unroll
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(sm + AB + raw16(r0 + 8 * h2, cc)));
+                        z3[nt][2 * h2] = a.x * c3[nt][2 * h2];
+                        z3[nt][2 * h2 + 1] = a.y * c3[nt][2 * h2 + 1];
+                    }
+                }
+            }
+            {
+                // diagonal block, tf32: A = dP_II^T, dA_II^T; B = q l, b k l
+                float c3[4][4] = {};
+#pragma unroll
+                for (int k0 = 0; k0 < 16; k0 += 8) {
+                    // a0 (j = g, r = t), a1 (g + 8, t), a2 (g, t + 4), a3 (g + 8, t + 4)
+                    const uint32_t aP[4] = {to_tf32(dgP[(k0 + tq) * 17 + gq]), to_tf32(dgP[(k0 + tq) * 17 + gq + 8]),
+                                            to_tf32(dgP[(k0 + tq + 4) * 17 + gq]), to_tf32(dgP[(k0 + tq + 4) * 17 + gq + 8])};
+                    const uint32_t aA[4] = {to_tf32(dgA[(k0 + tq) * 17 + gq]), to_tf32(dgA[(k0 + tq) * 17 + gq + 8]),
+                                            to_tf32(dgA[(k0 + tq + 4) * 17 + gq]), to_tf32(dgA[(k0 + tq + 4) * 17 + gq + 8])};
+#pragma unroll
+                    for (int nt = 0; nt < 4; ++nt) {
+                        const int cc = 32 * Q + 8 * nt + gq;
+                        uint32_t bqd[2], bbd[2];
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int r = 16 * I + k0 + tq + 4 * e;
+                            const float l = __expf(*reinterpret_cast<const float *>(sm + RG + raw32(r, cc)));
+                            const float qv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + RQ + raw16(r, cc)));
+                            const float kv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + RK + raw16(r, cc)));
+                            const float bv = *reinterpret_cast<const float *>(sm + RB + raw32(r, cc));
+                            bqd[e] = to_tf32(qv * l);
+                            bbd[e] = to_tf32(bv * kv * l);
+                        }
+                        mma_tf32_16x8x8(c3[nt], aP, bqd);
+                        mma_tf32_16x8x8(c3[nt], aA, bbd);
+                    }
+                }
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt) {
+                    const int cc = 32 * Q + 8 * nt + 2 * tq;
+#pragma unroll
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        const float2 dv = *reinterpret_cast<const float2 *>(sm + RG + raw32(r0 + 8 * h2, cc));
+                        z3[nt][2 * h2] += __expf(-dv.x) * c3[nt][2 * h2];
+                        z3[nt][2 * h2 + 1] += __expf(-dv.y) * c3[nt][2 * h2 + 1];
+                    }
+                }
+            }
+            __syncwarp();  // every read of this warp's raw region is done
+            // ---------------- dq, dk, db, dG in place; the chunk-end sum over Kb Y3
+            float endk[4][2];
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) {
+                float y1[4], y2[4], y3[4];
+                tmem_ld16x256x1(taddr(tm + TM_Y1 + 32 * Q + 8 * nt, I * 32, 0), y1);
+                tmem_ld16x256x1(taddr(tm + TM_Y2 + 32 * Q + 8 * nt, I * 32, 0), y2);
+                tmem_ld16x256x1(taddr(tm + TM_Y3 + 32 * Q + 8 * nt, I * 32, 0), y3);
+                tmem_wait_ld();
+                const int cc = 32 * Q + 8 * nt + 2 * tq;
+                const float2 es = *reinterpret_cast<const float2 *>(mes + I * 128 + cc);
+                const float2 ef = *reinterpret_cast<const float2 *>(mef + I * 128 + cc);
+                endk[nt][0] = endk[nt][1] = 0.f;
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const int r = r0 + 8 * h2;
+                    const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(sm + AL + raw16(r, cc)));
+                    const float2 ab = __half22float2(*reinterpret_cast<const __half2 *>(sm + AB + raw16(r, cc)));
+                    const float2 qf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(sm + RQ + raw16(r, cc)));
+                    const float2 kf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(sm + RK + raw16(r, cc)));
+                    const float2 bf = *reinterpret_cast<const float2 *>(sm + RB + raw32(r, cc));
+                    const float av[2] = {a.x, a.y}, abv[2] = {ab.x, ab.y}, qv[2] = {qf.x, qf.y},
+                                kv[2] = {kf.x, kf.y}, bv[2] = {bf.x, bf.y}, esv[2] = {es.x, es.y},
+                                efv[2] = {ef.x, ef.y};
+                    float dq[2], dk[2], db[2], dG[2];
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int x = 2 * h2 + e;
+                        const float E = av[e] * esv[e], F = abv[e] * efv[e];
+                        dq[e] = fmaf(y1[x], E, z1[nt][x]);
+                        const float dkc = fmaf(y2[x], E, z2[nt][x]);
+                        const float y3f = y3[x] * F;
+                        dk[e] = y3f + z3[nt][x] + dkc * bv[e];
+                        db[e] = dkc * kv[e];
+                        dG[e] = qv[e] * dq[e] + 2.f * bv[e] * kv[e] * dkc - kv[e] * dk[e];
+                        endk[nt][e] = fmaf(kv[e], y3f, endk[nt][e]);
+                    }
+                    *reinterpret_cast<uint32_t *>(sm + RQ + raw16(r, cc)) = pack_bf16(dq[0], dq[1]);
+                    *reinterpret_cast<uint32_t *>(sm + RK + raw16(r, cc)) = pack_bf16(dk[0], dk[1]);
+                    *reinterpret_cast<float2 *>(sm + RB + raw32(r, cc)) = make_float2(db[0], db[1]);
+                    *reinterpret_cast<float2 *>(sm + RG + raw32(r, cc)) = make_float2(dG[0], dG[1]);
+                }
+            }
+            // sum the Kb Y3 parts over this warp's 16 rows (lanes with equal t % 4)
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    float v = endk[nt][e];
+                    v += __shfl_xor_sync(0xffffffffu, v, 4);
+                    v += __shfl_xor_sync(0xffffffffu, v, 8);
+                    v += __shfl_xor_sync(0xffffffffu, v, 16);
+                    if (gq == 0) mendk[I * 128 + 32 * Q + 8 * nt + 2 * tq + e] = v;
+                }
+        }
         fence_proxy_async();
         fence_before_sync();
-        __syncthreads();
+        __syncthreads();  // dq, dk, db, dG formed; the pair-term data is consumed
         if (issuer) {
-            if (more) load_a2(nxt, (n + 1) & 1);  // Kh, Kc, E, 1/E, dP, dA are consumed
+            fence_after_sync();
+            if (more) {  // the next tile's operands into the space the pair terms used
+                load_a1(nxt);
+                load_a2(nxt);
+            }
             for (int x = 0; x < 2; ++x) {
                 tma_store_4d(&mdq, sm + RQ + x * 8192, 64 * x, h, c0, bb);
                 tma_store_4d(&mdk, sm + RK + x * 8192, 64 * x, h, c0, bb);
@@ -782,34 +937,25 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
             for (int x = 0; x < 4; ++x) tma_store_4d(&mdb, sm + RB + x * 8192, 32 * x, h, c0, bb);
             bulk_commit();
         }
-        // ---------------- dg: reverse in-chunk cumsum of dG with the chunk-end term
+        // ---------------- dg: reverse in-chunk cumsum of dG plus the chunk-end term
         if (compute) {
-            float run[4] = {0.f, 0.f, 0.f, 0.f}, x[4][4];
+            const int fc2 = 32 * Q + lane;
+            float x[16], run = 0.f;
 #pragma unroll
-            for (int m = 3; m >= 0; --m) {
-                const float4 t = *reinterpret_cast<const float4 *>(sm + RG + sw128_chunk(4 * warp + m, lane, 64));
-                run[0] += t.x; run[1] += t.y; run[2] += t.z; run[3] += t.w;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) x[m][i] = run[i];
+            for (int r = 15; r >= 0; --r) {
+                run += *reinterpret_cast<const float *>(sm + RG + raw32(16 * I + r, fc2));
+                x[r] = run;
             }
-            *reinterpret_cast<float4 *>(scan + warp * 128 + 4 * lane) = make_float4(run[0], run[1], run[2], run[3]);
+            mtot[I * 128 + fc2] = run;
             named_sync(1, kCompute);
-            if (tid < 128) {  // per channel: the end term plus the later warps' totals, in place
-                float acc = sEnd2[256 * par + tid] + sEnd2[256 * par + 128 + tid];
+            float after = mgam[fc2] * (mend1[fc2] + mend1[128 + fc2] + mend1[256 + fc2] + mend1[384 + fc2]) +
+                          mendk[fc2] + mendk[128 + fc2] + mendk[256 + fc2] + mendk[384 + fc2];
 #pragma unroll
-                for (int w2 = kWarps - 1; w2 >= 0; --w2) {
-                    const float t = scan[w2 * 128 + tid];
-                    scan[w2 * 128 + tid] = acc;
-                    acc += t;
-                }
-            }
-            named_sync(1, kCompute);
-            const float4 a4 = *reinterpret_cast<const float4 *>(scan + warp * 128 + 4 * lane);
-            const float after[4] = {a4.x, a4.y, a4.z, a4.w};
+            for (int J = 0; J < 4; ++J)
+                if (J > I) after += mtot[J * 128 + fc2];
 #pragma unroll
-            for (int m = 0; m < 4; ++m)
-                *reinterpret_cast<float4 *>(sm + RG + sw128_chunk(4 * warp + m, lane, 64)) =
-                    make_float4(x[m][0] + after[0], x[m][1] + after[1], x[m][2] + after[2], x[m][3] + after[3]);
+            for (int r = 0; r < 16; ++r)
+                *reinterpret_cast<float *>(sm + RG + raw32(16 * I + r, fc2)) = x[r] + after;
         }
         fence_proxy_async();
         fence_before_sync();
@@ -822,7 +968,7 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
         }
     }
     if (issuer) bulk_wait_all();
-    if (!(big <= kRange) || !(gbig <= 9.f)) record_status(status, GDN2_ERR_RANGE);
+    if (!(big <= kRange)) record_status(status, GDN2_ERR_RANGE);
     if (!ok && issuer) {
         record_status(status, GDN2_ERR_TIMEOUT);
         // every copy landed and every issued product done before the shared
@@ -831,8 +977,6 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
         if (issued[2] > 0) mbar_wait(&bars[3], (issued[2] - 1) & 1, kWait);
         mbar_wait(&bars[1], 0, kWait);
         mbar_wait(&bars[1], 1, kWait);
-        mbar_wait(&bars[2], 0, kWait);
-        mbar_wait(&bars[2], 1, kWait);
     }
     fence_before_sync();
     __syncthreads();

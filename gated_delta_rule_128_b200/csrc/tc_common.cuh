@@ -1,14 +1,27 @@
-// Pieces shared by the tensor-core forward and backward kernels: the in-chunk
-// cumulative log-decay, the decay-scaled fp16 operand tiles, and small store
-// helpers.  Thread layout of these helpers (256 threads, 64-row chunk, 128 key
-// channels): warp w owns rows 8w..8w+7, lane l owns channels 4l..4l+3.
+// Pieces shared by the tensor-core forward and backward kernels: the chunk's
+// decay frames, raw-tile addressing, fp16 store helpers and the warp-level
+// tf32 tile product.
 //
-// Decay factors are taken relative to the chunk's middle row m = 31
-// ("Gated DeltaNet-2", LIT-802 review, Key takeaways 2: the state is
-// normalised by the cumulative decay; here the normalisation point is moved
-// to the chunk's middle to keep every factor within fp16 range):
-//   E = e^(G - G_m),  Qb = q.E,  Kc = b.k.E,  Kh = k / E,
-//   gamma_m = e^(G_L - G_m) (sGam),  e^(G_m) (sRef).
+// Decay frames ("Gated DeltaNet-2", LIT-802 review, Key takeaways 2: the
+// state is normalised by the cumulative decay so that D_t folds into the two
+// factors of every rank-one erase).  Per chunk of 64 rows t and key channel c,
+// G_t = sum_{i <= t} g_i (rows past the sequence's end hold g = 0), and the
+// chunk splits into four 16-row blocks I with s_I = G_{16I-1} (s_0 = 0) and
+// e_I = G_{16I+15}:
+//   * state side, chunk-start frame, every factor <= 1 for any g <= 0:
+//       E_t = e^G_t,  F_t = e^(G_63 - G_t),  gamma = e^G_63;
+//   * pair factors e^(G_r - G_j) (r >= j) inside the chunk, which the chunk-
+//     start frame would split into e^G_r and e^-G_j (the second unbounded):
+//       - r and j in different blocks I > J: e^(G_r - s_I) * chi_IJ *
+//         e^(e_J - G_j) with chi_IJ = e^(s_I - e_J); all three are <= 1, so an
+//         fp16 operand can only underflow where the pair factor itself is
+//         below fp16's resolution;
+//       - r and j in the same block: l_r / l_j with l_t = e^(G'_t - G'_m),
+//         m the block's row 7, in float32 (tf32 products), where G' sums
+//         g' = max(g, -kClampG).  A clamped token lies between r and j only if
+//         the true factor is below e^-kClampG, and then the computed one is
+//         too; otherwise the two are equal.  Within a block |G' - G'_m| is at
+//         most 8 kClampG, inside float32's range.
 #pragma once
 
 #include "common.cuh"
@@ -17,6 +30,9 @@
 namespace gdn2 {
 namespace tcc {
 using namespace tc;
+
+// per-token floor of the log-decay inside the same-block pair factors
+constexpr float kClampG = 9.0f;
 
 __device__ __forceinline__ void st_h4(unsigned char *p, float a, float b, float c, float d) {
     uint2 v = make_uint2(pack_f16(a, b), pack_f16(c, d));
@@ -49,94 +65,59 @@ __device__ __forceinline__ void ld_h8(const unsigned char *p, float *x) {
     }
 }
 
-// Step 1 of the cumsum: local inclusive prefix over the warp's 8 rows (raw g
-// tile row-major [64][128] f32); the warp's totals go to scan[warp][128].
-__device__ __forceinline__ void cumsum_local(const float *rg, float *scan, int warp, int lane,
-                                             float G[8][4]) {
-    float run[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int m = 0; m < 8; ++m) {
-        float4 t = *reinterpret_cast<const float4 *>(rg + (8 * warp + m) * 128 + 4 * lane);
-        run[0] += t.x; run[1] += t.y; run[2] += t.z; run[3] += t.w;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) G[m][i] = run[i];
-    }
-    *reinterpret_cast<float4 *>(scan + warp * 128 + 4 * lane) = make_float4(run[0], run[1], run[2], run[3]);
+// Raw [64 rows][128 channels] tiles as TMA lands them with 128-byte swizzle:
+// bf16 tiles as two boxes of 64 channels, float32 tiles as four boxes of 32
+// channels, 8 KB per box.  Byte offset of element (t, c).
+__host__ __device__ __forceinline__ uint32_t raw16(int t, int c) {
+    return (uint32_t)((c >> 6) * 8192) + sw128_off(t, c & 63, 64);
+}
+__host__ __device__ __forceinline__ uint32_t raw32(int t, int c) {
+    return (uint32_t)((c >> 5) * 8192) + sw128_chunk(t, (c & 31) >> 2, 64) + (uint32_t)((c & 3) * 4);
 }
 
-// Step 2 (after a block barrier): add the earlier warps' totals and express G
-// relative to row 31; warp 0 writes e^(G_L - G_m) and e^(G_m) per channel.
-// Rows past the chunk's end hold g = 0 (zero-filled tiles), so row 63
-// carries G_L of a short last chunk.
-__device__ __forceinline__ void cumsum_finish(const float *scan, int warp, int lane, float G[8][4],
-                                              float *sGam, float *sRef) {
-    float pre[4] = {0.f, 0.f, 0.f, 0.f}, tot[4] = {0.f, 0.f, 0.f, 0.f}, ref[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int w2 = 0; w2 < 8; ++w2) {
-        float4 t = *reinterpret_cast<const float4 *>(scan + w2 * 128 + 4 * lane);
-        float tv[4] = {t.x, t.y, t.z, t.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            if (w2 < warp) pre[i] += tv[i];
-            if (w2 < 4) ref[i] += tv[i];
-            tot[i] += tv[i];
-        }
-    }
-#pragma unroll
-    for (int m = 0; m < 8; ++m)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) G[m][i] += pre[i] - ref[i];
-    if (warp == 0)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            sGam[4 * lane + i] = __expf(tot[i] - ref[i]);
-            sRef[4 * lane + i] = __expf(ref[i]);
-        }
+// Warp-level tf32 tile product D = A B + D (m16n8k8, f32 accumulate).
+// Fragments (g = lane / 4, t = lane % 4): a0 (g, t), a1 (g + 8, t),
+// a2 (g, t + 4), a3 (g + 8, t + 4); b0 (k = t, n = g), b1 (k = t + 4, n = g);
+// c0 (g, 2t), c1 (g, 2t + 1), c2 (g + 8, 2t), c3 (g + 8, 2t + 1).
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
 }
-
-// Operands of the chunk record from the raw q, k (bf16 [64][128]) and b (f32
-// [64][128]) tiles: Kc = b.k.E into rows 0..63 and Qb = q.E into rows
-// 64..127 of the [128][128] K-major tile at oWQ, Kh = k / E into the
-// [64][128] K-major tile at oKh (E = e^(G - G_m)).  Every input row is loaded
-// before the first store, so that the loads overlap.  Returns the largest
-// |G - G_m| seen: with |q|, |k|, |b| <= 8 every factor stays below 8 e^|G|,
-// so the fp16 range holds while that value stays below 9.
-__device__ __forceinline__ float write_factors_rec(const unsigned char *rq, const unsigned char *rk,
-                                                   const float *rb, const float G[8][4],
-                                                   unsigned char *oWQ, unsigned char *oKh,
-                                                   int warp, int lane) {
-    uint2 qr[8], kr[8];
-    float4 bv[8];
-#pragma unroll
-    for (int m = 0; m < 8; ++m) {
-        const int r = 8 * warp + m;
-        qr[m] = *reinterpret_cast<const uint2 *>(rq + r * 256 + lane * 8);
-        kr[m] = *reinterpret_cast<const uint2 *>(rk + r * 256 + lane * 8);
-        bv[m] = *reinterpret_cast<const float4 *>(rb + r * 128 + 4 * lane);
-    }
-    float gmax = 0.f;
-#pragma unroll
-    for (int m = 0; m < 8; ++m) {
-        const int r = 8 * warp + m;
-        const __nv_bfloat162 *q2 = reinterpret_cast<const __nv_bfloat162 *>(&qr[m]);
-        const __nv_bfloat162 *k2 = reinterpret_cast<const __nv_bfloat162 *>(&kr[m]);
-        const float qf[4] = {__low2float(q2[0]), __high2float(q2[0]), __low2float(q2[1]), __high2float(q2[1])};
-        const float kf[4] = {__low2float(k2[0]), __high2float(k2[0]), __low2float(k2[1]), __high2float(k2[1])};
-        const float bf[4] = {bv[m].x, bv[m].y, bv[m].z, bv[m].w};
-        float qb[4], kc[4], kh[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float e = __expf(G[m][i]), ei = __expf(-G[m][i]);
-            qb[i] = qf[i] * e;
-            kc[i] = bf[i] * kf[i] * e;
-            kh[i] = kf[i] * ei;
-            gmax = fmaxf(gmax, fabsf(G[m][i]));
-        }
-        st_h4(oWQ + sw128_off(r, 4 * lane, 128), kc[0], kc[1], kc[2], kc[3]);
-        st_h4(oWQ + sw128_off(r + 64, 4 * lane, 128), qb[0], qb[1], qb[2], qb[3]);
-        st_h4(oKh + sw128_off(r, 4 * lane, 64), kh[0], kh[1], kh[2], kh[3]);
-    }
-    return gmax;
+__device__ __forceinline__ void mma_tf32_16x8x8(float *c, const uint32_t *a, const uint32_t *b) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+// Warp-level fp16 tile product D = A B + D (m16n8k16, f32 accumulate).
+// Fragments: a0..a3 as f16 pairs: a0 (g, 2t..2t+1), a1 (g + 8, 2t..), a2 (g,
+// 2t + 8..), a3 (g + 8, 2t + 8..); b0 (k = 2t..2t+1, n = g), b1 (k = 2t + 8..,
+// n = g); c as for the tf32 product.
+__device__ __forceinline__ void mma_f16_16x8x16(float *c, const uint32_t *a, const uint32_t *b) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+// ldmatrix: four 8x8 b16 matrices from shared memory (rows addressed by
+// lanes 8i..8i+7 for matrix i), plain or transposed
+__device__ __forceinline__ void ldsm_x4(uint32_t *r, uint32_t saddr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(saddr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t *r, uint32_t saddr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(saddr));
+}
+// (x.lo s, x.hi s) for an f16 pair x, multiplied in float32 and rounded once
+__device__ __forceinline__ uint32_t h2scale(uint32_t x, float s) {
+    const float2 f = __half22float2(*reinterpret_cast<__half2 *>(&x));
+    return pack_f16(f.x * s, f.y * s);
 }
 
 }  // namespace tcc

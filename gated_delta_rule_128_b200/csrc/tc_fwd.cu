@@ -4,25 +4,27 @@
 //
 // "Gated DeltaNet-2" (LIT-802 review, Key takeaways 2; paper Secs. 3.3-3.4,
 // Apps. A-B): only the state crosses chunk borders.  Per chunk of 64 tokens
-// entering with state S (factors relative to the chunk's middle row m,
-// S_m = diag(e^G_m) S, U = w.v):
-//   Delta = T U - W S_m
-//   O = Qb S_m + P Delta,   S_next = diag(e^(G_L - G_m)) (S_m + Kh^T Delta)
+// entering with state S (chunk-start frame, tc_common.cuh; U = w.v):
+//   Delta = T U - W S
+//   O = Qb S + P Delta,   S_next = diag(gamma) S + Kb^T Delta
+// Every record factor is at most 1 in magnitude for any g <= 0, so the state
+// stays at its true scale and no factor can overflow.
 //
 // One CTA owns one (b, h) and one 64-column half of d_v and walks the
-// sequence's chunks in order with its fp32 state slice resident in tensor
-// memory.  The chunk records are double-buffered in shared memory and
-// requested two chunks ahead, since they do not depend on the state.
+// sequence's chunks in order with its fp32 state slice in registers (each
+// thread one key row, 32 columns).  The chunk records are double-buffered in
+// shared memory and requested two chunks ahead, since they do not depend on
+// the state.
 //
 // Both state-side products are M = 128 tcgen05.mma groups into one
 // [Delta; O] accumulator (rows 0..63 Delta, 64..127 O; two such accumulators
 // alternate between chunks):
-//   (1) [T; 0] U + [-W; Qb] S_m            -> Delta and Qb S_m
-//   (2) [0; P] Delta,  and  S += Kh^T Delta
-// Warp roles: warps 0, 1, 4, 5 (TMEM lanes 0..63) read Delta; warps 2, 3,
-// 6, 7 (lanes 64..127) read the previous chunk's O and form the next chunk's
-// U = w.v off the state's path; all warps rescale the state into the next
-// chunk's frame.
+//   (1) [T; 0] U + [-W; Qb] S              -> Delta and Qb S
+//   (2) [0; P] Delta,  and  X = Kb^T Delta (a fresh accumulator)
+// then S_next = gamma S + X in registers.  Warp roles: warps 0, 1, 4, 5 (TMEM
+// lanes 0..63) read Delta; warps 2, 3, 6, 7 (lanes 64..127) read the previous
+// chunk's O and form the next chunk's U = w.v off the state's path; all warps
+// update the state.
 //
 // Precision and range: fp16 operands carry 11 significant bits (bf16 carries
 // 8, which left the output error at the 5e-3 tolerance); Delta is formed in
@@ -30,8 +32,7 @@
 // GDN2_ERR_RANGE.
 //
 // For the backward the call can also leave in the workspace (TcWs): every
-// chunk's entry state in its own frame, S_m (fp16, a copy of the operand),
-// S_T (fp16, true scale) and Delta per chunk.
+// chunk's entry state S_c (fp16, a copy of the operand) and Delta per chunk.
 
 #include "common.cuh"
 #include "tc.cuh"
@@ -53,11 +54,11 @@ constexpr uint32_t STG = 0;                  // two record stages
 constexpr uint32_t RAW_V = 2 * STAGE;        // v half, bf16 [64 pos][64]
 constexpr uint32_t RAW_W = RAW_V + 8192;     // w half, f32  [64 pos][64]
 constexpr uint32_t OP_U = RAW_W + 16384;     // two U = w.v tiles [64 pos][64 v] MN-major, 8 KB each
-constexpr uint32_t OP_S = OP_U + 16384;      // S_m (fp16)   [128 key][64 v] MN-major
+constexpr uint32_t OP_S = OP_U + 16384;      // S (fp16)     [128 key][64 v] MN-major
 constexpr uint32_t OP_D = OP_S + 16384;      // Delta        [64 pos][64 v]  MN-major
 constexpr uint32_t MISC = OP_D + 8192;       // mbarriers, TMEM slot
 constexpr uint32_t SMEM_BYTES = MISC + 128 + 1024;
-// tensor memory columns (256 allocated): state, then two [Delta; O] accumulators
+// tensor memory columns (256 allocated): Kb^T Delta, then two [Delta; O] accumulators
 constexpr uint32_t TM_S = 0, TM_X = 64;
 constexpr uint32_t ID_KM128x64 = idesc_f16(128, 64, false, true);
 constexpr uint32_t ID_MM128x64 = idesc_f16(128, 64, true, true);
@@ -160,7 +161,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mv, const __grid_constant__ CU
         mma_commit(&bars[3]);
         ++groups[0];
     };
-    auto ckpt = [&](int c) { return ws + lay.ckS + ((bh * (NC + 1) + c) * 2 + vh) * 16384; };
+    auto ckpt = [&](int c) { return ws + lay.ckS + ((bh * NC + c) * 2 + vh) * 16384; };
     // O rows of chunk cc (O warps): accumulator rows 64..127, this warp's 32 columns
     auto store_o = [&](int cc) {
         float ov[32];
@@ -182,28 +183,22 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mv, const __grid_constant__ CU
     }
     if (tid == 64) load_vw(0);
 
-    // ---------------- prologue: S_m of chunk 0 (TMEM, OP_S); U of chunk 0
+    // ---------------- prologue: S of chunk 0 (registers, OP_S); U of chunk 0
     bool ok = mbar_wait(&bars[0], 0, kWait);
+    float sreg[32];  // this thread's state row `key`, columns v0 + 32 half + j
     {
         const size_t so = st_off(d, bb, h);
-        float x[32];
 #pragma unroll
         for (int j = 0; j < 32; j += 4) {
             float4 t = S0 ? *reinterpret_cast<const float4 *>(S0 + so + (size_t)key * 128 + v0 + 32 * half + j)
                           : make_float4(0.f, 0.f, 0.f, 0.f);
-            x[j] = t.x; x[j + 1] = t.y; x[j + 2] = t.z; x[j + 3] = t.w;
+            sreg[j] = t.x; sreg[j + 1] = t.y; sreg[j + 2] = t.z; sreg[j + 3] = t.w;
         }
-        const float e = reinterpret_cast<const float *>(sm + STG + S_FAC)[128 + key];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) x[j] *= e;
-        tmem_st16(taddr(tm + TM_S, quarter * 32, 32 * half), x);
-        tmem_st16(taddr(tm + TM_S, quarter * 32, 32 * half + 16), x + 16);
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
-            st_h8(sm + OP_S + sw128_chunk(key, 4 * half + jj, 128), x + 8 * jj);
-            big = absmax8(x + 8 * jj, big);
+            st_h8(sm + OP_S + sw128_chunk(key, 4 * half + jj, 128), sreg + 8 * jj);
+            big = absmax8(sreg + 8 * jj, big);
         }
-        tmem_wait_st();
     }
     if (!dwarp) {
         ok = mbar_wait(&bars[2], 0, kWait) && ok;
@@ -255,7 +250,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mv, const __grid_constant__ CU
                     mma_bf16(x, kstep_kmajor(dZP, 128, ks), kstep_mnmajor(dD, ks), ID_KM128x64, 1);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16(tm + TM_S, kstep_mnmajor(dK, ks), kstep_mnmajor(dD, ks), ID_MM128x64, 1);
+                    mma_bf16(tm + TM_S, kstep_mnmajor(dK, ks), kstep_mnmajor(dD, ks), ID_MM128x64, ks > 0);
                 mma_commit(&bars[4]);
                 ++groups[1];
                 if (keep) {  // Delta of this chunk and half, for the backward
@@ -274,43 +269,30 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mv, const __grid_constant__ CU
                 if (tid == 64 && c + 2 < NC) load_vw(c + 2);
             }
         }
-        // ---------------- state into the next chunk's frame
+        // ---------------- S_next = gamma S + Kb^T Delta
         ok = mbar_wait(&bars[4], par, kWait) && ok;
-        const float gam = reinterpret_cast<const float *>(stg + S_FAC)[key];  // e^(G_L - G_m)
-        float ref = 1.f;                                                      // next e^G_m
-        if (c + 1 < NC) {
-            ok = mbar_wait(&bars[s ^ 1], ((c + 1) >> 1) & 1, kWait) && ok;
-            ref = reinterpret_cast<const float *>(sm + STG + (s ^ 1) * STAGE + S_FAC)[128 + key];
-        }
+        const float gam = reinterpret_cast<const float *>(stg + S_FAC)[key];  // e^G_63
+        // the next chunk's record has landed before its first products are issued
+        if (c + 1 < NC) ok = mbar_wait(&bars[s ^ 1], ((c + 1) >> 1) & 1, kWait) && ok;
         fence_after_sync();
         {
-            float sv[32];
-            tmem_ld16(taddr(tm + TM_S, quarter * 32, 32 * half), sv);
-            tmem_ld16(taddr(tm + TM_S, quarter * 32, 32 * half + 16), sv + 16);
+            float xv[32];
+            tmem_ld16(taddr(tm + TM_S, quarter * 32, 32 * half), xv);
+            tmem_ld16(taddr(tm + TM_S, quarter * 32, 32 * half + 16), xv + 16);
             tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) sv[j] *= gam;  // S_{c+1}, true scale
+            for (int j = 0; j < 32; ++j) sreg[j] = fmaf(gam, sreg[j], xv[j]);
             if (c + 1 < NC) {
 #pragma unroll
-                for (int j = 0; j < 32; ++j) sv[j] *= ref;  // S_m of the next chunk
-                tmem_st16(taddr(tm + TM_S, quarter * 32, 32 * half), sv);
-                tmem_st16(taddr(tm + TM_S, quarter * 32, 32 * half + 16), sv + 16);
-#pragma unroll
                 for (int jj = 0; jj < 4; ++jj) {
-                    st_h8(sm + OP_S + sw128_chunk(key, 4 * half + jj, 128), sv + 8 * jj);
-                    big = absmax8(sv + 8 * jj, big);
+                    st_h8(sm + OP_S + sw128_chunk(key, 4 * half + jj, 128), sreg + 8 * jj);
+                    big = absmax8(sreg + 8 * jj, big);
                 }
-                tmem_wait_st();
-            } else {
-                if (ST) {
-                    float *dst = ST + st_off(d, bb, h) + (size_t)key * 128 + v0 + 32 * half;
+            } else if (ST) {
+                float *dst = ST + st_off(d, bb, h) + (size_t)key * 128 + v0 + 32 * half;
 #pragma unroll
-                    for (int j = 0; j < 32; j += 4)
-                        *reinterpret_cast<float4 *>(dst + j) = make_float4(sv[j], sv[j + 1], sv[j + 2], sv[j + 3]);
-                }
-                if (keep)
-#pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) st_h8(ckpt(NC) + sw128_chunk(key, 4 * half + jj, 128), sv + 8 * jj);
+                for (int j = 0; j < 32; j += 4)
+                    *reinterpret_cast<float4 *>(dst + j) = make_float4(sreg[j], sreg[j + 1], sreg[j + 2], sreg[j + 3]);
             }
         }
         if (tid == 0) bulk_wait_read();  // the Delta copy has left OP_D
