@@ -129,14 +129,21 @@ inline SimtWs simt_ws_layout(const Dims &d) {
 //   ckndU [bh][NC][2]          8 KB  -dU
 // A forward that is not followed by a backward needs `rec` only.
 //
-// Chunk record: chunk-start-frame operands (fp16, 128-byte swizzled; see
-// tc.cuh for the layouts and tc_common.cuh for the frames)
+// Chunk record: operands in the chunk's frame (fp16, 128-byte swizzled; see
+// tc.cuh for the layouts and tc_common.cuh for the frames).  With the frame
+// factor s (per key channel): s = 1 (the chunk-start frame) or, for a mild
+// chunk, s = e^G_31 (the frame of row 31):
 //   REC_WQ   [-W; Qb] as one [128 rows][128 key] K-major tile: rows 0..63
-//            -W = -T Kc (Kc = b.k.e^G), rows 64..127 Qb = q.e^G (32 KB)
-//   REC_KH   Kb = k.e^(G_63 - G)        [64 pos][128 key] K-major (16 KB)
+//            -W = -T Kc (Kc = b.k.e^G / s), rows 64..127 Qb = q.e^G / s (32 KB)
+//   REC_KH   Kx: Kb = k.e^(G_63 - G) (s = 1), or Kh = k.e^(G_31 - G) (mild)
+//            [64 pos][128 key] K-major (16 KB)
 //   REC_T    T = (I + A)^-1             [64][64] K-major (8 KB)
 //   REC_P    P                          [64][64] K-major (8 KB)
-//   REC_FAC  gamma = e^G_63 [128] f32, then 128 unused floats
+//   REC_FAC  gamma = e^G_63 [128] f32, then s [128] f32, stored as -1 where
+//            s = 1 (a negative value marks the chunk-start frame)
+// So that every consumer can handle both frames with per-channel scales:
+//   S_next = gamma S + r Kx^T Delta,  r = 1 (s = 1) or gamma / s (mild);
+//   the operand state is s S, the operand state gradient r dS'.
 constexpr uint32_t REC_WQ = 0, REC_KH = 32768, REC_T = 49152, REC_P = 57344, REC_FAC = 65536,
                    REC_BYTES = 66560;
 struct TcWs {

@@ -137,8 +137,10 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
         tma_load_4d(sm + VW + 8192, &mw, v0 + 32, h, cc * 64, bb, &bars[4]);
         ++issued[4];
     };
-    auto rec_gamma = [&](int cc) {  // gamma = e^G_63 of chunk cc
-        return reinterpret_cast<const float *>(sm + STG + (cc & 1) * REC_BYTES + REC_FAC)[key];
+    // the frame factor s of chunk cc (1 for the chunk-start frame)
+    auto rec_s = [&](int cc) {
+        const float sv = reinterpret_cast<const float *>(sm + STG + (cc & 1) * REC_BYTES + REC_FAC)[128 + key];
+        return sv < 0.f ? 1.f : sv;
     };
     // dO of the chunk in RAW_DO -> fp16 operand (each thread 16 values)
     auto convert_do = [&]() {
@@ -160,19 +162,24 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
         big = absmax8(x, big);
         big = absmax8(x + 8, big);
     };
-    // dS' of the next chunk to process: diag(gamma) dS' into TMEM (the
-    // products add the rest of dS_c to it), dS' as the fp16 operand (this
-    // thread's row, 32 columns)
-    auto put_ds = [&](const float *x, float gam) {
+    // dS' of the next chunk cc to process: diag(gamma / s) dS' into TMEM (the
+    // products add the rest of dS_c / s to it), r dS' as the fp16 operand
+    // (this thread's row, 32 columns); r = 1, or gamma / s for a mild chunk
+    auto put_ds = [&](const float *x, int cc) {
+        const float *fac = reinterpret_cast<const float *>(sm + STG + (cc & 1) * REC_BYTES + REC_FAC);
+        const float gam = fac[key], sv = fac[128 + key];
+        const float g_s = sv < 0.f ? gam : gam / sv, r = sv < 0.f ? 1.f : gam / sv;
         float y[32];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) y[j] = gam * x[j];
+        for (int j = 0; j < 32; ++j) y[j] = g_s * x[j];
         tmem_st16(taddr(tm + TM_DS, quarter * 32, 32 * half), y);
         tmem_st16(taddr(tm + TM_DS, quarter * 32, 32 * half + 16), y + 16);
 #pragma unroll
+        for (int j = 0; j < 32; ++j) y[j] = r * x[j];
+#pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
-            st_h8(sm + OP_DS + sw128_chunk(key, 4 * half + jj, 128), x + 8 * jj);
-            big = absmax8(x + 8 * jj, big);
+            st_h8(sm + OP_DS + sw128_chunk(key, 4 * half + jj, 128), y + 8 * jj);
+            big = absmax8(y + 8 * jj, big);
         }
     };
     // dU of chunk cc (TMEM) -> dv, dw in place of v, w; -dU staged (compute
@@ -235,7 +242,7 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
         }
         ok = mbar_wait(&bars[(NC - 1) & 1], 0, kWait);
         ok = mbar_wait(&bars[2], 0, kWait) && ok;
-        put_ds(x, rec_gamma(NC - 1));
+        put_ds(x, NC - 1);
         convert_do();
         tmem_wait_st();
     }
@@ -324,6 +331,9 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
             tmem_ld16(taddr(tm + TM_DS, quarter * 32, 32 * half), sv);
             tmem_ld16(taddr(tm + TM_DS, quarter * 32, 32 * half + 16), sv + 16);
             tmem_wait_ld();
+            const float se = rec_s(c);  // tensor memory holds dS_c / s
+#pragma unroll
+            for (int j = 0; j < 32; ++j) sv[j] *= se;
             if (c == 0) {
                 if (dS0) {
                     float *dst = dS0 + st_off(d, bb, h) + (size_t)key * 128 + v0 + 32 * half;
@@ -332,7 +342,7 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
                         *reinterpret_cast<float4 *>(dst + j) = make_float4(sv[j], sv[j + 1], sv[j + 2], sv[j + 3]);
                 }
             } else {
-                put_ds(sv, rec_gamma(c - 1));
+                put_ds(sv, c - 1);
                 convert_do();
                 tmem_wait_st();
             }
@@ -378,7 +388,7 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
 // ============================================================ chunk kernel
 namespace tbg {
 constexpr int kCompute = 512;             // warps 0..15 form operands and outputs
-constexpr int kThreads = kCompute + 32;   // warp 16 issues the copies and products
+constexpr int kThreads = kCompute;        // thread 0 also issues the copies and products
 constexpr int kWarps = kCompute / 32;
 // raw tiles (128-B swizzled TMA boxes, tc_common.cuh raw16 / raw32); the
 // outputs are formed in place
@@ -398,21 +408,28 @@ constexpr uint32_t QA = 114688;   // q e^(G - s_I)
 constexpr uint32_t BA = 131072;   // b k e^(G - s_I)
 constexpr uint32_t AL = 147456;   // e^(G - s_I)
 constexpr uint32_t AB = 163840;   // e^(e_I - G)
+// mild tiles: q E, b k E, k / E, E, 1 / E in the same five slots (E = e^(G - G_31))
+constexpr uint32_t MQB = KA, MKC = QA, MKH = BA, MEM = AL, MEI = AB;
 constexpr uint32_t PD = 180224;   // masked dP [64][64] fp16 (sw128, R = 64)
 constexpr uint32_t AD = 188416;   // masked dA
-constexpr uint32_t DG32 = 196608; // diagonal blocks of dP, dA in f32 [2][4][16][17]
+constexpr uint32_t DG32 = 196608; // diagonal blocks of dP, dA as tf32 bits [2][4][16][17]
+constexpr uint32_t ESF = 205824;  // e^s_I and e^(G_63 - e_I) per block and channel [2][4][128] f32
 constexpr uint32_t MISC = 212992; // per-channel values (below), mbarriers, TMEM slot
-constexpr uint32_t M_TOT = 0, M_ES = 2048, M_EF = 4096, M_CHI = 6144, M_END1 = 9216, M_ENDK = 11264,
-                   M_GAM = 13312, M_BAR = 13824;
+// 8-row totals of G and of the clamped G [2][8][128]; chi [6][128]; the
+// chunk-end parts [4][128] twice; gamma [128]
+constexpr uint32_t M_TOT = 0, M_CHI = 8192, M_END1 = 11264, M_ENDK = 13312, M_GAM = 15360,
+                   M_FLAG = 15872, M_BAR = 15936;
 constexpr uint32_t SMEM_BYTES = MISC + M_BAR + 128 + 1024;
 constexpr uint32_t LOAD_A = 32768 + 81920;  // dO, -dU; Delta, S_c, dS'
 constexpr uint32_t LOAD_B = 98304;          // raw q, k, b, g
 constexpr uint32_t TM_Y1 = 0, TM_Y2 = 128, TM_Y3 = 256, TM_PA = 384;  // 512 columns
 constexpr uint32_t ID_PA = idesc_f16(128, 64, false, false);
 constexpr uint32_t ID_KK128 = idesc_f16(64, 128, false, false);
+constexpr uint32_t ID_KM128 = idesc_f16(64, 128, false, true);
+constexpr uint32_t ID_MM128 = idesc_f16(64, 128, true, true);
 constexpr long long kWait = 2000000000LL;
 constexpr float kRange = 6.0e4f;
-static_assert(DG32 + 2 * 4 * 16 * 17 * 4 <= MISC, "pair-term data fits over the operands");
+static_assert(DG32 + 2 * 4 * 16 * 17 * 4 <= ESF && ESF + 4096 <= MISC, "pair-term data fits over the operands");
 static_assert(SMEM_BYTES <= 232448, "shared memory");
 }  // namespace tbg
 
@@ -436,11 +453,11 @@ __device__ __forceinline__ void tmem_ld16x256x1(uint32_t taddr, float *v) {
 // index of the block pair (I, J), I > J, among the six
 __host__ __device__ constexpr int pair_ix(int I, int J) { return I * (I - 1) / 2 + J; }
 
-// Persistent: one CTA per SM walks the (b, h, chunk) tiles, full d_v.  Warp 16
-// loads the tile (raw q, k, b, g, dO as 128-B swizzled TMA boxes; S_c, dS',
-// Delta, -dU from the workspace) and issues the tensor-core products; compute
-// warp w owns row block I = w % 4 (16 rows, TMEM lane quarter I) and channel
-// quarter Q = w / 4 (32 channels):
+// Persistent: one CTA per SM walks the (b, h, chunk) tiles, full d_v.  Thread
+// 0 also loads the tile (raw q, k, b, g, dO as 128-B swizzled TMA boxes; S_c,
+// dS', Delta, -dU from the workspace) and issues the tensor-core products (16
+// warps leave 128 registers per thread); warp w owns row block I = w % 4 (16
+// rows, TMEM lane quarter I) and channel quarter Q = w / 4 (32 channels):
 //   (1) [dP; dA] = [dO; -dU] Delta^T (M = 128), Y1 = dO S_c^T, Y2 = -dU S_c^T,
 //       Y3 = Delta dS'^T on the tensor cores, while the warps form the
 //       cumulative decay and the block factors;
@@ -463,13 +480,14 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
     extern __shared__ unsigned char smraw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smraw) + 1023) & ~static_cast<uintptr_t>(1023));
-    float *mtot = reinterpret_cast<float *>(sm + MISC + M_TOT);    // [4][128] block totals
-    float *mes = reinterpret_cast<float *>(sm + MISC + M_ES);      // [4][128] e^s_I
-    float *mef = reinterpret_cast<float *>(sm + MISC + M_EF);      // [4][128] e^(G_63 - e_I)
+    float *mtot = reinterpret_cast<float *>(sm + MISC + M_TOT);    // [8][128] 8-row totals (log2 units)
+    float *mtotc = mtot + 8 * 128;                                 // [8][128] the same, clamped
     float *mchi = reinterpret_cast<float *>(sm + MISC + M_CHI);    // [6][128] chi_IJ
     float *mend1 = reinterpret_cast<float *>(sm + MISC + M_END1);  // [4][128] rowsum(dS' . S_c) parts
     float *mendk = reinterpret_cast<float *>(sm + MISC + M_ENDK);  // [4][128] sum_t Kb Y3 parts
     float *mgam = reinterpret_cast<float *>(sm + MISC + M_GAM);    // [128] gamma
+    float *mes = reinterpret_cast<float *>(sm + ESF);              // [4][128] e^s_I (after the first products)
+    float *mef = mes + 4 * 128;                                    // [4][128] e^(G_63 - e_I)
     // 0 first-product operands (two parts), 1 products, 3 raw tiles, 4 dO
     // converted (one arrival per compute warp)
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + MISC + M_BAR);
@@ -481,7 +499,7 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
     const int ntiles = d.B * H * NC;
     const int I = warp & 3, Q = (warp >> 2) & 3;  // row block (TMEM lane quarter); channel quarter
     const int gq = lane >> 2, tq = lane & 3;
-    const bool compute = warp < kWarps, issuer = tid == kCompute;
+    const bool compute = true, issuer = tid == 0;
 
     if (warp == 0) {
         tmem_alloc(tslot, 512);
@@ -509,8 +527,9 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
         }
         ++issued[0];
     };
-    auto load_a2 = [&](int it) {  // Delta, S_c, dS'
-        mbar_expect_tx(&bars[0], LOAD_A - 32768);
+    auto load_a2 = [&](int it) {  // Delta, S_c, dS'; the chunk's frame factor (4 channels)
+        mbar_expect_tx(&bars[0], LOAD_A - 32768 + 16);
+        bulk_load(sm + MISC + M_FLAG, ws + lay.rec + (size_t)it * REC_BYTES + REC_FAC + 512, 16, &bars[0]);
         bulk_load(sm + DL, ws + lay.ckD + ((size_t)it * 2) * 8192, 16384, &bars[0]);
         bulk_load(sm + SMT, ws + lay.ckS + ((size_t)it * 2) * 16384, 32768, &bars[0]);
         bulk_load(sm + DXT, ws + lay.ckdS + ((size_t)it * 2) * 16384, 32768, &bars[0]);
@@ -536,36 +555,88 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
     }
 
     bool ok = true;
+    int nmild = 0;  // mild tiles done (second product groups committed to bars[2])
     for (int it = blockIdx.x, n = 0; it < ntiles; it += gridDim.x, ++n) {
         const int c = it % NC, bhi = it / NC, h = bhi % H, bb = bhi / H, c0 = c * 64;
         const uint32_t par = n & 1;
         const int nxt = it + (int)gridDim.x;
         const bool more = nxt < ntiles;
         ok = mbar_wait(&bars[0], par, kWait) && ok;
+        ok = mbar_wait(&bars[3], par, kWait) && ok;
 
-        // ---------------- dO to fp16; the issuer waits for this, then the
-        // first products run while the warps form the block factors
-        if (compute) {
+        // ---------------- dO to fp16, in place in the dO rows of [dO; -dU]
 #pragma unroll
-            for (int m = 0; m < 2; ++m) {  // the dO rows of [dO; -dU], in place
-                const int i = tid + kCompute * m;
-                unsigned char *p = sm + DN + (i >> 9) * 16384 + (i & 511) * 16;
-                uint4 raw = *reinterpret_cast<const uint4 *>(p);
-                const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-                float x[8];
+        for (int m = 0; m < 2; ++m) {
+            const int i = tid + kCompute * m;
+            unsigned char *p = sm + DN + (i >> 9) * 16384 + (i & 511) * 16;
+            uint4 raw = *reinterpret_cast<const uint4 *>(p);
+            const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+            float x[8];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    x[2 * e] = __low2float(b2[e]);
-                    x[2 * e + 1] = __high2float(b2[e]);
-                }
-                st_h8(p, x);
+            for (int e = 0; e < 4; ++e) {
+                x[2 * e] = __low2float(b2[e]);
+                x[2 * e + 1] = __high2float(b2[e]);
             }
-            fence_proxy_async();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[4]);
+            st_h8(p, x);
         }
+        // ---------------- cumulative decay (log2 units): warp w = rows 8 (w & 7)
+        // .. + 7 (block fb, half fh), channels fc, fc + 1 with fc = 64 (w >> 3) + 2 lane
+        const int frg = warp & 7, fb = frg >> 1, fh = frg & 1, fc = 64 * ((warp >> 3) & 1) + 2 * lane;
+        float gl[8][2], gc[8][2];
+        {
+            float run[2] = {0.f, 0.f}, runc[2] = {0.f, 0.f};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float2 g2 = *reinterpret_cast<const float2 *>(sm + RG + raw32(8 * frg + i, fc));
+                const float gv[2] = {g2.x * kLog2e, g2.y * kLog2e};
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    run[e] += gv[e];
+                    runc[e] += fmaxf(gv[e], -kClampG2);
+                    gl[i][e] = run[e];
+                    gc[i][e] = runc[e];
+                }
+            }
+            *reinterpret_cast<float2 *>(mtot + frg * 128 + fc) = make_float2(run[0], run[1]);
+            *reinterpret_cast<float2 *>(mtotc + frg * 128 + fc) = make_float2(runc[0], runc[1]);
+        }
+        named_sync(1, kCompute);
+        float btot[4][2], h0[2], h0c[2], sg[2], bt[2], all[2], pre[2] = {0.f, 0.f}, g31[2];
+#pragma unroll
+        for (int J = 0; J < 4; ++J) {
+            const float2 a2 = *reinterpret_cast<const float2 *>(mtot + (2 * J) * 128 + fc);
+            const float2 b2 = *reinterpret_cast<const float2 *>(mtot + (2 * J + 1) * 128 + fc);
+            btot[J][0] = a2.x + b2.x;
+            btot[J][1] = a2.y + b2.y;
+            if (J == fb) { h0[0] = a2.x; h0[1] = a2.y; }
+            if (2 * J < frg) { pre[0] += a2.x; pre[1] += a2.y; }
+            if (2 * J + 1 < frg) { pre[0] += b2.x; pre[1] += b2.y; }
+        }
+        {
+            const float2 c2 = *reinterpret_cast<const float2 *>(mtotc + 2 * fb * 128 + fc);
+            h0c[0] = c2.x;
+            h0c[1] = c2.y;
+        }
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            sg[e] = 0.f;
+            all[e] = 0.f;
+#pragma unroll
+            for (int J = 0; J < 4; ++J) {
+                if (J < fb) sg[e] += btot[J][e];
+                if (J == fb) bt[e] = btot[J][e];
+                all[e] += btot[J][e];
+            }
+            g31[e] = btot[0][e] + btot[1][e];
+        }
+        // ---------------- the frame of the chunk's record: mild (row 31, with S_c and
+        // dS' in the workspace as e^G_31 S_c and e^(G_63 - G_31) dS') or the
+        // chunk-start frame (a negative frame factor)
+        const bool mild = reinterpret_cast<const float *>(sm + MISC + M_FLAG)[0] > 0.f;
+        fence_proxy_async();
+        fence_before_sync();
+        __syncthreads();  // dO converted
         if (issuer) {
-            ok = mbar_wait(&bars[4], par, kWait) && ok;
             fence_after_sync();
             const uint64_t dn = desc_kmajor(smem_addr(sm + DN), 128, 0), dl = desc_kmajor(smem_addr(sm + DL), 64, 0),
                            s = desc_kmajor(smem_addr(sm + SMT), 128, 0), dx = desc_kmajor(smem_addr(sm + DXT), 128, 0),
@@ -580,328 +651,331 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
             }
             mma_commit(&bars[1]);
         }
-        // factor ownership: channel fc = 32 Q + lane, the 16 rows of block I
-        const int fc = 32 * Q + lane;
-        uint32_t pk[8][5];  // rows (2 i, 2 i + 1) as f16 pairs: k a_bar, q a, b k a, a, a_bar
-        if (compute) {
-            ok = mbar_wait(&bars[3], par, kWait) && ok;
-            float gl[16], gc[16];
-            {
-                float run = 0.f, runc = 0.f;
+        // ---------------- factors, held until the products have read S_c and dS':
+        // mild: q E, b k E, k / E, E, 1 / E (E = e^(G - G_31));
+        // else: k a_bar, q a, b k a, a, a_bar, and d = G' - G'_m in place of g
+        uint32_t pk[8][5];
+        if (!mild) {
+            float chi[4][2];
 #pragma unroll
-                for (int r = 0; r < 16; ++r) {
-                    const float gv = *reinterpret_cast<const float *>(sm + RG + raw32(16 * I + r, fc));
-                    run += gv;
-                    runc += fmaxf(gv, -kClampG);
-                    gl[r] = run;
-                    gc[r] = runc;
+            for (int e = 0; e < 2; ++e) {
+                float between = 0.f;  // block totals strictly between fb and I
+#pragma unroll
+                for (int I2 = 0; I2 < 4; ++I2) {
+                    chi[I2][e] = ex2(between);
+                    if (I2 > fb) between += btot[I2][e];
                 }
-                mtot[I * 128 + fc] = run;
             }
-            named_sync(1, kCompute);
-            float T4[4];
-#pragma unroll
-            for (int J = 0; J < 4; ++J) T4[J] = mtot[J * 128 + fc];
-            {
-                float s = 0.f, all = 0.f;
-#pragma unroll
-                for (int J = 0; J < 4; ++J) {
-                    if (J < I) s += T4[J];
-                    all += T4[J];
-                }
-                mes[I * 128 + fc] = __expf(s);
-                mef[I * 128 + fc] = __expf(all - s - T4[I]);
-                if (I == 0) mgam[fc] = __expf(all);
-                float between = 0.f;
+            if (fh == 0) {
 #pragma unroll
                 for (int I2 = 1; I2 < 4; ++I2)
-                    if (I2 > I) {
-                        mchi[pair_ix(I2, I) * 128 + fc] = I2 == I + 1 ? 1.f : __expf(between);
-                        between += T4[I2];
-                    }
-            }
-#pragma unroll
-            for (int r2 = 0; r2 < 8; ++r2) {
-                float v[2][5];
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int r = 2 * r2 + e, t = 16 * I + r;
-                    const float qv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + RQ + raw16(t, fc)));
-                    const float kv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + RK + raw16(t, fc)));
-                    const float bv = *reinterpret_cast<const float *>(sm + RB + raw32(t, fc));
-                    const float a = __expf(gl[r]), ab = __expf(T4[I] - gl[r]);
-                    v[e][0] = kv * ab;
-                    v[e][1] = qv * a;
-                    v[e][2] = bv * kv * a;
-                    v[e][3] = a;
-                    v[e][4] = ab;
-                    big = fmaxf(big, fmaxf(fabsf(v[e][0]), fmaxf(fabsf(v[e][1]), fabsf(v[e][2]))));
-                    *reinterpret_cast<float *>(sm + RG + raw32(t, fc)) = gc[r] - gc[7];
-                }
-#pragma unroll
-                for (int x = 0; x < 5; ++x) pk[r2][x] = pack_f16(v[0][x], v[1][x]);
-            }
-            // ---------------- chunk-end sum, once the products have read S_c and dS'
-            ok = mbar_wait(&bars[1], par, kWait) && ok;
-            fence_after_sync();
-            {
-                // channel fc, d_v quarter I: 32 values of S_c and dS'
-                float acc = 0.f;
-#pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                    const uint32_t off = (uint32_t)((I >> 1) * 16384) + sw128_chunk(fc, 4 * (I & 1) + jj, 128);
-                    float s8[8], d8[8];
-                    ld_h8(sm + SMT + off, s8);
-                    ld_h8(sm + DXT + off, d8);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) acc = fmaf(s8[e], d8[e], acc);
-                }
-                mend1[I * 128 + fc] = acc;
-            }
-            named_sync(1, kCompute);  // S_c, dS', Delta, [dO; -dU] are consumed
-            // ---------------- masked dP, dA (TMEM lanes 0..63 dP, 64..127 dA)
-            {
-                float row[16];
-                tmem_ld16(taddr(tm + TM_PA, I * 32, 16 * Q), row);
-                tmem_wait_ld();
-                const int pr = I * 32 + lane, r = pr & 63;
-                const bool isA = pr >= 64;
-#pragma unroll
-                for (int j = 0; j < 16; ++j) row[j] = (isA ? 16 * Q + j < r : 16 * Q + j <= r) ? row[j] : 0.f;
-                unsigned char *dst = sm + (isA ? AD : PD);
-#pragma unroll
-                for (int jj = 0; jj < 2; ++jj) {
-                    st_h8(dst + sw128_chunk(r, 2 * Q + jj, 64), row + 8 * jj);
-                    big = absmax8(row + 8 * jj, big);
-                }
-                if ((r >> 4) == Q) {
-                    float *dg32 = reinterpret_cast<float *>(sm + DG32) + ((isA ? 4 : 0) + Q) * 16 * 17 + (r & 15) * 17;
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) dg32[j] = row[j];
-                }
-            }
-            // ---------------- the block factors as fp16 tiles
-#pragma unroll
-            for (int r2 = 0; r2 < 8; ++r2) {
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const uint32_t off = raw16(16 * I + 2 * r2 + e, fc);
-#pragma unroll
-                    for (int x = 0; x < 5; ++x) {
-                        const uint32_t hv = e ? (pk[r2][x] >> 16) : (pk[r2][x] & 0xffffu);
-                        *reinterpret_cast<uint16_t *>(sm + KA + x * 16384 + off) = (uint16_t)hv;
-                    }
-                }
+                    if (I2 > fb + 1)
+                        *reinterpret_cast<float2 *>(mchi + pair_ix(I2, fb) * 128 + fc) = make_float2(chi[I2][0], chi[I2][1]);
             }
         }
+        if (fh == 0 && fb == 0) *reinterpret_cast<float2 *>(mgam + fc) = make_float2(ex2(all[0]), ex2(all[1]));
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int t = 8 * frg + i;
+            const float2 q2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(sm + RQ + raw16(t, fc)));
+            const float2 k2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(sm + RK + raw16(t, fc)));
+            const float2 b2 = *reinterpret_cast<const float2 *>(sm + RB + raw32(t, fc));
+            const float qv[2] = {q2.x, q2.y}, kv[2] = {k2.x, k2.y}, bv[2] = {b2.x, b2.y};
+            float v[5][2], dd[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                if (mild) {
+                    const float dl = pre[e] + gl[i][e] - g31[e];
+                    const float E = ex2(dl), Ei = ex2(-dl);
+                    v[0][e] = qv[e] * E;
+                    v[1][e] = bv[e] * kv[e] * E;
+                    v[2][e] = kv[e] * Ei;
+                    v[3][e] = E;
+                    v[4][e] = Ei;
+                } else {
+                    const float loc = fh ? h0[e] + gl[i][e] : gl[i][e];  // G_t - s_I
+                    const float a = ex2(loc), ab = ex2(bt[e] - loc);
+                    v[0][e] = kv[e] * ab;
+                    v[1][e] = qv[e] * a;
+                    v[2][e] = bv[e] * kv[e] * a;
+                    v[3][e] = a;
+                    v[4][e] = ab;
+                    dd[e] = fh ? gc[i][e] : gc[i][e] - h0c[e];  // G'_t - G'_m, m = the block's row 7
+                }
+                big = fmaxf(big, fmaxf(fabsf(v[0][e]), fmaxf(fabsf(v[1][e]), fabsf(v[2][e]))));
+            }
+#pragma unroll
+            for (int x = 0; x < 5; ++x) pk[i][x] = pack_f16(v[x][0], v[x][1]);
+            if (!mild) *reinterpret_cast<float2 *>(sm + RG + raw32(t, fc)) = make_float2(dd[0], dd[1]);
+        }
+        // ---------------- chunk-end sum, once the products have read S_c and dS'
+        ok = mbar_wait(&bars[1], par, kWait) && ok;
+        fence_after_sync();
+        {
+            // channel 32 (warp >> 2) + lane, d_v quarter warp & 3: 32 values of S_c
+            // and dS' (mild: of S_m and dX, whose product carries gamma already)
+            const int ec = 32 * ((warp >> 2) & 3) + lane, ev = warp & 3;
+            float acc = 0.f;
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                const uint32_t off = (uint32_t)((ev >> 1) * 16384) + sw128_chunk(ec, 4 * (ev & 1) + jj, 128);
+                float s8[8], d8[8];
+                ld_h8(sm + SMT + off, s8);
+                ld_h8(sm + DXT + off, d8);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc = fmaf(s8[e], d8[e], acc);
+            }
+            mend1[ev * 128 + ec] = acc;
+        }
+        named_sync(1, kCompute);  // S_c, dS', Delta, [dO; -dU] are consumed
+        if (!mild && fh == 0) {
+            *reinterpret_cast<float2 *>(mes + fb * 128 + fc) = make_float2(ex2(sg[0]), ex2(sg[1]));
+            *reinterpret_cast<float2 *>(mef + fb * 128 + fc) =
+                make_float2(ex2(all[0] - sg[0] - bt[0]), ex2(all[1] - sg[1] - bt[1]));
+        }
+        // ---------------- masked dP, dA (TMEM lanes 0..63 dP, 64..127 dA)
+        {
+            float row[16];
+            tmem_ld16(taddr(tm + TM_PA, I * 32, 16 * Q), row);
+            tmem_wait_ld();
+            const int pr = I * 32 + lane, r = pr & 63;
+            const bool isA = pr >= 64;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) row[j] = (isA ? 16 * Q + j < r : 16 * Q + j <= r) ? row[j] : 0.f;
+            unsigned char *dst = sm + (isA ? AD : PD);
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) {
+                st_h8(dst + sw128_chunk(r, 2 * Q + jj, 64), row + 8 * jj);
+                big = absmax8(row + 8 * jj, big);
+            }
+            if (!mild && (r >> 4) == Q) {
+                uint32_t *dg32 = reinterpret_cast<uint32_t *>(sm + DG32) + ((isA ? 4 : 0) + Q) * 16 * 17 + (r & 15) * 17;
+#pragma unroll
+                for (int j = 0; j < 16; ++j) dg32[j] = to_tf32(row[j]);
+            }
+        }
+        // ---------------- the factors as fp16 tiles
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint32_t off = raw16(8 * frg + i, fc);
+#pragma unroll
+            for (int x = 0; x < 5; ++x) *reinterpret_cast<uint32_t *>(sm + KA + x * 16384 + off) = pk[i][x];
+        }
+        fence_proxy_async();
+        fence_before_sync();
         __syncthreads();  // dP, dA and the factor tiles are in place
-        if (compute) {
+        if (mild) {
+            // ---------------- Kb^T Delta's share of the chunk-end term: sum_t Kh_m Y3
+            // with Y3 = Delta dX^T before the second products add to it
+            fence_after_sync();
+            const int r0 = 16 * I + gq;
+#pragma unroll 1
+            for (int nt = 0; nt < 4; ++nt) {
+                const int cc = 32 * Q + 8 * nt + 2 * tq;
+                float y3[4];
+                tmem_ld16x256x1(taddr(tm + TM_Y3 + 32 * Q + 8 * nt, I * 32, 0), y3);
+                tmem_wait_ld();
+                float part[2] = {0.f, 0.f};
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const float2 kh = __half22float2(*reinterpret_cast<const __half2 *>(sm + MKH + raw16(r0 + 8 * h2, cc)));
+                    part[0] = fmaf(kh.x, y3[2 * h2], part[0]);
+                    part[1] = fmaf(kh.y, y3[2 * h2 + 1], part[1]);
+                }
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    float v = part[e];
+                    v += __shfl_xor_sync(0xffffffffu, v, 4);
+                    v += __shfl_xor_sync(0xffffffffu, v, 8);
+                    v += __shfl_xor_sync(0xffffffffu, v, 16);
+                    if (gq == 0) mendk[I * 128 + cc + e] = v;
+                }
+            }
+            fence_before_sync();
+            __syncthreads();  // Y3 has been read
+            if (issuer) {
+                fence_after_sync();
+                const uint64_t kP = desc_kmajor(smem_addr(sm + PD), 64, 0), kA = desc_kmajor(smem_addr(sm + AD), 64, 0),
+                               mP = desc_mnmajor(smem_addr(sm + PD), 64, 0), mA = desc_mnmajor(smem_addr(sm + AD), 64, 0),
+                               qb = desc_mnmajor(smem_addr(sm + MQB), 64, 0), kc = desc_mnmajor(smem_addr(sm + MKC), 64, 0),
+                               kh = desc_mnmajor(smem_addr(sm + MKH), 64, 0);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                    const uint64_t b_kh = kstep_mnmajor(kh, ks);
+                    mma_bf16(tm + TM_Y1, kstep_kmajor(kP, 64, ks), b_kh, ID_KM128, 1);
+                    mma_bf16(tm + TM_Y2, kstep_kmajor(kA, 64, ks), b_kh, ID_KM128, 1);
+                    mma_bf16(tm + TM_Y3, kstep_mnmajor(mP, ks), kstep_mnmajor(qb, ks), ID_MM128, 1);
+                    mma_bf16(tm + TM_Y3, kstep_mnmajor(mA, ks), kstep_mnmajor(kc, ks), ID_MM128, 1);
+                }
+                mma_commit(&bars[2]);
+            }
+            ok = mbar_wait(&bars[2], nmild & 1, kWait) && ok;
+            ++nmild;
+            fence_after_sync();
+        }
+        if (!mild) {
             const uint32_t spd = smem_addr(sm + PD), sad = smem_addr(sm + AD);
-            const float *dgP = reinterpret_cast<const float *>(sm + DG32) + I * 16 * 17;
-            const float *dgA = dgP + 4 * 16 * 17;
+            const uint32_t *dgP = reinterpret_cast<const uint32_t *>(sm + DG32) + I * 16 * 17;
+            const uint32_t *dgA = dgP + 4 * 16 * 17;
             const int r0 = 16 * I + gq;  // this thread's fragment rows r0, r0 + 8
-            // ---------------- Z1, Z2: rows of block I, channels of quarter Q
-            float z1[4][4], z2[4][4];
-            {
-                float c1[4][4] = {}, c2[4][4] = {};
+            // per 8-channel n-tile: the pair terms Z1, Z2 (rows of block I), Z3
+            // (rows of block I as columns), then the outputs of those 8 channels
+#pragma unroll 1
+            for (int nt = 0; nt < 4; ++nt) {
+                const int cb = 32 * Q + 8 * nt;  // the n-tile's first channel
+                float c1[4] = {0.f, 0.f, 0.f, 0.f}, c2[4] = {0.f, 0.f, 0.f, 0.f}, c3[4] = {0.f, 0.f, 0.f, 0.f};
+                // blocks below the diagonal, fp16
                 for (int J = 0; J < I; ++J) {
-                    uint32_t aP[4], aA[4], bk[8];
-                    // A: rows 16 I + (l & 7) + 8 ((l >> 3) & 1), columns 16 J + 8 (l >> 4)
+                    uint32_t aP[4], aA[4], bk[2];
                     const int ar = 16 * I + (lane & 7) + 8 * ((lane >> 3) & 1), ac = 16 * J + 8 * (lane >> 4);
                     ldsm_x4(aP, spd + sw128_off(ar, ac, 64));
                     ldsm_x4(aA, sad + sw128_off(ar, ac, 64));
-                    // B: rows 16 J + (l & 7) + 8 ((l >> 3) & 1), channels 32 Q + 16 p + 8 (l >> 4)
-                    const int br = 16 * J + (lane & 7) + 8 * ((lane >> 3) & 1);
-                    ldsm_x4_t(bk, smem_addr(sm + KA + raw16(br, 32 * Q + 8 * (lane >> 4))));
-                    ldsm_x4_t(bk + 4, smem_addr(sm + KA + raw16(br, 32 * Q + 16 + 8 * (lane >> 4))));
+                    ldsm_x2_t(bk, smem_addr(sm + KA + raw16(16 * J + (lane & 7) + 8 * ((lane >> 3) & 1), cb)));
                     if (J + 1 < I) {
-#pragma unroll
-                        for (int nt = 0; nt < 4; ++nt) {
-                            const float chi = mchi[pair_ix(I, J) * 128 + 32 * Q + 8 * nt + gq];
-                            bk[2 * nt] = h2scale(bk[2 * nt], chi);
-                            bk[2 * nt + 1] = h2scale(bk[2 * nt + 1], chi);
-                        }
+                        const float chi = mchi[pair_ix(I, J) * 128 + cb + gq];
+                        bk[0] = h2scale(bk[0], chi);
+                        bk[1] = h2scale(bk[1], chi);
                     }
-#pragma unroll
-                    for (int nt = 0; nt < 4; ++nt) {
-                        mma_f16_16x8x16(c1[nt], aP, bk + 2 * nt);
-                        mma_f16_16x8x16(c2[nt], aA, bk + 2 * nt);
-                    }
+                    mma_f16_16x8x16(c1, aP, bk);
+                    mma_f16_16x8x16(c2, aA, bk);
                 }
-                // scale by a = e^(G_r - s_I)
-#pragma unroll
-                for (int nt = 0; nt < 4; ++nt) {
-                    const int cc = 32 * Q + 8 * nt + 2 * tq;
-#pragma unroll
-                    for (int h2 = 0; h2 < 2; ++h2) {
-                        const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(sm + AL + raw16(r0 + 8 * h2, cc)));
-                        z1[nt][2 * h2] = a.x * c1[nt][2 * h2];
-                        z1[nt][2 * h2 + 1] = a.y * c1[nt][2 * h2 + 1];
-                        z2[nt][2 * h2] = a.x * c2[nt][2 * h2];
-                        z2[nt][2 * h2 + 1] = a.y * c2[nt][2 * h2 + 1];
-                    }
-                }
-            }
-            {
-                // diagonal block: rows and columns of block I, tf32
-                float c1[4][4] = {}, c2[4][4] = {};
-#pragma unroll
-                for (int k0 = 0; k0 < 16; k0 += 8) {
-                    const uint32_t aP[4] = {to_tf32(dgP[gq * 17 + k0 + tq]), to_tf32(dgP[(gq + 8) * 17 + k0 + tq]),
-                                            to_tf32(dgP[gq * 17 + k0 + tq + 4]), to_tf32(dgP[(gq + 8) * 17 + k0 + tq + 4])};
-                    const uint32_t aA[4] = {to_tf32(dgA[gq * 17 + k0 + tq]), to_tf32(dgA[(gq + 8) * 17 + k0 + tq]),
-                                            to_tf32(dgA[gq * 17 + k0 + tq + 4]), to_tf32(dgA[(gq + 8) * 17 + k0 + tq + 4])};
-#pragma unroll
-                    for (int nt = 0; nt < 4; ++nt) {
-                        const int cc = 32 * Q + 8 * nt + gq;
-                        uint32_t bkd[2];
-#pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const int j = 16 * I + k0 + tq + 4 * e;
-                            const float kv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + RK + raw16(j, cc)));
-                            const float dv = *reinterpret_cast<const float *>(sm + RG + raw32(j, cc));
-                            bkd[e] = to_tf32(kv * __expf(-dv));
-                        }
-                        mma_tf32_16x8x8(c1[nt], aP, bkd);
-                        mma_tf32_16x8x8(c2[nt], aA, bkd);
-                    }
-                }
-                // scale by l = e^(G'_r - G'_m) and add
-#pragma unroll
-                for (int nt = 0; nt < 4; ++nt) {
-                    const int cc = 32 * Q + 8 * nt + 2 * tq;
-#pragma unroll
-                    for (int h2 = 0; h2 < 2; ++h2) {
-                        const float2 dv = *reinterpret_cast<const float2 *>(sm + RG + raw32(r0 + 8 * h2, cc));
-                        const float l0 = __expf(dv.x), l1 = __expf(dv.y);
-                        z1[nt][2 * h2] += l0 * c1[nt][2 * h2];
-                        z1[nt][2 * h2 + 1] += l1 * c1[nt][2 * h2 + 1];
-                        z2[nt][2 * h2] += l0 * c2[nt][2 * h2];
-                        z2[nt][2 * h2 + 1] += l1 * c2[nt][2 * h2 + 1];
-                    }
-                }
-            }
-            // ---------------- Z3: rows j of block I (as a column block), channels of quarter Q
-            float z3[4][4];
-            {
-                float c3[4][4] = {};
                 for (int I2 = I + 1; I2 < 4; ++I2) {
-                    uint32_t aP[4], aA[4], bq[8], bb2[8];
-                    // A = dP[r in I2][j in I]^T: stored rows 16 I2 + (l & 7) + 8 (l >> 4),
-                    // columns 16 I + 8 ((l >> 3) & 1)
+                    uint32_t aP[4], aA[4], bq[2], bb2[2];
                     const int sr = 16 * I2 + (lane & 7) + 8 * (lane >> 4), sc = 16 * I + 8 * ((lane >> 3) & 1);
                     ldsm_x4_t(aP, spd + sw128_off(sr, sc, 64));
                     ldsm_x4_t(aA, sad + sw128_off(sr, sc, 64));
                     const int br = 16 * I2 + (lane & 7) + 8 * ((lane >> 3) & 1);
-                    ldsm_x4_t(bq, smem_addr(sm + QA + raw16(br, 32 * Q + 8 * (lane >> 4))));
-                    ldsm_x4_t(bq + 4, smem_addr(sm + QA + raw16(br, 32 * Q + 16 + 8 * (lane >> 4))));
-                    ldsm_x4_t(bb2, smem_addr(sm + BA + raw16(br, 32 * Q + 8 * (lane >> 4))));
-                    ldsm_x4_t(bb2 + 4, smem_addr(sm + BA + raw16(br, 32 * Q + 16 + 8 * (lane >> 4))));
+                    ldsm_x2_t(bq, smem_addr(sm + QA + raw16(br, cb)));
+                    ldsm_x2_t(bb2, smem_addr(sm + BA + raw16(br, cb)));
                     if (I2 > I + 1) {
-#pragma unroll
-                        for (int nt = 0; nt < 4; ++nt) {
-                            const float chi = mchi[pair_ix(I2, I) * 128 + 32 * Q + 8 * nt + gq];
-#pragma unroll
-                            for (int e = 0; e < 2; ++e) {
-                                bq[2 * nt + e] = h2scale(bq[2 * nt + e], chi);
-                                bb2[2 * nt + e] = h2scale(bb2[2 * nt + e], chi);
-                            }
-                        }
+                        const float chi = mchi[pair_ix(I2, I) * 128 + cb + gq];
+                        bq[0] = h2scale(bq[0], chi);
+                        bq[1] = h2scale(bq[1], chi);
+                        bb2[0] = h2scale(bb2[0], chi);
+                        bb2[1] = h2scale(bb2[1], chi);
                     }
-#pragma unroll
-                    for (int nt = 0; nt < 4; ++nt) {
-                        mma_f16_16x8x16(c3[nt], aP, bq + 2 * nt);
-                        mma_f16_16x8x16(c3[nt], aA, bb2 + 2 * nt);
-                    }
+                    mma_f16_16x8x16(c3, aP, bq);
+                    mma_f16_16x8x16(c3, aA, bb2);
                 }
-                // scale by a_bar = e^(e_I - G_j)
-#pragma unroll
-                for (int nt = 0; nt < 4; ++nt) {
-                    const int cc = 32 * Q + 8 * nt + 2 * tq;
-#pragma unroll
-                    for (int h2 = 0; h2 < 2; ++h2) {
-                        const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(sm + AB + raw16(r0 + 8 * h2, cc)));
-                        z3[nt][2 * h2] = a.x * c3[nt][2 * h2];
-                        z3[nt][2 * h2 + 1] = a.y * c3[nt][2 * h2 + 1];
-                    }
-                }
-            }
-            {
-                // diagonal block, tf32: A = dP_II^T, dA_II^T; B = q l, b k l
-                float c3[4][4] = {};
+                // diagonal block in tf32: B operands k / l (Z1, Z2), q l and b k l (Z3)
+                // at rows 16 I + k0 + t (+4), channel cb + g
+                float d1[4] = {0.f, 0.f, 0.f, 0.f}, d2[4] = {0.f, 0.f, 0.f, 0.f}, d3[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int k0 = 0; k0 < 16; k0 += 8) {
-                    // a0 (j = g, r = t), a1 (g + 8, t), a2 (g, t + 4), a3 (g + 8, t + 4)
-                    const uint32_t aP[4] = {to_tf32(dgP[(k0 + tq) * 17 + gq]), to_tf32(dgP[(k0 + tq) * 17 + gq + 8]),
-                                            to_tf32(dgP[(k0 + tq + 4) * 17 + gq]), to_tf32(dgP[(k0 + tq + 4) * 17 + gq + 8])};
-                    const uint32_t aA[4] = {to_tf32(dgA[(k0 + tq) * 17 + gq]), to_tf32(dgA[(k0 + tq) * 17 + gq + 8]),
-                                            to_tf32(dgA[(k0 + tq + 4) * 17 + gq]), to_tf32(dgA[(k0 + tq + 4) * 17 + gq + 8])};
+                    uint32_t bkl[2], bql[2], bbl[2];
 #pragma unroll
-                    for (int nt = 0; nt < 4; ++nt) {
-                        const int cc = 32 * Q + 8 * nt + gq;
-                        uint32_t bqd[2], bbd[2];
-#pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const int r = 16 * I + k0 + tq + 4 * e;
-                            const float l = __expf(*reinterpret_cast<const float *>(sm + RG + raw32(r, cc)));
-                            const float qv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + RQ + raw16(r, cc)));
-                            const float kv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + RK + raw16(r, cc)));
-                            const float bv = *reinterpret_cast<const float *>(sm + RB + raw32(r, cc));
-                            bqd[e] = to_tf32(qv * l);
-                            bbd[e] = to_tf32(bv * kv * l);
-                        }
-                        mma_tf32_16x8x8(c3[nt], aP, bqd);
-                        mma_tf32_16x8x8(c3[nt], aA, bbd);
+                    for (int e = 0; e < 2; ++e) {
+                        const int j = 16 * I + k0 + tq + 4 * e, cc = cb + gq;
+                        const float dv = *reinterpret_cast<const float *>(sm + RG + raw32(j, cc));
+                        const float l = ex2(dv), il = ex2(-dv);
+                        const float kv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + RK + raw16(j, cc)));
+                        const float qv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + RQ + raw16(j, cc)));
+                        const float bv = *reinterpret_cast<const float *>(sm + RB + raw32(j, cc));
+                        bkl[e] = to_tf32(kv * il);
+                        bql[e] = to_tf32(qv * l);
+                        bbl[e] = to_tf32(bv * kv * l);
                     }
+                    // A = dP_II, dA_II: a0 (g, t), a1 (g + 8, t), a2 (g, t + 4), a3 (g + 8, t + 4)
+                    const uint32_t aP[4] = {dgP[gq * 17 + k0 + tq], dgP[(gq + 8) * 17 + k0 + tq],
+                                            dgP[gq * 17 + k0 + tq + 4], dgP[(gq + 8) * 17 + k0 + tq + 4]};
+                    const uint32_t aA[4] = {dgA[gq * 17 + k0 + tq], dgA[(gq + 8) * 17 + k0 + tq],
+                                            dgA[gq * 17 + k0 + tq + 4], dgA[(gq + 8) * 17 + k0 + tq + 4]};
+                    // their transposes (rows j, contraction over r)
+                    const uint32_t aPt[4] = {dgP[(k0 + tq) * 17 + gq], dgP[(k0 + tq) * 17 + gq + 8],
+                                             dgP[(k0 + tq + 4) * 17 + gq], dgP[(k0 + tq + 4) * 17 + gq + 8]};
+                    const uint32_t aAt[4] = {dgA[(k0 + tq) * 17 + gq], dgA[(k0 + tq) * 17 + gq + 8],
+                                             dgA[(k0 + tq + 4) * 17 + gq], dgA[(k0 + tq + 4) * 17 + gq + 8]};
+                    mma_tf32_16x8x8(d1, aP, bkl);
+                    mma_tf32_16x8x8(d2, aA, bkl);
+                    mma_tf32_16x8x8(d3, aPt, bql);
+                    mma_tf32_16x8x8(d3, aAt, bbl);
                 }
-#pragma unroll
-                for (int nt = 0; nt < 4; ++nt) {
-                    const int cc = 32 * Q + 8 * nt + 2 * tq;
-#pragma unroll
-                    for (int h2 = 0; h2 < 2; ++h2) {
-                        const float2 dv = *reinterpret_cast<const float2 *>(sm + RG + raw32(r0 + 8 * h2, cc));
-                        z3[nt][2 * h2] += __expf(-dv.x) * c3[nt][2 * h2];
-                        z3[nt][2 * h2 + 1] += __expf(-dv.y) * c3[nt][2 * h2 + 1];
-                    }
-                }
-            }
-            __syncwarp();  // every read of this warp's raw region is done
-            // ---------------- dq, dk, db, dG in place; the chunk-end sum over Kb Y3
-            float endk[4][2];
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt) {
+                // the outputs of rows r0, r0 + 8 and channels cb + 2 t, + 1
                 float y1[4], y2[4], y3[4];
-                tmem_ld16x256x1(taddr(tm + TM_Y1 + 32 * Q + 8 * nt, I * 32, 0), y1);
-                tmem_ld16x256x1(taddr(tm + TM_Y2 + 32 * Q + 8 * nt, I * 32, 0), y2);
-                tmem_ld16x256x1(taddr(tm + TM_Y3 + 32 * Q + 8 * nt, I * 32, 0), y3);
+                tmem_ld16x256x1(taddr(tm + TM_Y1 + cb, I * 32, 0), y1);
+                tmem_ld16x256x1(taddr(tm + TM_Y2 + cb, I * 32, 0), y2);
+                tmem_ld16x256x1(taddr(tm + TM_Y3 + cb, I * 32, 0), y3);
                 tmem_wait_ld();
-                const int cc = 32 * Q + 8 * nt + 2 * tq;
+                const int cc = cb + 2 * tq;
                 const float2 es = *reinterpret_cast<const float2 *>(mes + I * 128 + cc);
                 const float2 ef = *reinterpret_cast<const float2 *>(mef + I * 128 + cc);
-                endk[nt][0] = endk[nt][1] = 0.f;
+                const float esv[2] = {es.x, es.y}, efv[2] = {ef.x, ef.y};
+                float endk[2] = {0.f, 0.f};
+                __syncwarp();  // every read of this warp's raw region for these channels is done
 #pragma unroll
                 for (int h2 = 0; h2 < 2; ++h2) {
                     const int r = r0 + 8 * h2;
                     const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(sm + AL + raw16(r, cc)));
                     const float2 ab = __half22float2(*reinterpret_cast<const __half2 *>(sm + AB + raw16(r, cc)));
+                    const float2 dv = *reinterpret_cast<const float2 *>(sm + RG + raw32(r, cc));
                     const float2 qf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(sm + RQ + raw16(r, cc)));
                     const float2 kf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(sm + RK + raw16(r, cc)));
                     const float2 bf = *reinterpret_cast<const float2 *>(sm + RB + raw32(r, cc));
-                    const float av[2] = {a.x, a.y}, abv[2] = {ab.x, ab.y}, qv[2] = {qf.x, qf.y},
-                                kv[2] = {kf.x, kf.y}, bv[2] = {bf.x, bf.y}, esv[2] = {es.x, es.y},
-                                efv[2] = {ef.x, ef.y};
+                    const float av[2] = {a.x, a.y}, abv[2] = {ab.x, ab.y}, dvv[2] = {dv.x, dv.y},
+                                qv[2] = {qf.x, qf.y}, kv[2] = {kf.x, kf.y}, bv[2] = {bf.x, bf.y};
                     float dq[2], dk[2], db[2], dG[2];
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
                         const int x = 2 * h2 + e;
+                        const float l = ex2(dvv[e]), il = ex2(-dvv[e]);
+                        const float z1 = av[e] * c1[x] + l * d1[x];
+                        const float z2 = av[e] * c2[x] + l * d2[x];
+                        const float z3 = abv[e] * c3[x] + il * d3[x];
                         const float E = av[e] * esv[e], F = abv[e] * efv[e];
-                        dq[e] = fmaf(y1[x], E, z1[nt][x]);
-                        const float dkc = fmaf(y2[x], E, z2[nt][x]);
+                        dq[e] = fmaf(y1[x], E, z1);
+                        const float dkc = fmaf(y2[x], E, z2);
                         const float y3f = y3[x] * F;
-                        dk[e] = y3f + z3[nt][x] + dkc * bv[e];
+                        dk[e] = y3f + z3 + dkc * bv[e];
                         db[e] = dkc * kv[e];
                         dG[e] = qv[e] * dq[e] + 2.f * bv[e] * kv[e] * dkc - kv[e] * dk[e];
-                        endk[nt][e] = fmaf(kv[e], y3f, endk[nt][e]);
+                        endk[e] = fmaf(kv[e], y3f, endk[e]);
+                    }
+                    *reinterpret_cast<uint32_t *>(sm + RQ + raw16(r, cc)) = pack_bf16(dq[0], dq[1]);
+                    *reinterpret_cast<uint32_t *>(sm + RK + raw16(r, cc)) = pack_bf16(dk[0], dk[1]);
+                    *reinterpret_cast<float2 *>(sm + RB + raw32(r, cc)) = make_float2(db[0], db[1]);
+                    *reinterpret_cast<float2 *>(sm + RG + raw32(r, cc)) = make_float2(dG[0], dG[1]);
+                }
+                // sum the Kb Y3 parts over this warp's 16 rows (lanes with equal t % 4)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    float v = endk[e];
+                    v += __shfl_xor_sync(0xffffffffu, v, 4);
+                    v += __shfl_xor_sync(0xffffffffu, v, 8);
+                    v += __shfl_xor_sync(0xffffffffu, v, 16);
+                    if (gq == 0) mendk[I * 128 + cc + e] = v;
+                }
+                __syncwarp();
+            }
+        } else {
+            // ---------------- mild: dq = Y1 E, dKc = Y2 E, dk = Y3 / E + dKc b
+            const int r0 = 16 * I + gq;
+#pragma unroll 1
+            for (int nt = 0; nt < 4; ++nt) {
+                const int cb = 32 * Q + 8 * nt, cc = cb + 2 * tq;
+                float y1[4], y2[4], y3[4];
+                tmem_ld16x256x1(taddr(tm + TM_Y1 + cb, I * 32, 0), y1);
+                tmem_ld16x256x1(taddr(tm + TM_Y2 + cb, I * 32, 0), y2);
+                tmem_ld16x256x1(taddr(tm + TM_Y3 + cb, I * 32, 0), y3);
+                tmem_wait_ld();
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const int r = r0 + 8 * h2;
+                    const float2 E2 = __half22float2(*reinterpret_cast<const __half2 *>(sm + MEM + raw16(r, cc)));
+                    const float2 Ei2 = __half22float2(*reinterpret_cast<const __half2 *>(sm + MEI + raw16(r, cc)));
+                    const float2 qf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(sm + RQ + raw16(r, cc)));
+                    const float2 kf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(sm + RK + raw16(r, cc)));
+                    const float2 bf = *reinterpret_cast<const float2 *>(sm + RB + raw32(r, cc));
+                    const float Ev[2] = {E2.x, E2.y}, Eiv[2] = {Ei2.x, Ei2.y}, qv[2] = {qf.x, qf.y},
+                                kv[2] = {kf.x, kf.y}, bv[2] = {bf.x, bf.y};
+                    float dq[2], dk[2], db[2], dG[2];
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int x = 2 * h2 + e;
+                        dq[e] = y1[x] * Ev[e];
+                        const float dkc = y2[x] * Ev[e];
+                        dk[e] = y3[x] * Eiv[e] + dkc * bv[e];
+                        db[e] = dkc * kv[e];
+                        dG[e] = qv[e] * dq[e] + 2.f * bv[e] * kv[e] * dkc - kv[e] * dk[e];
                     }
                     *reinterpret_cast<uint32_t *>(sm + RQ + raw16(r, cc)) = pack_bf16(dq[0], dq[1]);
                     *reinterpret_cast<uint32_t *>(sm + RK + raw16(r, cc)) = pack_bf16(dk[0], dk[1]);
@@ -909,17 +983,6 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
                     *reinterpret_cast<float2 *>(sm + RG + raw32(r, cc)) = make_float2(dG[0], dG[1]);
                 }
             }
-            // sum the Kb Y3 parts over this warp's 16 rows (lanes with equal t % 4)
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    float v = endk[nt][e];
-                    v += __shfl_xor_sync(0xffffffffu, v, 4);
-                    v += __shfl_xor_sync(0xffffffffu, v, 8);
-                    v += __shfl_xor_sync(0xffffffffu, v, 16);
-                    if (gq == 0) mendk[I * 128 + 32 * Q + 8 * nt + 2 * tq + e] = v;
-                }
         }
         fence_proxy_async();
         fence_before_sync();
@@ -948,7 +1011,8 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
             }
             mtot[I * 128 + fc2] = run;
             named_sync(1, kCompute);
-            float after = mgam[fc2] * (mend1[fc2] + mend1[128 + fc2] + mend1[256 + fc2] + mend1[384 + fc2]) +
+            // rowsum(dS' . S_c) carries gamma already in the mild frame (S_m dX)
+            float after = (mild ? 1.f : mgam[fc2]) * (mend1[fc2] + mend1[128 + fc2] + mend1[256 + fc2] + mend1[384 + fc2]) +
                           mendk[fc2] + mendk[128 + fc2] + mendk[256 + fc2] + mendk[384 + fc2];
 #pragma unroll
             for (int J = 0; J < 4; ++J)
@@ -977,6 +1041,7 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
         if (issued[2] > 0) mbar_wait(&bars[3], (issued[2] - 1) & 1, kWait);
         mbar_wait(&bars[1], 0, kWait);
         mbar_wait(&bars[1], 1, kWait);
+        if (nmild > 0) mbar_wait(&bars[2], (nmild - 1) & 1, kWait);
     }
     fence_before_sync();
     __syncthreads();

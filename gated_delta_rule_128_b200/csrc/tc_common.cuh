@@ -33,6 +33,36 @@ using namespace tc;
 
 // per-token floor of the log-decay inside the same-block pair factors
 constexpr float kClampG = 9.0f;
+// the kernels carry cumulative decays in log2 units (g log2 e), so that every
+// factor is one ex2
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kClampG2 = kClampG * kLog2e;
+// A tile is mild when every channel's cumulative log-decay stays within
+// kMildG of its value at row 31 and |q|, |k|, |b k| <= kMildX: then every
+// factor e^(+-(G - G_31)) x stays within kMildX e^kMildG (1.4e4, inside fp16)
+// and no factor that matters falls below fp16's normal range, so one frame
+// serves the whole chunk.  Other tiles take the block frames.
+constexpr float kMildG = 4.0f;
+constexpr float kMildG2 = kMildG * kLog2e;
+constexpr float kMildX = 256.0f;
+
+// 2^x (the special-function unit's ex2; flushes denormal results to zero)
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float4 f4scale(float4 a, float s) { return make_float4(a.x * s, a.y * s, a.z * s, a.w * s); }
+// 4 bf16 values of an 8-byte chunk, widened
+__device__ __forceinline__ void ld_bf4(const unsigned char *p, float *x) {
+    const uint2 v = *reinterpret_cast<const uint2 *>(p);
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&v.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&v.y));
+    x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
+}
+__device__ __forceinline__ void st_h4v(unsigned char *p, const float *x) {
+    *reinterpret_cast<uint2 *>(p) = make_uint2(pack_f16(x[0], x[1]), pack_f16(x[2], x[3]));
+}
 
 __device__ __forceinline__ void st_h4(unsigned char *p, float a, float b, float c, float d) {
     uint2 v = make_uint2(pack_f16(a, b), pack_f16(c, d));
@@ -112,6 +142,12 @@ __device__ __forceinline__ void ldsm_x4(uint32_t *r, uint32_t saddr) {
 __device__ __forceinline__ void ldsm_x4_t(uint32_t *r, uint32_t saddr) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(saddr));
+}
+// two 8x8 b16 matrices, transposed (rows addressed by lanes 0..15)
+__device__ __forceinline__ void ldsm_x2_t(uint32_t *r, uint32_t saddr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];"
+                 : "=r"(r[0]), "=r"(r[1])
                  : "r"(saddr));
 }
 // (x.lo s, x.hi s) for an f16 pair x, multiplied in float32 and rounded once

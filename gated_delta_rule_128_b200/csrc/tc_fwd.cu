@@ -4,11 +4,12 @@
 //
 // "Gated DeltaNet-2" (LIT-802 review, Key takeaways 2; paper Secs. 3.3-3.4,
 // Apps. A-B): only the state crosses chunk borders.  Per chunk of 64 tokens
-// entering with state S (chunk-start frame, tc_common.cuh; U = w.v):
-//   Delta = T U - W S
-//   O = Qb S + P Delta,   S_next = diag(gamma) S + Kb^T Delta
-// Every record factor is at most 1 in magnitude for any g <= 0, so the state
-// stays at its true scale and no factor can overflow.
+// entering with state S (the chunk's frame, with frame factor s, see REC_* in
+// common.cuh; U = w.v):
+//   Delta = T U - W (s S)
+//   O = Qb (s S) + P Delta,   S_next = diag(gamma) S + r Kx^T Delta
+// The state stays at its true scale in registers; only the operand s S
+// changes frame from chunk to chunk.
 //
 // One CTA owns one (b, h) and one 64-column half of d_v and walks the
 // sequence's chunks in order with its fp32 state slice in registers (each
@@ -19,9 +20,9 @@
 // Both state-side products are M = 128 tcgen05.mma groups into one
 // [Delta; O] accumulator (rows 0..63 Delta, 64..127 O; two such accumulators
 // alternate between chunks):
-//   (1) [T; 0] U + [-W; Qb] S              -> Delta and Qb S
-//   (2) [0; P] Delta,  and  X = Kb^T Delta (a fresh accumulator)
-// then S_next = gamma S + X in registers.  Warp roles: warps 0, 1, 4, 5 (TMEM
+//   (1) [T; 0] U + [-W; Qb] (s S)          -> Delta and Qb (s S)
+//   (2) [0; P] Delta,  and  X = Kx^T Delta (a fresh accumulator)
+// then S_next = gamma S + r X in registers.  Warp roles: warps 0, 1, 4, 5 (TMEM
 // lanes 0..63) read Delta; warps 2, 3, 6, 7 (lanes 64..127) read the previous
 // chunk's O and form the next chunk's U = w.v off the state's path; all warps
 // update the state.
@@ -32,7 +33,8 @@
 // GDN2_ERR_RANGE.
 //
 // For the backward the call can also leave in the workspace (TcWs): every
-// chunk's entry state S_c (fp16, a copy of the operand) and Delta per chunk.
+// chunk's entry state in its frame, s S_c (fp16, a copy of the operand), and
+// Delta per chunk.
 
 #include "common.cuh"
 #include "tc.cuh"
@@ -194,10 +196,16 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mv, const __grid_constant__ CU
                           : make_float4(0.f, 0.f, 0.f, 0.f);
             sreg[j] = t.x; sreg[j + 1] = t.y; sreg[j + 2] = t.z; sreg[j + 3] = t.w;
         }
+        // the operand state s S in chunk 0's frame
+        const float s0 = reinterpret_cast<const float *>(sm + STG + S_FAC)[128 + key];
+        const float se = s0 < 0.f ? 1.f : s0;
+        float x[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) x[j] = se * sreg[j];
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
-            st_h8(sm + OP_S + sw128_chunk(key, 4 * half + jj, 128), sreg + 8 * jj);
-            big = absmax8(sreg + 8 * jj, big);
+            st_h8(sm + OP_S + sw128_chunk(key, 4 * half + jj, 128), x + 8 * jj);
+            big = absmax8(x + 8 * jj, big);
         }
     }
     if (!dwarp) {
@@ -272,8 +280,15 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mv, const __grid_constant__ CU
         // ---------------- S_next = gamma S + Kb^T Delta
         ok = mbar_wait(&bars[4], par, kWait) && ok;
         const float gam = reinterpret_cast<const float *>(stg + S_FAC)[key];  // e^G_63
+        const float sc = reinterpret_cast<const float *>(stg + S_FAC)[128 + key];
+        const float rr = sc < 0.f ? 1.f : gam / sc;  // Kx^T Delta's scale in S_next
         // the next chunk's record has landed before its first products are issued
-        if (c + 1 < NC) ok = mbar_wait(&bars[s ^ 1], ((c + 1) >> 1) & 1, kWait) && ok;
+        float sn = 1.f;  // the next chunk's frame factor
+        if (c + 1 < NC) {
+            ok = mbar_wait(&bars[s ^ 1], ((c + 1) >> 1) & 1, kWait) && ok;
+            const float sv = reinterpret_cast<const float *>(sm + STG + (s ^ 1) * STAGE + S_FAC)[128 + key];
+            sn = sv < 0.f ? 1.f : sv;
+        }
         fence_after_sync();
         {
             float xv[32];
@@ -281,12 +296,14 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mv, const __grid_constant__ CU
             tmem_ld16(taddr(tm + TM_S, quarter * 32, 32 * half + 16), xv + 16);
             tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) sreg[j] = fmaf(gam, sreg[j], xv[j]);
+            for (int j = 0; j < 32; ++j) sreg[j] = fmaf(gam, sreg[j], rr * xv[j]);
             if (c + 1 < NC) {
 #pragma unroll
+                for (int j = 0; j < 32; ++j) xv[j] = sn * sreg[j];  // the operand state s S
+#pragma unroll
                 for (int jj = 0; jj < 4; ++jj) {
-                    st_h8(sm + OP_S + sw128_chunk(key, 4 * half + jj, 128), sreg + 8 * jj);
-                    big = absmax8(sreg + 8 * jj, big);
+                    st_h8(sm + OP_S + sw128_chunk(key, 4 * half + jj, 128), xv + 8 * jj);
+                    big = absmax8(xv + 8 * jj, big);
                 }
             } else if (ST) {
                 float *dst = ST + st_off(d, bb, h) + (size_t)key * 128 + v0 + 32 * half;

@@ -11,9 +11,14 @@
 //   P[r][j] = sum_c q_r,c k_j,c e^(G_r,c - G_j,c)     (j <= r)
 //   T = (I + A)^-1,  W = T Kc,  Kc = b.k.e^G,  Qb = q.e^G,  Kb = k.e^(G_63 - G)
 // The chunk's record (layout REC_* in common.cuh) receives [-W; Qb], Kb, T,
-// P and gamma = e^G_63; the sequential state kernels read it.
+// P, gamma = e^G_63 and a frame factor s; the sequential state kernels read it.
 //
-// A and P come in two parts, so that no factor overflows for any g <= 0:
+// A mild tile (tc_common.cuh: every channel's G within e^4 of its row 31)
+// takes one frame for the whole chunk: Kc, Qb, Kb above are taken times
+// e^-G_31 (Kb times e^G_31 / e^G_63, i.e. Kh = k e^(G_31 - G)), s = e^G_31,
+// and A and P come from one fp16 product [Kc; Qb] Kh^T.  Any other tile keeps
+// the chunk-start frame (s = 1, stored as -1 to mark it) and takes A and P in
+// two parts, so that no factor overflows for any g <= 0:
 //  * blocks of rows I > J (16 rows each): one fp16 tcgen05.mma per row block
 //    I', M = 128 rows [b.k.a; q.a] (a = e^(G - s_I), <= 1) against
 //    R_I'[j] = k_j e^(s_I' - G_j) for j < 16 I' (<= 1), K = 128 channels;
@@ -47,7 +52,7 @@ constexpr uint32_t REC = RR + 24576;  // the tile's record, laid out as in the w
 constexpr uint32_t OP_WQ = REC + REC_WQ;  // [Kc; Qb], later [-W; Qb]
 constexpr uint32_t OP_KB = REC + REC_KH;
 constexpr uint32_t OP_T = REC + REC_T, OP_P = REC + REC_P, FAC = REC + REC_FAC;
-constexpr uint32_t TOT = OP_T;        // block totals of G [4][128] f32, before T is written
+constexpr uint32_t TOT = OP_T;        // 8-row totals of G [2][8][128] f32, before T and P are written
 // float32 scratch of the inversion, over CO / RR once the products have read them
 constexpr uint32_t SCR_A = CO, SCR_T = CO + 64 * 65 * 4, SCR_M = SCR_T + 64 * 65 * 4;
 constexpr uint32_t MISC = REC + REC_BYTES;  // mbarriers, TMEM slot
@@ -55,6 +60,7 @@ constexpr uint32_t SMEM_BYTES = MISC + 128 + 1024;
 constexpr uint32_t TM_C = 0, TM_W = 128;  // the three block products (96 columns); W
 __host__ __device__ constexpr uint32_t tm_coff(int I) { return I <= 1 ? 0u : (I == 2 ? 16u : 48u); }
 constexpr uint32_t ID_KM128 = idesc_f16(64, 128, false, true);
+constexpr uint32_t ID_KK128x64 = idesc_f16(128, 64, false, false);
 constexpr long long kWait = 2000000000LL;  // ~1 s of SM clocks per wait
 constexpr float kRange = 6.0e4f;
 static_assert(MISC % 8 == 0 && REC % 1024 == 0 && RR % 1024 == 0, "alignment");
@@ -150,7 +156,8 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
         (reinterpret_cast<uintptr_t>(smraw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + MISC);  // 0 raw tiles, 1 mma
     uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + MISC + 64);
-    float *tot = reinterpret_cast<float *>(sm + TOT);
+    float *tot = reinterpret_cast<float *>(sm + TOT);         // [8 row groups][128]
+    float *totc = reinterpret_cast<float *>(sm + TOT + 4096);  // the same, clamped
     float big = 0.f;  // range check: largest fp16 operand magnitude
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -188,8 +195,8 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
     };
     if (tid == 0 && (int)blockIdx.x < ntiles) load_raw(blockIdx.x);
 
-    // factor phase ownership: 16 rows of block fb, channels fc, fc + 1
-    const int fb = tid >> 6, fc = 2 * (tid & 63);
+    // factor phase ownership: warp = 8 rows (block fb, half fh), lane = 4 channels from fc4
+    const int fb = warp >> 1, fh = warp & 1, fc4 = 4 * lane;
 
     bool abort = false;
     int n = 0;  // tiles done by this CTA
@@ -199,83 +206,188 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
         if (tid == 0) bulk_wait_read();  // the previous tile's record has left shared memory
         if (__syncthreads_or(!ok)) { abort = true; break; }
 
-        // ---------------- cumulative decay of this block's 16 rows, exact and clamped
-        float gl[16][2], gc[16][2];
+        // ---------------- cumulative decay (log2 units) of this warp's 8 rows,
+        // exact and clamped; lane fq owns channels 4 fq .. 4 fq + 3
+        float gl[8][4], gc[8][4];
         {
-            float run[2] = {0.f, 0.f}, runc[2] = {0.f, 0.f};
+            float run[4] = {0.f, 0.f, 0.f, 0.f}, runc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                const float2 g2 = *reinterpret_cast<const float2 *>(sm + RAW_G + raw32(16 * fb + r, fc));
-                run[0] += g2.x;
-                run[1] += g2.y;
-                runc[0] += fmaxf(g2.x, -kClampG);
-                runc[1] += fmaxf(g2.y, -kClampG);
-                gl[r][0] = run[0];
-                gl[r][1] = run[1];
-                gc[r][0] = runc[0];
-                gc[r][1] = runc[1];
+            for (int i = 0; i < 8; ++i) {
+                const float4 g4 = *reinterpret_cast<const float4 *>(sm + RAW_G + raw32(8 * warp + i, fc4));
+                const float gv[4] = {g4.x * kLog2e, g4.y * kLog2e, g4.z * kLog2e, g4.w * kLog2e};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    run[e] += gv[e];
+                    runc[e] += fmaxf(gv[e], -kClampG2);
+                    gl[i][e] = run[e];
+                    gc[i][e] = runc[e];
+                }
             }
-            *reinterpret_cast<float2 *>(tot + fb * 128 + fc) = make_float2(run[0], run[1]);
+            *reinterpret_cast<float4 *>(tot + warp * 128 + fc4) = make_float4(run[0], run[1], run[2], run[3]);
+            *reinterpret_cast<float4 *>(totc + warp * 128 + fc4) = make_float4(runc[0], runc[1], runc[2], runc[3]);
         }
         __syncthreads();
+        // ---------------- mild tile?  Then the whole chunk fits one frame
+        // relative to its row 31: every factor e^(+-(G - G_31)) stays within
+        // e^kMildG, and one fp16 product gives A and P (tc_common.cuh).
+        bool mild;
+        {
+            float pre[4] = {0.f, 0.f, 0.f, 0.f}, g31[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int r8 = 0; r8 < 8; ++r8) {
+                const float4 t4 = *reinterpret_cast<const float4 *>(tot + r8 * 128 + fc4);
+                const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    if (r8 < warp) pre[e] += tv[e];
+                    if (r8 < 4) g31[e] += tv[e];
+                }
+            }
+            float dmax = 0.f, xmax = 0.f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                float qv[4], kv[4];
+                ld_bf4(sm + RAW_Q + raw16(8 * warp + i, fc4), qv);
+                ld_bf4(sm + RAW_K + raw16(8 * warp + i, fc4), kv);
+                const float4 b4 = *reinterpret_cast<const float4 *>(sm + RAW_B + raw32(8 * warp + i, fc4));
+                const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    dmax = fmaxf(dmax, fabsf(pre[e] + gl[i][e] - g31[e]));
+                    xmax = fmaxf(xmax, fmaxf(fabsf(qv[e]), fmaxf(fabsf(kv[e]), fabsf(bv[e] * kv[e]))));
+                }
+            }
+            mild = !__syncthreads_or(!(dmax <= kMildG2 && xmax <= kMildX));
+            if (mild) {
+                // ---------------- mild: the record takes the single frame of row 31
+                // (E = e^(G - G_31)): Kc = b k E, Qb = q E, Kh = k / E, and the frame
+                // factor s = e^G_31; A and P are [Kc; Qb] Kh^T
+                float all[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int r8 = 0; r8 < 8; ++r8) {
+                    const float4 t4 = *reinterpret_cast<const float4 *>(tot + r8 * 128 + fc4);
+                    all[0] += t4.x; all[1] += t4.y; all[2] += t4.z; all[3] += t4.w;
+                }
+                if (warp == 0) {
+                    *reinterpret_cast<float4 *>(sm + FAC + 4 * fc4) =
+                        make_float4(ex2(all[0]), ex2(all[1]), ex2(all[2]), ex2(all[3]));  // gamma
+                    *reinterpret_cast<float4 *>(sm + FAC + 512 + 4 * fc4) =
+                        make_float4(ex2(g31[0]), ex2(g31[1]), ex2(g31[2]), ex2(g31[3]));  // s
+                }
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int t = 8 * warp + i;
+                    float qv[4], kv[4];
+                    ld_bf4(sm + RAW_Q + raw16(t, fc4), qv);
+                    ld_bf4(sm + RAW_K + raw16(t, fc4), kv);
+                    const float4 b4 = *reinterpret_cast<const float4 *>(sm + RAW_B + raw32(t, fc4));
+                    const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
+                    float kcm[4], qbm[4], khm[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float dl = pre[e] + gl[i][e] - g31[e];
+                        const float E = ex2(dl), Ei = ex2(-dl);
+                        kcm[e] = bv[e] * kv[e] * E;
+                        qbm[e] = qv[e] * E;
+                        khm[e] = kv[e] * Ei;
+                    }
+                    st_h4v(sm + OP_WQ + sw128_off(t, fc4, 128), kcm);
+                    st_h4v(sm + OP_WQ + sw128_off(64 + t, fc4, 128), qbm);
+                    st_h4v(sm + OP_KB + sw128_off(t, fc4, 64), khm);
+                }
+                fence_proxy_async();
+                fence_before_sync();
+                __syncthreads();
+                if (tid == 0) {
+                    fence_after_sync();
+                    const uint64_t co = desc_kmajor(smem_addr(sm + OP_WQ), 128, 0),
+                                   kh = desc_kmajor(smem_addr(sm + OP_KB), 64, 0);
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks)
+                        mma_bf16(tm + TM_C, kstep_kmajor(co, 128, ks), kstep_kmajor(kh, 64, ks), ID_KK128x64, ks > 0);
+                    mma_commit(&bars[1]);
+                }
+            }
+        }
+        float cA[4] = {0.f, 0.f, 0.f, 0.f}, cP[4] = {0.f, 0.f, 0.f, 0.f};
+        const int db = warp >> 1, dn = warp & 1, gq = lane >> 2, tq = lane & 3;
+        if (!mild) {
         // ---------------- factors: record operands, block-product operands, d
         {
-            float T4[4][2];
+            // per channel: the four block totals; s (before this block), the
+            // block's first-half and whole totals, G_63; chi_{I', fb}
+            float btot[4][4], h0[4], h0c[4], sg[4], bt[4], all[4];
 #pragma unroll
-            for (int I = 0; I < 4; ++I) {
-                const float2 t2 = *reinterpret_cast<const float2 *>(tot + I * 128 + fc);
-                T4[I][0] = t2.x;
-                T4[I][1] = t2.y;
+            for (int J = 0; J < 4; ++J) {
+                const float4 a4 = *reinterpret_cast<const float4 *>(tot + (2 * J) * 128 + fc4);
+                const float4 b4 = *reinterpret_cast<const float4 *>(tot + (2 * J + 1) * 128 + fc4);
+                btot[J][0] = a4.x + b4.x; btot[J][1] = a4.y + b4.y; btot[J][2] = a4.z + b4.z; btot[J][3] = a4.w + b4.w;
+                if (J == fb) { h0[0] = a4.x; h0[1] = a4.y; h0[2] = a4.z; h0[3] = a4.w; }
             }
-            float eS[2], eF[2], chi[4][2];  // e^s_I, e^(G_63 - e_I), chi_{I', fb}
+            {
+                const float4 c4 = *reinterpret_cast<const float4 *>(totc + 2 * fb * 128 + fc4);
+                h0c[0] = c4.x; h0c[1] = c4.y; h0c[2] = c4.z; h0c[3] = c4.w;
+            }
+            float eS[4], eF[4], chi[4][4];
 #pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                float s = 0.f, all = 0.f;
+            for (int e = 0; e < 4; ++e) {
+                sg[e] = 0.f;
+                all[e] = 0.f;
+#pragma unroll
+                for (int J = 0; J < 4; ++J) {
+                    if (J < fb) sg[e] += btot[J][e];
+                    if (J == fb) bt[e] = btot[J][e];
+                    all[e] += btot[J][e];
+                }
+                eS[e] = ex2(sg[e]);
+                eF[e] = ex2(all[e] - sg[e] - bt[e]);
+                float between = 0.f;  // block totals strictly between fb and I
 #pragma unroll
                 for (int I = 0; I < 4; ++I) {
-                    if (I < fb) s += T4[I][i];
-                    all += T4[I][i];
+                    chi[I][e] = ex2(between);
+                    if (I > fb) between += btot[I][e];
                 }
-                eS[i] = __expf(s);
-                eF[i] = __expf(all - s - T4[fb][i]);
-                float between = 0.f;  // sum of the block totals strictly between fb and I'
-#pragma unroll
-                for (int I = 0; I < 4; ++I) {
-                    chi[I][i] = I == fb + 1 ? 1.f : __expf(between);
-                    if (I > fb) between += T4[I][i];
-                }
-                if (fb == 0) reinterpret_cast<float *>(sm + FAC)[fc + i] = __expf(all);  // gamma
+            }
+            if (warp == 0) {
+                *reinterpret_cast<float4 *>(sm + FAC + 4 * fc4) =
+                    make_float4(ex2(all[0]), ex2(all[1]), ex2(all[2]), ex2(all[3]));  // gamma
+                // the chunk-start frame: frame factor 1, marked by a negative s
+                *reinterpret_cast<float4 *>(sm + FAC + 512 + 4 * fc4) = make_float4(-1.f, -1.f, -1.f, -1.f);
             }
 #pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                const int t = 16 * fb + r;
-                const float2 q2 = ld_bf2(sm + RAW_Q + raw16(t, fc)), k2 = ld_bf2(sm + RAW_K + raw16(t, fc));
-                const float2 b2 = *reinterpret_cast<const float2 *>(sm + RAW_B + raw32(t, fc));
-                const float qv[2] = {q2.x, q2.y}, kv[2] = {k2.x, k2.y}, bv[2] = {b2.x, b2.y};
-                float bka[2], qa[2], kc[2], qb[2], kb[2], ka[2], dd[2];
+            for (int i = 0; i < 8; ++i) {
+                const int t = 8 * warp + i;
+                float qv[4], kv[4];
+                ld_bf4(sm + RAW_Q + raw16(t, fc4), qv);
+                ld_bf4(sm + RAW_K + raw16(t, fc4), kv);
+                const float4 b4 = *reinterpret_cast<const float4 *>(sm + RAW_B + raw32(t, fc4));
+                const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
+                float bka[4], qa[4], kc[4], qb[4], kb[4], ka[4], dd[4];
 #pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    const float a = __expf(gl[r][i]), ab = __expf(T4[fb][i] - gl[r][i]);
-                    bka[i] = bv[i] * kv[i] * a;
-                    qa[i] = qv[i] * a;
-                    kc[i] = bka[i] * eS[i];
-                    qb[i] = qa[i] * eS[i];
-                    kb[i] = kv[i] * ab * eF[i];
-                    ka[i] = kv[i] * ab;
-                    dd[i] = gc[r][i] - gc[7][i];
-                    big = fmaxf(big, fmaxf(fabsf(bka[i]), fmaxf(fabsf(qa[i]), fabsf(ka[i]))));
+                for (int e = 0; e < 4; ++e) {
+                    const float loc = fh ? h0[e] + gl[i][e] : gl[i][e];  // G_t - s_I
+                    const float a = ex2(loc), ab = ex2(bt[e] - loc);
+                    bka[e] = bv[e] * kv[e] * a;
+                    qa[e] = qv[e] * a;
+                    kc[e] = bka[e] * eS[e];
+                    qb[e] = qa[e] * eS[e];
+                    ka[e] = kv[e] * ab;
+                    kb[e] = ka[e] * eF[e];
+                    dd[e] = fh ? gc[i][e] : gc[i][e] - h0c[e];  // G'_t - G'_m, m = the block's row 7
+                    big = fmaxf(big, fmaxf(fabsf(bka[e]), fmaxf(fabsf(qa[e]), fabsf(ka[e]))));
                 }
-                *reinterpret_cast<uint32_t *>(sm + CO + sw128_off(t, fc, 128)) = pack_f16(bka[0], bka[1]);
-                *reinterpret_cast<uint32_t *>(sm + CO + sw128_off(64 + t, fc, 128)) = pack_f16(qa[0], qa[1]);
-                *reinterpret_cast<uint32_t *>(sm + OP_WQ + sw128_off(t, fc, 128)) = pack_f16(kc[0], kc[1]);
-                *reinterpret_cast<uint32_t *>(sm + OP_WQ + sw128_off(64 + t, fc, 128)) = pack_f16(qb[0], qb[1]);
-                *reinterpret_cast<uint32_t *>(sm + OP_KB + sw128_off(t, fc, 64)) = pack_f16(kb[0], kb[1]);
+                st_h4v(sm + CO + sw128_off(t, fc4, 128), bka);
+                st_h4v(sm + CO + sw128_off(64 + t, fc4, 128), qa);
+                st_h4v(sm + OP_WQ + sw128_off(t, fc4, 128), kc);
+                st_h4v(sm + OP_WQ + sw128_off(64 + t, fc4, 128), qb);
+                st_h4v(sm + OP_KB + sw128_off(t, fc4, 64), kb);
 #pragma unroll
                 for (int I = 1; I < 4; ++I)
-                    if (I > fb)
-                        *reinterpret_cast<uint32_t *>(sm + RR + rr_off(I) + sw128_off(t, fc, 16 * I)) =
-                            pack_f16(ka[0] * chi[I][0], ka[1] * chi[I][1]);
-                *reinterpret_cast<float2 *>(sm + RAW_G + raw32(t, fc)) = make_float2(dd[0], dd[1]);
+                    if (I > fb) {
+                        const float kx[4] = {ka[0] * chi[I][0], ka[1] * chi[I][1], ka[2] * chi[I][2], ka[3] * chi[I][3]};
+                        st_h4v(sm + RR + rr_off(I) + sw128_off(t, fc4, 16 * I), kx);
+                    }
+                *reinterpret_cast<float4 *>(sm + RAW_G + raw32(t, fc4)) = make_float4(dd[0], dd[1], dd[2], dd[3]);
             }
         }
         fence_proxy_async();
@@ -295,33 +407,50 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
             }
             mma_commit(&bars[1]);
         }
-        // ---------------- diagonal blocks: warp (block db, 8 columns dn) in tf32
-        const int db = warp >> 1, dn = warp & 1, gq = lane >> 2, tq = lane & 3;
-        float cA[4] = {0.f, 0.f, 0.f, 0.f}, cP[4] = {0.f, 0.f, 0.f, 0.f};
+        // ---------------- diagonal blocks: warp (block db, 8 columns dn) in tf32.
+        // The contraction runs over channels in the order that lets a lane
+        // load 4 consecutive channels at once: k-step 2p takes channels
+        // 16p + 4t, 16p + 4t + 1 as k = t, t + 4; k-step 2p + 1 takes
+        // 16p + 4t + 2, + 3.
         {
             const int r0 = 16 * db + gq, r1 = r0 + 8, jj = 16 * db + 8 * dn + gq;
-#pragma unroll 4
-            for (int k0 = 0; k0 < 128; k0 += 8) {
-                uint32_t aA[4], aP[4], bb[2];
+#pragma unroll 2
+            for (int p = 0; p < 8; ++p) {
+                const int c = 16 * p + 4 * tq;
+                uint32_t aA[2][4], aP[2][4], bb[4];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int r = (e & 1) ? r1 : r0, c = k0 + tq + ((e & 2) ? 4 : 0);
-                    const float l = __expf(*reinterpret_cast<const float *>(sm + RAW_G + raw32(r, c)));
-                    const float kv = ld_bf(sm + RAW_K + raw16(r, c)), qv = ld_bf(sm + RAW_Q + raw16(r, c));
-                    const float bv = *reinterpret_cast<const float *>(sm + RAW_B + raw32(r, c));
-                    aA[e] = to_tf32(bv * kv * l);
-                    aP[e] = to_tf32(qv * l);
-                }
+                for (int h = 0; h < 2; ++h) {  // rows r0, r1
+                    const int r = h ? r1 : r0;
+                    const float4 d4 = *reinterpret_cast<const float4 *>(sm + RAW_G + raw32(r, c));
+                    const float4 b4 = *reinterpret_cast<const float4 *>(sm + RAW_B + raw32(r, c));
+                    float qv[4], kv[4];
+                    ld_bf4(sm + RAW_Q + raw16(r, c), qv);
+                    ld_bf4(sm + RAW_K + raw16(r, c), kv);
+                    const float lv[4] = {ex2(d4.x), ex2(d4.y), ex2(d4.z), ex2(d4.w)};
+                    const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
 #pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int c = k0 + tq + 4 * e;
-                    const float il = __expf(-*reinterpret_cast<const float *>(sm + RAW_G + raw32(jj, c)));
-                    bb[e] = to_tf32(ld_bf(sm + RAW_K + raw16(jj, c)) * il);
+                    for (int e = 0; e < 4; ++e) {
+                        // channel c + e: k-step 2p + (e >> 1), k index t (+4 when e odd)
+                        aA[e >> 1][h + 2 * (e & 1)] = to_tf32(bv[e] * kv[e] * lv[e]);
+                        aP[e >> 1][h + 2 * (e & 1)] = to_tf32(qv[e] * lv[e]);
+                    }
                 }
-                mma_tf32_16x8x8(cA, aA, bb);
-                mma_tf32_16x8x8(cP, aP, bb);
+                {
+                    const float4 d4 = *reinterpret_cast<const float4 *>(sm + RAW_G + raw32(jj, c));
+                    float kv[4];
+                    ld_bf4(sm + RAW_K + raw16(jj, c), kv);
+                    bb[0] = to_tf32(kv[0] * ex2(-d4.x));
+                    bb[1] = to_tf32(kv[1] * ex2(-d4.y));
+                    bb[2] = to_tf32(kv[2] * ex2(-d4.z));
+                    bb[3] = to_tf32(kv[3] * ex2(-d4.w));
+                }
+                mma_tf32_16x8x8(cA, aA[0], bb);
+                mma_tf32_16x8x8(cP, aP[0], bb);
+                mma_tf32_16x8x8(cA, aA[1], bb + 2);
+                mma_tf32_16x8x8(cP, aP[1], bb + 2);
             }
         }
+        }  // !mild
         // ---------------- assemble A (float32, for the inversion) and P (record)
         ok = mbar_wait(&bars[1], 0, kWait);
         fence_after_sync();
@@ -329,7 +458,29 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
         if (tid == 0 && it + (int)gridDim.x < ntiles) load_raw(it + gridDim.x);
         float *sA = reinterpret_cast<float *>(sm + SCR_A);
         float *sT = reinterpret_cast<float *>(sm + SCR_T);
-        {
+        if (mild) {
+            // accumulator row quarter * 32 + lane: rows 0..63 are A, 64..127 are P;
+            // this warp's 32 columns start at 32 * (warp >> 2)
+            const int half = warp >> 2;
+            float row[32];
+            tmem_ld16(taddr(tm + TM_C, quarter * 32, 32 * half), row);
+            tmem_ld16(taddr(tm + TM_C, quarter * 32, 32 * half + 16), row + 16);
+            tmem_wait_ld();
+            if (quarter < 2) {
+                const int r = quarter * 32 + lane;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) sA[r * 65 + 32 * half + j] = 32 * half + j < r ? row[j] : 0.f;
+            } else {
+                const int r = quarter * 32 + lane - 64;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) row[j] = 32 * half + j <= r ? row[j] : 0.f;
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    st_h8(sm + OP_P + sw128_chunk(r, 4 * half + jj, 64), row + 8 * jj);
+                    big = absmax8(row + 8 * jj, big);
+                }
+            }
+        } else {
             // diagonal blocks from the warps' fragments: rows 16 db + gq (+ 8),
             // columns 16 db + 8 dn + 2 tq (+ 1)
 #pragma unroll

@@ -400,10 +400,16 @@ def _steep(kind, seed):
         g = torch.nn.functional.logsigmoid(torch.randn(x["g"].shape, generator=gen)) / 16
         g[..., ::3] = -30.0
         x["g"] = g
+    elif kind == "steep_then_mild":  # chunks 0, 1 steep, chunks 2, 3 mild: both tile paths in one call
+        g = torch.nn.functional.logsigmoid(torch.randn(x["g"].shape, generator=gen)) / 16
+        g[:, :128] = torch.nn.functional.logsigmoid(torch.randn(x["g"][:, :128].shape, generator=gen)) * 4
+        x["g"] = g
+    elif kind == "edge_-0.13":      # |G - G_31| reaches about 4.2: just past the single-frame bound
+        x["g"] = torch.full_like(x["g"], -0.13)
     return x
 
 
-@pytest.mark.parametrize("kind", ["logsigmoid_x4", "const_-2", "mixed_-30"])
+@pytest.mark.parametrize("kind", ["logsigmoid_x4", "const_-2", "mixed_-30", "steep_then_mild", "edge_-0.13"])
 def test_tensor_core_path_steep_decay(kind):
     """Any g <= 0 on the tensor-core path: the chunk-start frame keeps every
     state-side factor <= 1, and the in-chunk pair factors come from block
