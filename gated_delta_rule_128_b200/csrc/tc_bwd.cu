@@ -408,8 +408,10 @@ constexpr uint32_t QA = 114688;   // q e^(G - s_I)
 constexpr uint32_t BA = 131072;   // b k e^(G - s_I)
 constexpr uint32_t AL = 147456;   // e^(G - s_I)
 constexpr uint32_t AB = 163840;   // e^(e_I - G)
-// mild tiles: q E, b k E, k / E, E, 1 / E in the same five slots (E = e^(G - G_31))
-constexpr uint32_t MQB = KA, MKC = QA, MKH = BA, MEM = AL, MEI = AB;
+// mild tiles (E = e^(G - G_31)): q E in place of q; b k E, k / E, E, 1 / E over
+// Delta, S_c and the spare space, so that [dO; -dU] is free once the first
+// products have read it
+constexpr uint32_t MQB = RQ, MKC = DL, MKH = SMT, MEM = SMT + 16384, MEI = 196608;
 constexpr uint32_t PD = 180224;   // masked dP [64][64] fp16 (sw128, R = 64)
 constexpr uint32_t AD = 188416;   // masked dA
 constexpr uint32_t DG32 = 196608; // diagonal blocks of dP, dA as tf32 bits [2][4][16][17]
@@ -579,6 +581,24 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
             }
             st_h8(p, x);
         }
+        fence_proxy_async();
+        fence_before_sync();
+        __syncthreads();  // dO converted
+        if (issuer) {
+            fence_after_sync();
+            const uint64_t dn = desc_kmajor(smem_addr(sm + DN), 128, 0), dl = desc_kmajor(smem_addr(sm + DL), 64, 0),
+                           s = desc_kmajor(smem_addr(sm + SMT), 128, 0), dx = desc_kmajor(smem_addr(sm + DXT), 128, 0),
+                           ado = desc_kmajor(smem_addr(sm + DN), 64, 0), andu = desc_kmajor(smem_addr(sm + DN + 8192), 64, 0);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint64_t b_s = kstep_kmajor(s, 128, ks), a_dl = kstep_kmajor(dl, 64, ks);
+                mma_bf16(tm + TM_PA, kstep_kmajor(dn, 128, ks), a_dl, ID_PA, ks > 0);
+                mma_bf16(tm + TM_Y1, kstep_kmajor_blk(ado, 16384, ks), b_s, ID_KK128, ks > 0);
+                mma_bf16(tm + TM_Y2, kstep_kmajor_blk(andu, 16384, ks), b_s, ID_KK128, ks > 0);
+                mma_bf16(tm + TM_Y3, a_dl, kstep_kmajor(dx, 128, ks), ID_KK128, ks > 0);
+            }
+            mma_commit(&bars[1]);
+        }
         // ---------------- cumulative decay (log2 units): warp w = rows 8 (w & 7)
         // .. + 7 (block fb, half fh), channels fc, fc + 1 with fc = 64 (w >> 3) + 2 lane
         const int frg = warp & 7, fb = frg >> 1, fh = frg & 1, fc = 64 * ((warp >> 3) & 1) + 2 * lane;
@@ -633,24 +653,6 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
         // dS' in the workspace as e^G_31 S_c and e^(G_63 - G_31) dS') or the
         // chunk-start frame (a negative frame factor)
         const bool mild = reinterpret_cast<const float *>(sm + MISC + M_FLAG)[0] > 0.f;
-        fence_proxy_async();
-        fence_before_sync();
-        __syncthreads();  // dO converted
-        if (issuer) {
-            fence_after_sync();
-            const uint64_t dn = desc_kmajor(smem_addr(sm + DN), 128, 0), dl = desc_kmajor(smem_addr(sm + DL), 64, 0),
-                           s = desc_kmajor(smem_addr(sm + SMT), 128, 0), dx = desc_kmajor(smem_addr(sm + DXT), 128, 0),
-                           ado = desc_kmajor(smem_addr(sm + DN), 64, 0), andu = desc_kmajor(smem_addr(sm + DN + 8192), 64, 0);
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint64_t b_s = kstep_kmajor(s, 128, ks), a_dl = kstep_kmajor(dl, 64, ks);
-                mma_bf16(tm + TM_PA, kstep_kmajor(dn, 128, ks), a_dl, ID_PA, ks > 0);
-                mma_bf16(tm + TM_Y1, kstep_kmajor_blk(ado, 16384, ks), b_s, ID_KK128, ks > 0);
-                mma_bf16(tm + TM_Y2, kstep_kmajor_blk(andu, 16384, ks), b_s, ID_KK128, ks > 0);
-                mma_bf16(tm + TM_Y3, a_dl, kstep_kmajor(dx, 128, ks), ID_KK128, ks > 0);
-            }
-            mma_commit(&bars[1]);
-        }
         // ---------------- factors, held until the products have read S_c and dS':
         // mild: q E, b k E, k / E, E, 1 / E (E = e^(G - G_31));
         // else: k a_bar, q a, b k a, a, a_bar, and d = G' - G'_m in place of g
@@ -728,6 +730,7 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
             mend1[ev * 128 + ec] = acc;
         }
         named_sync(1, kCompute);  // S_c, dS', Delta, [dO; -dU] are consumed
+        if (issuer && mild && more) load_a1(nxt);  // the mild tiles leave [dO; -dU] free
         if (!mild && fh == 0) {
             *reinterpret_cast<float2 *>(mes + fb * 128 + fc) = make_float2(ex2(sg[0]), ex2(sg[1]));
             *reinterpret_cast<float2 *>(mef + fb * 128 + fc) =
@@ -755,11 +758,23 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
             }
         }
         // ---------------- the factors as fp16 tiles
+        if (mild) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const uint32_t off = raw16(8 * frg + i, fc);
+            for (int i = 0; i < 8; ++i) {
+                const uint32_t off = raw16(8 * frg + i, fc);
+                *reinterpret_cast<uint32_t *>(sm + MQB + off) = pk[i][0];
+                *reinterpret_cast<uint32_t *>(sm + MKC + off) = pk[i][1];
+                *reinterpret_cast<uint32_t *>(sm + MKH + off) = pk[i][2];
+                *reinterpret_cast<uint32_t *>(sm + MEM + off) = pk[i][3];
+                *reinterpret_cast<uint32_t *>(sm + MEI + off) = pk[i][4];
+            }
+        } else {
 #pragma unroll
-            for (int x = 0; x < 5; ++x) *reinterpret_cast<uint32_t *>(sm + KA + x * 16384 + off) = pk[i][x];
+            for (int i = 0; i < 8; ++i) {
+                const uint32_t off = raw16(8 * frg + i, fc);
+#pragma unroll
+                for (int x = 0; x < 5; ++x) *reinterpret_cast<uint32_t *>(sm + KA + x * 16384 + off) = pk[i][x];
+            }
         }
         fence_proxy_async();
         fence_before_sync();
@@ -962,11 +977,14 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
                     const int r = r0 + 8 * h2;
                     const float2 E2 = __half22float2(*reinterpret_cast<const __half2 *>(sm + MEM + raw16(r, cc)));
                     const float2 Ei2 = __half22float2(*reinterpret_cast<const __half2 *>(sm + MEI + raw16(r, cc)));
-                    const float2 qf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(sm + RQ + raw16(r, cc)));
+                    const float2 qe = __half22float2(*reinterpret_cast<const __half2 *>(sm + MQB + raw16(r, cc)));
+                    const float2 kc = __half22float2(*reinterpret_cast<const __half2 *>(sm + MKC + raw16(r, cc)));
+                    const float2 kh = __half22float2(*reinterpret_cast<const __half2 *>(sm + MKH + raw16(r, cc)));
                     const float2 kf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(sm + RK + raw16(r, cc)));
                     const float2 bf = *reinterpret_cast<const float2 *>(sm + RB + raw32(r, cc));
-                    const float Ev[2] = {E2.x, E2.y}, Eiv[2] = {Ei2.x, Ei2.y}, qv[2] = {qf.x, qf.y},
-                                kv[2] = {kf.x, kf.y}, bv[2] = {bf.x, bf.y};
+                    const float Ev[2] = {E2.x, E2.y}, Eiv[2] = {Ei2.x, Ei2.y}, qev[2] = {qe.x, qe.y},
+                                kcv[2] = {kc.x, kc.y}, khv[2] = {kh.x, kh.y}, kv[2] = {kf.x, kf.y},
+                                bv[2] = {bf.x, bf.y};
                     float dq[2], dk[2], db[2], dG[2];
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
@@ -975,7 +993,8 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
                         const float dkc = y2[x] * Ev[e];
                         dk[e] = y3[x] * Eiv[e] + dkc * bv[e];
                         db[e] = dkc * kv[e];
-                        dG[e] = qv[e] * dq[e] + 2.f * bv[e] * kv[e] * dkc - kv[e] * dk[e];
+                        // q dq + 2 b k dKc - k dk, with the factors E carries
+                        dG[e] = y1[x] * qev[e] + y2[x] * kcv[e] - y3[x] * khv[e];
                     }
                     *reinterpret_cast<uint32_t *>(sm + RQ + raw16(r, cc)) = pack_bf16(dq[0], dq[1]);
                     *reinterpret_cast<uint32_t *>(sm + RK + raw16(r, cc)) = pack_bf16(dk[0], dk[1]);
@@ -990,7 +1009,7 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
         if (issuer) {
             fence_after_sync();
             if (more) {  // the next tile's operands into the space the pair terms used
-                load_a1(nxt);
+                if (!mild) load_a1(nxt);
                 load_a2(nxt);
             }
             for (int x = 0; x < 2; ++x) {
