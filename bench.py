@@ -34,22 +34,29 @@ sys.path.insert(0, ROOT)
 WORKLOAD_INDEX = 2
 METRIC = "GDR-2 fwd+bwd tokens/s (H16, dk=dv=128) and % of HBM/tensor roofline"
 NAMES = ("q", "k", "v", "g", "b", "w", "S0")
-# algorithmic bytes per token-head (bf16 q,k,v,o,dO,dq,dk,dv; f32 g,b,w,dg,db,dw)
-FWD_BYTES = 3 * 128 * 2 + 3 * 128 * 4 + 128 * 2           # 2560
-BWD_BYTES = 3 * 128 * 2 + 3 * 128 * 4 + 128 * 2 + 3 * 128 * 2 + 3 * 128 * 4   # 4864
-# ... attributed to the kernel that first reads (or writes) each tensor
-KERNEL_BYTES = {
-    # q, k, g, b read
-    "tc_prep": 2 * 128 * 2 + 2 * 128 * 4,
-    # v, w read; o written
-    "tc_fwd": 128 * 2 + 128 * 4 + 128 * 2,
-    # q, k, g, b, dO, v, w read; dv, dw written
-    "tc_bwd_state": 2 * 128 * 2 + 2 * 128 * 4 + 128 * 2 + 128 * 2 + 128 * 4 + 128 * 2 + 128 * 4,
-    # dq, dk, db, dg written
-    "tc_bwd_grad": 2 * 128 * 2 + 2 * 128 * 4,
-}
-assert KERNEL_BYTES["tc_prep"] + KERNEL_BYTES["tc_fwd"] == FWD_BYTES
-assert KERNEL_BYTES["tc_bwd_state"] + KERNEL_BYTES["tc_bwd_grad"] == BWD_BYTES
+def byte_model(gs: int = 4):
+    """Algorithmic bytes per token-head at d = 128: bf16 q, k, v, o, dO, dq, dk,
+    dv and gates g, b, w, dg, db, dw of gs bytes (4 float32, 2 bf16).  Returns
+    (forward, backward, per-kernel), the per-kernel figures attributing each
+    tensor to the kernel that first reads (or writes) it."""
+    fwd = 3 * 128 * 2 + 3 * 128 * gs + 128 * 2
+    bwd = 3 * 128 * 2 + 3 * 128 * gs + 128 * 2 + 3 * 128 * 2 + 3 * 128 * gs
+    kern = {
+        # q, k, g, b read
+        "tc_prep": 2 * 128 * 2 + 2 * 128 * gs,
+        # v, w read; o written
+        "tc_fwd": 128 * 2 + 128 * gs + 128 * 2,
+        # q, k, g, b, dO, v, w read; dv, dw written
+        "tc_bwd_state": 2 * 128 * 2 + 2 * 128 * gs + 128 * 2 + 128 * 2 + 128 * gs + 128 * 2 + 128 * gs,
+        # dq, dk, db, dg written
+        "tc_bwd_grad": 2 * 128 * 2 + 2 * 128 * gs,
+    }
+    assert kern["tc_prep"] + kern["tc_fwd"] == fwd and kern["tc_bwd_state"] + kern["tc_bwd_grad"] == bwd
+    return fwd, bwd, kern
+
+
+# float32 gates: 2560 + 4864 = 7424; bf16 gates: 1792 + 3328 = 5120
+FWD_BYTES, BWD_BYTES, KERNEL_BYTES = byte_model(4)
 
 
 def parse():
@@ -152,16 +159,18 @@ def traffic_from_profiles(kernel_key: str, src_hash: str):
     return rec.get("dram_bytes_per_launch")
 
 
-# the files that make up the tensor-core kernels whose DRAM traffic
-# profiles/traffic.json records; the captured figures apply while these match
-TC_KERNEL_SOURCES = ("tc_prep.cu", "tc_fwd.cu", "tc_bwd.cu", "common.cuh", "tc.cuh", "tc_common.cuh",
-                     "tmap.cuh")
+# the files that make up each tensor-core kernel whose DRAM traffic
+# profiles/traffic.json records; a kernel's captured figure applies while these
+# match (the shared headers count for every kernel)
+TC_SHARED_SOURCES = ("common.cuh", "tc.cuh", "tc_common.cuh", "tmap.cuh")
+TC_KERNEL_SOURCES = {"tc_prep": ("tc_prep.cu",), "tc_fwd": ("tc_fwd.cu",),
+                     "tc_bwd_state": ("tc_bwd.cu",), "tc_bwd_grad": ("tc_bwd_grad.cu",)}
 
 
-def sources_hash() -> str:
+def sources_hash(kernel_key: str) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gated_delta_rule_128_b200", "csrc")
-    for n in TC_KERNEL_SOURCES:
+    for n in TC_KERNEL_SOURCES[kernel_key] + TC_SHARED_SOURCES:
         h.update(open(os.path.join(csrc, n), "rb").read())
     return h.hexdigest()
 
@@ -172,7 +181,7 @@ def _peak():
     return peaks.get("hbm_gbs", 6650.0), ("of measured" if "hbm_gbs" in peaks else "of fallback")
 
 
-def kernel_split(gdn, run_steps, steps, token_heads, peak, stream):
+def kernel_split(gdn, run_steps, steps, token_heads, peak, stream, kernel_bytes=None):
     """Per-kernel device time from the library's event timer, taken in a pass
     of its own (the timer records two events around every launch, so it is
     never on while a headline number is timed)."""
@@ -188,7 +197,7 @@ def kernel_split(gdn, run_steps, steps, token_heads, peak, stream):
     for name, (cnt, tot) in ktimes.items():
         avg = tot / cnt
         ent = {"launches": cnt, "avg_ms": avg}
-        per = KERNEL_BYTES.get(name)
+        per = (kernel_bytes or KERNEL_BYTES).get(name)
         if per is not None:
             gbs = per * token_heads / (avg * 1e-3) / 1e9
             ent.update(alg_bytes_per_launch=per * token_heads, achieved_gbs=gbs, frac=gbs / peak)
@@ -198,9 +207,9 @@ def kernel_split(gdn, run_steps, steps, token_heads, peak, stream):
 
 class FwdBwdCase:
     """Device buffers and the fwd+bwd step of one workload shape (bf16 I/O,
-    float32 gates and state), inputs resident in HBM."""
+    float32 or bf16 gates, float32 state), inputs resident in HBM."""
 
-    def __init__(self, wl, B, seed, dev, with_bwd=True):
+    def __init__(self, wl, B, seed, dev, with_bwd=True, gates="f32"):
         import torch
 
         import gated_delta_rule_128_b200 as gdn
@@ -213,7 +222,11 @@ class FwdBwdCase:
                            erase_scale=wl.erase_scale, with_dO=with_bwd)
         bf = torch.bfloat16
         io_names = ("q", "k", "v", "dO")
-        self.host = {n: (t.to(bf) if n in io_names else t).contiguous() for n, t in x.items()}
+        gate_t = bf if gates == "bf16" else torch.float32
+        self.host = {n: (t.to(bf) if n in io_names else t.to(gate_t) if n in ("g", "b", "w") else t)
+                     .contiguous() for n, t in x.items()}
+        self.gate_io = gdn.GDN2_IO_BF16 if gates == "bf16" else gdn.GDN2_IO_F32
+        self.fwd_bytes, self.bwd_bytes, self.kernel_bytes = byte_model(2 if gates == "bf16" else 4)
         self.d = {n: t.to(dev) for n, t in self.host.items()}
         self.io = gdn.GDN2_IO_BF16
         self.ws = gdn.workspace(B, wl.T, wl.H, wl.dk, wl.dv, wl.chunk, self.io, with_bwd, dev)
@@ -232,15 +245,15 @@ class FwdBwdCase:
     def fwd(self, inp=None, out=None):
         inp, out = inp or self.d, out or dict(o=self.o, **self.grads)
         g = self.gdn
-        g.gdn2_fwd(*(inp[n] for n in NAMES), out["o"], self.ST, self.ws, self.ws.numel(), self.B,
-                   self.T, self.H, self.dk, self.dv, self.C, self.io, self.stream)
+        g.gdn2_fwd_ex(*(inp[n] for n in NAMES), out["o"], self.ST, self.ws, self.ws.numel(), self.B,
+                      self.T, self.H, self.dk, self.dv, self.C, self.io, self.gate_io, self.stream)
 
     def bwd(self, inp=None, out=None):
         inp, out = inp or self.d, out or dict(o=self.o, **self.grads)
-        self.gdn.gdn2_bwd(*(inp[n] for n in NAMES), inp["dO"], None, out["dq"], out["dk"],
-                          out["dv"], out["dg"], out["db"], out["dw"], None, self.ws,
-                          self.ws.numel(), 1, self.B, self.T, self.H, self.dk, self.dv, self.C,
-                          self.io, self.stream)
+        self.gdn.gdn2_bwd_ex(*(inp[n] for n in NAMES), inp["dO"], None, out["dq"], out["dk"],
+                             out["dv"], out["dg"], out["db"], out["dw"], None, self.ws,
+                             self.ws.numel(), 1, self.B, self.T, self.H, self.dk, self.dv, self.C,
+                             self.io, self.gate_io, self.stream)
 
     def step(self, inp=None, out=None):
         self.fwd(inp, out)
@@ -287,26 +300,29 @@ class FwdBwdCase:
         return start.elapsed_time(end) / steps, fwd_ms, bwd_ms, launches
 
 
-def sub_workload(index, args, rank, dev, peak, peak_src):
+def sub_workload(index, args, rank, dev, peak, peak_src, gates="f32"):
     """A secondary workload of the default line (1: forward only B8 T2048;
-    3: fwd+bwd B1 T16384 with b in [0, 2]), device-timed like the headline."""
+    3: fwd+bwd B1 T16384 with b in [0, 2]; 2 with bf16 gates), device-timed
+    like the headline."""
     import torch
 
     from gated_delta_rule_128_b200 import dist as gd
     from gated_delta_rule_128_b200 import workloads
 
     wl = workloads.WORKLOADS[index]
-    case = FwdBwdCase(wl, wl.B, gd.rank_seed(wl.seed, rank), dev, with_bwd=wl.backward)
+    case = FwdBwdCase(wl, wl.B, gd.rank_seed(wl.seed, rank), dev, with_bwd=wl.backward, gates=gates)
     steps = max(5, args.steps // 2)
     ms, fwd_ms, bwd_ms, _ = case.timed(steps, args.warmup, gd.barrier)
-    kernels = kernel_split(case.gdn, case.run, steps, case.token_heads, peak, case.stream)
+    kernels = kernel_split(case.gdn, case.run, steps, case.token_heads, peak, case.stream,
+                           case.kernel_bytes)
     ms = gd.max_over_ranks([ms], dev)[0]
     if wl.backward:
-        alg = case.token_heads * (FWD_BYTES + BWD_BYTES)
+        alg = case.token_heads * (case.fwd_bytes + case.bwd_bytes)
     else:  # the forward's bytes per token-head plus S0 read and S_T written
-        alg = case.token_heads * FWD_BYTES + 2 * wl.B * wl.H * wl.dk * wl.dv * 4
+        alg = case.token_heads * case.fwd_bytes + 2 * wl.B * wl.H * wl.dk * wl.dv * 4
     gbs = alg / (ms * 1e-3) / 1e9
-    out = {"workload": wl.name, "ms_per_step": ms, "steps": steps,
+    name = wl.name + (" bf16 gates" if gates == "bf16" else "")
+    out = {"workload": name, "ms_per_step": ms, "steps": steps,
            "tokens_per_s": wl.B * wl.T / (ms * 1e-3),
            "roofline_step": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
                              "frac": gbs / peak, "alg_bytes_per_step": alg,
@@ -401,20 +417,23 @@ def run_ours(args, rank, world, local_rank):
     decode = run_decode(args, rank, dev) if not args.no_decode else None
     subs = {} if (args.no_sub or WORKLOAD_INDEX != 2) else {
         f"workload{i}": sub_workload(i, args, rank, dev, peak, peak_src) for i in (1, 3)}
+    if subs:
+        subs["workload2_bf16_gates"] = sub_workload(2, args, rank, dev, peak, peak_src, gates="bf16")
     ms_step, e2e_ms, fwd_ms, bwd_ms = gd.max_over_ranks([ms_step, e2e_ms, fwd_ms, bwd_ms], dev)
     if decode is not None:
         decode["us_per_step"] = gd.max_over_ranks([decode["us_per_step"]], dev)[0]
     tokens = B * T * world
     value = tokens / (ms_step * 1e-3)
     alg_bytes = token_heads * (FWD_BYTES + BWD_BYTES)
-    src = sources_hash()
+    for n, kd in kernels.items():
+        kd["traffic"] = (traffic_from_profiles(n, sources_hash(n)) if n in TC_KERNEL_SOURCES else None)
     dom = max(kernels, key=lambda n: kernels[n]["launches"] * kernels[n]["avg_ms"])
     dk_ = kernels[dom]
     roofline = {"bound": "hbm", "kernel": dom, "achieved": dk_.get("achieved_gbs"), "peak": peak,
                 "unit": "GB/s", "frac": dk_.get("frac"), "peak_source": peak_src,
                 "alg_bytes_per_launch": dk_.get("alg_bytes_per_launch"),
                 "avg_launch_ms": dk_["avg_ms"],
-                "traffic": traffic_from_profiles(dom, src)}
+                "traffic": dk_["traffic"]}
     step_achieved = alg_bytes / (ms_step * 1e-3) / 1e9
     roofline_step = {"bound": "hbm", "achieved": step_achieved, "peak": peak, "unit": "GB/s",
                      "frac": step_achieved / peak, "alg_bytes_per_step": alg_bytes,

@@ -7,7 +7,8 @@ gated_delta_rule_128_b200.build``).
 
 Two layers:
 
-* ``gdn2_fwd``, ``gdn2_bwd``, ``gdn2_decode_step``, ``gdn2_workspace_bytes``,
+* ``gdn2_fwd``, ``gdn2_bwd``, ``gdn2_decode_step`` (and their ``_ex`` forms with
+  the gates' own type), ``gdn2_workspace_bytes``,
   ``gdn2_get_device_status``: the C entry points of ``include/gdn2.h`` under
   the same names, taking torch tensors (or None) where the C call takes
   pointers, and raising ``Gdn2Error`` on a non-zero status.
@@ -61,6 +62,12 @@ def lib() -> ctypes.CDLL:
         L.gdn2_bwd.argtypes = [vp] * 17 + [sz, i] + [i] * 7 + [vp]
         L.gdn2_bwd.restype = i
         L.gdn2_decode_step.argtypes = [vp] * 8 + [i] * 5 + [vp]
+        L.gdn2_fwd_ex.argtypes = [vp] * 10 + [sz] + [i] * 8 + [vp]
+        L.gdn2_fwd_ex.restype = i
+        L.gdn2_bwd_ex.argtypes = [vp] * 17 + [sz, i] + [i] * 8 + [vp]
+        L.gdn2_bwd_ex.restype = i
+        L.gdn2_decode_step_ex.argtypes = [vp] * 8 + [i] * 6 + [vp]
+        L.gdn2_decode_step_ex.restype = i
         L.gdn2_decode_step.restype = i
         L.gdn2_get_device_status.argtypes = [vp]
         L.gdn2_get_device_status.restype = i
@@ -102,6 +109,16 @@ def _io_of(t: torch.Tensor) -> int:
     raise TypeError(f"q/k/v must be float32 or bfloat16, got {t.dtype}")
 
 
+def _gate_io_of(g: torch.Tensor, b: torch.Tensor, w: torch.Tensor) -> int:
+    if not (g.dtype == b.dtype == w.dtype):
+        raise TypeError(f"g, b, w must share one dtype, got {g.dtype}, {b.dtype}, {w.dtype}")
+    if g.dtype == torch.bfloat16:
+        return GDN2_IO_BF16
+    if g.dtype == torch.float32:
+        return GDN2_IO_F32
+    raise TypeError(f"g/b/w must be float32 or bfloat16, got {g.dtype}")
+
+
 def _stream(stream=None):
     s = torch.cuda.current_stream() if stream is None else stream
     return ctypes.c_void_p(s.cuda_stream)
@@ -139,6 +156,29 @@ def gdn2_bwd(q, k, v, g, b, w, S0, dO, dST, dq, dk, dv, dg, db, dw, dS0, ws, ws_
                         _ptr(dS0), _ptr(ws), ws_bytes, int(ws_has_fwd), B, T, H, d_k, d_v, chunk,
                         io, _stream(stream))
     _check("gdn2_bwd", rc)
+
+
+def gdn2_fwd_ex(q, k, v, g, b, w, S0, o, ST, ws, ws_bytes, B, T, H, d_k, d_v, chunk, io,
+                gate_io, stream=None):
+    rc = lib().gdn2_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b), _ptr(w), _ptr(S0), _ptr(o),
+                           _ptr(ST), _ptr(ws), ws_bytes, B, T, H, d_k, d_v, chunk, io, gate_io,
+                           _stream(stream))
+    _check("gdn2_fwd_ex", rc)
+
+
+def gdn2_bwd_ex(q, k, v, g, b, w, S0, dO, dST, dq, dk, dv, dg, db, dw, dS0, ws, ws_bytes,
+                ws_has_fwd, B, T, H, d_k, d_v, chunk, io, gate_io, stream=None):
+    rc = lib().gdn2_bwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b), _ptr(w), _ptr(S0), _ptr(dO),
+                           _ptr(dST), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg), _ptr(db), _ptr(dw),
+                           _ptr(dS0), _ptr(ws), ws_bytes, int(ws_has_fwd), B, T, H, d_k, d_v, chunk,
+                           io, gate_io, _stream(stream))
+    _check("gdn2_bwd_ex", rc)
+
+
+def gdn2_decode_step_ex(q, k, v, g, b, w, S, o, N, H, d_k, d_v, io, gate_io, stream=None):
+    rc = lib().gdn2_decode_step_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b), _ptr(w), _ptr(S),
+                                   _ptr(o), N, H, d_k, d_v, io, gate_io, _stream(stream))
+    _check("gdn2_decode_step_ex", rc)
 
 
 def gdn2_decode_step(q, k, v, g, b, w, S, o, N, H, d_k, d_v, io, stream=None):
@@ -196,6 +236,7 @@ def forward(q, k, v, g, b, w, S0=None, *, chunk: int = 64, want_state: bool = Tr
             ws: Optional[torch.Tensor] = None, for_bwd: bool = False, stream=None,
             check: bool = True):
     """Returns (o, S_T or None, ws).  Shapes: q, k, g, b [B,T,H,dk]; v, w [B,T,H,dv].
+    g, b, w may be bfloat16 (all three) on the tensor-core path.
 
     check=True (the default) waits for the stream and raises Gdn2Error if a
     kernel recorded an error during the call; check=False leaves the call
@@ -207,7 +248,8 @@ def forward(q, k, v, g, b, w, S0=None, *, chunk: int = 64, want_state: bool = Tr
         ws = workspace(B, T, H, dk, dv, chunk, io, for_bwd, q.device)
     o = torch.empty(B, T, H, dv, dtype=q.dtype, device=q.device)
     ST = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device) if want_state else None
-    gdn2_fwd(q, k, v, g, b, w, S0, o, ST, ws, ws.numel(), B, T, H, dk, dv, chunk, io, stream)
+    gdn2_fwd_ex(q, k, v, g, b, w, S0, o, ST, ws, ws.numel(), B, T, H, dk, dv, chunk, io,
+                _gate_io_of(g, b, w), stream)
     if check:
         check_device_status(stream)
     return o, ST, ws
@@ -216,8 +258,8 @@ def forward(q, k, v, g, b, w, S0=None, *, chunk: int = 64, want_state: bool = Tr
 def backward(q, k, v, g, b, w, S0, dO, dST=None, *, chunk: int = 64,
              ws: Optional[torch.Tensor] = None, ws_has_fwd: bool = False,
              want_dS0: bool = True, stream=None, check: bool = True) -> Dict[str, torch.Tensor]:
-    """Gradients dq, dk, dv, dg, db, dw, dS0 (None unless want_dS0).  check as
-    in forward()."""
+    """Gradients dq, dk, dv, dg, db, dw, dS0 (None unless want_dS0); dg, db, dw
+    take the gates' dtype.  check as in forward()."""
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     io = _io_of(q)
@@ -228,8 +270,9 @@ def backward(q, k, v, g, b, w, S0, dO, dST=None, *, chunk: int = 64,
                dg=torch.empty_like(g), db=torch.empty_like(b), dw=torch.empty_like(w))
     out["dS0"] = (torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device)
                   if want_dS0 else None)
-    gdn2_bwd(q, k, v, g, b, w, S0, dO, dST, out["dq"], out["dk"], out["dv"], out["dg"], out["db"],
-             out["dw"], out["dS0"], ws, ws.numel(), ws_has_fwd, B, T, H, dk, dv, chunk, io, stream)
+    gdn2_bwd_ex(q, k, v, g, b, w, S0, dO, dST, out["dq"], out["dk"], out["dv"], out["dg"],
+                out["db"], out["dw"], out["dS0"], ws, ws.numel(), ws_has_fwd, B, T, H, dk, dv, chunk,
+                io, _gate_io_of(g, b, w), stream)
     if check:
         check_device_status(stream)
     return out
@@ -242,5 +285,6 @@ def decode_step(q, k, v, g, b, w, S, o=None, stream=None):
     dv = v.shape[-1]
     if o is None:
         o = torch.empty(N, H, dv, dtype=q.dtype, device=q.device)
-    gdn2_decode_step(q, k, v, g, b, w, S, o, N, H, dk, dv, _io_of(q), stream)
+    gdn2_decode_step_ex(q, k, v, g, b, w, S, o, N, H, dk, dv, _io_of(q), _gate_io_of(g, b, w),
+                        stream)
     return o

@@ -25,15 +25,15 @@ template <typename E>
 cudaError_t simt_bwd_launch(const void *, const void *, const void *, const float *, const float *,
                             const void *, const float *, void *, void *, void *, float *, float *,
                             float *, float *, void *, const Dims &, cudaStream_t);
-cudaError_t decode_launch(const void *, const void *, const void *, const float *, const float *,
-                          const float *, float *, void *, int, int, int, int, gdn2_io,
+cudaError_t decode_launch(const void *, const void *, const void *, const void *, const void *,
+                          const void *, float *, void *, int, int, int, int, gdn2_io, gdn2_io,
                           cudaStream_t);
-cudaError_t tc_fwd_launch(const void *, const void *, const void *, const float *, const float *,
-                          const float *, const float *, void *, float *, void *, int,
+cudaError_t tc_fwd_launch(const void *, const void *, const void *, const void *, const void *,
+                          const void *, const float *, void *, float *, void *, int,
                           unsigned int *, const Dims &, cudaStream_t);
-cudaError_t tc_bwd_launch(const void *, const void *, const void *, const float *, const float *,
-                          const float *, const void *, const float *, void *, void *, void *,
-                          float *, float *, float *, float *, void *, unsigned int *, const Dims &,
+cudaError_t tc_bwd_launch(const void *, const void *, const void *, const void *, const void *,
+                          const void *, const void *, const float *, void *, void *, void *,
+                          void *, void *, void *, float *, void *, unsigned int *, const Dims &,
                           cudaStream_t);
 
 // The device status word (GDN2_OK or the first error a kernel recorded), and
@@ -115,7 +115,7 @@ static gdn2_status check_dims(int B, int T, int H, int dk, int dv, int chunk, gd
 }
 
 static Dims make_dims(int B, int T, int H, int dk, int dv, int chunk) {
-    return Dims{B, T, H, dk, dv, chunk, (T + chunk - 1) / chunk};
+    return Dims{B, T, H, dk, dv, chunk, (T + chunk - 1) / chunk, 0};
 }
 
 // every required pointer non-null and 16-byte aligned; optional ones aligned
@@ -168,16 +168,25 @@ size_t gdn2_workspace_bytes(int B, int T, int H, int d_k, int d_v, int chunk, gd
     return ws_bytes_for(make_dims(B, T, H, d_k, d_v, chunk), io, for_bwd);
 }
 
-gdn2_status gdn2_fwd(const void *q, const void *k, const void *v, const float *g, const float *b,
-                     const float *w, const float *S0, void *o, float *ST, void *ws,
-                     size_t ws_bytes, int B, int T, int H, int d_k, int d_v, int chunk,
-                     gdn2_io io, gdn2_stream_t stream) {
+// gate tensors in bf16 need the tensor-core path
+static gdn2_status check_gate_io(const Dims &d, gdn2_io io, gdn2_io gate_io) {
+    if (gate_io != GDN2_IO_F32 && gate_io != GDN2_IO_BF16) return GDN2_ERR_INVALID_ARG;
+    if (gate_io == GDN2_IO_BF16 && !use_tc(d, io)) return GDN2_ERR_UNSUPPORTED;
+    return GDN2_OK;
+}
+
+gdn2_status gdn2_fwd_ex(const void *q, const void *k, const void *v, const void *g, const void *b,
+                        const void *w, const float *S0, void *o, float *ST, void *ws,
+                        size_t ws_bytes, int B, int T, int H, int d_k, int d_v, int chunk,
+                        gdn2_io io, gdn2_io gate_io, gdn2_stream_t stream) {
     gdn2_status st = check_dims(B, T, H, d_k, d_v, chunk, io);
     if (st != GDN2_OK) return st;
+    Dims d = make_dims(B, T, H, d_k, d_v, chunk);
+    if ((st = check_gate_io(d, io, gate_io)) != GDN2_OK) return st;
     st = check_ptrs({q, k, v, g, b, w, o}, {S0, ST});
     if (st != GDN2_OK) return st;
-    Dims d = make_dims(B, T, H, d_k, d_v, chunk);
     if (!ws || !aligned16(ws) || ws_bytes < ws_bytes_for(d, io, 0)) return GDN2_ERR_WORKSPACE;
+    d.gb = gate_io == GDN2_IO_BF16;
     if (use_tc(d, io)) {
         unsigned int *status = status_word();
         if (!status) return GDN2_ERR_CUDA;
@@ -185,20 +194,32 @@ gdn2_status gdn2_fwd(const void *q, const void *k, const void *v, const float *g
         return cuda_status(tc_fwd_launch(q, k, v, g, b, w, S0, o, ST, ws, keep, status, d,
                                          (cudaStream_t)stream));
     }
-    return cuda_status(run_forward(q, k, v, g, b, w, S0, o, ST, ws, d, io, (cudaStream_t)stream));
+    return cuda_status(run_forward(q, k, v, static_cast<const float *>(g), static_cast<const float *>(b),
+                                   static_cast<const float *>(w), S0, o, ST, ws, d, io,
+                                   (cudaStream_t)stream));
 }
 
-gdn2_status gdn2_bwd(const void *q, const void *k, const void *v, const float *g, const float *b,
-                     const float *w, const float *S0, const void *dO, const float *dST, void *dq,
-                     void *dk, void *dv, float *dg, float *db, float *dw, float *dS0, void *ws,
-                     size_t ws_bytes, int ws_has_fwd, int B, int T, int H, int d_k, int d_v,
-                     int chunk, gdn2_io io, gdn2_stream_t stream) {
+gdn2_status gdn2_fwd(const void *q, const void *k, const void *v, const float *g, const float *b,
+                     const float *w, const float *S0, void *o, float *ST, void *ws,
+                     size_t ws_bytes, int B, int T, int H, int d_k, int d_v, int chunk,
+                     gdn2_io io, gdn2_stream_t stream) {
+    return gdn2_fwd_ex(q, k, v, g, b, w, S0, o, ST, ws, ws_bytes, B, T, H, d_k, d_v, chunk, io,
+                       GDN2_IO_F32, stream);
+}
+
+gdn2_status gdn2_bwd_ex(const void *q, const void *k, const void *v, const void *g, const void *b,
+                        const void *w, const float *S0, const void *dO, const float *dST, void *dq,
+                        void *dk, void *dv, void *dg, void *db, void *dw, float *dS0, void *ws,
+                        size_t ws_bytes, int ws_has_fwd, int B, int T, int H, int d_k, int d_v,
+                        int chunk, gdn2_io io, gdn2_io gate_io, gdn2_stream_t stream) {
     gdn2_status st = check_dims(B, T, H, d_k, d_v, chunk, io);
     if (st != GDN2_OK) return st;
+    Dims d = make_dims(B, T, H, d_k, d_v, chunk);
+    if ((st = check_gate_io(d, io, gate_io)) != GDN2_OK) return st;
     st = check_ptrs({q, k, v, g, b, w, dO, dq, dk, dv, dg, db, dw}, {S0, dST, dS0});
     if (st != GDN2_OK) return st;
-    Dims d = make_dims(B, T, H, d_k, d_v, chunk);
     if (!ws || !aligned16(ws) || ws_bytes < ws_bytes_for(d, io, 1)) return GDN2_ERR_WORKSPACE;
+    d.gb = gate_io == GDN2_IO_BF16;
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e;
     if (use_tc(d, io)) {
@@ -211,28 +232,47 @@ gdn2_status gdn2_bwd(const void *q, const void *k, const void *v, const float *g
         return cuda_status(tc_bwd_launch(q, k, v, g, b, w, dO, dST, dq, dk, dv, dg, db, dw, dS0, ws,
                                          status, d, s));
     }
+    const float *gf = static_cast<const float *>(g), *bf = static_cast<const float *>(b),
+                *wf = static_cast<const float *>(w);
+    float *dgf = static_cast<float *>(dg), *dbf = static_cast<float *>(db), *dwf = static_cast<float *>(dw);
     if (!ws_has_fwd) {
-        e = run_forward(q, k, v, g, b, w, S0, nullptr, nullptr, ws, d, io, s);
+        e = run_forward(q, k, v, gf, bf, wf, S0, nullptr, nullptr, ws, d, io, s);
         if (e != cudaSuccess) return GDN2_ERR_CUDA;
     }
     if (io == GDN2_IO_BF16)
-        e = simt_bwd_launch<__nv_bfloat16>(q, k, v, b, w, dO, dST, dq, dk, dv, dg, db, dw, dS0, ws,
+        e = simt_bwd_launch<__nv_bfloat16>(q, k, v, bf, wf, dO, dST, dq, dk, dv, dgf, dbf, dwf, dS0, ws,
                                            d, s);
     else
-        e = simt_bwd_launch<float>(q, k, v, b, w, dO, dST, dq, dk, dv, dg, db, dw, dS0, ws, d, s);
+        e = simt_bwd_launch<float>(q, k, v, bf, wf, dO, dST, dq, dk, dv, dgf, dbf, dwf, dS0, ws, d, s);
     return cuda_status(e);
+}
+
+gdn2_status gdn2_bwd(const void *q, const void *k, const void *v, const float *g, const float *b,
+                     const float *w, const float *S0, const void *dO, const float *dST, void *dq,
+                     void *dk, void *dv, float *dg, float *db, float *dw, float *dS0, void *ws,
+                     size_t ws_bytes, int ws_has_fwd, int B, int T, int H, int d_k, int d_v,
+                     int chunk, gdn2_io io, gdn2_stream_t stream) {
+    return gdn2_bwd_ex(q, k, v, g, b, w, S0, dO, dST, dq, dk, dv, dg, db, dw, dS0, ws, ws_bytes,
+                       ws_has_fwd, B, T, H, d_k, d_v, chunk, io, GDN2_IO_F32, stream);
+}
+
+gdn2_status gdn2_decode_step_ex(const void *q, const void *k, const void *v, const void *g,
+                                const void *b, const void *w, float *S, void *o, int N, int H,
+                                int d_k, int d_v, gdn2_io io, gdn2_io gate_io, gdn2_stream_t stream) {
+    if (N < 1 || H < 1 || (io != GDN2_IO_F32 && io != GDN2_IO_BF16)) return GDN2_ERR_INVALID_ARG;
+    if (gate_io != GDN2_IO_F32 && gate_io != GDN2_IO_BF16) return GDN2_ERR_INVALID_ARG;
+    if (!supported_d(d_k) || !supported_d(d_v)) return GDN2_ERR_UNSUPPORTED;
+    if ((long long)N * H > 0x7fffffffLL) return GDN2_ERR_UNSUPPORTED;
+    gdn2_status st = check_ptrs({q, k, v, g, b, w, S, o}, {});
+    if (st != GDN2_OK) return st;
+    return cuda_status(decode_launch(q, k, v, g, b, w, S, o, N, H, d_k, d_v, io, gate_io,
+                                     (cudaStream_t)stream));
 }
 
 gdn2_status gdn2_decode_step(const void *q, const void *k, const void *v, const float *g,
                              const float *b, const float *w, float *S, void *o, int N, int H,
                              int d_k, int d_v, gdn2_io io, gdn2_stream_t stream) {
-    if (N < 1 || H < 1 || (io != GDN2_IO_F32 && io != GDN2_IO_BF16)) return GDN2_ERR_INVALID_ARG;
-    if (!supported_d(d_k) || !supported_d(d_v)) return GDN2_ERR_UNSUPPORTED;
-    if ((long long)N * H > 0x7fffffffLL) return GDN2_ERR_UNSUPPORTED;
-    gdn2_status st = check_ptrs({q, k, v, g, b, w, S, o}, {});
-    if (st != GDN2_OK) return st;
-    return cuda_status(decode_launch(q, k, v, g, b, w, S, o, N, H, d_k, d_v, io,
-                                     (cudaStream_t)stream));
+    return gdn2_decode_step_ex(q, k, v, g, b, w, S, o, N, H, d_k, d_v, io, GDN2_IO_F32, stream);
 }
 
 // One block, one waiting thread: an mbarrier that no copy or product will
@@ -278,12 +318,12 @@ const char *gdn2_status_string(gdn2_status status) {
         case GDN2_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
         case GDN2_ERR_CUDA: return "CUDA error";
         case GDN2_ERR_TIMEOUT: return "a kernel gave up on a bounded wait";
-        case GDN2_ERR_RANGE: return "input outside the tensor-core path's range (see gdn2.h)";
+        case GDN2_ERR_RANGE: return "an fp16 operand of the tensor-core path overflowed (see gdn2.h)";
     }
     return "unknown status";
 }
 
-int gdn2_version(void) { return 100; }
+int gdn2_version(void) { return 200; }
 
 unsigned long long gdn2_kernel_launches(void) { return g_launches.load(); }
 

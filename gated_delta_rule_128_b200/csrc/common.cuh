@@ -15,6 +15,7 @@ constexpr int kMaxChunk = 64;  // largest chunk
 
 struct Dims {
     int B, T, H, dk, dv, C, NC;
+    int gb;  // gate tensors g, b, w and dg, db, dw in bf16 (tensor-core path), else float32
 };
 
 // ---- element access in the io type (float or bf16), computing in float
@@ -123,7 +124,8 @@ inline SimtWs simt_ws_layout(const Dims &d) {
 // with plain bulk copies.  Offsets in bytes; bh = b * H + h.
 //   rec   [bh][NC]        66560 B  the chunk's record, written by the chunk-
 //                                  parallel prep kernel (layout REC_* below)
-//   ckS   [bh][NC][2 halves]  16 KB  chunk-entry states S_c (true scale)
+//   ckS   [bh][NC][2 halves]  16 KB  chunk-entry states in the chunk's frame, s S_c
+//                                  (a copy of the forward's fp16 operand)
 //   ckD   [bh][NC][2]          8 KB  Delta (columns of one d_v half)
 //   ckdS  [bh][NC][2]         16 KB  dL/dS_{c+1}, the state gradient leaving chunk c
 //   ckndU [bh][NC][2]          8 KB  -dU

@@ -28,11 +28,12 @@ template <int CL> __device__ __forceinline__ void vstore(float *p, const float *
     else { *p = x[0]; }
 }
 
-template <typename E, int DK, int DV>
+// E: the io type of q, k, v, o; GE: the gate type of g, b, w (float or bf16)
+template <typename E, typename GE, int DK, int DV>
 __global__ void __launch_bounds__(kDecThreads)
 decode_step_kernel(const E *__restrict__ q, const E *__restrict__ k, const E *__restrict__ v,
-                   const float *__restrict__ g, const float *__restrict__ b,
-                   const float *__restrict__ w, float *__restrict__ S, E *__restrict__ o, int H) {
+                   const GE *__restrict__ g, const GE *__restrict__ b,
+                   const GE *__restrict__ w, float *__restrict__ S, E *__restrict__ o, int H) {
     constexpr int RW = DK / kDecWarps;  // rows per warp
     constexpr int CL = DV / 32;         // columns per lane
     __shared__ float sk[DK], sbk[DK], sq[DK], sa[DK], su[DV], sdelta[DV];
@@ -50,9 +51,9 @@ decode_step_kernel(const E *__restrict__ q, const E *__restrict__ k, const E *__
 
     for (int i = tid; i < DK; i += kDecThreads) {
         float kv = ldx(k, hk + i), qv = ldx(q, hk + i);
-        sk[i] = kv; sq[i] = qv; sbk[i] = b[hk + i] * kv; sa[i] = __expf(g[hk + i]);
+        sk[i] = kv; sq[i] = qv; sbk[i] = ldx(b, hk + i) * kv; sa[i] = __expf(ldx(g, hk + i));
     }
-    for (int j = tid; j < DV; j += kDecThreads) su[j] = w[hv + j] * ldx(v, hv + j);
+    for (int j = tid; j < DV; j += kDecThreads) su[j] = ldx(w, hv + j) * ldx(v, hv + j);
     if (warp == 0) {
         float acc = 0.f;
         for (int i = lane; i < DK; i += 32) acc += ldx(k, hk + i) * ldx(q, hk + i);
@@ -101,23 +102,24 @@ decode_step_kernel(const E *__restrict__ q, const E *__restrict__ k, const E *__
     }
 }
 
-template <typename E, int DK, int DV>
-static cudaError_t launch_dec(const void *q, const void *k, const void *v, const float *g,
-                              const float *b, const float *w, float *S, void *o, int N, int H,
+template <typename E, typename GE, int DK, int DV>
+static cudaError_t launch_dec(const void *q, const void *k, const void *v, const void *g,
+                              const void *b, const void *w, float *S, void *o, int N, int H,
                               cudaStream_t s) {
     launch_begin(K_DECODE, s);
-    decode_step_kernel<E, DK, DV><<<(unsigned)N * (unsigned)H, kDecThreads, 0, s>>>(
-        (const E *)q, (const E *)k, (const E *)v, g, b, w, S, (E *)o, H);
+    decode_step_kernel<E, GE, DK, DV><<<(unsigned)N * (unsigned)H, kDecThreads, 0, s>>>(
+        (const E *)q, (const E *)k, (const E *)v, (const GE *)g, (const GE *)b, (const GE *)w, S,
+        (E *)o, H);
     launch_end(K_DECODE, s);
     return cudaGetLastError();
 }
 
-template <typename E>
-static cudaError_t dispatch_dec(const void *q, const void *k, const void *v, const float *g,
-                                const float *b, const float *w, float *S, void *o, int N, int H,
+template <typename E, typename GE>
+static cudaError_t dispatch_dec(const void *q, const void *k, const void *v, const void *g,
+                                const void *b, const void *w, float *S, void *o, int N, int H,
                                 int dk, int dv, cudaStream_t s) {
 #define GDN2_DEC(DK_, DV_) \
-    if (dk == DK_ && dv == DV_) return launch_dec<E, DK_, DV_>(q, k, v, g, b, w, S, o, N, H, s);
+    if (dk == DK_ && dv == DV_) return launch_dec<E, GE, DK_, DV_>(q, k, v, g, b, w, S, o, N, H, s);
     GDN2_DEC(32, 32) GDN2_DEC(32, 64) GDN2_DEC(32, 128)
     GDN2_DEC(64, 32) GDN2_DEC(64, 64) GDN2_DEC(64, 128)
     GDN2_DEC(128, 32) GDN2_DEC(128, 64) GDN2_DEC(128, 128)
@@ -125,12 +127,15 @@ static cudaError_t dispatch_dec(const void *q, const void *k, const void *v, con
     return cudaErrorInvalidValue;
 }
 
-cudaError_t decode_launch(const void *q, const void *k, const void *v, const float *g,
-                          const float *b, const float *w, float *S, void *o, int N, int H,
-                          int dk, int dv, gdn2_io io, cudaStream_t s) {
+cudaError_t decode_launch(const void *q, const void *k, const void *v, const void *g,
+                          const void *b, const void *w, float *S, void *o, int N, int H,
+                          int dk, int dv, gdn2_io io, gdn2_io gate_io, cudaStream_t s) {
+    using BF = __nv_bfloat16;
     if (io == GDN2_IO_BF16)
-        return dispatch_dec<__nv_bfloat16>(q, k, v, g, b, w, S, o, N, H, dk, dv, s);
-    return dispatch_dec<float>(q, k, v, g, b, w, S, o, N, H, dk, dv, s);
+        return gate_io == GDN2_IO_BF16 ? dispatch_dec<BF, BF>(q, k, v, g, b, w, S, o, N, H, dk, dv, s)
+                                       : dispatch_dec<BF, float>(q, k, v, g, b, w, S, o, N, H, dk, dv, s);
+    return gate_io == GDN2_IO_BF16 ? dispatch_dec<float, BF>(q, k, v, g, b, w, S, o, N, H, dk, dv, s)
+                                   : dispatch_dec<float, float>(q, k, v, g, b, w, S, o, N, H, dk, dv, s);
 }
 
 }  // namespace gdn2

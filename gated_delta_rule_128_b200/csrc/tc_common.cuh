@@ -105,6 +105,41 @@ __host__ __device__ __forceinline__ uint32_t raw32(int t, int c) {
     return (uint32_t)((c >> 5) * 8192) + sw128_chunk(t, (c & 31) >> 2, 64) + (uint32_t)((c & 3) * 4);
 }
 
+// Gate tiles (g, b, w and their gradients) come as float32 or bf16.  GB
+// selects bf16: two 64-channel boxes (raw16) instead of four 32-channel ones
+// (raw32), half the bytes.  Values are widened to float32 on load and rounded
+// once on store.
+template <bool GB> __host__ __device__ __forceinline__ uint32_t graw(int t, int c) {
+    return GB ? raw16(t, c) : raw32(t, c);
+}
+template <bool GB> constexpr int gate_box_cols() { return GB ? 64 : 32; }
+template <bool GB> constexpr uint32_t gate_tile_bytes() { return GB ? 16384u : 32768u; }
+template <bool GB> __device__ __forceinline__ float gld1(const unsigned char *p) {
+    if constexpr (GB) return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(p));
+    else return *reinterpret_cast<const float *>(p);
+}
+template <bool GB> __device__ __forceinline__ float2 gld2(const unsigned char *p) {
+    if constexpr (GB) return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(p));
+    else return *reinterpret_cast<const float2 *>(p);
+}
+template <bool GB> __device__ __forceinline__ float4 gld4(const unsigned char *p) {
+    if constexpr (GB) {
+        float x[4];
+        ld_bf4(p, x);
+        return make_float4(x[0], x[1], x[2], x[3]);
+    } else {
+        return *reinterpret_cast<const float4 *>(p);
+    }
+}
+template <bool GB> __device__ __forceinline__ void gst1(unsigned char *p, float a) {
+    if constexpr (GB) *reinterpret_cast<__nv_bfloat16 *>(p) = __float2bfloat16_rn(a);
+    else *reinterpret_cast<float *>(p) = a;
+}
+template <bool GB> __device__ __forceinline__ void gst2(unsigned char *p, float a, float b) {
+    if constexpr (GB) *reinterpret_cast<uint32_t *>(p) = pack_bf16(a, b);
+    else *reinterpret_cast<float2 *>(p) = make_float2(a, b);
+}
+
 // Warp-level tf32 tile product D = A B + D (m16n8k8, f32 accumulate).
 // Fragments (g = lane / 4, t = lane % 4): a0 (g, t), a1 (g + 8, t),
 // a2 (g, t + 4), a3 (g + 8, t + 4); b0 (k = t, n = g), b1 (k = t + 4, n = g);

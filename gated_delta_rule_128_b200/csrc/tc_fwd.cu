@@ -54,7 +54,7 @@ constexpr uint32_t STAGE = 74752;
 // shared memory map (bytes from a 1024-aligned base)
 constexpr uint32_t STG = 0;                  // two record stages
 constexpr uint32_t RAW_V = 2 * STAGE;        // v half, bf16 [64 pos][64]
-constexpr uint32_t RAW_W = RAW_V + 8192;     // w half, f32  [64 pos][64]
+constexpr uint32_t RAW_W = RAW_V + 8192;     // w half, f32 or bf16 [64 pos][64]
 constexpr uint32_t OP_U = RAW_W + 16384;     // two U = w.v tiles [64 pos][64 v] MN-major, 8 KB each
 constexpr uint32_t OP_S = OP_U + 16384;      // S (fp16)     [128 key][64 v] MN-major
 constexpr uint32_t OP_D = OP_S + 16384;      // Delta        [64 pos][64 v]  MN-major
@@ -67,8 +67,10 @@ constexpr uint32_t ID_MM128x64 = idesc_f16(128, 64, true, true);
 constexpr long long kWait = 2000000000LL;  // ~1 s of SM clocks per wait
 constexpr float kRange = 6.0e4f;           // largest operand magnitude kept in fp16
 static_assert(STAGE % 1024 == 0 && MISC % 1024 == 0, "alignment");
+static_assert(SMEM_BYTES <= 232448, "shared memory");
 }  // namespace tfwd
 
+template <bool GB>  // w as bf16 (else float32)
 __global__ void __launch_bounds__(tfwd::kThreads, 1)
 tc_fwd_kernel(const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mw,
               const float *__restrict__ S0, __nv_bfloat16 *__restrict__ o, float *__restrict__ ST,
@@ -122,7 +124,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mv, const __grid_constant__ CU
         ++issued[s];
     };
     auto load_vw = [&](int cc) {  // thread 64
-        mbar_expect_tx(&bars[2], 8192 + 16384);
+        mbar_expect_tx(&bars[2], 8192 + (GB ? 8192 : 16384));
         tma_load_4d(sm + RAW_V, &mv, v0, h, cc * 64, bb, &bars[2]);
         tma_load_4d(sm + RAW_W, &mw, v0, h, cc * 64, bb, &bars[2]);
         ++issued[2];
@@ -135,8 +137,14 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mv, const __grid_constant__ CU
         for (int i = 0; i < 4; ++i) {
             const int r = (ot >> 3) + 16 * i;
             const uint4 vr = *reinterpret_cast<const uint4 *>(sm + RAW_V + r * 128 + jv * 16);
-            const float4 w0 = *reinterpret_cast<const float4 *>(sm + RAW_W + r * 256 + jv * 32);
-            const float4 w1 = *reinterpret_cast<const float4 *>(sm + RAW_W + r * 256 + jv * 32 + 16);
+            float4 w0, w1;
+            if constexpr (GB) {
+                w0 = gld4<true>(sm + RAW_W + r * 128 + jv * 16);
+                w1 = gld4<true>(sm + RAW_W + r * 128 + jv * 16 + 8);
+            } else {
+                w0 = *reinterpret_cast<const float4 *>(sm + RAW_W + r * 256 + jv * 32);
+                w1 = *reinterpret_cast<const float4 *>(sm + RAW_W + r * 256 + jv * 32 + 16);
+            }
             const __nv_bfloat162 *v2 = reinterpret_cast<const __nv_bfloat162 *>(&vr);
             float u[8] = {w0.x * __low2float(v2[0]), w0.y * __high2float(v2[0]),
                           w0.z * __low2float(v2[1]), w0.w * __high2float(v2[1]),
@@ -346,27 +354,34 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mv, const __grid_constant__ CU
 }
 
 // ---------------------------------------------------------------- launcher
-cudaError_t tc_prep_launch(const void *q, const void *k, const float *g, const float *b, void *ws,
+cudaError_t tc_prep_launch(const void *q, const void *k, const void *g, const void *b, void *ws,
                            unsigned int *status, const Dims &d, cudaStream_t s);
 
-// keep != 0: also leave the chunk states and Delta for the backward
-cudaError_t tc_fwd_launch(const void *q, const void *k, const void *v, const float *g,
-                          const float *b, const float *w, const float *S0, void *o, float *ST,
-                          void *ws, int keep, unsigned int *status, const Dims &d, cudaStream_t s) {
-    cudaError_t e = tc_prep_launch(q, k, g, b, ws, status, d, s);
-    if (e != cudaSuccess) return e;
+template <bool GB>
+static cudaError_t tc_fwd_run(const void *v, const void *w, const float *S0, void *o, float *ST,
+                              void *ws, int keep, unsigned int *status, const Dims &d, cudaStream_t s) {
     CUtensorMap mv, mw;
     if (!make_btHd_map(&mv, v, true, d.B, d.T, d.H, 128, 64, 64) ||
-        !make_btHd_map(&mw, w, false, d.B, d.T, d.H, 128, 64, 64))
+        !make_btHd_map(&mw, w, GB, d.B, d.T, d.H, 128, 64, 64))
         return cudaErrorInvalidValue;
-    e = cudaFuncSetAttribute(tc_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)tfwd::SMEM_BYTES);
+    cudaError_t e = cudaFuncSetAttribute(tc_fwd_kernel<GB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)tfwd::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     launch_begin(K_TC_FWD, s);
-    tc_fwd_kernel<<<dim3(2, d.H, d.B), tfwd::kThreads, tfwd::SMEM_BYTES, s>>>(
+    tc_fwd_kernel<GB><<<dim3(2, d.H, d.B), tfwd::kThreads, tfwd::SMEM_BYTES, s>>>(
         mv, mw, S0, (__nv_bfloat16 *)o, ST, (unsigned char *)ws, keep, tc_ws_layout(d), status, d);
     launch_end(K_TC_FWD, s);
     return cudaGetLastError();
+}
+
+// keep != 0: also leave the chunk states and Delta for the backward
+cudaError_t tc_fwd_launch(const void *q, const void *k, const void *v, const void *g,
+                          const void *b, const void *w, const float *S0, void *o, float *ST,
+                          void *ws, int keep, unsigned int *status, const Dims &d, cudaStream_t s) {
+    cudaError_t e = tc_prep_launch(q, k, g, b, ws, status, d, s);
+    if (e != cudaSuccess) return e;
+    return d.gb ? tc_fwd_run<true>(v, w, S0, o, ST, ws, keep, status, d, s)
+                : tc_fwd_run<false>(v, w, S0, o, ST, ws, keep, status, d, s);
 }
 
 }  // namespace gdn2

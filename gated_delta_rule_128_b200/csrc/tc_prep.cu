@@ -42,8 +42,9 @@ using namespace tcc;
 
 namespace tprep {
 constexpr int kThreads = 256;
-// raw tiles (128-B swizzled boxes, tc_common.cuh raw16 / raw32); the g tile
-// later holds d = G' - G'_m per element
+// raw tiles (128-B swizzled boxes, tc_common.cuh raw16 / raw32; g and b as
+// float32 or bf16, graw); the g tile later holds d = G' - G'_m per element
+// (float32, raw32), once the cumulative decay has read g
 constexpr uint32_t RAW_Q = 0, RAW_K = 16384, RAW_G = 32768, RAW_B = 65536;
 constexpr uint32_t CO = 98304;        // [b.k.a; q.a] fp16 [128][128] K-major
 constexpr uint32_t RR = CO + 32768;   // R_1 (16 rows), R_2 (32), R_3 (48): fp16 K-major
@@ -146,6 +147,7 @@ __device__ __forceinline__ float ld_bf(const unsigned char *p) {
     return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(p));
 }
 
+template <bool GB>  // g, b as bf16 (else float32)
 __global__ void __launch_bounds__(tprep::kThreads, 1)
 tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                const __grid_constant__ CUtensorMap mg, const __grid_constant__ CUtensorMap mb,
@@ -182,14 +184,14 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
     int issued = 0;  // raw-tile loads requested (thread 0)
     auto load_raw = [&](int it) {
         const int c = it % NC, bh = it / NC, h = bh % H, bb = bh / H;
-        mbar_expect_tx(&bars[0], 16384 * 2 + 32768 * 2);
+        mbar_expect_tx(&bars[0], 16384 * 2 + gate_tile_bytes<GB>() * 2);
         for (int x = 0; x < 2; ++x) {
             tma_load_4d(sm + RAW_Q + x * 8192, &mq, 64 * x, h, c * 64, bb, &bars[0]);
             tma_load_4d(sm + RAW_K + x * 8192, &mk, 64 * x, h, c * 64, bb, &bars[0]);
         }
-        for (int x = 0; x < 4; ++x) {
-            tma_load_4d(sm + RAW_G + x * 8192, &mg, 32 * x, h, c * 64, bb, &bars[0]);
-            tma_load_4d(sm + RAW_B + x * 8192, &mb, 32 * x, h, c * 64, bb, &bars[0]);
+        for (int x = 0; x < 128 / gate_box_cols<GB>(); ++x) {
+            tma_load_4d(sm + RAW_G + x * 8192, &mg, gate_box_cols<GB>() * x, h, c * 64, bb, &bars[0]);
+            tma_load_4d(sm + RAW_B + x * 8192, &mb, gate_box_cols<GB>() * x, h, c * 64, bb, &bars[0]);
         }
         ++issued;
     };
@@ -213,7 +215,7 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
             float run[4] = {0.f, 0.f, 0.f, 0.f}, runc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                const float4 g4 = *reinterpret_cast<const float4 *>(sm + RAW_G + raw32(8 * warp + i, fc4));
+                const float4 g4 = gld4<GB>(sm + RAW_G + graw<GB>(8 * warp + i, fc4));
                 const float gv[4] = {g4.x * kLog2e, g4.y * kLog2e, g4.z * kLog2e, g4.w * kLog2e};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
@@ -243,25 +245,40 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
                     if (r8 < 4) g31[e] += tv[e];
                 }
             }
+            // the mild test, and the mild tile's operands written speculatively (a
+            // steep tile overwrites them): Kc = b k E, Qb = q E, Kh = k / E with
+            // E = e^(G - G_31)
             float dmax = 0.f, xmax = 0.f;
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
+                const int t = 8 * warp + i;
                 float qv[4], kv[4];
-                ld_bf4(sm + RAW_Q + raw16(8 * warp + i, fc4), qv);
-                ld_bf4(sm + RAW_K + raw16(8 * warp + i, fc4), kv);
-                const float4 b4 = *reinterpret_cast<const float4 *>(sm + RAW_B + raw32(8 * warp + i, fc4));
+                ld_bf4(sm + RAW_Q + raw16(t, fc4), qv);
+                ld_bf4(sm + RAW_K + raw16(t, fc4), kv);
+                const float4 b4 = gld4<GB>(sm + RAW_B + graw<GB>(t, fc4));
                 const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
+                float kcm[4], qbm[4], khm[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    dmax = fmaxf(dmax, fabsf(pre[e] + gl[i][e] - g31[e]));
-                    xmax = fmaxf(xmax, fmaxf(fabsf(qv[e]), fmaxf(fabsf(kv[e]), fabsf(bv[e] * kv[e]))));
+                    const float dl = pre[e] + gl[i][e] - g31[e];
+                    dmax = fmaxf(dmax, fabsf(dl));
+                    const float bk = bv[e] * kv[e];
+                    xmax = fmaxf(xmax, fmaxf(fabsf(qv[e]), fmaxf(fabsf(kv[e]), fabsf(bk))));
+                    const float E = ex2(dl), Ei = ex2(-dl);
+                    kcm[e] = bk * E;
+                    qbm[e] = qv[e] * E;
+                    khm[e] = kv[e] * Ei;
                 }
+                st_h4v(sm + OP_WQ + sw128_off(t, fc4, 128), kcm);
+                st_h4v(sm + OP_WQ + sw128_off(64 + t, fc4, 128), qbm);
+                st_h4v(sm + OP_KB + sw128_off(t, fc4, 64), khm);
             }
+            fence_proxy_async();
+            fence_before_sync();
             mild = !__syncthreads_or(!(dmax <= kMildG2 && xmax <= kMildX));
             if (mild) {
-                // ---------------- mild: the record takes the single frame of row 31
-                // (E = e^(G - G_31)): Kc = b k E, Qb = q E, Kh = k / E, and the frame
-                // factor s = e^G_31; A and P are [Kc; Qb] Kh^T
+                // ---------------- mild: the record takes the single frame of row 31:
+                // the frame factor s = e^G_31; A and P are [Kc; Qb] Kh^T
                 float all[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int r8 = 0; r8 < 8; ++r8) {
@@ -274,30 +291,6 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
                     *reinterpret_cast<float4 *>(sm + FAC + 512 + 4 * fc4) =
                         make_float4(ex2(g31[0]), ex2(g31[1]), ex2(g31[2]), ex2(g31[3]));  // s
                 }
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int t = 8 * warp + i;
-                    float qv[4], kv[4];
-                    ld_bf4(sm + RAW_Q + raw16(t, fc4), qv);
-                    ld_bf4(sm + RAW_K + raw16(t, fc4), kv);
-                    const float4 b4 = *reinterpret_cast<const float4 *>(sm + RAW_B + raw32(t, fc4));
-                    const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
-                    float kcm[4], qbm[4], khm[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float dl = pre[e] + gl[i][e] - g31[e];
-                        const float E = ex2(dl), Ei = ex2(-dl);
-                        kcm[e] = bv[e] * kv[e] * E;
-                        qbm[e] = qv[e] * E;
-                        khm[e] = kv[e] * Ei;
-                    }
-                    st_h4v(sm + OP_WQ + sw128_off(t, fc4, 128), kcm);
-                    st_h4v(sm + OP_WQ + sw128_off(64 + t, fc4, 128), qbm);
-                    st_h4v(sm + OP_KB + sw128_off(t, fc4, 64), khm);
-                }
-                fence_proxy_async();
-                fence_before_sync();
-                __syncthreads();
                 if (tid == 0) {
                     fence_after_sync();
                     const uint64_t co = desc_kmajor(smem_addr(sm + OP_WQ), 128, 0),
@@ -360,7 +353,7 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
                 float qv[4], kv[4];
                 ld_bf4(sm + RAW_Q + raw16(t, fc4), qv);
                 ld_bf4(sm + RAW_K + raw16(t, fc4), kv);
-                const float4 b4 = *reinterpret_cast<const float4 *>(sm + RAW_B + raw32(t, fc4));
+                const float4 b4 = gld4<GB>(sm + RAW_B + graw<GB>(t, fc4));
                 const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
                 float bka[4], qa[4], kc[4], qb[4], kb[4], ka[4], dd[4];
 #pragma unroll
@@ -422,7 +415,7 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
                 for (int h = 0; h < 2; ++h) {  // rows r0, r1
                     const int r = h ? r1 : r0;
                     const float4 d4 = *reinterpret_cast<const float4 *>(sm + RAW_G + raw32(r, c));
-                    const float4 b4 = *reinterpret_cast<const float4 *>(sm + RAW_B + raw32(r, c));
+                    const float4 b4 = gld4<GB>(sm + RAW_B + graw<GB>(r, c));
                     float qv[4], kv[4];
                     ld_bf4(sm + RAW_Q + raw16(r, c), qv);
                     ld_bf4(sm + RAW_K + raw16(r, c), kv);
@@ -599,24 +592,31 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
     if (warp == 0) tmem_dealloc(tm, 256);
 }
 
-cudaError_t tc_prep_launch(const void *q, const void *k, const float *g, const float *b, void *ws,
-                           unsigned int *status, const Dims &d, cudaStream_t s) {
+template <bool GB>
+static cudaError_t tc_prep_run(const void *q, const void *k, const void *g, const void *b, void *ws,
+                               unsigned int *status, const Dims &d, cudaStream_t s) {
     CUtensorMap mq, mk, mg, mb;
     if (!make_btHd_map(&mq, q, true, d.B, d.T, d.H, 128, 64, 64, true) ||
         !make_btHd_map(&mk, k, true, d.B, d.T, d.H, 128, 64, 64, true) ||
-        !make_btHd_map(&mg, g, false, d.B, d.T, d.H, 128, 64, 32, true) ||
-        !make_btHd_map(&mb, b, false, d.B, d.T, d.H, 128, 64, 32, true))
+        !make_btHd_map(&mg, g, GB, d.B, d.T, d.H, 128, 64, gate_box_cols<GB>(), true) ||
+        !make_btHd_map(&mb, b, GB, d.B, d.T, d.H, 128, 64, gate_box_cols<GB>(), true))
         return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(tc_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(tc_prep_kernel<GB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)tprep::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     const long long ntiles = (long long)d.B * d.H * d.NC;
     const int grid = (int)(ntiles < sm_count() ? ntiles : sm_count());
     launch_begin(K_TC_PREP, s);
-    tc_prep_kernel<<<grid, tprep::kThreads, tprep::SMEM_BYTES, s>>>(
+    tc_prep_kernel<GB><<<grid, tprep::kThreads, tprep::SMEM_BYTES, s>>>(
         mq, mk, mg, mb, (unsigned char *)ws, tc_ws_layout(d), status, d);
     launch_end(K_TC_PREP, s);
     return cudaGetLastError();
+}
+
+cudaError_t tc_prep_launch(const void *q, const void *k, const void *g, const void *b, void *ws,
+                           unsigned int *status, const Dims &d, cudaStream_t s) {
+    return d.gb ? tc_prep_run<true>(q, k, g, b, ws, status, d, s)
+                : tc_prep_run<false>(q, k, g, b, ws, status, d, s);
 }
 
 }  // namespace gdn2

@@ -24,7 +24,8 @@
  * Decode uses the same layouts with T = 1 removed: [N, H, d] and
  * [N, H, d_k, d_v].
  * Element types: q, k, v, o, dO, dq, dk, dv are float32 (GDN2_IO_F32) or
- *   bfloat16 (GDN2_IO_BF16); g, b, w, dg, db, dw and every state are float32.
+ *   bfloat16 (GDN2_IO_BF16); g, b, w, dg, db, dw are float32, or bfloat16
+ *   through the *_ex entry points (gate_io); every state is float32.
  * Supported sizes: B, T, H, N >= 1; d_k, d_v in {32, 64, 128}; chunk in
  *   {16, 32, 64}.  T need not be a multiple of chunk (the last chunk is short).
  *   The chunk size changes only the order of rounding, never the result.
@@ -41,14 +42,21 @@
  *   bounded wait records GDN2_ERR_TIMEOUT in a device status word that
  *   gdn2_get_device_status reports.
  * Paths: bf16 I/O with d_k = d_v = 128 and chunk 64 runs on the tensor cores
- *   (fp16 operands, fp32 accumulation and state); every other combination
- *   runs on the float32 CUDA-core path.  The tensor-core path forms the decay
- *   factors relative to the middle of each chunk, so it needs every key
- *   channel's cumulative log-decay to move by at most 9 within any 32-token
- *   half-chunk (and |q|, |k|, |b| <= 8 per element, |w v| and the state below
- *   6e4); a kernel that meets an input outside that range records
- *   GDN2_ERR_RANGE (the results of that call are then not valid).  The
- *   float32 path has no such limit.
+ *   (fp16 and tf32 operands, fp32 accumulation and state); every other
+ *   combination runs on the float32 CUDA-core path.  Both take any log-decay
+ *   g <= 0.  The tensor-core path forms every decay factor so that it stays
+ *   within fp16's range: state-side factors relative to the chunk's start
+ *   (all <= 1), in-chunk pair factors relative to 16-row block boundaries
+ *   (<= 1), and the 16 x 16 diagonal blocks in float32 relative to the block's
+ *   middle with each token's log-decay floored at -9 for those factors only
+ *   (a pair factor changes only where it is below e^-9 already, by at most
+ *   e^-9).  Chunks whose decay stays within e^4 of the chunk's row 31 (and
+ *   |q|, |k|, |b k| <= 256) take one frame for the whole chunk instead, which
+ *   is exact and faster.  An fp16 operand beyond 6e4 in magnitude (inputs or
+ *   states far outside the usual range) records GDN2_ERR_RANGE in the device
+ *   status word (the results of that call are then not valid); the float32
+ *   path has no such limit.  g > 0 is accepted but is not a decay: the
+ *   tensor-core path may then report GDN2_ERR_RANGE.
  */
 #ifndef GDN2_H
 #define GDN2_H
@@ -70,7 +78,7 @@ typedef enum {
     GDN2_ERR_WORKSPACE = 3,    /* workspace missing or smaller than required   */
     GDN2_ERR_CUDA = 4,         /* a CUDA launch or runtime call failed          */
     GDN2_ERR_TIMEOUT = 5,      /* a kernel gave up on a bounded wait            */
-    GDN2_ERR_RANGE = 6         /* inputs outside the tensor-core path's range   */
+    GDN2_ERR_RANGE = 6         /* an fp16 operand of the tensor-core path overflowed */
 } gdn2_status;
 
 typedef enum {
@@ -133,6 +141,33 @@ gdn2_status gdn2_bwd(const void *q, const void *k, const void *v, const float *g
 gdn2_status gdn2_decode_step(const void *q, const void *k, const void *v, const float *g,
                              const float *b, const float *w, float *S, void *o, int N, int H,
                              int d_k, int d_v, gdn2_io io, gdn2_stream_t stream);
+
+/* The same three calls with the gate tensors in a type of their own.
+ *   gate_io : type of g, b, w and of dg, db, dw.  GDN2_IO_F32 makes each call
+ *             identical to gdn2_fwd / gdn2_bwd / gdn2_decode_step.  GDN2_IO_BF16
+ *             halves the gate bytes ("Gated DeltaNet-2" LIT-802 review, "Key
+ *             takeaways" 1: b and w are sigmoid gates, values in (0, 1) or
+ *             (0, 2), which bf16 holds to 3 significant digits); values are
+ *             widened to float32 on load and the gradients rounded once on
+ *             store.  For gdn2_fwd_ex / gdn2_bwd_ex it needs the tensor-core
+ *             path (io = GDN2_IO_BF16, d_k = d_v = 128, chunk = 64) and returns
+ *             GDN2_ERR_UNSUPPORTED otherwise; gdn2_decode_step_ex takes it for
+ *             every size.
+ * Every other argument, the layouts, the workspace size and the error
+ * behaviour are those of the call without the suffix. */
+gdn2_status gdn2_fwd_ex(const void *q, const void *k, const void *v, const void *g, const void *b,
+                        const void *w, const float *S0, void *o, float *ST, void *ws,
+                        size_t ws_bytes, int B, int T, int H, int d_k, int d_v, int chunk,
+                        gdn2_io io, gdn2_io gate_io, gdn2_stream_t stream);
+gdn2_status gdn2_bwd_ex(const void *q, const void *k, const void *v, const void *g, const void *b,
+                        const void *w, const float *S0, const void *dO, const float *dST, void *dq,
+                        void *dk, void *dv, void *dg, void *db, void *dw, float *dS0, void *ws,
+                        size_t ws_bytes, int ws_has_fwd, int B, int T, int H, int d_k, int d_v,
+                        int chunk, gdn2_io io, gdn2_io gate_io, gdn2_stream_t stream);
+gdn2_status gdn2_decode_step_ex(const void *q, const void *k, const void *v, const void *g,
+                                const void *b, const void *w, float *S, void *o, int N, int H,
+                                int d_k, int d_v, gdn2_io io, gdn2_io gate_io,
+                                gdn2_stream_t stream);
 
 /* Bytes of the scratch array behind gdn2_fwd_noalloc (64 MiB). */
 #define GDN2_NOALLOC_SCRATCH_BYTES (64u << 20)

@@ -113,6 +113,26 @@ def test_decode_rejects_bad_arguments(L):
     assert f(*bad) == 1
 
 
+def test_ex_entry_points_check_the_gate_type(L):
+    """bf16 gates need the tensor-core path: any other size or io type is
+    rejected as unsupported, an unknown gate type as invalid, and float32
+    gates behave as the calls without the suffix."""
+    def fwd_ex(gate_io, dk=32, dv=32, chunk=16, io=0, ws_bytes=1 << 40):
+        return L.gdn2_fwd_ex(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, None, FAKE, ws_bytes,
+                             1, 16, 1, dk, dv, chunk, io, gate_io, None)
+    assert fwd_ex(1) == 2                              # f32 io, d = 32
+    assert fwd_ex(1, dk=128, dv=128, chunk=64) == 2    # still f32 io
+    assert fwd_ex(1, dk=128, dv=128, chunk=32, io=1) == 2
+    assert fwd_ex(5) == 1
+    assert fwd_ex(0, ws_bytes=10) == 3 == fwd(L, ws_bytes=10)
+    assert fwd_ex(1, dk=128, dv=128, chunk=64, io=1, ws_bytes=10) == 3   # passes the gate check
+    args = [FAKE] * 6 + [None, FAKE, None] + [FAKE] * 6 + [None, FAKE]
+    assert L.gdn2_bwd_ex(*args, 1 << 40, 1, 1, 16, 1, 32, 32, 16, 0, 1, None) == 2
+    assert L.gdn2_bwd_ex(*args, 1 << 40, 1, 1, 16, 1, 32, 32, 16, 0, 9, None) == 1
+    assert L.gdn2_decode_step_ex(*([FAKE] * 8), 1, 1, 32, 32, 0, 7, None) == 1
+    assert L.gdn2_decode_step_ex(*([FAKE] * 8), 1, 1, 16, 32, 0, 1, None) == 2
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(gdn, "_lib", None)
     monkeypatch.setattr(gdn, "LIB_PATH", str(tmp_path / "missing.so"))

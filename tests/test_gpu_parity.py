@@ -36,8 +36,8 @@ def tols(io):
     return (TOL_F32, TOL_F32) if io == "f32" else (TOL_BF16_OUT, TOL_BF16_GRAD)
 
 
-def gpu_fwd_bwd(x, io, chunk, backward=True, use_dST=True):
-    d = to_device(x, io)
+def gpu_fwd_bwd(x, io, chunk, backward=True, use_dST=True, gates="f32"):
+    d = to_device(x, io, gates=gates)
     o, ST, ws = gdn.forward(*(d[n] for n in NAMES), chunk=chunk, for_bwd=backward)
     out = {"o": o, "ST": ST}
     if backward:
@@ -49,14 +49,14 @@ def gpu_fwd_bwd(x, io, chunk, backward=True, use_dST=True):
     return {n: t.float().cpu().numpy() for n, t in out.items() if t is not None}
 
 
-def oracle_fwd_bwd(x, io, backward=True, use_dST=True, pairs=None):
+def oracle_fwd_bwd(x, io, backward=True, use_dST=True, pairs=None, gates="f32"):
     """Oracle on all (b, h) pairs, or on the listed ones (results stacked in
     the order given, as batch 1 with len(pairs) heads)."""
     if pairs is not None:
         x = {n: (torch.stack([t[bb, h] for bb, h in pairs])[None] if n in ("S0", "dST")
                  else torch.stack([t[bb, :, h] for bb, h in pairs], dim=1)[None]).contiguous()
              for n, t in x.items() if t.dim() == 4}
-    r = to_np64(io_round(x, io))
+    r = to_np64(io_round(x, io, gates))
     o, ST = oracle.forward(*(r[n] for n in NAMES))
     out = {"o": o, "ST": ST}
     if backward:
@@ -270,20 +270,63 @@ def test_full_workload_sampled_heads(index):
     compare(gpu, ref, wl.io, names, pairs=SAMPLE[index])
 
 
+# --------------------------------------------------------------- bf16 gates
+
+@pytest.mark.parametrize("index", [1, 2])
+def test_bf16_gates_full_workload_sampled_heads(index):
+    """g, b, w in bf16 (and dg, db, dw returned in bf16) on the tensor-core
+    path at full size: the oracle takes the same bf16-rounded gate values."""
+    wl = workloads.WORKLOADS[index]
+    x = workloads.draw_workload(index)
+    if wl.backward:
+        x["dST"] = torch.zeros(wl.B, wl.H, wl.dk, wl.dv)
+    gpu = gpu_fwd_bwd(x, wl.io, wl.chunk, backward=wl.backward, gates="bf16")
+    ref = oracle_fwd_bwd(x, wl.io, backward=wl.backward, pairs=SAMPLE[index], gates="bf16")
+    names = ("o", "ST") + (GRADS if wl.backward else ())
+    compare(gpu, ref, wl.io, names, pairs=SAMPLE[index])
+
+
+@pytest.mark.parametrize("kind", ["ragged", "steep_then_mild"])
+def test_bf16_gates_small(kind):
+    """bf16 gates on a ragged length (T = 200: three full chunks and a short
+    one) and on a call that takes both the steep and the mild tile paths."""
+    if kind == "ragged":
+        x = workloads.draw(2, 200, 2, 128, 128, 77, s0_std=0.1, with_dST=True)
+    else:
+        x = _steep(kind, 931)
+    gpu = gpu_fwd_bwd(x, "bf16", 64, gates="bf16")
+    ref = oracle_fwd_bwd(x, "bf16", gates="bf16")
+    compare(gpu, ref, "bf16", ("o", "ST") + GRADS)
+
+
+def test_bf16_gates_match_f32_gates_on_rounded_values():
+    """The two gate types give the same results when the float32 gates hold
+    the bf16-rounded values: the bf16 path only changes the storage."""
+    x = io_round(workloads.draw(1, 256, 2, 128, 128, 58, s0_std=0.1, with_dST=True), "f32", "bf16")
+    a = gpu_fwd_bwd(x, "bf16", 64, gates="f32")
+    b = gpu_fwd_bwd(x, "bf16", 64, gates="bf16")
+    for n in ("o", "ST", "dq", "dk", "dv", "dS0"):
+        assert np.array_equal(a[n], b[n]), n
+    for n in ("dg", "db", "dw"):   # rounded once more to bf16
+        assert rel(b[n], a[n]) < 4e-3, n
+
+
 # ------------------------------------------------------------------ decode
 
-@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("io,gates", [("f32", "f32"), ("bf16", "f32"), ("bf16", "bf16"),
+                                      ("f32", "bf16")])
 @pytest.mark.parametrize("dk,dv", [(128, 128), (64, 32), (32, 128)])
-def test_decode_small_step_by_step(io, dk, dv):
+def test_decode_small_step_by_step(io, gates, dk, dv):
     N, H, steps = 3, 2, 12
     S_gpu = (workloads.decode_state(N, H, dk, dv, 7, 0.3)).cuda()
     S_ref = S_gpu.double().cpu().numpy()
     dt = torch.bfloat16 if io == "bf16" else torch.float32
+    gt = torch.bfloat16 if gates == "bf16" else torch.float32
     tol = TOL_F32 if io == "f32" else TOL_BF16_OUT
     for s in range(steps):
         x = workloads.decode_step_inputs(N, H, dk, dv, 7, s, erase_scale=2.0 if s % 2 else 1.0)
-        xr = io_round(x, io)
-        d = {n: (t.to(dt) if n in ("q", "k", "v") else t).cuda() for n, t in x.items()}
+        xr = io_round(x, io, gates)
+        d = {n: (t.to(dt) if n in ("q", "k", "v") else t.to(gt)).cuda() for n, t in x.items()}
         o = gdn.decode_step(d["q"], d["k"], d["v"], d["g"], d["b"], d["w"], S_gpu)
         r = {n: t.double().numpy()[:, None] for n, t in xr.items()}
         o_ref, S_ref = oracle.forward(r["q"], r["k"], r["v"], r["g"], r["b"], r["w"], S_ref)
