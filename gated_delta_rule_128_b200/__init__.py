@@ -68,6 +68,12 @@ def lib() -> ctypes.CDLL:
         L.gdn2_bwd_ex.restype = i
         L.gdn2_decode_step_ex.argtypes = [vp] * 8 + [i] * 6 + [vp]
         L.gdn2_decode_step_ex.restype = i
+        L.gdn2_workspace_bytes_varlen.argtypes = [i] * 8
+        L.gdn2_workspace_bytes_varlen.restype = sz
+        L.gdn2_fwd_varlen.argtypes = [vp] * 10 + [sz, vp] + [i] * 8 + [vp]
+        L.gdn2_fwd_varlen.restype = i
+        L.gdn2_bwd_varlen.argtypes = [vp] * 17 + [sz, i, vp] + [i] * 8 + [vp]
+        L.gdn2_bwd_varlen.restype = i
         L.gdn2_decode_step.restype = i
         L.gdn2_get_device_status.argtypes = [vp]
         L.gdn2_get_device_status.restype = i
@@ -181,6 +187,28 @@ def gdn2_decode_step_ex(q, k, v, g, b, w, S, o, N, H, d_k, d_v, io, gate_io, str
     _check("gdn2_decode_step_ex", rc)
 
 
+def gdn2_workspace_bytes_varlen(N, T, H, d_k, d_v, chunk, io, for_bwd) -> int:
+    return int(lib().gdn2_workspace_bytes_varlen(N, T, H, d_k, d_v, chunk, io, int(for_bwd)))
+
+
+def gdn2_fwd_varlen(q, k, v, g, b, w, S0, o, ST, ws, ws_bytes, cu_seqlens, N, T, H, d_k, d_v,
+                    chunk, io, gate_io, stream=None):
+    rc = lib().gdn2_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b), _ptr(w), _ptr(S0),
+                               _ptr(o), _ptr(ST), _ptr(ws), ws_bytes, _ptr(cu_seqlens), N, T, H,
+                               d_k, d_v, chunk, io, gate_io, _stream(stream))
+    _check("gdn2_fwd_varlen", rc)
+
+
+def gdn2_bwd_varlen(q, k, v, g, b, w, S0, dO, dST, dq, dk, dv, dg, db, dw, dS0, ws, ws_bytes,
+                    ws_has_fwd, cu_seqlens, N, T, H, d_k, d_v, chunk, io, gate_io, stream=None):
+    rc = lib().gdn2_bwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b), _ptr(w), _ptr(S0),
+                               _ptr(dO), _ptr(dST), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg),
+                               _ptr(db), _ptr(dw), _ptr(dS0), _ptr(ws), ws_bytes, int(ws_has_fwd),
+                               _ptr(cu_seqlens), N, T, H, d_k, d_v, chunk, io, gate_io,
+                               _stream(stream))
+    _check("gdn2_bwd_varlen", rc)
+
+
 def gdn2_decode_step(q, k, v, g, b, w, S, o, N, H, d_k, d_v, io, stream=None):
     rc = lib().gdn2_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b), _ptr(w), _ptr(S),
                                 _ptr(o), N, H, d_k, d_v, io, _stream(stream))
@@ -273,6 +301,56 @@ def backward(q, k, v, g, b, w, S0, dO, dST=None, *, chunk: int = 64,
     gdn2_bwd_ex(q, k, v, g, b, w, S0, dO, dST, out["dq"], out["dk"], out["dv"], out["dg"],
                 out["db"], out["dw"], out["dS0"], ws, ws.numel(), ws_has_fwd, B, T, H, dk, dv, chunk,
                 io, _gate_io_of(g, b, w), stream)
+    if check:
+        check_device_status(stream)
+    return out
+
+
+def forward_varlen(q, k, v, g, b, w, cu_seqlens, S0=None, *, chunk: int = 64,
+                   want_state: bool = True, ws: Optional[torch.Tensor] = None,
+                   for_bwd: bool = False, stream=None, check: bool = True):
+    """Packed sequences: q, k, g, b [1,T,H,dk]; v, w [1,T,H,dv]; cu_seqlens
+    int32 [N+1] on the device; S0 [N,H,dk,dv] or None.  Returns (o, S_T [N,...]
+    or None, ws)."""
+    _, T, H, dk = q.shape
+    dv = v.shape[-1]
+    N = cu_seqlens.numel() - 1
+    io = _io_of(q)
+    if ws is None:
+        n = gdn2_workspace_bytes_varlen(N, T, H, dk, dv, chunk, io, for_bwd)
+        if n == 0:
+            raise Gdn2Error("gdn2_workspace_bytes_varlen", 2)
+        ws = torch.empty(n, dtype=torch.uint8, device=q.device)
+    o = torch.empty(1, T, H, dv, dtype=q.dtype, device=q.device)
+    ST = torch.empty(N, H, dk, dv, dtype=torch.float32, device=q.device) if want_state else None
+    gdn2_fwd_varlen(q, k, v, g, b, w, S0, o, ST, ws, ws.numel(), cu_seqlens, N, T, H, dk, dv, chunk,
+                    io, _gate_io_of(g, b, w), stream)
+    if check:
+        check_device_status(stream)
+    return o, ST, ws
+
+
+def backward_varlen(q, k, v, g, b, w, cu_seqlens, S0, dO, dST=None, *, chunk: int = 64,
+                    ws: Optional[torch.Tensor] = None, ws_has_fwd: bool = False,
+                    want_dS0: bool = True, stream=None, check: bool = True) -> Dict[str, torch.Tensor]:
+    """Gradients of forward_varlen: dq, dk, dv, dg, db, dw and dS0 [N,...]."""
+    _, T, H, dk = q.shape
+    dv = v.shape[-1]
+    N = cu_seqlens.numel() - 1
+    io = _io_of(q)
+    if ws is None:
+        n = gdn2_workspace_bytes_varlen(N, T, H, dk, dv, chunk, io, True)
+        if n == 0:
+            raise Gdn2Error("gdn2_workspace_bytes_varlen", 2)
+        ws = torch.empty(n, dtype=torch.uint8, device=q.device)
+        ws_has_fwd = False
+    out = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
+               dg=torch.empty_like(g), db=torch.empty_like(b), dw=torch.empty_like(w))
+    out["dS0"] = (torch.empty(N, H, dk, dv, dtype=torch.float32, device=q.device)
+                  if want_dS0 else None)
+    gdn2_bwd_varlen(q, k, v, g, b, w, S0, dO, dST, out["dq"], out["dk"], out["dv"], out["dg"],
+                    out["db"], out["dw"], out["dS0"], ws, ws.numel(), ws_has_fwd, cu_seqlens, N, T,
+                    H, dk, dv, chunk, io, _gate_io_of(g, b, w), stream)
     if check:
         check_device_status(stream)
     return out

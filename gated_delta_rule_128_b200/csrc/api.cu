@@ -75,7 +75,7 @@ static unsigned long long g_kind_count[K_KINDS];
 static double g_kind_ms[K_KINDS];
 static const char *const g_kind_names[K_KINDS] = {
     "simt_chunk_prep", "simt_state_fwd", "simt_out_fwd", "simt_state_bwd", "simt_chunk_bwd_a",
-    "simt_chunk_bwd_b", "decode_step", "tc_prep", "tc_fwd", "tc_bwd_state", "tc_bwd_grad"};
+    "simt_chunk_bwd_b", "decode_step", "tc_prep", "tc_fwd", "tc_bwd_state", "tc_bwd_grad", "seq_table"};
 
 void launch_begin(int kind, cudaStream_t s) {
     g_launches.fetch_add(1, std::memory_order_relaxed);
@@ -254,6 +254,151 @@ gdn2_status gdn2_bwd(const void *q, const void *k, const void *v, const float *g
                      int chunk, gdn2_io io, gdn2_stream_t stream) {
     return gdn2_bwd_ex(q, k, v, g, b, w, S0, dO, dST, dq, dk, dv, dg, db, dw, dS0, ws, ws_bytes,
                        ws_has_fwd, B, T, H, d_k, d_v, chunk, io, GDN2_IO_F32, stream);
+}
+
+// ---------------------------------------------------------- packed sequences
+// Chunk offsets co[0..N] of the sequences cu[0..N] (chunk C): one block,
+// a block-wide scan in steps of its 1024 threads.  A table that is not
+// non-decreasing from 0 to T gets co = 0 throughout (every sequence empty)
+// and records GDN2_ERR_INVALID_ARG.
+static __global__ void __launch_bounds__(1024) seq_table_kernel(const int *cu, int N, int T, int C, int *co,
+                                                               unsigned int *status) {
+    __shared__ int warp_tot[32];
+    __shared__ int carry;
+    __shared__ int bad;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (tid == 0) {
+        carry = 0;
+        bad = (cu[0] != 0 || cu[N] != T);
+    }
+    __syncthreads();
+    for (int base = 0; base < N; base += 1024) {
+        const int n = base + tid;
+        int cnt = 0;
+        if (n < N) {
+            const int len = cu[n + 1] - cu[n];
+            if (len < 0) bad = 1;
+            cnt = len > 0 ? (len + C - 1) / C : 0;
+        }
+        int x = cnt;  // inclusive scan: warps, then warp totals
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, off);
+            if (lane >= off) x += y;
+        }
+        if (lane == 31) warp_tot[warp] = x;
+        __syncthreads();
+        if (warp == 0) {
+            int t = warp_tot[lane];
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, t, off);
+                if (lane >= off) t += y;
+            }
+            warp_tot[lane] = t;
+        }
+        __syncthreads();
+        const int incl = carry + x + (warp > 0 ? warp_tot[warp - 1] : 0);
+        if (n < N) co[n + 1] = incl;
+        __syncthreads();
+        if (tid == 1023) carry = incl;
+        __syncthreads();
+    }
+    if (tid == 0) co[0] = 0;
+    __syncthreads();
+    if (bad) {
+        for (int n = tid; n <= N; n += 1024) co[n] = 0;
+        if (tid == 0) record_status(status, GDN2_ERR_INVALID_ARG);
+    }
+}
+
+// a packed call: B = 1 row of T tokens holding N sequences, the chunk bound
+// ceil(T / C) + N, and the chunk table at the end of the workspace
+static Dims varlen_dims(int N, int T, int H, int dk, int dv, int chunk) {
+    Dims d = make_dims(1, T, H, dk, dv, chunk);
+    d.NC = (T + chunk - 1) / chunk + N;
+    d.N = N;
+    return d;
+}
+// the chunk table follows the records (a forward-only workspace) or the whole
+// layout (a workspace that keeps the forward for the backward)
+static size_t varlen_table_at(const Dims &d, int for_bwd) {
+    const TcWs t = tc_ws_layout(d);
+    return for_bwd ? t.bwd_end : t.rec_end;
+}
+static size_t varlen_ws_bytes(const Dims &d, int for_bwd) {
+    return varlen_table_at(d, for_bwd) + align256((size_t)(d.N + 1) * sizeof(int));
+}
+static gdn2_status check_varlen(int N, int T, int H, int dk, int dv, int chunk, gdn2_io io, gdn2_io gate_io,
+                                const int *cu) {
+    if (N < 1 || !cu || !aligned16(cu)) return GDN2_ERR_INVALID_ARG;
+    gdn2_status st = check_dims(1, T, H, dk, dv, chunk, io);
+    if (st != GDN2_OK) return st;
+    if (gate_io != GDN2_IO_F32 && gate_io != GDN2_IO_BF16) return GDN2_ERR_INVALID_ARG;
+    if (!use_tc(make_dims(1, T, H, dk, dv, chunk), io)) return GDN2_ERR_UNSUPPORTED;
+    if (N > 65535 || (long long)H * ((T + chunk - 1) / chunk + N) > 0x7fffffffLL) return GDN2_ERR_UNSUPPORTED;
+    return GDN2_OK;
+}
+static cudaError_t seq_table_launch(Dims &d, void *ws, int for_bwd, unsigned int *status, cudaStream_t s) {
+    int *co = reinterpret_cast<int *>(static_cast<char *>(ws) + varlen_table_at(d, for_bwd));
+    launch_begin(K_SEQ_TABLE, s);
+    seq_table_kernel<<<1, 1024, 0, s>>>(d.cu, d.N, d.T, d.C, co, status);
+    launch_end(K_SEQ_TABLE, s);
+    d.co = co;
+    return cudaGetLastError();
+}
+
+size_t gdn2_workspace_bytes_varlen(int N, int T, int H, int d_k, int d_v, int chunk, gdn2_io io, int for_bwd) {
+    if (N < 1 || check_dims(1, T, H, d_k, d_v, chunk, io) != GDN2_OK) return 0;
+    if (!use_tc(make_dims(1, T, H, d_k, d_v, chunk), io)) return 0;
+    return varlen_ws_bytes(varlen_dims(N, T, H, d_k, d_v, chunk), for_bwd);
+}
+
+gdn2_status gdn2_fwd_varlen(const void *q, const void *k, const void *v, const void *g, const void *b,
+                            const void *w, const float *S0, void *o, float *ST, void *ws, size_t ws_bytes,
+                            const int *cu_seqlens, int N, int T, int H, int d_k, int d_v, int chunk,
+                            gdn2_io io, gdn2_io gate_io, gdn2_stream_t stream) {
+    gdn2_status st = check_varlen(N, T, H, d_k, d_v, chunk, io, gate_io, cu_seqlens);
+    if (st != GDN2_OK) return st;
+    st = check_ptrs({q, k, v, g, b, w, o}, {S0, ST});
+    if (st != GDN2_OK) return st;
+    Dims d = varlen_dims(N, T, H, d_k, d_v, chunk);
+    d.cu = cu_seqlens;
+    d.gb = gate_io == GDN2_IO_BF16;
+    if (!ws || !aligned16(ws) || ws_bytes < varlen_ws_bytes(d, 0)) return GDN2_ERR_WORKSPACE;
+    unsigned int *status = status_word();
+    if (!status) return GDN2_ERR_CUDA;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int keep = ws_bytes >= varlen_ws_bytes(d, 1);
+    cudaError_t e = seq_table_launch(d, ws, keep, status, s);
+    if (e != cudaSuccess) return GDN2_ERR_CUDA;
+    return cuda_status(tc_fwd_launch(q, k, v, g, b, w, S0, o, ST, ws, keep, status, d, s));
+}
+
+gdn2_status gdn2_bwd_varlen(const void *q, const void *k, const void *v, const void *g, const void *b,
+                            const void *w, const float *S0, const void *dO, const float *dST, void *dq,
+                            void *dk, void *dv, void *dg, void *db, void *dw, float *dS0, void *ws,
+                            size_t ws_bytes, int ws_has_fwd, const int *cu_seqlens, int N, int T, int H,
+                            int d_k, int d_v, int chunk, gdn2_io io, gdn2_io gate_io, gdn2_stream_t stream) {
+    gdn2_status st = check_varlen(N, T, H, d_k, d_v, chunk, io, gate_io, cu_seqlens);
+    if (st != GDN2_OK) return st;
+    st = check_ptrs({q, k, v, g, b, w, dO, dq, dk, dv, dg, db, dw}, {S0, dST, dS0});
+    if (st != GDN2_OK) return st;
+    Dims d = varlen_dims(N, T, H, d_k, d_v, chunk);
+    d.cu = cu_seqlens;
+    d.gb = gate_io == GDN2_IO_BF16;
+    if (!ws || !aligned16(ws) || ws_bytes < varlen_ws_bytes(d, 1)) return GDN2_ERR_WORKSPACE;
+    unsigned int *status = status_word();
+    if (!status) return GDN2_ERR_CUDA;
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = seq_table_launch(d, ws, 1, status, s);
+    if (e != cudaSuccess) return GDN2_ERR_CUDA;
+    if (!ws_has_fwd) {
+        e = tc_fwd_launch(q, k, v, g, b, w, S0, nullptr, nullptr, ws, 1, status, d, s);
+        if (e != cudaSuccess) return GDN2_ERR_CUDA;
+    }
+    return cuda_status(tc_bwd_launch(q, k, v, g, b, w, dO, dST, dq, dk, dv, dg, db, dw, dS0, ws, status,
+                                     d, s));
 }
 
 gdn2_status gdn2_decode_step_ex(const void *q, const void *k, const void *v, const void *g,

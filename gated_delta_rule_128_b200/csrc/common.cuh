@@ -16,7 +16,57 @@ constexpr int kMaxChunk = 64;  // largest chunk
 struct Dims {
     int B, T, H, dk, dv, C, NC;
     int gb;  // gate tensors g, b, w and dg, db, dw in bf16 (tensor-core path), else float32
+    // Packed variable-length sequences (tensor-core path): N sequences whose
+    // tokens lie at rows cu[n] .. cu[n + 1] - 1 of a B = 1 batch, cu (device,
+    // N + 1 entries) as given by the caller, co (workspace, N + 1 entries) the
+    // first chunk of each sequence in chunk order; NC then bounds the total
+    // chunks.  cu == nullptr: B rows of T tokens each.
+    const int *cu, *co;
+    int N;
 };
+
+// One sequence as the kernels see it: its first row in the T axis of its
+// batch row `brow`, its length, its chunks and the first of them (global).
+struct Seq {
+    int bos, len, nc, c0, brow;
+};
+__device__ __forceinline__ Seq seq_of(const Dims &d, int n) {
+    if (!d.cu) return Seq{0, d.T, d.NC, n * d.NC, n};
+    const int bos = __ldg(d.cu + n), c0 = __ldg(d.co + n);
+    return Seq{bos, __ldg(d.cu + n + 1) - bos, __ldg(d.co + n + 1) - c0, c0, 0};
+}
+// sequences (rows of the batch, or packed sequences)
+__host__ __device__ __forceinline__ int num_seqs(const Dims &d) { return d.cu ? d.N : d.B; }
+// chunk tiles of the call, in the order (sequence, head, chunk)
+__device__ __forceinline__ int total_tiles(const Dims &d) {
+    return d.cu ? d.H * __ldg(d.co + d.N) : d.B * d.H * d.NC;
+}
+// workspace tile index of chunk c of head h of sequence s (B rows: (b H + h) NC + c)
+__device__ __forceinline__ int tile_of(const Dims &d, const Seq &s, int h, int c) {
+    return s.c0 * d.H + h * s.nc + c;
+}
+// the sequence, head and chunk of tile `it`
+__device__ __forceinline__ void tile_decode(const Dims &d, int it, int &n, int &h, int &c) {
+    if (!d.cu) {
+        c = it % d.NC;
+        const int bhi = it / d.NC;
+        h = bhi % d.H;
+        n = bhi / d.H;
+        return;
+    }
+    // the last sequence whose first tile is at or before it (it has chunks:
+    // the next sequence, or the end, starts after it)
+    int lo = 0, hi = d.N;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (__ldg(d.co + mid) * d.H <= it) lo = mid;
+        else hi = mid;
+    }
+    n = lo;
+    const int c0 = __ldg(d.co + lo), nc = __ldg(d.co + lo + 1) - c0, rem = it - c0 * d.H;
+    h = rem / nc;
+    c = rem - h * nc;
+}
 
 // ---- element access in the io type (float or bf16), computing in float
 template <typename E> __device__ __forceinline__ float ldx(const E *p, size_t i);
@@ -74,7 +124,7 @@ struct SimtWs {
 // with launch_begin / launch_end (kernel kind ids below)
 enum KernelKind {
     K_SIMT_PREP = 0, K_SIMT_STATE_FWD, K_SIMT_OUT, K_SIMT_STATE_BWD, K_SIMT_BWD_A, K_SIMT_BWD_B,
-    K_DECODE, K_TC_PREP, K_TC_FWD, K_TC_BWD_STATE, K_TC_BWD_GRAD, K_KINDS
+    K_DECODE, K_TC_PREP, K_TC_FWD, K_TC_BWD_STATE, K_TC_BWD_GRAD, K_SEQ_TABLE, K_KINDS
 };
 void launch_begin(int kind, cudaStream_t s);
 void launch_end(int kind, cudaStream_t s);

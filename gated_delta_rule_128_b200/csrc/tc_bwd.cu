@@ -68,8 +68,8 @@ __global__ void __launch_bounds__(tbs::kThreads, 1)
 tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_constant__ CUtensorMap mv,
                     const __grid_constant__ CUtensorMap mw, const __grid_constant__ CUtensorMap mdv,
                     const __grid_constant__ CUtensorMap mdw, const float *__restrict__ dST,
-                    float *__restrict__ dS0, unsigned char *__restrict__ ws, TcWs lay,
-                    unsigned int *status, Dims d) {
+                    float *__restrict__ dS0, void *__restrict__ dv_out, void *__restrict__ dw_out,
+                    unsigned char *__restrict__ ws, TcWs lay, unsigned int *status, Dims d) {
     using namespace tbs;
     extern __shared__ unsigned char smraw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(
@@ -81,13 +81,23 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
     float big = 0.f;  // range check: operand magnitude
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int vh = blockIdx.x, h = blockIdx.y, bb = blockIdx.z, v0 = vh * 64;
-    const int NC = d.NC, H = d.H;
+    const int vh = blockIdx.x, h = blockIdx.y, n = blockIdx.z, v0 = vh * 64;
+    // sequence n: tokens bos .. bos + T - 1 of batch row bb, chunks NC
+    const Seq sq = seq_of(d, n);
+    const int NC = sq.nc, T = sq.len, bb = sq.brow, bos = sq.bos;
     const bool compute = tid < kCompute, issuer = tid == kCompute, copier = tid == kCompute + 32;
+    const bool copy_warp = warp == kCompute / 32 + 1;
     const int quarter = warp & 3, half = (warp >> 2) & 1;
     const int key = quarter * 32 + lane;
-    const size_t bh = (size_t)bb * H + h;
-    const unsigned char *recs = ws + lay.rec + bh * NC * (size_t)REC_BYTES;
+    const size_t tile0 = (size_t)tile_of(d, sq, h, 0);  // workspace tile of chunk 0
+    const unsigned char *recs = ws + lay.rec + tile0 * (size_t)REC_BYTES;
+    if (NC <= 0) {  // an empty sequence: dS0 = dS_T
+        if (dS0 && tid < 256) {
+            const size_t so = st_off(d, n, h) + (size_t)(tid >> 1) * 128 + v0 + 32 * (tid & 1);
+            for (int j = 0; j < 32; ++j) dS0[so + j] = dST ? dST[so + j] : 0.f;
+        }
+        return;
+    }
 
     if (warp == 0) {
         tmem_alloc(tslot, 256);
@@ -112,14 +122,14 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
     };
     auto load_do = [&](int cc) {
         mbar_expect_tx(&bars[2], 8192);
-        tma_load_4d(sm + RAW_DO, &mdo, v0, h, cc * 64, bb, &bars[2]);
+        tma_load_4d(sm + RAW_DO, &mdo, v0, h, bos + cc * 64, bb, &bars[2]);
         ++issued[2];
     };
     auto load_vw = [&](int cc) {
         mbar_expect_tx(&bars[4], 8192 + (GB ? 8192 : 16384));
-        tma_load_4d(sm + VV, &mv, v0, h, cc * 64, bb, &bars[4]);
-        tma_load_4d(sm + VW, &mw, v0, h, cc * 64, bb, &bars[4]);
-        if (!GB) tma_load_4d(sm + VW + 8192, &mw, v0 + 32, h, cc * 64, bb, &bars[4]);
+        tma_load_4d(sm + VV, &mv, v0, h, bos + cc * 64, bb, &bars[4]);
+        tma_load_4d(sm + VW, &mw, v0, h, bos + cc * 64, bb, &bars[4]);
+        if (!GB) tma_load_4d(sm + VW + 8192, &mw, v0 + 32, h, bos + cc * 64, bb, &bars[4]);
         ++issued[4];
     };
     // the frame factor s of chunk cc (1 for the chunk-start frame)
@@ -127,11 +137,13 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
         const float sv = reinterpret_cast<const float *>(sm + STG + (cc & 1) * REC_BYTES + REC_FAC)[128 + key];
         return sv < 0.f ? 1.f : sv;
     };
-    // dO of the chunk in RAW_DO -> fp16 operand (each thread 16 values)
-    auto convert_do = [&]() {
+    // dO of chunk cc in RAW_DO -> fp16 operand (each thread 16 values); rows
+    // past the sequence's end (a packed layout's next sequence) count as zero
+    auto convert_do = [&](int cc) {
         const int r = tid >> 2, cg = tid & 3;
-        const uint4 d0 = *reinterpret_cast<const uint4 *>(sm + RAW_DO + r * 128 + cg * 32);
-        const uint4 d1 = *reinterpret_cast<const uint4 *>(sm + RAW_DO + r * 128 + cg * 32 + 16);
+        uint4 d0 = *reinterpret_cast<const uint4 *>(sm + RAW_DO + r * 128 + cg * 32);
+        uint4 d1 = *reinterpret_cast<const uint4 *>(sm + RAW_DO + r * 128 + cg * 32 + 16);
+        if (r >= T - 64 * cc) d0 = d1 = make_uint4(0u, 0u, 0u, 0u);
         const __nv_bfloat162 *a = reinterpret_cast<const __nv_bfloat162 *>(&d0);
         const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&d1);
         float x[16];
@@ -198,15 +210,41 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
         fence_proxy_async();
         return fine;
     };
-    // the copier: dv, dw and -dU of chunk cc out, then the v, w tiles of chunk cc - 1
+    // the copy warp: dv, dw and -dU of chunk cc out, then the v, w tiles of
+    // chunk cc - 1.  A chunk that ends inside a packed layout (rows past its
+    // sequence's end belong to the next sequence) leaves row by row from the
+    // whole warp instead of by TMA stores, which would write all 64 rows.
     auto store_du = [&](int cc) {
-        tma_store_4d(&mdv, sm + VV, v0, h, cc * 64, bb);
-        tma_store_4d(&mdw, sm + VW, v0, h, cc * 64, bb);
-        if (!GB) tma_store_4d(&mdw, sm + VW + 8192, v0 + 32, h, cc * 64, bb);
-        bulk_store(ws + lay.ckndU + ((bh * NC + cc) * 2 + vh) * 8192, sm + NDU, 8192);
-        bulk_commit();
-        bulk_wait_read();  // VV, VW and NDU may be rewritten
-        if (cc > 0) load_vw(cc - 1);
+        const int L = T - 64 * cc;
+        if (d.cu && L < 64) {
+            __nv_bfloat16 *dvp = reinterpret_cast<__nv_bfloat16 *>(dv_out);
+            for (int i = lane; i < L * 8; i += 32) {  // dv: 8 chunks of 8 bf16 per row
+                const int r = i >> 3, j = i & 7;
+                const size_t row = tok(d, bb, bos + 64 * cc + r, h, 128) + v0;
+                *reinterpret_cast<uint4 *>(dvp + row + 8 * j) =
+                    *reinterpret_cast<const uint4 *>(sm + VV + sw128_chunk(r, j, 64));
+                if constexpr (GB) {
+                    *reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(dw_out) + row + 8 * j) =
+                        *reinterpret_cast<const uint4 *>(sm + VW + sw128_chunk(r, j, 64));
+                } else {  // two [64][32] float32 boxes: 4 floats per 16-byte chunk
+                    for (int x = 0; x < 2; ++x)
+                        *reinterpret_cast<uint4 *>(reinterpret_cast<float *>(dw_out) + row + 32 * x + 4 * j) =
+                            *reinterpret_cast<const uint4 *>(sm + VW + x * 8192 + sw128_chunk(r, j, 64));
+                }
+            }
+            fence_proxy_async();
+            __syncwarp();
+        } else if (lane == 0) {
+            tma_store_4d(&mdv, sm + VV, v0, h, bos + cc * 64, bb);
+            tma_store_4d(&mdw, sm + VW, v0, h, bos + cc * 64, bb);
+            if (!GB) tma_store_4d(&mdw, sm + VW + 8192, v0 + 32, h, bos + cc * 64, bb);
+        }
+        if (lane == 0) {
+            bulk_store(ws + lay.ckndU + ((tile0 + cc) * 2 + vh) * 8192, sm + NDU, 8192);
+            bulk_commit();
+            bulk_wait_read();  // VV, VW and NDU may be rewritten
+            if (cc > 0) load_vw(cc - 1);
+        }
     };
 
     if (copier) {
@@ -219,7 +257,7 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
     bool ok = true;
     if (compute) {
         float x[32];
-        const size_t so = st_off(d, bb, h);
+        const size_t so = st_off(d, n, h);
 #pragma unroll
         for (int j = 0; j < 32; j += 4) {
             float4 t = dST ? *reinterpret_cast<const float4 *>(dST + so + (size_t)key * 128 + v0 + 32 * half + j)
@@ -229,7 +267,7 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
         ok = mbar_wait(&bars[(NC - 1) & 1], 0, kWait);
         ok = mbar_wait(&bars[2], 0, kWait) && ok;
         put_ds(x, NC - 1);
-        convert_do();
+        convert_do(NC - 1);
         tmem_wait_st();
     }
     fence_proxy_async();
@@ -237,7 +275,7 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
     bool abort = __syncthreads_or(!ok);
     if (!abort && copier) {
         fence_after_sync();
-        bulk_store(ws + lay.ckdS + ((bh * NC + NC - 1) * 2 + vh) * 16384, sm + OP_DS, 16384);
+        bulk_store(ws + lay.ckdS + ((tile0 + NC - 1) * 2 + vh) * 16384, sm + OP_DS, 16384);
         bulk_commit();
         if (NC > 1) load_do(NC - 2);
         bulk_wait_read();  // the dS' copy has left OP_DS
@@ -288,7 +326,7 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
         fence_proxy_async();
         fence_before_sync();
         __syncthreads();
-        if (copier && c + 1 < NC) store_du(c + 1);
+        if (copy_warp && c + 1 < NC) store_du(c + 1);
         if (issuer) {
             fence_after_sync();
             const uint32_t st = smem_addr(stg);
@@ -322,14 +360,14 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
             for (int j = 0; j < 32; ++j) sv[j] *= se;
             if (c == 0) {
                 if (dS0) {
-                    float *dst = dS0 + st_off(d, bb, h) + (size_t)key * 128 + v0 + 32 * half;
+                    float *dst = dS0 + st_off(d, n, h) + (size_t)key * 128 + v0 + 32 * half;
 #pragma unroll
                     for (int j = 0; j < 32; j += 4)
                         *reinterpret_cast<float4 *>(dst + j) = make_float4(sv[j], sv[j + 1], sv[j + 2], sv[j + 3]);
                 }
             } else {
                 put_ds(sv, c - 1);
-                convert_do();
+                convert_do(c - 1);
                 tmem_wait_st();
             }
         }
@@ -339,7 +377,7 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
         if (c > 0) {
             if (copier) {
                 fence_after_sync();
-                bulk_store(ws + lay.ckdS + ((bh * NC + c - 1) * 2 + vh) * 16384, sm + OP_DS, 16384);
+                bulk_store(ws + lay.ckdS + ((tile0 + c - 1) * 2 + vh) * 16384, sm + OP_DS, 16384);
                 bulk_commit();
                 if (c >= 2) {
                     load_do(c - 2);           // raw dO consumed
@@ -354,7 +392,7 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
     if (!abort && compute) ok = flush_du(0, (NC - 1) & 1, (NC - 1) & 1);
     fence_before_sync();
     const bool bad = __syncthreads_or(abort || !ok);
-    if (!bad && copier) store_du(0);
+    if (!bad && copy_warp) store_du(0);
     if (!(big <= kRange)) record_status(status, GDN2_ERR_RANGE);
     if (copier) bulk_wait_all();
     if (bad && copier) {
@@ -393,8 +431,8 @@ static cudaError_t tc_bwd_state_run(const void *v, const void *w, const void *dO
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tbs::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     launch_begin(K_TC_BWD_STATE, s);
-    tc_bwd_state_kernel<GB><<<dim3(2, d.H, d.B), tbs::kThreads, tbs::SMEM_BYTES, s>>>(
-        mdo_half, mv, mw, mdv, mdw, dST, dS0, (unsigned char *)ws, lay, status, d);
+    tc_bwd_state_kernel<GB><<<dim3(2, d.H, num_seqs(d)), tbs::kThreads, tbs::SMEM_BYTES, s>>>(
+        mdo_half, mv, mw, mdv, mdw, dST, dS0, dv, dw, (unsigned char *)ws, lay, status, d);
     launch_end(K_TC_BWD_STATE, s);
     return cudaGetLastError();
 }

@@ -123,8 +123,9 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
                    const __grid_constant__ CUtensorMap mb, const __grid_constant__ CUtensorMap mg,
                    const __grid_constant__ CUtensorMap mdo, const __grid_constant__ CUtensorMap mdq,
                    const __grid_constant__ CUtensorMap mdk, const __grid_constant__ CUtensorMap mdb,
-                   const __grid_constant__ CUtensorMap mdg, unsigned char *__restrict__ ws, TcWs lay,
-                   unsigned int *status, Dims d) {
+                   const __grid_constant__ CUtensorMap mdg, void *__restrict__ dq_out,
+                   void *__restrict__ dk_out, void *__restrict__ db_out, void *__restrict__ dg_out,
+                   unsigned char *__restrict__ ws, TcWs lay, unsigned int *status, Dims d) {
     using namespace tbg;
     extern __shared__ unsigned char smraw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(
@@ -144,8 +145,7 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
     float big = 0.f;  // range check: largest fp16 operand magnitude
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int NC = d.NC, H = d.H;
-    const int ntiles = d.B * H * NC;
+    const int ntiles = total_tiles(d);
     const int I = warp & 3, Q = (warp >> 2) & 3;  // row block (TMEM lane quarter); channel quarter
     const int gq = lane >> 2, tq = lane & 3;
     const bool compute = true, issuer = tid == 0;
@@ -165,13 +165,22 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
     fence_after_sync();
     const uint32_t tm = *tslot;
 
-    // tile `it` = (b * H + h) * NC + c; copies requested by the issuer
+    // tile `it` in (sequence, head, chunk) order (tile_decode); copies requested by the issuer
     int issued[3] = {0, 0, 0};  // operand parts 1, 2 and raw tiles
+    // the tile's head, first row and batch row
+    auto tile_rows = [&](int it, int &h, int &row0, int &bb) {
+        int n, c;
+        tile_decode(d, it, n, h, c);
+        const Seq sq = seq_of(d, n);
+        row0 = sq.bos + 64 * c;
+        bb = sq.brow;
+    };
     auto load_a1 = [&](int it) {  // dO (TMA) and -dU: [dO; -dU]
-        const int c = it % NC, bhi = it / NC, h = bhi % H, bb = bhi / H;
+        int h, row0, bb;
+        tile_rows(it, h, row0, bb);
         mbar_expect_tx(&bars[0], 32768);
         for (int x = 0; x < 2; ++x) {
-            tma_load_4d(sm + DN + x * 16384, &mdo, 64 * x, h, c * 64, bb, &bars[0]);
+            tma_load_4d(sm + DN + x * 16384, &mdo, 64 * x, h, row0, bb, &bars[0]);
             bulk_load(sm + DN + x * 16384 + 8192, ws + lay.ckndU + ((size_t)it * 2 + x) * 8192, 8192, &bars[0]);
         }
         ++issued[0];
@@ -185,15 +194,16 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
         ++issued[1];
     };
     auto load_b = [&](int it) {  // raw q, k, b, g
-        const int c = it % NC, bhi = it / NC, h = bhi % H, bb = bhi / H;
+        int h, row0, bb;
+        tile_rows(it, h, row0, bb);
         mbar_expect_tx(&bars[3], 32768 + 2 * gate_tile_bytes<GB>());
         for (int x = 0; x < 2; ++x) {
-            tma_load_4d(sm + RQ + x * 8192, &mq, 64 * x, h, c * 64, bb, &bars[3]);
-            tma_load_4d(sm + RK + x * 8192, &mk, 64 * x, h, c * 64, bb, &bars[3]);
+            tma_load_4d(sm + RQ + x * 8192, &mq, 64 * x, h, row0, bb, &bars[3]);
+            tma_load_4d(sm + RK + x * 8192, &mk, 64 * x, h, row0, bb, &bars[3]);
         }
         for (int x = 0; x < 128 / gate_box_cols<GB>(); ++x) {
-            tma_load_4d(sm + RG + x * 8192, &mg, gate_box_cols<GB>() * x, h, c * 64, bb, &bars[3]);
-            tma_load_4d(sm + RB + x * 8192, &mb, gate_box_cols<GB>() * x, h, c * 64, bb, &bars[3]);
+            tma_load_4d(sm + RG + x * 8192, &mg, gate_box_cols<GB>() * x, h, row0, bb, &bars[3]);
+            tma_load_4d(sm + RB + x * 8192, &mb, gate_box_cols<GB>() * x, h, row0, bb, &bars[3]);
         }
         ++issued[2];
     };
@@ -206,7 +216,13 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
     bool ok = true;
     int nmild = 0;  // mild tiles done (second product groups committed to bars[2])
     for (int it = blockIdx.x, n = 0; it < ntiles; it += gridDim.x, ++n) {
-        const int c = it % NC, bhi = it / NC, h = bhi % H, bb = bhi / H, c0 = c * 64;
+        int tn, h, c;
+        tile_decode(d, it, tn, h, c);
+        const Seq sq = seq_of(d, tn);
+        const int c0 = sq.bos + 64 * c, bb = sq.brow;
+        // a packed sequence's tail chunk: rows L..63 hold the next sequence's tokens
+        const int L = sq.len - 64 * c;
+        const bool tail = d.cu != nullptr && L < 64;
         const uint32_t par = n & 1;
         const int nxt = it + (int)gridDim.x;
         const bool more = nxt < ntiles;
@@ -218,6 +234,7 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
             const int i = tid + kCompute * m;
             unsigned char *p = sm + DN + (i >> 9) * 16384 + (i & 511) * 16;
             uint4 raw = *reinterpret_cast<const uint4 *>(p);
+            if (((i & 511) >> 3) >= L) raw = make_uint4(0u, 0u, 0u, 0u);  // rows past the sequence's end
             const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
             float x[8];
 #pragma unroll
@@ -246,6 +263,10 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
             mma_commit(&bars[1]);
         }
         ok = mbar_wait(&bars[3], par, kWait) && ok;  // raw q, k, b, g
+        if (tail) {
+            zero_rows(sm + RQ, 12, L, tid, kThreads);  // q, k, b, g: 96 KB of 8 KB boxes
+            __syncthreads();
+        }
         // ---------------- cumulative decay (log2 units): warp w = rows 8 (w & 7)
         // .. + 7 (block fb, half fh), channels fc, fc + 1 with fc = 64 (w >> 3) + 2 lane
         const int frg = warp & 7, fb = frg >> 1, fh = frg & 1, fc = 64 * ((warp >> 3) & 1) + 2 * lane;
@@ -668,13 +689,23 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
                 load_a1(nxt);
                 load_a2(nxt);
             }
-            for (int x = 0; x < 2; ++x) {
-                tma_store_4d(&mdq, sm + RQ + x * 8192, 64 * x, h, c0, bb);
-                tma_store_4d(&mdk, sm + RK + x * 8192, 64 * x, h, c0, bb);
+            if (!tail) {
+                for (int x = 0; x < 2; ++x) {
+                    tma_store_4d(&mdq, sm + RQ + x * 8192, 64 * x, h, c0, bb);
+                    tma_store_4d(&mdk, sm + RK + x * 8192, 64 * x, h, c0, bb);
+                }
+                for (int x = 0; x < 128 / gate_box_cols<GB>(); ++x)
+                    tma_store_4d(&mdb, sm + RB + x * 8192, gate_box_cols<GB>() * x, h, c0, bb);
+                bulk_commit();
             }
-            for (int x = 0; x < 128 / gate_box_cols<GB>(); ++x)
-                tma_store_4d(&mdb, sm + RB + x * 8192, gate_box_cols<GB>() * x, h, c0, bb);
-            bulk_commit();
+        }
+        if (tail) {  // rows 0 .. L - 1 only
+            const size_t row = tok(d, bb, c0, h, 128);
+            const size_t st16 = (size_t)d.H * 128 * 2, stg = (size_t)d.H * 128 * (GB ? 2 : 4);
+            store_rows(reinterpret_cast<unsigned char *>(dq_out) + row * 2, st16, sm + RQ, 2, L, tid, kThreads);
+            store_rows(reinterpret_cast<unsigned char *>(dk_out) + row * 2, st16, sm + RK, 2, L, tid, kThreads);
+            store_rows(reinterpret_cast<unsigned char *>(db_out) + row * (GB ? 2 : 4), stg, sm + RB, GB ? 2 : 4, L,
+                       tid, kThreads);
         }
         if (mild) {  // dG over E and 1 / E, which every thread has read
 #pragma unroll
@@ -709,10 +740,18 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
         fence_proxy_async();
         fence_before_sync();
         if (__syncthreads_or(!ok)) break;
+        if (tail) {
+            store_rows(reinterpret_cast<unsigned char *>(dg_out) + tok(d, bb, c0, h, 128) * (GB ? 2 : 4),
+                       (size_t)d.H * 128 * (GB ? 2 : 4), sm + RG, GB ? 2 : 4, L, tid, kThreads);
+            fence_proxy_async();
+            __syncthreads();  // every row has left the raw tiles
+        }
         if (issuer) {
-            for (int x = 0; x < 128 / gate_box_cols<GB>(); ++x)
-                tma_store_4d(&mdg, sm + RG + x * 8192, gate_box_cols<GB>() * x, h, c0, bb);
-            bulk_commit();
+            if (!tail) {
+                for (int x = 0; x < 128 / gate_box_cols<GB>(); ++x)
+                    tma_store_4d(&mdg, sm + RG + x * 8192, gate_box_cols<GB>() * x, h, c0, bb);
+                bulk_commit();
+            }
             bulk_wait_read();  // the tiles may be refilled
             if (more) load_b(nxt);
         }
@@ -759,7 +798,7 @@ static cudaError_t tc_bwd_grad_run(const void *q, const void *k, const void *g, 
     const long long ntiles = (long long)d.B * d.H * d.NC;
     const int grid = (int)(ntiles < sm_count() ? ntiles : sm_count());
     tc_bwd_grad_kernel<GB><<<grid, tbg::kThreads, tbg::SMEM_BYTES, s>>>(
-        mq, mk, mb, mg, mdo, mdq, mdk, mdb, mdg, (unsigned char *)ws, lay, status, d);
+        mq, mk, mb, mg, mdo, mdq, mdk, mdb, mdg, dq, dk, db, dg, (unsigned char *)ws, lay, status, d);
     launch_end(K_TC_BWD_GRAD, s);
     return cudaGetLastError();
 }

@@ -140,6 +140,35 @@ template <bool GB> __device__ __forceinline__ void gst2(unsigned char *p, float 
     else *reinterpret_cast<float2 *>(p) = make_float2(a, b);
 }
 
+// Zero rows L..63 of `boxes` consecutive 8 KB boxes of 64 rows x 128 B (the
+// rows of a chunk past its sequence's end, which a packed layout fills with
+// the next sequence's tokens).  A 128-byte swizzle permutes 16-byte chunks
+// within a row only, so whole rows are zeroed the same way in any layout.
+// Every thread of the block takes part; the caller supplies the barrier.
+__device__ __forceinline__ void zero_rows(unsigned char *base, int boxes, int L, int tid, int nthreads) {
+    const int per_box = (64 - L) * 8;
+    for (int i = tid; i < boxes * per_box; i += nthreads) {
+        const int box = i / per_box, rem = i - box * per_box;
+        *reinterpret_cast<uint4 *>(base + box * 8192 + (L + (rem >> 3)) * 128 + (rem & 7) * 16) =
+            make_uint4(0u, 0u, 0u, 0u);
+    }
+}
+
+// Copy rows 0..L-1 of a [64 rows][128 channels] raw tile (8 KB boxes of
+// 128-byte swizzled rows: es = 2 bytes per element, two boxes; es = 4, four)
+// to global rows dst + r * stride, 128 channels each: the tail chunk of a
+// packed sequence, whose TMA store would also write the next sequence's rows.
+// Every thread of the block takes part; the caller supplies the barriers.
+__device__ __forceinline__ void store_rows(unsigned char *dst, size_t stride, const unsigned char *tile,
+                                           int es, int L, int tid, int nthreads) {
+    const int per_row = es * 8;  // 16-byte chunks per row
+    for (int i = tid; i < L * per_row; i += nthreads) {
+        const int r = i / per_row, rem = i - r * per_row, x = rem >> 3, j = rem & 7;
+        *reinterpret_cast<uint4 *>(dst + r * stride + x * 128 + j * 16) =
+            *reinterpret_cast<const uint4 *>(tile + x * 8192 + sw128_chunk(r, j, 64));
+    }
+}
+
 // Warp-level tf32 tile product D = A B + D (m16n8k8, f32 accumulate).
 // Fragments (g = lane / 4, t = lane % 4): a0 (g, t), a1 (g + 8, t),
 // a2 (g, t + 4), a3 (g + 8, t + 4); b0 (k = t, n = g), b1 (k = t + 4, n = g);

@@ -85,14 +85,23 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mv, const __grid_constant__ CU
     float big = 0.f;  // largest operand magnitude seen (range check)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int vh = blockIdx.x, h = blockIdx.y, bb = blockIdx.z, v0 = vh * 64;
-    const int NC = d.NC, T = d.T, H = d.H;
+    const int vh = blockIdx.x, h = blockIdx.y, n = blockIdx.z, v0 = vh * 64;
+    // sequence n: tokens bos .. bos + T - 1 of batch row bb, chunks NC
+    const Seq sq = seq_of(d, n);
+    const int NC = sq.nc, T = sq.len, bb = sq.brow, bos = sq.bos;
     const int quarter = warp & 3, half = warp >> 2;
     const int key = quarter * 32 + lane;          // state row (TMEM lane) of this thread
     const bool dwarp = quarter < 2;               // reads Delta (lanes 0..63), else O (64..127)
     const int ot = (half * 2 + (quarter - 2)) * 32 + lane;  // 0..127 among the O warps
-    const size_t bh = (size_t)bb * H + h;
-    const unsigned char *recs = ws + lay.rec + bh * NC * (size_t)REC_BYTES;
+    const size_t tile0 = (size_t)tile_of(d, sq, h, 0);  // workspace tile of chunk 0
+    const unsigned char *recs = ws + lay.rec + tile0 * (size_t)REC_BYTES;
+    if (NC <= 0) {  // an empty sequence: S_T = S0
+        if (ST) {
+            const size_t so = st_off(d, n, h) + (size_t)(tid >> 1) * 128 + v0 + 32 * (tid & 1);
+            for (int j = 0; j < 32; ++j) ST[so + j] = S0 ? S0[so + j] : 0.f;
+        }
+        return;
+    }
 
     if (warp == 0) {
         tmem_alloc(tslot, 256);
@@ -125,8 +134,8 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mv, const __grid_constant__ CU
     };
     auto load_vw = [&](int cc) {  // thread 64
         mbar_expect_tx(&bars[2], 8192 + (GB ? 8192 : 16384));
-        tma_load_4d(sm + RAW_V, &mv, v0, h, cc * 64, bb, &bars[2]);
-        tma_load_4d(sm + RAW_W, &mw, v0, h, cc * 64, bb, &bars[2]);
+        tma_load_4d(sm + RAW_V, &mv, v0, h, bos + cc * 64, bb, &bars[2]);
+        tma_load_4d(sm + RAW_W, &mw, v0, h, bos + cc * 64, bb, &bars[2]);
         ++issued[2];
     };
     // U = w.v of chunk cc into OP_U[cc & 1] (O warps: 4 rows x 8 columns each)
@@ -150,6 +159,10 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mv, const __grid_constant__ CU
                           w0.z * __low2float(v2[1]), w0.w * __high2float(v2[1]),
                           w1.x * __low2float(v2[2]), w1.y * __high2float(v2[2]),
                           w1.z * __low2float(v2[3]), w1.w * __high2float(v2[3])};
+            if (r >= T - 64 * cc) {  // past the sequence's end (a packed layout's next sequence)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) u[e] = 0.f;
+            }
             st_h8(dst + sw128_chunk(r, jv, 64), u);
             big = absmax8(u, big);
         }
@@ -171,7 +184,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mv, const __grid_constant__ CU
         mma_commit(&bars[3]);
         ++groups[0];
     };
-    auto ckpt = [&](int c) { return ws + lay.ckS + ((bh * NC + c) * 2 + vh) * 16384; };
+    auto ckpt = [&](int c) { return ws + lay.ckS + ((tile0 + c) * 2 + vh) * 16384; };
     // O rows of chunk cc (O warps): accumulator rows 64..127, this warp's 32 columns
     auto store_o = [&](int cc) {
         float ov[32];
@@ -181,7 +194,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mv, const __grid_constant__ CU
         tmem_wait_ld();
         const int t = cc * 64 + key - 64;
         if (o && t < T) {
-            unsigned char *dst = reinterpret_cast<unsigned char *>(o + tok(d, bb, t, h, 128) + v0 + 32 * half);
+            unsigned char *dst = reinterpret_cast<unsigned char *>(o + tok(d, bb, bos + t, h, 128) + v0 + 32 * half);
 #pragma unroll
             for (int jj = 0; jj < 4; ++jj) st_bf16x8(dst + 16 * jj, ov + 8 * jj);
         }
@@ -197,7 +210,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mv, const __grid_constant__ CU
     bool ok = mbar_wait(&bars[0], 0, kWait);
     float sreg[32];  // this thread's state row `key`, columns v0 + 32 half + j
     {
-        const size_t so = st_off(d, bb, h);
+        const size_t so = st_off(d, n, h);
 #pragma unroll
         for (int j = 0; j < 32; j += 4) {
             float4 t = S0 ? *reinterpret_cast<const float4 *>(S0 + so + (size_t)key * 128 + v0 + 32 * half + j)
@@ -270,7 +283,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mv, const __grid_constant__ CU
                 mma_commit(&bars[4]);
                 ++groups[1];
                 if (keep) {  // Delta of this chunk and half, for the backward
-                    bulk_store(ws + lay.ckD + ((bh * NC + c) * 2 + vh) * 8192, sm + OP_D, 8192);
+                    bulk_store(ws + lay.ckD + ((tile0 + c) * 2 + vh) * 8192, sm + OP_D, 8192);
                     bulk_commit();
                 }
             }
@@ -314,7 +327,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mv, const __grid_constant__ CU
                     big = absmax8(xv + 8 * jj, big);
                 }
             } else if (ST) {
-                float *dst = ST + st_off(d, bb, h) + (size_t)key * 128 + v0 + 32 * half;
+                float *dst = ST + st_off(d, n, h) + (size_t)key * 128 + v0 + 32 * half;
 #pragma unroll
                 for (int j = 0; j < 32; j += 4)
                     *reinterpret_cast<float4 *>(dst + j) = make_float4(sreg[j], sreg[j + 1], sreg[j + 2], sreg[j + 3]);
@@ -368,7 +381,7 @@ static cudaError_t tc_fwd_run(const void *v, const void *w, const float *S0, voi
                                          (int)tfwd::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     launch_begin(K_TC_FWD, s);
-    tc_fwd_kernel<GB><<<dim3(2, d.H, d.B), tfwd::kThreads, tfwd::SMEM_BYTES, s>>>(
+    tc_fwd_kernel<GB><<<dim3(2, d.H, num_seqs(d)), tfwd::kThreads, tfwd::SMEM_BYTES, s>>>(
         mv, mw, S0, (__nv_bfloat16 *)o, ST, (unsigned char *)ws, keep, tc_ws_layout(d), status, d);
     launch_end(K_TC_FWD, s);
     return cudaGetLastError();

@@ -164,8 +164,7 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quarter = warp & 3;
-    const int NC = d.NC, H = d.H;
-    const int ntiles = d.B * H * NC;
+    const int ntiles = total_tiles(d);
 
     if (warp == 0) {
         tmem_alloc(tslot, 256);
@@ -183,15 +182,18 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
 
     int issued = 0;  // raw-tile loads requested (thread 0)
     auto load_raw = [&](int it) {
-        const int c = it % NC, bh = it / NC, h = bh % H, bb = bh / H;
+        int n, h, c;
+        tile_decode(d, it, n, h, c);
+        const Seq sq = seq_of(d, n);
+        const int row0 = sq.bos + 64 * c, bb = sq.brow;
         mbar_expect_tx(&bars[0], 16384 * 2 + gate_tile_bytes<GB>() * 2);
         for (int x = 0; x < 2; ++x) {
-            tma_load_4d(sm + RAW_Q + x * 8192, &mq, 64 * x, h, c * 64, bb, &bars[0]);
-            tma_load_4d(sm + RAW_K + x * 8192, &mk, 64 * x, h, c * 64, bb, &bars[0]);
+            tma_load_4d(sm + RAW_Q + x * 8192, &mq, 64 * x, h, row0, bb, &bars[0]);
+            tma_load_4d(sm + RAW_K + x * 8192, &mk, 64 * x, h, row0, bb, &bars[0]);
         }
         for (int x = 0; x < 128 / gate_box_cols<GB>(); ++x) {
-            tma_load_4d(sm + RAW_G + x * 8192, &mg, gate_box_cols<GB>() * x, h, c * 64, bb, &bars[0]);
-            tma_load_4d(sm + RAW_B + x * 8192, &mb, gate_box_cols<GB>() * x, h, c * 64, bb, &bars[0]);
+            tma_load_4d(sm + RAW_G + x * 8192, &mg, gate_box_cols<GB>() * x, h, row0, bb, &bars[0]);
+            tma_load_4d(sm + RAW_B + x * 8192, &mb, gate_box_cols<GB>() * x, h, row0, bb, &bars[0]);
         }
         ++issued;
     };
@@ -207,6 +209,15 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
         bool ok = mbar_wait(&bars[0], n & 1, kWait);
         if (tid == 0) bulk_wait_read();  // the previous tile's record has left shared memory
         if (__syncthreads_or(!ok)) { abort = true; break; }
+        if (d.cu) {  // packed sequences: rows past the sequence's end belong to the next one
+            int tn, th, tc;
+            tile_decode(d, it, tn, th, tc);
+            const int L = seq_of(d, tn).len - 64 * tc;
+            if (L < 64) {
+                zero_rows(sm + RAW_Q, 12, L, tid, kThreads);  // q, k, g, b: 96 KB of 8 KB boxes
+                __syncthreads();
+            }
+        }
 
         // ---------------- cumulative decay (log2 units) of this warp's 8 rows,
         // exact and clamped; lane fq owns channels 4 fq .. 4 fq + 3
@@ -604,6 +615,7 @@ static cudaError_t tc_prep_run(const void *q, const void *k, const void *g, cons
     cudaError_t e = cudaFuncSetAttribute(tc_prep_kernel<GB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)tprep::SMEM_BYTES);
     if (e != cudaSuccess) return e;
+    // (packed sequences: NC bounds the total chunks; the kernel reads the count)
     const long long ntiles = (long long)d.B * d.H * d.NC;
     const int grid = (int)(ntiles < sm_count() ? ntiles : sm_count());
     launch_begin(K_TC_PREP, s);

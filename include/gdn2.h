@@ -169,6 +169,42 @@ gdn2_status gdn2_decode_step_ex(const void *q, const void *k, const void *v, con
                                 int d_k, int d_v, gdn2_io io, gdn2_io gate_io,
                                 gdn2_stream_t stream);
 
+/* Packed variable-length sequences: N sequences stored back to back along one
+ * token axis, each with its own initial and final state (no state crosses from
+ * one sequence to the next; "Gated DeltaNet-2" LIT-802 review, "Where the
+ * hedges are": the mixer runs inside a language model, whose training packs
+ * documents of mixed lengths).
+ *   q, k, g, b, dq, dk, dg, db : [1, T, H, d_k];  v, w, o, dO, dv, dw : [1, T, H, d_v]
+ *   S0, ST, dST, dS0 : [N, H, d_k, d_v]
+ *   cu_seqlens : device int32 [N + 1]: sequence n holds tokens cu_seqlens[n]
+ *       .. cu_seqlens[n + 1] - 1.  It must rise from 0 to T (a sequence may be
+ *       empty: its S_T is S0).  The table is read on the device only (the call
+ *       does not synchronise): a table that breaks this rule makes the call
+ *       treat every sequence as empty and records GDN2_ERR_INVALID_ARG in the
+ *       device status word.
+ *   N : 1 .. 65535 sequences.
+ * Tensor-core path only: io = GDN2_IO_BF16, d_k = d_v = 128, chunk = 64, gate_io
+ * either type; other sizes return GDN2_ERR_UNSUPPORTED.  Chunks never cross a
+ * sequence boundary: a sequence of length L takes ceil(L / 64) chunks, the last
+ * one short.
+ * Workspace: gdn2_workspace_bytes_varlen (for_bwd as for gdn2_workspace_bytes,
+ * sized for the worst case of N sequences over T tokens); the workspace also
+ * holds the chunk table the call derives from cu_seqlens.  ws_has_fwd as for
+ * gdn2_bwd, with the same cu_seqlens. */
+size_t gdn2_workspace_bytes_varlen(int N, int T, int H, int d_k, int d_v, int chunk, gdn2_io io,
+                                   int for_bwd);
+gdn2_status gdn2_fwd_varlen(const void *q, const void *k, const void *v, const void *g,
+                            const void *b, const void *w, const float *S0, void *o, float *ST,
+                            void *ws, size_t ws_bytes, const int *cu_seqlens, int N, int T, int H,
+                            int d_k, int d_v, int chunk, gdn2_io io, gdn2_io gate_io,
+                            gdn2_stream_t stream);
+gdn2_status gdn2_bwd_varlen(const void *q, const void *k, const void *v, const void *g,
+                            const void *b, const void *w, const float *S0, const void *dO,
+                            const float *dST, void *dq, void *dk, void *dv, void *dg, void *db,
+                            void *dw, float *dS0, void *ws, size_t ws_bytes, int ws_has_fwd,
+                            const int *cu_seqlens, int N, int T, int H, int d_k, int d_v, int chunk,
+                            gdn2_io io, gdn2_io gate_io, gdn2_stream_t stream);
+
 /* Bytes of the scratch array behind gdn2_fwd_noalloc (64 MiB). */
 #define GDN2_NOALLOC_SCRATCH_BYTES (64u << 20)
 

@@ -311,6 +311,77 @@ def test_bf16_gates_match_f32_gates_on_rounded_values():
         assert rel(b[n], a[n]) < 4e-3, n
 
 
+# -------------------------------------------------------- packed sequences
+
+VARLEN_LENS = [65, 1, 200, 64, 0, 3, 130, 17]
+
+
+def _varlen_inputs(lens, H, seed):
+    cu = [0] + list(np.cumsum(lens))
+    N, T = len(lens), int(cu[-1])
+    x = workloads.draw(1, T, H, 128, 128, seed)
+    x["S0"] = workloads.draw(N, 1, H, 128, 128, seed + 1, s0_std=0.1)["S0"]
+    x["dST"] = workloads.draw(N, 1, H, 128, 128, seed + 2, s0_std=0.1)["S0"]
+    return x, [int(c) for c in cu]
+
+
+def gpu_varlen(x, cu, gates="f32"):
+    d = to_device(x, "bf16", gates=gates)
+    cu_d = torch.tensor(cu, dtype=torch.int32, device="cuda")
+    o, ST, ws = gdn.forward_varlen(*(d[n] for n in NAMES[:-1]), cu_d, d["S0"], for_bwd=True)
+    gr = gdn.backward_varlen(*(d[n] for n in NAMES[:-1]), cu_d, d["S0"], d["dO"], d["dST"], ws=ws,
+                             ws_has_fwd=True)
+    torch.cuda.synchronize()
+    assert gdn.gdn2_get_device_status() == 0
+    out = {"o": o, "ST": ST, **gr}
+    return {n: t.float().cpu().numpy() for n, t in out.items()}
+
+
+@pytest.mark.parametrize("gates", ["f32", "bf16"])
+def test_varlen_mixed_lengths(gates):
+    """Packed sequences of lengths 65, 1, 200, 64, 0, 3, 130 and 17 (short
+    tails, a sequence of one token, an empty one) against the oracle run on
+    each sequence alone from its own S0."""
+    from oracle import varlen
+    x, cu = _varlen_inputs(VARLEN_LENS, 2, 950)
+    gpu = gpu_varlen(x, cu, gates)
+    r = to_np64(io_round(x, "bf16", gates))
+    names = ("q", "k", "v", "g", "b", "w")
+    o, ST = varlen.forward(*(r[n] for n in names), cu, r["S0"])
+    ref = {"o": o, "ST": ST, **varlen.backward(*(r[n] for n in names), cu, r["S0"], r["dO"], r["dST"])}
+    compare(gpu, ref, "bf16", ("o", "ST") + GRADS)
+
+
+def test_varlen_equal_lengths_match_the_batch_bit_for_bit():
+    """Three sequences of 200 tokens packed back to back give exactly the
+    batch call's results: the same tiles, masked tails instead of the
+    tensor's end."""
+    B, T, H = 3, 200, 2
+    x = workloads.draw(B, T, H, 128, 128, 951, s0_std=0.1, with_dST=True)
+    dense = gpu_fwd_bwd(x, "bf16", 64)
+    packed = {n: (t.reshape(1, B * T, *t.shape[2:]) if n not in ("S0", "dST") else t) for n, t in x.items()}
+    pv = gpu_varlen(packed, [0, T, 2 * T, 3 * T])
+    for n in ("o", "dq", "dk", "dv", "dg", "db", "dw"):
+        assert np.array_equal(pv[n], dense[n].reshape(pv[n].shape)), n
+    for n in ("ST", "dS0"):
+        assert np.array_equal(pv[n], dense[n]), n
+
+
+def test_varlen_rejects_a_bad_table_on_the_device():
+    """A table that falls (0, 30, 20, 64) is caught on the device: the call
+    records GDN2_ERR_INVALID_ARG, treats every sequence as empty, and the
+    next valid call runs clean."""
+    x, cu = _varlen_inputs([30, 0, 44], 1, 952)
+    d = to_device(x, "bf16")
+    bad = torch.tensor([0, 30, 20, 74], dtype=torch.int32, device="cuda")
+    o, ST, _ = gdn.forward_varlen(*(d[n] for n in NAMES[:-1]), bad, d["S0"], check=False)
+    torch.cuda.synchronize()
+    assert gdn.gdn2_get_device_status() == 1
+    assert torch.equal(ST, d["S0"])
+    gpu = gpu_varlen(x, cu)          # asserts a clean status itself
+    assert np.isfinite(gpu["o"]).all()
+
+
 # ------------------------------------------------------------------ decode
 
 @pytest.mark.parametrize("io,gates", [("f32", "f32"), ("bf16", "f32"), ("bf16", "bf16"),

@@ -342,3 +342,55 @@ def test_forward_substitution_inverse():
     T = chunkwise._forward_substitution_inverse(A)
     np.testing.assert_allclose(T @ (np.eye(20) + A), np.eye(20), atol=1e-12)
     assert math.isclose(np.linalg.det(T), 1.0, rel_tol=1e-12)
+
+
+# ------------------------------------------------------ packed sequences
+
+def _packed(x, lens):
+    """Equal-length batch rows -> one packed row (for lens all equal to T)."""
+    return {n: (t.reshape(1, -1, *t.shape[2:]) if t.dim() == 4 and n not in ("S0", "dST") else t)
+            for n, t in x.items()}
+
+
+def test_varlen_oracle_equals_the_batch_for_equal_lengths():
+    """B rows of T tokens packed back to back with cu_seqlens = 0, T, 2T, ...
+    give the batch oracle's results: each sequence starts from its own S0."""
+    from oracle import varlen
+    B, T, H, dk, dv = 3, 37, 2, 8, 6
+    x = workloads.draw(B, T, H, dk, dv, 611, s0_std=0.3, with_dST=True)
+    r = {n: t.double().numpy() for n, t in x.items()}
+    o, ST = oracle.forward(*(r[n] for n in ("q", "k", "v", "g", "b", "w", "S0")))
+    gr = oracle.backward(*(r[n] for n in ("q", "k", "v", "g", "b", "w", "S0")), r["dO"], r["dST"])
+    p = {n: t.double().numpy() for n, t in _packed(x, None).items()}
+    cu = [0, T, 2 * T, 3 * T]
+    o2, ST2 = varlen.forward(*(p[n] for n in ("q", "k", "v", "g", "b", "w")), cu, p["S0"])
+    gr2 = varlen.backward(*(p[n] for n in ("q", "k", "v", "g", "b", "w")), cu, p["S0"], p["dO"], p["dST"])
+    assert np.array_equal(o2, o.reshape(1, B * T, H, dv)) and np.array_equal(ST2, ST)
+    for n in ("dq", "dk", "dv", "dg", "db", "dw"):
+        assert np.array_equal(gr2[n], gr[n].reshape(1, B * T, H, -1)), n
+    assert np.array_equal(gr2["dS0"], gr["dS0"])
+
+
+def test_varlen_oracle_sequences_are_independent():
+    """Changing one sequence's inputs leaves every other sequence's outputs
+    and gradients bit for bit; an empty sequence passes S0 through to S_T and
+    dS_T through to dS0."""
+    from oracle import varlen
+    lens = [5, 1, 0, 9]
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    T, H, dk, dv = int(cu[-1]), 2, 4, 3
+    x = workloads.draw(1, T, H, dk, dv, 612, with_dST=True)
+    S0 = workloads.draw(len(lens), 1, H, dk, dv, 613, s0_std=0.5)["S0"]
+    dST = workloads.draw(len(lens), 1, H, dk, dv, 614, s0_std=0.5)["S0"]
+    r = {n: t.double().numpy() for n, t in x.items()}
+    names = ("q", "k", "v", "g", "b", "w")
+    o, ST = varlen.forward(*(r[n] for n in names), cu, S0.double().numpy())
+    gr = varlen.backward(*(r[n] for n in names), cu, S0.double().numpy(), r["dO"], dST.double().numpy())
+    assert np.array_equal(ST[2], S0[2].double().numpy()) and np.array_equal(gr["dS0"][2], dST[2].double().numpy())
+    r2 = dict(r)
+    r2["v"] = r["v"].copy()
+    r2["v"][:, 5] += 1.0            # the length-1 sequence
+    o2, ST2 = varlen.forward(*(r2[n] for n in names), cu, S0.double().numpy())
+    keep = np.r_[0:5, 6:T]
+    assert np.array_equal(o2[:, keep], o[:, keep]) and not np.array_equal(o2[:, 5], o[:, 5])
+    assert np.array_equal(ST2[[0, 2, 3]], ST[[0, 2, 3]]) and not np.array_equal(ST2[1], ST[1])
