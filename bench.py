@@ -246,14 +246,14 @@ class FwdBwdCase:
         inp, out = inp or self.d, out or dict(o=self.o, **self.grads)
         g = self.gdn
         g.gdn2_fwd_ex(*(inp[n] for n in NAMES), out["o"], self.ST, self.ws, self.ws.numel(), self.B,
-                      self.T, self.H, self.dk, self.dv, self.C, self.io, self.gate_io, self.stream)
+                      self.T, self.H, self.H, self.dk, self.dv, self.C, self.io, self.gate_io, self.stream)
 
     def bwd(self, inp=None, out=None):
         inp, out = inp or self.d, out or dict(o=self.o, **self.grads)
         self.gdn.gdn2_bwd_ex(*(inp[n] for n in NAMES), inp["dO"], None, out["dq"], out["dk"],
                              out["dv"], out["dg"], out["db"], out["dw"], None, self.ws,
-                             self.ws.numel(), 1, self.B, self.T, self.H, self.dk, self.dv, self.C,
-                             self.io, self.gate_io, self.stream)
+                             self.ws.numel(), 1, self.B, self.T, self.H, self.H, self.dk, self.dv,
+                             self.C, self.io, self.gate_io, self.stream)
 
     def step(self, inp=None, out=None):
         self.fwd(inp, out)
@@ -331,6 +331,69 @@ def sub_workload(index, args, rank, dev, peak, peak_src, gates="f32"):
     if wl.backward:
         out.update(fwd_ms=fwd_ms, bwd_ms=bwd_ms)
     del case
+    torch.cuda.empty_cache()
+    return out
+
+
+def sub_packed(args, rank, dev, peak, peak_src):
+    """Workload 2's 16384 tokens per head as one packed row of sequences of
+    mixed lengths (uniform in [1, 2048], seeded), fwd+bwd through the packed
+    entry points: the step a training run on packed documents takes."""
+    import torch
+
+    import gated_delta_rule_128_b200 as gdn
+    from gated_delta_rule_128_b200 import dist as gd
+    from gated_delta_rule_128_b200 import workloads
+
+    wl = workloads.WORKLOADS[2]
+    T, H, dk, dv, C = wl.B * wl.T, wl.H, wl.dk, wl.dv, wl.chunk
+    seed = gd.rank_seed(1005, rank)
+    lens = workloads.packed_lengths(T, seed)
+    N = len(lens)
+    cu = torch.tensor([0] + list(torch.tensor(lens).cumsum(0).tolist()), dtype=torch.int32, device=dev)
+    x = workloads.draw(1, T, H, dk, dv, seed)
+    bf = torch.bfloat16
+    d = {n: (t.to(bf) if n in ("q", "k", "v", "dO") else t).contiguous().to(dev) for n, t in x.items()}
+    io, gio = gdn.GDN2_IO_BF16, gdn.GDN2_IO_F32
+    ws = torch.empty(gdn.gdn2_workspace_bytes_varlen(N, T, H, H, dk, dv, C, io, gio, 1), dtype=torch.uint8,
+                     device=dev)
+    o = torch.empty(1, T, H, dv, dtype=bf, device=dev)
+    gr = {n: torch.empty_like(d[m]) for n, m in (("dq", "q"), ("dk", "k"), ("dv", "v"), ("dg", "g"),
+                                                 ("db", "b"), ("dw", "w"))}
+    stream = torch.cuda.current_stream(dev)
+    names = ("q", "k", "v", "g", "b", "w")
+
+    def step():
+        gdn.gdn2_fwd_varlen(*(d[n] for n in names), None, o, None, ws, ws.numel(), cu, N, T, H, H, dk, dv,
+                            C, io, gio, stream)
+        gdn.gdn2_bwd_varlen(*(d[n] for n in names), None, d["dO"], None, gr["dq"], gr["dk"], gr["dv"],
+                            gr["dg"], gr["db"], gr["dw"], None, ws, ws.numel(), 1, cu, N, T, H, H, dk, dv,
+                            C, io, gio, stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    if gdn.gdn2_get_device_status(stream) != 0:
+        raise RuntimeError("device status reports an error in the packed workload")
+    steps = max(5, args.steps // 2)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    gd.barrier()
+    torch.cuda.synchronize(dev)
+    start.record(stream)
+    for _ in range(steps):
+        step()
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    gd.barrier()
+    ms = gd.max_over_ranks([start.elapsed_time(end) / steps], dev)[0]
+    alg = T * H * (FWD_BYTES + BWD_BYTES)
+    gbs = alg / (ms * 1e-3) / 1e9
+    out = {"workload": f"fwd+bwd packed {N} sequences (lengths 1..2048, {T} tokens) H{H} d{dk} C{C} bf16",
+           "ms_per_step": ms, "steps": steps, "tokens_per_s": T / (ms * 1e-3),
+           "sequences": N, "longest": max(lens), "shortest": min(lens),
+           "roofline_step": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
+                             "frac": gbs / peak, "alg_bytes_per_step": alg, "peak_source": peak_src}}
+    del ws, d, gr
     torch.cuda.empty_cache()
     return out
 
@@ -419,6 +482,7 @@ def run_ours(args, rank, world, local_rank):
         f"workload{i}": sub_workload(i, args, rank, dev, peak, peak_src) for i in (1, 3)}
     if subs:
         subs["workload2_bf16_gates"] = sub_workload(2, args, rank, dev, peak, peak_src, gates="bf16")
+        subs["packed"] = sub_packed(args, rank, dev, peak, peak_src)
     ms_step, e2e_ms, fwd_ms, bwd_ms = gd.max_over_ranks([ms_step, e2e_ms, fwd_ms, bwd_ms], dev)
     if decode is not None:
         decode["us_per_step"] = gd.max_over_ranks([decode["us_per_step"]], dev)[0]

@@ -62,17 +62,19 @@ def lib() -> ctypes.CDLL:
         L.gdn2_bwd.argtypes = [vp] * 17 + [sz, i] + [i] * 7 + [vp]
         L.gdn2_bwd.restype = i
         L.gdn2_decode_step.argtypes = [vp] * 8 + [i] * 5 + [vp]
-        L.gdn2_fwd_ex.argtypes = [vp] * 10 + [sz] + [i] * 8 + [vp]
+        L.gdn2_workspace_bytes_ex.argtypes = [i] * 10
+        L.gdn2_workspace_bytes_ex.restype = sz
+        L.gdn2_fwd_ex.argtypes = [vp] * 10 + [sz] + [i] * 9 + [vp]
         L.gdn2_fwd_ex.restype = i
-        L.gdn2_bwd_ex.argtypes = [vp] * 17 + [sz, i] + [i] * 8 + [vp]
+        L.gdn2_bwd_ex.argtypes = [vp] * 17 + [sz, i] + [i] * 9 + [vp]
         L.gdn2_bwd_ex.restype = i
-        L.gdn2_decode_step_ex.argtypes = [vp] * 8 + [i] * 6 + [vp]
+        L.gdn2_decode_step_ex.argtypes = [vp] * 8 + [i] * 7 + [vp]
         L.gdn2_decode_step_ex.restype = i
-        L.gdn2_workspace_bytes_varlen.argtypes = [i] * 8
+        L.gdn2_workspace_bytes_varlen.argtypes = [i] * 10
         L.gdn2_workspace_bytes_varlen.restype = sz
-        L.gdn2_fwd_varlen.argtypes = [vp] * 10 + [sz, vp] + [i] * 8 + [vp]
+        L.gdn2_fwd_varlen.argtypes = [vp] * 10 + [sz, vp] + [i] * 9 + [vp]
         L.gdn2_fwd_varlen.restype = i
-        L.gdn2_bwd_varlen.argtypes = [vp] * 17 + [sz, i, vp] + [i] * 8 + [vp]
+        L.gdn2_bwd_varlen.argtypes = [vp] * 17 + [sz, i, vp] + [i] * 9 + [vp]
         L.gdn2_bwd_varlen.restype = i
         L.gdn2_decode_step.restype = i
         L.gdn2_get_device_status.argtypes = [vp]
@@ -164,47 +166,53 @@ def gdn2_bwd(q, k, v, g, b, w, S0, dO, dST, dq, dk, dv, dg, db, dw, dS0, ws, ws_
     _check("gdn2_bwd", rc)
 
 
-def gdn2_fwd_ex(q, k, v, g, b, w, S0, o, ST, ws, ws_bytes, B, T, H, d_k, d_v, chunk, io,
+def gdn2_workspace_bytes_ex(B, T, H, H_v, d_k, d_v, chunk, io, gate_io, for_bwd) -> int:
+    return int(lib().gdn2_workspace_bytes_ex(B, T, H, H_v, d_k, d_v, chunk, io, gate_io, int(for_bwd)))
+
+
+def gdn2_fwd_ex(q, k, v, g, b, w, S0, o, ST, ws, ws_bytes, B, T, H, H_v, d_k, d_v, chunk, io,
                 gate_io, stream=None):
     rc = lib().gdn2_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b), _ptr(w), _ptr(S0), _ptr(o),
-                           _ptr(ST), _ptr(ws), ws_bytes, B, T, H, d_k, d_v, chunk, io, gate_io,
+                           _ptr(ST), _ptr(ws), ws_bytes, B, T, H, H_v, d_k, d_v, chunk, io, gate_io,
                            _stream(stream))
     _check("gdn2_fwd_ex", rc)
 
 
 def gdn2_bwd_ex(q, k, v, g, b, w, S0, dO, dST, dq, dk, dv, dg, db, dw, dS0, ws, ws_bytes,
-                ws_has_fwd, B, T, H, d_k, d_v, chunk, io, gate_io, stream=None):
+                ws_has_fwd, B, T, H, H_v, d_k, d_v, chunk, io, gate_io, stream=None):
     rc = lib().gdn2_bwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b), _ptr(w), _ptr(S0), _ptr(dO),
                            _ptr(dST), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg), _ptr(db), _ptr(dw),
-                           _ptr(dS0), _ptr(ws), ws_bytes, int(ws_has_fwd), B, T, H, d_k, d_v, chunk,
-                           io, gate_io, _stream(stream))
+                           _ptr(dS0), _ptr(ws), ws_bytes, int(ws_has_fwd), B, T, H, H_v, d_k, d_v,
+                           chunk, io, gate_io, _stream(stream))
     _check("gdn2_bwd_ex", rc)
 
 
-def gdn2_decode_step_ex(q, k, v, g, b, w, S, o, N, H, d_k, d_v, io, gate_io, stream=None):
+def gdn2_decode_step_ex(q, k, v, g, b, w, S, o, N, H, H_v, d_k, d_v, io, gate_io, stream=None):
     rc = lib().gdn2_decode_step_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b), _ptr(w), _ptr(S),
-                                   _ptr(o), N, H, d_k, d_v, io, gate_io, _stream(stream))
+                                   _ptr(o), N, H, H_v, d_k, d_v, io, gate_io, _stream(stream))
     _check("gdn2_decode_step_ex", rc)
 
 
-def gdn2_workspace_bytes_varlen(N, T, H, d_k, d_v, chunk, io, for_bwd) -> int:
-    return int(lib().gdn2_workspace_bytes_varlen(N, T, H, d_k, d_v, chunk, io, int(for_bwd)))
+def gdn2_workspace_bytes_varlen(N, T, H, H_v, d_k, d_v, chunk, io, gate_io, for_bwd) -> int:
+    return int(lib().gdn2_workspace_bytes_varlen(N, T, H, H_v, d_k, d_v, chunk, io, gate_io,
+                                                 int(for_bwd)))
 
 
-def gdn2_fwd_varlen(q, k, v, g, b, w, S0, o, ST, ws, ws_bytes, cu_seqlens, N, T, H, d_k, d_v,
+def gdn2_fwd_varlen(q, k, v, g, b, w, S0, o, ST, ws, ws_bytes, cu_seqlens, N, T, H, H_v, d_k, d_v,
                     chunk, io, gate_io, stream=None):
     rc = lib().gdn2_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b), _ptr(w), _ptr(S0),
                                _ptr(o), _ptr(ST), _ptr(ws), ws_bytes, _ptr(cu_seqlens), N, T, H,
-                               d_k, d_v, chunk, io, gate_io, _stream(stream))
+                               H_v, d_k, d_v, chunk, io, gate_io, _stream(stream))
     _check("gdn2_fwd_varlen", rc)
 
 
 def gdn2_bwd_varlen(q, k, v, g, b, w, S0, dO, dST, dq, dk, dv, dg, db, dw, dS0, ws, ws_bytes,
-                    ws_has_fwd, cu_seqlens, N, T, H, d_k, d_v, chunk, io, gate_io, stream=None):
+                    ws_has_fwd, cu_seqlens, N, T, H, H_v, d_k, d_v, chunk, io, gate_io,
+                    stream=None):
     rc = lib().gdn2_bwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b), _ptr(w), _ptr(S0),
                                _ptr(dO), _ptr(dST), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg),
                                _ptr(db), _ptr(dw), _ptr(dS0), _ptr(ws), ws_bytes, int(ws_has_fwd),
-                               _ptr(cu_seqlens), N, T, H, d_k, d_v, chunk, io, gate_io,
+                               _ptr(cu_seqlens), N, T, H, H_v, d_k, d_v, chunk, io, gate_io,
                                _stream(stream))
     _check("gdn2_bwd_varlen", rc)
 
@@ -260,24 +268,32 @@ def check_device_status(stream=None) -> None:
         raise Gdn2Error("device status", st)
 
 
+def _alloc_ws(n: int, fn: str, device) -> torch.Tensor:
+    if n == 0:
+        raise Gdn2Error(fn, 2)
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
 def forward(q, k, v, g, b, w, S0=None, *, chunk: int = 64, want_state: bool = True,
             ws: Optional[torch.Tensor] = None, for_bwd: bool = False, stream=None,
             check: bool = True):
-    """Returns (o, S_T or None, ws).  Shapes: q, k, g, b [B,T,H,dk]; v, w [B,T,H,dv].
-    g, b, w may be bfloat16 (all three) on the tensor-core path.
+    """Returns (o, S_T or None, ws).  Shapes: q, k, g, b [B,T,H,dk]; v, w [B,T,H_v,dv]
+    (H_v a multiple of H: grouped value heads); S0, S_T [B,H_v,dk,dv].  g, b, w
+    may be bfloat16 (all three) on the tensor-core path.
 
     check=True (the default) waits for the stream and raises Gdn2Error if a
     kernel recorded an error during the call; check=False leaves the call
     asynchronous (read the status later with check_device_status)."""
     B, T, H, dk = q.shape
-    dv = v.shape[-1]
-    io = _io_of(q)
+    Hv, dv = v.shape[2], v.shape[3]
+    io, gio = _io_of(q), _gate_io_of(g, b, w)
     if ws is None:
-        ws = workspace(B, T, H, dk, dv, chunk, io, for_bwd, q.device)
-    o = torch.empty(B, T, H, dv, dtype=q.dtype, device=q.device)
-    ST = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device) if want_state else None
-    gdn2_fwd_ex(q, k, v, g, b, w, S0, o, ST, ws, ws.numel(), B, T, H, dk, dv, chunk, io,
-                _gate_io_of(g, b, w), stream)
+        ws = _alloc_ws(gdn2_workspace_bytes_ex(B, T, H, Hv, dk, dv, chunk, io, gio, for_bwd),
+                       "gdn2_workspace_bytes_ex", q.device)
+    o = torch.empty(B, T, Hv, dv, dtype=q.dtype, device=q.device)
+    ST = torch.empty(B, Hv, dk, dv, dtype=torch.float32, device=q.device) if want_state else None
+    gdn2_fwd_ex(q, k, v, g, b, w, S0, o, ST, ws, ws.numel(), B, T, H, Hv, dk, dv, chunk, io, gio,
+                stream)
     if check:
         check_device_status(stream)
     return o, ST, ws
@@ -289,18 +305,19 @@ def backward(q, k, v, g, b, w, S0, dO, dST=None, *, chunk: int = 64,
     """Gradients dq, dk, dv, dg, db, dw, dS0 (None unless want_dS0); dg, db, dw
     take the gates' dtype.  check as in forward()."""
     B, T, H, dk = q.shape
-    dv = v.shape[-1]
-    io = _io_of(q)
+    Hv, dv = v.shape[2], v.shape[3]
+    io, gio = _io_of(q), _gate_io_of(g, b, w)
     if ws is None:
-        ws = workspace(B, T, H, dk, dv, chunk, io, True, q.device)
+        ws = _alloc_ws(gdn2_workspace_bytes_ex(B, T, H, Hv, dk, dv, chunk, io, gio, True),
+                       "gdn2_workspace_bytes_ex", q.device)
         ws_has_fwd = False
     out = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
                dg=torch.empty_like(g), db=torch.empty_like(b), dw=torch.empty_like(w))
-    out["dS0"] = (torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device)
+    out["dS0"] = (torch.empty(B, Hv, dk, dv, dtype=torch.float32, device=q.device)
                   if want_dS0 else None)
     gdn2_bwd_ex(q, k, v, g, b, w, S0, dO, dST, out["dq"], out["dk"], out["dv"], out["dg"],
-                out["db"], out["dw"], out["dS0"], ws, ws.numel(), ws_has_fwd, B, T, H, dk, dv, chunk,
-                io, _gate_io_of(g, b, w), stream)
+                out["db"], out["dw"], out["dS0"], ws, ws.numel(), ws_has_fwd, B, T, H, Hv, dk, dv,
+                chunk, io, gio, stream)
     if check:
         check_device_status(stream)
     return out
@@ -309,22 +326,20 @@ def backward(q, k, v, g, b, w, S0, dO, dST=None, *, chunk: int = 64,
 def forward_varlen(q, k, v, g, b, w, cu_seqlens, S0=None, *, chunk: int = 64,
                    want_state: bool = True, ws: Optional[torch.Tensor] = None,
                    for_bwd: bool = False, stream=None, check: bool = True):
-    """Packed sequences: q, k, g, b [1,T,H,dk]; v, w [1,T,H,dv]; cu_seqlens
-    int32 [N+1] on the device; S0 [N,H,dk,dv] or None.  Returns (o, S_T [N,...]
-    or None, ws)."""
+    """Packed sequences: q, k, g, b [1,T,H,dk]; v, w [1,T,H_v,dv]; cu_seqlens
+    int32 [N+1] on the device; S0 [N,H_v,dk,dv] or None.  Returns (o, S_T
+    [N,...] or None, ws)."""
     _, T, H, dk = q.shape
-    dv = v.shape[-1]
+    Hv, dv = v.shape[2], v.shape[3]
     N = cu_seqlens.numel() - 1
-    io = _io_of(q)
+    io, gio = _io_of(q), _gate_io_of(g, b, w)
     if ws is None:
-        n = gdn2_workspace_bytes_varlen(N, T, H, dk, dv, chunk, io, for_bwd)
-        if n == 0:
-            raise Gdn2Error("gdn2_workspace_bytes_varlen", 2)
-        ws = torch.empty(n, dtype=torch.uint8, device=q.device)
-    o = torch.empty(1, T, H, dv, dtype=q.dtype, device=q.device)
-    ST = torch.empty(N, H, dk, dv, dtype=torch.float32, device=q.device) if want_state else None
-    gdn2_fwd_varlen(q, k, v, g, b, w, S0, o, ST, ws, ws.numel(), cu_seqlens, N, T, H, dk, dv, chunk,
-                    io, _gate_io_of(g, b, w), stream)
+        ws = _alloc_ws(gdn2_workspace_bytes_varlen(N, T, H, Hv, dk, dv, chunk, io, gio, for_bwd),
+                       "gdn2_workspace_bytes_varlen", q.device)
+    o = torch.empty(1, T, Hv, dv, dtype=q.dtype, device=q.device)
+    ST = torch.empty(N, Hv, dk, dv, dtype=torch.float32, device=q.device) if want_state else None
+    gdn2_fwd_varlen(q, k, v, g, b, w, S0, o, ST, ws, ws.numel(), cu_seqlens, N, T, H, Hv, dk, dv,
+                    chunk, io, gio, stream)
     if check:
         check_device_status(stream)
     return o, ST, ws
@@ -335,34 +350,32 @@ def backward_varlen(q, k, v, g, b, w, cu_seqlens, S0, dO, dST=None, *, chunk: in
                     want_dS0: bool = True, stream=None, check: bool = True) -> Dict[str, torch.Tensor]:
     """Gradients of forward_varlen: dq, dk, dv, dg, db, dw and dS0 [N,...]."""
     _, T, H, dk = q.shape
-    dv = v.shape[-1]
+    Hv, dv = v.shape[2], v.shape[3]
     N = cu_seqlens.numel() - 1
-    io = _io_of(q)
+    io, gio = _io_of(q), _gate_io_of(g, b, w)
     if ws is None:
-        n = gdn2_workspace_bytes_varlen(N, T, H, dk, dv, chunk, io, True)
-        if n == 0:
-            raise Gdn2Error("gdn2_workspace_bytes_varlen", 2)
-        ws = torch.empty(n, dtype=torch.uint8, device=q.device)
+        ws = _alloc_ws(gdn2_workspace_bytes_varlen(N, T, H, Hv, dk, dv, chunk, io, gio, True),
+                       "gdn2_workspace_bytes_varlen", q.device)
         ws_has_fwd = False
     out = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
                dg=torch.empty_like(g), db=torch.empty_like(b), dw=torch.empty_like(w))
-    out["dS0"] = (torch.empty(N, H, dk, dv, dtype=torch.float32, device=q.device)
+    out["dS0"] = (torch.empty(N, Hv, dk, dv, dtype=torch.float32, device=q.device)
                   if want_dS0 else None)
     gdn2_bwd_varlen(q, k, v, g, b, w, S0, dO, dST, out["dq"], out["dk"], out["dv"], out["dg"],
                     out["db"], out["dw"], out["dS0"], ws, ws.numel(), ws_has_fwd, cu_seqlens, N, T,
-                    H, dk, dv, chunk, io, _gate_io_of(g, b, w), stream)
+                    H, Hv, dk, dv, chunk, io, gio, stream)
     if check:
         check_device_status(stream)
     return out
 
 
 def decode_step(q, k, v, g, b, w, S, o=None, stream=None):
-    """One token for N sequences: q, k, g, b [N,H,dk]; v, w [N,H,dv]; S [N,H,dk,dv]
-    float32, updated in place.  Returns o [N,H,dv]."""
+    """One token for N sequences: q, k, g, b [N,H,dk]; v, w [N,H_v,dv]; S
+    [N,H_v,dk,dv] float32, updated in place.  Returns o [N,H_v,dv]."""
     N, H, dk = q.shape
-    dv = v.shape[-1]
+    Hv, dv = v.shape[1], v.shape[2]
     if o is None:
-        o = torch.empty(N, H, dv, dtype=q.dtype, device=q.device)
-    gdn2_decode_step_ex(q, k, v, g, b, w, S, o, N, H, dk, dv, _io_of(q), _gate_io_of(g, b, w),
+        o = torch.empty(N, Hv, dv, dtype=q.dtype, device=q.device)
+    gdn2_decode_step_ex(q, k, v, g, b, w, S, o, N, H, Hv, dk, dv, _io_of(q), _gate_io_of(g, b, w),
                         stream)
     return o

@@ -26,7 +26,7 @@ cudaError_t simt_bwd_launch(const void *, const void *, const void *, const floa
                             const void *, const float *, void *, void *, void *, float *, float *,
                             float *, float *, void *, const Dims &, cudaStream_t);
 cudaError_t decode_launch(const void *, const void *, const void *, const void *, const void *,
-                          const void *, float *, void *, int, int, int, int, gdn2_io, gdn2_io,
+                          const void *, float *, void *, int, int, int, int, int, gdn2_io, gdn2_io,
                           cudaStream_t);
 cudaError_t tc_fwd_launch(const void *, const void *, const void *, const void *, const void *,
                           const void *, const float *, void *, float *, void *, int,
@@ -75,7 +75,8 @@ static unsigned long long g_kind_count[K_KINDS];
 static double g_kind_ms[K_KINDS];
 static const char *const g_kind_names[K_KINDS] = {
     "simt_chunk_prep", "simt_state_fwd", "simt_out_fwd", "simt_state_bwd", "simt_chunk_bwd_a",
-    "simt_chunk_bwd_b", "decode_step", "tc_prep", "tc_fwd", "tc_bwd_state", "tc_bwd_grad", "seq_table"};
+    "simt_chunk_bwd_b", "decode_step", "tc_prep", "tc_fwd", "tc_bwd_state", "tc_bwd_grad", "seq_table",
+    "permute_state"};
 
 void launch_begin(int kind, cudaStream_t s) {
     g_launches.fetch_add(1, std::memory_order_relaxed);
@@ -175,86 +176,42 @@ static gdn2_status check_gate_io(const Dims &d, gdn2_io io, gdn2_io gate_io) {
     return GDN2_OK;
 }
 
-gdn2_status gdn2_fwd_ex(const void *q, const void *k, const void *v, const void *g, const void *b,
-                        const void *w, const float *S0, void *o, float *ST, void *ws,
-                        size_t ws_bytes, int B, int T, int H, int d_k, int d_v, int chunk,
-                        gdn2_io io, gdn2_io gate_io, gdn2_stream_t stream) {
-    gdn2_status st = check_dims(B, T, H, d_k, d_v, chunk, io);
-    if (st != GDN2_OK) return st;
-    Dims d = make_dims(B, T, H, d_k, d_v, chunk);
-    if ((st = check_gate_io(d, io, gate_io)) != GDN2_OK) return st;
-    st = check_ptrs({q, k, v, g, b, w, o}, {S0, ST});
-    if (st != GDN2_OK) return st;
-    if (!ws || !aligned16(ws) || ws_bytes < ws_bytes_for(d, io, 0)) return GDN2_ERR_WORKSPACE;
-    d.gb = gate_io == GDN2_IO_BF16;
-    if (use_tc(d, io)) {
-        unsigned int *status = status_word();
-        if (!status) return GDN2_ERR_CUDA;
-        const int keep = ws_bytes >= ws_bytes_for(d, io, 1);
-        return cuda_status(tc_fwd_launch(q, k, v, g, b, w, S0, o, ST, ws, keep, status, d,
-                                         (cudaStream_t)stream));
-    }
-    return cuda_status(run_forward(q, k, v, static_cast<const float *>(g), static_cast<const float *>(b),
-                                   static_cast<const float *>(w), S0, o, ST, ws, d, io,
-                                   (cudaStream_t)stream));
+// ------------------------------------------------------ grouped value heads
+// H_v value heads over H key heads, G = H_v / H consecutive value heads per
+// key head.  Value head h G + j reads q, k, g, b of key head h, so the G
+// states of a key head evolve as one state of G d_v columns: the kernels run
+// that wide problem (d_v' = G d_v) on v, w, o, dO, dv, dw unchanged in memory
+// ([.., H_v, d_v] is [.., H, G d_v]).  Only the states are laid out per value
+// head, [S, H_v, d_k, d_v]; they pass through the wide layout [S, H, d_k, G d_v]
+// in two workspace buffers.
+static int value_groups(int H, int H_v) {
+    if (H_v == 0 || H_v == H) return 1;
+    if (H_v < H || H_v % H != 0) return 0;
+    return H_v / H;
 }
 
-gdn2_status gdn2_fwd(const void *q, const void *k, const void *v, const float *g, const float *b,
-                     const float *w, const float *S0, void *o, float *ST, void *ws,
-                     size_t ws_bytes, int B, int T, int H, int d_k, int d_v, int chunk,
-                     gdn2_io io, gdn2_stream_t stream) {
-    return gdn2_fwd_ex(q, k, v, g, b, w, S0, o, ST, ws, ws_bytes, B, T, H, d_k, d_v, chunk, io,
-                       GDN2_IO_F32, stream);
-}
-
-gdn2_status gdn2_bwd_ex(const void *q, const void *k, const void *v, const void *g, const void *b,
-                        const void *w, const float *S0, const void *dO, const float *dST, void *dq,
-                        void *dk, void *dv, void *dg, void *db, void *dw, float *dS0, void *ws,
-                        size_t ws_bytes, int ws_has_fwd, int B, int T, int H, int d_k, int d_v,
-                        int chunk, gdn2_io io, gdn2_io gate_io, gdn2_stream_t stream) {
-    gdn2_status st = check_dims(B, T, H, d_k, d_v, chunk, io);
-    if (st != GDN2_OK) return st;
-    Dims d = make_dims(B, T, H, d_k, d_v, chunk);
-    if ((st = check_gate_io(d, io, gate_io)) != GDN2_OK) return st;
-    st = check_ptrs({q, k, v, g, b, w, dO, dq, dk, dv, dg, db, dw}, {S0, dST, dS0});
-    if (st != GDN2_OK) return st;
-    if (!ws || !aligned16(ws) || ws_bytes < ws_bytes_for(d, io, 1)) return GDN2_ERR_WORKSPACE;
-    d.gb = gate_io == GDN2_IO_BF16;
-    cudaStream_t s = (cudaStream_t)stream;
-    cudaError_t e;
-    if (use_tc(d, io)) {
-        unsigned int *status = status_word();
-        if (!status) return GDN2_ERR_CUDA;
-        if (!ws_has_fwd) {
-            e = tc_fwd_launch(q, k, v, g, b, w, S0, nullptr, nullptr, ws, 1, status, d, s);
-            if (e != cudaSuccess) return GDN2_ERR_CUDA;
-        }
-        return cuda_status(tc_bwd_launch(q, k, v, g, b, w, dO, dST, dq, dk, dv, dg, db, dw, dS0, ws,
-                                         status, d, s));
+// state layouts: per value head [S][H G][dk][dvh]  <->  wide [S][H][dk][G dvh]
+static __global__ void permute_state_kernel(const float *src, float *dst, long long total, int G, int dk,
+                                            int dvh, int to_wide) {
+    const int dvw = G * dvh;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+         i += (long long)gridDim.x * blockDim.x) {
+        const int col = (int)(i % dvw), key = (int)((i / dvw) % dk);
+        const long long sh = i / ((long long)dvw * dk);  // s H + h
+        const long long j = ((sh * G + col / dvh) * dk + key) * dvh + col % dvh;
+        if (to_wide) dst[i] = src[j];
+        else dst[j] = src[i];
     }
-    const float *gf = static_cast<const float *>(g), *bf = static_cast<const float *>(b),
-                *wf = static_cast<const float *>(w);
-    float *dgf = static_cast<float *>(dg), *dbf = static_cast<float *>(db), *dwf = static_cast<float *>(dw);
-    if (!ws_has_fwd) {
-        e = run_forward(q, k, v, gf, bf, wf, S0, nullptr, nullptr, ws, d, io, s);
-        if (e != cudaSuccess) return GDN2_ERR_CUDA;
-    }
-    if (io == GDN2_IO_BF16)
-        e = simt_bwd_launch<__nv_bfloat16>(q, k, v, bf, wf, dO, dST, dq, dk, dv, dgf, dbf, dwf, dS0, ws,
-                                           d, s);
-    else
-        e = simt_bwd_launch<float>(q, k, v, bf, wf, dO, dST, dq, dk, dv, dgf, dbf, dwf, dS0, ws, d, s);
-    return cuda_status(e);
 }
-
-gdn2_status gdn2_bwd(const void *q, const void *k, const void *v, const float *g, const float *b,
-                     const float *w, const float *S0, const void *dO, const float *dST, void *dq,
-                     void *dk, void *dv, float *dg, float *db, float *dw, float *dS0, void *ws,
-                     size_t ws_bytes, int ws_has_fwd, int B, int T, int H, int d_k, int d_v,
-                     int chunk, gdn2_io io, gdn2_stream_t stream) {
-    return gdn2_bwd_ex(q, k, v, g, b, w, S0, dO, dST, dq, dk, dv, dg, db, dw, dS0, ws, ws_bytes,
-                       ws_has_fwd, B, T, H, d_k, d_v, chunk, io, GDN2_IO_F32, stream);
+static cudaError_t permute_state(const float *src, float *dst, const Dims &d, int G, int to_wide, cudaStream_t s) {
+    const long long total = (long long)num_seqs(d) * d.H * d.dk * d.dv;
+    const int blocks = (int)((total + 255) / 256 < 4 * sm_count() ? (total + 255) / 256 : 4 * sm_count());
+    launch_begin(K_PERMUTE_STATE, s);
+    permute_state_kernel<<<blocks, 256, 0, s>>>(src, dst, total, G, d.dk, d.dv / G, to_wide);
+    launch_end(K_PERMUTE_STATE, s);
+    return cudaGetLastError();
 }
+static size_t state_bytes(const Dims &d) { return align256((size_t)num_seqs(d) * d.H * d.dk * d.dv * sizeof(float)); }
 
 // ---------------------------------------------------------- packed sequences
 // Chunk offsets co[0..N] of the sequences cu[0..N] (chunk C): one block,
@@ -312,112 +269,256 @@ static __global__ void __launch_bounds__(1024) seq_table_kernel(const int *cu, i
     }
 }
 
-// a packed call: B = 1 row of T tokens holding N sequences, the chunk bound
-// ceil(T / C) + N, and the chunk table at the end of the workspace
-static Dims varlen_dims(int N, int T, int H, int dk, int dv, int chunk) {
-    Dims d = make_dims(1, T, H, dk, dv, chunk);
-    d.NC = (T + chunk - 1) / chunk + N;
-    d.N = N;
-    return d;
-}
-// the chunk table follows the records (a forward-only workspace) or the whole
-// layout (a workspace that keeps the forward for the backward)
-static size_t varlen_table_at(const Dims &d, int for_bwd) {
-    const TcWs t = tc_ws_layout(d);
-    return for_bwd ? t.bwd_end : t.rec_end;
-}
-static size_t varlen_ws_bytes(const Dims &d, int for_bwd) {
-    return varlen_table_at(d, for_bwd) + align256((size_t)(d.N + 1) * sizeof(int));
-}
-static gdn2_status check_varlen(int N, int T, int H, int dk, int dv, int chunk, gdn2_io io, gdn2_io gate_io,
-                                const int *cu) {
-    if (N < 1 || !cu || !aligned16(cu)) return GDN2_ERR_INVALID_ARG;
-    gdn2_status st = check_dims(1, T, H, dk, dv, chunk, io);
+// ------------------------------------------------------------ one call
+// The problem after the host checks: the (wide) sizes, the path, and the
+// workspace regions that follow the path's own layout: the packed
+// sequences' chunk table, then two wide state buffers when G > 1.
+struct Call {
+    Dims d;
+    gdn2_io io;
+    int G;
+    int for_bwd;
+    size_t table_at, states_at, total;
+};
+
+// packed: N sequences of the table cu (which only a launch reads; sizing
+// passes none)
+static gdn2_status plan_call(Call &c, int B, int T, int H, int H_v, int dk, int dv, int chunk, gdn2_io io,
+                             gdn2_io gate_io, bool packed, int N, const int *cu, int for_bwd) {
+    c.G = value_groups(H, H_v);
+    if (c.G == 0 || H < 1) return GDN2_ERR_INVALID_ARG;
+    if (c.G > 1 && !supported_d(dv)) return GDN2_ERR_UNSUPPORTED;
+    const int dvw = c.G * dv;
+    gdn2_status st = check_dims(packed ? 1 : B, T, H, dk, dvw, chunk, io);
     if (st != GDN2_OK) return st;
-    if (gate_io != GDN2_IO_F32 && gate_io != GDN2_IO_BF16) return GDN2_ERR_INVALID_ARG;
-    if (!use_tc(make_dims(1, T, H, dk, dv, chunk), io)) return GDN2_ERR_UNSUPPORTED;
-    if (N > 65535 || (long long)H * ((T + chunk - 1) / chunk + N) > 0x7fffffffLL) return GDN2_ERR_UNSUPPORTED;
+    c.io = io;
+    c.for_bwd = for_bwd;
+    c.d = make_dims(packed ? 1 : B, T, H, dk, dvw, chunk);
+    if ((st = check_gate_io(c.d, io, gate_io)) != GDN2_OK) return st;
+    c.d.gb = gate_io == GDN2_IO_BF16;
+    size_t o;
+    if (packed) {
+        if (N < 1 || ((uintptr_t)cu & 3u) != 0) return GDN2_ERR_INVALID_ARG;
+        if (!use_tc(c.d, io)) return GDN2_ERR_UNSUPPORTED;
+        if (N > 65535 || (long long)H * ((T + chunk - 1) / chunk + N) > 0x7fffffffLL) return GDN2_ERR_UNSUPPORTED;
+        c.d.NC = (T + chunk - 1) / chunk + N;  // bounds the chunks of N sequences over T tokens
+        c.d.N = N;
+        c.d.cu = cu;
+        const TcWs t = tc_ws_layout(c.d);
+        c.table_at = for_bwd ? t.bwd_end : t.rec_end;
+        o = c.table_at + align256((size_t)(N + 1) * sizeof(int));
+    } else {
+        c.table_at = 0;
+        o = ws_bytes_for(c.d, io, for_bwd);
+    }
+    c.states_at = align256(o);
+    c.total = c.G > 1 ? c.states_at + 2 * state_bytes(c.d) : o;
     return GDN2_OK;
 }
-static cudaError_t seq_table_launch(Dims &d, void *ws, int for_bwd, unsigned int *status, cudaStream_t s) {
-    int *co = reinterpret_cast<int *>(static_cast<char *>(ws) + varlen_table_at(d, for_bwd));
+
+static cudaError_t seq_table_launch(Call &c, void *ws, unsigned int *status, cudaStream_t s) {
+    if (c.d.N == 0) return cudaSuccess;
+    int *co = reinterpret_cast<int *>(static_cast<char *>(ws) + c.table_at);
     launch_begin(K_SEQ_TABLE, s);
-    seq_table_kernel<<<1, 1024, 0, s>>>(d.cu, d.N, d.T, d.C, co, status);
+    seq_table_kernel<<<1, 1024, 0, s>>>(c.d.cu, c.d.N, c.d.T, c.d.C, co, status);
     launch_end(K_SEQ_TABLE, s);
-    d.co = co;
+    c.d.co = co;
     return cudaGetLastError();
 }
+static float *state_buf(const Call &c, void *ws, int i) {
+    return reinterpret_cast<float *>(static_cast<char *>(ws) + c.states_at + i * state_bytes(c.d));
+}
 
-size_t gdn2_workspace_bytes_varlen(int N, int T, int H, int d_k, int d_v, int chunk, gdn2_io io, int for_bwd) {
-    if (N < 1 || check_dims(1, T, H, d_k, d_v, chunk, io) != GDN2_OK) return 0;
-    if (!use_tc(make_dims(1, T, H, d_k, d_v, chunk), io)) return 0;
-    return varlen_ws_bytes(varlen_dims(N, T, H, d_k, d_v, chunk), for_bwd);
+static gdn2_status fwd_call(Call &c, const void *q, const void *k, const void *v, const void *g,
+                            const void *b, const void *w, const float *S0, void *o, float *ST, void *ws,
+                            size_t ws_bytes, gdn2_stream_t stream) {
+    gdn2_status st = check_ptrs({q, k, v, g, b, w, o}, {S0, ST});
+    if (st != GDN2_OK) return st;
+    if (!ws || !aligned16(ws) || ws_bytes < c.total) return GDN2_ERR_WORKSPACE;
+    cudaStream_t s = (cudaStream_t)stream;
+    // keep the forward for the backward when the workspace is the backward's
+    Call full = c;
+    if (!c.for_bwd) {
+        Call cb;
+        if (plan_call(cb, c.d.B, c.d.T, c.d.H, c.d.H * c.G, c.d.dk, c.d.dv / c.G, c.d.C, c.io,
+                      c.d.gb ? GDN2_IO_BF16 : GDN2_IO_F32, c.d.N > 0, c.d.N, c.d.cu, 1) == GDN2_OK &&
+            ws_bytes >= cb.total)
+            full = cb;
+    }
+    const int keep = full.for_bwd;
+    const float *wS0 = S0;
+    float *wST = ST;
+    cudaError_t e = cudaSuccess;
+    if (full.G > 1) {
+        if (S0) {
+            wS0 = state_buf(full, ws, 0);
+            if ((e = permute_state(S0, state_buf(full, ws, 0), full.d, full.G, 1, s)) != cudaSuccess) return GDN2_ERR_CUDA;
+        }
+        if (ST) wST = state_buf(full, ws, 1);
+    }
+    if (use_tc(full.d, full.io)) {
+        unsigned int *status = status_word();
+        if (!status) return GDN2_ERR_CUDA;
+        if ((e = seq_table_launch(full, ws, status, s)) != cudaSuccess) return GDN2_ERR_CUDA;
+        e = tc_fwd_launch(q, k, v, g, b, w, wS0, o, wST, ws, keep, status, full.d, s);
+    } else {
+        e = run_forward(q, k, v, static_cast<const float *>(g), static_cast<const float *>(b),
+                        static_cast<const float *>(w), wS0, o, wST, ws, full.d, full.io, s);
+    }
+    if (e != cudaSuccess) return GDN2_ERR_CUDA;
+    if (full.G > 1 && ST) e = permute_state(wST, ST, full.d, full.G, 0, s);
+    return cuda_status(e);
+}
+
+static gdn2_status bwd_call(Call &c, const void *q, const void *k, const void *v, const void *g,
+                            const void *b, const void *w, const float *S0, const void *dO, const float *dST,
+                            void *dq, void *dk, void *dv, void *dg, void *db, void *dw, float *dS0, void *ws,
+                            size_t ws_bytes, int ws_has_fwd, gdn2_stream_t stream) {
+    gdn2_status st = check_ptrs({q, k, v, g, b, w, dO, dq, dk, dv, dg, db, dw}, {S0, dST, dS0});
+    if (st != GDN2_OK) return st;
+    if (!ws || !aligned16(ws) || ws_bytes < c.total) return GDN2_ERR_WORKSPACE;
+    cudaStream_t s = (cudaStream_t)stream;
+    const float *wS0 = S0, *wdST = dST;
+    float *wdS0 = dS0;
+    cudaError_t e = cudaSuccess;
+    if (c.G > 1) {
+        // S0 (read by a recomputed forward) and then dS0 share buffer 0: the
+        // stream runs the forward's reads before the backward's writes
+        if (S0 && !ws_has_fwd) {
+            wS0 = state_buf(c, ws, 0);
+            if ((e = permute_state(S0, state_buf(c, ws, 0), c.d, c.G, 1, s)) != cudaSuccess) return GDN2_ERR_CUDA;
+        }
+        if (dST) {
+            wdST = state_buf(c, ws, 1);
+            if ((e = permute_state(dST, state_buf(c, ws, 1), c.d, c.G, 1, s)) != cudaSuccess) return GDN2_ERR_CUDA;
+        }
+        if (dS0) wdS0 = state_buf(c, ws, 0);
+    }
+    if (use_tc(c.d, c.io)) {
+        unsigned int *status = status_word();
+        if (!status) return GDN2_ERR_CUDA;
+        if ((e = seq_table_launch(c, ws, status, s)) != cudaSuccess) return GDN2_ERR_CUDA;
+        if (!ws_has_fwd) {
+            e = tc_fwd_launch(q, k, v, g, b, w, wS0, nullptr, nullptr, ws, 1, status, c.d, s);
+            if (e != cudaSuccess) return GDN2_ERR_CUDA;
+        }
+        e = tc_bwd_launch(q, k, v, g, b, w, dO, wdST, dq, dk, dv, dg, db, dw, wdS0, ws, status, c.d, s);
+    } else {
+        const float *gf = static_cast<const float *>(g), *bf = static_cast<const float *>(b),
+                    *wf = static_cast<const float *>(w);
+        float *dgf = static_cast<float *>(dg), *dbf = static_cast<float *>(db), *dwf = static_cast<float *>(dw);
+        if (!ws_has_fwd) {
+            e = run_forward(q, k, v, gf, bf, wf, wS0, nullptr, nullptr, ws, c.d, c.io, s);
+            if (e != cudaSuccess) return GDN2_ERR_CUDA;
+        }
+        if (c.io == GDN2_IO_BF16)
+            e = simt_bwd_launch<__nv_bfloat16>(q, k, v, bf, wf, dO, wdST, dq, dk, dv, dgf, dbf, dwf, wdS0, ws,
+                                               c.d, s);
+        else
+            e = simt_bwd_launch<float>(q, k, v, bf, wf, dO, wdST, dq, dk, dv, dgf, dbf, dwf, wdS0, ws, c.d, s);
+    }
+    if (e != cudaSuccess) return GDN2_ERR_CUDA;
+    if (c.G > 1 && dS0) e = permute_state(wdS0, dS0, c.d, c.G, 0, s);
+    return cuda_status(e);
+}
+
+size_t gdn2_workspace_bytes_ex(int B, int T, int H, int H_v, int d_k, int d_v, int chunk, gdn2_io io,
+                               gdn2_io gate_io, int for_bwd) {
+    Call c;
+    if (plan_call(c, B, T, H, H_v, d_k, d_v, chunk, io, gate_io, false, 0, nullptr, for_bwd) != GDN2_OK) return 0;
+    return c.total;
+}
+
+gdn2_status gdn2_fwd_ex(const void *q, const void *k, const void *v, const void *g, const void *b,
+                        const void *w, const float *S0, void *o, float *ST, void *ws,
+                        size_t ws_bytes, int B, int T, int H, int H_v, int d_k, int d_v, int chunk,
+                        gdn2_io io, gdn2_io gate_io, gdn2_stream_t stream) {
+    Call c;
+    gdn2_status st = plan_call(c, B, T, H, H_v, d_k, d_v, chunk, io, gate_io, false, 0, nullptr, 0);
+    if (st != GDN2_OK) return st;
+    return fwd_call(c, q, k, v, g, b, w, S0, o, ST, ws, ws_bytes, stream);
+}
+
+gdn2_status gdn2_fwd(const void *q, const void *k, const void *v, const float *g, const float *b,
+                     const float *w, const float *S0, void *o, float *ST, void *ws,
+                     size_t ws_bytes, int B, int T, int H, int d_k, int d_v, int chunk,
+                     gdn2_io io, gdn2_stream_t stream) {
+    return gdn2_fwd_ex(q, k, v, g, b, w, S0, o, ST, ws, ws_bytes, B, T, H, H, d_k, d_v, chunk, io,
+                       GDN2_IO_F32, stream);
+}
+
+gdn2_status gdn2_bwd_ex(const void *q, const void *k, const void *v, const void *g, const void *b,
+                        const void *w, const float *S0, const void *dO, const float *dST, void *dq,
+                        void *dk, void *dv, void *dg, void *db, void *dw, float *dS0, void *ws,
+                        size_t ws_bytes, int ws_has_fwd, int B, int T, int H, int H_v, int d_k, int d_v,
+                        int chunk, gdn2_io io, gdn2_io gate_io, gdn2_stream_t stream) {
+    Call c;
+    gdn2_status st = plan_call(c, B, T, H, H_v, d_k, d_v, chunk, io, gate_io, false, 0, nullptr, 1);
+    if (st != GDN2_OK) return st;
+    return bwd_call(c, q, k, v, g, b, w, S0, dO, dST, dq, dk, dv, dg, db, dw, dS0, ws, ws_bytes, ws_has_fwd,
+                    stream);
+}
+
+gdn2_status gdn2_bwd(const void *q, const void *k, const void *v, const float *g, const float *b,
+                     const float *w, const float *S0, const void *dO, const float *dST, void *dq,
+                     void *dk, void *dv, float *dg, float *db, float *dw, float *dS0, void *ws,
+                     size_t ws_bytes, int ws_has_fwd, int B, int T, int H, int d_k, int d_v,
+                     int chunk, gdn2_io io, gdn2_stream_t stream) {
+    return gdn2_bwd_ex(q, k, v, g, b, w, S0, dO, dST, dq, dk, dv, dg, db, dw, dS0, ws, ws_bytes,
+                       ws_has_fwd, B, T, H, H, d_k, d_v, chunk, io, GDN2_IO_F32, stream);
+}
+
+size_t gdn2_workspace_bytes_varlen(int N, int T, int H, int H_v, int d_k, int d_v, int chunk, gdn2_io io,
+                                   gdn2_io gate_io, int for_bwd) {
+    Call c;
+    if (plan_call(c, 1, T, H, H_v, d_k, d_v, chunk, io, gate_io, true, N, nullptr, for_bwd) != GDN2_OK) return 0;
+    return c.total;
 }
 
 gdn2_status gdn2_fwd_varlen(const void *q, const void *k, const void *v, const void *g, const void *b,
                             const void *w, const float *S0, void *o, float *ST, void *ws, size_t ws_bytes,
-                            const int *cu_seqlens, int N, int T, int H, int d_k, int d_v, int chunk,
+                            const int *cu_seqlens, int N, int T, int H, int H_v, int d_k, int d_v, int chunk,
                             gdn2_io io, gdn2_io gate_io, gdn2_stream_t stream) {
-    gdn2_status st = check_varlen(N, T, H, d_k, d_v, chunk, io, gate_io, cu_seqlens);
+    if (!cu_seqlens) return GDN2_ERR_INVALID_ARG;
+    Call c;
+    gdn2_status st = plan_call(c, 1, T, H, H_v, d_k, d_v, chunk, io, gate_io, true, N, cu_seqlens, 0);
     if (st != GDN2_OK) return st;
-    st = check_ptrs({q, k, v, g, b, w, o}, {S0, ST});
-    if (st != GDN2_OK) return st;
-    Dims d = varlen_dims(N, T, H, d_k, d_v, chunk);
-    d.cu = cu_seqlens;
-    d.gb = gate_io == GDN2_IO_BF16;
-    if (!ws || !aligned16(ws) || ws_bytes < varlen_ws_bytes(d, 0)) return GDN2_ERR_WORKSPACE;
-    unsigned int *status = status_word();
-    if (!status) return GDN2_ERR_CUDA;
-    cudaStream_t s = (cudaStream_t)stream;
-    const int keep = ws_bytes >= varlen_ws_bytes(d, 1);
-    cudaError_t e = seq_table_launch(d, ws, keep, status, s);
-    if (e != cudaSuccess) return GDN2_ERR_CUDA;
-    return cuda_status(tc_fwd_launch(q, k, v, g, b, w, S0, o, ST, ws, keep, status, d, s));
+    return fwd_call(c, q, k, v, g, b, w, S0, o, ST, ws, ws_bytes, stream);
 }
 
 gdn2_status gdn2_bwd_varlen(const void *q, const void *k, const void *v, const void *g, const void *b,
                             const void *w, const float *S0, const void *dO, const float *dST, void *dq,
                             void *dk, void *dv, void *dg, void *db, void *dw, float *dS0, void *ws,
                             size_t ws_bytes, int ws_has_fwd, const int *cu_seqlens, int N, int T, int H,
-                            int d_k, int d_v, int chunk, gdn2_io io, gdn2_io gate_io, gdn2_stream_t stream) {
-    gdn2_status st = check_varlen(N, T, H, d_k, d_v, chunk, io, gate_io, cu_seqlens);
+                            int H_v, int d_k, int d_v, int chunk, gdn2_io io, gdn2_io gate_io,
+                            gdn2_stream_t stream) {
+    if (!cu_seqlens) return GDN2_ERR_INVALID_ARG;
+    Call c;
+    gdn2_status st = plan_call(c, 1, T, H, H_v, d_k, d_v, chunk, io, gate_io, true, N, cu_seqlens, 1);
     if (st != GDN2_OK) return st;
-    st = check_ptrs({q, k, v, g, b, w, dO, dq, dk, dv, dg, db, dw}, {S0, dST, dS0});
-    if (st != GDN2_OK) return st;
-    Dims d = varlen_dims(N, T, H, d_k, d_v, chunk);
-    d.cu = cu_seqlens;
-    d.gb = gate_io == GDN2_IO_BF16;
-    if (!ws || !aligned16(ws) || ws_bytes < varlen_ws_bytes(d, 1)) return GDN2_ERR_WORKSPACE;
-    unsigned int *status = status_word();
-    if (!status) return GDN2_ERR_CUDA;
-    cudaStream_t s = (cudaStream_t)stream;
-    cudaError_t e = seq_table_launch(d, ws, 1, status, s);
-    if (e != cudaSuccess) return GDN2_ERR_CUDA;
-    if (!ws_has_fwd) {
-        e = tc_fwd_launch(q, k, v, g, b, w, S0, nullptr, nullptr, ws, 1, status, d, s);
-        if (e != cudaSuccess) return GDN2_ERR_CUDA;
-    }
-    return cuda_status(tc_bwd_launch(q, k, v, g, b, w, dO, dST, dq, dk, dv, dg, db, dw, dS0, ws, status,
-                                     d, s));
+    return bwd_call(c, q, k, v, g, b, w, S0, dO, dST, dq, dk, dv, dg, db, dw, dS0, ws, ws_bytes, ws_has_fwd,
+                    stream);
 }
 
 gdn2_status gdn2_decode_step_ex(const void *q, const void *k, const void *v, const void *g,
-                                const void *b, const void *w, float *S, void *o, int N, int H,
+                                const void *b, const void *w, float *S, void *o, int N, int H, int H_v,
                                 int d_k, int d_v, gdn2_io io, gdn2_io gate_io, gdn2_stream_t stream) {
     if (N < 1 || H < 1 || (io != GDN2_IO_F32 && io != GDN2_IO_BF16)) return GDN2_ERR_INVALID_ARG;
     if (gate_io != GDN2_IO_F32 && gate_io != GDN2_IO_BF16) return GDN2_ERR_INVALID_ARG;
+    const int G = value_groups(H, H_v);
+    if (G == 0) return GDN2_ERR_INVALID_ARG;
     if (!supported_d(d_k) || !supported_d(d_v)) return GDN2_ERR_UNSUPPORTED;
-    if ((long long)N * H > 0x7fffffffLL) return GDN2_ERR_UNSUPPORTED;
+    if ((long long)N * H * G > 0x7fffffffLL) return GDN2_ERR_UNSUPPORTED;
     gdn2_status st = check_ptrs({q, k, v, g, b, w, S, o}, {});
     if (st != GDN2_OK) return st;
-    return cuda_status(decode_launch(q, k, v, g, b, w, S, o, N, H, d_k, d_v, io, gate_io,
+    return cuda_status(decode_launch(q, k, v, g, b, w, S, o, N, H, G, d_k, d_v, io, gate_io,
                                      (cudaStream_t)stream));
 }
 
 gdn2_status gdn2_decode_step(const void *q, const void *k, const void *v, const float *g,
                              const float *b, const float *w, float *S, void *o, int N, int H,
                              int d_k, int d_v, gdn2_io io, gdn2_stream_t stream) {
-    return gdn2_decode_step_ex(q, k, v, g, b, w, S, o, N, H, d_k, d_v, io, GDN2_IO_F32, stream);
+    return gdn2_decode_step_ex(q, k, v, g, b, w, S, o, N, H, H, d_k, d_v, io, GDN2_IO_F32, stream);
 }
 
 // One block, one waiting thread: an mbarrier that no copy or product will

@@ -36,7 +36,7 @@ __device__ __forceinline__ Seq seq_of(const Dims &d, int n) {
     return Seq{bos, __ldg(d.cu + n + 1) - bos, __ldg(d.co + n + 1) - c0, c0, 0};
 }
 // sequences (rows of the batch, or packed sequences)
-__host__ __device__ __forceinline__ int num_seqs(const Dims &d) { return d.cu ? d.N : d.B; }
+__host__ __device__ __forceinline__ int num_seqs(const Dims &d) { return d.N > 0 ? d.N : d.B; }
 // chunk tiles of the call, in the order (sequence, head, chunk)
 __device__ __forceinline__ int total_tiles(const Dims &d) {
     return d.cu ? d.H * __ldg(d.co + d.N) : d.B * d.H * d.NC;
@@ -124,7 +124,8 @@ struct SimtWs {
 // with launch_begin / launch_end (kernel kind ids below)
 enum KernelKind {
     K_SIMT_PREP = 0, K_SIMT_STATE_FWD, K_SIMT_OUT, K_SIMT_STATE_BWD, K_SIMT_BWD_A, K_SIMT_BWD_B,
-    K_DECODE, K_TC_PREP, K_TC_FWD, K_TC_BWD_STATE, K_TC_BWD_GRAD, K_SEQ_TABLE, K_KINDS
+    K_DECODE, K_TC_PREP, K_TC_FWD, K_TC_BWD_STATE, K_TC_BWD_GRAD, K_SEQ_TABLE,
+    K_PERMUTE_STATE, K_KINDS
 };
 void launch_begin(int kind, cudaStream_t s);
 void launch_end(int kind, cudaStream_t s);

@@ -33,16 +33,17 @@ template <typename E, typename GE, int DK, int DV>
 __global__ void __launch_bounds__(kDecThreads)
 decode_step_kernel(const E *__restrict__ q, const E *__restrict__ k, const E *__restrict__ v,
                    const GE *__restrict__ g, const GE *__restrict__ b,
-                   const GE *__restrict__ w, float *__restrict__ S, E *__restrict__ o, int H) {
+                   const GE *__restrict__ w, float *__restrict__ S, E *__restrict__ o, int H, int G) {
     constexpr int RW = DK / kDecWarps;  // rows per warp
     constexpr int CL = DV / 32;         // columns per lane
     __shared__ float sk[DK], sbk[DK], sq[DK], sa[DK], su[DV], sdelta[DV];
     __shared__ float red_r[kDecWarps][DV], red_p[kDecWarps][DV];
     __shared__ float s_kq;
-    const int h = blockIdx.x % H, n = blockIdx.x / H, tid = threadIdx.x;
+    // block = (sequence n, value head hv); value head hv reads key head hv / G
+    const int HV = H * G, hv = blockIdx.x % HV, n = blockIdx.x / HV, tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
-    const size_t hk = ((size_t)n * H + h) * DK, hv = ((size_t)n * H + h) * DV;
-    float *Sp = S + ((size_t)n * H + h) * DK * DV;
+    const size_t hk = ((size_t)n * H + hv / G) * DK, hvo = ((size_t)n * HV + hv) * DV;
+    float *Sp = S + ((size_t)n * HV + hv) * DK * DV;
 
     // issue the state loads first: they are the bulk of the traffic
     float x[RW][CL];
@@ -53,7 +54,7 @@ decode_step_kernel(const E *__restrict__ q, const E *__restrict__ k, const E *__
         float kv = ldx(k, hk + i), qv = ldx(q, hk + i);
         sk[i] = kv; sq[i] = qv; sbk[i] = ldx(b, hk + i) * kv; sa[i] = __expf(ldx(g, hk + i));
     }
-    for (int j = tid; j < DV; j += kDecThreads) su[j] = ldx(w, hv + j) * ldx(v, hv + j);
+    for (int j = tid; j < DV; j += kDecThreads) su[j] = ldx(w, hvo + j) * ldx(v, hvo + j);
     if (warp == 0) {
         float acc = 0.f;
         for (int i = lane; i < DK; i += 32) acc += ldx(k, hk + i) * ldx(q, hk + i);
@@ -89,7 +90,7 @@ decode_step_kernel(const E *__restrict__ q, const E *__restrict__ k, const E *__
         for (int wi = 0; wi < kDecWarps; ++wi) { r += red_r[wi][j]; p += red_p[wi][j]; }
         float dlt = su[j] - r;
         sdelta[j] = dlt;
-        stx(o, hv + j, p + s_kq * dlt);
+        stx(o, hvo + j, p + s_kq * dlt);
     }
     __syncthreads();
 #pragma unroll
@@ -104,22 +105,22 @@ decode_step_kernel(const E *__restrict__ q, const E *__restrict__ k, const E *__
 
 template <typename E, typename GE, int DK, int DV>
 static cudaError_t launch_dec(const void *q, const void *k, const void *v, const void *g,
-                              const void *b, const void *w, float *S, void *o, int N, int H,
+                              const void *b, const void *w, float *S, void *o, int N, int H, int G,
                               cudaStream_t s) {
     launch_begin(K_DECODE, s);
-    decode_step_kernel<E, GE, DK, DV><<<(unsigned)N * (unsigned)H, kDecThreads, 0, s>>>(
+    decode_step_kernel<E, GE, DK, DV><<<(unsigned)N * (unsigned)(H * G), kDecThreads, 0, s>>>(
         (const E *)q, (const E *)k, (const E *)v, (const GE *)g, (const GE *)b, (const GE *)w, S,
-        (E *)o, H);
+        (E *)o, H, G);
     launch_end(K_DECODE, s);
     return cudaGetLastError();
 }
 
 template <typename E, typename GE>
 static cudaError_t dispatch_dec(const void *q, const void *k, const void *v, const void *g,
-                                const void *b, const void *w, float *S, void *o, int N, int H,
+                                const void *b, const void *w, float *S, void *o, int N, int H, int G,
                                 int dk, int dv, cudaStream_t s) {
 #define GDN2_DEC(DK_, DV_) \
-    if (dk == DK_ && dv == DV_) return launch_dec<E, GE, DK_, DV_>(q, k, v, g, b, w, S, o, N, H, s);
+    if (dk == DK_ && dv == DV_) return launch_dec<E, GE, DK_, DV_>(q, k, v, g, b, w, S, o, N, H, G, s);
     GDN2_DEC(32, 32) GDN2_DEC(32, 64) GDN2_DEC(32, 128)
     GDN2_DEC(64, 32) GDN2_DEC(64, 64) GDN2_DEC(64, 128)
     GDN2_DEC(128, 32) GDN2_DEC(128, 64) GDN2_DEC(128, 128)
@@ -128,14 +129,14 @@ static cudaError_t dispatch_dec(const void *q, const void *k, const void *v, con
 }
 
 cudaError_t decode_launch(const void *q, const void *k, const void *v, const void *g,
-                          const void *b, const void *w, float *S, void *o, int N, int H,
+                          const void *b, const void *w, float *S, void *o, int N, int H, int G,
                           int dk, int dv, gdn2_io io, gdn2_io gate_io, cudaStream_t s) {
     using BF = __nv_bfloat16;
     if (io == GDN2_IO_BF16)
-        return gate_io == GDN2_IO_BF16 ? dispatch_dec<BF, BF>(q, k, v, g, b, w, S, o, N, H, dk, dv, s)
-                                       : dispatch_dec<BF, float>(q, k, v, g, b, w, S, o, N, H, dk, dv, s);
-    return gate_io == GDN2_IO_BF16 ? dispatch_dec<float, BF>(q, k, v, g, b, w, S, o, N, H, dk, dv, s)
-                                   : dispatch_dec<float, float>(q, k, v, g, b, w, S, o, N, H, dk, dv, s);
+        return gate_io == GDN2_IO_BF16 ? dispatch_dec<BF, BF>(q, k, v, g, b, w, S, o, N, H, G, dk, dv, s)
+                                       : dispatch_dec<BF, float>(q, k, v, g, b, w, S, o, N, H, G, dk, dv, s);
+    return gate_io == GDN2_IO_BF16 ? dispatch_dec<float, BF>(q, k, v, g, b, w, S, o, N, H, G, dk, dv, s)
+                                   : dispatch_dec<float, float>(q, k, v, g, b, w, S, o, N, H, G, dk, dv, s);
 }
 
 }  // namespace gdn2

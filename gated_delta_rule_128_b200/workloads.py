@@ -152,3 +152,16 @@ def decode_step_inputs(N: int, H: int, dk: int, dv: int, seed: int, step: int,
     d = draw(N, 1, H, dk, dv, seed * 1_000_003 + step, erase_scale=erase_scale,
              with_dO=False)
     return {n: d[n][:, 0].contiguous() for n in ("q", "k", "v", "g", "b", "w")}
+
+
+def packed_lengths(total: int, seed: int, lo: int = 1, hi: int = 2048) -> list:
+    """Sequence lengths for a packed batch of `total` tokens: drawn uniformly
+    from [lo, hi] (seeded) until they fill `total`, the last one cut to fit.
+    A stand-in for documents of mixed lengths packed into one training row."""
+    gen = torch.Generator().manual_seed(seed)
+    lens, left = [], total
+    while left > 0:
+        n = int(torch.randint(lo, hi + 1, (1,), generator=gen).item())
+        lens.append(min(n, left))
+        left -= lens[-1]
+    return lens

@@ -142,68 +142,78 @@ gdn2_status gdn2_decode_step(const void *q, const void *k, const void *v, const 
                              const float *b, const float *w, float *S, void *o, int N, int H,
                              int d_k, int d_v, gdn2_io io, gdn2_stream_t stream);
 
-/* The same three calls with the gate tensors in a type of their own.
- *   gate_io : type of g, b, w and of dg, db, dw.  GDN2_IO_F32 makes each call
- *             identical to gdn2_fwd / gdn2_bwd / gdn2_decode_step.  GDN2_IO_BF16
- *             halves the gate bytes ("Gated DeltaNet-2" LIT-802 review, "Key
- *             takeaways" 1: b and w are sigmoid gates, values in (0, 1) or
- *             (0, 2), which bf16 holds to 3 significant digits); values are
- *             widened to float32 on load and the gradients rounded once on
- *             store.  For gdn2_fwd_ex / gdn2_bwd_ex it needs the tensor-core
- *             path (io = GDN2_IO_BF16, d_k = d_v = 128, chunk = 64) and returns
- *             GDN2_ERR_UNSUPPORTED otherwise; gdn2_decode_step_ex takes it for
- *             every size.
- * Every other argument, the layouts, the workspace size and the error
- * behaviour are those of the call without the suffix. */
+/* The same calls with two more choices: the gate tensors' type and grouped
+ * value heads.
+ *   gate_io : type of g, b, w and of dg, db, dw.  GDN2_IO_F32 gives the calls
+ *       above.  GDN2_IO_BF16 halves the gate bytes ("Gated DeltaNet-2"
+ *       LIT-802 review, "Key takeaways" 1: b and w are sigmoid gates, values in
+ *       (0, 1) or (0, 2), which bf16 holds to 3 significant digits); values
+ *       are widened to float32 on load and the gradients rounded once on store.
+ *       For the chunkwise calls it needs the tensor-core path (io =
+ *       GDN2_IO_BF16, d_k = d_v = 128 after grouping, chunk = 64) and returns
+ *       GDN2_ERR_UNSUPPORTED otherwise; the decode step takes it at every size.
+ *   H_v : value heads, a multiple of H (H_v = H or 0: one value head per key
+ *       head).  The LIT-802 review's "Where the hedges are" gives the write
+ *       gate H_v d_v outputs against H d_k for the erase gate: value head
+ *       j uses query/key head j / (H_v / H), so q, k, g, b keep H heads and v,
+ *       w, o, dO, dv, dw take H_v: [B, T, H_v, d_v]; states are
+ *       [B, H_v, d_k, d_v].  The G = H_v / H value heads of one key head evolve
+ *       together as one state of G d_v columns, so the chunkwise calls need
+ *       G d_v in {32, 64, 128} (and 128 for the tensor-core path); d_v is then
+ *       32 or 64.  The decode step takes any d_k, d_v of the supported set.
+ * Every other argument, the layouts and the error behaviour are those of the
+ * call without the suffix.  The workspace comes from gdn2_workspace_bytes_ex,
+ * which also counts two state buffers when H_v > H. */
+size_t gdn2_workspace_bytes_ex(int B, int T, int H, int H_v, int d_k, int d_v, int chunk, gdn2_io io,
+                               gdn2_io gate_io, int for_bwd);
 gdn2_status gdn2_fwd_ex(const void *q, const void *k, const void *v, const void *g, const void *b,
                         const void *w, const float *S0, void *o, float *ST, void *ws,
-                        size_t ws_bytes, int B, int T, int H, int d_k, int d_v, int chunk,
+                        size_t ws_bytes, int B, int T, int H, int H_v, int d_k, int d_v, int chunk,
                         gdn2_io io, gdn2_io gate_io, gdn2_stream_t stream);
 gdn2_status gdn2_bwd_ex(const void *q, const void *k, const void *v, const void *g, const void *b,
                         const void *w, const float *S0, const void *dO, const float *dST, void *dq,
                         void *dk, void *dv, void *dg, void *db, void *dw, float *dS0, void *ws,
-                        size_t ws_bytes, int ws_has_fwd, int B, int T, int H, int d_k, int d_v,
-                        int chunk, gdn2_io io, gdn2_io gate_io, gdn2_stream_t stream);
+                        size_t ws_bytes, int ws_has_fwd, int B, int T, int H, int H_v, int d_k,
+                        int d_v, int chunk, gdn2_io io, gdn2_io gate_io, gdn2_stream_t stream);
 gdn2_status gdn2_decode_step_ex(const void *q, const void *k, const void *v, const void *g,
                                 const void *b, const void *w, float *S, void *o, int N, int H,
-                                int d_k, int d_v, gdn2_io io, gdn2_io gate_io,
+                                int H_v, int d_k, int d_v, gdn2_io io, gdn2_io gate_io,
                                 gdn2_stream_t stream);
 
 /* Packed variable-length sequences: N sequences stored back to back along one
  * token axis, each with its own initial and final state (no state crosses from
- * one sequence to the next; "Gated DeltaNet-2" LIT-802 review, "Where the
- * hedges are": the mixer runs inside a language model, whose training packs
- * documents of mixed lengths).
- *   q, k, g, b, dq, dk, dg, db : [1, T, H, d_k];  v, w, o, dO, dv, dw : [1, T, H, d_v]
- *   S0, ST, dST, dS0 : [N, H, d_k, d_v]
+ * one sequence to the next; the mixer runs inside a language model, whose
+ * training packs documents of mixed lengths).
+ *   q, k, g, b, dq, dk, dg, db : [1, T, H, d_k];  v, w, o, dO, dv, dw : [1, T, H_v, d_v]
+ *   S0, ST, dST, dS0 : [N, H_v, d_k, d_v]
  *   cu_seqlens : device int32 [N + 1]: sequence n holds tokens cu_seqlens[n]
  *       .. cu_seqlens[n + 1] - 1.  It must rise from 0 to T (a sequence may be
  *       empty: its S_T is S0).  The table is read on the device only (the call
  *       does not synchronise): a table that breaks this rule makes the call
  *       treat every sequence as empty and records GDN2_ERR_INVALID_ARG in the
- *       device status word.
+ *       device status word.  4-byte alignment suffices.
  *   N : 1 .. 65535 sequences.
- * Tensor-core path only: io = GDN2_IO_BF16, d_k = d_v = 128, chunk = 64, gate_io
- * either type; other sizes return GDN2_ERR_UNSUPPORTED.  Chunks never cross a
- * sequence boundary: a sequence of length L takes ceil(L / 64) chunks, the last
- * one short.
+ * Tensor-core path only: io = GDN2_IO_BF16, d_k = 128, G d_v = 128, chunk = 64,
+ * gate_io and H_v as for the _ex calls; other sizes return
+ * GDN2_ERR_UNSUPPORTED.  Chunks never cross a sequence boundary: a sequence of
+ * length L takes ceil(L / 64) chunks, the last one short.
  * Workspace: gdn2_workspace_bytes_varlen (for_bwd as for gdn2_workspace_bytes,
- * sized for the worst case of N sequences over T tokens); the workspace also
- * holds the chunk table the call derives from cu_seqlens.  ws_has_fwd as for
- * gdn2_bwd, with the same cu_seqlens. */
-size_t gdn2_workspace_bytes_varlen(int N, int T, int H, int d_k, int d_v, int chunk, gdn2_io io,
-                                   int for_bwd);
+ * sized for the worst case of N sequences over T tokens); it also holds the
+ * chunk table the call derives from cu_seqlens.  ws_has_fwd as for gdn2_bwd,
+ * with the same cu_seqlens. */
+size_t gdn2_workspace_bytes_varlen(int N, int T, int H, int H_v, int d_k, int d_v, int chunk,
+                                   gdn2_io io, gdn2_io gate_io, int for_bwd);
 gdn2_status gdn2_fwd_varlen(const void *q, const void *k, const void *v, const void *g,
                             const void *b, const void *w, const float *S0, void *o, float *ST,
                             void *ws, size_t ws_bytes, const int *cu_seqlens, int N, int T, int H,
-                            int d_k, int d_v, int chunk, gdn2_io io, gdn2_io gate_io,
+                            int H_v, int d_k, int d_v, int chunk, gdn2_io io, gdn2_io gate_io,
                             gdn2_stream_t stream);
 gdn2_status gdn2_bwd_varlen(const void *q, const void *k, const void *v, const void *g,
                             const void *b, const void *w, const float *S0, const void *dO,
                             const float *dST, void *dq, void *dk, void *dv, void *dg, void *db,
                             void *dw, float *dS0, void *ws, size_t ws_bytes, int ws_has_fwd,
-                            const int *cu_seqlens, int N, int T, int H, int d_k, int d_v, int chunk,
-                            gdn2_io io, gdn2_io gate_io, gdn2_stream_t stream);
+                            const int *cu_seqlens, int N, int T, int H, int H_v, int d_k, int d_v,
+                            int chunk, gdn2_io io, gdn2_io gate_io, gdn2_stream_t stream);
 
 /* Bytes of the scratch array behind gdn2_fwd_noalloc (64 MiB). */
 #define GDN2_NOALLOC_SCRATCH_BYTES (64u << 20)

@@ -113,24 +113,47 @@ def test_decode_rejects_bad_arguments(L):
     assert f(*bad) == 1
 
 
-def test_ex_entry_points_check_the_gate_type(L):
+def test_ex_entry_points_check_the_gate_type_and_value_heads(L):
     """bf16 gates need the tensor-core path: any other size or io type is
     rejected as unsupported, an unknown gate type as invalid, and float32
-    gates behave as the calls without the suffix."""
-    def fwd_ex(gate_io, dk=32, dv=32, chunk=16, io=0, ws_bytes=1 << 40):
+    gates with H_v = H behave as the calls without the suffix.  H_v must be a
+    multiple of H whose group width G d_v is a supported d_v."""
+    def fwd_ex(gate_io, dk=32, dv=32, chunk=16, io=0, ws_bytes=1 << 40, H=1, Hv=1):
         return L.gdn2_fwd_ex(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, None, FAKE, ws_bytes,
-                             1, 16, 1, dk, dv, chunk, io, gate_io, None)
+                             1, 16, H, Hv, dk, dv, chunk, io, gate_io, None)
     assert fwd_ex(1) == 2                              # f32 io, d = 32
     assert fwd_ex(1, dk=128, dv=128, chunk=64) == 2    # still f32 io
     assert fwd_ex(1, dk=128, dv=128, chunk=32, io=1) == 2
     assert fwd_ex(5) == 1
     assert fwd_ex(0, ws_bytes=10) == 3 == fwd(L, ws_bytes=10)
     assert fwd_ex(1, dk=128, dv=128, chunk=64, io=1, ws_bytes=10) == 3   # passes the gate check
+    assert fwd_ex(0, H=2, Hv=3) == 1                   # not a multiple
+    assert fwd_ex(0, H=2, Hv=1) == 1                   # fewer value heads
+    assert fwd_ex(0, H=1, Hv=8, dv=32) == 2            # G d_v = 256
+    assert fwd_ex(0, H=1, Hv=4, dv=32, ws_bytes=10) == 3   # G d_v = 128: passes
+    assert fwd_ex(1, dk=128, dv=64, chunk=64, io=1, H=1, Hv=2, ws_bytes=10) == 3  # tensor cores
     args = [FAKE] * 6 + [None, FAKE, None] + [FAKE] * 6 + [None, FAKE]
-    assert L.gdn2_bwd_ex(*args, 1 << 40, 1, 1, 16, 1, 32, 32, 16, 0, 1, None) == 2
-    assert L.gdn2_bwd_ex(*args, 1 << 40, 1, 1, 16, 1, 32, 32, 16, 0, 9, None) == 1
-    assert L.gdn2_decode_step_ex(*([FAKE] * 8), 1, 1, 32, 32, 0, 7, None) == 1
-    assert L.gdn2_decode_step_ex(*([FAKE] * 8), 1, 1, 16, 32, 0, 1, None) == 2
+    assert L.gdn2_bwd_ex(*args, 1 << 40, 1, 1, 16, 1, 1, 32, 32, 16, 0, 1, None) == 2
+    assert L.gdn2_bwd_ex(*args, 1 << 40, 1, 1, 16, 1, 1, 32, 32, 16, 0, 9, None) == 1
+    assert L.gdn2_decode_step_ex(*([FAKE] * 8), 1, 1, 1, 32, 32, 0, 7, None) == 1
+    assert L.gdn2_decode_step_ex(*([FAKE] * 8), 1, 1, 1, 16, 32, 0, 1, None) == 2
+    assert L.gdn2_decode_step_ex(*([FAKE] * 8), 1, 2, 3, 32, 32, 0, 0, None) == 1
+
+
+def test_workspace_sizes_of_the_ex_and_packed_calls(L):
+    """H_v = H sizes as the plain call; grouped heads add two state buffers;
+    packed sequences size for ceil(T / 64) + N chunks and need the tensor-core
+    path."""
+    plain = gdn.gdn2_workspace_bytes(2, 300, 4, 128, 128, 64, 1, 1)
+    assert gdn.gdn2_workspace_bytes_ex(2, 300, 4, 4, 128, 128, 64, 1, 0, 1) == plain
+    assert gdn.gdn2_workspace_bytes_ex(2, 300, 4, 0, 128, 128, 64, 1, 1, 1) == plain
+    grouped = gdn.gdn2_workspace_bytes_ex(2, 300, 4, 8, 128, 64, 64, 1, 0, 1)
+    assert grouped >= plain + 2 * 2 * 4 * 128 * 128 * 4
+    one = gdn.gdn2_workspace_bytes_varlen(1, 600, 4, 4, 128, 128, 64, 1, 0, 1)
+    many = gdn.gdn2_workspace_bytes_varlen(50, 600, 4, 4, 128, 128, 64, 1, 0, 1)
+    assert 0 < one < many
+    assert gdn.gdn2_workspace_bytes_varlen(1, 600, 4, 4, 64, 64, 64, 1, 0, 1) == 0   # no tensor cores
+    assert gdn.gdn2_workspace_bytes_varlen(0, 600, 4, 4, 128, 128, 64, 1, 0, 1) == 0
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):

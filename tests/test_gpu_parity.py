@@ -382,6 +382,53 @@ def test_varlen_rejects_a_bad_table_on_the_device():
     assert np.isfinite(gpu["o"]).all()
 
 
+# ------------------------------------------------------ grouped value heads
+
+def _grouped_inputs(B, T, H, Hv, dk, dv, seed):
+    x = workloads.draw(B, T, H, dk, dv, seed)
+    xv = workloads.draw(B, T, Hv, dk, dv, seed + 1, s0_std=0.1, with_dST=True)
+    for n in ("v", "w", "S0", "dO", "dST"):
+        x[n] = xv[n]
+    return x
+
+
+@pytest.mark.parametrize("io,H,Hv,dk,dv,chunk", [
+    ("bf16", 2, 4, 128, 64, 64),     # tensor cores: G d_v = 128
+    ("f32", 1, 2, 64, 32, 32),       # CUDA cores: G d_v = 64
+    ("bf16", 1, 4, 32, 32, 16),      # CUDA cores, bf16 I/O: G d_v = 128
+])
+def test_grouped_value_heads(io, H, Hv, dk, dv, chunk):
+    """H_v value heads over H key heads: value head j reads key head
+    j / (H_v / H); states per value head.  Against the oracle's grouped form
+    (the token loop on repeated q, k, g, b, key-side gradients summed)."""
+    from oracle import grouped
+    x = _grouped_inputs(2, 150, H, Hv, dk, dv, 960 + Hv)
+    gpu = gpu_fwd_bwd(x, io, chunk)
+    r = to_np64(io_round(x, io))
+    names = ("q", "k", "v", "g", "b", "w", "S0")
+    o, ST = grouped.forward(*(r[n] for n in names))
+    ref = {"o": o, "ST": ST, **grouped.backward(*(r[n] for n in names), r["dO"], r["dST"])}
+    compare(gpu, ref, io, ("o", "ST") + GRADS)
+
+
+def test_grouped_value_heads_packed():
+    """Grouped value heads and packed sequences together (tensor cores)."""
+    from oracle import varlen
+    cu = [0, 70, 71, 200]       # lengths 70, 1, 129
+    x = _grouped_inputs(1, 200, 1, 2, 128, 64, 970)
+    x["S0"] = workloads.draw(3, 1, 2, 128, 64, 971, s0_std=0.1)["S0"]
+    x["dST"] = workloads.draw(3, 1, 2, 128, 64, 972, s0_std=0.1)["S0"]
+    gpu = gpu_varlen(x, cu)
+    r = to_np64(io_round(x, "bf16"))
+    rep = {n: (np.repeat(r[n], 2, axis=2) if n in ("q", "k", "g", "b") else r[n]) for n in r}
+    names = ("q", "k", "v", "g", "b", "w")
+    o, ST = varlen.forward(*(rep[n] for n in names), cu, rep["S0"])
+    gr = varlen.backward(*(rep[n] for n in names), cu, rep["S0"], rep["dO"], rep["dST"])
+    for n in ("q", "k", "g", "b"):
+        gr["d" + n] = gr["d" + n].reshape(1, 200, 1, 2, 128).sum(axis=3)
+    compare(gpu, {"o": o, "ST": ST, **gr}, "bf16", ("o", "ST") + GRADS)
+
+
 # ------------------------------------------------------------------ decode
 
 @pytest.mark.parametrize("io,gates", [("f32", "f32"), ("bf16", "f32"), ("bf16", "bf16"),
@@ -403,6 +450,26 @@ def test_decode_small_step_by_step(io, gates, dk, dv):
         o_ref, S_ref = oracle.forward(r["q"], r["k"], r["v"], r["g"], r["b"], r["w"], S_ref)
         assert rel(o.float().cpu().numpy(), o_ref[:, 0]) < tol, s
         assert rel(S_gpu.cpu().numpy(), S_ref) < tol, s
+
+
+@pytest.mark.parametrize("H,Hv,dk,dv", [(2, 4, 64, 32), (1, 2, 128, 128)])
+def test_decode_grouped_value_heads(H, Hv, dk, dv):
+    """The decode step with H_v value heads over H key heads, against the
+    oracle's grouped form, step by step from the same state."""
+    from oracle import grouped
+    N, steps = 3, 6
+    S_gpu = workloads.decode_state(N, Hv, dk, dv, 11, 0.3).cuda()
+    S_ref = S_gpu.double().cpu().numpy()
+    for s_ in range(steps):
+        xk = workloads.decode_step_inputs(N, H, dk, dv, 12, s_)
+        xv = workloads.decode_step_inputs(N, Hv, dk, dv, 13, s_)
+        x = {n: (xk[n] if n in ("q", "k", "g", "b") else xv[n]) for n in ("q", "k", "v", "g", "b", "w")}
+        d = {n: t.cuda() for n, t in x.items()}
+        o = gdn.decode_step(d["q"], d["k"], d["v"], d["g"], d["b"], d["w"], S_gpu)
+        r = {n: t.double().numpy()[:, None] for n, t in x.items()}
+        o_ref, S_ref = grouped.forward(r["q"], r["k"], r["v"], r["g"], r["b"], r["w"], S_ref)
+        assert rel(o.cpu().numpy(), o_ref[:, 0]) < TOL_F32, s_
+        assert rel(S_gpu.cpu().numpy(), S_ref) < TOL_F32, s_
 
 
 def test_decode_equals_chunked_forward():

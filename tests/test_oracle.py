@@ -394,3 +394,39 @@ def test_varlen_oracle_sequences_are_independent():
     keep = np.r_[0:5, 6:T]
     assert np.array_equal(o2[:, keep], o[:, keep]) and not np.array_equal(o2[:, 5], o[:, 5])
     assert np.array_equal(ST2[[0, 2, 3]], ST[[0, 2, 3]]) and not np.array_equal(ST2[1], ST[1])
+
+
+# ------------------------------------------------------ grouped value heads
+
+def test_grouped_oracle_gradients_match_finite_differences():
+    """H = 1 key head, H_v = 2 value heads: the grouped forward's gradients
+    (the key side summed over the group) against central differences of the
+    grouped forward itself."""
+    from oracle import grouped
+    B, T, H, Hv, dk, dv = 1, 7, 1, 2, 3, 2
+    x = workloads.draw(B, T, H, dk, dv, 621)
+    xv = workloads.draw(B, T, Hv, dk, dv, 622, s0_std=0.4, with_dST=True)
+    r = {n: t.double().numpy() for n, t in x.items()}
+    for n in ("v", "w", "S0", "dO", "dST"):
+        r[n] = xv[n].double().numpy()
+    names = ("q", "k", "v", "g", "b", "w", "S0")
+    gr = grouped.backward(*(r[n] for n in names), r["dO"], r["dST"])
+    num = fd.gradients({n: r[n] for n in names}, r["dO"], r["dST"], fn=grouped.forward)
+    for n in names:
+        assert np.max(np.abs(gr["d" + n] - num["d" + n])) < 1e-7, n
+
+
+def test_grouped_oracle_is_the_plain_recurrence_per_value_head():
+    """Each value head of a grouped call equals a plain call on its key head:
+    value heads 2 and 3 of H = 2, H_v = 4 read key head 1."""
+    from oracle import grouped
+    B, T, H, Hv, dk, dv = 2, 9, 2, 4, 4, 3
+    x = workloads.draw(B, T, H, dk, dv, 623)
+    xv = workloads.draw(B, T, Hv, dk, dv, 624, s0_std=0.3)
+    r = {n: t.double().numpy() for n, t in x.items()}
+    for n in ("v", "w", "S0"):
+        r[n] = xv[n].double().numpy()
+    o, ST = grouped.forward(*(r[n] for n in ("q", "k", "v", "g", "b", "w", "S0")))
+    o3, ST3 = oracle.forward(r["q"][:, :, 1:2], r["k"][:, :, 1:2], r["v"][:, :, 3:4], r["g"][:, :, 1:2],
+                             r["b"][:, :, 1:2], r["w"][:, :, 3:4], r["S0"][:, 3:4])
+    assert np.array_equal(o[:, :, 3:4], o3) and np.array_equal(ST[:, 3:4], ST3)
