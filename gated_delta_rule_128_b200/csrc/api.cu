@@ -76,7 +76,7 @@ static double g_kind_ms[K_KINDS];
 static const char *const g_kind_names[K_KINDS] = {
     "simt_chunk_prep", "simt_state_fwd", "simt_out_fwd", "simt_state_bwd", "simt_chunk_bwd_a",
     "simt_chunk_bwd_b", "decode_step", "tc_prep", "tc_fwd", "tc_bwd_state", "tc_bwd_grad", "seq_table",
-    "permute_state"};
+    "permute_state", "seg_link"};
 
 void launch_begin(int kind, cudaStream_t s) {
     g_launches.fetch_add(1, std::memory_order_relaxed);

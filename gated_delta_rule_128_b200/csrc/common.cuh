@@ -93,6 +93,43 @@ __device__ __forceinline__ size_t tile(const Dims &d, int bb, int h, int c) {
     return ((size_t)bb * d.H + h) * d.NC + c;
 }
 
+// ---- segment-parallel state passes.  A long sequence with few (b, h) leaves
+// most SMs idle in the sequential state kernels; its chunks then split into P
+// segments, and S_end = M_s S_begin + N_s over segment s (M_s the product of
+// the chunks' transitions, N_s the state reached from zero):
+//   phase 1: segment 0 for real; for every middle segment s = 1 .. P-2, N_s
+//            (a run from a zero state) and M_s (a run from the identity with no
+//            input), all in parallel;
+//   link:    entries S_{s+1} = M_s S_s + N_s, s = 1 .. P-2 (a short scan);
+//   phase 2: segments 1 .. P-1 for real from their entries, in parallel.
+// The backward runs the same way in reverse with M_s^T (dS_entry = M_s^T
+// dS_exit + R_s, R_s the gradient reached from a zero exit gradient).
+// buf holds [bh][P][3][128 x 128] float32: entry (kind 0), zero-run result
+// (kind 1) and map M_s (kind 2), rows of 128 like a state.
+struct SegPass {
+    int P;      // segments per sequence (1: one run over the whole sequence)
+    int phase;  // 0: the whole sequence; 1, 2: the passes above
+    float *buf;
+};
+enum SegKind { SEG_ENTRY = 0, SEG_ZERO = 1, SEG_MAP = 2 };
+__host__ __device__ __forceinline__ float *seg_buf(const SegPass &sp, size_t bh, int s, int kind) {
+    return sp.buf + ((bh * sp.P + s) * 3 + kind) * (size_t)(128 * 128);
+}
+// chunk range of segment s (P segments over nc chunks, every one non-empty)
+__host__ __device__ __forceinline__ int seg_len(int nc, int P) { return (nc + P - 1) / P; }
+// the largest useful P: every segment non-empty, at least 4 chunks each, and
+// the first pass (2 + 4 (P - 2) CTAs per (b, h)) within one wave of 148 SMs
+inline int seg_count(int B, int H, int nc) {
+    int best = 1;
+    for (int P = 3; P <= 8; ++P) {
+        const int L = seg_len(nc, P);
+        if (L < 4 || (P - 1) * L >= nc) break;
+        if ((long long)(2 + 4 * (P - 2)) * B * H > 148) break;
+        best = P;
+    }
+    return best;
+}
+
 // ---- the device status word (GDN2_OK or the first error recorded); kernels
 // that can give up on a bounded wait receive its device address.
 __device__ __forceinline__ void record_status(unsigned int *status, unsigned int s) {
@@ -125,7 +162,7 @@ struct SimtWs {
 enum KernelKind {
     K_SIMT_PREP = 0, K_SIMT_STATE_FWD, K_SIMT_OUT, K_SIMT_STATE_BWD, K_SIMT_BWD_A, K_SIMT_BWD_B,
     K_DECODE, K_TC_PREP, K_TC_FWD, K_TC_BWD_STATE, K_TC_BWD_GRAD, K_SEQ_TABLE,
-    K_PERMUTE_STATE, K_KINDS
+    K_PERMUTE_STATE, K_SEG_LINK, K_KINDS
 };
 void launch_begin(int kind, cudaStream_t s);
 void launch_end(int kind, cudaStream_t s);
@@ -200,7 +237,8 @@ inline SimtWs simt_ws_layout(const Dims &d) {
 constexpr uint32_t REC_WQ = 0, REC_KH = 32768, REC_T = 49152, REC_P = 57344, REC_FAC = 65536,
                    REC_BYTES = 66560;
 struct TcWs {
-    size_t rec, rec_end, ckS, ckD, fwd_end, ckdS, ckndU, bwd_end;
+    size_t rec, rec_end, ckS, ckD, seg, fwd_end, ckdS, ckndU, bwd_end;
+    int P;  // segments per sequence of the state passes (1: none)
 };
 inline TcWs tc_ws_layout(const Dims &d) {
     const size_t bh = (size_t)d.B * d.H, nc = (size_t)d.NC;
@@ -211,6 +249,8 @@ inline TcWs tc_ws_layout(const Dims &d) {
     w.rec_end = o;
     w.ckS = take(bh * nc * 2 * 16384);
     w.ckD = take(bh * nc * 2 * 8192);
+    w.P = d.N > 0 ? 1 : seg_count(d.B, d.H, d.NC);
+    w.seg = take(w.P > 1 ? bh * w.P * 3 * 128 * 128 * sizeof(float) : 0);
     w.fwd_end = o;
     w.ckdS = take(bh * nc * 2 * 16384);
     w.ckndU = take(bh * nc * 2 * 8192);

@@ -69,7 +69,7 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
                     const __grid_constant__ CUtensorMap mw, const __grid_constant__ CUtensorMap mdv,
                     const __grid_constant__ CUtensorMap mdw, const float *__restrict__ dST,
                     float *__restrict__ dS0, void *__restrict__ dv_out, void *__restrict__ dw_out,
-                    unsigned char *__restrict__ ws, TcWs lay, unsigned int *status, Dims d) {
+                    unsigned char *__restrict__ ws, TcWs lay, SegPass sp, unsigned int *status, Dims d) {
     using namespace tbs;
     extern __shared__ unsigned char smraw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(
@@ -81,20 +81,50 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
     float big = 0.f;  // range check: operand magnitude
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int vh = blockIdx.x, h = blockIdx.y, n = blockIdx.z, v0 = vh * 64;
-    // sequence n: tokens bos .. bos + T - 1 of batch row bb, chunks NC
+    const int h = blockIdx.y, n = blockIdx.z;
+    // this CTA's task (SegPass in common.cuh): a real run of segment sg, or in
+    // the first pass of a split sequence a run from a zero exit gradient (R_s)
+    int vh, sg = 0, mode = 0;  // mode 0 real, 1 from zero
+    {
+        const int x = blockIdx.x;
+        if (sp.P == 1) { vh = x; }
+        else if (sp.phase == 2) { sg = x >> 1; vh = x & 1; }
+        else if (x < 2) { sg = sp.P - 1; vh = x; }
+        else { mode = 1; sg = 1 + ((x - 2) >> 1); vh = (x - 2) & 1; }
+    }
+    const int v0 = vh * 64;
+    // sequence n: tokens bos .. bos + T - 1 of batch row bb, chunks NC; a
+    // segment narrows these to its own chunks
     const Seq sq = seq_of(d, n);
-    const int NC = sq.nc, T = sq.len, bb = sq.brow, bos = sq.bos;
+    int NC = sq.nc, T = sq.len, bos = sq.bos;
+    const int bb = sq.brow;
+    const size_t bhx = (size_t)n * d.H + h;
+    size_t tile0 = (size_t)tile_of(d, sq, h, 0);  // workspace tile of the run's first chunk
+    if (sp.P > 1) {
+        const int L = seg_len(NC, sp.P), cb = sg * L;
+        NC = min(L, NC - cb);
+        T = min(T - 64 * cb, 64 * NC);
+        bos += 64 * cb;
+        tile0 += cb;
+    }
+    // the exit gradient (null: zero) and where the entry gradient goes (null:
+    // nowhere); only real runs write dv, dw, -dU and dS'
+    const bool real = mode == 0;
+    const float *ext = !real ? nullptr
+                     : (sp.P == 1 || sg == sp.P - 1) ? (dST ? dST + st_off(d, n, h) : nullptr)
+                     : seg_buf(sp, bhx, sg, SEG_ENTRY);
+    float *fin = !real ? seg_buf(sp, bhx, sg, SEG_ZERO)
+               : (sp.P == 1 || sg == 0) ? (dS0 ? dS0 + st_off(d, n, h) : nullptr)
+               : (sp.phase == 1 ? seg_buf(sp, bhx, sp.P - 2, SEG_ENTRY) : nullptr);
     const bool compute = tid < kCompute, issuer = tid == kCompute, copier = tid == kCompute + 32;
     const bool copy_warp = warp == kCompute / 32 + 1;
     const int quarter = warp & 3, half = (warp >> 2) & 1;
     const int key = quarter * 32 + lane;
-    const size_t tile0 = (size_t)tile_of(d, sq, h, 0);  // workspace tile of chunk 0
     const unsigned char *recs = ws + lay.rec + tile0 * (size_t)REC_BYTES;
     if (NC <= 0) {  // an empty sequence: dS0 = dS_T
-        if (dS0 && tid < 256) {
-            const size_t so = st_off(d, n, h) + (size_t)(tid >> 1) * 128 + v0 + 32 * (tid & 1);
-            for (int j = 0; j < 32; ++j) dS0[so + j] = dST ? dST[so + j] : 0.f;
+        if (fin && tid < 256) {
+            const size_t so = (size_t)(tid >> 1) * 128 + v0 + 32 * (tid & 1);
+            for (int j = 0; j < 32; ++j) fin[so + j] = ext ? ext[so + j] : 0.f;
         }
         return;
     }
@@ -216,7 +246,9 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
     // whole warp instead of by TMA stores, which would write all 64 rows.
     auto store_du = [&](int cc) {
         const int L = T - 64 * cc;
-        if (d.cu && L < 64) {
+        if (!real) {
+            // a run from a zero exit gradient keeps only its entry gradient
+        } else if (d.cu && L < 64) {
             __nv_bfloat16 *dvp = reinterpret_cast<__nv_bfloat16 *>(dv_out);
             for (int i = lane; i < L * 8; i += 32) {  // dv: 8 chunks of 8 bf16 per row
                 const int r = i >> 3, j = i & 7;
@@ -240,7 +272,7 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
             if (!GB) tma_store_4d(&mdw, sm + VW + 8192, v0 + 32, h, bos + cc * 64, bb);
         }
         if (lane == 0) {
-            bulk_store(ws + lay.ckndU + ((tile0 + cc) * 2 + vh) * 8192, sm + NDU, 8192);
+            if (real) bulk_store(ws + lay.ckndU + ((tile0 + cc) * 2 + vh) * 8192, sm + NDU, 8192);
             bulk_commit();
             bulk_wait_read();  // VV, VW and NDU may be rewritten
             if (cc > 0) load_vw(cc - 1);
@@ -257,10 +289,9 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
     bool ok = true;
     if (compute) {
         float x[32];
-        const size_t so = st_off(d, n, h);
 #pragma unroll
         for (int j = 0; j < 32; j += 4) {
-            float4 t = dST ? *reinterpret_cast<const float4 *>(dST + so + (size_t)key * 128 + v0 + 32 * half + j)
+            float4 t = ext ? *reinterpret_cast<const float4 *>(ext + (size_t)key * 128 + v0 + 32 * half + j)
                            : make_float4(0.f, 0.f, 0.f, 0.f);
             x[j] = t.x; x[j + 1] = t.y; x[j + 2] = t.z; x[j + 3] = t.w;
         }
@@ -275,7 +306,7 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
     bool abort = __syncthreads_or(!ok);
     if (!abort && copier) {
         fence_after_sync();
-        bulk_store(ws + lay.ckdS + ((tile0 + NC - 1) * 2 + vh) * 16384, sm + OP_DS, 16384);
+        if (real) bulk_store(ws + lay.ckdS + ((tile0 + NC - 1) * 2 + vh) * 16384, sm + OP_DS, 16384);
         bulk_commit();
         if (NC > 1) load_do(NC - 2);
         bulk_wait_read();  // the dS' copy has left OP_DS
@@ -359,8 +390,8 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
 #pragma unroll
             for (int j = 0; j < 32; ++j) sv[j] *= se;
             if (c == 0) {
-                if (dS0) {
-                    float *dst = dS0 + st_off(d, n, h) + (size_t)key * 128 + v0 + 32 * half;
+                if (fin) {
+                    float *dst = fin + (size_t)key * 128 + v0 + 32 * half;
 #pragma unroll
                     for (int j = 0; j < 32; j += 4)
                         *reinterpret_cast<float4 *>(dst + j) = make_float4(sv[j], sv[j + 1], sv[j + 2], sv[j + 3]);
@@ -377,7 +408,7 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
         if (c > 0) {
             if (copier) {
                 fence_after_sync();
-                bulk_store(ws + lay.ckdS + ((tile0 + c - 1) * 2 + vh) * 16384, sm + OP_DS, 16384);
+                if (real) bulk_store(ws + lay.ckdS + ((tile0 + c - 1) * 2 + vh) * 16384, sm + OP_DS, 16384);
                 bulk_commit();
                 if (c >= 2) {
                     load_do(c - 2);           // raw dO consumed
@@ -415,6 +446,9 @@ cudaError_t tc_bwd_grad_launch(const void *q, const void *k, const void *g, cons
                                const void *dO, void *dq, void *dk, void *dg, void *db, void *ws,
                                unsigned int *status, const Dims &d, cudaStream_t s);
 
+// the link step between the passes (seg_link.cu)
+cudaError_t seg_link_launch(const SegPass &sp, int nbh, bool backward, cudaStream_t s);
+
 template <bool GB>
 static cudaError_t tc_bwd_state_run(const void *v, const void *w, const void *dO, const float *dST,
                                     void *dv, void *dw, float *dS0, void *ws, unsigned int *status,
@@ -430,10 +464,23 @@ static cudaError_t tc_bwd_state_run(const void *v, const void *w, const void *dO
     cudaError_t e = cudaFuncSetAttribute(tc_bwd_state_kernel<GB>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tbs::SMEM_BYTES);
     if (e != cudaSuccess) return e;
+    // a split sequence takes the maps M_s the split forward left in the workspace
+    SegPass sp{1, 0, nullptr};
+    if (lay.P > 1) sp = SegPass{lay.P, 1, reinterpret_cast<float *>(static_cast<char *>(ws) + lay.seg)};
     launch_begin(K_TC_BWD_STATE, s);
-    tc_bwd_state_kernel<GB><<<dim3(2, d.H, num_seqs(d)), tbs::kThreads, tbs::SMEM_BYTES, s>>>(
-        mdo_half, mv, mw, mdv, mdw, dST, dS0, dv, dw, (unsigned char *)ws, lay, status, d);
+    tc_bwd_state_kernel<GB><<<dim3(sp.P > 1 ? 2 * (sp.P - 1) : 2, d.H, num_seqs(d)), tbs::kThreads,
+                              tbs::SMEM_BYTES, s>>>(mdo_half, mv, mw, mdv, mdw, dST, dS0, dv, dw,
+                                                    (unsigned char *)ws, lay, sp, status, d);
     launch_end(K_TC_BWD_STATE, s);
+    if (sp.P > 1) {
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if ((e = seg_link_launch(sp, d.B * d.H, true, s)) != cudaSuccess) return e;
+        sp.phase = 2;
+        launch_begin(K_TC_BWD_STATE, s);
+        tc_bwd_state_kernel<GB><<<dim3(2 * (sp.P - 1), d.H, d.B), tbs::kThreads, tbs::SMEM_BYTES, s>>>(
+            mdo_half, mv, mw, mdv, mdw, dST, dS0, dv, dw, (unsigned char *)ws, lay, sp, status, d);
+        launch_end(K_TC_BWD_STATE, s);
+    }
     return cudaGetLastError();
 }
 

@@ -465,12 +465,13 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
             // ---------------- Kb^T Delta's share of the chunk-end term: sum_t Kh_m Y3
             // with Y3 = Delta dX^T before the second products add to it
             const int r0 = 16 * I + gq;
-#pragma unroll 1
+            float y3a[16];  // the four 8-column groups of this warp's 32 channels
+            tmem_ld16x256x4(taddr(tm + TM_Y3 + 32 * Q, I * 32, 0), y3a);
+            tmem_wait_ld();
+#pragma unroll
             for (int nt = 0; nt < 4; ++nt) {
                 const int cc = 32 * Q + 8 * nt + 2 * tq;
-                float y3[4];
-                tmem_ld16x256x1(taddr(tm + TM_Y3 + 32 * Q + 8 * nt, I * 32, 0), y3);
-                tmem_wait_ld();
+                const float *y3 = y3a + 4 * nt;
                 float part[2] = {0.f, 0.f};
 #pragma unroll
                 for (int h2 = 0; h2 < 2; ++h2) {
@@ -644,14 +645,15 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
             // ---------------- mild: dq = Y1 E, dKc = Y2 E, dk = Y3 / E + dKc b; dG
             // waits in registers until every thread has read E and 1 / E
             const int r0 = 16 * I + gq;
+            float y1a[16], y2a[16], y3a[16];  // all four 8-column groups at once
+            tmem_ld16x256x4(taddr(tm + TM_Y1 + 32 * Q, I * 32, 0), y1a);
+            tmem_ld16x256x4(taddr(tm + TM_Y2 + 32 * Q, I * 32, 0), y2a);
+            tmem_ld16x256x4(taddr(tm + TM_Y3 + 32 * Q, I * 32, 0), y3a);
+            tmem_wait_ld();
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt) {
                 const int cb = 32 * Q + 8 * nt, cc = cb + 2 * tq;
-                float y1[4], y2[4], y3[4];
-                tmem_ld16x256x1(taddr(tm + TM_Y1 + cb, I * 32, 0), y1);
-                tmem_ld16x256x1(taddr(tm + TM_Y2 + cb, I * 32, 0), y2);
-                tmem_ld16x256x1(taddr(tm + TM_Y3 + cb, I * 32, 0), y3);
-                tmem_wait_ld();
+                const float *y1 = y1a + 4 * nt, *y2 = y2a + 4 * nt, *y3 = y3a + 4 * nt;
 #pragma unroll
                 for (int h2 = 0; h2 < 2; ++h2) {
                     const int r = r0 + 8 * h2;

@@ -112,8 +112,8 @@ __host__ __device__ __forceinline__ uint32_t raw32(int t, int c) {
 template <bool GB> __host__ __device__ __forceinline__ uint32_t graw(int t, int c) {
     return GB ? raw16(t, c) : raw32(t, c);
 }
-template <bool GB> constexpr int gate_box_cols() { return GB ? 64 : 32; }
-template <bool GB> constexpr uint32_t gate_tile_bytes() { return GB ? 16384u : 32768u; }
+template <bool GB> __host__ __device__ constexpr int gate_box_cols() { return GB ? 64 : 32; }
+template <bool GB> __host__ __device__ constexpr uint32_t gate_tile_bytes() { return GB ? 16384u : 32768u; }
 template <bool GB> __device__ __forceinline__ float gld1(const unsigned char *p) {
     if constexpr (GB) return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(p));
     else return *reinterpret_cast<const float *>(p);

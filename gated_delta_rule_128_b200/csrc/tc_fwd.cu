@@ -74,7 +74,7 @@ template <bool GB>  // w as bf16 (else float32)
 __global__ void __launch_bounds__(tfwd::kThreads, 1)
 tc_fwd_kernel(const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mw,
               const float *__restrict__ S0, __nv_bfloat16 *__restrict__ o, float *__restrict__ ST,
-              unsigned char *__restrict__ ws, int keep, TcWs lay, unsigned int *status, Dims d) {
+              unsigned char *__restrict__ ws, int keep, TcWs lay, SegPass sp, unsigned int *status, Dims d) {
     using namespace tfwd;
     extern __shared__ unsigned char smraw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(
@@ -85,20 +85,55 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mv, const __grid_constant__ CU
     float big = 0.f;  // largest operand magnitude seen (range check)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int vh = blockIdx.x, h = blockIdx.y, n = blockIdx.z, v0 = vh * 64;
-    // sequence n: tokens bos .. bos + T - 1 of batch row bb, chunks NC
+    const int h = blockIdx.y, n = blockIdx.z;
+    // this CTA's task (SegPass in common.cuh): a real run of segment sg, or in
+    // the first pass of a split sequence a run from zero (N_s) or from the
+    // identity with no input (M_s); vh is the 64-column half
+    int vh, sg = 0, mode = 0;  // mode 0 real, 1 from zero, 2 from the identity
+    {
+        const int x = blockIdx.x, mid = 2 * (sp.P - 2);
+        if (sp.phase == 2) { sg = 1 + (x >> 1); vh = x & 1; }
+        else if (x < 2) { vh = x; }
+        else if (x < 2 + mid) { mode = 1; sg = 1 + ((x - 2) >> 1); vh = (x - 2) & 1; }
+        else { mode = 2; sg = 1 + ((x - 2 - mid) >> 1); vh = (x - 2 - mid) & 1; }
+    }
+    const int v0 = vh * 64;
+    // sequence n: tokens bos .. bos + T - 1 of batch row bb, chunks NC; a
+    // segment narrows these to its own chunks
     const Seq sq = seq_of(d, n);
-    const int NC = sq.nc, T = sq.len, bb = sq.brow, bos = sq.bos;
+    int NC = sq.nc, T = sq.len, bos = sq.bos;
+    const int bb = sq.brow;
+    size_t tile0 = (size_t)tile_of(d, sq, h, 0);  // workspace tile of the run's first chunk
+    const size_t bhx = (size_t)n * d.H + h;
+    if (sp.P > 1) {
+        const int L = seg_len(NC, sp.P), cb = sg * L;
+        NC = min(L, NC - cb);
+        T = min(T - 64 * cb, 64 * NC);
+        bos += 64 * cb;
+        tile0 += cb;
+    }
+    // the entry state (null: zero) and where the final state goes (null: nowhere)
+    const bool first_seg = sp.P == 1 || (mode == 0 && sg == 0);
+    const float *ent = mode != 0 ? nullptr : first_seg ? (S0 ? S0 + st_off(d, n, h) : nullptr)
+                                                      : seg_buf(sp, bhx, sg, SEG_ENTRY);
+    float *fin = mode == 1 ? seg_buf(sp, bhx, sg, SEG_ZERO)
+               : mode == 2 ? seg_buf(sp, bhx, sg, SEG_MAP)
+               : (sp.P == 1 || sg == sp.P - 1) ? (ST ? ST + st_off(d, n, h) : nullptr)
+               : (sp.phase == 1 ? seg_buf(sp, bhx, 1, SEG_ENTRY) : nullptr);
+    if (mode != 0) {  // no outputs of its own
+        o = nullptr;
+        keep = 0;
+    }
+    const bool use_u = mode != 2;  // the identity run has no input
     const int quarter = warp & 3, half = warp >> 2;
     const int key = quarter * 32 + lane;          // state row (TMEM lane) of this thread
     const bool dwarp = quarter < 2;               // reads Delta (lanes 0..63), else O (64..127)
     const int ot = (half * 2 + (quarter - 2)) * 32 + lane;  // 0..127 among the O warps
-    const size_t tile0 = (size_t)tile_of(d, sq, h, 0);  // workspace tile of chunk 0
     const unsigned char *recs = ws + lay.rec + tile0 * (size_t)REC_BYTES;
     if (NC <= 0) {  // an empty sequence: S_T = S0
-        if (ST) {
-            const size_t so = st_off(d, n, h) + (size_t)(tid >> 1) * 128 + v0 + 32 * (tid & 1);
-            for (int j = 0; j < 32; ++j) ST[so + j] = S0 ? S0[so + j] : 0.f;
+        if (fin) {
+            const size_t so = (size_t)(tid >> 1) * 128 + v0 + 32 * (tid & 1);
+            for (int j = 0; j < 32; ++j) fin[so + j] = ent ? ent[so + j] : 0.f;
         }
         return;
     }
@@ -142,6 +177,12 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mv, const __grid_constant__ CU
     auto make_u = [&](int cc) {
         const int jv = ot & 7;
         unsigned char *dst = sm + OP_U + (cc & 1) * 8192;
+        if (!use_u) {  // no input: U = 0
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                *reinterpret_cast<uint4 *>(dst + sw128_chunk((ot >> 3) + 16 * i, jv, 64)) = make_uint4(0u, 0u, 0u, 0u);
+            return;
+        }
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int r = (ot >> 3) + 16 * i;
@@ -204,18 +245,21 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mv, const __grid_constant__ CU
         load_rec(0);
         if (NC > 1) load_rec(1);
     }
-    if (tid == 64) load_vw(0);
+    if (tid == 64 && use_u) load_vw(0);
 
     // ---------------- prologue: S of chunk 0 (registers, OP_S); U of chunk 0
     bool ok = mbar_wait(&bars[0], 0, kWait);
     float sreg[32];  // this thread's state row `key`, columns v0 + 32 half + j
     {
-        const size_t so = st_off(d, n, h);
 #pragma unroll
         for (int j = 0; j < 32; j += 4) {
-            float4 t = S0 ? *reinterpret_cast<const float4 *>(S0 + so + (size_t)key * 128 + v0 + 32 * half + j)
-                          : make_float4(0.f, 0.f, 0.f, 0.f);
+            float4 t = ent ? *reinterpret_cast<const float4 *>(ent + (size_t)key * 128 + v0 + 32 * half + j)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
             sreg[j] = t.x; sreg[j + 1] = t.y; sreg[j + 2] = t.z; sreg[j + 3] = t.w;
+        }
+        if (mode == 2) {  // the identity: column v0 + 32 half + j of I
+#pragma unroll
+            for (int j = 0; j < 32; ++j) sreg[j] = key == v0 + 32 * half + j ? 1.f : 0.f;
         }
         // the operand state s S in chunk 0's frame
         const float s0 = reinterpret_cast<const float *>(sm + STG + S_FAC)[128 + key];
@@ -230,10 +274,10 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mv, const __grid_constant__ CU
         }
     }
     if (!dwarp) {
-        ok = mbar_wait(&bars[2], 0, kWait) && ok;
+        if (use_u) ok = mbar_wait(&bars[2], 0, kWait) && ok;
         make_u(0);
         named_sync(2, 128);  // raw v, w consumed
-        if (tid == 64 && NC > 1) load_vw(1);
+        if (tid == 64 && NC > 1 && use_u) load_vw(1);
     }
     fence_proxy_async();
     fence_before_sync();
@@ -291,11 +335,11 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mv, const __grid_constant__ CU
             // ---------------- previous chunk's O; next chunk's U
             if (c > 0) store_o(c - 1);
             if (c + 1 < NC) {
-                ok = mbar_wait(&bars[2], (c + 1) & 1, kWait) && ok;
+                if (use_u) ok = mbar_wait(&bars[2], (c + 1) & 1, kWait) && ok;
                 make_u(c + 1);
                 fence_proxy_async();
                 named_sync(2, 128);  // raw v, w consumed
-                if (tid == 64 && c + 2 < NC) load_vw(c + 2);
+                if (tid == 64 && c + 2 < NC && use_u) load_vw(c + 2);
             }
         }
         // ---------------- S_next = gamma S + Kb^T Delta
@@ -326,8 +370,8 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mv, const __grid_constant__ CU
                     st_h8(sm + OP_S + sw128_chunk(key, 4 * half + jj, 128), xv + 8 * jj);
                     big = absmax8(xv + 8 * jj, big);
                 }
-            } else if (ST) {
-                float *dst = ST + st_off(d, n, h) + (size_t)key * 128 + v0 + 32 * half;
+            } else if (fin) {
+                float *dst = fin + (size_t)key * 128 + v0 + 32 * half;
 #pragma unroll
                 for (int j = 0; j < 32; j += 4)
                     *reinterpret_cast<float4 *>(dst + j) = make_float4(sreg[j], sreg[j + 1], sreg[j + 2], sreg[j + 3]);
@@ -370,6 +414,9 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mv, const __grid_constant__ CU
 cudaError_t tc_prep_launch(const void *q, const void *k, const void *g, const void *b, void *ws,
                            unsigned int *status, const Dims &d, cudaStream_t s);
 
+// the link step between the passes (seg_link.cu)
+cudaError_t seg_link_launch(const SegPass &sp, int nbh, bool backward, cudaStream_t s);
+
 template <bool GB>
 static cudaError_t tc_fwd_run(const void *v, const void *w, const float *S0, void *o, float *ST,
                               void *ws, int keep, unsigned int *status, const Dims &d, cudaStream_t s) {
@@ -380,10 +427,24 @@ static cudaError_t tc_fwd_run(const void *v, const void *w, const float *S0, voi
     cudaError_t e = cudaFuncSetAttribute(tc_fwd_kernel<GB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)tfwd::SMEM_BYTES);
     if (e != cudaSuccess) return e;
+    const TcWs lay = tc_ws_layout(d);
+    SegPass sp{1, 0, nullptr};
+    // a split sequence needs the workspace that keeps the forward (its segment buffers)
+    if (lay.P > 1 && keep) sp = SegPass{lay.P, 1, reinterpret_cast<float *>(static_cast<char *>(ws) + lay.seg)};
     launch_begin(K_TC_FWD, s);
-    tc_fwd_kernel<GB><<<dim3(2, d.H, num_seqs(d)), tfwd::kThreads, tfwd::SMEM_BYTES, s>>>(
-        mv, mw, S0, (__nv_bfloat16 *)o, ST, (unsigned char *)ws, keep, tc_ws_layout(d), status, d);
+    tc_fwd_kernel<GB><<<dim3(sp.P > 1 ? 2 + 4 * (sp.P - 2) : 2, d.H, num_seqs(d)), tfwd::kThreads,
+                        tfwd::SMEM_BYTES, s>>>(mv, mw, S0, (__nv_bfloat16 *)o, ST, (unsigned char *)ws, keep,
+                                               lay, sp, status, d);
     launch_end(K_TC_FWD, s);
+    if (sp.P > 1) {
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if ((e = seg_link_launch(sp, d.B * d.H, false, s)) != cudaSuccess) return e;
+        sp.phase = 2;
+        launch_begin(K_TC_FWD, s);
+        tc_fwd_kernel<GB><<<dim3(2 * (sp.P - 1), d.H, d.B), tfwd::kThreads, tfwd::SMEM_BYTES, s>>>(
+            mv, mw, S0, (__nv_bfloat16 *)o, ST, (unsigned char *)ws, keep, lay, sp, status, d);
+        launch_end(K_TC_FWD, s);
+    }
     return cudaGetLastError();
 }
 

@@ -270,6 +270,30 @@ def test_full_workload_sampled_heads(index):
     compare(gpu, ref, wl.io, names, pairs=SAMPLE[index])
 
 
+# ------------------------------------------- segment-parallel state passes
+
+@pytest.mark.parametrize("T", [768, 837, 1024])
+def test_split_state_passes(T):
+    """Few (b, h) and many chunks: the state passes split each sequence into
+    segments (maps M_s, N_s in parallel, a link, then the segments' real runs).
+    T = 768, 837 and 1024 with B = 1, H = 2 take 3, 4 and 4 segments (837: a
+    short last segment with a ragged tail).  Against the oracle."""
+    x = workloads.draw(1, T, 2, 128, 128, 980 + T, s0_std=0.1, with_dST=True)
+    gpu = gpu_fwd_bwd(x, "bf16", 64)
+    ref = oracle_fwd_bwd(x, "bf16")
+    compare(gpu, ref, "bf16", ("o", "ST") + GRADS)
+
+
+def test_split_state_passes_steep_decay_and_bf16_gates():
+    """The split passes under a steep decay (g = 4 logsigmoid) with bf16 gates."""
+    x = workloads.draw(1, 1024, 2, 128, 128, 985, s0_std=0.1, with_dST=True)
+    gen = torch.Generator().manual_seed(986)
+    x["g"] = torch.nn.functional.logsigmoid(torch.randn(x["g"].shape, generator=gen)) * 4
+    gpu = gpu_fwd_bwd(x, "bf16", 64, gates="bf16")
+    ref = oracle_fwd_bwd(x, "bf16", gates="bf16")
+    compare(gpu, ref, "bf16", ("o", "ST") + GRADS)
+
+
 # --------------------------------------------------------------- bf16 gates
 
 @pytest.mark.parametrize("index", [1, 2])
