@@ -53,11 +53,13 @@ constexpr uint32_t REC = RR + 24576;  // the tile's record, laid out as in the w
 constexpr uint32_t OP_WQ = REC + REC_WQ;  // [Kc; Qb], later [-W; Qb]
 constexpr uint32_t OP_KB = REC + REC_KH;
 constexpr uint32_t OP_T = REC + REC_T, OP_P = REC + REC_P, FAC = REC + REC_FAC;
-constexpr uint32_t TOT = OP_T;        // 8-row totals of G [2][8][128] f32, before T and P are written
 // float32 scratch of the inversion, over CO / RR once the products have read them
 constexpr uint32_t SCR_A = CO, SCR_T = CO + 64 * 65 * 4, SCR_M = SCR_T + 64 * 65 * 4;
 constexpr uint32_t MISC = REC + REC_BYTES;  // mbarriers, TMEM slot
-constexpr uint32_t SMEM_BYTES = MISC + 128 + 1024;
+// 8-row totals of G [2][8][128] f32, outside the record so that they can be
+// formed while the previous tile's record is still leaving
+constexpr uint32_t TOT = MISC + 128;
+constexpr uint32_t SMEM_BYTES = TOT + 8192 + 1024;
 constexpr uint32_t TM_C = 0, TM_W = 128;  // the three block products (96 columns); W
 __host__ __device__ constexpr uint32_t tm_coff(int I) { return I <= 1 ? 0u : (I == 2 ? 16u : 48u); }
 constexpr uint32_t ID_KM128 = idesc_f16(64, 128, false, true);
@@ -88,14 +90,18 @@ __device__ __forceinline__ void tile_mma(float *c, const float *X, int r0, int k
 // barrier.
 __device__ __forceinline__ void invert_unit_lower(const float *sA, float *sT, float *sM, int tid) {
     if (tid < 64) {
+        // column cl of the block's inverse, right-looking: once x[j] is final,
+        // every later row takes its term at once, so the dependent chain is
+        // 16 multiply-adds long instead of 120
         const int o16 = (tid >> 4) * 16, cl = tid & 15;
         float x[16];
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            float acc = r == cl ? 1.f : 0.f;
+        for (int r = 0; r < 16; ++r) x[r] = r == cl ? 1.f : 0.f;
 #pragma unroll
-            for (int j = 0; j < r; ++j) acc -= sA[(o16 + r) * 65 + o16 + j] * x[j];
-            x[r] = acc;
+        for (int j = 0; j < 15; ++j) {
+            const float xj = x[j];
+#pragma unroll
+            for (int r = j + 1; r < 16; ++r) x[r] = fmaf(-sA[(o16 + r) * 65 + o16 + j], xj, x[r]);
         }
 #pragma unroll
         for (int r = 0; r < 16; ++r) sT[(o16 + r) * 65 + o16 + cl] = x[r];
@@ -207,7 +213,6 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
     for (int it = blockIdx.x; it < ntiles; it += gridDim.x, ++n) {
         unsigned char *rec = ws + lay.rec + (size_t)it * REC_BYTES;
         bool ok = mbar_wait(&bars[0], n & 1, kWait);
-        if (tid == 0) bulk_wait_read();  // the previous tile's record has left shared memory
         if (__syncthreads_or(!ok)) { abort = true; break; }
         if (d.cu) {  // packed sequences: rows past the sequence's end belong to the next one
             int tn, th, tc;
@@ -239,6 +244,7 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
             *reinterpret_cast<float4 *>(tot + warp * 128 + fc4) = make_float4(run[0], run[1], run[2], run[3]);
             *reinterpret_cast<float4 *>(totc + warp * 128 + fc4) = make_float4(runc[0], runc[1], runc[2], runc[3]);
         }
+        if (tid == 0) bulk_wait_read();  // the previous tile's record has left shared memory
         __syncthreads();
         // ---------------- mild tile?  Then the whole chunk fits one frame
         // relative to its row 31: every factor e^(+-(G - G_31)) stays within
