@@ -31,6 +31,9 @@ LIB_PATH = os.path.join(PKG, "libgdn2.so")
 
 GDN2_IO_F32 = 0
 GDN2_IO_BF16 = 1
+GDN2_GATE_LOGITS = 0x100   # g, b, w are logits: g = logsigmoid, b = sigmoid (x2 with B_X2), w = sigmoid
+GDN2_GATE_B_X2 = 0x200
+GATE_FLAGS = {"activated": 0, "logits": GDN2_GATE_LOGITS, "logits_b2": GDN2_GATE_LOGITS | GDN2_GATE_B_X2}
 STATUS = {0: "GDN2_OK", 1: "GDN2_ERR_INVALID_ARG", 2: "GDN2_ERR_UNSUPPORTED",
           3: "GDN2_ERR_WORKSPACE", 4: "GDN2_ERR_CUDA", 5: "GDN2_ERR_TIMEOUT",
           6: "GDN2_ERR_RANGE"}
@@ -117,13 +120,17 @@ def _io_of(t: torch.Tensor) -> int:
     raise TypeError(f"q/k/v must be float32 or bfloat16, got {t.dtype}")
 
 
-def _gate_io_of(g: torch.Tensor, b: torch.Tensor, w: torch.Tensor) -> int:
+def _gate_io_of(g: torch.Tensor, b: torch.Tensor, w: torch.Tensor, gates: str = "activated") -> int:
+    """The gate_io argument: the gates' dtype, or-ed with the flags of the
+    gate encoding ("activated" values, "logits", or "logits_b2")."""
     if not (g.dtype == b.dtype == w.dtype):
         raise TypeError(f"g, b, w must share one dtype, got {g.dtype}, {b.dtype}, {w.dtype}")
+    if gates not in GATE_FLAGS:
+        raise ValueError(f"gates must be one of {sorted(GATE_FLAGS)}, got {gates!r}")
     if g.dtype == torch.bfloat16:
-        return GDN2_IO_BF16
+        return GDN2_IO_BF16 | GATE_FLAGS[gates]
     if g.dtype == torch.float32:
-        return GDN2_IO_F32
+        return GDN2_IO_F32 | GATE_FLAGS[gates]
     raise TypeError(f"g/b/w must be float32 or bfloat16, got {g.dtype}")
 
 
@@ -276,7 +283,7 @@ def _alloc_ws(n: int, fn: str, device) -> torch.Tensor:
 
 def forward(q, k, v, g, b, w, S0=None, *, chunk: int = 64, want_state: bool = True,
             ws: Optional[torch.Tensor] = None, for_bwd: bool = False, stream=None,
-            check: bool = True):
+            check: bool = True, gates: str = "activated"):
     """Returns (o, S_T or None, ws).  Shapes: q, k, g, b [B,T,H,dk]; v, w [B,T,H_v,dv]
     (H_v a multiple of H: grouped value heads); S0, S_T [B,H_v,dk,dv].  g, b, w
     may be bfloat16 (all three) on the tensor-core path.
@@ -286,7 +293,7 @@ def forward(q, k, v, g, b, w, S0=None, *, chunk: int = 64, want_state: bool = Tr
     asynchronous (read the status later with check_device_status)."""
     B, T, H, dk = q.shape
     Hv, dv = v.shape[2], v.shape[3]
-    io, gio = _io_of(q), _gate_io_of(g, b, w)
+    io, gio = _io_of(q), _gate_io_of(g, b, w, gates)
     if ws is None:
         ws = _alloc_ws(gdn2_workspace_bytes_ex(B, T, H, Hv, dk, dv, chunk, io, gio, for_bwd),
                        "gdn2_workspace_bytes_ex", q.device)
@@ -301,12 +308,14 @@ def forward(q, k, v, g, b, w, S0=None, *, chunk: int = 64, want_state: bool = Tr
 
 def backward(q, k, v, g, b, w, S0, dO, dST=None, *, chunk: int = 64,
              ws: Optional[torch.Tensor] = None, ws_has_fwd: bool = False,
-             want_dS0: bool = True, stream=None, check: bool = True) -> Dict[str, torch.Tensor]:
+             want_dS0: bool = True, stream=None, check: bool = True,
+             gates: str = "activated") -> Dict[str, torch.Tensor]:
     """Gradients dq, dk, dv, dg, db, dw, dS0 (None unless want_dS0); dg, db, dw
-    take the gates' dtype.  check as in forward()."""
+    take the gates' dtype (and are of the logits with gates="logits").  check
+    as in forward()."""
     B, T, H, dk = q.shape
     Hv, dv = v.shape[2], v.shape[3]
-    io, gio = _io_of(q), _gate_io_of(g, b, w)
+    io, gio = _io_of(q), _gate_io_of(g, b, w, gates)
     if ws is None:
         ws = _alloc_ws(gdn2_workspace_bytes_ex(B, T, H, Hv, dk, dv, chunk, io, gio, True),
                        "gdn2_workspace_bytes_ex", q.device)
@@ -325,14 +334,14 @@ def backward(q, k, v, g, b, w, S0, dO, dST=None, *, chunk: int = 64,
 
 def forward_varlen(q, k, v, g, b, w, cu_seqlens, S0=None, *, chunk: int = 64,
                    want_state: bool = True, ws: Optional[torch.Tensor] = None,
-                   for_bwd: bool = False, stream=None, check: bool = True):
+                   for_bwd: bool = False, stream=None, check: bool = True, gates: str = "activated"):
     """Packed sequences: q, k, g, b [1,T,H,dk]; v, w [1,T,H_v,dv]; cu_seqlens
     int32 [N+1] on the device; S0 [N,H_v,dk,dv] or None.  Returns (o, S_T
     [N,...] or None, ws)."""
     _, T, H, dk = q.shape
     Hv, dv = v.shape[2], v.shape[3]
     N = cu_seqlens.numel() - 1
-    io, gio = _io_of(q), _gate_io_of(g, b, w)
+    io, gio = _io_of(q), _gate_io_of(g, b, w, gates)
     if ws is None:
         ws = _alloc_ws(gdn2_workspace_bytes_varlen(N, T, H, Hv, dk, dv, chunk, io, gio, for_bwd),
                        "gdn2_workspace_bytes_varlen", q.device)
@@ -347,12 +356,13 @@ def forward_varlen(q, k, v, g, b, w, cu_seqlens, S0=None, *, chunk: int = 64,
 
 def backward_varlen(q, k, v, g, b, w, cu_seqlens, S0, dO, dST=None, *, chunk: int = 64,
                     ws: Optional[torch.Tensor] = None, ws_has_fwd: bool = False,
-                    want_dS0: bool = True, stream=None, check: bool = True) -> Dict[str, torch.Tensor]:
+                    want_dS0: bool = True, stream=None, check: bool = True,
+                    gates: str = "activated") -> Dict[str, torch.Tensor]:
     """Gradients of forward_varlen: dq, dk, dv, dg, db, dw and dS0 [N,...]."""
     _, T, H, dk = q.shape
     Hv, dv = v.shape[2], v.shape[3]
     N = cu_seqlens.numel() - 1
-    io, gio = _io_of(q), _gate_io_of(g, b, w)
+    io, gio = _io_of(q), _gate_io_of(g, b, w, gates)
     if ws is None:
         ws = _alloc_ws(gdn2_workspace_bytes_varlen(N, T, H, Hv, dk, dv, chunk, io, gio, True),
                        "gdn2_workspace_bytes_varlen", q.device)
@@ -369,13 +379,13 @@ def backward_varlen(q, k, v, g, b, w, cu_seqlens, S0, dO, dST=None, *, chunk: in
     return out
 
 
-def decode_step(q, k, v, g, b, w, S, o=None, stream=None):
+def decode_step(q, k, v, g, b, w, S, o=None, stream=None, gates: str = "activated"):
     """One token for N sequences: q, k, g, b [N,H,dk]; v, w [N,H_v,dv]; S
     [N,H_v,dk,dv] float32, updated in place.  Returns o [N,H_v,dv]."""
     N, H, dk = q.shape
     Hv, dv = v.shape[1], v.shape[2]
     if o is None:
         o = torch.empty(N, Hv, dv, dtype=q.dtype, device=q.device)
-    gdn2_decode_step_ex(q, k, v, g, b, w, S, o, N, H, Hv, dk, dv, _io_of(q), _gate_io_of(g, b, w),
+    gdn2_decode_step_ex(q, k, v, g, b, w, S, o, N, H, Hv, dk, dv, _io_of(q), _gate_io_of(g, b, w, gates),
                         stream)
     return o

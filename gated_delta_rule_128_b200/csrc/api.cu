@@ -26,7 +26,7 @@ cudaError_t simt_bwd_launch(const void *, const void *, const void *, const floa
                             const void *, const float *, void *, void *, void *, float *, float *,
                             float *, float *, void *, const Dims &, cudaStream_t);
 cudaError_t decode_launch(const void *, const void *, const void *, const void *, const void *,
-                          const void *, float *, void *, int, int, int, int, int, gdn2_io, gdn2_io,
+                          const void *, float *, void *, int, int, int, int, int, gdn2_io, gdn2_io, int,
                           cudaStream_t);
 cudaError_t tc_fwd_launch(const void *, const void *, const void *, const void *, const void *,
                           const void *, const float *, void *, float *, void *, int,
@@ -116,7 +116,7 @@ static gdn2_status check_dims(int B, int T, int H, int dk, int dv, int chunk, gd
 }
 
 static Dims make_dims(int B, int T, int H, int dk, int dv, int chunk) {
-    return Dims{B, T, H, dk, dv, chunk, (T + chunk - 1) / chunk, 0};
+    return Dims{B, T, H, dk, dv, chunk, (T + chunk - 1) / chunk, 0, 0};
 }
 
 // every required pointer non-null and 16-byte aligned; optional ones aligned
@@ -169,10 +169,18 @@ size_t gdn2_workspace_bytes(int B, int T, int H, int d_k, int d_v, int chunk, gd
     return ws_bytes_for(make_dims(B, T, H, d_k, d_v, chunk), io, for_bwd);
 }
 
-// gate tensors in bf16 need the tensor-core path
+// gate_io: the gate tensors' type in its low byte, GDN2_GATE_* flags above it
+static gdn2_io gate_type(gdn2_io gate_io) { return (gdn2_io)((int)gate_io & 0xff); }
+static int gate_flags(gdn2_io gate_io) { return ((int)gate_io >> 8) & 3; }
+static bool gate_io_valid(gdn2_io gate_io) {
+    const int t = (int)gate_io & 0xff, f = (int)gate_io >> 8;
+    return (t == GDN2_IO_F32 || t == GDN2_IO_BF16) && (f & ~3) == 0 && (f != 2);  // B_X2 needs LOGITS
+}
+// gate tensors in bf16, and gate logits, need the tensor-core path
 static gdn2_status check_gate_io(const Dims &d, gdn2_io io, gdn2_io gate_io) {
-    if (gate_io != GDN2_IO_F32 && gate_io != GDN2_IO_BF16) return GDN2_ERR_INVALID_ARG;
-    if (gate_io == GDN2_IO_BF16 && !use_tc(d, io)) return GDN2_ERR_UNSUPPORTED;
+    if (!gate_io_valid(gate_io)) return GDN2_ERR_INVALID_ARG;
+    if ((gate_type(gate_io) == GDN2_IO_BF16 || gate_flags(gate_io) != 0) && !use_tc(d, io))
+        return GDN2_ERR_UNSUPPORTED;
     return GDN2_OK;
 }
 
@@ -295,7 +303,8 @@ static gdn2_status plan_call(Call &c, int B, int T, int H, int H_v, int dk, int 
     c.for_bwd = for_bwd;
     c.d = make_dims(packed ? 1 : B, T, H, dk, dvw, chunk);
     if ((st = check_gate_io(c.d, io, gate_io)) != GDN2_OK) return st;
-    c.d.gb = gate_io == GDN2_IO_BF16;
+    c.d.gb = gate_type(gate_io) == GDN2_IO_BF16;
+    c.d.act = gate_flags(gate_io);
     size_t o;
     if (packed) {
         if (N < 1 || ((uintptr_t)cu & 3u) != 0) return GDN2_ERR_INVALID_ARG;
@@ -341,7 +350,8 @@ static gdn2_status fwd_call(Call &c, const void *q, const void *k, const void *v
     if (!c.for_bwd) {
         Call cb;
         if (plan_call(cb, c.d.B, c.d.T, c.d.H, c.d.H * c.G, c.d.dk, c.d.dv / c.G, c.d.C, c.io,
-                      c.d.gb ? GDN2_IO_BF16 : GDN2_IO_F32, c.d.N > 0, c.d.N, c.d.cu, 1) == GDN2_OK &&
+                      (gdn2_io)((c.d.gb ? GDN2_IO_BF16 : GDN2_IO_F32) | (c.d.act << 8)), c.d.N > 0, c.d.N,
+                      c.d.cu, 1) == GDN2_OK &&
             ws_bytes >= cb.total)
             full = cb;
     }
@@ -504,15 +514,15 @@ gdn2_status gdn2_decode_step_ex(const void *q, const void *k, const void *v, con
                                 const void *b, const void *w, float *S, void *o, int N, int H, int H_v,
                                 int d_k, int d_v, gdn2_io io, gdn2_io gate_io, gdn2_stream_t stream) {
     if (N < 1 || H < 1 || (io != GDN2_IO_F32 && io != GDN2_IO_BF16)) return GDN2_ERR_INVALID_ARG;
-    if (gate_io != GDN2_IO_F32 && gate_io != GDN2_IO_BF16) return GDN2_ERR_INVALID_ARG;
+    if (!gate_io_valid(gate_io)) return GDN2_ERR_INVALID_ARG;
     const int G = value_groups(H, H_v);
     if (G == 0) return GDN2_ERR_INVALID_ARG;
     if (!supported_d(d_k) || !supported_d(d_v)) return GDN2_ERR_UNSUPPORTED;
     if ((long long)N * H * G > 0x7fffffffLL) return GDN2_ERR_UNSUPPORTED;
     gdn2_status st = check_ptrs({q, k, v, g, b, w, S, o}, {});
     if (st != GDN2_OK) return st;
-    return cuda_status(decode_launch(q, k, v, g, b, w, S, o, N, H, G, d_k, d_v, io, gate_io,
-                                     (cudaStream_t)stream));
+    return cuda_status(decode_launch(q, k, v, g, b, w, S, o, N, H, G, d_k, d_v, io, gate_type(gate_io),
+                                     gate_flags(gate_io), (cudaStream_t)stream));
 }
 
 gdn2_status gdn2_decode_step(const void *q, const void *k, const void *v, const float *g,

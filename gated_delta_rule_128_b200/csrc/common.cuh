@@ -16,6 +16,10 @@ constexpr int kMaxChunk = 64;  // largest chunk
 struct Dims {
     int B, T, H, dk, dv, C, NC;
     int gb;  // gate tensors g, b, w and dg, db, dw in bf16 (tensor-core path), else float32
+    // gate logits (tensor-core path and decode): bit 0 set: g, b, w arrive as
+    // pre-activation logits and are activated on load (GateAct below), and
+    // dg, db, dw leave as gradients of the logits; bit 1: b = 2 sigmoid(x)
+    int act;
     // Packed variable-length sequences (tensor-core path): N sequences whose
     // tokens lie at rows cu[n] .. cu[n + 1] - 1 of a B = 1 batch, cu (device,
     // N + 1 entries) as given by the caller, co (workspace, N + 1 entries) the
@@ -67,6 +71,45 @@ __device__ __forceinline__ void tile_decode(const Dims &d, int it, int &n, int &
     h = rem / nc;
     c = rem - h * nc;
 }
+
+// ---- gate activations ("Gated DeltaNet-2", LIT-802 review, Key takeaways 1:
+// the erase and write gates are sigmoid outputs, 2 sigmoid for erase
+// eigenvalues in [-1, 1]; the decay a log-sigmoid) for calls that pass logits
+__device__ __forceinline__ float sigmoid_act(float x) { return 1.f / (1.f + __expf(-x)); }
+// log(sigmoid(x)) = min(x, 0) - log(1 + e^-|x|), without overflow
+__device__ __forceinline__ float logsigmoid_act(float x) { return fminf(x, 0.f) - log1pf(__expf(-fabsf(x))); }
+struct GateAct {
+    bool on;      // logits in, logit gradients out
+    float bscale; // 1 or 2
+    __device__ __forceinline__ float g(float x) const { return on ? logsigmoid_act(x) : x; }
+    __device__ __forceinline__ float b(float x) const { return on ? bscale * sigmoid_act(x) : x; }
+    __device__ __forceinline__ float w(float x) const { return on ? sigmoid_act(x) : x; }
+    // d(activation)/dx at logit x: g' = sigmoid(-x), b' = s sigma (1 - sigma), w' = sigma (1 - sigma)
+    __device__ __forceinline__ float dg(float x) const { return on ? sigmoid_act(-x) : 1.f; }
+    __device__ __forceinline__ float db(float x) const {
+        if (!on) return 1.f;
+        const float s = sigmoid_act(x);
+        return bscale * s * (1.f - s);
+    }
+    __device__ __forceinline__ float dw(float x) const {
+        if (!on) return 1.f;
+        const float s = sigmoid_act(x);
+        return s * (1.f - s);
+    }
+};
+__device__ __forceinline__ GateAct gate_act(int act) { return GateAct{(act & 1) != 0, (act & 2) ? 2.f : 1.f}; }
+__device__ __forceinline__ float4 act_g4(const GateAct &a, float4 v) {
+    return a.on ? make_float4(a.g(v.x), a.g(v.y), a.g(v.z), a.g(v.w)) : v;
+}
+__device__ __forceinline__ float4 act_b4(const GateAct &a, float4 v) {
+    return a.on ? make_float4(a.b(v.x), a.b(v.y), a.b(v.z), a.b(v.w)) : v;
+}
+__device__ __forceinline__ float4 act_w4(const GateAct &a, float4 v) {
+    return a.on ? make_float4(a.w(v.x), a.w(v.y), a.w(v.z), a.w(v.w)) : v;
+}
+__device__ __forceinline__ float2 act_g2(const GateAct &a, float2 v) { return a.on ? make_float2(a.g(v.x), a.g(v.y)) : v; }
+__device__ __forceinline__ float2 act_b2(const GateAct &a, float2 v) { return a.on ? make_float2(a.b(v.x), a.b(v.y)) : v; }
+__device__ __forceinline__ float2 act_w2(const GateAct &a, float2 v) { return a.on ? make_float2(a.w(v.x), a.w(v.y)) : v; }
 
 // ---- element access in the io type (float or bf16), computing in float
 template <typename E> __device__ __forceinline__ float ldx(const E *p, size_t i);

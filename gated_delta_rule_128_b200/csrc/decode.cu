@@ -28,12 +28,14 @@ template <int CL> __device__ __forceinline__ void vstore(float *p, const float *
     else { *p = x[0]; }
 }
 
-// E: the io type of q, k, v, o; GE: the gate type of g, b, w (float or bf16)
-template <typename E, typename GE, int DK, int DV>
+// E: the io type of q, k, v, o; GE: the gate type of g, b, w (float or bf16);
+// ACT: gate logits (GateAct)
+template <typename E, typename GE, bool ACT, int DK, int DV>
 __global__ void __launch_bounds__(kDecThreads)
 decode_step_kernel(const E *__restrict__ q, const E *__restrict__ k, const E *__restrict__ v,
                    const GE *__restrict__ g, const GE *__restrict__ b,
-                   const GE *__restrict__ w, float *__restrict__ S, E *__restrict__ o, int H, int G) {
+                   const GE *__restrict__ w, float *__restrict__ S, E *__restrict__ o, int H, int G, int act) {
+    const GateAct ga = ACT ? gate_act(act) : GateAct{false, 1.f};  // logits in: activated on load
     constexpr int RW = DK / kDecWarps;  // rows per warp
     constexpr int CL = DV / 32;         // columns per lane
     __shared__ float sk[DK], sbk[DK], sq[DK], sa[DK], su[DV], sdelta[DV];
@@ -52,9 +54,9 @@ decode_step_kernel(const E *__restrict__ q, const E *__restrict__ k, const E *__
 
     for (int i = tid; i < DK; i += kDecThreads) {
         float kv = ldx(k, hk + i), qv = ldx(q, hk + i);
-        sk[i] = kv; sq[i] = qv; sbk[i] = ldx(b, hk + i) * kv; sa[i] = __expf(ldx(g, hk + i));
+        sk[i] = kv; sq[i] = qv; sbk[i] = ga.b(ldx(b, hk + i)) * kv; sa[i] = __expf(ga.g(ldx(g, hk + i)));
     }
-    for (int j = tid; j < DV; j += kDecThreads) su[j] = ldx(w, hvo + j) * ldx(v, hvo + j);
+    for (int j = tid; j < DV; j += kDecThreads) su[j] = ga.w(ldx(w, hvo + j)) * ldx(v, hvo + j);
     if (warp == 0) {
         float acc = 0.f;
         for (int i = lane; i < DK; i += 32) acc += ldx(k, hk + i) * ldx(q, hk + i);
@@ -103,24 +105,24 @@ decode_step_kernel(const E *__restrict__ q, const E *__restrict__ k, const E *__
     }
 }
 
-template <typename E, typename GE, int DK, int DV>
+template <typename E, typename GE, bool ACT, int DK, int DV>
 static cudaError_t launch_dec(const void *q, const void *k, const void *v, const void *g,
                               const void *b, const void *w, float *S, void *o, int N, int H, int G,
-                              cudaStream_t s) {
+                              int act, cudaStream_t s) {
     launch_begin(K_DECODE, s);
-    decode_step_kernel<E, GE, DK, DV><<<(unsigned)N * (unsigned)(H * G), kDecThreads, 0, s>>>(
+    decode_step_kernel<E, GE, ACT, DK, DV><<<(unsigned)N * (unsigned)(H * G), kDecThreads, 0, s>>>(
         (const E *)q, (const E *)k, (const E *)v, (const GE *)g, (const GE *)b, (const GE *)w, S,
-        (E *)o, H, G);
+        (E *)o, H, G, act);
     launch_end(K_DECODE, s);
     return cudaGetLastError();
 }
 
-template <typename E, typename GE>
+template <typename E, typename GE, bool ACT>
 static cudaError_t dispatch_dec(const void *q, const void *k, const void *v, const void *g,
                                 const void *b, const void *w, float *S, void *o, int N, int H, int G,
-                                int dk, int dv, cudaStream_t s) {
+                                int act, int dk, int dv, cudaStream_t s) {
 #define GDN2_DEC(DK_, DV_) \
-    if (dk == DK_ && dv == DV_) return launch_dec<E, GE, DK_, DV_>(q, k, v, g, b, w, S, o, N, H, G, s);
+    if (dk == DK_ && dv == DV_) return launch_dec<E, GE, ACT, DK_, DV_>(q, k, v, g, b, w, S, o, N, H, G, act, s);
     GDN2_DEC(32, 32) GDN2_DEC(32, 64) GDN2_DEC(32, 128)
     GDN2_DEC(64, 32) GDN2_DEC(64, 64) GDN2_DEC(64, 128)
     GDN2_DEC(128, 32) GDN2_DEC(128, 64) GDN2_DEC(128, 128)
@@ -128,15 +130,24 @@ static cudaError_t dispatch_dec(const void *q, const void *k, const void *v, con
     return cudaErrorInvalidValue;
 }
 
-cudaError_t decode_launch(const void *q, const void *k, const void *v, const void *g,
-                          const void *b, const void *w, float *S, void *o, int N, int H, int G,
-                          int dk, int dv, gdn2_io io, gdn2_io gate_io, cudaStream_t s) {
+template <bool ACT>
+static cudaError_t decode_types(const void *q, const void *k, const void *v, const void *g, const void *b,
+                                const void *w, float *S, void *o, int N, int H, int G, int dk, int dv,
+                                gdn2_io io, gdn2_io gate_io, int act, cudaStream_t s) {
     using BF = __nv_bfloat16;
     if (io == GDN2_IO_BF16)
-        return gate_io == GDN2_IO_BF16 ? dispatch_dec<BF, BF>(q, k, v, g, b, w, S, o, N, H, G, dk, dv, s)
-                                       : dispatch_dec<BF, float>(q, k, v, g, b, w, S, o, N, H, G, dk, dv, s);
-    return gate_io == GDN2_IO_BF16 ? dispatch_dec<float, BF>(q, k, v, g, b, w, S, o, N, H, G, dk, dv, s)
-                                   : dispatch_dec<float, float>(q, k, v, g, b, w, S, o, N, H, G, dk, dv, s);
+        return gate_io == GDN2_IO_BF16
+                   ? dispatch_dec<BF, BF, ACT>(q, k, v, g, b, w, S, o, N, H, G, act, dk, dv, s)
+                   : dispatch_dec<BF, float, ACT>(q, k, v, g, b, w, S, o, N, H, G, act, dk, dv, s);
+    return gate_io == GDN2_IO_BF16 ? dispatch_dec<float, BF, ACT>(q, k, v, g, b, w, S, o, N, H, G, act, dk, dv, s)
+                                   : dispatch_dec<float, float, ACT>(q, k, v, g, b, w, S, o, N, H, G, act, dk, dv, s);
+}
+
+cudaError_t decode_launch(const void *q, const void *k, const void *v, const void *g,
+                          const void *b, const void *w, float *S, void *o, int N, int H, int G,
+                          int dk, int dv, gdn2_io io, gdn2_io gate_io, int act, cudaStream_t s) {
+    return act ? decode_types<true>(q, k, v, g, b, w, S, o, N, H, G, dk, dv, io, gate_io, act, s)
+               : decode_types<false>(q, k, v, g, b, w, S, o, N, H, G, dk, dv, io, gate_io, act, s);
 }
 
 }  // namespace gdn2

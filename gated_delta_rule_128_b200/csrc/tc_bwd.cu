@@ -63,7 +63,7 @@ static_assert(SMEM_BYTES <= 232448, "shared memory");
 // the accumulators and form the operands and outputs; warp 8 issues the
 // products (an issuing thread is held for about as long as the products
 // run); warp 9 requests every copy, so that neither delays the readouts.
-template <bool GB>  // w and dw as bf16 (else float32)
+template <bool GB, bool ACT>  // w and dw as bf16 (else float32); ACT: gate logits (GateAct)
 __global__ void __launch_bounds__(tbs::kThreads, 1)
 tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_constant__ CUtensorMap mv,
                     const __grid_constant__ CUtensorMap mw, const __grid_constant__ CUtensorMap mdv,
@@ -110,6 +110,7 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
     // the exit gradient (null: zero) and where the entry gradient goes (null:
     // nowhere); only real runs write dv, dw, -dU and dS'
     const bool real = mode == 0;
+    const GateAct ga = ACT ? gate_act(d.act) : GateAct{false, 1.f};  // logits in: w activated on load, dw by the chain rule
     const float *ext = !real ? nullptr
                      : (sp.P == 1 || sg == sp.P - 1) ? (dST ? dST + st_off(d, n, h) : nullptr)
                      : seg_buf(sp, bhx, sg, SEG_ENTRY);
@@ -230,9 +231,11 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
                 unsigned char *pw = sm + VW + (GB ? sw128_off(rr, c, 64)
                                                   : (c >> 5) * 8192 + sw128_chunk(rr, (c & 31) >> 2, 64) + (c & 3) * 4);
                 const float2 vf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(pv));
-                const float2 wf = gld2<GB>(pw);
+                const float2 wx = gld2<GB>(pw);  // w, or its logit
+                const float2 wf = act_w2(ga, wx);
                 *reinterpret_cast<uint32_t *>(pv) = pack_bf16(u0 * wf.x, u1 * wf.y);
-                gst2<GB>(pw, u0 * vf.x, u1 * vf.y);
+                // dw = dU v, times dw/dx for logits
+                gst2<GB>(pw, u0 * vf.x * ga.dw(wx.x), u1 * vf.y * ga.dw(wx.y));
                 *reinterpret_cast<uint32_t *>(sm + NDU + sw128_off(rr, c, 64)) = pack_f16(-u0, -u1);
                 big = fmaxf(big, fmaxf(fabsf(u0), fabsf(u1)));
             }
@@ -449,7 +452,7 @@ cudaError_t tc_bwd_grad_launch(const void *q, const void *k, const void *g, cons
 // the link step between the passes (seg_link.cu)
 cudaError_t seg_link_launch(const SegPass &sp, int nbh, bool backward, cudaStream_t s);
 
-template <bool GB>
+template <bool GB, bool ACT>
 static cudaError_t tc_bwd_state_run(const void *v, const void *w, const void *dO, const float *dST,
                                     void *dv, void *dw, float *dS0, void *ws, unsigned int *status,
                                     const Dims &d, cudaStream_t s) {
@@ -461,14 +464,14 @@ static cudaError_t tc_bwd_state_run(const void *v, const void *w, const void *dO
         !make_btHd_map(&mdw, dw, GB, d.B, d.T, d.H, 128, 64, gate_box_cols<GB>(), true))
         return cudaErrorInvalidValue;
     const TcWs lay = tc_ws_layout(d);
-    cudaError_t e = cudaFuncSetAttribute(tc_bwd_state_kernel<GB>,
+    cudaError_t e = cudaFuncSetAttribute(tc_bwd_state_kernel<GB, ACT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tbs::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     // a split sequence takes the maps M_s the split forward left in the workspace
     SegPass sp{1, 0, nullptr};
     if (lay.P > 1) sp = SegPass{lay.P, 1, reinterpret_cast<float *>(static_cast<char *>(ws) + lay.seg)};
     launch_begin(K_TC_BWD_STATE, s);
-    tc_bwd_state_kernel<GB><<<dim3(sp.P > 1 ? 2 * (sp.P - 1) : 2, d.H, num_seqs(d)), tbs::kThreads,
+    tc_bwd_state_kernel<GB, ACT><<<dim3(sp.P > 1 ? 2 * (sp.P - 1) : 2, d.H, num_seqs(d)), tbs::kThreads,
                               tbs::SMEM_BYTES, s>>>(mdo_half, mv, mw, mdv, mdw, dST, dS0, dv, dw,
                                                     (unsigned char *)ws, lay, sp, status, d);
     launch_end(K_TC_BWD_STATE, s);
@@ -477,7 +480,7 @@ static cudaError_t tc_bwd_state_run(const void *v, const void *w, const void *dO
         if ((e = seg_link_launch(sp, d.B * d.H, true, s)) != cudaSuccess) return e;
         sp.phase = 2;
         launch_begin(K_TC_BWD_STATE, s);
-        tc_bwd_state_kernel<GB><<<dim3(2 * (sp.P - 1), d.H, d.B), tbs::kThreads, tbs::SMEM_BYTES, s>>>(
+        tc_bwd_state_kernel<GB, ACT><<<dim3(2 * (sp.P - 1), d.H, d.B), tbs::kThreads, tbs::SMEM_BYTES, s>>>(
             mdo_half, mv, mw, mdv, mdw, dST, dS0, dv, dw, (unsigned char *)ws, lay, sp, status, d);
         launch_end(K_TC_BWD_STATE, s);
     }
@@ -489,8 +492,11 @@ cudaError_t tc_bwd_launch(const void *q, const void *k, const void *v, const voi
                           void *dq, void *dk, void *dv, void *dg, void *db, void *dw,
                           float *dS0, void *ws, unsigned int *status, const Dims &d,
                           cudaStream_t s) {
-    cudaError_t e = d.gb ? tc_bwd_state_run<true>(v, w, dO, dST, dv, dw, dS0, ws, status, d, s)
-                         : tc_bwd_state_run<false>(v, w, dO, dST, dv, dw, dS0, ws, status, d, s);
+    cudaError_t e =
+        d.act ? (d.gb ? tc_bwd_state_run<true, true>(v, w, dO, dST, dv, dw, dS0, ws, status, d, s)
+                      : tc_bwd_state_run<false, true>(v, w, dO, dST, dv, dw, dS0, ws, status, d, s))
+              : (d.gb ? tc_bwd_state_run<true, false>(v, w, dO, dST, dv, dw, dS0, ws, status, d, s)
+                      : tc_bwd_state_run<false, false>(v, w, dO, dST, dv, dw, dS0, ws, status, d, s));
     if (e != cudaSuccess) return e;
     return tc_bwd_grad_launch(q, k, g, b, dO, dq, dk, dg, db, ws, status, d, s);
 }

@@ -117,13 +117,13 @@ __host__ __device__ constexpr int pair_ix(int I, int J) { return I * (I - 1) / 2
 //       which the 16x256b tensor-memory loads share, written in place of q,
 //       k, b, g; then dg, the reverse in-chunk cumsum of dG plus the chunk-end
 //       term, and TMA stores.
-template <bool GB>  // g, b, dg, db as bf16 (else float32)
+template <bool GB, bool ACT>  // g, b, dg, db as bf16 (else float32); ACT: gate logits (GateAct)
 __global__ void __launch_bounds__(tbg::kThreads, 1)
 tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                    const __grid_constant__ CUtensorMap mb, const __grid_constant__ CUtensorMap mg,
                    const __grid_constant__ CUtensorMap mdo, const __grid_constant__ CUtensorMap mdq,
                    const __grid_constant__ CUtensorMap mdk, const __grid_constant__ CUtensorMap mdb,
-                   const __grid_constant__ CUtensorMap mdg, void *__restrict__ dq_out,
+                   const __grid_constant__ CUtensorMap mdg, const void *__restrict__ g_in, void *__restrict__ dq_out,
                    void *__restrict__ dk_out, void *__restrict__ db_out, void *__restrict__ dg_out,
                    unsigned char *__restrict__ ws, TcWs lay, unsigned int *status, Dims d) {
     using namespace tbg;
@@ -146,6 +146,7 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int ntiles = total_tiles(d);
+    const GateAct ga = ACT ? gate_act(d.act) : GateAct{false, 1.f};  // logits in: g, b activated on load, db and dg by the chain rule
     const int I = warp & 3, Q = (warp >> 2) & 3;  // row block (TMEM lane quarter); channel quarter
     const int gq = lane >> 2, tq = lane & 3;
     const bool compute = true, issuer = tid == 0;
@@ -275,7 +276,9 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
             float run[2] = {0.f, 0.f}, runc[2] = {0.f, 0.f};
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                const float2 g2 = gld2<GB>(sm + RG + graw<GB>(8 * frg + i, fc));
+                // past the end, no decay (a zero logit would activate to log 1/2)
+                const float2 g2 = 8 * frg + i < L ? act_g2(ga, gld2<GB>(sm + RG + graw<GB>(8 * frg + i, fc)))
+                                                  : make_float2(0.f, 0.f);
                 const float gv[2] = {g2.x * kLog2e, g2.y * kLog2e};
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
@@ -349,7 +352,7 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
             const int t = 8 * frg + i;
             const float2 q2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(sm + RQ + raw16(t, fc)));
             const float2 k2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(sm + RK + raw16(t, fc)));
-            const float2 b2 = gld2<GB>(sm + RB + graw<GB>(t, fc));
+            const float2 b2 = act_b2(ga, gld2<GB>(sm + RB + graw<GB>(t, fc)));
             const float qv[2] = {q2.x, q2.y}, kv[2] = {k2.x, k2.y}, bv[2] = {b2.x, b2.y};
             float v[5][2], dd[2];
 #pragma unroll
@@ -565,7 +568,7 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
                         const float l = ex2(dv), il = ex2(-dv);
                         const float kv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + RK + raw16(j, cc)));
                         const float qv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + RQ + raw16(j, cc)));
-                        const float bv = gld1<GB>(sm + RB + graw<GB>(j, cc));
+                        const float bv = ga.b(gld1<GB>(sm + RB + graw<GB>(j, cc)));
                         bkl[e] = to_tf32(kv * il);
                         bql[e] = to_tf32(qv * l);
                         bbl[e] = to_tf32(bv * kv * l);
@@ -605,9 +608,10 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
                     const float2 dv = *reinterpret_cast<const float2 *>(sm + RG + raw32(r, cc));
                     const float2 qf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(sm + RQ + raw16(r, cc)));
                     const float2 kf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(sm + RK + raw16(r, cc)));
-                    const float2 bf = gld2<GB>(sm + RB + graw<GB>(r, cc));
+                    const float2 bx = gld2<GB>(sm + RB + graw<GB>(r, cc)), bf = act_b2(ga, bx);
                     const float av[2] = {a.x, a.y}, abv[2] = {ab.x, ab.y}, dvv[2] = {dv.x, dv.y},
-                                qv[2] = {qf.x, qf.y}, kv[2] = {kf.x, kf.y}, bv[2] = {bf.x, bf.y};
+                                qv[2] = {qf.x, qf.y}, kv[2] = {kf.x, kf.y}, bv[2] = {bf.x, bf.y},
+                                bxv[2] = {bx.x, bx.y};
                     float dq[2], dk[2], db[2], dG[2];
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
@@ -621,7 +625,7 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
                         const float dkc = fmaf(y2[x], E, z2);
                         const float y3f = y3[x] * F;
                         dk[e] = y3f + z3 + dkc * bv[e];
-                        db[e] = dkc * kv[e];
+                        db[e] = dkc * kv[e] * ga.db(bxv[e]);  // of b, or of its logit
                         dG[e] = qv[e] * dq[e] + 2.f * bv[e] * kv[e] * dkc - kv[e] * dk[e];
                         endk[e] = fmaf(kv[e], y3f, endk[e]);
                     }
@@ -661,9 +665,9 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
                     const float2 Ei2 = __half22float2(*reinterpret_cast<const __half2 *>(sm + MEI + raw16(r, cc)));
                     const float2 qf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(sm + RQ + raw16(r, cc)));
                     const float2 kf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(sm + RK + raw16(r, cc)));
-                    const float2 bf = gld2<GB>(sm + RB + graw<GB>(r, cc));
+                    const float2 bx = gld2<GB>(sm + RB + graw<GB>(r, cc)), bf = act_b2(ga, bx);
                     const float Ev[2] = {E2.x, E2.y}, Eiv[2] = {Ei2.x, Ei2.y}, qv[2] = {qf.x, qf.y},
-                                kv[2] = {kf.x, kf.y}, bv[2] = {bf.x, bf.y};
+                                kv[2] = {kf.x, kf.y}, bv[2] = {bf.x, bf.y}, bxv[2] = {bx.x, bx.y};
                     float dq[2], dk[2], db[2];
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
@@ -672,7 +676,7 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
                         const float dkc = y2[x] * Ev[e];
                         const float y3e = y3[x] * Eiv[e];
                         dk[e] = fmaf(dkc, bv[e], y3e);
-                        db[e] = dkc * kv[e];
+                        db[e] = dkc * kv[e] * ga.db(bxv[e]);  // of b, or of its logit
                         // q dq + 2 b k dKc - k dk = q dq + k (b dKc - Y3 / E)
                         mdG[nt][x] = fmaf(qv[e], dq[e], kv[e] * fmaf(dkc, bv[e], -y3e));
                     }
@@ -728,6 +732,16 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
                 x[r] = run;
             }
             mtot[I * 128 + fc2] = run;
+            // logits in: dg of the logit x_g is dg sigmoid(-x_g); x_g comes back from
+            // global memory (L2), since g's tile now holds dG
+            float sx[16];
+            if (ga.on) {
+#pragma unroll
+                for (int r = 0; r < 16; ++r)
+                    sx[r] = 16 * I + r < L ? gld1<GB>(static_cast<const unsigned char *>(g_in) +
+                                                      (tok(d, bb, c0 + 16 * I + r, h, 128) + fc2) * (GB ? 2 : 4))
+                                           : 0.f;
+            }
             named_sync(1, kCompute);
             // rowsum(dS' . S_c) carries gamma already in the mild frame (S_m dX)
             float after = (mild ? 1.f : mgam[fc2]) * (mend1[fc2] + mend1[128 + fc2] + mend1[256 + fc2] + mend1[384 + fc2]) +
@@ -737,7 +751,7 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
                 if (J > I) after += mtot[J * 128 + fc2];
 #pragma unroll
             for (int r = 0; r < 16; ++r)
-                gst1<GB>(sm + RG + graw<GB>(16 * I + r, fc2), x[r] + after);
+                gst1<GB>(sm + RG + graw<GB>(16 * I + r, fc2), ga.on ? (x[r] + after) * ga.dg(sx[r]) : x[r] + after);
         }
         fence_proxy_async();
         fence_before_sync();
@@ -776,7 +790,7 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
 }
 
 // ---------------------------------------------------------------- launcher
-template <bool GB>
+template <bool GB, bool ACT>
 static cudaError_t tc_bwd_grad_run(const void *q, const void *k, const void *g, const void *b,
                                    const void *dO, void *dq, void *dk, void *dg, void *db, void *ws,
                                    unsigned int *status, const Dims &d, cudaStream_t s) {
@@ -793,14 +807,14 @@ static cudaError_t tc_bwd_grad_run(const void *q, const void *k, const void *g, 
         !make_btHd_map(&mdg, dg, GB, d.B, d.T, d.H, 128, 64, gc, true))
         return cudaErrorInvalidValue;
     const TcWs lay = tc_ws_layout(d);
-    cudaError_t e = cudaFuncSetAttribute(tc_bwd_grad_kernel<GB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(tc_bwd_grad_kernel<GB, ACT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)tbg::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     launch_begin(K_TC_BWD_GRAD, s);
     const long long ntiles = (long long)d.B * d.H * d.NC;
     const int grid = (int)(ntiles < sm_count() ? ntiles : sm_count());
-    tc_bwd_grad_kernel<GB><<<grid, tbg::kThreads, tbg::SMEM_BYTES, s>>>(
-        mq, mk, mb, mg, mdo, mdq, mdk, mdb, mdg, dq, dk, db, dg, (unsigned char *)ws, lay, status, d);
+    tc_bwd_grad_kernel<GB, ACT><<<grid, tbg::kThreads, tbg::SMEM_BYTES, s>>>(
+        mq, mk, mb, mg, mdo, mdq, mdk, mdb, mdg, g, dq, dk, db, dg, (unsigned char *)ws, lay, status, d);
     launch_end(K_TC_BWD_GRAD, s);
     return cudaGetLastError();
 }
@@ -808,8 +822,10 @@ static cudaError_t tc_bwd_grad_run(const void *q, const void *k, const void *g, 
 cudaError_t tc_bwd_grad_launch(const void *q, const void *k, const void *g, const void *b,
                                const void *dO, void *dq, void *dk, void *dg, void *db, void *ws,
                                unsigned int *status, const Dims &d, cudaStream_t s) {
-    return d.gb ? tc_bwd_grad_run<true>(q, k, g, b, dO, dq, dk, dg, db, ws, status, d, s)
-                : tc_bwd_grad_run<false>(q, k, g, b, dO, dq, dk, dg, db, ws, status, d, s);
+    if (d.act) return d.gb ? tc_bwd_grad_run<true, true>(q, k, g, b, dO, dq, dk, dg, db, ws, status, d, s)
+                           : tc_bwd_grad_run<false, true>(q, k, g, b, dO, dq, dk, dg, db, ws, status, d, s);
+    return d.gb ? tc_bwd_grad_run<true, false>(q, k, g, b, dO, dq, dk, dg, db, ws, status, d, s)
+                : tc_bwd_grad_run<false, false>(q, k, g, b, dO, dq, dk, dg, db, ws, status, d, s);
 }
 
 }  // namespace gdn2

@@ -70,7 +70,7 @@ static_assert(STAGE % 1024 == 0 && MISC % 1024 == 0, "alignment");
 static_assert(SMEM_BYTES <= 232448, "shared memory");
 }  // namespace tfwd
 
-template <bool GB>  // w as bf16 (else float32)
+template <bool GB, bool ACT>  // w as bf16 (else float32); ACT: gate logits (GateAct)
 __global__ void __launch_bounds__(tfwd::kThreads, 1)
 tc_fwd_kernel(const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mw,
               const float *__restrict__ S0, __nv_bfloat16 *__restrict__ o, float *__restrict__ ST,
@@ -125,6 +125,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mv, const __grid_constant__ CU
         keep = 0;
     }
     const bool use_u = mode != 2;  // the identity run has no input
+    const GateAct ga = ACT ? gate_act(d.act) : GateAct{false, 1.f};  // logits in: w activated on load
     const int quarter = warp & 3, half = warp >> 2;
     const int key = quarter * 32 + lane;          // state row (TMEM lane) of this thread
     const bool dwarp = quarter < 2;               // reads Delta (lanes 0..63), else O (64..127)
@@ -195,6 +196,8 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mv, const __grid_constant__ CU
                 w0 = *reinterpret_cast<const float4 *>(sm + RAW_W + r * 256 + jv * 32);
                 w1 = *reinterpret_cast<const float4 *>(sm + RAW_W + r * 256 + jv * 32 + 16);
             }
+            w0 = act_w4(ga, w0);
+            w1 = act_w4(ga, w1);
             const __nv_bfloat162 *v2 = reinterpret_cast<const __nv_bfloat162 *>(&vr);
             float u[8] = {w0.x * __low2float(v2[0]), w0.y * __high2float(v2[0]),
                           w0.z * __low2float(v2[1]), w0.w * __high2float(v2[1]),
@@ -417,14 +420,14 @@ cudaError_t tc_prep_launch(const void *q, const void *k, const void *g, const vo
 // the link step between the passes (seg_link.cu)
 cudaError_t seg_link_launch(const SegPass &sp, int nbh, bool backward, cudaStream_t s);
 
-template <bool GB>
+template <bool GB, bool ACT>
 static cudaError_t tc_fwd_run(const void *v, const void *w, const float *S0, void *o, float *ST,
                               void *ws, int keep, unsigned int *status, const Dims &d, cudaStream_t s) {
     CUtensorMap mv, mw;
     if (!make_btHd_map(&mv, v, true, d.B, d.T, d.H, 128, 64, 64) ||
         !make_btHd_map(&mw, w, GB, d.B, d.T, d.H, 128, 64, 64))
         return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(tc_fwd_kernel<GB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(tc_fwd_kernel<GB, ACT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)tfwd::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     const TcWs lay = tc_ws_layout(d);
@@ -432,7 +435,7 @@ static cudaError_t tc_fwd_run(const void *v, const void *w, const float *S0, voi
     // a split sequence needs the workspace that keeps the forward (its segment buffers)
     if (lay.P > 1 && keep) sp = SegPass{lay.P, 1, reinterpret_cast<float *>(static_cast<char *>(ws) + lay.seg)};
     launch_begin(K_TC_FWD, s);
-    tc_fwd_kernel<GB><<<dim3(sp.P > 1 ? 2 + 4 * (sp.P - 2) : 2, d.H, num_seqs(d)), tfwd::kThreads,
+    tc_fwd_kernel<GB, ACT><<<dim3(sp.P > 1 ? 2 + 4 * (sp.P - 2) : 2, d.H, num_seqs(d)), tfwd::kThreads,
                         tfwd::SMEM_BYTES, s>>>(mv, mw, S0, (__nv_bfloat16 *)o, ST, (unsigned char *)ws, keep,
                                                lay, sp, status, d);
     launch_end(K_TC_FWD, s);
@@ -441,7 +444,7 @@ static cudaError_t tc_fwd_run(const void *v, const void *w, const float *S0, voi
         if ((e = seg_link_launch(sp, d.B * d.H, false, s)) != cudaSuccess) return e;
         sp.phase = 2;
         launch_begin(K_TC_FWD, s);
-        tc_fwd_kernel<GB><<<dim3(2 * (sp.P - 1), d.H, d.B), tfwd::kThreads, tfwd::SMEM_BYTES, s>>>(
+        tc_fwd_kernel<GB, ACT><<<dim3(2 * (sp.P - 1), d.H, d.B), tfwd::kThreads, tfwd::SMEM_BYTES, s>>>(
             mv, mw, S0, (__nv_bfloat16 *)o, ST, (unsigned char *)ws, keep, lay, sp, status, d);
         launch_end(K_TC_FWD, s);
     }
@@ -454,8 +457,10 @@ cudaError_t tc_fwd_launch(const void *q, const void *k, const void *v, const voi
                           void *ws, int keep, unsigned int *status, const Dims &d, cudaStream_t s) {
     cudaError_t e = tc_prep_launch(q, k, g, b, ws, status, d, s);
     if (e != cudaSuccess) return e;
-    return d.gb ? tc_fwd_run<true>(v, w, S0, o, ST, ws, keep, status, d, s)
-                : tc_fwd_run<false>(v, w, S0, o, ST, ws, keep, status, d, s);
+    if (d.act) return d.gb ? tc_fwd_run<true, true>(v, w, S0, o, ST, ws, keep, status, d, s)
+                           : tc_fwd_run<false, true>(v, w, S0, o, ST, ws, keep, status, d, s);
+    return d.gb ? tc_fwd_run<true, false>(v, w, S0, o, ST, ws, keep, status, d, s)
+                : tc_fwd_run<false, false>(v, w, S0, o, ST, ws, keep, status, d, s);
 }
 
 }  // namespace gdn2

@@ -153,7 +153,7 @@ __device__ __forceinline__ float ld_bf(const unsigned char *p) {
     return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(p));
 }
 
-template <bool GB>  // g, b as bf16 (else float32)
+template <bool GB, bool ACT>  // g, b as bf16 (else float32); ACT: gate logits (GateAct)
 __global__ void __launch_bounds__(tprep::kThreads, 1)
 tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                const __grid_constant__ CUtensorMap mg, const __grid_constant__ CUtensorMap mb,
@@ -171,6 +171,7 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quarter = warp & 3;
     const int ntiles = total_tiles(d);
+    const GateAct ga = ACT ? gate_act(d.act) : GateAct{false, 1.f};  // logits in: g, b activated on load
 
     if (warp == 0) {
         tmem_alloc(tslot, 256);
@@ -214,14 +215,16 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
         unsigned char *rec = ws + lay.rec + (size_t)it * REC_BYTES;
         bool ok = mbar_wait(&bars[0], n & 1, kWait);
         if (__syncthreads_or(!ok)) { abort = true; break; }
-        if (d.cu) {  // packed sequences: rows past the sequence's end belong to the next one
+        // rows L.. of the tile lie past its sequence's end
+        int L;
+        {
             int tn, th, tc;
             tile_decode(d, it, tn, th, tc);
-            const int L = seq_of(d, tn).len - 64 * tc;
-            if (L < 64) {
-                zero_rows(sm + RAW_Q, 12, L, tid, kThreads);  // q, k, g, b: 96 KB of 8 KB boxes
-                __syncthreads();
-            }
+            L = seq_of(d, tn).len - 64 * tc;
+        }
+        if (d.cu && L < 64) {  // packed sequences: those rows belong to the next one
+            zero_rows(sm + RAW_Q, 12, L, tid, kThreads);  // q, k, g, b: 96 KB of 8 KB boxes
+            __syncthreads();
         }
 
         // ---------------- cumulative decay (log2 units) of this warp's 8 rows,
@@ -231,7 +234,9 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
             float run[4] = {0.f, 0.f, 0.f, 0.f}, runc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                const float4 g4 = gld4<GB>(sm + RAW_G + graw<GB>(8 * warp + i, fc4));
+                // past the end, no decay (a zero logit would activate to log 1/2)
+                const float4 g4 = 8 * warp + i < L ? act_g4(ga, gld4<GB>(sm + RAW_G + graw<GB>(8 * warp + i, fc4)))
+                                                   : make_float4(0.f, 0.f, 0.f, 0.f);
                 const float gv[4] = {g4.x * kLog2e, g4.y * kLog2e, g4.z * kLog2e, g4.w * kLog2e};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
@@ -272,7 +277,7 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
                 float qv[4], kv[4];
                 ld_bf4(sm + RAW_Q + raw16(t, fc4), qv);
                 ld_bf4(sm + RAW_K + raw16(t, fc4), kv);
-                const float4 b4 = gld4<GB>(sm + RAW_B + graw<GB>(t, fc4));
+                const float4 b4 = act_b4(ga, gld4<GB>(sm + RAW_B + graw<GB>(t, fc4)));
                 const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
                 float kcm[4], qbm[4], khm[4];
 #pragma unroll
@@ -370,7 +375,7 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
                 float qv[4], kv[4];
                 ld_bf4(sm + RAW_Q + raw16(t, fc4), qv);
                 ld_bf4(sm + RAW_K + raw16(t, fc4), kv);
-                const float4 b4 = gld4<GB>(sm + RAW_B + graw<GB>(t, fc4));
+                const float4 b4 = act_b4(ga, gld4<GB>(sm + RAW_B + graw<GB>(t, fc4)));
                 const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
                 float bka[4], qa[4], kc[4], qb[4], kb[4], ka[4], dd[4];
 #pragma unroll
@@ -432,7 +437,7 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
                 for (int h = 0; h < 2; ++h) {  // rows r0, r1
                     const int r = h ? r1 : r0;
                     const float4 d4 = *reinterpret_cast<const float4 *>(sm + RAW_G + raw32(r, c));
-                    const float4 b4 = gld4<GB>(sm + RAW_B + graw<GB>(r, c));
+                    const float4 b4 = act_b4(ga, gld4<GB>(sm + RAW_B + graw<GB>(r, c)));
                     float qv[4], kv[4];
                     ld_bf4(sm + RAW_Q + raw16(r, c), qv);
                     ld_bf4(sm + RAW_K + raw16(r, c), kv);
@@ -609,7 +614,7 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
     if (warp == 0) tmem_dealloc(tm, 256);
 }
 
-template <bool GB>
+template <bool GB, bool ACT>
 static cudaError_t tc_prep_run(const void *q, const void *k, const void *g, const void *b, void *ws,
                                unsigned int *status, const Dims &d, cudaStream_t s) {
     CUtensorMap mq, mk, mg, mb;
@@ -618,14 +623,14 @@ static cudaError_t tc_prep_run(const void *q, const void *k, const void *g, cons
         !make_btHd_map(&mg, g, GB, d.B, d.T, d.H, 128, 64, gate_box_cols<GB>(), true) ||
         !make_btHd_map(&mb, b, GB, d.B, d.T, d.H, 128, 64, gate_box_cols<GB>(), true))
         return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(tc_prep_kernel<GB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(tc_prep_kernel<GB, ACT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)tprep::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     // (packed sequences: NC bounds the total chunks; the kernel reads the count)
     const long long ntiles = (long long)d.B * d.H * d.NC;
     const int grid = (int)(ntiles < sm_count() ? ntiles : sm_count());
     launch_begin(K_TC_PREP, s);
-    tc_prep_kernel<GB><<<grid, tprep::kThreads, tprep::SMEM_BYTES, s>>>(
+    tc_prep_kernel<GB, ACT><<<grid, tprep::kThreads, tprep::SMEM_BYTES, s>>>(
         mq, mk, mg, mb, (unsigned char *)ws, tc_ws_layout(d), status, d);
     launch_end(K_TC_PREP, s);
     return cudaGetLastError();
@@ -633,8 +638,10 @@ static cudaError_t tc_prep_run(const void *q, const void *k, const void *g, cons
 
 cudaError_t tc_prep_launch(const void *q, const void *k, const void *g, const void *b, void *ws,
                            unsigned int *status, const Dims &d, cudaStream_t s) {
-    return d.gb ? tc_prep_run<true>(q, k, g, b, ws, status, d, s)
-                : tc_prep_run<false>(q, k, g, b, ws, status, d, s);
+    if (d.act) return d.gb ? tc_prep_run<true, true>(q, k, g, b, ws, status, d, s)
+                           : tc_prep_run<false, true>(q, k, g, b, ws, status, d, s);
+    return d.gb ? tc_prep_run<true, false>(q, k, g, b, ws, status, d, s)
+                : tc_prep_run<false, false>(q, k, g, b, ws, status, d, s);
 }
 
 }  // namespace gdn2

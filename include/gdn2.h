@@ -142,9 +142,21 @@ gdn2_status gdn2_decode_step(const void *q, const void *k, const void *v, const 
                              const float *b, const float *w, float *S, void *o, int N, int H,
                              int d_k, int d_v, gdn2_io io, gdn2_stream_t stream);
 
+/* Flags or-ed into gate_io (the _ex and _varlen calls): the fused gate
+ * prologue.  With GDN2_GATE_LOGITS, g, b and w arrive as pre-activation logits
+ * x_g, x_b, x_w and the kernels activate them on load ("Gated DeltaNet-2",
+ * LIT-802 review, "Key takeaways" 1: sigmoid erase and write gates, a
+ * log-sigmoid decay): g = log sigmoid(x_g), b = sigmoid(x_b), w = sigmoid(x_w);
+ * dg, db, dw are then the gradients of the logits.  GDN2_GATE_B_X2 (only with
+ * LOGITS) takes b = 2 sigmoid(x_b), erase eigenvalues in [-1, 1] (the review's
+ * Table 5).  The chunkwise calls need the tensor-core path for either flag. */
+#define GDN2_GATE_LOGITS 0x100
+#define GDN2_GATE_B_X2 0x200
+
 /* The same calls with two more choices: the gate tensors' type and grouped
  * value heads.
- *   gate_io : type of g, b, w and of dg, db, dw.  GDN2_IO_F32 gives the calls
+ *   gate_io : type of g, b, w and of dg, db, dw, or-ed with the GDN2_GATE_*
+ *       flags above.  GDN2_IO_F32 without flags gives the calls
  *       above.  GDN2_IO_BF16 halves the gate bytes ("Gated DeltaNet-2"
  *       LIT-802 review, "Key takeaways" 1: b and w are sigmoid gates, values in
  *       (0, 1) or (0, 2), which bf16 holds to 3 significant digits); values

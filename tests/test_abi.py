@@ -132,6 +132,11 @@ def test_ex_entry_points_check_the_gate_type_and_value_heads(L):
     assert fwd_ex(0, H=1, Hv=8, dv=32) == 2            # G d_v = 256
     assert fwd_ex(0, H=1, Hv=4, dv=32, ws_bytes=10) == 3   # G d_v = 128: passes
     assert fwd_ex(1, dk=128, dv=64, chunk=64, io=1, H=1, Hv=2, ws_bytes=10) == 3  # tensor cores
+    # gate logits: tensor-core path only; B_X2 needs LOGITS; unknown flags are invalid
+    assert fwd_ex(0x100) == 2
+    assert fwd_ex(0x100 | 0x200, dk=128, dv=128, chunk=64, io=1, ws_bytes=10) == 3
+    assert fwd_ex(0x200, dk=128, dv=128, chunk=64, io=1) == 1
+    assert fwd_ex(0x400, dk=128, dv=128, chunk=64, io=1) == 1
     args = [FAKE] * 6 + [None, FAKE, None] + [FAKE] * 6 + [None, FAKE]
     assert L.gdn2_bwd_ex(*args, 1 << 40, 1, 1, 16, 1, 1, 32, 32, 16, 0, 1, None) == 2
     assert L.gdn2_bwd_ex(*args, 1 << 40, 1, 1, 16, 1, 1, 32, 32, 16, 0, 9, None) == 1

@@ -36,13 +36,13 @@ def tols(io):
     return (TOL_F32, TOL_F32) if io == "f32" else (TOL_BF16_OUT, TOL_BF16_GRAD)
 
 
-def gpu_fwd_bwd(x, io, chunk, backward=True, use_dST=True, gates="f32"):
+def gpu_fwd_bwd(x, io, chunk, backward=True, use_dST=True, gates="f32", encoding="activated"):
     d = to_device(x, io, gates=gates)
-    o, ST, ws = gdn.forward(*(d[n] for n in NAMES), chunk=chunk, for_bwd=backward)
+    o, ST, ws = gdn.forward(*(d[n] for n in NAMES), chunk=chunk, for_bwd=backward, gates=encoding)
     out = {"o": o, "ST": ST}
     if backward:
         gr = gdn.backward(*(d[n] for n in NAMES), d["dO"], d.get("dST") if use_dST else None,
-                          chunk=chunk, ws=ws, ws_has_fwd=True)
+                          chunk=chunk, ws=ws, ws_has_fwd=True, gates=encoding)
         out.update(gr)
     torch.cuda.synchronize()
     assert gdn.gdn2_get_device_status() == 0
@@ -404,6 +404,89 @@ def test_varlen_rejects_a_bad_table_on_the_device():
     assert torch.equal(ST, d["S0"])
     gpu = gpu_varlen(x, cu)          # asserts a clean status itself
     assert np.isfinite(gpu["o"]).all()
+
+
+# ------------------------------------------------------ fused gate prologue
+
+def _logit_inputs(B, T, H, seed, g_shift):
+    """Gate logits: x_g ~ N(g_shift, 1) (g = log sigmoid(x_g): shift 3 gives a
+    mild decay near -0.05 per token, shift 0 a steep one near -0.8), x_b, x_w ~ N(0, 1.5)."""
+    x = workloads.draw(B, T, H, 128, 128, seed, s0_std=0.1, with_dST=True)
+    gen = torch.Generator().manual_seed(seed + 1)
+    x["g"] = torch.randn(x["g"].shape, generator=gen) + g_shift
+    x["b"] = torch.randn(x["b"].shape, generator=gen) * 1.5
+    x["w"] = torch.randn(x["w"].shape, generator=gen) * 1.5
+    return x
+
+
+@pytest.mark.parametrize("encoding,gates,T,g_shift", [
+    ("logits", "f32", 200, 3.0),        # mild tiles, ragged
+    ("logits_b2", "bf16", 200, 0.0),    # steep tiles, b = 2 sigmoid, bf16 logits
+    ("logits", "f32", 1024, 3.0),       # the split state passes (B1 H2: 4 segments)
+])
+def test_gate_logits(encoding, gates, T, g_shift):
+    """The fused gate prologue: g, b, w arrive as logits, the kernels activate
+    them on load, and dg, db, dw leave as gradients of the logits.  Against
+    the oracle's gate layer (fp64 activations, chain rule) on the same
+    (rounded) logits."""
+    from oracle import gates as ogates
+    B = 2 if T == 200 else 1
+    x = _logit_inputs(B, T, 2, 990 + T, g_shift)
+    gpu = gpu_fwd_bwd(x, "bf16", 64, gates=gates, encoding=encoding)
+    r = to_np64(io_round(x, "bf16", gates))
+    bs = 2.0 if encoding == "logits_b2" else 1.0
+    args = (r["q"], r["k"], r["v"], r["g"], r["b"], r["w"], r["S0"])
+    o, ST = ogates.forward(*args, b_scale=bs)
+    ref = {"o": o, "ST": ST, **ogates.backward(*args, r["dO"], r["dST"], b_scale=bs)}
+    compare(gpu, ref, "bf16", ("o", "ST") + GRADS)
+
+
+def test_gate_logits_packed():
+    """Gate logits with packed sequences (65, 1, 130 tokens): the rows past each
+    sequence's end keep no decay, as a zero logit would otherwise activate to
+    log 1/2."""
+    from oracle import gates as ogates, varlen
+    cu = [0, 65, 66, 196]
+    x = _logit_inputs(1, 196, 2, 995, 1.0)
+    x["S0"] = workloads.draw(3, 1, 2, 128, 128, 996, s0_std=0.1)["S0"]
+    x["dST"] = workloads.draw(3, 1, 2, 128, 128, 997, s0_std=0.1)["S0"]
+    d = to_device(x, "bf16")
+    cu_d = torch.tensor(cu, dtype=torch.int32, device="cuda")
+    o, ST, ws = gdn.forward_varlen(*(d[n] for n in NAMES[:-1]), cu_d, d["S0"], for_bwd=True, gates="logits")
+    gr = gdn.backward_varlen(*(d[n] for n in NAMES[:-1]), cu_d, d["S0"], d["dO"], d["dST"], ws=ws,
+                             ws_has_fwd=True, gates="logits")
+    torch.cuda.synchronize()
+    assert gdn.gdn2_get_device_status() == 0
+    gpu = {n: t.float().cpu().numpy() for n, t in {"o": o, "ST": ST, **gr}.items()}
+    r = to_np64(io_round(x, "bf16"))
+    ga, gb_, gw = ogates.activate(r["g"], r["b"], r["w"])
+    names = ("q", "k", "v")
+    o_ref, ST_ref = varlen.forward(*(r[n] for n in names), ga, gb_, gw, cu, r["S0"])
+    ref = varlen.backward(*(r[n] for n in names), ga, gb_, gw, cu, r["S0"], r["dO"], r["dST"])
+    sig = lambda z: 0.5 * (1.0 + np.tanh(0.5 * z))  # noqa: E731
+    ref["dg"] = ref["dg"] * sig(-r["g"])
+    ref["db"] = ref["db"] * sig(r["b"]) * (1 - sig(r["b"]))
+    ref["dw"] = ref["dw"] * sig(r["w"]) * (1 - sig(r["w"]))
+    compare(gpu, {"o": o_ref, "ST": ST_ref, **ref}, "bf16", ("o", "ST") + GRADS)
+
+
+def test_gate_logits_decode():
+    """The decode step with gate logits (b = 2 sigmoid) against the oracle's gate layer."""
+    from oracle import gates as ogates
+    N, H, dk, dv = 3, 2, 64, 64
+    S_gpu = workloads.decode_state(N, H, dk, dv, 21, 0.3).cuda()
+    S_ref = S_gpu.double().cpu().numpy()
+    for s_ in range(6):
+        x = workloads.decode_step_inputs(N, H, dk, dv, 22, s_)
+        gen = torch.Generator().manual_seed(23 + s_)
+        for n in ("g", "b", "w"):
+            x[n] = torch.randn(x[n].shape, generator=gen) + (2.0 if n == "g" else 0.0)
+        d = {n: t.cuda() for n, t in x.items()}
+        o = gdn.decode_step(d["q"], d["k"], d["v"], d["g"], d["b"], d["w"], S_gpu, gates="logits_b2")
+        r = {n: t.double().numpy()[:, None] for n, t in x.items()}
+        o_ref, S_ref = ogates.forward(r["q"], r["k"], r["v"], r["g"], r["b"], r["w"], S_ref, b_scale=2.0)
+        assert rel(o.cpu().numpy(), o_ref[:, 0]) < TOL_F32, s_
+        assert rel(S_gpu.cpu().numpy(), S_ref) < TOL_F32, s_
 
 
 # ------------------------------------------------------ grouped value heads

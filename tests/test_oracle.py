@@ -430,3 +430,29 @@ def test_grouped_oracle_is_the_plain_recurrence_per_value_head():
     o3, ST3 = oracle.forward(r["q"][:, :, 1:2], r["k"][:, :, 1:2], r["v"][:, :, 3:4], r["g"][:, :, 1:2],
                              r["b"][:, :, 1:2], r["w"][:, :, 3:4], r["S0"][:, 3:4])
     assert np.array_equal(o[:, :, 3:4], o3) and np.array_equal(ST[:, 3:4], ST3)
+
+
+# ------------------------------------------------------ fused gate prologue
+
+@pytest.mark.parametrize("b_scale", [1.0, 2.0])
+def test_gate_logits_oracle_matches_finite_differences(b_scale):
+    """Logits in: the chain-rule gradients of x_g, x_b, x_w against central
+    differences of the logit forward; the activations themselves against
+    their definitions at a few points."""
+    from oracle import gates
+    B, T, H, dk, dv = 1, 6, 1, 3, 2
+    x = workloads.draw(B, T, H, dk, dv, 631, s0_std=0.3, with_dST=True)
+    r = {n: t.double().numpy() for n, t in x.items()}
+    gen = np.random.default_rng(632)
+    xs = {"g": gen.normal(1.0, 1.5, r["g"].shape), "b": gen.normal(0, 1.5, r["b"].shape),
+          "w": gen.normal(0, 1.5, r["w"].shape)}
+    fn = lambda q, k, v, xg, xb, xw, S0: gates.forward(q, k, v, xg, xb, xw, S0, b_scale=b_scale)  # noqa: E731
+    inputs = {"q": r["q"], "k": r["k"], "v": r["v"], "g": xs["g"], "b": xs["b"], "w": xs["w"], "S0": r["S0"]}
+    gr = gates.backward(r["q"], r["k"], r["v"], xs["g"], xs["b"], xs["w"], r["S0"], r["dO"], r["dST"],
+                        b_scale=b_scale)
+    num = fd.gradients(inputs, r["dO"], r["dST"], fn=fn)
+    for n in ("dg", "db", "dw", "dq", "dk", "dv", "dS0"):
+        assert np.max(np.abs(gr[n] - num[n])) < 1e-7, n
+    g, b, w = gates.activate(np.array([0.0, -40.0, 40.0]), np.array([0.0]), np.array([0.0]), b_scale)
+    assert abs(g[0] + math.log(2.0)) < 1e-15 and abs(g[1] + 40.0) < 1e-12 and abs(g[2]) < 1e-17
+    assert b[0] == 0.5 * b_scale and w[0] == 0.5
