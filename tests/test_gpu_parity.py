@@ -272,13 +272,14 @@ def test_full_workload_sampled_heads(index):
 
 # ------------------------------------------- segment-parallel state passes
 
-@pytest.mark.parametrize("T", [768, 837, 1024])
-def test_split_state_passes(T):
+@pytest.mark.parametrize("T,H", [(768, 2), (837, 2), (1024, 2), (4096, 1)])
+def test_split_state_passes(T, H):
     """Few (b, h) and many chunks: the state passes split each sequence into
     segments (maps M_s, N_s in parallel, a link, then the segments' real runs).
     T = 768, 837 and 1024 with B = 1, H = 2 take 3, 4 and 4 segments (837: a
-    short last segment with a ragged tail).  Against the oracle."""
-    x = workloads.draw(1, T, 2, 128, 128, 980 + T, s0_std=0.1, with_dST=True)
+    short last segment with a ragged tail); T = 4096 with H = 1 takes the
+    largest count, 8, whose link runs six steps.  Against the oracle."""
+    x = workloads.draw(1, T, H, 128, 128, 980 + T, s0_std=0.1, with_dST=True)
     gpu = gpu_fwd_bwd(x, "bf16", 64)
     ref = oracle_fwd_bwd(x, "bf16")
     compare(gpu, ref, "bf16", ("o", "ST") + GRADS)
