@@ -25,11 +25,14 @@
 //  * the four 16 x 16 diagonal blocks: warp-level tf32 products of
 //    [b.k.l; q.l] against k / l (l = e^(G' - G'_m), clamped, see
 //    tc_common.cuh), each warp one diagonal block and one 8-column half of it.
-// T is inverted in float32 on the CUDA cores; W = T Kc is a tcgen05.mma.
+// T is inverted on the CUDA cores (float32 diagonal blocks, tf32 block
+// columns); W = T Kc is a tcgen05.mma.
 //
 // Persistent: one CTA per SM walks the (b, h, chunk) tiles with a stride of
 // the grid size.  TMA brings the raw q, k, g, b tiles; the next tile's are
-// requested as soon as the diagonal products have read this tile's.
+// requested as soon as this tile's have been read (after the mild test on a
+// mild tile, after the diagonal products otherwise).  The record leaves by
+// bulk copies in four pieces, each as soon as it is final.
 
 #include "common.cuh"
 #include "tc.cuh"
@@ -53,8 +56,11 @@ constexpr uint32_t REC = RR + 24576;  // the tile's record, laid out as in the w
 constexpr uint32_t OP_WQ = REC + REC_WQ;  // [Kc; Qb], later [-W; Qb]
 constexpr uint32_t OP_KB = REC + REC_KH;
 constexpr uint32_t OP_T = REC + REC_T, OP_P = REC + REC_P, FAC = REC + REC_FAC;
-// float32 scratch of the inversion, over CO / RR once the products have read them
-constexpr uint32_t SCR_A = CO, SCR_T = CO + 64 * 65 * 4, SCR_M = SCR_T + 64 * 65 * 4;
+// float32 scratch of the inversion, over CO / RR once the products have read them:
+// A with rows kSA floats apart and T with rows kST apart (row strides chosen so
+// that the warp-level tile loads of either operand role avoid bank conflicts)
+constexpr int kSA = 68, kST = 72;
+constexpr uint32_t SCR_A = CO, SCR_T = CO + 64 * kSA * 4, SCR_M = SCR_T + 64 * kST * 4;
 constexpr uint32_t MISC = REC + REC_BYTES;  // mbarriers, TMEM slot
 // 8-row totals of G [2][8][128] f32, outside the record so that they can be
 // formed while the previous tile's record is still leaving
@@ -71,24 +77,33 @@ static_assert(SCR_M + 8 * 16 * 9 * 4 <= REC, "inversion scratch fits over CO / R
 static_assert(SMEM_BYTES <= 232448, "shared memory");
 }  // namespace tprep
 
-// c += X[r0.., k0..k0+8) * Y[k0..k0+8, n0..n0+8) for row-major [.][65] f32 tiles
+// c += X[r0.., k0..k0+8) * Y[k0..k0+8, n0..n0+8) for row-major f32 tiles with
+// rows SX and SY floats apart
+template <int SX, int SY>
 __device__ __forceinline__ void tile_mma(float *c, const float *X, int r0, int k0, const float *Y,
                                          int n0, int lane) {
     const int g = lane >> 2, t = lane & 3;
-    uint32_t a[4] = {to_tf32(X[(r0 + g) * 65 + k0 + t]), to_tf32(X[(r0 + g + 8) * 65 + k0 + t]),
-                     to_tf32(X[(r0 + g) * 65 + k0 + t + 4]), to_tf32(X[(r0 + g + 8) * 65 + k0 + t + 4])};
-    uint32_t b[2] = {to_tf32(Y[(k0 + t) * 65 + n0 + g]), to_tf32(Y[(k0 + t + 4) * 65 + n0 + g])};
+    uint32_t a[4] = {to_tf32(X[(r0 + g) * SX + k0 + t]), to_tf32(X[(r0 + g + 8) * SX + k0 + t]),
+                     to_tf32(X[(r0 + g) * SX + k0 + t + 4]), to_tf32(X[(r0 + g + 8) * SX + k0 + t + 4])};
+    uint32_t b[2] = {to_tf32(Y[(k0 + t) * SY + n0 + g]), to_tf32(Y[(k0 + t + 4) * SY + n0 + g])};
     mma_tf32_16x8x8(c, a, b);
 }
 
-// T = (I + A)^-1 for the strictly-lower 64x64 A in sA ([64][65] f32), into
-// sT ([64][65] f32), by blocks of 16: the diagonal blocks by forward
-// substitution (one column per thread), then level by level
-// T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ (I - J = 1, 2, 3) as warp-level
-// tf32 tile products, each warp owning 8 columns of one block.  sM holds one
-// 16x8 intermediate per warp ([8][16][9] f32).  All 256 threads; ends with a
-// barrier.
-__device__ __forceinline__ void invert_unit_lower(const float *sA, float *sT, float *sM, int tid) {
+// T = (I + A)^-1 for the strictly-lower 64x64 A in sA (f32, rows kSA apart),
+// written as fp16 into the record's T tile rT ([64][64] K-major, 128-byte
+// swizzle); returns the running largest magnitude of T.  Blocks of 16: the
+// four diagonal blocks by forward substitution (one column per thread, 64
+// threads) into sT (f32, rows kST apart), while the other warps clear the
+// blocks above the diagonal of rT.  Then warp w owns the 8 columns n0 = 8 w of
+// block column J = w / 2 and walks down it, T_IJ = -T_II sum_{K=J}^{I-1}
+// A_IK T_KJ for I = J+1 .. 3, as warp-level tf32 tile products.  A warp reads
+// back only the diagonal blocks and what it wrote itself, so the block levels
+// need no barrier across warps.  sM holds one 16x8 intermediate per warp
+// ([8][16][9] f32).  All 256 threads; the caller fences and synchronises.
+__device__ __forceinline__ float invert_unit_lower(const float *sA, float *sT, float *sM,
+                                                   unsigned char *rT, int tid, float big) {
+    using tprep::kSA;
+    using tprep::kST;
     if (tid < 64) {
         // column cl of the block's inverse, right-looking: once x[j] is final,
         // every later row takes its term at once, so the dependent chain is
@@ -101,49 +116,59 @@ __device__ __forceinline__ void invert_unit_lower(const float *sA, float *sT, fl
         for (int j = 0; j < 15; ++j) {
             const float xj = x[j];
 #pragma unroll
-            for (int r = j + 1; r < 16; ++r) x[r] = fmaf(-sA[(o16 + r) * 65 + o16 + j], xj, x[r]);
+            for (int r = j + 1; r < 16; ++r) x[r] = fmaf(-sA[(o16 + r) * kSA + o16 + j], xj, x[r]);
         }
 #pragma unroll
-        for (int r = 0; r < 16; ++r) sT[(o16 + r) * 65 + o16 + cl] = x[r];
-    }
-    for (int e = tid; e < 64 * 64; e += 256) {
-        const int r = e >> 6, j = e & 63;
-        if ((j >> 4) > (r >> 4)) sT[r * 65 + j] = 0.f;
+        for (int r = 0; r < 16; ++r) sT[(o16 + r) * kST + o16 + cl] = x[r];
+    } else {
+        // 16-byte chunks of rT above the diagonal blocks
+        for (int e = tid - 64; e < 64 * 8; e += 192) {
+            const int r = e >> 3, jc = e & 7;
+            if ((jc >> 1) > (r >> 4)) *reinterpret_cast<uint4 *>(rT + sw128_chunk(r, jc, 64)) = make_uint4(0, 0, 0, 0);
+        }
     }
     __syncthreads();
     const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
-    float *mw = sM + warp * 16 * 9;
-    for (int lvl = 1; lvl < 4; ++lvl) {
-        const int nb = 4 - lvl;  // blocks on this level, two warps each
-        if (warp < 2 * nb) {
-            const int J = warp >> 1, I = J + lvl, n0 = 16 * J + 8 * (warp & 1);
-            float c[4] = {0.f, 0.f, 0.f, 0.f};
-            for (int K = J; K < I; ++K) {
-                tile_mma(c, sA, 16 * I, 16 * K, sT, n0, lane);
-                tile_mma(c, sA, 16 * I, 16 * K + 8, sT, n0, lane);
-            }
-            mw[g * 9 + 2 * t] = c[0];
-            mw[g * 9 + 2 * t + 1] = c[1];
-            mw[(g + 8) * 9 + 2 * t] = c[2];
-            mw[(g + 8) * 9 + 2 * t + 1] = c[3];
-            __syncwarp();
-            float e[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int k0 = 0; k0 < 16; k0 += 8) {
-                uint32_t a[4] = {to_tf32(sT[(16 * I + g) * 65 + 16 * I + k0 + t]),
-                                 to_tf32(sT[(16 * I + g + 8) * 65 + 16 * I + k0 + t]),
-                                 to_tf32(sT[(16 * I + g) * 65 + 16 * I + k0 + t + 4]),
-                                 to_tf32(sT[(16 * I + g + 8) * 65 + 16 * I + k0 + t + 4])};
-                uint32_t b[2] = {to_tf32(mw[(k0 + t) * 9 + g]), to_tf32(mw[(k0 + t + 4) * 9 + g])};
-                mma_tf32_16x8x8(e, a, b);
-            }
-            sT[(16 * I + g) * 65 + n0 + 2 * t] = -e[0];
-            sT[(16 * I + g) * 65 + n0 + 2 * t + 1] = -e[1];
-            sT[(16 * I + g + 8) * 65 + n0 + 2 * t] = -e[2];
-            sT[(16 * I + g + 8) * 65 + n0 + 2 * t + 1] = -e[3];
-        }
-        __syncthreads();
+    const int J = warp >> 1, n0 = 8 * warp;
+    if (lane < 16) {  // this warp's columns of the diagonal block, one row a lane
+        const float *src = sT + (16 * J + lane) * kST + n0;
+        st_h8(rT + sw128_chunk(16 * J + lane, warp, 64), src);
+        big = absmax8(src, big);
     }
+    float *mw = sM + warp * 16 * 9;
+    for (int I = J + 1; I < 4; ++I) {
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int K = J; K < I; ++K) {
+            tile_mma<kSA, kST>(c, sA, 16 * I, 16 * K, sT, n0, lane);
+            tile_mma<kSA, kST>(c, sA, 16 * I, 16 * K + 8, sT, n0, lane);
+        }
+        mw[g * 9 + 2 * t] = c[0];
+        mw[g * 9 + 2 * t + 1] = c[1];
+        mw[(g + 8) * 9 + 2 * t] = c[2];
+        mw[(g + 8) * 9 + 2 * t + 1] = c[3];
+        __syncwarp();
+        float e[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int k0 = 0; k0 < 16; k0 += 8) {
+            uint32_t a[4] = {to_tf32(sT[(16 * I + g) * kST + 16 * I + k0 + t]),
+                             to_tf32(sT[(16 * I + g + 8) * kST + 16 * I + k0 + t]),
+                             to_tf32(sT[(16 * I + g) * kST + 16 * I + k0 + t + 4]),
+                             to_tf32(sT[(16 * I + g + 8) * kST + 16 * I + k0 + t + 4])};
+            uint32_t b[2] = {to_tf32(mw[(k0 + t) * 9 + g]), to_tf32(mw[(k0 + t + 4) * 9 + g])};
+            mma_tf32_16x8x8(e, a, b);
+        }
+        // T_IJ = -e: rows 16 I + g (+ 8), columns n0 + 2 t (+ 1)
+        const int r = 16 * I + g, cc = n0 + 2 * t;
+        sT[r * kST + cc] = -e[0];
+        sT[r * kST + cc + 1] = -e[1];
+        sT[(r + 8) * kST + cc] = -e[2];
+        sT[(r + 8) * kST + cc + 1] = -e[3];
+        *reinterpret_cast<uint32_t *>(rT + sw128_off(r, cc, 64)) = pack_f16(-e[0], -e[1]);
+        *reinterpret_cast<uint32_t *>(rT + sw128_off(r + 8, cc, 64)) = pack_f16(-e[2], -e[3]);
+        big = fmaxf(big, fmaxf(fmaxf(fabsf(e[0]), fabsf(e[1])), fmaxf(fabsf(e[2]), fabsf(e[3]))));
+        __syncwarp();  // this block of T before the next step reads it; mw free again
+    }
+    return big;
 }
 
 __device__ __forceinline__ float2 ld_bf2(const unsigned char *p) {
@@ -187,7 +212,9 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
     fence_after_sync();
     const uint32_t tm = *tslot;
 
-    int issued = 0;  // raw-tile loads requested (thread 0)
+    // raw-tile loads requested: counted by every thread (the conditions are
+    // uniform); thread 0 requests the first tile, thread 32 the later ones
+    int issued = 0;
     auto load_raw = [&](int it) {
         int n, h, c;
         tile_decode(d, it, n, h, c);
@@ -202,9 +229,32 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
             tma_load_4d(sm + RAW_G + x * 8192, &mg, gate_box_cols<GB>() * x, h, row0, bb, &bars[0]);
             tma_load_4d(sm + RAW_B + x * 8192, &mb, gate_box_cols<GB>() * x, h, row0, bb, &bars[0]);
         }
-        ++issued;
     };
-    if (tid == 0 && (int)blockIdx.x < ntiles) load_raw(blockIdx.x);
+    if ((int)blockIdx.x < ntiles) {
+        if (tid == 0) load_raw(blockIdx.x);
+        issued = 1;
+    }
+    // the next tile's raw tiles, once this tile's have been read
+    auto load_next = [&](int it) {
+        if (it + (int)gridDim.x < ntiles) {
+            if (tid == 32) load_raw(it + gridDim.x);
+            ++issued;
+        }
+    };
+    // the record leaves in pieces, each as soon as it is final (thread 64's
+    // bulk group): [Kx] and the Qb rows of [-W; Qb]; P and the factors; T; -W
+    auto store_piece = [&](unsigned char *rec, uint32_t off, uint32_t bytes) {
+        bulk_store(rec + off, sm + REC + off, bytes);
+    };
+    auto store_early = [&](unsigned char *rec) {
+        if (tid == 64) {
+            fence_after_sync();
+            store_piece(rec, REC_KH, 16384);
+            store_piece(rec, REC_WQ + 8192, 8192);
+            store_piece(rec, REC_WQ + 24576, 8192);
+            bulk_commit();
+        }
+    };
 
     // factor phase ownership: warp = 8 rows (block fb, half fh), lane = 4 channels from fc4
     const int fb = warp >> 1, fh = warp & 1, fc4 = 4 * lane;
@@ -249,7 +299,7 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
             *reinterpret_cast<float4 *>(tot + warp * 128 + fc4) = make_float4(run[0], run[1], run[2], run[3]);
             *reinterpret_cast<float4 *>(totc + warp * 128 + fc4) = make_float4(runc[0], runc[1], runc[2], runc[3]);
         }
-        if (tid == 0) bulk_wait_read();  // the previous tile's record has left shared memory
+        if (tid == 64) bulk_wait_read();  // the previous tile's record has left shared memory
         __syncthreads();
         // ---------------- mild tile?  Then the whole chunk fits one frame
         // relative to its row 31: every factor e^(+-(G - G_31)) stays within
@@ -322,6 +372,8 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
                         mma_bf16(tm + TM_C, kstep_kmajor(co, 128, ks), kstep_kmajor(kh, 64, ks), ID_KK128x64, ks > 0);
                     mma_commit(&bars[1]);
                 }
+                load_next(it);  // the mild path reads the raw tiles no more
+                store_early(rec);
             }
         }
         float cA[4] = {0.f, 0.f, 0.f, 0.f}, cP[4] = {0.f, 0.f, 0.f, 0.f};
@@ -408,6 +460,7 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
         fence_proxy_async();
         fence_before_sync();
         __syncthreads();
+        store_early(rec);
         if (tid == 0) {
             fence_after_sync();
             const uint64_t co = desc_kmajor(smem_addr(sm + CO), 128, 0);
@@ -470,7 +523,7 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
         ok = mbar_wait(&bars[1], 0, kWait);
         fence_after_sync();
         __syncthreads();  // the block products have read CO / RR; the raw tiles are consumed
-        if (tid == 0 && it + (int)gridDim.x < ntiles) load_raw(it + gridDim.x);
+        if (!mild) load_next(it);
         float *sA = reinterpret_cast<float *>(sm + SCR_A);
         float *sT = reinterpret_cast<float *>(sm + SCR_T);
         if (mild) {
@@ -484,7 +537,11 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
             if (quarter < 2) {
                 const int r = quarter * 32 + lane;
 #pragma unroll
-                for (int j = 0; j < 32; ++j) sA[r * 65 + 32 * half + j] = 32 * half + j < r ? row[j] : 0.f;
+                for (int j = 0; j < 32; ++j) row[j] = 32 * half + j < r ? row[j] : 0.f;
+#pragma unroll
+                for (int j4 = 0; j4 < 8; ++j4)
+                    *reinterpret_cast<float4 *>(sA + r * kSA + 32 * half + 4 * j4) =
+                        make_float4(row[4 * j4], row[4 * j4 + 1], row[4 * j4 + 2], row[4 * j4 + 3]);
             } else {
                 const int r = quarter * 32 + lane - 64;
 #pragma unroll
@@ -502,7 +559,7 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
             for (int e = 0; e < 4; ++e) {
                 const int rl = gq + ((e & 2) ? 8 : 0), jl = 8 * dn + 2 * tq + (e & 1);
                 const int r = 16 * db + rl, j = 16 * db + jl;
-                sA[r * 65 + j] = jl < rl ? cA[e] : 0.f;
+                sA[r * kSA + j] = jl < rl ? cA[e] : 0.f;
                 cP[e] = jl <= rl ? cP[e] : 0.f;
             }
             const int rA = 16 * db + gq, jA = 16 * db + 8 * dn + 2 * tq;
@@ -531,7 +588,9 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
                     if (I == prod) {
                         if (!isP) {
 #pragma unroll
-                            for (int j = 0; j < 16; ++j) sA[row * 65 + c0 + j] = v[j];
+                            for (int j4 = 0; j4 < 4; ++j4)
+                                *reinterpret_cast<float4 *>(sA + row * kSA + c0 + 4 * j4) =
+                                    make_float4(v[4 * j4], v[4 * j4 + 1], v[4 * j4 + 2], v[4 * j4 + 3]);
                         } else {
 #pragma unroll
                             for (int jj = 0; jj < 2; ++jj) {
@@ -545,16 +604,22 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
         }
         fence_proxy_async();
         if (__syncthreads_or(!ok)) { abort = true; break; }
-        // ---------------- T = (I + A)^-1
-        invert_unit_lower(sA, sT, reinterpret_cast<float *>(sm + SCR_M), tid);
-        for (int e = tid; e < 64 * 8; e += kThreads) {
-            const int r = e >> 3, jj = e & 7;
-            st_h8(sm + OP_T + sw128_chunk(r, jj, 64), sT + r * 65 + 8 * jj);
-            big = absmax8(sT + r * 65 + 8 * jj, big);
+        if (tid == 64) {  // P and the factors are final
+            fence_after_sync();
+            store_piece(rec, REC_P, 8192);
+            store_piece(rec, REC_FAC, REC_BYTES - REC_FAC);
+            bulk_commit();
         }
+        // ---------------- T = (I + A)^-1, into the record as fp16
+        big = invert_unit_lower(sA, sT, reinterpret_cast<float *>(sm + SCR_M), sm + OP_T, tid, big);
         fence_proxy_async();
         fence_before_sync();
         __syncthreads();
+        if (tid == 64) {
+            fence_after_sync();
+            store_piece(rec, REC_T, 8192);
+            bulk_commit();
+        }
         if (tid == 0) {
             fence_after_sync();
             // Kc (rows 0..63 of the [Kc; Qb] tile) as the MN-major B: its two
@@ -591,15 +656,16 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
         fence_proxy_async();
         fence_before_sync();
         if (__syncthreads_or(!ok)) { abort = true; break; }
-        if (tid == 0) {
+        if (tid == 64) {  // -W: rows 0..63 of both 64-key blocks
             fence_after_sync();
-            bulk_store(rec, sm + REC, REC_BYTES);
+            store_piece(rec, REC_WQ, 8192);
+            store_piece(rec, REC_WQ + 16384, 8192);
             bulk_commit();
         }
     }
     if (!(big <= kRange)) record_status(status, GDN2_ERR_RANGE);
+    if (tid == 64) bulk_wait_all();
     if (tid == 0) {
-        bulk_wait_all();
         if (abort) {
             record_status(status, GDN2_ERR_TIMEOUT);
             // let every requested tile land, and every issued product finish,
