@@ -198,14 +198,10 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
         int h, row0, bb;
         tile_rows(it, h, row0, bb);
         mbar_expect_tx(&bars[3], 32768 + 2 * gate_tile_bytes<GB>());
-        for (int x = 0; x < 2; ++x) {
-            tma_load_4d(sm + RQ + x * 8192, &mq, 64 * x, h, row0, bb, &bars[3]);
-            tma_load_4d(sm + RK + x * 8192, &mk, 64 * x, h, row0, bb, &bars[3]);
-        }
-        for (int x = 0; x < 128 / gate_box_cols<GB>(); ++x) {
-            tma_load_4d(sm + RG + x * 8192, &mg, gate_box_cols<GB>() * x, h, row0, bb, &bars[3]);
-            tma_load_4d(sm + RB + x * 8192, &mb, gate_box_cols<GB>() * x, h, row0, bb, &bars[3]);
-        }
+        tma_load_5d(sm + RQ, &mq, 0, h, row0, 0, bb, &bars[3]);
+        tma_load_5d(sm + RK, &mk, 0, h, row0, 0, bb, &bars[3]);
+        tma_load_5d(sm + RG, &mg, 0, h, row0, 0, bb, &bars[3]);
+        tma_load_5d(sm + RB, &mb, 0, h, row0, 0, bb, &bars[3]);
         ++issued[2];
     };
     if (issuer && (int)blockIdx.x < ntiles) {
@@ -697,12 +693,9 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
                 load_a2(nxt);
             }
             if (!tail) {
-                for (int x = 0; x < 2; ++x) {
-                    tma_store_4d(&mdq, sm + RQ + x * 8192, 64 * x, h, c0, bb);
-                    tma_store_4d(&mdk, sm + RK + x * 8192, 64 * x, h, c0, bb);
-                }
-                for (int x = 0; x < 128 / gate_box_cols<GB>(); ++x)
-                    tma_store_4d(&mdb, sm + RB + x * 8192, gate_box_cols<GB>() * x, h, c0, bb);
+                tma_store_5d(&mdq, sm + RQ, 0, h, c0, 0, bb);
+                tma_store_5d(&mdk, sm + RK, 0, h, c0, 0, bb);
+                tma_store_5d(&mdb, sm + RB, 0, h, c0, 0, bb);
                 bulk_commit();
             }
         }
@@ -765,8 +758,7 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
         }
         if (issuer) {
             if (!tail) {
-                for (int x = 0; x < 128 / gate_box_cols<GB>(); ++x)
-                    tma_store_4d(&mdg, sm + RG + x * 8192, gate_box_cols<GB>() * x, h, c0, bb);
+                tma_store_5d(&mdg, sm + RG, 0, h, c0, 0, bb);
                 bulk_commit();
             }
             bulk_wait_read();  // the tiles may be refilled
@@ -796,16 +788,11 @@ static cudaError_t tc_bwd_grad_run(const void *q, const void *k, const void *g, 
                                    const void *dO, void *dq, void *dk, void *dg, void *db, void *ws,
                                    unsigned int *status, const Dims &d, cudaStream_t s) {
     CUtensorMap mq, mk, mb, mg, mdo, mdq, mdk, mdb, mdg;
-    constexpr int gc = gate_box_cols<GB>();
-    if (!make_btHd_map(&mq, q, true, d.B, d.T, d.H, 128, 64, 64, true) ||
-        !make_btHd_map(&mk, k, true, d.B, d.T, d.H, 128, 64, 64, true) ||
-        !make_btHd_map(&mb, b, GB, d.B, d.T, d.H, 128, 64, gc, true) ||
-        !make_btHd_map(&mg, g, GB, d.B, d.T, d.H, 128, 64, gc, true) ||
+    if (!make_wide_map(&mq, q, true, d.B, d.T, d.H, 128, 64) || !make_wide_map(&mk, k, true, d.B, d.T, d.H, 128, 64) ||
+        !make_wide_map(&mb, b, GB, d.B, d.T, d.H, 128, 64) || !make_wide_map(&mg, g, GB, d.B, d.T, d.H, 128, 64) ||
         !make_btHd_map(&mdo, dO, true, d.B, d.T, d.H, 128, 64, 64, true) ||
-        !make_btHd_map(&mdq, dq, true, d.B, d.T, d.H, 128, 64, 64, true) ||
-        !make_btHd_map(&mdk, dk, true, d.B, d.T, d.H, 128, 64, 64, true) ||
-        !make_btHd_map(&mdb, db, GB, d.B, d.T, d.H, 128, 64, gc, true) ||
-        !make_btHd_map(&mdg, dg, GB, d.B, d.T, d.H, 128, 64, gc, true))
+        !make_wide_map(&mdq, dq, true, d.B, d.T, d.H, 128, 64) || !make_wide_map(&mdk, dk, true, d.B, d.T, d.H, 128, 64) ||
+        !make_wide_map(&mdb, db, GB, d.B, d.T, d.H, 128, 64) || !make_wide_map(&mdg, dg, GB, d.B, d.T, d.H, 128, 64))
         return cudaErrorInvalidValue;
     const TcWs lay = tc_ws_layout(d);
     cudaError_t e = cudaFuncSetAttribute(tc_bwd_grad_kernel<GB, ACT>, cudaFuncAttributeMaxDynamicSharedMemorySize,

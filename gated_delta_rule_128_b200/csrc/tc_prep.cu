@@ -30,9 +30,9 @@
 //
 // Persistent: one CTA per SM walks the (b, h, chunk) tiles with a stride of
 // the grid size.  TMA brings the raw q, k, g, b tiles; the next tile's are
-// requested as soon as this tile's have been read (after the mild test on a
-// mild tile, after the diagonal products otherwise).  The record leaves by
-// bulk copies in four pieces, each as soon as it is final.
+// requested during the inversion, by a warp that is idle then (issuing a TMA
+// load holds its thread a long time).  The record leaves by bulk copies in
+// four pieces, each as soon as it is final.
 
 #include "common.cuh"
 #include "tc.cuh"
@@ -99,9 +99,12 @@ __device__ __forceinline__ void tile_mma(float *c, const float *X, int r0, int k
 // A_IK T_KJ for I = J+1 .. 3, as warp-level tf32 tile products.  A warp reads
 // back only the diagonal blocks and what it wrote itself, so the block levels
 // need no barrier across warps.  sM holds one 16x8 intermediate per warp
-// ([8][16][9] f32).  All 256 threads; the caller fences and synchronises.
+// ([8][16][9] f32).  Warp 7 has no block below its diagonal block: its lane 0
+// runs `idle` during the block columns.  All 256 threads; the caller fences
+// and synchronises.
+template <typename Idle>
 __device__ __forceinline__ float invert_unit_lower(const float *sA, float *sT, float *sM,
-                                                   unsigned char *rT, int tid, float big) {
+                                                   unsigned char *rT, int tid, float big, Idle &&idle) {
     using tprep::kSA;
     using tprep::kST;
     if (tid < 64) {
@@ -135,17 +138,25 @@ __device__ __forceinline__ float invert_unit_lower(const float *sA, float *sT, f
         st_h8(rT + sw128_chunk(16 * J + lane, warp, 64), src);
         big = absmax8(src, big);
     }
+    if (tid == 224) idle();
+    // right-looking over the block rows: acc[I] collects sum_K A_IK T_KJ, and
+    // once T_IJ is final every lower block row takes its term at once, so the
+    // dependent chain is two tile products per block row
     float *mw = sM + warp * 16 * 9;
-    for (int I = J + 1; I < 4; ++I) {
-        float c[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int K = J; K < I; ++K) {
-            tile_mma<kSA, kST>(c, sA, 16 * I, 16 * K, sT, n0, lane);
-            tile_mma<kSA, kST>(c, sA, 16 * I, 16 * K + 8, sT, n0, lane);
+    float acc[4][4] = {};
+#pragma unroll
+    for (int I = 1; I < 4; ++I)
+        if (I > J) {
+            tile_mma<kSA, kST>(acc[I], sA, 16 * I, 16 * J, sT, n0, lane);
+            tile_mma<kSA, kST>(acc[I], sA, 16 * I, 16 * J + 8, sT, n0, lane);
         }
-        mw[g * 9 + 2 * t] = c[0];
-        mw[g * 9 + 2 * t + 1] = c[1];
-        mw[(g + 8) * 9 + 2 * t] = c[2];
-        mw[(g + 8) * 9 + 2 * t + 1] = c[3];
+#pragma unroll
+    for (int I = 1; I < 4; ++I) {
+        if (I <= J) continue;
+        mw[g * 9 + 2 * t] = acc[I][0];
+        mw[g * 9 + 2 * t + 1] = acc[I][1];
+        mw[(g + 8) * 9 + 2 * t] = acc[I][2];
+        mw[(g + 8) * 9 + 2 * t + 1] = acc[I][3];
         __syncwarp();
         float e[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -166,7 +177,12 @@ __device__ __forceinline__ float invert_unit_lower(const float *sA, float *sT, f
         *reinterpret_cast<uint32_t *>(rT + sw128_off(r, cc, 64)) = pack_f16(-e[0], -e[1]);
         *reinterpret_cast<uint32_t *>(rT + sw128_off(r + 8, cc, 64)) = pack_f16(-e[2], -e[3]);
         big = fmaxf(big, fmaxf(fmaxf(fabsf(e[0]), fabsf(e[1])), fmaxf(fabsf(e[2]), fabsf(e[3]))));
-        __syncwarp();  // this block of T before the next step reads it; mw free again
+        __syncwarp();  // T_IJ before the lower block rows read it; mw free again
+#pragma unroll
+        for (int I2 = I + 1; I2 < 4; ++I2) {
+            tile_mma<kSA, kST>(acc[I2], sA, 16 * I2, 16 * I, sT, n0, lane);
+            tile_mma<kSA, kST>(acc[I2], sA, 16 * I2, 16 * I + 8, sT, n0, lane);
+        }
     }
     return big;
 }
@@ -213,7 +229,7 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
     const uint32_t tm = *tslot;
 
     // raw-tile loads requested: counted by every thread (the conditions are
-    // uniform); thread 0 requests the first tile, thread 32 the later ones
+    // uniform); thread 0 requests the first tile, thread 224 the later ones
     int issued = 0;
     auto load_raw = [&](int it) {
         int n, h, c;
@@ -221,26 +237,16 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
         const Seq sq = seq_of(d, n);
         const int row0 = sq.bos + 64 * c, bb = sq.brow;
         mbar_expect_tx(&bars[0], 16384 * 2 + gate_tile_bytes<GB>() * 2);
-        for (int x = 0; x < 2; ++x) {
-            tma_load_4d(sm + RAW_Q + x * 8192, &mq, 64 * x, h, row0, bb, &bars[0]);
-            tma_load_4d(sm + RAW_K + x * 8192, &mk, 64 * x, h, row0, bb, &bars[0]);
-        }
-        for (int x = 0; x < 128 / gate_box_cols<GB>(); ++x) {
-            tma_load_4d(sm + RAW_G + x * 8192, &mg, gate_box_cols<GB>() * x, h, row0, bb, &bars[0]);
-            tma_load_4d(sm + RAW_B + x * 8192, &mb, gate_box_cols<GB>() * x, h, row0, bb, &bars[0]);
-        }
+        tma_load_5d(sm + RAW_Q, &mq, 0, h, row0, 0, bb, &bars[0]);
+        tma_load_5d(sm + RAW_K, &mk, 0, h, row0, 0, bb, &bars[0]);
+        tma_load_5d(sm + RAW_G, &mg, 0, h, row0, 0, bb, &bars[0]);
+        tma_load_5d(sm + RAW_B, &mb, 0, h, row0, 0, bb, &bars[0]);
     };
     if ((int)blockIdx.x < ntiles) {
         if (tid == 0) load_raw(blockIdx.x);
         issued = 1;
     }
-    // the next tile's raw tiles, once this tile's have been read
-    auto load_next = [&](int it) {
-        if (it + (int)gridDim.x < ntiles) {
-            if (tid == 32) load_raw(it + gridDim.x);
-            ++issued;
-        }
-    };
+
     // the record leaves in pieces, each as soon as it is final (thread 64's
     // bulk group): [Kx] and the Qb rows of [-W; Qb]; P and the factors; T; -W
     auto store_piece = [&](unsigned char *rec, uint32_t off, uint32_t bytes) {
@@ -261,17 +267,19 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
 
     bool abort = false;
     int n = 0;  // tiles done by this CTA
+    // rows of tile `it` inside its sequence (64 unless a packed sequence ends in it)
+    auto rows_of = [&](int it) {
+        int tn, th, tc;
+        tile_decode(d, it, tn, th, tc);
+        return seq_of(d, tn).len - 64 * tc;
+    };
+    int L_next = (int)blockIdx.x < ntiles ? rows_of(blockIdx.x) : 0;
     for (int it = blockIdx.x; it < ntiles; it += gridDim.x, ++n) {
         unsigned char *rec = ws + lay.rec + (size_t)it * REC_BYTES;
         bool ok = mbar_wait(&bars[0], n & 1, kWait);
         if (__syncthreads_or(!ok)) { abort = true; break; }
         // rows L.. of the tile lie past its sequence's end
-        int L;
-        {
-            int tn, th, tc;
-            tile_decode(d, it, tn, th, tc);
-            L = seq_of(d, tn).len - 64 * tc;
-        }
+        const int L = L_next;  // found during the previous tile
         if (d.cu && L < 64) {  // packed sequences: those rows belong to the next one
             zero_rows(sm + RAW_Q, 12, L, tid, kThreads);  // q, k, g, b: 96 KB of 8 KB boxes
             __syncthreads();
@@ -372,7 +380,6 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
                         mma_bf16(tm + TM_C, kstep_kmajor(co, 128, ks), kstep_kmajor(kh, 64, ks), ID_KK128x64, ks > 0);
                     mma_commit(&bars[1]);
                 }
-                load_next(it);  // the mild path reads the raw tiles no more
                 store_early(rec);
             }
         }
@@ -523,7 +530,6 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
         ok = mbar_wait(&bars[1], 0, kWait);
         fence_after_sync();
         __syncthreads();  // the block products have read CO / RR; the raw tiles are consumed
-        if (!mild) load_next(it);
         float *sA = reinterpret_cast<float *>(sm + SCR_A);
         float *sT = reinterpret_cast<float *>(sm + SCR_T);
         if (mild) {
@@ -611,7 +617,13 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
             bulk_commit();
         }
         // ---------------- T = (I + A)^-1, into the record as fp16
-        big = invert_unit_lower(sA, sT, reinterpret_cast<float *>(sm + SCR_M), sm + OP_T, tid, big);
+        // the raw tiles are consumed: the next tile's are requested by a warp
+        // that is idle during the inversion's block columns
+        const bool has_next = it + (int)gridDim.x < ntiles;
+        big = invert_unit_lower(sA, sT, reinterpret_cast<float *>(sm + SCR_M), sm + OP_T, tid, big, [&] {
+            if (has_next) load_raw(it + gridDim.x);
+        });
+        issued += has_next;
         fence_proxy_async();
         fence_before_sync();
         __syncthreads();
@@ -632,6 +644,7 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
             mma_commit(&bars[1]);
         }
         // ---------------- -W to fp16 (over Kc, consumed by the product); the record
+        if (it + (int)gridDim.x < ntiles) L_next = rows_of(it + gridDim.x);  // while W runs
         ok = mbar_wait(&bars[1], 1, kWait);
         fence_after_sync();
         {
@@ -684,10 +697,8 @@ template <bool GB, bool ACT>
 static cudaError_t tc_prep_run(const void *q, const void *k, const void *g, const void *b, void *ws,
                                unsigned int *status, const Dims &d, cudaStream_t s) {
     CUtensorMap mq, mk, mg, mb;
-    if (!make_btHd_map(&mq, q, true, d.B, d.T, d.H, 128, 64, 64, true) ||
-        !make_btHd_map(&mk, k, true, d.B, d.T, d.H, 128, 64, 64, true) ||
-        !make_btHd_map(&mg, g, GB, d.B, d.T, d.H, 128, 64, gate_box_cols<GB>(), true) ||
-        !make_btHd_map(&mb, b, GB, d.B, d.T, d.H, 128, 64, gate_box_cols<GB>(), true))
+    if (!make_wide_map(&mq, q, true, d.B, d.T, d.H, 128, 64) || !make_wide_map(&mk, k, true, d.B, d.T, d.H, 128, 64) ||
+        !make_wide_map(&mg, g, GB, d.B, d.T, d.H, 128, 64) || !make_wide_map(&mb, b, GB, d.B, d.T, d.H, 128, 64))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(tc_prep_kernel<GB, ACT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)tprep::SMEM_BYTES);
