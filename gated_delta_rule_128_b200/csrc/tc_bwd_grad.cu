@@ -115,15 +115,16 @@ __host__ __device__ constexpr int pair_ix(int I, int J) { return I * (I - 1) / 2
 //       diagonal blocks in tf32 (m16n8k8) with the clamped mid-block frame;
 //   (4) dq, dk, db, dG per (row, channel) in the accumulator-fragment layout,
 //       which the 16x256b tensor-memory loads share, written in place of q,
-//       k, b, g; then dg, the reverse in-chunk cumsum of dG plus the chunk-end
-//       term, and TMA stores.
+//       k, b, g, and dq, dk, db leave by TMA stores; then dg, the reverse
+//       in-chunk cumsum of dG plus the chunk-end term, straight from the scan
+//       to global memory.
 template <bool GB, bool ACT>  // g, b, dg, db as bf16 (else float32); ACT: gate logits (GateAct)
 __global__ void __launch_bounds__(tbg::kThreads, 1)
 tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                    const __grid_constant__ CUtensorMap mb, const __grid_constant__ CUtensorMap mg,
                    const __grid_constant__ CUtensorMap mdo, const __grid_constant__ CUtensorMap mdq,
                    const __grid_constant__ CUtensorMap mdk, const __grid_constant__ CUtensorMap mdb,
-                   const __grid_constant__ CUtensorMap mdg, const void *__restrict__ g_in, void *__restrict__ dq_out,
+                   const void *__restrict__ g_in, void *__restrict__ dq_out,
                    void *__restrict__ dk_out, void *__restrict__ db_out, void *__restrict__ dg_out,
                    unsigned char *__restrict__ ws, TcWs lay, unsigned int *status, Dims d) {
     using namespace tbg;
@@ -194,23 +195,34 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
         bulk_load(sm + DXT, ws + lay.ckdS + ((size_t)it * 2) * 16384, 32768, &bars[0]);
         ++issued[1];
     };
-    auto load_b = [&](int it) {  // raw q, k, b, g
+    // raw q, k, b, g in two parts: g as soon as the scan has read dG out of its
+    // tile, then q, k, b once dq, dk, db have left theirs; the first part
+    // expects the bytes of all four
+    int pend_b = -1;  // tile whose g has been requested but not its q, k, b
+    auto load_b_g = [&](int it) {
         int h, row0, bb;
         tile_rows(it, h, row0, bb);
         mbar_expect_tx(&bars[3], 32768 + 2 * gate_tile_bytes<GB>());
+        tma_load_5d(sm + RG, &mg, 0, h, row0, 0, bb, &bars[3]);
+        ++issued[2];
+        pend_b = it;
+    };
+    auto load_b_rest = [&](int it) {
+        int h, row0, bb;
+        tile_rows(it, h, row0, bb);
         tma_load_5d(sm + RQ, &mq, 0, h, row0, 0, bb, &bars[3]);
         tma_load_5d(sm + RK, &mk, 0, h, row0, 0, bb, &bars[3]);
-        tma_load_5d(sm + RG, &mg, 0, h, row0, 0, bb, &bars[3]);
         tma_load_5d(sm + RB, &mb, 0, h, row0, 0, bb, &bars[3]);
-        ++issued[2];
+        pend_b = -1;
     };
     if (issuer && (int)blockIdx.x < ntiles) {
         load_a1(blockIdx.x);
         load_a2(blockIdx.x);
-        load_b(blockIdx.x);
+        load_b_g(blockIdx.x);
+        load_b_rest(blockIdx.x);
     }
 
-    bool ok = true;
+    bool ok = true, aborted = false;  // aborted: some thread's wait gave up (block-wide)
     int nmild = 0;  // mild tiles done (second product groups committed to bars[2])
     for (int it = blockIdx.x, n = 0; it < ntiles; it += gridDim.x, ++n) {
         int tn, h, c;
@@ -736,42 +748,41 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
                                                       (tok(d, bb, c0 + 16 * I + r, h, 128) + fc2) * (GB ? 2 : 4))
                                            : 0.f;
             }
-            named_sync(1, kCompute);
+            named_sync(1, kCompute);  // dG is read: g's tile is free
+            if (issuer && more) load_b_g(nxt);
             // rowsum(dS' . S_c) carries gamma already in the mild frame (S_m dX)
             float after = (mild ? 1.f : mgam[fc2]) * (mend1[fc2] + mend1[128 + fc2] + mend1[256 + fc2] + mend1[384 + fc2]) +
                           mendk[fc2] + mendk[128 + fc2] + mendk[256 + fc2] + mendk[384 + fc2];
 #pragma unroll
             for (int J = 0; J < 4; ++J)
                 if (J > I) after += mtot[J * 128 + fc2];
+            // dg leaves from the scan's registers: for each row a warp writes 32
+            // consecutive channels, so g's tile is free once the scan has read dG
+            constexpr int ges = GB ? 2 : 4;
+            unsigned char *dgp = static_cast<unsigned char *>(dg_out) + (tok(d, bb, c0 + 16 * I, h, 128) + fc2) * ges;
+            const size_t rstride = (size_t)d.H * 128 * ges;
 #pragma unroll
             for (int r = 0; r < 16; ++r)
-                gst1<GB>(sm + RG + graw<GB>(16 * I + r, fc2), ga.on ? (x[r] + after) * ga.dg(sx[r]) : x[r] + after);
+                if (16 * I + r < L) gst1<GB>(dgp + r * rstride, ga.on ? (x[r] + after) * ga.dg(sx[r]) : x[r] + after);
         }
-        fence_proxy_async();
         fence_before_sync();
-        if (__syncthreads_or(!ok)) break;
-        if (tail) {
-            store_rows(reinterpret_cast<unsigned char *>(dg_out) + tok(d, bb, c0, h, 128) * (GB ? 2 : 4),
-                       (size_t)d.H * 128 * (GB ? 2 : 4), sm + RG, GB ? 2 : 4, L, tid, kThreads);
-            fence_proxy_async();
-            __syncthreads();  // every row has left the raw tiles
+        if (__syncthreads_or(!ok)) {
+            aborted = true;
+            break;
         }
         if (issuer) {
-            if (!tail) {
-                tma_store_5d(&mdg, sm + RG, 0, h, c0, 0, bb);
-                bulk_commit();
-            }
-            bulk_wait_read();  // the tiles may be refilled
-            if (more) load_b(nxt);
+            bulk_wait_read();  // dq, dk, db have left the raw tiles
+            if (more) load_b_rest(nxt);
         }
     }
     if (issuer) bulk_wait_all();
     if (!(big <= kRange)) record_status(status, GDN2_ERR_RANGE);
-    if (!ok && issuer) {
+    if (aborted && issuer) {
         record_status(status, GDN2_ERR_TIMEOUT);
         // every copy landed and every issued product done before the shared
         // and tensor memory go away
         if (issued[0] > 0) mbar_wait(&bars[0], (issued[0] - 1) & 1, kWait);
+        if (pend_b >= 0) load_b_rest(pend_b);  // the requested tile's bytes complete its phase
         if (issued[2] > 0) mbar_wait(&bars[3], (issued[2] - 1) & 1, kWait);
         mbar_wait(&bars[1], 0, kWait);
         mbar_wait(&bars[1], 1, kWait);
@@ -787,12 +798,12 @@ template <bool GB, bool ACT>
 static cudaError_t tc_bwd_grad_run(const void *q, const void *k, const void *g, const void *b,
                                    const void *dO, void *dq, void *dk, void *dg, void *db, void *ws,
                                    unsigned int *status, const Dims &d, cudaStream_t s) {
-    CUtensorMap mq, mk, mb, mg, mdo, mdq, mdk, mdb, mdg;
+    CUtensorMap mq, mk, mb, mg, mdo, mdq, mdk, mdb;
     if (!make_wide_map(&mq, q, true, d.B, d.T, d.H, 128, 64) || !make_wide_map(&mk, k, true, d.B, d.T, d.H, 128, 64) ||
         !make_wide_map(&mb, b, GB, d.B, d.T, d.H, 128, 64) || !make_wide_map(&mg, g, GB, d.B, d.T, d.H, 128, 64) ||
         !make_btHd_map(&mdo, dO, true, d.B, d.T, d.H, 128, 64, 64, true) ||
         !make_wide_map(&mdq, dq, true, d.B, d.T, d.H, 128, 64) || !make_wide_map(&mdk, dk, true, d.B, d.T, d.H, 128, 64) ||
-        !make_wide_map(&mdb, db, GB, d.B, d.T, d.H, 128, 64) || !make_wide_map(&mdg, dg, GB, d.B, d.T, d.H, 128, 64))
+        !make_wide_map(&mdb, db, GB, d.B, d.T, d.H, 128, 64))
         return cudaErrorInvalidValue;
     const TcWs lay = tc_ws_layout(d);
     cudaError_t e = cudaFuncSetAttribute(tc_bwd_grad_kernel<GB, ACT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -802,7 +813,7 @@ static cudaError_t tc_bwd_grad_run(const void *q, const void *k, const void *g, 
     const long long ntiles = (long long)d.B * d.H * d.NC;
     const int grid = (int)(ntiles < sm_count() ? ntiles : sm_count());
     tc_bwd_grad_kernel<GB, ACT><<<grid, tbg::kThreads, tbg::SMEM_BYTES, s>>>(
-        mq, mk, mb, mg, mdo, mdq, mdk, mdb, mdg, g, dq, dk, db, dg, (unsigned char *)ws, lay, status, d);
+        mq, mk, mb, mg, mdo, mdq, mdk, mdb, g, dq, dk, db, dg, (unsigned char *)ws, lay, status, d);
     launch_end(K_TC_BWD_GRAD, s);
     return cudaGetLastError();
 }
