@@ -139,8 +139,8 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
     float *mgam = reinterpret_cast<float *>(sm + MISC + M_GAM);    // [128] gamma
     float *mes = reinterpret_cast<float *>(sm + ESF);              // [4][128] e^s_I (after the first products)
     float *mef = mes + 4 * 128;                                    // [4][128] e^(G_63 - e_I)
-    // 0 first-product operands (two parts), 1 products, 3 raw tiles, 4 dO
-    // converted (one arrival per compute warp)
+    // 0 first-product operands (two parts), 1 products, 2 second products
+    // (mild), 3 raw g, 4 raw q, k, b
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + MISC + M_BAR);
     uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + MISC + M_BAR + 64);
     float big = 0.f;  // range check: largest fp16 operand magnitude
@@ -159,7 +159,7 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
     if (issuer) {
         mbar_init(&bars[0], 2);
         for (int i = 1; i < 4; ++i) mbar_init(&bars[i], 1);
-        mbar_init(&bars[4], kWarps);
+        mbar_init(&bars[4], 1);
         mbar_fence_init();
     }
     fence_before_sync();
@@ -195,14 +195,14 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
         bulk_load(sm + DXT, ws + lay.ckdS + ((size_t)it * 2) * 16384, 32768, &bars[0]);
         ++issued[1];
     };
-    // raw q, k, b, g in two parts: g as soon as the scan has read dG out of its
-    // tile, then q, k, b once dq, dk, db have left theirs; the first part
-    // expects the bytes of all four
+    // raw q, k, b, g in two parts on two barriers: g (bars[3]) as soon as the
+    // scan has read dG out of its tile, then q, k, b (bars[4]) once dq, dk, db
+    // have left theirs
     int pend_b = -1;  // tile whose g has been requested but not its q, k, b
     auto load_b_g = [&](int it) {
         int h, row0, bb;
         tile_rows(it, h, row0, bb);
-        mbar_expect_tx(&bars[3], 32768 + 2 * gate_tile_bytes<GB>());
+        mbar_expect_tx(&bars[3], gate_tile_bytes<GB>());
         tma_load_5d(sm + RG, &mg, 0, h, row0, 0, bb, &bars[3]);
         ++issued[2];
         pend_b = it;
@@ -210,9 +210,10 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
     auto load_b_rest = [&](int it) {
         int h, row0, bb;
         tile_rows(it, h, row0, bb);
-        tma_load_5d(sm + RQ, &mq, 0, h, row0, 0, bb, &bars[3]);
-        tma_load_5d(sm + RK, &mk, 0, h, row0, 0, bb, &bars[3]);
-        tma_load_5d(sm + RB, &mb, 0, h, row0, 0, bb, &bars[3]);
+        mbar_expect_tx(&bars[4], 32768 + gate_tile_bytes<GB>());
+        tma_load_5d(sm + RQ, &mq, 0, h, row0, 0, bb, &bars[4]);
+        tma_load_5d(sm + RK, &mk, 0, h, row0, 0, bb, &bars[4]);
+        tma_load_5d(sm + RB, &mb, 0, h, row0, 0, bb, &bars[4]);
         pend_b = -1;
     };
     if (issuer && (int)blockIdx.x < ntiles) {
@@ -271,8 +272,9 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
             }
             mma_commit(&bars[1]);
         }
-        ok = mbar_wait(&bars[3], par, kWait) && ok;  // raw q, k, b, g
+        ok = mbar_wait(&bars[3], par, kWait) && ok;  // raw g
         if (tail) {
+            ok = mbar_wait(&bars[4], par, kWait) && ok;  // raw q, k, b
             zero_rows(sm + RQ, 12, L, tid, kThreads);  // q, k, b, g: 96 KB of 8 KB boxes
             __syncthreads();
         }
@@ -355,6 +357,7 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
             }
         }
         if (fh == 0 && fb == 0) *reinterpret_cast<float2 *>(mgam + fc) = make_float2(ex2(all[0]), ex2(all[1]));
+        if (!tail) ok = mbar_wait(&bars[4], par, kWait) && ok;  // raw q, k, b
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const int t = 8 * frg + i;
@@ -783,7 +786,10 @@ tc_bwd_grad_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
         // and tensor memory go away
         if (issued[0] > 0) mbar_wait(&bars[0], (issued[0] - 1) & 1, kWait);
         if (pend_b >= 0) load_b_rest(pend_b);  // the requested tile's bytes complete its phase
-        if (issued[2] > 0) mbar_wait(&bars[3], (issued[2] - 1) & 1, kWait);
+        if (issued[2] > 0) {
+            mbar_wait(&bars[3], (issued[2] - 1) & 1, kWait);
+            mbar_wait(&bars[4], (issued[2] - 1) & 1, kWait);
+        }
         mbar_wait(&bars[1], 0, kWait);
         mbar_wait(&bars[1], 1, kWait);
         if (nmild > 0) mbar_wait(&bars[2], (nmild - 1) & 1, kWait);
