@@ -312,6 +312,11 @@ __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t b
         "l"(src), "r"(bytes), "r"(smem_addr(bar))
         : "memory");
 }
+// global -> L2 only (no shared memory, no completion); address 16-B aligned,
+// size a multiple of 16
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
 // shared -> global, tracked by the issuing thread's bulk group
 __device__ __forceinline__ void bulk_store(void *dst, const void *src, uint32_t bytes) {
     asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),

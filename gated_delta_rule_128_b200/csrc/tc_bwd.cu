@@ -418,6 +418,8 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
                     // this chunk's record is consumed once T^T dDelta has read T
                     if (!mbar_wait(&bars[7], par, kWait)) record_status(status, GDN2_ERR_TIMEOUT);
                     load_rec(c - 2);
+                    // and the one after it into L2, so that its copy takes the L2 latency
+                    if (c >= 3) bulk_prefetch_l2(recs + (size_t)(c - 3) * REC_BYTES, REC_BYTES);
                 }
                 bulk_wait_read();  // the dS' copy has left OP_DS before it is rewritten
             }

@@ -394,6 +394,8 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mv, const __grid_constant__ CU
                 }
                 group1(c + 1);
             }
+            // the record after the next into L2, so that its copy takes the L2 latency
+            if (c + 3 < NC) bulk_prefetch_l2(recs + (size_t)(c + 3) * REC_BYTES, REC_BYTES);
         }
     }
     if (!abort && !dwarp) store_o(NC - 1);
