@@ -68,7 +68,7 @@ constexpr uint32_t TOT = MISC + 128;
 constexpr uint32_t SMEM_BYTES = TOT + 8192 + 1024;
 constexpr uint32_t TM_C = 0, TM_W = 128;  // the three block products (96 columns); W
 __host__ __device__ constexpr uint32_t tm_coff(int I) { return I <= 1 ? 0u : (I == 2 ? 16u : 48u); }
-constexpr uint32_t ID_KM128 = idesc_f16(64, 128, false, true);
+constexpr uint32_t ID_WP128 = idesc_f16(128, 128, false, true);
 constexpr uint32_t ID_KK128x64 = idesc_f16(128, 64, false, false);
 constexpr long long kWait = 2000000000LL;  // ~1 s of SM clocks per wait
 constexpr float kRange = 6.0e4f;
@@ -636,33 +636,31 @@ tc_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
             fence_after_sync();
             // Kc (rows 0..63 of the [Kc; Qb] tile) as the MN-major B: its two
             // 64-key blocks lie 16 KB apart
-            const uint64_t t = desc_kmajor(smem_addr(sm + OP_T), 64, 0),
+            // [T; P] (the record's T and P tiles follow each other) as one M = 128
+            // A operand, so that W lands one row per tensor-memory lane; P Kc in
+            // lanes 64..127 is not read
+            const uint64_t t = desc_kmajor(smem_addr(sm + OP_T), 128, 0),
                            kc = desc_mnmajor_lbo(smem_addr(sm + OP_WQ), 16384, 0);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tm + TM_W, kstep_kmajor(t, 64, ks), kstep_mnmajor(kc, ks), ID_KM128, ks > 0);
+                mma_bf16(tm + TM_W, kstep_kmajor(t, 128, ks), kstep_mnmajor(kc, ks), ID_WP128, ks > 0);
             mma_commit(&bars[1]);
         }
         // ---------------- -W to fp16 (over Kc, consumed by the product); the record
         if (it + (int)gridDim.x < ntiles) L_next = rows_of(it + gridDim.x);  // while W runs
         ok = mbar_wait(&bars[1], 1, kWait);
         fence_after_sync();
-        {
+        if (quarter < 2) {  // lanes 0..63: row 32 quarter + lane, 64 columns from 64 half
             float wv[64];
-            const int half = warp >> 2;
+            const int half = warp >> 2, r = quarter * 32 + lane;
 #pragma unroll
             for (int j = 0; j < 4; ++j) tmem_ld16(taddr(tm + TM_W, quarter * 32, 64 * half + 16 * j), wv + 16 * j);
             tmem_wait_ld();
-            // lanes 0..15 hold the rows; lane l + 16 takes columns 32..63 of row l
-            const int r = quarter * 16 + (lane & 15), hi = lane >> 4;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const float t = __shfl_sync(0xffffffffu, wv[32 + j], lane & 15);
-                wv[j] = -(hi ? t : wv[j]);
-            }
+            for (int j = 0; j < 64; ++j) wv[j] = -wv[j];
 #pragma unroll
-            for (int j2 = 0; j2 < 4; ++j2) {
-                st_h8(sm + OP_WQ + sw128_chunk(r, 8 * half + 4 * hi + j2, 128), wv + 8 * j2);
+            for (int j2 = 0; j2 < 8; ++j2) {
+                st_h8(sm + OP_WQ + sw128_chunk(r, 8 * half + j2, 128), wv + 8 * j2);
                 big = absmax8(wv + 8 * j2, big);
             }
         }
