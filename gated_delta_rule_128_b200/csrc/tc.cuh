@@ -277,6 +277,14 @@ __device__ __forceinline__ void tma_store_5d(const CUtensorMap *map, const void 
         : "memory");
 }
 
+// ---- TMA: 4-D tile prefetch into L2 (no shared memory, no completion)
+__device__ __forceinline__ void tma_prefetch_4d(const CUtensorMap *map, int c0, int c1, int c2, int c3) {
+    asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+                 : "memory");
+}
+
 // ---- TMA: 4-D tiled store shared -> global, tracked by the issuing
 // thread's bulk group (coordinates must not be negative)
 __device__ __forceinline__ void tma_store_4d(const CUtensorMap *map, const void *src, int c0, int c1,

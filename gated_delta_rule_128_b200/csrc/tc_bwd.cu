@@ -279,6 +279,12 @@ tc_bwd_state_kernel(const __grid_constant__ CUtensorMap mdo, const __grid_consta
             bulk_commit();
             bulk_wait_read();  // VV, VW and NDU may be rewritten
             if (cc > 0) load_vw(cc - 1);
+            if (cc > 1) {  // the v, w after those into L2, so that their copy takes the L2 latency
+                tma_prefetch_4d(&mv, v0, h, bos + (cc - 2) * 64, bb);
+                tma_prefetch_4d(&mw, v0, h, bos + (cc - 2) * 64, bb);
+                if (!GB) tma_prefetch_4d(&mw, v0 + 32, h, bos + (cc - 2) * 64, bb);
+            }
+            if (cc > 3) tma_prefetch_4d(&mdo, v0, h, bos + (cc - 4) * 64, bb);  // dO two requests ahead
         }
     };
 

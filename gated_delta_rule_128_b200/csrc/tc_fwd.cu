@@ -342,7 +342,13 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap mv, const __grid_constant__ CU
                 make_u(c + 1);
                 fence_proxy_async();
                 named_sync(2, 128);  // raw v, w consumed
-                if (tid == 64 && c + 2 < NC && use_u) load_vw(c + 2);
+                if (tid == 64 && c + 2 < NC && use_u) {
+                    load_vw(c + 2);
+                    if (c + 3 < NC) {  // the v, w after those into L2
+                        tma_prefetch_4d(&mv, v0, h, bos + (c + 3) * 64, bb);
+                        tma_prefetch_4d(&mw, v0, h, bos + (c + 3) * 64, bb);
+                    }
+                }
             }
         }
         // ---------------- S_next = gamma S + Kb^T Delta
