@@ -6,8 +6,9 @@
 //
 // Grid (8, B H): a CTA owns 16 of the 128 columns of one (b, h) and keeps them
 // in shared memory from step to step; the map M is staged in shared memory 32
-// rows (or columns) at a time with coalesced loads.  Thread t computes row
-// t / 2, 8 columns.  float32 throughout.
+// rows (or columns) at a time, each thread's four 16-byte loads issued before
+// any of them is stored, so that a stage waits for one round trip to L2.
+// Thread t computes row t / 2, 8 columns.  float32 throughout.
 
 #include "common.cuh"
 
@@ -22,7 +23,20 @@ __global__ void __launch_bounds__(256) seg_link_kernel(SegPass sp) {
     const int first = TRANSPOSE ? sp.P - 2 : 1;
     {
         const float *E = seg_buf(sp, bh, first, SEG_ENTRY);
-        for (int e = tid; e < 128 * 16; e += 256) Es[e >> 4][e & 15] = E[(e >> 4) * 128 + c0 + (e & 15)];
+        float4 ev[2];
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {  // 128 rows x 4 float4 of this CTA's 16 columns
+            const int q = tid + 256 * m;
+            ev[m] = *reinterpret_cast<const float4 *>(E + (q >> 2) * 128 + c0 + 4 * (q & 3));
+        }
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+            const int q = tid + 256 * m, r = q >> 2, c = 4 * (q & 3);
+            Es[r][c] = ev[m].x;
+            Es[r][c + 1] = ev[m].y;
+            Es[r][c + 2] = ev[m].z;
+            Es[r][c + 3] = ev[m].w;
+        }
     }
     __syncthreads();
     for (int step = 0; step < sp.P - 2; ++step) {
@@ -32,14 +46,32 @@ __global__ void __launch_bounds__(256) seg_link_kernel(SegPass sp) {
         const float *M = seg_buf(sp, bh, s_map, SEG_MAP);
         const float *A = seg_buf(sp, bh, s_map, SEG_ZERO) + (size_t)i * 128 + c0 + j0;
         float acc[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc[j] = A[j];
+        {
+            const float4 a0 = *reinterpret_cast<const float4 *>(A), a1 = *reinterpret_cast<const float4 *>(A + 4);
+            acc[0] = a0.x; acc[1] = a0.y; acc[2] = a0.z; acc[3] = a0.w;
+            acc[4] = a1.x; acc[5] = a1.y; acc[6] = a1.z; acc[7] = a1.w;
+        }
         for (int k0 = 0; k0 < 128; k0 += 32) {
-            // Ms[kk][r] = the factor of E[k0 + kk] in output row r
-            for (int e = tid; e < 32 * 128; e += 256) {
-                const int a = e >> 7, b = e & 127;  // coalesced over b
-                if (TRANSPOSE) Ms[a][b] = M[(size_t)(k0 + a) * 128 + b];  // M[k][i], k = k0 + a, i = b
-                else Ms[e & 31][e >> 5] = M[(size_t)(e >> 5) * 128 + k0 + (e & 31)];  // M[i][k]
+            // Ms[kk][r] = the factor of E[k0 + kk] in output row r: 32 x 128
+            // floats, four float4 per thread
+            float4 mv[4];
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const int q = tid + 256 * m;
+                // TRANSPOSE: M[k][i] for k = k0 + q / 32, i = 4 (q % 32) ..;
+                // else M[i][k] for i = q / 8, k = k0 + 4 (q % 8) ..
+                mv[m] = TRANSPOSE ? *reinterpret_cast<const float4 *>(M + (size_t)(k0 + (q >> 5)) * 128 + 4 * (q & 31))
+                                  : *reinterpret_cast<const float4 *>(M + (size_t)(q >> 3) * 128 + k0 + 4 * (q & 7));
+            }
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const int q = tid + 256 * m;
+                const float v[4] = {mv[m].x, mv[m].y, mv[m].z, mv[m].w};
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    if (TRANSPOSE) Ms[q >> 5][4 * (q & 31) + x] = v[x];
+                    else Ms[4 * (q & 7) + x][q >> 3] = v[x];
+                }
             }
             __syncthreads();
 #pragma unroll 4
