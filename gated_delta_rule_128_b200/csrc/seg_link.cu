@@ -5,19 +5,23 @@
 // so a segment of chunks acts on it as one affine map.
 //
 // Grid (8, B H): a CTA owns 16 of the 128 columns of one (b, h) and keeps them
-// in shared memory from step to step; the map M is staged in shared memory 32
-// rows (or columns) at a time, each thread's four 16-byte loads issued before
-// any of them is stored, so that a stage waits for one round trip to L2.
+// in shared memory from step to step.  The whole map M (64 KB) is staged in
+// dynamic shared memory per step, each thread's sixteen 16-byte loads issued
+// before any is stored, so that a step waits for one round trip to L2.
 // Thread t computes row t / 2, 8 columns.  float32 throughout.
 
 #include "common.cuh"
 
 namespace gdn2 {
 
+constexpr int kLinkMs = 128 * 129;                         // floats of the staged map
+constexpr int kLinkSmem = (kLinkMs + 128 * 17) * 4;        // + the carried columns
+
 template <bool TRANSPOSE>
 __global__ void __launch_bounds__(256) seg_link_kernel(SegPass sp) {
-    __shared__ float Es[128][17];  // the carried columns
-    __shared__ float Ms[32][129];  // 32 k-rows of M (TRANSPOSE: M[k][i]) or of M^T (M[i][k] at [k][i])
+    extern __shared__ float link_sm[];
+    float(*Ms)[129] = reinterpret_cast<float(*)[129]>(link_sm);             // Ms[k][i]: factor of E[k] in row i
+    float(*Es)[17] = reinterpret_cast<float(*)[17]>(link_sm + kLinkMs);    // the carried columns
     const int tid = threadIdx.x, i = tid >> 1, j0 = 8 * (tid & 1), c0 = 16 * blockIdx.x;
     const size_t bh = blockIdx.y;
     const int first = TRANSPOSE ? sp.P - 2 : 1;
@@ -38,7 +42,6 @@ __global__ void __launch_bounds__(256) seg_link_kernel(SegPass sp) {
             Es[r][c + 3] = ev[m].w;
         }
     }
-    __syncthreads();
     for (int step = 0; step < sp.P - 2; ++step) {
         // forward: from segment s = 1 + step to s + 1; backward: from s + 1 = P - 2 - step to s
         const int s_map = TRANSPOSE ? sp.P - 2 - step : 1 + step;
@@ -51,51 +54,49 @@ __global__ void __launch_bounds__(256) seg_link_kernel(SegPass sp) {
             acc[0] = a0.x; acc[1] = a0.y; acc[2] = a0.z; acc[3] = a0.w;
             acc[4] = a1.x; acc[5] = a1.y; acc[6] = a1.z; acc[7] = a1.w;
         }
-        for (int k0 = 0; k0 < 128; k0 += 32) {
-            // Ms[kk][r] = the factor of E[k0 + kk] in output row r: 32 x 128
-            // floats, four float4 per thread
-            float4 mv[4];
+        // the whole map, 128 rows of 32 float4: row q / 32, float4 q % 32, with
+        // q = tid + 256 m; stored as Ms[k][i]
+        float4 mv[16];
 #pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const int q = tid + 256 * m;
-                // TRANSPOSE: M[k][i] for k = k0 + q / 32, i = 4 (q % 32) ..;
-                // else M[i][k] for i = q / 8, k = k0 + 4 (q % 8) ..
-                mv[m] = TRANSPOSE ? *reinterpret_cast<const float4 *>(M + (size_t)(k0 + (q >> 5)) * 128 + 4 * (q & 31))
-                                  : *reinterpret_cast<const float4 *>(M + (size_t)(q >> 3) * 128 + k0 + 4 * (q & 7));
-            }
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const int q = tid + 256 * m;
-                const float v[4] = {mv[m].x, mv[m].y, mv[m].z, mv[m].w};
-#pragma unroll
-                for (int x = 0; x < 4; ++x) {
-                    if (TRANSPOSE) Ms[q >> 5][4 * (q & 31) + x] = v[x];
-                    else Ms[4 * (q & 7) + x][q >> 3] = v[x];
-                }
-            }
-            __syncthreads();
-#pragma unroll 4
-            for (int kk = 0; kk < 32; ++kk) {
-                const float m = Ms[kk][i];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) acc[j] = fmaf(m, Es[k0 + kk][j0 + j], acc[j]);
-            }
-            __syncthreads();
+        for (int m = 0; m < 16; ++m) {
+            const int q = tid + 256 * m;
+            mv[m] = *reinterpret_cast<const float4 *>(M + (size_t)(q >> 5) * 128 + 4 * (q & 31));
         }
+#pragma unroll
+        for (int m = 0; m < 16; ++m) {
+            const int q = tid + 256 * m, row = q >> 5, col = 4 * (q & 31);
+            const float v[4] = {mv[m].x, mv[m].y, mv[m].z, mv[m].w};
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+                if (TRANSPOSE) Ms[row][col + x] = v[x];  // M[k][i]: k = row, i = col + x
+                else Ms[col + x][row] = v[x];            // M[i][k]: i = row, k = col + x
+            }
+        }
+        __syncthreads();  // the map and the carried columns are in place
+#pragma unroll 8
+        for (int k = 0; k < 128; ++k) {
+            const float mk = Ms[k][i];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[j] = fmaf(mk, Es[k][j0 + j], acc[j]);
+        }
+        __syncthreads();  // every thread has read the carried columns and the map
         float *out = seg_buf(sp, bh, s_out, SEG_ENTRY) + (size_t)i * 128 + c0 + j0;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             Es[i][j0 + j] = acc[j];
             out[j] = acc[j];
         }
-        __syncthreads();
     }
 }
 
 cudaError_t seg_link_launch(const SegPass &sp, int nbh, bool backward, cudaStream_t s) {
+    cudaError_t e = cudaFuncSetAttribute(seg_link_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kLinkSmem);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(seg_link_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kLinkSmem);
+    if (e != cudaSuccess) return e;
     launch_begin(K_SEG_LINK, s);
-    if (backward) seg_link_kernel<true><<<dim3(8, nbh), 256, 0, s>>>(sp);
-    else seg_link_kernel<false><<<dim3(8, nbh), 256, 0, s>>>(sp);
+    if (backward) seg_link_kernel<true><<<dim3(8, nbh), 256, kLinkSmem, s>>>(sp);
+    else seg_link_kernel<false><<<dim3(8, nbh), 256, kLinkSmem, s>>>(sp);
     launch_end(K_SEG_LINK, s);
     return cudaGetLastError();
 }
